@@ -1,0 +1,178 @@
+"""fp64 CPU oracle for the gated delta-rule forward (numpy front end).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline / reference legs of ``bench.py``.  The CUDA product path
+never imports, links or calls anything here, and this package imports nothing
+from the product package.
+
+The arithmetic lives in ``gdr_oracle.c`` (plain C99 + OpenMP, fp64); this file
+only marshals numpy arrays.  Citations for each routine are in the C source:
+the token recurrence follows "Systolic Linear Attention: Co-Designing
+Tile-Grouped Gated Delta Attention for TPUs" §2.1 Eq. (2); the chunkwise WY
+form follows its §2.3 Table 2 and §2.4.2; the truncated Neumann inverse follows
+"When Good Enough Is Optimal: Multiplication-Only Matrix Inversion
+Approximation for Quantized Gated DeltaNet" (Lemma 3.1, §4.1).
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+closed forms, invariants and hand-worked examples in ``tests/golden/``.
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_gdr_oracle.so")
+_lib = None
+
+INV_EXACT = 0
+INV_NEUMANN = 1
+NV_NEWTON = 0      # residual step X <- X + X (I - (I+N) X)
+NV_REFINE = 1      # residual step X <- X + X0 (I - (I+N) X)
+NV_BANDCUT = 2     # zero X0 outside the band i - j <= order
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle C source into a shared library with gcc + OpenMP."""
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(src)):
+        return out
+    tmp = out + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+           "-Wall", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def load_library(path: str):
+    """Load an oracle build (the default one, or a test's mutated copy)."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    i = ctypes.c_int
+    lib.gdro_recurrent.argtypes = [i] * 7 + [dp] * 8 + [i]
+    lib.gdro_chunked.argtypes = [i] * 12 + [dp] * 8 + [i]
+    lib.gdro_tril_inverse.argtypes = [i, dp, dp]
+    lib.gdro_neumann_inverse.argtypes = [i, dp, i, i, i, dp]
+    lib.gdro_chunk_matrices.argtypes = [i, i, i] + [dp] * 7
+    lib.gdro_max_threads.argtypes = []
+    for f in (lib.gdro_recurrent, lib.gdro_chunked, lib.gdro_tril_inverse,
+              lib.gdro_neumann_inverse, lib.gdro_chunk_matrices, lib.gdro_max_threads):
+        f.restype = ctypes.c_int
+    return lib
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Temporarily route every oracle call through another build (tests only)."""
+    global _lib
+    saved = _load()
+    _lib = load_library(path)
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().gdro_max_threads())
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _dims(q, v, g):
+    B, Hk, T, dk = q.shape
+    Bv, Hv, Tv, dv = v.shape
+    G = g.shape[-1]
+    if Bv != B or Tv != T:
+        raise ValueError("q and v disagree on B or T")
+    return B, T, Hk, Hv, dk, dv, G
+
+
+def _check(code, what):
+    if code != 0:
+        raise ValueError("%s failed with code %d" % (what, code))
+
+
+def recurrent(q, k, v, g, beta, S0=None, nthreads=0):
+    """Token-by-token fp64 recurrence.  Returns (o [B,Hv,T,dv], S_final [B,Hv,dk,dv])."""
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    S0 = None if S0 is None else _f64(S0)
+    B, T, Hk, Hv, dk, dv, G = _dims(q, v, g)
+    o = np.zeros((B, Hv, T, dv), np.float64)
+    Sf = np.zeros((B, Hv, dk, dv), np.float64)
+    _check(_load().gdro_recurrent(B, T, Hk, Hv, dk, dv, G, _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(g), _ptr(beta), _ptr(S0), _ptr(o), _ptr(Sf),
+                                  int(nthreads)), "gdro_recurrent")
+    return o, Sf
+
+
+def chunked(q, k, v, g, beta, S0=None, chunk=64, inverse="exact", order=4, resid=1,
+            variant=NV_NEWTON, nthreads=0):
+    """Chunkwise WY form in fp64 with an exact (forward substitution) or truncated
+    Neumann chunk inverse.  Returns (o, S_final)."""
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    S0 = None if S0 is None else _f64(S0)
+    B, T, Hk, Hv, dk, dv, G = _dims(q, v, g)
+    mode = {"exact": INV_EXACT, "neumann": INV_NEUMANN}[inverse]
+    o = np.zeros((B, Hv, T, dv), np.float64)
+    Sf = np.zeros((B, Hv, dk, dv), np.float64)
+    _check(_load().gdro_chunked(B, T, Hk, Hv, dk, dv, G, int(chunk), mode, int(order),
+                                int(resid), int(variant), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(g), _ptr(beta), _ptr(S0), _ptr(o), _ptr(Sf),
+                                int(nthreads)), "gdro_chunked")
+    return o, Sf
+
+
+def tril_inverse(N):
+    """(I + N)^{-1} for strictly lower-triangular N, by forward substitution."""
+    N = _f64(N)
+    n = N.shape[0]
+    X = np.zeros((n, n), np.float64)
+    _check(_load().gdro_tril_inverse(n, _ptr(N), _ptr(X)), "gdro_tril_inverse")
+    return X
+
+
+def neumann_inverse(N, order=4, resid=1, variant=NV_NEWTON):
+    """Truncated Neumann approximation of (I + N)^{-1} with structural masking
+    and `resid` residual-correction steps."""
+    N = _f64(N)
+    n = N.shape[0]
+    X = np.zeros((n, n), np.float64)
+    _check(_load().gdro_neumann_inverse(n, _ptr(N), int(order), int(resid), int(variant),
+                                        _ptr(X)), "gdro_neumann_inverse")
+    return X
+
+
+def chunk_matrices(qc, kc, gc, bc):
+    """Cumulative log-decay Lam [C,dk], Gram M [C,C] and score L [C,C] of one
+    chunk of one key head (qc, kc [C,dk]; gc [C,G]; bc [C])."""
+    qc, kc, gc, bc = map(_f64, (qc, kc, gc, bc))
+    C, dk = kc.shape
+    G = gc.shape[-1]
+    Lam = np.zeros((C, dk), np.float64)
+    M = np.zeros((C, C), np.float64)
+    L = np.zeros((C, C), np.float64)
+    _check(_load().gdro_chunk_matrices(C, dk, G, _ptr(qc), _ptr(kc), _ptr(gc), _ptr(bc),
+                                       _ptr(Lam), _ptr(M), _ptr(L)), "gdro_chunk_matrices")
+    return Lam, M, L

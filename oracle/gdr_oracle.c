@@ -1,0 +1,424 @@
+/*
+ * gdr_oracle.c -- plain, slow, fp64 CPU oracle for the gated delta-rule forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may load, link or
+ * call this file.  It is used by tests/, by __graft_entry__.smoke() and by the
+ * CPU-baseline / reference legs of bench.py, and nowhere else.  It shares no
+ * code, header, table or helper with the CUDA library.
+ *
+ * Sources (page title, section/equation):
+ *  [SLA]  "Systolic Linear Attention: Co-Designing Tile-Grouped Gated Delta
+ *         Attention for TPUs".
+ *  [MOMI] "When Good Enough Is Optimal: Multiplication-Only Matrix Inversion
+ *         Approximation for Quantized Gated DeltaNet".
+ *
+ * Layouts (all row-major, contiguous, fp64):
+ *   q, k   [B, Hk, T, dk]      query / key of key head hk
+ *   v      [B, Hv, T, dv]      value of value head hv; hv uses key head hv / R,
+ *                              R = Hv / Hk (grouped value heads, [SLA] §2.3,
+ *                              §2.4.1)
+ *   g      [B, Hk, T, G]       log forget gate (<= 0); channel i of a key head
+ *                              uses group floor(i * G / dk)  ([SLA] §2.1 GDN
+ *                              G=1, KDA G=dk; §2.3 four 64-channel tiles)
+ *   beta   [B, Hk, T]          write gate, shared by the R value heads
+ *   S0     [B, Hv, dk, dv]     initial state, or NULL for zeros
+ *   o      [B, Hv, T, dv]      output o_t = S_t^T q_t (post-update state)
+ *   S_final[B, Hv, dk, dv]     state after the last token
+ *
+ * Every function returns 0 on success and a negative code on a bad argument.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define GDRO_ERR_ARG (-1)
+#define GDRO_ERR_NOMEM (-2)
+
+/* Inverse modes and Neumann variant bits (mirrors nothing; the CUDA library
+ * defines its own enums). */
+#define GDRO_INV_EXACT 0
+#define GDRO_INV_NEUMANN 1
+#define GDRO_NV_REFINE 1   /* residual step uses X0 instead of X_k        */
+#define GDRO_NV_BANDCUT 2  /* zero X0 outside the band i - j <= order      */
+
+static int check_dims(int B, int T, int Hk, int Hv, int dk, int dv, int G)
+{
+    if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0 || G <= 0)
+        return GDRO_ERR_ARG;
+    if (Hv % Hk != 0 || dk % G != 0)
+        return GDRO_ERR_ARG;
+    return 0;
+}
+
+static void set_threads(int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+int gdro_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Token-by-token recurrence, the definition of the operation.
+ * [SLA] §2.1, Eq. (2), prediction-error form:
+ *     S_t = F_t S_{t-1} + beta_t k_t (v_t - (F_t S_{t-1})^T k_t)^T,
+ *     o_t = S_t^T q_t,   F_t = diag(exp(g_t expanded to dk channels)).
+ * Each step: decay the rows of S, read the current prediction r = S^T k,
+ * write beta * k (v - r)^T, read out with q.
+ */
+int gdro_recurrent(int B, int T, int Hk, int Hv, int dk, int dv, int G,
+                   const double *q, const double *k, const double *v,
+                   const double *g, const double *beta, const double *S0,
+                   double *o, double *S_final, int nthreads)
+{
+    if (check_dims(B, T, Hk, Hv, dk, dv, G))
+        return GDRO_ERR_ARG;
+    const int R = Hv / Hk;
+    const long nseq = (long)B * Hv;
+    int err = 0;
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long s = 0; s < nseq; ++s) {
+        const long b = s / Hv, hv = s % Hv, hk = hv / R;
+        double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+        double *r = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *f = (double *)malloc(sizeof(double) * (size_t)dk);
+        if (!S || !r || !f) {
+            free(S); free(r); free(f);
+#pragma omp atomic write
+            err = GDRO_ERR_NOMEM;
+            continue;
+        }
+        if (S0)
+            memcpy(S, S0 + s * (long)dk * dv, sizeof(double) * (size_t)dk * dv);
+        else
+            memset(S, 0, sizeof(double) * (size_t)dk * dv);
+        const long kh = b * Hk + hk;
+        for (long t = 0; t < T; ++t) {
+            const double *qt = q + (kh * T + t) * dk;
+            const double *kt = k + (kh * T + t) * dk;
+            const double *vt = v + (s * T + t) * dv;
+            const double *gt = g + (kh * T + t) * G;
+            const double bt = beta[kh * T + t];
+            for (int i = 0; i < dk; ++i)
+                f[i] = exp(gt[(long)i * G / dk]);
+            /* decay: S <- F_t S */
+            for (int i = 0; i < dk; ++i)
+                for (int n = 0; n < dv; ++n)
+                    S[i * dv + n] *= f[i];
+            /* current prediction r = S^T k */
+            for (int n = 0; n < dv; ++n)
+                r[n] = 0.0;
+            for (int i = 0; i < dk; ++i)
+                for (int n = 0; n < dv; ++n)
+                    r[n] += S[i * dv + n] * kt[i];
+            /* delta write */
+            for (int i = 0; i < dk; ++i) {
+                const double bk = bt * kt[i];
+                for (int n = 0; n < dv; ++n)
+                    S[i * dv + n] += bk * (vt[n] - r[n]);
+            }
+            /* readout with the post-update state */
+            double *ot = o + (s * T + t) * dv;
+            for (int n = 0; n < dv; ++n)
+                ot[n] = 0.0;
+            for (int i = 0; i < dk; ++i)
+                for (int n = 0; n < dv; ++n)
+                    ot[n] += S[i * dv + n] * qt[i];
+        }
+        if (S_final)
+            memcpy(S_final + s * (long)dk * dv, S, sizeof(double) * (size_t)dk * dv);
+        free(S); free(r); free(f);
+    }
+    return err;
+}
+
+/*
+ * X = (I + N)^{-1} for strictly lower-triangular N (n x n, row-major), by
+ * forward substitution (row t of X from rows j < t).  This is the
+ * "sequential substitution" that [SLA] §2.2 Bottleneck 3 describes; it is a
+ * different algorithm from the block-doubling the GPU uses.
+ */
+int gdro_tril_inverse(int n, const double *N, double *X)
+{
+    if (n < 0)
+        return GDRO_ERR_ARG;
+    for (int t = 0; t < n; ++t) {
+        for (int c = 0; c < n; ++c) {
+            double acc = (t == c) ? 1.0 : 0.0;
+            for (int j = c; j < t; ++j)
+                acc -= N[t * n + j] * X[j * n + c];
+            X[t * n + c] = (c <= t) ? acc : 0.0;
+        }
+    }
+    return 0;
+}
+
+static void matmul_nn(int n, const double *A, const double *B, double *C)
+{
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int l = 0; l < n; ++l)
+                acc += A[i * n + l] * B[l * n + j];
+            C[i * n + j] = acc;
+        }
+}
+
+/*
+ * Truncated Neumann approximation of (I + N)^{-1}, N strictly lower
+ * triangular, following [MOMI] (abstract; Lemma 3.1; §4.1 settings):
+ *   1. powers with structural masking: P_1 = N, P_p = mask_p(P_{p-1} N),
+ *      mask_p zeroing entries with i - j < p (Lemma 3.1: those entries of
+ *      N^p vanish, so the mask keeps only the structurally non-zero band);
+ *   2. X_0 = sum_{p=0}^{order} (-1)^p P_p;
+ *   3. residual correction, `resid` times:
+ *        Newton (default):  X_{s+1} = X_s + X_s (I - (I + N) X_s)
+ *        refine (flag 1) :  X_{s+1} = X_s + X_0 (I - (I + N) X_s)
+ *      (identical for one step).
+ * Flag 2 zeroes X_0 outside the band i - j <= order before the correction.
+ */
+int gdro_neumann_inverse(int n, const double *N, int order, int resid, int variant,
+                         double *X)
+{
+    if (n < 0 || order < 0 || resid < 0)
+        return GDRO_ERR_ARG;
+    const size_t nn = (size_t)n * n;
+    double *P = (double *)malloc(sizeof(double) * (nn ? nn : 1));
+    double *T1 = (double *)malloc(sizeof(double) * (nn ? nn : 1));
+    double *X0 = (double *)malloc(sizeof(double) * (nn ? nn : 1));
+    double *Rm = (double *)malloc(sizeof(double) * (nn ? nn : 1));
+    if (!P || !T1 || !X0 || !Rm) {
+        free(P); free(T1); free(X0); free(Rm);
+        return GDRO_ERR_NOMEM;
+    }
+    /* X0 = I (p = 0) */
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j)
+            X0[i * n + j] = (i == j) ? 1.0 : 0.0;
+    if (order >= 1) {
+        memcpy(P, N, sizeof(double) * nn);
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j)
+                if (i - j < 1)
+                    P[i * n + j] = 0.0;
+        for (size_t e = 0; e < nn; ++e)
+            X0[e] -= P[e];
+    }
+    for (int p = 2; p <= order; ++p) {
+        matmul_nn(n, P, N, T1);
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j)
+                if (i - j < p)
+                    T1[i * n + j] = 0.0;
+        memcpy(P, T1, sizeof(double) * nn);
+        const double sgn = (p % 2 == 0) ? 1.0 : -1.0;
+        for (size_t e = 0; e < nn; ++e)
+            X0[e] += sgn * P[e];
+    }
+    if (variant & GDRO_NV_BANDCUT)
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j)
+                if (i - j > order)
+                    X0[i * n + j] = 0.0;
+    memcpy(X, X0, sizeof(double) * nn);
+    for (int s = 0; s < resid; ++s) {
+        /* Rm = I - (I + N) X = -(N X) + (I - X) */
+        matmul_nn(n, N, X, T1);
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j)
+                Rm[i * n + j] = ((i == j) ? 1.0 : 0.0) - X[i * n + j] - T1[i * n + j];
+        matmul_nn(n, (variant & GDRO_NV_REFINE) ? X0 : X, Rm, T1);
+        for (size_t e = 0; e < nn; ++e)
+            X[e] += T1[e];
+    }
+    free(P); free(T1); free(X0); free(Rm);
+    return 0;
+}
+
+/*
+ * Chunk matrices of one chunk for one key head, [SLA] §2.2 Bottleneck 2 and
+ * §2.3 Table 2 (Gram M, score L, cumulative log-decay Lambda):
+ *   Lam[t][i] = sum_{s<=t} g_s(i)                       (summed, never log o exp)
+ *   M[t][j]   = 1[t>j]  beta_j sum_i k_ti k_ji exp(Lam_ti - Lam_ji)
+ *   L[t][j]   = 1[t>=j]        sum_i q_ti k_ji exp(Lam_ti - Lam_ji)
+ * The exponent is always of a difference with t >= j, so it is <= 0 and
+ * needs no pivot in fp64.  Arrays: qc,kc [Cl][dk], gc [Cl][G], bc [Cl].
+ */
+static void chunk_matrices(int Cl, int dk, int G, const double *qc, const double *kc,
+                           const double *gc, const double *bc, double *Lam,
+                           double *M, double *L)
+{
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        for (int t = 0; t < Cl; ++t) {
+            acc += gc[(long)t * G + (long)i * G / dk];
+            Lam[t * dk + i] = acc;
+        }
+    }
+    for (int t = 0; t < Cl; ++t)
+        for (int j = 0; j < Cl; ++j) {
+            double m = 0.0, l = 0.0;
+            if (j <= t) {
+                for (int i = 0; i < dk; ++i) {
+                    const double d = exp(Lam[t * dk + i] - Lam[j * dk + i]);
+                    m += kc[t * dk + i] * kc[j * dk + i] * d;
+                    l += qc[t * dk + i] * kc[j * dk + i] * d;
+                }
+            }
+            M[t * Cl + j] = (j < t) ? bc[j] * m : 0.0;
+            L[t * Cl + j] = (j <= t) ? l : 0.0;
+        }
+}
+
+int gdro_chunk_matrices(int Cl, int dk, int G, const double *qc, const double *kc,
+                        const double *gc, const double *bc, double *Lam, double *M,
+                        double *L)
+{
+    if (Cl < 0 || dk <= 0 || G <= 0 || dk % G != 0)
+        return GDRO_ERR_ARG;
+    chunk_matrices(Cl, dk, G, qc, kc, gc, bc, Lam, M, L);
+    return 0;
+}
+
+/*
+ * Chunkwise WY form ([SLA] §2.1 "Chunkwise WY parallelization", §2.3 Table 2,
+ * §2.4.2 "Proof of tile-grouped packed WY equivalence", §2.5):
+ *   A  = (I + M)^{-1}                     (exact: forward substitution;
+ *                                          NEUMANN: gdro_neumann_inverse)
+ *   Kb = P_{t<-0} k_t,  Qb = P_{t<-0} q_t,  Kh = P_{C<-t} k_t,  F = P_{C<-0}
+ *   E  = diag(beta) A (V - Kb S)          (= U - W S with U, W of Table 2)
+ *   O  = Qb S + L E
+ *   S <- F S + Kh^T E
+ * A ragged last chunk (T % C != 0) is a chunk of length T - start.
+ * Processed per value head (one S of dk x dv), so the packed grouped-value
+ * form is reached by running the R value heads of a key head separately.
+ */
+int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
+                 int inverse_mode, int neumann_order, int neumann_resid,
+                 int neumann_variant, const double *q, const double *k,
+                 const double *v, const double *g, const double *beta,
+                 const double *S0, double *o, double *S_final, int nthreads)
+{
+    if (check_dims(B, T, Hk, Hv, dk, dv, G) || C <= 0)
+        return GDRO_ERR_ARG;
+    if (inverse_mode != GDRO_INV_EXACT && inverse_mode != GDRO_INV_NEUMANN)
+        return GDRO_ERR_ARG;
+    if (inverse_mode == GDRO_INV_NEUMANN && (neumann_order < 0 || neumann_resid < 0))
+        return GDRO_ERR_ARG;
+    const int R = Hv / Hk;
+    const long nseq = (long)B * Hv;
+    int err = 0;
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long s = 0; s < nseq; ++s) {
+        const long b = s / Hv, hv = s % Hv, hk = hv / R;
+        const long kh = b * Hk + hk;
+        const size_t CC = (size_t)C * C;
+        double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+        double *Lam = (double *)malloc(sizeof(double) * (size_t)C * dk);
+        double *M = (double *)malloc(sizeof(double) * CC);
+        double *L = (double *)malloc(sizeof(double) * CC);
+        double *A = (double *)malloc(sizeof(double) * CC);
+        double *RHS = (double *)malloc(sizeof(double) * (size_t)C * dv);
+        double *E = (double *)malloc(sizeof(double) * (size_t)C * dv);
+        double *Kb = (double *)malloc(sizeof(double) * (size_t)C * dk);
+        double *Qb = (double *)malloc(sizeof(double) * (size_t)C * dk);
+        double *Kh = (double *)malloc(sizeof(double) * (size_t)C * dk);
+        double *F = (double *)malloc(sizeof(double) * (size_t)dk);
+        if (!S || !Lam || !M || !L || !A || !RHS || !E || !Kb || !Qb || !Kh || !F) {
+            free(S); free(Lam); free(M); free(L); free(A); free(RHS); free(E);
+            free(Kb); free(Qb); free(Kh); free(F);
+#pragma omp atomic write
+            err = GDRO_ERR_NOMEM;
+            continue;
+        }
+        if (S0)
+            memcpy(S, S0 + s * (long)dk * dv, sizeof(double) * (size_t)dk * dv);
+        else
+            memset(S, 0, sizeof(double) * (size_t)dk * dv);
+        for (long c0 = 0; c0 < T; c0 += C) {
+            const int Cl = (int)((T - c0 < C) ? (T - c0) : C);
+            const double *qc = q + (kh * T + c0) * dk;
+            const double *kc = k + (kh * T + c0) * dk;
+            const double *vc = v + (s * T + c0) * dv;
+            const double *gc = g + (kh * T + c0) * G;
+            const double *bc = beta + kh * T + c0;
+            chunk_matrices(Cl, dk, G, qc, kc, gc, bc, Lam, M, L);
+            if (inverse_mode == GDRO_INV_EXACT)
+                gdro_tril_inverse(Cl, M, A);
+            else if (gdro_neumann_inverse(Cl, M, neumann_order, neumann_resid,
+                                          neumann_variant, A) != 0) {
+#pragma omp atomic write
+                err = GDRO_ERR_NOMEM;
+                break;
+            }
+            /* decayed operands: Kb_t = P_{t<-0} k_t, Qb_t = P_{t<-0} q_t,
+             * Kh_t = P_{C<-t} k_t, F = P_{C<-0} (Table 2 of [SLA] §2.3) */
+            for (int i = 0; i < dk; ++i) {
+                const double LamC = Lam[(Cl - 1) * dk + i];
+                F[i] = exp(LamC);
+                for (int t = 0; t < Cl; ++t) {
+                    Kb[t * dk + i] = kc[t * dk + i] * exp(Lam[t * dk + i]);
+                    Qb[t * dk + i] = qc[t * dk + i] * exp(Lam[t * dk + i]);
+                    Kh[t * dk + i] = kc[t * dk + i] * exp(LamC - Lam[t * dk + i]);
+                }
+            }
+            /* RHS = V - Kb S */
+            for (int t = 0; t < Cl; ++t)
+                for (int n = 0; n < dv; ++n) {
+                    double acc = vc[t * dv + n];
+                    for (int i = 0; i < dk; ++i)
+                        acc -= Kb[t * dk + i] * S[i * dv + n];
+                    RHS[t * dv + n] = acc;
+                }
+            /* E = diag(beta) A RHS */
+            for (int t = 0; t < Cl; ++t)
+                for (int n = 0; n < dv; ++n) {
+                    double acc = 0.0;
+                    for (int j = 0; j < Cl; ++j)
+                        acc += A[t * Cl + j] * RHS[j * dv + n];
+                    E[t * dv + n] = bc[t] * acc;
+                }
+            /* O = Qb S + L E (uses the chunk-entry state) */
+            for (int t = 0; t < Cl; ++t) {
+                double *ot = o + (s * T + c0 + t) * dv;
+                for (int n = 0; n < dv; ++n) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i)
+                        acc += Qb[t * dk + i] * S[i * dv + n];
+                    for (int j = 0; j <= t; ++j)
+                        acc += L[t * Cl + j] * E[j * dv + n];
+                    ot[n] = acc;
+                }
+            }
+            /* S <- F S + Kh^T E */
+            for (int i = 0; i < dk; ++i)
+                for (int n = 0; n < dv; ++n) {
+                    double acc = F[i] * S[i * dv + n];
+                    for (int t = 0; t < Cl; ++t)
+                        acc += Kh[t * dk + i] * E[t * dv + n];
+                    S[i * dv + n] = acc;
+                }
+        }
+        if (S_final)
+            memcpy(S_final + s * (long)dk * dv, S, sizeof(double) * (size_t)dk * dv);
+        free(S); free(Lam); free(M); free(L); free(A); free(RHS); free(E);
+        free(Kb); free(Qb); free(Kh); free(F);
+    }
+    return err;
+}
