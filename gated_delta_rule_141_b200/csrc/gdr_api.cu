@@ -1,0 +1,196 @@
+// gdr_api.cu -- the C ABI of libgdr.so (declared in include/gdr.h): argument
+// validation, kernel selection and the host-buffer convenience entry point.
+// Every computation happens in the kernels of gdr_simt.cu / gdr_tc.cu.
+#include <cstdint>
+
+#include "gdr.h"
+#include "gdr_internal.h"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(gdr_dtype d) { return d == GDR_BF16 ? 2 : 4; }
+
+gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inverse_mode im,
+                       gdr::Params *p)
+{
+    if (s == nullptr)
+        return GDR_ERR_ARG;
+    if (s->in_dtype != GDR_F32 && s->in_dtype != GDR_BF16)
+        return GDR_ERR_DTYPE;
+    if (s->out_dtype != GDR_F32 && s->out_dtype != GDR_BF16)
+        return GDR_ERR_DTYPE;
+    if (s->kernel != GDR_KERNEL_AUTO && s->kernel != GDR_KERNEL_SIMT && s->kernel != GDR_KERNEL_TC)
+        return GDR_ERR_ARG;
+    if (s->B < 0 || s->T < 0 || s->Hk < 1 || s->Hv < 1 || s->Hv % s->Hk != 0)
+        return GDR_ERR_SHAPE;
+    if (s->dk < 1 || s->dk > 256 || s->dv < 1 || s->dv > 256)
+        return GDR_ERR_SHAPE;
+    if (chunk < 1 || chunk > 128)
+        return GDR_ERR_SHAPE;
+    int G;
+    switch (gm) {
+    case GDR_GATE_SCALAR: G = 1; break;
+    case GDR_GATE_GROUP64:
+        if (s->dk % 64 != 0)
+            return GDR_ERR_SHAPE;
+        G = s->dk / 64;
+        break;
+    case GDR_GATE_CHANNEL: G = s->dk; break;
+    default: return GDR_ERR_ARG;
+    }
+    if (im != GDR_INV_EXACT && im != GDR_INV_NEUMANN)
+        return GDR_ERR_ARG;
+    if (im == GDR_INV_NEUMANN &&
+        (s->neumann_order < 0 || s->neumann_order > 256 || s->neumann_residual_steps < 0 ||
+         s->neumann_residual_steps > 16))
+        return GDR_ERR_SHAPE;
+    *p = gdr::Params{};
+    p->B = s->B; p->T = s->T; p->Hk = s->Hk; p->Hv = s->Hv; p->dk = s->dk; p->dv = s->dv;
+    p->G = G; p->C = chunk; p->R = s->Hv / s->Hk;
+    p->in_bf16 = s->in_dtype == GDR_BF16;
+    p->out_bf16 = s->out_dtype == GDR_BF16;
+    p->neumann = im == GDR_INV_NEUMANN;
+    p->neu_order = p->neumann ? s->neumann_order : 0;
+    p->neu_resid = p->neumann ? s->neumann_residual_steps : 0;
+    return GDR_OK;
+}
+
+// GDR_KERNEL_SIMT / GDR_KERNEL_TC, or -status.
+int choose(const gdr::Params &p, gdr_kernel want)
+{
+    const bool tc = gdr::tc_supports(p);
+    const bool simt = gdr::simt_smem_bytes(p) <= 227 * 1024;
+    if (want == GDR_KERNEL_TC)
+        return tc ? GDR_KERNEL_TC : -GDR_ERR_UNSUPPORTED;
+    if (want == GDR_KERNEL_SIMT)
+        return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
+    if (tc)
+        return GDR_KERNEL_TC;
+    return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, const float *S0, int chunk,
+                         gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode, void *o,
+                         float *S_final, void *stream)
+{
+    gdr::Params p;
+    gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return st;
+    const bool has_tokens = (long)p.B * p.T > 0;
+    if (has_tokens && (!q || !k || !v || !g || !beta || !o))
+        return GDR_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_final};
+    for (const void *ptr : ptrs)
+        if (ptr != nullptr && !aligned16(ptr))
+            return GDR_ERR_ALIGN;
+    const int which = choose(p, shape->kernel);
+    if (which < 0)
+        return static_cast<gdr_status>(-which);
+    if (p.B == 0)
+        return GDR_OK;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S0 = S0; p.o = o; p.S_final = S_final;
+    auto s = static_cast<cudaStream_t>(stream);
+    const int rc = which == GDR_KERNEL_TC ? gdr::launch_tc(p, s) : gdr::launch_simt(p, s);
+    return static_cast<gdr_status>(rc);
+}
+
+gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const gdr_io *dev,
+                              int chunk, gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode,
+                              void *stream)
+{
+    if (host == nullptr || dev == nullptr)
+        return GDR_ERR_ARG;
+    gdr::Params p;
+    gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return st;
+    const bool has_tokens = (long)p.B * p.T > 0;
+    if (has_tokens && (!host->q || !host->k || !host->v || !host->g || !host->beta || !host->o))
+        return GDR_ERR_ARG;
+    if ((host->S0 == nullptr) != (dev->S0 == nullptr) ||
+        (host->S_final == nullptr) != (dev->S_final == nullptr))
+        return GDR_ERR_ARG;
+    const size_t si = elem_size(shape->in_dtype), so = elem_size(shape->out_dtype);
+    const size_t nk = (size_t)p.B * p.Hk * p.T, nv = (size_t)p.B * p.Hv * p.T;
+    const size_t nstate = (size_t)p.B * p.Hv * p.dk * p.dv;
+    auto s = static_cast<cudaStream_t>(stream);
+    struct Copy { void *dst; const void *src; size_t bytes; };
+    const Copy in[] = {
+        {const_cast<void *>(dev->q), host->q, nk * p.dk * si},
+        {const_cast<void *>(dev->k), host->k, nk * p.dk * si},
+        {const_cast<void *>(dev->v), host->v, nv * p.dv * si},
+        {const_cast<float *>(dev->g), host->g, nk * p.G * sizeof(float)},
+        {const_cast<float *>(dev->beta), host->beta, nk * sizeof(float)},
+        {const_cast<float *>(dev->S0), host->S0, nstate * sizeof(float)},
+    };
+    for (const Copy &c : in) {
+        if (c.bytes == 0 || c.src == nullptr)
+            continue;
+        if (c.dst == nullptr)
+            return GDR_ERR_ARG;
+        if (cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return GDR_ERR_CUDA;
+    }
+    st = gdr_chunk_fwd(shape, dev->q, dev->k, dev->v, dev->g, dev->beta, dev->S0, chunk,
+                       gate_mode, inverse_mode, dev->o, dev->S_final, stream);
+    if (st != GDR_OK)
+        return st;
+    if (has_tokens &&
+        cudaMemcpyAsync(host->o, dev->o, nv * p.dv * so, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    if (host->S_final && nstate &&
+        cudaMemcpyAsync(host->S_final, dev->S_final, nstate * sizeof(float),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    return GDR_OK;
+}
+
+int gdr_select_kernel(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                      gdr_inverse_mode inverse_mode)
+{
+    gdr::Params p;
+    const gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return -static_cast<int>(st);
+    return choose(p, shape->kernel);
+}
+
+gdr_status gdr_device_status(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    const int v = gdr::read_and_clear_device_status();
+    if (v < 0)
+        return GDR_ERR_CUDA;
+    return v == 0 ? GDR_OK : GDR_ERR_TIMEOUT;
+}
+
+const char *gdr_status_string(gdr_status status)
+{
+    switch (status) {
+    case GDR_OK: return "ok";
+    case GDR_ERR_ARG: return "invalid argument (null pointer or bad enum)";
+    case GDR_ERR_SHAPE: return "sizes outside the supported envelope";
+    case GDR_ERR_DTYPE: return "unsupported dtype";
+    case GDR_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case GDR_ERR_UNSUPPORTED: return "no kernel implements this request";
+    case GDR_ERR_CUDA: return "CUDA runtime error";
+    case GDR_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case GDR_ERR_NONFINITE: return "non-finite input";
+    }
+    return "unknown status";
+}
+
+int gdr_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,40 @@
+// gdr_internal.h -- launch parameters shared by the C-ABI layer and the kernels
+// of libgdr.so (not part of the public ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace gdr {
+
+// One validated gdr_chunk_fwd request, flattened for the kernels.
+struct Params {
+    int B, T, Hk, Hv, dk, dv;
+    int G;          // decay groups: 1, dk/64 or dk
+    int C;          // chunk length
+    int R;          // value heads per key head
+    int in_bf16;    // q, k, v are bf16 (else fp32)
+    int out_bf16;   // o is bf16 (else fp32)
+    int neumann;    // 0 exact inverse, 1 truncated Neumann
+    int neu_order;  // Neumann order m
+    int neu_resid;  // Newton residual corrections
+    const void *q, *k, *v;
+    const float *g, *beta, *S0;
+    void *o;
+    float *S_final;
+};
+
+// Status word that kernels set when a bounded wait gives up (0 = fine).  It
+// lives in gdr_tc.cu, the translation unit whose kernels wait; this reads it
+// (after the caller synchronised) and clears it.  Returns -1 on a CUDA error.
+int read_and_clear_device_status();
+
+// CUDA-core kernel (fp32 arithmetic).  Returns 0 on launch, or a gdr_status
+// code if the request does not fit the kernel's shared-memory budget.
+int simt_smem_bytes(const Params &p);
+int launch_simt(const Params &p, cudaStream_t stream);
+
+// Tensor-core kernel (tcgen05 + TMEM + TMA, bf16 operands, fp32 accumulate).
+bool tc_supports(const Params &p);
+int launch_tc(const Params &p, cudaStream_t stream);
+
+}  // namespace gdr

@@ -1,0 +1,333 @@
+// gdr_simt.cu -- chunkwise gated delta-rule forward on the CUDA cores, in fp32.
+//
+// The general kernel of the library: any gate mode, any chunk length up to 128,
+// fp32 or bf16 inputs, fp32 arithmetic throughout.  It is the fp32 path
+// (spec tolerance 1e-4) and serves every request the tensor-core kernel
+// does not take.  It follows the chunkwise WY algebra of "Systolic Linear
+// Attention: Co-Designing Tile-Grouped Gated Delta Attention for TPUs"
+// (§2.1 "Chunkwise WY parallelization", §2.3 Table 2, §2.4.2):
+//   Lambda_t = cumsum g,  M_tj = 1[t>j] beta_j sum_i k_ti k_ji e^{Lambda_ti - Lambda_ji},
+//   A = (I + M)^{-1},  E = diag(beta) A (V - Kbar S),  O = Qbar S + L E,
+//   S <- F S + Khat^T E,
+// with every decay factor formed as the exponential of a non-positive
+// difference of cumulative log-decays (no division by decay prefixes).  The
+// exact inverse is forward substitution in shared memory; the Neumann inverse
+// follows "When Good Enough Is Optimal: Multiplication-Only Matrix Inversion
+// Approximation for Quantized Gated DeltaNet" (masked powers, Lemma 3.1, then
+// Newton residual corrections).
+//
+// One CTA owns one value head and NV value columns; chunks run in order.
+#include <cuda_bf16.h>
+
+#include "gdr_internal.h"
+
+namespace gdr {
+namespace {
+
+constexpr int NT = 256;  // threads per CTA
+constexpr int NV = 32;   // value columns per CTA
+constexpr int LB = 16;   // rows per row block (L readout, Neumann products)
+
+struct SimtLayout {      // offsets in floats into dynamic shared memory
+    int lam, A, P, X, S, rhs, qs, E, blk, beta, row, total;
+};
+
+__host__ __device__ inline SimtLayout simt_layout(int C, int G, int dk, bool neumann)
+{
+    SimtLayout s;
+    int off = 0;
+    s.lam = off;  off += C * G;
+    s.A = off;    off += C * C;
+    s.P = off;    off += neumann ? C * C : 0;
+    s.X = off;    off += neumann ? C * C : 0;
+    s.S = off;    off += dk * NV;
+    s.rhs = off;  off += C * NV;
+    s.qs = off;   off += C * NV;
+    s.E = off;    off += C * NV;
+    s.blk = off;  off += LB * C;
+    s.beta = off; off += C;
+    s.row = off;  off += C;
+    s.total = off;
+    return s;
+}
+
+template <bool BF>
+__device__ __forceinline__ float ld_in(const void *p, long i)
+{
+    if constexpr (BF)
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+    else
+        return static_cast<const float *>(p)[i];
+}
+
+template <bool BF>
+__device__ __forceinline__ void st_out(void *p, long i, float x)
+{
+    if constexpr (BF)
+        static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+    else
+        static_cast<float *>(p)[i] = x;
+}
+
+template <bool IN_BF16, bool OUT_BF16>
+__global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
+{
+    extern __shared__ float sm[];
+    const int C = p.C, G = p.G, dk = p.dk, dv = p.dv, T = p.T;
+    const bool neu = p.neumann != 0;
+    const SimtLayout Ly = simt_layout(C, G, dk, neu);
+    float *lam = sm + Ly.lam, *A = sm + Ly.A, *P = sm + Ly.P, *X = sm + Ly.X;
+    float *S = sm + Ly.S, *rhs = sm + Ly.rhs, *qs = sm + Ly.qs, *E = sm + Ly.E;
+    float *blk = sm + Ly.blk, *sbeta = sm + Ly.beta, *row = sm + Ly.row;
+
+    const int tid = threadIdx.x;
+    const int n0 = blockIdx.x * NV;           // first value column of this CTA
+    const int hv = blockIdx.y, b = blockIdx.z;
+    const int hk = hv / p.R;                  // key head read by this value head
+    const int nv = min(NV, dv - n0);          // live columns of this CTA
+    const long kh = (long)b * p.Hk + hk;      // key-head sequence
+    const long vh = (long)b * p.Hv + hv;      // value-head sequence
+    const int width = dk / G;                 // channels per decay group
+
+    for (int idx = tid; idx < dk * NV; idx += NT) {
+        const int i = idx / NV, n = idx % NV;
+        S[idx] = (p.S0 != nullptr && n < nv) ? p.S0[(vh * dk + i) * dv + n0 + n] : 0.f;
+    }
+
+    for (int c0 = 0; c0 < T; c0 += C) {
+        const int Cl = min(C, T - c0);        // a ragged last chunk is shorter
+        __syncthreads();
+        // --- write gates and cumulative log-decay Lambda (summed, per group)
+        for (int t = tid; t < Cl; t += NT)
+            sbeta[t] = p.beta[kh * T + c0 + t];
+        for (int gi = tid; gi < G; gi += NT) {
+            float acc = 0.f;
+            for (int t = 0; t < Cl; ++t) {
+                acc += p.g[(kh * T + c0 + t) * G + gi];
+                lam[t * G + gi] = acc;
+            }
+        }
+        __syncthreads();
+        // --- Gram M (strictly lower, beta on the column) into A
+        for (int idx = tid; idx < Cl * Cl; idx += NT) {
+            const int t = idx / Cl, j = idx % Cl;
+            float m = 0.f;
+            if (j < t) {
+                const long kt = (kh * T + c0 + t) * dk, kj = (kh * T + c0 + j) * dk;
+                for (int gi = 0; gi < G; ++gi) {
+                    float s = 0.f;
+                    for (int i = gi * width; i < (gi + 1) * width; ++i)
+                        s += ld_in<IN_BF16>(p.k, kt + i) * ld_in<IN_BF16>(p.k, kj + i);
+                    m += expf(lam[t * G + gi] - lam[j * G + gi]) * s;
+                }
+                m *= sbeta[j];
+            }
+            A[t * C + j] = m;
+        }
+        __syncthreads();
+        // --- chunk inverse
+        if (!neu) {
+            // forward substitution in place: row t of M becomes row t of A
+            for (int t = tid; t < Cl; t += NT)
+                A[t * C + t] = 1.f;
+            __syncthreads();
+            for (int t = 1; t < Cl; ++t) {
+                for (int j = tid; j < t; j += NT)
+                    row[j] = A[t * C + j];
+                __syncthreads();
+                for (int c = tid; c < t; c += NT) {
+                    float acc = -row[c];
+                    for (int j = c + 1; j < t; ++j)
+                        acc -= row[j] * A[j * C + c];
+                    A[t * C + c] = acc;
+                }
+                __syncthreads();
+            }
+        } else {
+            // X0 = sum_{p<=m} (-N)^p with masked powers, N = M (in A)
+            for (int idx = tid; idx < Cl * Cl; idx += NT) {
+                const int i = idx / Cl, j = idx % Cl;
+                const float nij = A[i * C + j];
+                P[i * C + j] = nij;
+                X[i * C + j] = (i == j ? 1.f : 0.f) - (p.neu_order >= 1 ? nij : 0.f);
+            }
+            __syncthreads();
+            for (int pw = 2; pw <= p.neu_order; ++pw) {
+                const float sgn = (pw & 1) ? -1.f : 1.f;
+                for (int r0 = 0; r0 < Cl; r0 += LB) {
+                    const int nr = min(LB, Cl - r0);
+                    for (int idx = tid; idx < nr * Cl; idx += NT) {
+                        const int r = idx / Cl, c = idx % Cl, i = r0 + r;
+                        float acc = 0.f;
+                        if (i - c >= pw)   // mask: (N^p)_ic = 0 when i - c < p
+                            for (int l = c + 1; l < i; ++l)
+                                acc += P[i * C + l] * A[l * C + c];
+                        blk[r * C + c] = acc;
+                    }
+                    __syncthreads();
+                    for (int idx = tid; idx < nr * Cl; idx += NT) {
+                        const int r = idx / Cl, c = idx % Cl, i = r0 + r;
+                        P[i * C + c] = blk[r * C + c];
+                        X[i * C + c] += sgn * blk[r * C + c];
+                    }
+                    __syncthreads();
+                }
+            }
+            for (int s = 0; s < p.neu_resid; ++s) {
+                // residual Rm = I - (I + N) X  (into P)
+                for (int idx = tid; idx < Cl * Cl; idx += NT) {
+                    const int i = idx / Cl, c = idx % Cl;
+                    float acc = (i == c ? 1.f : 0.f) - X[i * C + c];
+                    for (int l = 0; l < Cl; ++l)
+                        acc -= A[i * C + l] * X[l * C + c];
+                    P[i * C + c] = acc;
+                }
+                __syncthreads();
+                // Newton correction X <- X + X Rm, one row block at a time
+                for (int r0 = 0; r0 < Cl; r0 += LB) {
+                    const int nr = min(LB, Cl - r0);
+                    for (int idx = tid; idx < nr * Cl; idx += NT) {
+                        const int r = idx / Cl, c = idx % Cl, i = r0 + r;
+                        float acc = X[i * C + c];
+                        for (int l = 0; l < Cl; ++l)
+                            acc += X[i * C + l] * P[l * C + c];
+                        blk[r * C + c] = acc;
+                    }
+                    __syncthreads();
+                    for (int idx = tid; idx < nr * Cl; idx += NT) {
+                        const int r = idx / Cl, c = idx % Cl;
+                        X[(r0 + r) * C + c] = blk[r * C + c];
+                    }
+                    __syncthreads();
+                }
+            }
+        }
+        const float *Ai = neu ? X : A;
+        // --- RHS = V - Kbar S and Qbar S, Kbar_t = k_t e^{Lambda_t}, Qbar_t = q_t e^{Lambda_t}
+        for (int idx = tid; idx < Cl * (NV / 8); idx += NT) {
+            const int t = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
+            float ar[8], aq[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                ar[u] = aq[u] = 0.f;
+            const long kt = (kh * T + c0 + t) * dk;
+            for (int i = 0; i < dk; ++i) {
+                const float e = expf(lam[t * G + i / width]);
+                const float kb = ld_in<IN_BF16>(p.k, kt + i) * e;
+                const float qb = ld_in<IN_BF16>(p.q, kt + i) * e;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float s = S[i * NV + nb + u];
+                    ar[u] += kb * s;
+                    aq[u] += qb * s;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int n = nb + u;
+                const float vv = (n < nv) ? ld_in<IN_BF16>(p.v, (vh * T + c0 + t) * dv + n0 + n) : 0.f;
+                rhs[t * NV + n] = vv - ar[u];
+                qs[t * NV + n] = aq[u];
+            }
+        }
+        __syncthreads();
+        // --- E = diag(beta) A RHS
+        for (int idx = tid; idx < Cl * NV; idx += NT) {
+            const int t = idx / NV, n = idx % NV;
+            float acc = 0.f;
+            for (int j = 0; j <= t; ++j)
+                acc += Ai[t * C + j] * rhs[j * NV + n];
+            E[t * NV + n] = sbeta[t] * acc;
+        }
+        __syncthreads();
+        // --- O = Qbar S + L E, L formed one row block at a time
+        for (int r0 = 0; r0 < Cl; r0 += LB) {
+            const int nr = min(LB, Cl - r0);
+            for (int idx = tid; idx < nr * Cl; idx += NT) {
+                const int r = idx / Cl, j = idx % Cl, t = r0 + r;
+                float l = 0.f;
+                if (j <= t) {
+                    const long qt = (kh * T + c0 + t) * dk, kj = (kh * T + c0 + j) * dk;
+                    for (int gi = 0; gi < G; ++gi) {
+                        float s = 0.f;
+                        for (int i = gi * width; i < (gi + 1) * width; ++i)
+                            s += ld_in<IN_BF16>(p.q, qt + i) * ld_in<IN_BF16>(p.k, kj + i);
+                        l += expf(lam[t * G + gi] - lam[j * G + gi]) * s;
+                    }
+                }
+                blk[r * C + j] = l;
+            }
+            __syncthreads();
+            for (int idx = tid; idx < nr * NV; idx += NT) {
+                const int r = idx / NV, n = idx % NV, t = r0 + r;
+                if (n < nv) {
+                    float acc = qs[t * NV + n];
+                    for (int j = 0; j <= t; ++j)
+                        acc += blk[r * C + j] * E[j * NV + n];
+                    st_out<OUT_BF16>(p.o, (vh * T + c0 + t) * dv + n0 + n, acc);
+                }
+            }
+            __syncthreads();
+        }
+        // --- S <- F S + Khat^T E,  F = e^{Lambda_C}, Khat_t = k_t e^{Lambda_C - Lambda_t}
+        for (int idx = tid; idx < dk * (NV / 8); idx += NT) {
+            const int i = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
+            const float lc = lam[(Cl - 1) * G + i / width];
+            const float f = expf(lc);
+            float acc[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                acc[u] = f * S[i * NV + nb + u];
+            for (int t = 0; t < Cl; ++t) {
+                const float w = ld_in<IN_BF16>(p.k, (kh * T + c0 + t) * dk + i) *
+                                expf(lc - lam[t * G + i / width]);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    acc[u] += w * E[t * NV + nb + u];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                S[i * NV + nb + u] = acc[u];
+        }
+    }
+    __syncthreads();
+    if (p.S_final != nullptr)
+        for (int idx = tid; idx < dk * NV; idx += NT) {
+            const int i = idx / NV, n = idx % NV;
+            if (n < nv)
+                p.S_final[(vh * dk + i) * dv + n0 + n] = S[idx];
+        }
+}
+
+template <bool I, bool O>
+int launch_variant(const Params &p, int smem, cudaStream_t stream)
+{
+    auto kern = simt_fwd_kernel<I, O>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 6;  // GDR_ERR_CUDA
+    dim3 grid((p.dv + NV - 1) / NV, p.Hv, p.B);
+    kern<<<grid, NT, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? 0 : 6;
+}
+
+}  // namespace
+
+int simt_smem_bytes(const Params &p)
+{
+    return simt_layout(p.C, p.G, p.dk, p.neumann != 0).total * (int)sizeof(float);
+}
+
+int launch_simt(const Params &p, cudaStream_t stream)
+{
+    const int smem = simt_smem_bytes(p);
+    if (smem > 227 * 1024)
+        return 5;  // GDR_ERR_UNSUPPORTED
+    if (p.in_bf16) {
+        return p.out_bf16 ? launch_variant<true, true>(p, smem, stream)
+                          : launch_variant<true, false>(p, smem, stream);
+    }
+    return p.out_bf16 ? launch_variant<false, true>(p, smem, stream)
+                      : launch_variant<false, false>(p, smem, stream);
+}
+
+}  // namespace gdr

@@ -1,0 +1,190 @@
+"""Thin ctypes binding of libgdr.so (C ABI in include/gdr.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libgdr.so.  PyTorch supplies device memory and streams.  There is
+no fallback: if the library is missing or the request is rejected, the call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgdr.so")
+
+# gdr_status
+OK, ERR_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, \
+    ERR_NONFINITE = range(9)
+# gdr_dtype
+F32, BF16 = 0, 1
+# gdr_gate_mode
+GATE_SCALAR, GATE_GROUP64, GATE_CHANNEL = 0, 1, 2
+# gdr_inverse_mode
+INV_EXACT, INV_NEUMANN = 0, 1
+# gdr_kernel
+KERNEL_AUTO, KERNEL_SIMT, KERNEL_TC = 0, 1, 2
+
+_KERNELS = {"auto": KERNEL_AUTO, "simt": KERNEL_SIMT, "tc": KERNEL_TC}
+_INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN}
+
+# Every symbol include/gdr.h declares.
+EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_select_kernel", "gdr_device_status",
+           "gdr_status_string", "gdr_version")
+
+
+class GdrShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("Hk", ctypes.c_int),
+                ("Hv", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
+                ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("neumann_order", ctypes.c_int), ("neumann_residual_steps", ctypes.c_int),
+                ("kernel", ctypes.c_int)]
+
+
+class GdrIO(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("S0", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("S_final", ctypes.c_void_p)]
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status: int, what: str = "gdr_chunk_fwd"):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libgdr.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("libgdr.so not found at %s; build it with "
+                           "`python -m gated_delta_rule_141_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.gdr_chunk_fwd.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i, i,
+                                  vp, vp, vp]
+    lib.gdr_chunk_fwd.restype = i
+    lib.gdr_chunk_fwd_host.argtypes = [ctypes.POINTER(GdrShape), ctypes.POINTER(GdrIO),
+                                       ctypes.POINTER(GdrIO), i, i, i, vp]
+    lib.gdr_chunk_fwd_host.restype = i
+    lib.gdr_select_kernel.argtypes = [ctypes.POINTER(GdrShape), i, i, i]
+    lib.gdr_select_kernel.restype = i
+    lib.gdr_device_status.argtypes = [vp]
+    lib.gdr_device_status.restype = i
+    lib.gdr_status_string.argtypes = [i]
+    lib.gdr_status_string.restype = ctypes.c_char_p
+    lib.gdr_version.argtypes = []
+    lib.gdr_version.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().gdr_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(load().gdr_version())
+
+
+def make_shape(B, T, Hk, Hv, dk, dv, in_dtype=BF16, out_dtype=BF16, neumann_order=4,
+               neumann_residual_steps=1, kernel="auto") -> GdrShape:
+    return GdrShape(int(B), int(T), int(Hk), int(Hv), int(dk), int(dv), int(in_dtype),
+                    int(out_dtype), int(neumann_order), int(neumann_residual_steps),
+                    _KERNELS[kernel] if isinstance(kernel, str) else int(kernel))
+
+
+def gate_mode_for(G: int, dk: int) -> int:
+    if G == 1:
+        return GATE_SCALAR
+    if G == dk:
+        return GATE_CHANNEL
+    if dk % 64 == 0 and G == dk // 64:
+        return GATE_GROUP64
+    raise ValueError("no gate mode has G=%d for dk=%d" % (G, dk))
+
+
+def select_kernel(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "exact") -> int:
+    return int(load().gdr_select_kernel(ctypes.byref(shape), int(chunk), int(gate_mode),
+                                        _INVERSES[inverse]))
+
+
+def device_status(stream=None) -> int:
+    return int(load().gdr_device_status(_stream_handle(stream)))
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(getattr(stream, "cuda_stream", stream)))
+
+
+def _dtype_code(t):
+    import torch
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float32:
+        return F32
+    raise TypeError("unsupported dtype %s (bf16 or fp32)" % t)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def chunk_fwd(q, k, v, g, beta, S0=None, chunk=64, gate_mode=None, inverse="exact",
+              neumann_order=4, neumann_residual_steps=1, out_dtype=None, o=None,
+              S_final=None, want_state=True, kernel="auto", stream=None):
+    """Chunkwise gated delta-rule forward on the current CUDA device.
+
+    q, k [B,Hk,T,dk] and v [B,Hv,T,dv] (bf16 or fp32, same dtype); g [B,Hk,T,G] and
+    beta [B,Hk,T] fp32; S0 [B,Hv,dk,dv] fp32 or None.  Returns (o, S_final);
+    S_final is None when want_state is False.  Outputs are allocated with torch
+    unless passed in.  Runs asynchronously on `stream` (default: torch's current).
+    """
+    import torch
+    B, Hk, T, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[3]
+    G = g.shape[-1]
+    if gate_mode is None:
+        gate_mode = gate_mode_for(G, dk)
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("S0", S0)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if o is None:
+        o = torch.empty((B, Hv, T, dv), dtype=out_dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    shape = make_shape(B, T, Hk, Hv, dk, dv, _dtype_code(q.dtype), _dtype_code(o.dtype),
+                       neumann_order, neumann_residual_steps, kernel)
+    st = load().gdr_chunk_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                              _ptr(beta), _ptr(S0), int(chunk), int(gate_mode),
+                              _INVERSES[inverse], _ptr(o), _ptr(S_final),
+                              _stream_handle(stream))
+    if st != OK:
+        raise GdrError(st)
+    return o, S_final
+
+
+def chunk_fwd_host(host: dict, dev: dict, shape: GdrShape, chunk: int, gate_mode: int,
+                   inverse: str = "exact", stream=None):
+    """gdr_chunk_fwd_host: inputs/outputs in (pinned) host tensors, device buffers
+    supplied by the caller.  Both dicts map q, k, v, g, beta, S0, o, S_final to
+    tensors (S0 / S_final may be None)."""
+    names = ("q", "k", "v", "g", "beta", "S0", "o", "S_final")
+    h = GdrIO(*[_ptr(host.get(n)) for n in names])
+    d = GdrIO(*[_ptr(dev.get(n)) for n in names])
+    st = load().gdr_chunk_fwd_host(ctypes.byref(shape), ctypes.byref(h), ctypes.byref(d),
+                                   int(chunk), int(gate_mode), _INVERSES[inverse],
+                                   _stream_handle(stream))
+    if st != OK:
+        raise GdrError(st, "gdr_chunk_fwd_host")

@@ -1,0 +1,136 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Bounds (relative error max|x - x_ref| / max|x_ref| on o and
+S_final): 1e-4 for the fp32 path, 2e-2 for bf16 inputs with fp32 state and
+accumulation.  Neumann mode is compared with the oracle's chunked Neumann form
+(same order and residual steps); its distance from the exact inverse is
+reported separately."""
+import numpy as np
+import pytest
+
+import gpu_util as U
+from gated_delta_rule_141_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from gated_delta_rule_141_b200 import build as gdr_build
+    gdr_build.build()
+
+
+# (workload index, overrides, chunk, inverse, kernel)
+SMALL = [
+    # fp32 path, tiny GDN workload at its own size (the whole workload, every output)
+    (0, {}, 64, "exact", "auto"),
+    (0, {}, 64, "exact", "simt"),
+    # ragged last chunk, odd sizes, S0 present, fp32
+    (0, dict(T=203, Hk=1, Hv=3, dv=40, s0_std=0.5), 64, "exact", "simt"),
+    (0, dict(T=77, dk=32, dv=16, s0_std=0.3), 16, "exact", "simt"),
+    (0, dict(T=130, gate_mode=W.GATE_CHANNEL), 32, "neumann", "simt"),
+    # bf16 inputs, each gate mode, both inverse modes, shrunk workloads
+    (1, dict(B=1, Hk=2, Hv=2, T=320), 64, "exact", "auto"),
+    (1, dict(B=1, Hk=2, Hv=2, T=320), 64, "exact", "simt"),
+    (2, dict(B=1, Hk=2, Hv=2, T=448), 64, "exact", "auto"),
+    (2, dict(B=1, Hk=2, Hv=2, T=448), 64, "neumann", "auto"),
+    (3, dict(B=1, Hk=2, Hv=8, T=384), 64, "exact", "auto"),
+    (3, dict(B=1, Hk=2, Hv=8, T=384), 64, "neumann", "auto"),
+    (3, dict(B=1, Hk=1, Hv=4, T=384, chunk=128), 128, "exact", "auto"),
+    (4, dict(Hk=2, Hv=2, T=640), 128, "exact", "auto"),
+    (4, dict(Hk=2, Hv=2, T=704 - 37), 128, "exact", "auto"),
+]
+
+
+@pytest.mark.parametrize("idx,over,chunk,inverse,kernel", SMALL,
+                         ids=["w%d-%s-C%d-%s-%s" % (c[0], "-".join("%s%s" % kv for kv in c[1].items())
+                                                     or "full", c[2], c[3], c[4]) for c in SMALL])
+def test_small_parity(idx, over, chunk, inverse, kernel):
+    w, x = W.workload_inputs(idx, **over)
+    o, Sf = U.run_gpu(x, w.in_dtype, chunk, inverse, kernel=kernel)
+    o_ref, S_ref = U.oracle_reference(x, chunk, inverse)
+    tol = U.tol_for(w.in_dtype)
+    eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
+    print("rel err o %.3e  S_final %.3e  (tol %.0e)" % (eo, es, tol))
+    assert eo <= tol and es <= tol
+
+
+def test_edge_cases():
+    # T = 0: no tokens, S_final = S0
+    w, x = W.workload_inputs(0, T=0, s0_std=0.4)
+    o, Sf = U.run_gpu(x, "f32", 64)
+    assert o.shape == (1, 2, 0, 64)
+    assert np.array_equal(Sf, x["S0"].astype(np.float64))
+    # T = 1 and T = C + 1 with and without S0, bf16 in / fp32 out
+    for T in (1, 65):
+        for s0 in (0.0, 0.3):
+            w, x = W.workload_inputs(1, B=1, Hk=1, Hv=1, T=T, s0_std=s0)
+            o, Sf = U.run_gpu(x, "bf16", 64, out_dtype=__import__("torch").float32)
+            o_ref, S_ref = U.oracle_reference(x, 64, "exact")
+            assert U.rel_err(o, o_ref) <= U.TOL_BF16
+            assert U.rel_err(Sf, S_ref) <= U.TOL_BF16
+    # no S_final requested
+    w, x = W.workload_inputs(0, T=64)
+    o, Sf = U.run_gpu(x, "f32", 64, want_state=False)
+    assert Sf is None
+    assert U.rel_err(o, U.oracle_reference(x, 64, "exact")[0]) <= U.TOL_F32
+
+
+def test_host_entry_matches_device_entry():
+    import torch
+    from gated_delta_rule_141_b200 import gdr
+    w, x = W.workload_inputs(1, B=1, Hk=2, Hv=2, T=256)
+    dev_in = U.to_device(x, "bf16")
+    o_dev, S_dev = gdr.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"],
+                                 dev_in["beta"], dev_in["S0"], chunk=64)
+    host = {n: (None if t is None else t.cpu().pin_memory()) for n, t in dev_in.items()}
+    host["o"] = torch.empty(o_dev.shape, dtype=o_dev.dtype).pin_memory()
+    host["S_final"] = torch.empty(S_dev.shape, dtype=torch.float32).pin_memory()
+    dev = {n: (None if t is None else torch.empty_like(t)) for n, t in dev_in.items()}
+    dev["o"] = torch.empty_like(o_dev)
+    dev["S_final"] = torch.empty_like(S_dev)
+    shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv)
+    gdr.chunk_fwd_host(host, dev, shape, 64, gdr.GATE_SCALAR)
+    torch.cuda.synchronize()
+    assert torch.equal(host["o"], o_dev.cpu())
+    assert torch.equal(host["S_final"], S_dev.cpu())
+
+
+# Full-size workloads, in the launch configuration bench.py times, checked on a
+# deterministic sample of sequences that the oracle computes one by one.
+FULL = [
+    (1, 64, "exact"),
+    (2, 64, "exact"),
+    (3, 64, "exact"),
+    (3, 128, "exact"),
+    (3, 64, "neumann"),
+    (3, 128, "neumann"),
+    (4, 128, "exact"),
+    (4, 128, "neumann"),
+]
+
+
+@pytest.mark.parametrize("idx,chunk,inverse", FULL,
+                         ids=["w%d-C%d-%s" % c for c in FULL])
+def test_full_size_sampled(idx, chunk, inverse):
+    w, x = W.workload_inputs(idx)
+    o, Sf = U.run_gpu(x, w.in_dtype, chunk, inverse)
+    assert np.isfinite(o).all() and np.isfinite(Sf).all()
+    seqs = U.sample_sequences(w)
+    xs = U.slice_sequences(x, w.R, seqs)
+    o_ref, S_ref = U.oracle_reference(xs, chunk, inverse)
+    idx_b = [b for b, _ in seqs]
+    idx_h = [h for _, h in seqs]
+    o_s = o[idx_b, idx_h][:, None]
+    S_s = Sf[idx_b, idx_h][:, None]
+    eo, es = U.rel_err(o_s, o_ref), U.rel_err(S_s, S_ref)
+    msg = "rel err o %.3e  S_final %.3e" % (eo, es)
+    if inverse == "neumann":
+        o_ex, S_ex = U.oracle_reference(xs, chunk, "exact")
+        msg += "  | Neumann vs exact: o %.3e  S_final %.3e" % (U.rel_err(o_s, o_ex),
+                                                              U.rel_err(S_s, S_ex))
+    print(msg)
+    tol = U.tol_for(w.in_dtype)
+    assert eo <= tol and es <= tol, msg
