@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Throughput of the chunkwise gated delta-rule forward on B200 GPUs.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--chunk C]
+                [--inverse exact|neumann] [--impl ours|reference]
+
+One step = one gdr_chunk_fwd pass over the whole workload (all sequences, all
+chunks) with inputs resident in HBM.  Prints ONE JSON line on rank 0.
+
+* value: tokens/s (B*T per step) over all ranks; N>1 runs one process per GPU,
+  each rank processing its own copy of the workload (independent sequences, no
+  collective on the data path: weak scaling); time = max over ranks of the
+  CUDA-event time of K steps between barriers.
+* e2e: the same metric through gdr_chunk_fwd_host with pinned host buffers
+  (host->device copies of every input and device->host copies of o and
+  S_final inside the timed region).
+* roofline: algorithmic bytes (or flops) of one launch / its average duration,
+  against the measured peaks in MEASURED_PEAKS.json.
+* cpu_baseline: the fp64 oracle timed on this host's cores on a bounded sample
+  of the same workload (rank 0, N = 1 only).
+* --impl reference: the oracle alone on the host cores (a bounded sample per
+  step), the only comparison arm this method has.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gated_delta_rule_141_b200 import workloads as W  # noqa: E402
+
+METRIC = "tokens/s and TFLOP/s (% of bf16 TC peak) for chunkwise gated-delta fwd, 1 B200"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--inverse", default="exact", choices=["exact", "neumann"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "simt"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work of one pass (per token and key head, summed over the workload)
+def algorithmic(w: W.Workload, chunk: int, inverse: str, order=4, resid=1):
+    C, dk, Dv, G = chunk, w.dk, w.R * w.dv, w.G
+    s_in = 4 if w.in_dtype == "f32" else 2
+    s_out = s_in
+    inv = C * C / 3.0 if inverse == "exact" else (order - 1 + 2 * resid) * C * C / 3.0
+    flop_tok = 3 * C * dk + 2 * C * Dv + 6 * dk * Dv + inv
+    byte_tok = 2 * dk * s_in + Dv * s_in + Dv * s_out + 4 * G + 4
+    units = w.B * w.Hk * w.T
+    state = w.B * w.Hk * dk * Dv * 4 * (2 if w.s0_std > 0 else 1)
+    return flop_tok * units, byte_tok * units + state
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_fingerprint():
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "gated_delta_rule_141_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(workload_name: str, chunk: int, inverse: str):
+    """dram bytes per launch from a committed ncu summary of the same kernel
+    build (profiles/traffic.json), or None if absent or stale."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get("%s/C%d/%s" % (workload_name, chunk, inverse))
+    if not e or e.get("fingerprint") != kernel_fingerprint():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, flag in zip(names, parts[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * (mx or max(sm))] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def oracle_sample(w: W.Workload, x: dict, chunk: int, inverse: str, budget_s: float = 12.0):
+    """Time the fp64 oracle on a bounded sample of the workload's sequences on
+    all host cores.  Returns (tokens/s equivalent, threads, description)."""
+    import oracle
+    threads = max(1, oracle.max_threads())
+    total = w.B * w.Hv
+
+    def run(n):
+        seqs = [(s // w.Hv, s % w.Hv) for s in range(n)]
+        xs = {}
+        for name in ("q", "k", "g", "beta"):
+            xs[name] = np.stack([x[name][b, hv // w.R] for b, hv in seqs])[:, None]
+        xs["v"] = np.stack([x["v"][b, hv] for b, hv in seqs])[:, None]
+        xs["S0"] = None if x["S0"] is None else np.stack([x["S0"][b, hv] for b, hv in seqs])[:, None]
+        t0 = time.perf_counter()
+        if inverse == "exact":
+            oracle.recurrent(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["S0"],
+                             nthreads=threads)
+        else:
+            oracle.chunked(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["S0"],
+                           chunk=chunk, inverse="neumann", nthreads=threads)
+        return time.perf_counter() - t0
+
+    n = min(total, threads)
+    dt = run(n)
+    # grow the sample (multiples of the thread count) towards the time budget
+    want = int(n * max(1.0, budget_s / max(dt, 1e-3)))
+    n2 = min(total, max(n, (want // threads) * threads))
+    if n2 > n:
+        dt = run(n2)
+        n = n2
+    tokens = n * w.T / w.Hv            # value-head sequences -> tokens of B*T
+    kind = "recurrent" if inverse == "exact" else "chunked-neumann"
+    desc = "%d of %d (batch, value-head) sequences, all %d tokens each, fp64 %s" % (
+        n, total, w.T, kind)
+    return tokens / dt, threads, desc, dt
+
+
+# ---------------------------------------------------------------------------
+def run_reference(args, w, chunk, rank):
+    if rank != 0:
+        return 0
+    x = W.make_inputs(w, 1000 + args.workload)
+    times, rate_list = [], []
+    desc, threads = "", 1
+    for step in range(args.warmup + args.steps):
+        rate, threads, desc, dt = oracle_sample(w, x, chunk, args.inverse, budget_s=2.0)
+        if step >= args.warmup:
+            rate_list.append(rate)
+            times.append(dt)
+    value = statistics.median(rate_list)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, chunk, args.inverse, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, chunk, inverse, world):
+    in_bytes = (w.B * w.T * (2 * w.Hk * w.dk + w.Hv * w.dv) * (2 if w.in_dtype == "bf16" else 4)
+                + w.B * w.Hk * w.T * (w.G + 1) * 4)
+    return {"workload": w.name, "B": w.B, "T": w.T, "Hk": w.Hk, "Hv": w.Hv, "dk": w.dk,
+            "dv": w.dv, "G": w.G, "chunk": chunk, "inverse": inverse,
+            "in_dtype": w.in_dtype, "S0": w.s0_std > 0,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": ("inputs larger than L2" if in_bytes >= L2_BYTES
+                   else "L2 flushed between steps")}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = W.WORKLOADS[args.workload]
+    chunk = args.chunk or w.chunk
+    if args.impl == "reference":
+        return run_reference(args, w, chunk, rank)
+
+    import torch
+    from gated_delta_rule_141_b200 import gdr
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    x = W.make_inputs(w, 1000 + args.workload + 7919 * rank)
+    dt_in = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
+    dev = {n: torch.from_numpy(x[n]).to("cuda").to(dt_in) for n in ("q", "k", "v")}
+    dev["g"] = torch.from_numpy(x["g"]).cuda()
+    dev["beta"] = torch.from_numpy(x["beta"]).cuda()
+    dev["S0"] = None if x["S0"] is None else torch.from_numpy(x["S0"]).cuda()
+    o = torch.empty((w.B, w.Hv, w.T, w.dv), dtype=dt_in, device="cuda")
+    Sf = torch.empty((w.B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    in_bytes = sum(t.numel() * t.element_size() for t in dev.values() if t is not None)
+    flush = None
+    if in_bytes < L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    # with an L2 flush between steps, only the launches themselves are timed
+    step_events = []
+
+    def step(timed=False):
+        if flush is not None:
+            flush.zero_()
+        if timed and flush is not None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        gdr.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
+                      chunk=chunk, inverse=args.inverse, o=o, S_final=Sf, kernel=args.kernel,
+                      stream=stream)
+        if timed and flush is not None:
+            e1.record(stream)
+            step_events.append((e0, e1))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if gdr.device_status(stream) != gdr.OK:
+        raise RuntimeError("device status reported a timeout during warm-up")
+
+    sampler = ClockSampler(local)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(timed=True)
+        ev1.record(stream)
+        barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    if step_events:
+        ms_total = sum(a.elapsed_time(b) for a, b in step_events)
+    if dist is not None:
+        t = torch.tensor([ms_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_step = w.B * w.T
+    value = world * tokens_step / (ms_step * 1e-3)
+
+    # kernel-only launch time, for the roofline (no L2 flush between launches
+    # when the inputs exceed L2 anyway)
+    flop, byts = algorithmic(w, chunk, args.inverse)
+    peaks, peak_src = measured_peaks()
+    hbm_frac = (byts / (ms_step * 1e-3)) / (peaks["hbm_gbs"] * 1e9)
+    tc_frac = (flop / (ms_step * 1e-3)) / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if byts / (peaks["hbm_gbs"] * 1e9) >= flop / (peaks["bf16_tflops"] * 1e12) else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": byts / (ms_step * 1e-3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm_frac}
+    else:
+        roof = {"bound": "tensor", "achieved": flop / (ms_step * 1e-3) / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tc_frac}
+    roof["peak_source"] = peak_src + " (burst)"
+    roof["traffic"] = recorded_traffic(w.name, chunk, args.inverse)
+    roof["tflops"] = flop / (ms_step * 1e-3) / 1e12
+    roof["tc_frac"] = tc_frac
+    roof["hbm_frac"] = hbm_frac
+
+    # end to end through the host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        host = {n: (None if t is None else t.cpu().pin_memory()) for n, t in dev.items()}
+        host["o"] = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        host["S_final"] = torch.empty(Sf.shape, dtype=torch.float32).pin_memory()
+        dbuf = {n: (None if t is None else torch.empty_like(t)) for n, t in dev.items()}
+        dbuf["o"], dbuf["S_final"] = torch.empty_like(o), torch.empty_like(Sf)
+        shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
+                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                               kernel=args.kernel)
+        gm = gdr.gate_mode_for(w.G, w.dk)
+        h2d = sum(t.numel() * t.element_size() for n, t in host.items()
+                  if t is not None and n not in ("o", "S_final"))
+        d2h = host["o"].numel() * host["o"].element_size() + host["S_final"].numel() * 4
+        e2e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, stream)
+        barrier()
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, stream)
+        ev1.record(stream)
+        barrier()
+        ms_e2e = ev0.elapsed_time(ev1)
+        if dist is not None:
+            t = torch.tensor([ms_e2e], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * tokens_step / (ms_e2e / e2e_steps * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, desc, _ = oracle_sample(w, x, chunk, args.inverse)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    kern = gdr.select_kernel(gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
+                                            gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                                            gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                                            kernel=args.kernel),
+                             chunk, gdr.gate_mode_for(w.G, w.dk), args.inverse)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.in_dtype == "bf16" else "f32",
+        "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
+        "config": config_dict(w, chunk, args.inverse, world),
+        "tflops": roof["tflops"], "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps, "kernel": {1: "simt", 2: "tc"}.get(kern, str(kern)),
+        "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
