@@ -589,6 +589,8 @@ int launch_scalar(const Params &p, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }
 
+#include "gdr_tc_ws.cuh"
+
 }  // namespace
 
 bool tc_supports(const Params &p)
@@ -599,6 +601,8 @@ bool tc_supports(const Params &p)
 
 int launch_tc(const Params &p, cudaStream_t stream)
 {
+    if (ws::supports(p))
+        return p.out_bf16 ? ws::launch<true>(p, stream) : ws::launch<false>(p, stream);
     if (p.dk == 64)
         return p.out_bf16 ? launch_scalar<64, true>(p, stream) : launch_scalar<64, false>(p, stream);
     return p.out_bf16 ? launch_scalar<128, true>(p, stream) : launch_scalar<128, false>(p, stream);
