@@ -25,24 +25,28 @@ namespace gdr {
 namespace {
 
 constexpr int NT = 256;  // threads per CTA
-constexpr int NV = 32;   // value columns per CTA
 constexpr int LB = 16;   // rows per row block (L readout, Neumann products)
 
 struct SimtLayout {      // offsets in floats into dynamic shared memory
     int lam, A, P, X, S, rhs, qs, E, blk, beta, row, total;
 };
 
-__host__ __device__ inline SimtLayout simt_layout(int C, int G, int dk, bool neumann)
+// Neumann mode keeps N (in A) and the series X; a third C x C buffer P is only
+// needed for more than one residual step (the single-step correction writes
+// its residual over N).  Q S is staged in X once X has been applied.
+__host__ __device__ inline SimtLayout simt_layout(int C, int G, int dk, bool neumann, int resid,
+                                                  int NV)
 {
     SimtLayout s;
     int off = 0;
     s.lam = off;  off += C * G;
     s.A = off;    off += C * C;
-    s.P = off;    off += neumann ? C * C : 0;
     s.X = off;    off += neumann ? C * C : 0;
+    s.P = off;    off += (neumann && resid > 1) ? C * C : 0;
     s.S = off;    off += dk * NV;
     s.rhs = off;  off += C * NV;
-    s.qs = off;   off += C * NV;
+    s.qs = neumann ? s.X : off;
+    off += neumann ? 0 : C * NV;
     s.E = off;    off += C * NV;
     s.blk = off;  off += LB * C;
     s.beta = off; off += C;
@@ -69,13 +73,13 @@ __device__ __forceinline__ void st_out(void *p, long i, float x)
         static_cast<float *>(p)[i] = x;
 }
 
-template <bool IN_BF16, bool OUT_BF16>
+template <bool IN_BF16, bool OUT_BF16, int NV>
 __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
 {
     extern __shared__ float sm[];
     const int C = p.C, G = p.G, dk = p.dk, dv = p.dv, T = p.T;
     const bool neu = p.neumann != 0;
-    const SimtLayout Ly = simt_layout(C, G, dk, neu);
+    const SimtLayout Ly = simt_layout(C, G, dk, neu, p.neu_resid, NV);
     float *lam = sm + Ly.lam, *A = sm + Ly.A, *P = sm + Ly.P, *X = sm + Ly.X;
     float *S = sm + Ly.S, *rhs = sm + Ly.rhs, *qs = sm + Ly.qs, *E = sm + Ly.E;
     float *blk = sm + Ly.blk, *sbeta = sm + Ly.beta, *row = sm + Ly.row;
@@ -144,53 +148,61 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
                 __syncthreads();
             }
         } else {
-            // X0 = sum_{p<=m} (-N)^p with masked powers, N = M (in A)
+            // X0 = sum_{p<=m} (-N)^p, N = M (in A), by Horner's rule X <- I - N X
+            // (m times from X = I).  N is strictly lower triangular, so row i of
+            // N X reads only rows above i: the update runs in place, one row block
+            // at a time from the bottom up.  This equals the sum of the masked
+            // powers of N (the masks only drop entries that are exactly zero).
             for (int idx = tid; idx < Cl * Cl; idx += NT) {
                 const int i = idx / Cl, j = idx % Cl;
-                const float nij = A[i * C + j];
-                P[i * C + j] = nij;
-                X[i * C + j] = (i == j ? 1.f : 0.f) - (p.neu_order >= 1 ? nij : 0.f);
+                X[i * C + j] = (i == j) ? 1.f : 0.f;
             }
             __syncthreads();
-            for (int pw = 2; pw <= p.neu_order; ++pw) {
-                const float sgn = (pw & 1) ? -1.f : 1.f;
-                for (int r0 = 0; r0 < Cl; r0 += LB) {
+            for (int pw = 1; pw <= p.neu_order; ++pw) {
+                for (int r0 = ((Cl - 1) / LB) * LB; r0 >= 0; r0 -= LB) {
                     const int nr = min(LB, Cl - r0);
                     for (int idx = tid; idx < nr * Cl; idx += NT) {
                         const int r = idx / Cl, c = idx % Cl, i = r0 + r;
-                        float acc = 0.f;
-                        if (i - c >= pw)   // mask: (N^p)_ic = 0 when i - c < p
-                            for (int l = c + 1; l < i; ++l)
-                                acc += P[i * C + l] * A[l * C + c];
+                        float acc = (i == c) ? 1.f : 0.f;
+                        for (int l = c; l < i; ++l)
+                            acc -= A[i * C + l] * X[l * C + c];
                         blk[r * C + c] = acc;
                     }
                     __syncthreads();
                     for (int idx = tid; idx < nr * Cl; idx += NT) {
-                        const int r = idx / Cl, c = idx % Cl, i = r0 + r;
-                        P[i * C + c] = blk[r * C + c];
-                        X[i * C + c] += sgn * blk[r * C + c];
+                        const int r = idx / Cl, c = idx % Cl;
+                        X[(r0 + r) * C + c] = blk[r * C + c];
                     }
                     __syncthreads();
                 }
             }
             for (int s = 0; s < p.neu_resid; ++s) {
-                // residual Rm = I - (I + N) X  (into P)
-                for (int idx = tid; idx < Cl * Cl; idx += NT) {
-                    const int i = idx / Cl, c = idx % Cl;
-                    float acc = (i == c ? 1.f : 0.f) - X[i * C + c];
-                    for (int l = 0; l < Cl; ++l)
-                        acc -= A[i * C + l] * X[l * C + c];
-                    P[i * C + c] = acc;
+                // residual Rm = I - (I + N) X; the last step may overwrite N
+                float *Rm = (s + 1 < p.neu_resid) ? P : A;
+                for (int r0 = 0; r0 < Cl; r0 += LB) {
+                    const int nr = min(LB, Cl - r0);
+                    for (int idx = tid; idx < nr * Cl; idx += NT) {
+                        const int r = idx / Cl, c = idx % Cl, i = r0 + r;
+                        float acc = (i == c ? 1.f : 0.f) - X[i * C + c];
+                        for (int l = c; l < i; ++l)
+                            acc -= A[i * C + l] * X[l * C + c];
+                        blk[r * C + c] = acc;
+                    }
+                    __syncthreads();
+                    for (int idx = tid; idx < nr * Cl; idx += NT) {
+                        const int r = idx / Cl, c = idx % Cl;
+                        Rm[(r0 + r) * C + c] = blk[r * C + c];
+                    }
+                    __syncthreads();
                 }
-                __syncthreads();
                 // Newton correction X <- X + X Rm, one row block at a time
                 for (int r0 = 0; r0 < Cl; r0 += LB) {
                     const int nr = min(LB, Cl - r0);
                     for (int idx = tid; idx < nr * Cl; idx += NT) {
                         const int r = idx / Cl, c = idx % Cl, i = r0 + r;
                         float acc = X[i * C + c];
-                        for (int l = 0; l < Cl; ++l)
-                            acc += X[i * C + l] * P[l * C + c];
+                        for (int l = c; l <= i; ++l)
+                            acc += X[i * C + l] * Rm[l * C + c];
                         blk[r * C + c] = acc;
                     }
                     __syncthreads();
@@ -203,31 +215,25 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
             }
         }
         const float *Ai = neu ? X : A;
-        // --- RHS = V - Kbar S and Qbar S, Kbar_t = k_t e^{Lambda_t}, Qbar_t = q_t e^{Lambda_t}
+        // --- RHS = V - Kbar S, Kbar_t = k_t e^{Lambda_t}
         for (int idx = tid; idx < Cl * (NV / 8); idx += NT) {
             const int t = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
-            float ar[8], aq[8];
+            float ar[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                ar[u] = aq[u] = 0.f;
+                ar[u] = 0.f;
             const long kt = (kh * T + c0 + t) * dk;
             for (int i = 0; i < dk; ++i) {
-                const float e = expf(lam[t * G + i / width]);
-                const float kb = ld_in<IN_BF16>(p.k, kt + i) * e;
-                const float qb = ld_in<IN_BF16>(p.q, kt + i) * e;
+                const float kb = ld_in<IN_BF16>(p.k, kt + i) * expf(lam[t * G + i / width]);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float s = S[i * NV + nb + u];
-                    ar[u] += kb * s;
-                    aq[u] += qb * s;
-                }
+                for (int u = 0; u < 8; ++u)
+                    ar[u] += kb * S[i * NV + nb + u];
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int n = nb + u;
                 const float vv = (n < nv) ? ld_in<IN_BF16>(p.v, (vh * T + c0 + t) * dv + n0 + n) : 0.f;
                 rhs[t * NV + n] = vv - ar[u];
-                qs[t * NV + n] = aq[u];
             }
         }
         __syncthreads();
@@ -238,6 +244,25 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
             for (int j = 0; j <= t; ++j)
                 acc += Ai[t * C + j] * rhs[j * NV + n];
             E[t * NV + n] = sbeta[t] * acc;
+        }
+        __syncthreads();
+        // --- Qbar S, Qbar_t = q_t e^{Lambda_t} (staged in X in Neumann mode: X is spent)
+        for (int idx = tid; idx < Cl * (NV / 8); idx += NT) {
+            const int t = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
+            float aq[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                aq[u] = 0.f;
+            const long qt = (kh * T + c0 + t) * dk;
+            for (int i = 0; i < dk; ++i) {
+                const float qb = ld_in<IN_BF16>(p.q, qt + i) * expf(lam[t * G + i / width]);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    aq[u] += qb * S[i * NV + nb + u];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                qs[t * NV + nb + u] = aq[u];
         }
         __syncthreads();
         // --- O = Qbar S + L E, L formed one row block at a time
@@ -299,10 +324,10 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
         }
 }
 
-template <bool I, bool O>
+template <bool I, bool O, int NV>
 int launch_variant(const Params &p, int smem, cudaStream_t stream)
 {
-    auto kern = simt_fwd_kernel<I, O>;
+    auto kern = simt_fwd_kernel<I, O, NV>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 6;  // GDR_ERR_CUDA
     dim3 grid((p.dv + NV - 1) / NV, p.Hv, p.B);
@@ -310,24 +335,41 @@ int launch_variant(const Params &p, int smem, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }
 
+constexpr int kMaxSmem = 227 * 1024;
+
+int smem_for(const Params &p, int NV)
+{
+    return simt_layout(p.C, p.G, p.dk, p.neumann != 0, p.neu_resid, NV).total * (int)sizeof(float);
+}
+
+template <int NV>
+int launch_nv(const Params &p, int smem, cudaStream_t stream)
+{
+    if (p.in_bf16)
+        return p.out_bf16 ? launch_variant<true, true, NV>(p, smem, stream)
+                          : launch_variant<true, false, NV>(p, smem, stream);
+    return p.out_bf16 ? launch_variant<false, true, NV>(p, smem, stream)
+                      : launch_variant<false, false, NV>(p, smem, stream);
+}
+
 }  // namespace
 
+// Shared memory of the widest value tile (32, else 16 columns) that fits.
 int simt_smem_bytes(const Params &p)
 {
-    return simt_layout(p.C, p.G, p.dk, p.neumann != 0).total * (int)sizeof(float);
+    const int s32 = smem_for(p, 32);
+    return s32 <= kMaxSmem ? s32 : smem_for(p, 16);
 }
 
 int launch_simt(const Params &p, cudaStream_t stream)
 {
-    const int smem = simt_smem_bytes(p);
-    if (smem > 227 * 1024)
-        return 5;  // GDR_ERR_UNSUPPORTED
-    if (p.in_bf16) {
-        return p.out_bf16 ? launch_variant<true, true>(p, smem, stream)
-                          : launch_variant<true, false>(p, smem, stream);
-    }
-    return p.out_bf16 ? launch_variant<false, true>(p, smem, stream)
-                      : launch_variant<false, false>(p, smem, stream);
+    const int s32 = smem_for(p, 32);
+    if (s32 <= kMaxSmem)
+        return launch_nv<32>(p, s32, stream);
+    const int s16 = smem_for(p, 16);
+    if (s16 <= kMaxSmem)
+        return launch_nv<16>(p, s16, stream);
+    return 5;  // GDR_ERR_UNSUPPORTED
 }
 
 }  // namespace gdr

@@ -12,7 +12,7 @@
 // Four roles run them concurrently, handing tiles over through mbarriers:
 //   warp 0       TMA producer (q, k, v tiles; gates) for a 2-stage ring
 //   warp 1       MMA issuer (one thread issues every tcgen05.mma)
-//   warps 2-5    state group: E, S update, O epilogue (S stays in registers)
+//   warps 2-5    state group: E, S update, O epilogue (fp32 S kept in TMEM)
 //   warps 6-13   intra team: gates, Gram read-back, chunk inverse, W read-back
 // MMA operands are stacked so that every MMA has M = 128:
 //   [Q; K] K^T,  [Ab; Abe] V -> U,  [Ab; Abe] K -> W,  [W; Qbar] S -> P, Qbar S,
@@ -39,6 +39,7 @@ constexpr uint32_t T_U = 64;         // [Ab;Abe] V        64 cols (rows 0-63 = U
 constexpr uint32_t T_W = 128;        // [Ab;Abe] K        128 cols (rows 64-127 = W)
 constexpr uint32_t T_PO = 256;       // [W;Qbar] S (+[V;L] E)  rows 0-63 P, 64-127 O
 constexpr uint32_t T_DS = 320;       // K^T E_hat         64 cols
+constexpr uint32_t T_S = 384;        // fp32 state master 64 cols
 constexpr uint32_t TMEM_COLS = 512;
 
 enum Bar { FULL0, FULL1, FREE0, FREE1, GRAM_FULL, GRAM_FREE, AB_READY, WU_FULL, W_READY,
@@ -97,21 +98,29 @@ __device__ __forceinline__ bool named_vote_or(int id, int n, bool pred)
 }
 
 // Bounded wait that also gives up when another role raised the abort flag.
+// Waiting warps back off with short sleeps so that their probes do not crowd
+// the shared-memory pipe that the working roles need.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
                                               volatile int *abort_flag)
 {
     if (ptx::mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = ptx::globaltimer_ns();
-    while (true) {
+    uint32_t nap = 32;
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(nap);
+        if (nap < 256)
+            nap <<= 1;
         if (ptx::mbar_try_wait(bar, parity))
             return true;
-        if (*abort_flag)
-            return false;
-        if (ptx::globaltimer_ns() - t0 > 2000000000ull) {
-            *abort_flag = 1;
-            atomicExch(&g_device_status, kTimeoutStatus);
-            return false;
+        if ((it & 63) == 0) {
+            if (*abort_flag)
+                return false;
+            if (ptx::globaltimer_ns() - t0 > 2000000000ull) {
+                *abort_flag = 1;
+                atomicExch(&g_device_status, kTimeoutStatus);
+                return false;
+            }
         }
     }
 }
@@ -139,13 +148,15 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
     const int T = p.T;
     const int N = (T + CC - 1) / CC;
 
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 4);
-    float *Mf = reinterpret_cast<float *>(base + Ly.Mf);
-    float *Af = reinterpret_cast<float *>(base + Ly.Af);
-    float *Tf = reinterpret_cast<float *>(base + Ly.Tf);
-    auto gates = [&](int s) { return reinterpret_cast<Gates *>(base + Ly.gates[s]); };
+    const uint32_t pad = base_u32 - smem_u32(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + pad + Ly.bar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + pad + Ly.misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + pad + Ly.misc + 4);
+    float *Mf = reinterpret_cast<float *>(smem_raw + pad + Ly.Mf);
+    float *Af = reinterpret_cast<float *>(smem_raw + pad + Ly.Af);
+    float *Tf = reinterpret_cast<float *>(smem_raw + pad + Ly.Tf);
+    Gates *gates0 = reinterpret_cast<Gates *>(smem_raw + pad + Ly.gates[0]);
+    Gates *gates1 = reinterpret_cast<Gates *>(smem_raw + pad + Ly.gates[1]);
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i)
@@ -170,8 +181,8 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
 
     if (warp == W_PROD) {
         // ------------------------------------------------------------ producer
-        bool pend[2] = {false, false};
-        uint32_t pend_par[2] = {0, 0};
+        // outstanding loads per stage: bit s of pend, completion parity in par_s
+        uint32_t pend = 0, par0 = 0, par1 = 0;
         for (int c = 0; c < N; ++c) {
             const int s = c & 1;
             if (c >= 2) {
@@ -181,7 +192,7 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             }
             const long c0 = (long)c * CC;
             const int Cl = (int)min((long)CC, T - c0);
-            Gates *gt = gates(s);
+            Gates *gt = s ? gates1 : gates0;
             for (int t = lane; t < CC; t += 32) {
                 gt->graw[t] = (t < Cl) ? p.g[kh * T + c0 + t] : 0.f;
                 gt->beta[t] = (t < Cl) ? p.beta[kh * T + c0 + t] : 0.f;
@@ -190,20 +201,25 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars[FULL0 + s], 4u * CC * 64 * 2 + CC * NVC * 2);
                 for (int kb = 0; kb < KD / 64; ++kb) {
-                    uint8_t *blk = base + Ly.wqk[s] + kb * 192 * 128;
+                    uint8_t *blk = base + (s ? Ly.wqk[1] : Ly.wqk[0]) + kb * 192 * 128;
                     tma_load_3d(blk + 64 * 128, &tm_q, &bars[FULL0 + s], 64 * kb, (int)c0, (int)kh);
                     tma_load_3d(blk + 128 * 128, &tm_k, &bars[FULL0 + s], 64 * kb, (int)c0, (int)kh);
                 }
-                tma_load_3d(base + Ly.vl[s], &tm_v, &bars[FULL0 + s], n0, (int)c0, (int)vh);
+                tma_load_3d(base + (s ? Ly.vl[1] : Ly.vl[0]), &tm_v, &bars[FULL0 + s], n0, (int)c0, (int)vh);
             }
-            pend[s] = true;
-            pend_par[s] = (c >> 1) & 1;
+            pend |= 1u << s;
+            if (s)
+                par1 = (c >> 1) & 1;
+            else
+                par0 = (c >> 1) & 1;
         }
         // drain loads that may still be landing (bounded)
-        if (lane == 0)
-            for (int s = 0; s < 2; ++s)
-                if (pend[s])
-                    mbar_wait(&bars[FULL0 + s], pend_par[s], 200000000ull);
+        if (lane == 0) {
+            if (pend & 1u)
+                mbar_wait(&bars[FULL0], par0, 200000000ull);
+            if (pend & 2u)
+                mbar_wait(&bars[FULL1], par1, 200000000ull);
+        }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -214,7 +230,7 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             const uint32_t id_ds = idesc_bf16(KD, NVC, true, true);
             const uint32_t ab = base_u32 + Ly.AB;
             auto gram = [&](int s) {
-                const uint32_t t = base_u32 + Ly.wqk[s];
+                const uint32_t t = base_u32 + (s ? Ly.wqk[1] : Ly.wqk[0]);
                 for (int k0 = 0; k0 < KD; k0 += 16)
                     mma_bf16(tmem + T_GRAM, desc_kmajor(t, 192, 64, k0), desc_kmajor(t, 192, 128, k0),
                              id_gram, k0 > 0);
@@ -231,7 +247,7 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             for (int c = 0; c < N && ok; ++c) {
                 const int s = c & 1;
                 const uint32_t par = c & 1;
-                const uint32_t wqk = base_u32 + Ly.wqk[s], vl = base_u32 + Ly.vl[s];
+                const uint32_t wqk = base_u32 + (s ? Ly.wqk[1] : Ly.wqk[0]), vl = base_u32 + (s ? Ly.vl[1] : Ly.vl[0]);
                 if (!(ok = wait_or_abort(&bars[AB_READY], par, abort_flag)))
                     break;
                 tc_fence_after();
@@ -279,21 +295,25 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         // ------------------------------------------------------------ state group
         const int stid = tid - W_STATE0 * 32;
         const int R = 32 * (warp & 3) + lane;    // state row / TMEM lane
-        float sreg[NVC];
 #pragma unroll
-        for (int n = 0; n < NVC; ++n)
-            sreg[n] = 0.f;
-        if (p.S0 != nullptr) {
-            const float *src = p.S0 + (vh * KD + R) * p.dv + n0;
+        for (int cb = 0; cb < NVC; cb += 16) {
+            float sv[16];
 #pragma unroll
-            for (int n = 0; n < NVC; n += 4) {
-                const float4 v4 = *reinterpret_cast<const float4 *>(src + n);
-                sreg[n] = v4.x; sreg[n + 1] = v4.y; sreg[n + 2] = v4.z; sreg[n + 3] = v4.w;
+            for (int n = 0; n < 16; ++n)
+                sv[n] = 0.f;
+            if (p.S0 != nullptr) {
+                const float *src = p.S0 + (vh * KD + R) * p.dv + n0 + cb;
+#pragma unroll
+                for (int n = 0; n < 16; n += 4) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(src + n);
+                    sv[n] = v4.x; sv[n + 1] = v4.y; sv[n + 2] = v4.z; sv[n + 3] = v4.w;
+                }
             }
+            tmem_st16(tq + T_S + cb, sv);
+            st_tile8(base_u32 + Ly.S, KD, R, cb, &sv[0]);
+            st_tile8(base_u32 + Ly.S, KD, R, cb + 8, &sv[8]);
         }
-#pragma unroll
-        for (int n = 0; n < NVC; n += 8)
-            st_tile8(base_u32 + Ly.S, KD, R, n, &sreg[n]);
+        tmem_st_wait();
         fence_proxy_async_smem();
         named_sync(NB_STATE, N_STATE);
         if (stid == 0)
@@ -306,7 +326,7 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             if (named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[P_FULL], par, abort_flag)))
                 break;
             tc_fence_after();
-            const Gates *gt = gates(s);
+            const Gates *gt = s ? gates1 : gates0;
             const float F = gt->ea[CC - 1];
             if (R < CC) {
                 const float f = gt->eb[R];
@@ -337,15 +357,18 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < NVC; cb += 16) {
-                float ds[16];
+                float ds[16], sv[16];
                 tmem_ld16(tq + T_DS + cb, ds);
+                tmem_ld16(tq + T_S + cb, sv);
                 tmem_ld_wait();
 #pragma unroll
                 for (int n = 0; n < 16; ++n)
-                    sreg[cb + n] = F * sreg[cb + n] + ds[n];
-                st_tile8(base_u32 + Ly.S, KD, R, cb, &sreg[cb]);
-                st_tile8(base_u32 + Ly.S, KD, R, cb + 8, &sreg[cb + 8]);
+                    sv[n] = F * sv[n] + ds[n];
+                tmem_st16(tq + T_S + cb, sv);
+                st_tile8(base_u32 + Ly.S, KD, R, cb, &sv[0]);
+                st_tile8(base_u32 + Ly.S, KD, R, cb + 8, &sv[8]);
             }
+            tmem_st_wait();
             if (R >= CC) {
                 const int t = R - CC;
                 const bool live = t < Cl;
@@ -380,8 +403,14 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (p.S_final != nullptr && !*abort_flag) {
             float *dst = p.S_final + (vh * KD + R) * p.dv + n0;
 #pragma unroll
-            for (int n = 0; n < NVC; n += 4)
-                *reinterpret_cast<float4 *>(dst + n) = make_float4(sreg[n], sreg[n + 1], sreg[n + 2], sreg[n + 3]);
+            for (int cb = 0; cb < NVC; cb += 16) {
+                float sv[16];
+                tmem_ld16(tq + T_S + cb, sv);
+                tmem_ld_wait();
+#pragma unroll
+                for (int n = 0; n < 16; n += 4)
+                    *reinterpret_cast<float4 *>(dst + cb + n) = make_float4(sv[n], sv[n + 1], sv[n + 2], sv[n + 3]);
+            }
         }
     } else {
         // ------------------------------------------------------------ intra team
@@ -392,8 +421,8 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         for (int c = 0; c < N; ++c) {
             const int s = c & 1;
             const uint32_t par = c & 1;
-            const uint32_t wqk = base_u32 + Ly.wqk[s], vl = base_u32 + Ly.vl[s];
-            Gates *gt = gates(s);
+            const uint32_t wqk = base_u32 + (s ? Ly.wqk[1] : Ly.wqk[0]), vl = base_u32 + (s ? Ly.vl[1] : Ly.vl[0]);
+            Gates *gt = s ? gates1 : gates0;
             if (named_vote_or(NB_INTRA, N_INTRA,
                               !wait_or_abort(&bars[FULL0 + s], (c >> 1) & 1, abort_flag)))
                 break;
@@ -424,34 +453,39 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             // decay masks: rows 0-63 of the Gram are Q K^T (-> L), rows 64-127 K K^T (-> M)
             {
                 const int j0 = 32 * h;
-                float gv[32];
-                tmem_ld16(tq + T_GRAM + j0, *reinterpret_cast<float(*)[16]>(&gv[0]));
-                tmem_ld16(tq + T_GRAM + j0 + 16, *reinterpret_cast<float(*)[16]>(&gv[16]));
+                float gv0[16], gv1[16];
+                tmem_ld16(tq + T_GRAM + j0, gv0);
+                tmem_ld16(tq + T_GRAM + j0 + 16, gv1);
                 tmem_ld_wait();
-                if (R < CC) {
-                    const int t = R;
-                    const float lt = gt->lam[t];
-                    float lr[32];
+                const bool qrow = R < CC;
+                const int t = qrow ? R : R - CC;
+                const float lt = gt->lam[t];
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int j = j0 + u;
-                        lr[u] = (j <= t) ? __expf(lt - gt->lam[j]) * gv[u] : 0.f;
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int jb = j0 + 16 * hh;
+                    float lj[16], bj[16], out[16];
+#pragma unroll
+                    for (int u = 0; u < 16; u += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(&gt->lam[jb + u]);
+                        const float4 b4 = *reinterpret_cast<const float4 *>(&gt->beta[jb + u]);
+                        lj[u] = l4.x; lj[u + 1] = l4.y; lj[u + 2] = l4.z; lj[u + 3] = l4.w;
+                        bj[u] = b4.x; bj[u + 1] = b4.y; bj[u + 2] = b4.z; bj[u + 3] = b4.w;
                     }
 #pragma unroll
-                    for (int u = 0; u < 32; u += 8)
-                        st_tile8(vl, 128, CC + t, j0 + u, &lr[u]);
-                } else {
-                    const int t = R - CC;
-                    const float lt = gt->lam[t];
+                    for (int u = 0; u < 16; ++u) {
+                        const int j = jb + u;
+                        const float g = hh ? gv1[u] : gv0[u];
+                        const float d = __expf(lt - lj[u]) * g;
+                        out[u] = qrow ? ((j <= t) ? d : 0.f) : ((j < t) ? bj[u] * d : 0.f);
+                    }
+                    if (qrow) {
+                        st_tile8(vl, 128, CC + t, jb, &out[0]);
+                        st_tile8(vl, 128, CC + t, jb + 8, &out[8]);
+                    } else {
 #pragma unroll
-                    for (int u = 0; u < 32; u += 4) {
-                        float m4[4];
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const int j = j0 + u + v;
-                            m4[v] = (j < t) ? gt->beta[j] * __expf(lt - gt->lam[j]) * gv[u + v] : 0.f;
-                        }
-                        *reinterpret_cast<float4 *>(&Mf[t * LDM + j0 + u]) = make_float4(m4[0], m4[1], m4[2], m4[3]);
+                        for (int u = 0; u < 16; u += 4)
+                            *reinterpret_cast<float4 *>(&Mf[t * LDM + jb + u]) =
+                                make_float4(out[u], out[u + 1], out[u + 2], out[u + 3]);
                     }
                 }
             }
@@ -485,8 +519,9 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
                     const float *mrow = Mf + (o + t) * LDM + o;
                     float acc = (t == cc) ? 1.f : 0.f;
 #pragma unroll
-                    for (int j = 0; j < t; ++j)
-                        acc -= mrow[j] * x[j];
+                    for (int j = 0; j < 16; ++j)
+                        if (j < t)
+                            acc -= mrow[j] * x[j];
                     x[t] = acc;
                 }
 #pragma unroll
@@ -497,59 +532,91 @@ ws_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
             // ... merged pairwise: X21 = -X22 (M21 X11), 16 -> 32
             {
                 const int pr = itid >> 7, r = (itid >> 3) & 15, c2 = (itid & 7) * 2, o = 32 * pr;
+                float mr[16];
+#pragma unroll
+                for (int l = 0; l < 16; l += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4 *>(&Mf[(o + 16 + r) * LDM + o + l]);
+                    mr[l] = m4.x; mr[l + 1] = m4.y; mr[l + 2] = m4.z; mr[l + 3] = m4.w;
+                }
                 float t0 = 0.f, t1 = 0.f;
 #pragma unroll
                 for (int l = 0; l < 16; ++l) {
-                    const float m = Mf[(o + 16 + r) * LDM + o + l];
-                    t0 += m * Af[(o + l) * LDM + o + c2];
-                    t1 += m * Af[(o + l) * LDM + o + c2 + 1];
+                    const float2 a2 = *reinterpret_cast<const float2 *>(&Af[(o + l) * LDM + o + c2]);
+                    t0 += mr[l] * a2.x;
+                    t1 += mr[l] * a2.y;
                 }
-                Tf[(pr * 16 + r) * LDT + c2] = t0;
-                Tf[(pr * 16 + r) * LDT + c2 + 1] = t1;
+                *reinterpret_cast<float2 *>(&Tf[(pr * 16 + r) * LDT + c2]) = make_float2(t0, t1);
                 named_sync(NB_INTRA, N_INTRA);
+                float ar[16];
+#pragma unroll
+                for (int l = 0; l < 16; l += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(&Af[(o + 16 + r) * LDM + o + 16 + l]);
+                    ar[l] = a4.x; ar[l + 1] = a4.y; ar[l + 2] = a4.z; ar[l + 3] = a4.w;
+                }
                 float x0 = 0.f, x1 = 0.f;
 #pragma unroll
                 for (int l = 0; l < 16; ++l) {
-                    const float a = Af[(o + 16 + r) * LDM + o + 16 + l];
-                    x0 += a * Tf[(pr * 16 + l) * LDT + c2];
-                    x1 += a * Tf[(pr * 16 + l) * LDT + c2 + 1];
+                    const float2 t2 = *reinterpret_cast<const float2 *>(&Tf[(pr * 16 + l) * LDT + c2]);
+                    x0 += ar[l] * t2.x;
+                    x1 += ar[l] * t2.y;
                 }
-                Af[(o + 16 + r) * LDM + o + c2] = -x0;
-                Af[(o + 16 + r) * LDM + o + c2 + 1] = -x1;
+                *reinterpret_cast<float2 *>(&Af[(o + 16 + r) * LDM + o + c2]) = make_float2(-x0, -x1);
             }
             named_sync(NB_INTRA, N_INTRA);
             // ... and 32 -> 64
             {
                 const int r = itid >> 3, c4 = (itid & 7) * 4;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-                for (int l = 0; l < 32; ++l) {
-                    const float m = Mf[(32 + r) * LDM + l];
+                float mr[32];
+#pragma unroll
+                for (int l = 0; l < 32; l += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4 *>(&Mf[(32 + r) * LDM + l]);
+                    mr[l] = m4.x; mr[l + 1] = m4.y; mr[l + 2] = m4.z; mr[l + 3] = m4.w;
+                }
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
+#pragma unroll
+                for (int l = 0; l < 32; l += 2) {
                     const float4 a = *reinterpret_cast<const float4 *>(&Af[l * LDM + c4]);
-                    acc.x += m * a.x; acc.y += m * a.y; acc.z += m * a.z; acc.w += m * a.w;
+                    const float4 b2 = *reinterpret_cast<const float4 *>(&Af[(l + 1) * LDM + c4]);
+                    acc.x += mr[l] * a.x; acc.y += mr[l] * a.y; acc.z += mr[l] * a.z; acc.w += mr[l] * a.w;
+                    acc2.x += mr[l + 1] * b2.x; acc2.y += mr[l + 1] * b2.y;
+                    acc2.z += mr[l + 1] * b2.z; acc2.w += mr[l + 1] * b2.w;
                 }
-                *reinterpret_cast<float4 *>(&Tf[r * LDT + c4]) = acc;
+                *reinterpret_cast<float4 *>(&Tf[r * LDT + c4]) =
+                    make_float4(acc.x + acc2.x, acc.y + acc2.y, acc.z + acc2.z, acc.w + acc2.w);
                 named_sync(NB_INTRA, N_INTRA);
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-                for (int l = 0; l < 32; ++l) {
-                    const float a = Af[(32 + r) * LDM + 32 + l];
-                    const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[l * LDT + c4]);
-                    x.x += a * t4.x; x.y += a * t4.y; x.z += a * t4.z; x.w += a * t4.w;
+                float ar[32];
+#pragma unroll
+                for (int l = 0; l < 32; l += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(&Af[(32 + r) * LDM + 32 + l]);
+                    ar[l] = a4.x; ar[l + 1] = a4.y; ar[l + 2] = a4.z; ar[l + 3] = a4.w;
                 }
-                *reinterpret_cast<float4 *>(&Af[(32 + r) * LDM + c4]) = make_float4(-x.x, -x.y, -x.z, -x.w);
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), x2 = x;
+#pragma unroll
+                for (int l = 0; l < 32; l += 2) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[l * LDT + c4]);
+                    const float4 u4 = *reinterpret_cast<const float4 *>(&Tf[(l + 1) * LDT + c4]);
+                    x.x += ar[l] * t4.x; x.y += ar[l] * t4.y; x.z += ar[l] * t4.z; x.w += ar[l] * t4.w;
+                    x2.x += ar[l + 1] * u4.x; x2.y += ar[l + 1] * u4.y;
+                    x2.z += ar[l + 1] * u4.z; x2.w += ar[l + 1] * u4.w;
+                }
+                *reinterpret_cast<float4 *>(&Af[(32 + r) * LDM + c4]) =
+                    make_float4(-(x.x + x2.x), -(x.y + x2.y), -(x.z + x2.z), -(x.w + x2.w));
             }
             named_sync(NB_INTRA, N_INTRA);
             // [Ab; Abe] = [diag(beta) A; diag(beta) A diag(e^Lambda)]  (bf16, 128 x 64)
-            for (int u = itid; u < CC * 8; u += N_INTRA) {
+#pragma unroll
+            for (int rep = 0; rep < (CC * 8) / N_INTRA; ++rep) {
+                const int u = itid + rep * N_INTRA;
                 const int t = u >> 3, j = (u & 7) * 8;
                 const float bt = gt->beta[t];
-                float a[8], ae[8];
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    a[v] = bt * Af[t * LDM + j + v];
-                    ae[v] = a[v] * gt->ea[j + v];
-                }
+                const float4 a0 = *reinterpret_cast<const float4 *>(&Af[t * LDM + j]);
+                const float4 a1 = *reinterpret_cast<const float4 *>(&Af[t * LDM + j + 4]);
+                const float4 e0 = *reinterpret_cast<const float4 *>(&gt->ea[j]);
+                const float4 e1 = *reinterpret_cast<const float4 *>(&gt->ea[j + 4]);
+                const float a[8] = {bt * a0.x, bt * a0.y, bt * a0.z, bt * a0.w,
+                                    bt * a1.x, bt * a1.y, bt * a1.z, bt * a1.w};
+                const float ae[8] = {a[0] * e0.x, a[1] * e0.y, a[2] * e0.z, a[3] * e0.w,
+                                     a[4] * e1.x, a[5] * e1.y, a[6] * e1.z, a[7] * e1.w};
                 st_tile8(base_u32 + Ly.AB, 128, t, j, a);
                 st_tile8(base_u32 + Ly.AB, 128, CC + t, j, ae);
             }
