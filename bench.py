@@ -75,6 +75,27 @@ def algorithmic(w: W.Workload, chunk: int, inverse: str, order=4, resid=1):
     return flop_tok * units, byte_tok * units + state
 
 
+def rank_seed(workload_index: int, rank: int) -> int:
+    """Each rank draws its own copy of the workload (weak scaling, independent
+    sequences); rank 0 uses the standard seed."""
+    return 1000 + workload_index + 7919 * rank
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """Slowest rank's time: the whole job is done when the last rank is."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank_step: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own tokens each step."""
+    return world * tokens_per_rank_step / (ms_per_step * 1e-3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -208,7 +229,7 @@ def oracle_sample(w: W.Workload, x: dict, chunk: int, inverse: str, budget_s: fl
 def run_reference(args, w, chunk, rank):
     if rank != 0:
         return 0
-    x = W.make_inputs(w, 1000 + args.workload)
+    x = W.make_inputs(w, rank_seed(args.workload, 0))
     times, rate_list = [], []
     desc, threads = "", 1
     for step in range(args.warmup + args.steps):
@@ -262,7 +283,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    x = W.make_inputs(w, 1000 + args.workload + 7919 * rank)
+    x = W.make_inputs(w, rank_seed(args.workload, rank))
     dt_in = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
     dev = {n: torch.from_numpy(x[n]).to("cuda").to(dt_in) for n in ("q", "k", "v")}
     dev["g"] = torch.from_numpy(x["g"]).cuda()
@@ -314,13 +335,10 @@ def main():
     ms_total = ev0.elapsed_time(ev1)
     if step_events:
         ms_total = sum(a.elapsed_time(b) for a, b in step_events)
-    if dist is not None:
-        t = torch.tensor([ms_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dist, torch.device("cuda", local))
     ms_step = ms_total / args.steps
     tokens_step = w.B * w.T
-    value = world * tokens_step / (ms_step * 1e-3)
+    value = job_tokens_per_s(world, tokens_step, ms_step)
 
     # kernel-only launch time, for the roofline (no L2 flush between launches
     # when the inputs exceed L2 anyway)
@@ -366,12 +384,8 @@ def main():
             gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, stream)
         ev1.record(stream)
         barrier()
-        ms_e2e = ev0.elapsed_time(ev1)
-        if dist is not None:
-            t = torch.tensor([ms_e2e], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * tokens_step / (ms_e2e / e2e_steps * 1e-3), "unit": UNIT,
+        ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), dist, torch.device("cuda", local))
+        e2e = {"value": job_tokens_per_s(world, tokens_step, ms_e2e / e2e_steps), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
