@@ -590,22 +590,29 @@ int launch_scalar(const Params &p, cudaStream_t stream)
 }
 
 #include "gdr_tc_ws.cuh"
+#include "gdr_tc_gen.cuh"
 
 }  // namespace
 
 bool tc_supports(const Params &p)
 {
-    return p.in_bf16 && p.G == 1 && p.C == CH && (p.dk == 64 || p.dk == 128) && p.dv % NV == 0 &&
-           !p.neumann && p.T >= 1 && p.B <= 65535;
+    const bool scalar64 = p.in_bf16 && p.G == 1 && p.C == CH && p.dk == 64 && p.dv % NV == 0 &&
+                          !p.neumann && p.T >= 1 && p.B <= 65535;
+    return ws::supports(p) || scalar64 || gen::supports(p);
 }
 
 int launch_tc(const Params &p, cudaStream_t stream)
 {
     if (ws::supports(p))
         return p.out_bf16 ? ws::launch<true>(p, stream) : ws::launch<false>(p, stream);
+    if (gen::supports(p)) {
+        if (p.dk == 128)
+            return p.out_bf16 ? gen::launch<128, true>(p, stream) : gen::launch<128, false>(p, stream);
+        return p.out_bf16 ? gen::launch<256, true>(p, stream) : gen::launch<256, false>(p, stream);
+    }
     if (p.dk == 64)
         return p.out_bf16 ? launch_scalar<64, true>(p, stream) : launch_scalar<64, false>(p, stream);
-    return p.out_bf16 ? launch_scalar<128, true>(p, stream) : launch_scalar<128, false>(p, stream);
+    return 5;
 }
 
 }  // namespace gdr

@@ -1,0 +1,872 @@
+// gdr_tc_gen.cuh -- tensor-core kernel for grouped and per-channel decay
+// (G = dk/64 or dk), key width 128 or 256, chunk C = 64, exact or truncated
+// Neumann chunk inverse.  Included by gdr_tc.cu.
+//
+// One CTA (256 threads) owns one (batch, value head, 64 value columns) and runs
+// the chunk steps in order ("Systolic Linear Attention: Co-Designing
+// Tile-Grouped Gated Delta Attention for TPUs", §2.1, §2.3 Table 2, §2.4.2):
+//   1. TMA: q, k (as one [q; k] block of 128 rows), v and (for G >= 4) the
+//      chunk's log-gates, zero-filled past T; beta (and the gates when G < 4)
+//      are prefetched a chunk ahead through registers, zero past T.  Zero gates
+//      and beta leave the recurrence untouched.
+//   2. Lambda = cumsum g per decay group.  Decayed operands in place, with the
+//      chunk boundaries as pivots (no division by a decay prefix):
+//        Khat = k e^{Lambda_C - Lambda_t} (<= 1), and for the Gram
+//        Kr = k e^{Lambda_t - Lambda_C}, Qr = q e^{Lambda_t - Lambda_C}, whose
+//      factor is bounded by e^{-Lambda_C}; the kernel uses this single-MMA Gram
+//      only while max_i(-Lambda_C,i) <= 60, and otherwise forms the chunk's
+//      Gram exactly in fp32 from exp(Lambda_t - Lambda_j) (t >= j).
+//   3. tcgen05: [Qr; Kr] Khat^T -> L (rows 0-63) and M (rows 64-127, beta_j).
+//   4. A = (I + M)^{-1}: exact fp32 block doubling in place (16 x 16 diagonal
+//      blocks, merges X21 = -X22 M21 X11), or the truncated Neumann series by
+//      Horner's rule plus Newton residual steps, both products on tcgen05
+//      ("When Good Enough Is Optimal: Multiplication-Only Matrix Inversion
+//      Approximation for Quantized Gated DeltaNet", Lemma 3.1, §4.1).
+//   5. Kbar = Kr e^{Lambda_C} = k e^{Lambda_t}, Qbar likewise (in place).
+//   6. tcgen05: [Qbar; Kbar] S -> Q S, Kbar S;  RHS = V - Kbar S (bf16).
+//   7. tcgen05: E = diag(beta) A RHS   (= U - W S of Table 2).
+//   8. tcgen05: dS = Khat^T E, O = Qbar S + L E;  S <- diag(e^{Lambda_C}) S + dS.
+
+namespace gen {
+
+constexpr int NT = 256;
+constexpr int CC = 64;
+constexpr int NVC = 64;
+constexpr int LDM = 68;
+constexpr float kGrowthLimit = 60.f;
+
+// Widest gate tile per key width: G <= 128 for dk = 128 (per channel); for
+// dk = 256 only the scalar and 64-channel-tile gates (G <= 4) run here.
+__host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
+
+constexpr uint32_t T_G = 0;      // [Qr;Kr] Khat^T : rows 0-63 L', 64-127 M'
+constexpr uint32_t T_Y = 64;     // [Qbar;Kbar] S : rows 0-63 QS (+ L E), 64-127 Kbar S
+constexpr uint32_t T_E = 128;    // [Ab;0] RHS : rows 0-63 E
+constexpr uint32_t T_N = 192;    // Neumann products (M = 64)
+constexpr uint32_t T_DS = 256;   // dS, 64 columns per 128 key channels
+constexpr uint32_t TMEM_COLS = 512;
+
+enum Bar { TMA_QK, TMA_V, TMA_G, MMA, NBARS };
+
+template <int DK>
+struct Plan {
+    uint32_t QK, KH, V, S, L, AB, RHS, E, gates, beta, Mf, Tf, fac, bar, misc, total;
+};
+
+template <int DK>
+__host__ __device__ inline Plan<DK> plan()
+{
+    Plan<DK> s;
+    uint32_t o = 0;
+    auto take = [&](uint32_t bytes) {
+        const uint32_t at = o;
+        o += (bytes + 1023u) & ~1023u;
+        return at;
+    };
+    s.QK = take((DK / 64) * 128 * 128);   // rows 0-63 q, 64-127 k
+    s.KH = take((DK / 64) * 64 * 128);
+    s.V = take(64 * 128);
+    s.S = take(DK * 128);
+    s.L = take(128 * 128);                // rows 64-127 stay zero
+    s.AB = take(128 * 128);               // rows 64-127 stay zero
+    s.RHS = take(64 * 128);
+    s.E = take(64 * 128);
+    s.gates = take(CC * gmax(DK) * 4);    // C x G fp32
+    s.beta = take(CC * 4 + 2 * DK * 4);   // beta, then Lambda_C and e^{Lambda_C} per channel
+    s.Mf = take(CC * LDM * 4);
+    s.Tf = take(32 * 36 * 4);
+    s.fac = take(2 * CC * 8 * 4);         // per (t, group) factors when G <= 8
+    s.bar = take(NBARS * 8 + 16);
+    s.misc = s.bar + NBARS * 8;
+    s.total = o + 1024;
+    return s;
+}
+
+struct GenArgs {
+    Params p;
+    int nvt;
+    int g_flat;                           // G < 4: gates prefetched through registers
+};
+
+// Row of an M = 64 accumulator held by this thread (lanes 0-15 of each quarter).
+__device__ __forceinline__ int row64g(int warp, int lane) { return lane < 16 ? 16 * (warp & 3) + lane : -1; }
+
+// In-place exact inverse of I + M (64 x 64, M strictly lower) by block doubling.
+__device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
+{
+    // diagonal 16 x 16 blocks, exact forward substitution (into Tf, then back)
+    if (tid < 64) {
+        const int blk = tid >> 4, cc = tid & 15, o = 16 * blk;
+        float x[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const float *mrow = Mf + (o + t) * LDM + o;
+            float acc = (t == cc) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (j < t)
+                    acc -= mrow[j] * x[j];
+            x[t] = acc;
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+            Tf[blk * 256 + t * 16 + cc] = x[t];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < 4 * 256; idx += NT) {
+        const int blk = idx >> 8, t = (idx >> 4) & 15, cc = idx & 15;
+        Mf[(16 * blk + t) * LDM + 16 * blk + cc] = Tf[idx];
+    }
+    __syncthreads();
+    // 16 -> 32 (two pairs): T = M21 X11, X21 = -X22 T
+    {
+        const int pr = tid >> 7, r = (tid >> 3) & 15, c2 = (tid & 7) * 2, o = 32 * pr;
+        float mr[16];
+#pragma unroll
+        for (int l = 0; l < 16; l += 4) {
+            const float4 m4 = *reinterpret_cast<const float4 *>(&Mf[(o + 16 + r) * LDM + o + l]);
+            mr[l] = m4.x; mr[l + 1] = m4.y; mr[l + 2] = m4.z; mr[l + 3] = m4.w;
+        }
+        float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {
+            const float2 a2 = *reinterpret_cast<const float2 *>(&Mf[(o + l) * LDM + o + c2]);
+            t0 += mr[l] * a2.x;
+            t1 += mr[l] * a2.y;
+        }
+        __syncthreads();
+        *reinterpret_cast<float2 *>(&Tf[(pr * 16 + r) * 36 + c2]) = make_float2(t0, t1);
+        __syncthreads();
+        float ar[16];
+#pragma unroll
+        for (int l = 0; l < 16; l += 4) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(&Mf[(o + 16 + r) * LDM + o + 16 + l]);
+            ar[l] = a4.x; ar[l + 1] = a4.y; ar[l + 2] = a4.z; ar[l + 3] = a4.w;
+        }
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {
+            const float2 t2 = *reinterpret_cast<const float2 *>(&Tf[(pr * 16 + l) * 36 + c2]);
+            x0 += ar[l] * t2.x;
+            x1 += ar[l] * t2.y;
+        }
+        *reinterpret_cast<float2 *>(&Mf[(o + 16 + r) * LDM + o + c2]) = make_float2(-x0, -x1);
+    }
+    __syncthreads();
+    // 32 -> 64
+    {
+        const int r = tid >> 3, c4 = (tid & 7) * 4;
+        float mr[32];
+#pragma unroll
+        for (int l = 0; l < 32; l += 4) {
+            const float4 m4 = *reinterpret_cast<const float4 *>(&Mf[(32 + r) * LDM + l]);
+            mr[l] = m4.x; mr[l + 1] = m4.y; mr[l + 2] = m4.z; mr[l + 3] = m4.w;
+        }
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
+#pragma unroll
+        for (int l = 0; l < 32; l += 2) {
+            const float4 a = *reinterpret_cast<const float4 *>(&Mf[l * LDM + c4]);
+            const float4 b2 = *reinterpret_cast<const float4 *>(&Mf[(l + 1) * LDM + c4]);
+            acc.x += mr[l] * a.x; acc.y += mr[l] * a.y; acc.z += mr[l] * a.z; acc.w += mr[l] * a.w;
+            acc2.x += mr[l + 1] * b2.x; acc2.y += mr[l + 1] * b2.y;
+            acc2.z += mr[l + 1] * b2.z; acc2.w += mr[l + 1] * b2.w;
+        }
+        *reinterpret_cast<float4 *>(&Tf[r * 36 + c4]) =
+            make_float4(acc.x + acc2.x, acc.y + acc2.y, acc.z + acc2.z, acc.w + acc2.w);
+        __syncthreads();
+        float ar[32];
+#pragma unroll
+        for (int l = 0; l < 32; l += 4) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(&Mf[(32 + r) * LDM + 32 + l]);
+            ar[l] = a4.x; ar[l + 1] = a4.y; ar[l + 2] = a4.z; ar[l + 3] = a4.w;
+        }
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f), x2 = x;
+#pragma unroll
+        for (int l = 0; l < 32; l += 2) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[l * 36 + c4]);
+            const float4 u4 = *reinterpret_cast<const float4 *>(&Tf[(l + 1) * 36 + c4]);
+            x.x += ar[l] * t4.x; x.y += ar[l] * t4.y; x.z += ar[l] * t4.z; x.w += ar[l] * t4.w;
+            x2.x += ar[l + 1] * u4.x; x2.y += ar[l + 1] * u4.y;
+            x2.z += ar[l + 1] * u4.z; x2.w += ar[l + 1] * u4.w;
+        }
+        __syncthreads();
+        *reinterpret_cast<float4 *>(&Mf[(32 + r) * LDM + c4]) =
+            make_float4(-(x.x + x2.x), -(x.y + x2.y), -(x.z + x2.z), -(x.w + x2.w));
+    }
+    __syncthreads();
+}
+
+template <int DK, bool OUT_BF16>
+__global__ void __launch_bounds__(NT, 1)
+gen_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+           const GenArgs args)
+{
+    using namespace ptx;
+    extern __shared__ uint8_t smem_raw[];
+    const Params &p = args.p;
+    const Plan<DK> Ly = plan<DK>();
+    const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t pad = base_u32 - smem_u32(smem_raw);
+    uint8_t *base = smem_raw + pad;
+    float *gts = reinterpret_cast<float *>(smem_raw + pad + Ly.gates);
+    float *sbeta = reinterpret_cast<float *>(smem_raw + pad + Ly.beta);
+    float *lamc = sbeta + CC;          // Lambda_C per channel
+    float *fch = lamc + DK;            // e^{Lambda_C} per channel
+    float *Mf = reinterpret_cast<float *>(smem_raw + pad + Ly.Mf);
+    float *Tf = reinterpret_cast<float *>(smem_raw + pad + Ly.Tf);
+    float *fac = reinterpret_cast<float *>(smem_raw + pad + Ly.fac);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + pad + Ly.bar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + pad + Ly.misc);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nt = blockIdx.x % args.nvt, hv = blockIdx.x / args.nvt, b = blockIdx.y;
+    const int hk = hv / p.R, n0 = nt * NVC;
+    const long kh = (long)b * p.Hk + hk, vh = (long)b * p.Hv + hv;
+    const int T = p.T, G = p.G, width = DK / G;
+    const int N = (T + CC - 1) / CC;
+    const uint32_t QK = base_u32 + Ly.QK, KH = base_u32 + Ly.KH, VT = base_u32 + Ly.V;
+    const uint32_t ST = base_u32 + Ly.S, LT = base_u32 + Ly.L, AB = base_u32 + Ly.AB;
+    const uint32_t RT = base_u32 + Ly.RHS, ET = base_u32 + Ly.E;
+
+    if (tid == 0) {
+        for (int i = 0; i < NBARS; ++i)
+            mbar_init(&bars[i], 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    // zero rows 64-127 of L and [Ab; 0] once (stacked MMA padding)
+    for (int i = tid; i < 64 * 8; i += NT) {
+        const int r = 64 + (i >> 3), c = (i & 7) * 8;
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        st_tile8(LT, 128, r, c, z);
+        st_tile8(AB, 128, r, c, z);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const int half = warp >> 2;
+    const uint32_t gbytes = (uint32_t)(CC * G * 4);
+
+    // phase parities
+    uint32_t ph_qk = 0, ph_v = 0, ph_g = 0, ph_mma = 0;
+    uint32_t pend = 0;     // bit per TMA barrier with a load in flight (thread 0's view)
+    bool failed = false;
+    auto wait_all = [&](int bar, uint32_t &ph) {
+        const bool gave_up = !mbar_wait(&bars[bar], ph);
+        if (!gave_up) {
+            ph ^= 1u;
+            if (bar != MMA)
+                pend &= ~(1u << bar);
+        }
+        if (gave_up)
+            atomicExch(&g_device_status, kTimeoutStatus);
+        return __syncthreads_or(gave_up ? 1 : 0) != 0;
+    };
+    auto issue_qk = [&](int c) {
+        pend |= 1u << TMA_QK;
+        mbar_arrive_expect_tx(&bars[TMA_QK], 2u * CC * DK * 2u);
+        for (int kb = 0; kb < DK / 64; ++kb) {
+            tma_load_3d(base + Ly.QK + kb * 128 * 128, &tm_q, &bars[TMA_QK], 64 * kb, c * CC, (int)kh);
+            tma_load_3d(base + Ly.QK + kb * 128 * 128 + 64 * 128, &tm_k, &bars[TMA_QK], 64 * kb, c * CC, (int)kh);
+        }
+    };
+    auto issue_v = [&](int c) {
+        pend |= 1u << TMA_V;
+        mbar_arrive_expect_tx(&bars[TMA_V], CC * NVC * 2u);
+        tma_load_3d(base + Ly.V, &tm_v, &bars[TMA_V], n0, c * CC, (int)vh);
+    };
+    auto issue_g = [&](int c) {
+        pend |= 1u << TMA_G;
+        mbar_arrive_expect_tx(&bars[TMA_G], gbytes);
+        tma_load_3d(gts, &tm_g, &bars[TMA_G], 0, c * CC, (int)kh);
+    };
+    // beta (and the flattened gates when G < 4) of chunk c, one value per thread
+    float pf_b = 0.f, pf_g = 0.f;
+    auto prefetch_small = [&](int c) {
+        const long cs = (long)c * CC;
+        if (tid < CC)
+            pf_b = (cs + tid < T) ? p.beta[kh * T + cs + tid] : 0.f;
+        if (args.g_flat && tid < CC * G)
+            pf_g = (cs + tid / G < T) ? p.g[(kh * T + cs) * G + tid] : 0.f;
+    };
+    auto mma_sync_wait = [&]() {   // called by all threads after tid 0 committed
+        return wait_all(MMA, ph_mma);
+    };
+
+    // state: row i = 32 * (warp & 3) + lane (+128 for the second half), columns 32*half..+32
+    constexpr int NH = DK / 128;
+    float sreg[NH][32];
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+        const int row = 128 * hh + 32 * (warp & 3) + lane;
+#pragma unroll
+        for (int n = 0; n < 32; ++n)
+            sreg[hh][n] = 0.f;
+        if (p.S0 != nullptr) {
+            const float *src = p.S0 + (vh * DK + row) * p.dv + n0 + 32 * half;
+#pragma unroll
+            for (int n = 0; n < 32; n += 4) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(src + n);
+                sreg[hh][n] = v4.x; sreg[hh][n + 1] = v4.y; sreg[hh][n + 2] = v4.z; sreg[hh][n + 3] = v4.w;
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < 32; n += 8)
+            st_tile8(ST, DK, row, 32 * half + n, &sreg[hh][n]);
+    }
+    if (tid == 0 && N > 0) {
+        prefetch_tensormap(&tm_q);
+        issue_qk(0);
+        issue_v(0);
+        if (!args.g_flat)
+            issue_g(0);
+    }
+    prefetch_small(0);
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    for (int c = 0; c < N && !failed; ++c) {
+        const long c0 = (long)c * CC;
+        const int Cl = (int)min((long)CC, T - c0);
+        if (tid < CC)
+            sbeta[tid] = pf_b;
+        if (args.g_flat && tid < CC * G)
+            gts[tid] = pf_g;
+        if (args.g_flat) {
+            __syncthreads();
+        } else if (wait_all(TMA_G, ph_g)) {
+            failed = true;
+            break;
+        }
+        // ---- Lambda = cumsum over the chunk, one thread per decay group
+        for (int gi = tid; gi < G; gi += NT) {
+            float acc = 0.f;
+            for (int t = 0; t < CC; ++t) {
+                acc += gts[t * G + gi];
+                gts[t * G + gi] = acc;
+            }
+        }
+        __syncthreads();
+        // per-channel Lambda_C, e^{Lambda_C}; growth guard
+        bool strong = false;
+        for (int i = tid; i < DK; i += NT) {
+            const float lc = gts[(CC - 1) * G + i / width];
+            lamc[i] = lc;
+            fch[i] = __expf(lc);
+            strong |= (-lc > kGrowthLimit);
+        }
+        if (G <= 8)
+            for (int u = tid; u < CC * G; u += NT) {
+                const int t = u / G, gi = u % G;
+                const float d = gts[t * G + gi] - gts[(CC - 1) * G + gi];   // Lambda_t - Lambda_C >= 0
+                fac[u] = __expf(-d);                                         // e^{Lambda_C - Lambda_t}
+                fac[CC * 8 + u] = __expf(fminf(d, kGrowthLimit));            // e^{Lambda_t - Lambda_C}
+            }
+        strong = __syncthreads_or(strong ? 1 : 0) != 0;
+        if (wait_all(TMA_QK, ph_qk)) {
+            failed = true;
+            break;
+        }
+        // ---- decayed operands: Khat (new tile), Qr / Kr in place (or raw for the exact Gram)
+        for (int u = tid; u < CC * (DK / 8); u += NT) {
+            const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+            float qv[8], kv[8], kh8[8];
+            ld_tile8(QK, 128, t, i0, qv);
+            ld_tile8(QK, 128, 64 + t, i0, kv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int gi = (i0 + e) / width;
+                float fd, fu;
+                if (G <= 8) {
+                    fd = fac[t * G + gi];
+                    fu = fac[CC * 8 + t * G + gi];
+                } else {
+                    const float d = gts[t * G + gi] - lamc[i0 + e];
+                    fd = __expf(-d);
+                    fu = __expf(fminf(d, kGrowthLimit));
+                }
+                kh8[e] = kv[e] * fd;
+                if (!strong) {
+                    kv[e] *= fu;
+                    qv[e] *= fu;
+                }
+            }
+            st_tile8(KH, 64, t, i0, kh8);
+            if (!strong) {
+                st_tile8(QK, 128, t, i0, qv);
+                st_tile8(QK, 128, 64 + t, i0, kv);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (!strong) {
+            // ---- Gram: [Qr; Kr] Khat^T  (M = 128, N = 64, K = dk)
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, CC, false, false);
+                for (int k0 = 0; k0 < DK; k0 += 16)
+                    mma_bf16(tmem + T_G, desc_kmajor(QK, 128, 0, k0), desc_kmajor(KH, 64, 0, k0), id, k0 > 0);
+                mma_commit(&bars[MMA]);
+            }
+            if (mma_sync_wait()) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            {
+                const int R = 32 * (warp & 3) + lane, j0 = 32 * half;
+                float g0[16], g1[16];
+                tmem_ld16(tq + T_G + j0, g0);
+                tmem_ld16(tq + T_G + j0 + 16, g1);
+                tmem_ld_wait();
+                const bool qrow = R < CC;
+                const int t = qrow ? R : R - CC;
+                float out[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const int j = j0 + u;
+                    const float d = u < 16 ? g0[u] : g1[u - 16];
+                    out[u] = qrow ? ((j <= t) ? d : 0.f) : ((j < t) ? sbeta[j] * d : 0.f);
+                }
+                if (qrow) {
+#pragma unroll
+                    for (int u = 0; u < 32; u += 8)
+                        st_tile8(LT, 128, t, j0 + u, &out[u]);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 32; u += 4)
+                        *reinterpret_cast<float4 *>(&Mf[t * LDM + j0 + u]) =
+                            make_float4(out[u], out[u + 1], out[u + 2], out[u + 3]);
+                }
+            }
+            tc_fence_before();
+            // Kbar = Kr e^{Lambda_C}, Qbar = Qr e^{Lambda_C} (in place)
+            for (int u = tid; u < CC * (DK / 8); u += NT) {
+                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                float qv[8], kv[8];
+                ld_tile8(QK, 128, t, i0, qv);
+                ld_tile8(QK, 128, 64 + t, i0, kv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    qv[e] *= fch[i0 + e];
+                    kv[e] *= fch[i0 + e];
+                }
+                st_tile8(QK, 128, t, i0, qv);
+                st_tile8(QK, 128, 64 + t, i0, kv);
+            }
+        } else {
+            // ---- strong decay: the chunk's Gram exactly in fp32 from the raw tiles
+            for (int u = tid; u < CC * CC; u += NT) {
+                const int t = u / CC, j = u % CC;
+                float m = 0.f, l = 0.f;
+                if (j <= t) {
+                    for (int i0 = 0; i0 < DK; i0 += 8) {
+                        float qv[8], kt8[8], kj8[8];
+                        ld_tile8(QK, 128, t, i0, qv);
+                        ld_tile8(QK, 128, 64 + t, i0, kt8);
+                        ld_tile8(QK, 128, 64 + j, i0, kj8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int gi = (i0 + e) / width;
+                            const float d = __expf(gts[t * G + gi] - gts[j * G + gi]);
+                            m += kt8[e] * kj8[e] * d;
+                            l += qv[e] * kj8[e] * d;
+                        }
+                    }
+                }
+                Mf[t * LDM + j] = (j < t) ? sbeta[j] * m : 0.f;
+                // one bf16 element of L, stored into its place in the swizzled tile
+                const float lv = (j <= t) ? l : 0.f;
+                const uint32_t addr = LT + sw128_off(128, t, j & ~7) + (j & 7) * 2;
+                const uint32_t hi = __float_as_uint(lv);
+                const uint16_t h = static_cast<uint16_t>((hi + 0x7FFFu + ((hi >> 16) & 1u)) >> 16);
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(h));
+            }
+            __syncthreads();
+            // Kbar = k e^{Lambda_t}, Qbar = q e^{Lambda_t}
+            for (int u = tid; u < CC * (DK / 8); u += NT) {
+                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                float qv[8], kv[8];
+                ld_tile8(QK, 128, t, i0, qv);
+                ld_tile8(QK, 128, 64 + t, i0, kv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float f = __expf(gts[t * G + (i0 + e) / width]);
+                    qv[e] *= f;
+                    kv[e] *= f;
+                }
+                st_tile8(QK, 128, t, i0, qv);
+                st_tile8(QK, 128, 64 + t, i0, kv);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        // gates of this chunk are no longer needed except Lambda_C / e^{Lambda_C}: prefetch
+        if (tid == 0 && c + 1 < N && !args.g_flat)
+            issue_g(c + 1);
+        // ---- chunk inverse -> Mf
+        if (!p.neumann) {
+            inverse64_inplace(Mf, Tf, tid);
+        } else {
+            // N (bf16, in the [Ab; 0] tile rows 0-63); X (bf16, in RHS tile); fp32 X in Mf
+            for (int u = tid; u < CC * 8; u += NT) {
+                const int t = u >> 3, j = (u & 7) * 8;
+                float v8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v8[e] = Mf[t * LDM + j + e];
+                st_tile8(AB, 128, t, j, v8);
+                float x8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    x8[e] = (t == j + e) ? 1.f : 0.f;
+                st_tile8(RT, 64, t, j, x8);
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+            const int rr = row64g(warp, lane);
+            const int cb = 32 * half;
+            // Horner: X <- I - N X, `order` times (from X = I)
+            for (int pw = 1; pw <= p.neu_order; ++pw) {
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(64, 64, false, true);
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tmem + T_N, desc_kmajor(AB, 128, 0, k0), desc_mnmajor(RT, 64, k0, 0), id, k0 > 0);
+                    mma_commit(&bars[MMA]);
+                }
+                if (mma_sync_wait()) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                float d0[16], d1[16];
+                tmem_ld16(tq + T_N + cb, d0);
+                tmem_ld16(tq + T_N + cb + 16, d1);
+                tmem_ld_wait();
+                if (rr >= 0) {
+                    float x[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        x[u] = ((rr == cb + u) ? 1.f : 0.f) - (u < 16 ? d0[u] : d1[u - 16]);
+#pragma unroll
+                    for (int u = 0; u < 32; u += 8)
+                        st_tile8(RT, 64, rr, cb + u, &x[u]);
+                    if (pw == p.neu_order)
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            Mf[rr * LDM + cb + u] = x[u];
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+            }
+            if (failed)
+                break;
+            if (p.neu_order == 0) {
+                for (int u = tid; u < CC * CC; u += NT)
+                    Mf[(u / CC) * LDM + (u % CC)] = ((u / CC) == (u % CC)) ? 1.f : 0.f;
+                __syncthreads();
+            }
+            // Newton residual steps: Rm = I - X - N X ; X <- X + X Rm
+            for (int st = 0; st < p.neu_resid && !failed; ++st) {
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(64, 64, false, true);
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tmem + T_N, desc_kmajor(AB, 128, 0, k0), desc_mnmajor(RT, 64, k0, 0), id, k0 > 0);
+                    mma_commit(&bars[MMA]);
+                }
+                if (mma_sync_wait()) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                float d0[16], d1[16];
+                tmem_ld16(tq + T_N + cb, d0);
+                tmem_ld16(tq + T_N + cb + 16, d1);
+                tmem_ld_wait();
+                if (rr >= 0) {
+                    float rm[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        rm[u] = ((rr == cb + u) ? 1.f : 0.f) - Mf[rr * LDM + cb + u] - (u < 16 ? d0[u] : d1[u - 16]);
+#pragma unroll
+                    for (int u = 0; u < 32; u += 8)
+                        st_tile8(ET, 64, rr, cb + u, &rm[u]);     // Rm as an MN-major B operand
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                // X Rm with X (bf16, RHS tile) as a K-major A operand
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(64, 64, false, true);
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tmem + T_N, desc_kmajor(RT, 64, 0, k0), desc_mnmajor(ET, 64, k0, 0), id, k0 > 0);
+                    mma_commit(&bars[MMA]);
+                }
+                if (mma_sync_wait()) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                tmem_ld16(tq + T_N + cb, d0);
+                tmem_ld16(tq + T_N + cb + 16, d1);
+                tmem_ld_wait();
+                if (rr >= 0) {
+                    float x[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        x[u] = Mf[rr * LDM + cb + u] + (u < 16 ? d0[u] : d1[u - 16]);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        Mf[rr * LDM + cb + u] = x[u];
+#pragma unroll
+                    for (int u = 0; u < 32; u += 8)
+                        st_tile8(RT, 64, rr, cb + u, &x[u]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+            }
+            if (failed)
+                break;
+        }
+        // ---- [Ab; 0] = diag(beta) A  (rows 0-63)
+        for (int u = tid; u < CC * 8; u += NT) {
+            const int t = u >> 3, j = (u & 7) * 8;
+            const float bt = sbeta[t];
+            float a[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                a[e] = bt * Mf[t * LDM + j + e];
+            st_tile8(AB, 128, t, j, a);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        // ---- [Qbar; Kbar] S  (M = 128, N = 64, K = dk)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, NVC, false, true);
+            for (int k0 = 0; k0 < DK; k0 += 16)
+                mma_bf16(tmem + T_Y, desc_kmajor(QK, 128, 0, k0), desc_mnmajor(ST, DK, k0, 0), id, k0 > 0);
+            mma_commit(&bars[MMA]);
+        }
+        if (mma_sync_wait()) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        if (wait_all(TMA_V, ph_v)) {
+            failed = true;
+            break;
+        }
+        // q, k of this chunk are spent (Khat has its own tile): prefetch the next ones
+        if (tid == 0 && c + 1 < N)
+            issue_qk(c + 1);
+        // ---- RHS = V - Kbar S  (rows 64-127 of T_Y)
+        if ((warp & 3) >= 2) {
+            const int t = 32 * (warp & 3) + lane - CC;
+            float y0[16], y1[16];
+            tmem_ld16(tq + T_Y + 32 * half, y0);
+            tmem_ld16(tq + T_Y + 32 * half + 16, y1);
+            tmem_ld_wait();
+            float r[32];
+#pragma unroll
+            for (int u = 0; u < 32; u += 8) {
+                float v8[8];
+                ld_tile8(VT, 64, t, 32 * half + u, v8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    r[u + e] = v8[e] - (u + e < 16 ? y0[u + e] : y1[u + e - 16]);
+            }
+#pragma unroll
+            for (int u = 0; u < 32; u += 8)
+                st_tile8(RT, 64, t, 32 * half + u, &r[u]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && c + 1 < N) {
+            issue_v(c + 1);
+        }
+        // ---- E = [Ab; 0] RHS
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, NVC, false, true);
+            for (int k0 = 0; k0 < CC; k0 += 16)
+                mma_bf16(tmem + T_E, desc_kmajor(AB, 128, 0, k0), desc_mnmajor(RT, 64, k0, 0), id, k0 > 0);
+            mma_commit(&bars[MMA]);
+        }
+        if (mma_sync_wait()) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        if ((warp & 3) < 2) {
+            const int t = 32 * (warp & 3) + lane;
+            float e0[16], e1[16];
+            tmem_ld16(tq + T_E + 32 * half, e0);
+            tmem_ld16(tq + T_E + 32 * half + 16, e1);
+            tmem_ld_wait();
+            st_tile8(ET, 64, t, 32 * half, &e0[0]);
+            st_tile8(ET, 64, t, 32 * half + 8, &e0[8]);
+            st_tile8(ET, 64, t, 32 * half + 16, &e1[0]);
+            st_tile8(ET, 64, t, 32 * half + 24, &e1[8]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (c + 1 < N)
+            prefetch_small(c + 1);
+        // ---- dS = Khat^T E  (M = 128 per half of dk),  O = QS + [L; 0] E
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_ds = idesc_bf16(128, NVC, true, true);
+            const uint32_t id_o = idesc_bf16(128, NVC, false, true);
+            for (int hh = 0; hh < NH; ++hh)
+                for (int k0 = 0; k0 < CC; k0 += 16)
+                    mma_bf16(tmem + T_DS + 64 * hh, desc_mnmajor(KH, 64, k0, 128 * hh),
+                             desc_mnmajor(ET, 64, k0, 0), id_ds, k0 > 0);
+            for (int k0 = 0; k0 < CC; k0 += 16)
+                mma_bf16(tmem + T_Y, desc_kmajor(LT, 128, 0, k0), desc_mnmajor(ET, 64, k0, 0), id_o, 1u);
+            mma_commit(&bars[MMA]);
+        }
+        if (mma_sync_wait()) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        // ---- S <- diag(e^{Lambda_C}) S + dS ; O (rows 0-63 of T_Y)
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+            const int row = 128 * hh + 32 * (warp & 3) + lane;
+            const float F = fch[row];
+            float d0[16], d1[16];
+            tmem_ld16(tq + T_DS + 64 * hh + 32 * half, d0);
+            tmem_ld16(tq + T_DS + 64 * hh + 32 * half + 16, d1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int n = 0; n < 32; ++n)
+                sreg[hh][n] = F * sreg[hh][n] + (n < 16 ? d0[n] : d1[n - 16]);
+#pragma unroll
+            for (int n = 0; n < 32; n += 8)
+                st_tile8(ST, DK, row, 32 * half + n, &sreg[hh][n]);
+        }
+        if ((warp & 3) < 2) {
+            const int t = 32 * (warp & 3) + lane;
+            float o0[16], o1[16];
+            tmem_ld16(tq + T_Y + 32 * half, o0);
+            tmem_ld16(tq + T_Y + 32 * half + 16, o1);
+            tmem_ld_wait();
+            if (t < Cl) {
+                const long orow = (vh * T + c0 + t) * p.dv + n0 + 32 * half;
+                if constexpr (OUT_BF16) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow);
+                    dst[0] = make_uint4(pack_bf16(o0[0], o0[1]), pack_bf16(o0[2], o0[3]), pack_bf16(o0[4], o0[5]), pack_bf16(o0[6], o0[7]));
+                    dst[1] = make_uint4(pack_bf16(o0[8], o0[9]), pack_bf16(o0[10], o0[11]), pack_bf16(o0[12], o0[13]), pack_bf16(o0[14], o0[15]));
+                    dst[2] = make_uint4(pack_bf16(o1[0], o1[1]), pack_bf16(o1[2], o1[3]), pack_bf16(o1[4], o1[5]), pack_bf16(o1[6], o1[7]));
+                    dst[3] = make_uint4(pack_bf16(o1[8], o1[9]), pack_bf16(o1[10], o1[11]), pack_bf16(o1[12], o1[13]), pack_bf16(o1[14], o1[15]));
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow);
+#pragma unroll
+                    for (int n = 0; n < 4; ++n)
+                        dst[n] = make_float4(o0[4 * n], o0[4 * n + 1], o0[4 * n + 2], o0[4 * n + 3]);
+#pragma unroll
+                    for (int n = 0; n < 4; ++n)
+                        dst[4 + n] = make_float4(o1[4 * n], o1[4 * n + 1], o1[4 * n + 2], o1[4 * n + 3]);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    }
+    if (!failed && p.S_final != nullptr) {
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+            const int row = 128 * hh + 32 * (warp & 3) + lane;
+            float *dst = p.S_final + (vh * DK + row) * p.dv + n0 + 32 * half;
+#pragma unroll
+            for (int n = 0; n < 32; n += 4)
+                *reinterpret_cast<float4 *>(dst + n) =
+                    make_float4(sreg[hh][n], sreg[hh][n + 1], sreg[hh][n + 2], sreg[hh][n + 3]);
+        }
+    }
+    // drain: let every load and product this CTA started finish (bounded)
+    if (tid == 0) {
+        mma_commit(&bars[MMA]);
+        mbar_wait(&bars[MMA], ph_mma, 200000000ull);
+        if (pend & (1u << TMA_QK))
+            mbar_wait(&bars[TMA_QK], ph_qk, 200000000ull);
+        if (pend & (1u << TMA_V))
+            mbar_wait(&bars[TMA_V], ph_v, 200000000ull);
+        if (pend & (1u << TMA_G))
+            mbar_wait(&bars[TMA_G], ph_g, 200000000ull);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// fp32 3-D map, no swizzle
+inline bool make_map_f32(CUtensorMap *m, const void *ptr, const cuuint64_t (&dims)[3],
+                         const cuuint64_t (&strides)[2], const cuuint32_t (&box)[3])
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr)
+        return false;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK, bool OB>
+int launch(const Params &p, cudaStream_t stream)
+{
+    CUtensorMap mq, mk, mv, mg;
+    const long sk = (long)p.B * p.Hk;
+    GenArgs a;
+    a.p = p;
+    a.nvt = p.dv / NVC;
+    a.g_flat = p.G < 4;
+    bool ok = make_map(&mq, p.q, DK, p.T, sk, CC) && make_map(&mk, p.k, DK, p.T, sk, CC) &&
+              make_map(&mv, p.v, p.dv, p.T, (long)p.B * p.Hv, CC);
+    if (!a.g_flat) {
+        const cuuint64_t dims[3] = {(cuuint64_t)p.G, (cuuint64_t)p.T, (cuuint64_t)sk};
+        const cuuint64_t str[2] = {(cuuint64_t)p.G * 4, (cuuint64_t)p.G * 4 * p.T};
+        const cuuint32_t box[3] = {(cuuint32_t)p.G, CC, 1};
+        ok = ok && make_map_f32(&mg, p.g, dims, str, box);
+    } else {
+        mg = mq;   // unused
+    }
+    if (!ok)
+        return 6;
+    const Plan<DK> Ly = plan<DK>();
+    auto kern = gen_kernel<DK, OB>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
+        cudaSuccess)
+        return 6;
+    dim3 grid(a.nvt * p.Hv, p.B);
+    kern<<<grid, NT, Ly.total, stream>>>(mq, mk, mv, mg, a);
+    return cudaGetLastError() == cudaSuccess ? 0 : 6;
+}
+
+inline bool supports(const Params &p)
+{
+    return p.in_bf16 && p.C == CC && (p.dk == 128 || p.dk == 256) && p.dv % NVC == 0 &&
+           p.G >= 1 && p.G <= gmax(p.dk) && p.T >= 1 && p.B <= 65535;
+}
+
+}  // namespace gen

@@ -41,6 +41,13 @@ SMALL = [
     (3, dict(B=1, Hk=1, Hv=4, T=384, chunk=128), 128, "exact", "auto"),
     (4, dict(Hk=2, Hv=2, T=640), 128, "exact", "auto"),
     (4, dict(Hk=2, Hv=2, T=704 - 37), 128, "exact", "auto"),
+    # tensor-core kernel for grouped / per-channel decay, forced
+    (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 64, "exact", "tc"),
+    (2, dict(B=1, Hk=1, Hv=1, T=256, gate_mode=W.GATE_GROUP64), 64, "exact", "tc"),
+    (3, dict(B=1, Hk=1, Hv=4, T=256, gate_mode=W.GATE_SCALAR), 64, "exact", "tc"),
+    (3, dict(B=1, Hk=1, Hv=4, T=256 - 21), 64, "neumann", "tc"),
+    (4, dict(Hk=1, Hv=1, T=384), 64, "exact", "tc"),      # strong decay: exact fp32 Gram
+    (4, dict(Hk=1, Hv=1, T=384), 64, "neumann", "tc"),
 ]
 
 
