@@ -105,25 +105,29 @@ def measured_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_fingerprint():
+def files_fingerprint(files):
     h = hashlib.sha1()
-    csrc = os.path.join(ROOT, "gated_delta_rule_141_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+    for name in files:
+        with open(os.path.join(ROOT, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:12]
 
 
 def recorded_traffic(workload_name: str, chunk: int, inverse: str):
-    """dram bytes per launch from a committed ncu summary of the same kernel
-    build (profiles/traffic.json), or None if absent or stale."""
+    """DRAM bytes per launch from a committed ncu summary (profiles/traffic.json),
+    or None if there is none or the kernel's source files changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get("%s/C%d/%s" % (workload_name, chunk, inverse))
-    if not e or e.get("fingerprint") != kernel_fingerprint():
+    if not e:
+        return None
+    try:
+        if files_fingerprint(e["files"]) != e["fingerprint"]:
+            return None
+    except OSError:
         return None
     return e.get("bytes_per_launch")
 
