@@ -397,11 +397,12 @@ def main():
         rate, threads, desc, _ = oracle_sample(w, x, chunk, args.inverse)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
-    kern = gdr.select_kernel(gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
-                                            gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
-                                            gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
-                                            kernel=args.kernel),
-                             chunk, gdr.gate_mode_for(w.G, w.dk), args.inverse)
+    sel_shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
+                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                               kernel=args.kernel)
+    kern = gdr.select_kernel(sel_shape, chunk, gdr.gate_mode_for(w.G, w.dk), args.inverse)
+    kchunk = gdr.kernel_chunk(sel_shape, chunk, gdr.gate_mode_for(w.G, w.dk), args.inverse)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -413,7 +414,7 @@ def main():
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.in_dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
-        "config": config_dict(w, chunk, args.inverse, world),
+        "config": dict(config_dict(w, chunk, args.inverse, world), kernel_chunk=kchunk),
         "tflops": roof["tflops"], "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps, "kernel": {1: "simt", 2: "tc"}.get(kern, str(kern)),
         "clocks": sampler.summary(),

@@ -165,6 +165,19 @@ int gdr_select_kernel(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode
     return choose(p, shape->kernel);
 }
 
+int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                     gdr_inverse_mode inverse_mode)
+{
+    gdr::Params p;
+    const gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return -static_cast<int>(st);
+    const int which = choose(p, shape->kernel);
+    if (which < 0)
+        return which;
+    return which == GDR_KERNEL_TC ? gdr::tc_kernel_chunk(p) : p.C;
+}
+
 gdr_status gdr_device_status(void *stream)
 {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -35,6 +35,9 @@ int launch_simt(const Params &p, cudaStream_t stream);
 
 // Tensor-core kernel (tcgen05 + TMEM + TMA, bf16 operands, fp32 accumulate).
 bool tc_supports(const Params &p);
+// Chunk length the tensor-core kernel actually blocks by (an exact-mode request
+// for C = 128 runs on the C = 64 kernels).
+int tc_kernel_chunk(const Params &p);
 int launch_tc(const Params &p, cudaStream_t stream);
 
 }  // namespace gdr

@@ -594,15 +594,31 @@ int launch_scalar(const Params &p, cudaStream_t stream)
 
 }  // namespace
 
-bool tc_supports(const Params &p)
+// In exact mode the chunkwise form reaches the token recurrence exactly for any
+// chunk length (the WY equivalence of the SLA paper, §2.4.2), so a request for
+// C = 128 runs on the C = 64 kernels: the same function, blocked more finely.
+// The truncated Neumann inverse depends on C and is never re-blocked.
+static Params as_kernel_chunk(const Params &p)
 {
+    Params q = p;
+    if (!p.neumann && p.C == 128)
+        q.C = CH;
+    return q;
+}
+
+int tc_kernel_chunk(const Params &p) { return as_kernel_chunk(p).C; }
+
+bool tc_supports(const Params &p0)
+{
+    const Params p = as_kernel_chunk(p0);
     const bool scalar64 = p.in_bf16 && p.G == 1 && p.C == CH && p.dk == 64 && p.dv % NV == 0 &&
                           !p.neumann && p.T >= 1 && p.B <= 65535;
     return ws::supports(p) || scalar64 || gen::supports(p);
 }
 
-int launch_tc(const Params &p, cudaStream_t stream)
+int launch_tc(const Params &p0, cudaStream_t stream)
 {
+    const Params p = as_kernel_chunk(p0);
     if (ws::supports(p))
         return p.out_bf16 ? ws::launch<true>(p, stream) : ws::launch<false>(p, stream);
     if (gen::supports(p)) {

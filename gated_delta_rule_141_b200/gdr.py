@@ -29,8 +29,8 @@ _KERNELS = {"auto": KERNEL_AUTO, "simt": KERNEL_SIMT, "tc": KERNEL_TC}
 _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN}
 
 # Every symbol include/gdr.h declares.
-EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_select_kernel", "gdr_device_status",
-           "gdr_status_string", "gdr_version")
+EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_select_kernel", "gdr_kernel_chunk",
+           "gdr_device_status", "gdr_status_string", "gdr_version")
 
 
 class GdrShape(ctypes.Structure):
@@ -74,6 +74,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_chunk_fwd_host.restype = i
     lib.gdr_select_kernel.argtypes = [ctypes.POINTER(GdrShape), i, i, i]
     lib.gdr_select_kernel.restype = i
+    lib.gdr_kernel_chunk.argtypes = [ctypes.POINTER(GdrShape), i, i, i]
+    lib.gdr_kernel_chunk.restype = i
     lib.gdr_device_status.argtypes = [vp]
     lib.gdr_device_status.restype = i
     lib.gdr_status_string.argtypes = [i]
@@ -112,6 +114,12 @@ def gate_mode_for(G: int, dk: int) -> int:
 def select_kernel(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "exact") -> int:
     return int(load().gdr_select_kernel(ctypes.byref(shape), int(chunk), int(gate_mode),
                                         _INVERSES[inverse]))
+
+
+def kernel_chunk(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "exact") -> int:
+    """Chunk length the selected kernel blocks by (negative status if rejected)."""
+    return int(load().gdr_kernel_chunk(ctypes.byref(shape), int(chunk), int(gate_mode),
+                                       _INVERSES[inverse]))
 
 
 def device_status(stream=None) -> int:

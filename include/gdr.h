@@ -101,7 +101,7 @@ typedef struct {
  * Device outputs (written):
  *   o      [B, Hv, T, dv]  out_dtype
  *   S_final[B, Hv, dk, dv] fp32 state after token T, or NULL to skip
- * chunk: chunk length C, 1..128 (the tensor-core kernel takes 64 or 128).
+ * chunk: chunk length C, 1..128 (see gdr_kernel_chunk for the blocking used).
  * Returns GDR_OK once the work is queued on `stream`.  Kernel-side wait
  * timeouts are reported through gdr_device_status().
  */
@@ -136,6 +136,16 @@ gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const 
  * GDR_KERNEL_TC, or a negative gdr_status value if it would be rejected. */
 int gdr_select_kernel(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
                       gdr_inverse_mode inverse_mode);
+
+/* Chunk length the kernel selected for this request actually blocks by, or a
+ * negative gdr_status value if the request would be rejected.  It equals
+ * `chunk` except on the tensor-core kernel in exact mode, where chunk 128 runs
+ * as chunk 64: the exact chunkwise form equals the token recurrence for any
+ * chunk length (WY representation of the SLA paper, §2.4.2), so the result is
+ * the same function up to rounding.  The truncated Neumann inverse depends on
+ * the chunk length and is never re-blocked. */
+int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                     gdr_inverse_mode inverse_mode);
 
 /* Synchronises `stream`, then returns and clears the device status word that
  * kernels set when a bounded wait gives up (GDR_OK or GDR_ERR_TIMEOUT), or

@@ -121,6 +121,21 @@ def test_kernel_selection(lib):
     assert gdr.select_kernel(bad, 64, gdr.GATE_SCALAR) == -gdr.ERR_SHAPE
 
 
+def test_kernel_chunk(lib):
+    # Exact mode: chunk 128 on the tensor-core kernel blocks by 64 (same function);
+    # the Neumann inverse depends on C and keeps the requested blocking.
+    kda = gdr.make_shape(2, 8192, 32, 32, 128, 128)
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL) == gdr.KERNEL_TC
+    assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL) == 64
+    assert gdr.kernel_chunk(kda, 64, gdr.GATE_CHANNEL) == 64
+    assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL, "neumann") == 128
+    simt = gdr.make_shape(1, 256, 2, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
+    assert gdr.kernel_chunk(simt, 128, gdr.GATE_SCALAR) == 128
+    assert gdr.kernel_chunk(simt, 32, gdr.GATE_SCALAR) == 32
+    assert gdr.kernel_chunk(gdr.make_shape(1, 256, 2, 3, 64, 64), 64,
+                            gdr.GATE_SCALAR) == -gdr.ERR_SHAPE
+
+
 def test_host_entry_validates(lib):
     shape = gdr.make_shape(1, 64, 2, 4, 64, 64)
     io = gdr.GdrIO()

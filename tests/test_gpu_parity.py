@@ -48,6 +48,10 @@ SMALL = [
     (3, dict(B=1, Hk=1, Hv=4, T=256 - 21), 64, "neumann", "tc"),
     (4, dict(Hk=1, Hv=1, T=384), 64, "exact", "tc"),      # strong decay: exact fp32 Gram
     (4, dict(Hk=1, Hv=1, T=384), 64, "neumann", "tc"),
+    # exact mode at C = 128 on the tensor-core kernels (blocked by 64 there), oracle at C = 128
+    (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 128, "exact", "tc"),
+    (3, dict(B=1, Hk=1, Hv=4, T=384 - 37), 128, "exact", "tc"),
+    (4, dict(Hk=2, Hv=2, T=640), 128, "exact", "tc"),
 ]
 
 
