@@ -55,7 +55,7 @@ def parse_args():
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--inverse", default="exact", choices=["exact", "neumann"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "simt"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -300,6 +300,14 @@ def main():
     if in_bytes < L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+    shape_run = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
+                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32, kernel=args.kernel)
+    gm_run = gdr.gate_mode_for(w.G, w.dk)
+    ws_bytes = gdr.workspace_bytes(shape_run, chunk, gm_run, args.inverse)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda") if ws_bytes else None
+    kern = gdr.select_kernel(shape_run, chunk, gm_run, args.inverse)
+    launches_per_step = 2 if kern == gdr.KERNEL_TC2 else 1
     # with an L2 flush between steps, only the launches themselves are timed
     step_events = []
 
@@ -311,7 +319,7 @@ def main():
             e0.record(stream)
         gdr.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
                       chunk=chunk, inverse=args.inverse, o=o, S_final=Sf, kernel=args.kernel,
-                      stream=stream)
+                      workspace=workspace, stream=stream)
         if timed and flush is not None:
             e1.record(stream)
             step_events.append((e0, e1))
@@ -362,6 +370,8 @@ def main():
     roof["tflops"] = flop / (ms_step * 1e-3) / 1e12
     roof["tc_frac"] = tc_frac
     roof["hbm_frac"] = hbm_frac
+    roof["kernel"] = gdr.KERNEL_NAMES.get(kern, str(kern))
+    roof["launches_per_step"] = launches_per_step
 
     # end to end through the host-buffer entry point
     e2e = None
@@ -371,21 +381,17 @@ def main():
         host["S_final"] = torch.empty(Sf.shape, dtype=torch.float32).pin_memory()
         dbuf = {n: (None if t is None else torch.empty_like(t)) for n, t in dev.items()}
         dbuf["o"], dbuf["S_final"] = torch.empty_like(o), torch.empty_like(Sf)
-        shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
-                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
-                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
-                               kernel=args.kernel)
-        gm = gdr.gate_mode_for(w.G, w.dk)
+        shape, gm = shape_run, gm_run
         h2d = sum(t.numel() * t.element_size() for n, t in host.items()
                   if t is not None and n not in ("o", "S_final"))
         d2h = host["o"].numel() * host["o"].element_size() + host["S_final"].numel() * 4
         e2e_steps = max(3, min(args.steps, 20))
         for _ in range(2):
-            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, stream)
+            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, workspace, stream)
         barrier()
         ev0.record(stream)
         for _ in range(e2e_steps):
-            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, stream)
+            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, workspace, stream)
         ev1.record(stream)
         barrier()
         ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), dist, torch.device("cuda", local))
@@ -397,12 +403,7 @@ def main():
         rate, threads, desc, _ = oracle_sample(w, x, chunk, args.inverse)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
-    sel_shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
-                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
-                               gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
-                               kernel=args.kernel)
-    kern = gdr.select_kernel(sel_shape, chunk, gdr.gate_mode_for(w.G, w.dk), args.inverse)
-    kchunk = gdr.kernel_chunk(sel_shape, chunk, gdr.gate_mode_for(w.G, w.dk), args.inverse)
+    kchunk = gdr.kernel_chunk(shape_run, chunk, gm_run, args.inverse)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -416,7 +417,7 @@ def main():
         "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
         "config": dict(config_dict(w, chunk, args.inverse, world), kernel_chunk=kchunk),
         "tflops": roof["tflops"], "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": args.steps, "kernel": {1: "simt", 2: "tc"}.get(kern, str(kern)),
+        "gpu_launches": args.steps * launches_per_step, "kernel": gdr.KERNEL_NAMES.get(kern, str(kern)),
         "clocks": sampler.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -2,6 +2,7 @@
 // validation, kernel selection and the host-buffer convenience entry point.
 // Every computation happens in the kernels of gdr_simt.cu / gdr_tc.cu.
 #include <cstdint>
+#include <cstddef>
 
 #include "gdr.h"
 #include "gdr_internal.h"
@@ -23,7 +24,8 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
         return GDR_ERR_DTYPE;
     if (s->out_dtype != GDR_F32 && s->out_dtype != GDR_BF16)
         return GDR_ERR_DTYPE;
-    if (s->kernel != GDR_KERNEL_AUTO && s->kernel != GDR_KERNEL_SIMT && s->kernel != GDR_KERNEL_TC)
+    if (s->kernel != GDR_KERNEL_AUTO && s->kernel != GDR_KERNEL_SIMT && s->kernel != GDR_KERNEL_TC &&
+        s->kernel != GDR_KERNEL_TC2)
         return GDR_ERR_ARG;
     if (s->B < 0 || s->T < 0 || s->Hk < 1 || s->Hv < 1 || s->Hv % s->Hk != 0)
         return GDR_ERR_SHAPE;
@@ -59,15 +61,25 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
     return GDR_OK;
 }
 
-// GDR_KERNEL_SIMT / GDR_KERNEL_TC, or -status.
-int choose(const gdr::Params &p, gdr_kernel want)
+// GDR_KERNEL_SIMT / GDR_KERNEL_TC / GDR_KERNEL_TC2, or -status, for a call
+// that brings `ws_bytes` of workspace (SIZE_MAX: as much as TC2 asks for).
+int choose(const gdr::Params &p, gdr_kernel want, size_t ws_bytes)
 {
+    const bool tc2 = gdr::tc2_supports(p);
+    const bool tc2_fits = tc2 && ws_bytes >= gdr::tc2_workspace_bytes(p);
     const bool tc = gdr::tc_supports(p);
     const bool simt = gdr::simt_smem_bytes(p) <= 227 * 1024;
-    if (want == GDR_KERNEL_TC)
-        return tc ? GDR_KERNEL_TC : -GDR_ERR_UNSUPPORTED;
-    if (want == GDR_KERNEL_SIMT)
-        return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
+    switch (want) {
+    case GDR_KERNEL_TC2:
+        if (!tc2)
+            return -GDR_ERR_UNSUPPORTED;
+        return tc2_fits ? GDR_KERNEL_TC2 : -GDR_ERR_WORKSPACE;
+    case GDR_KERNEL_TC: return tc ? GDR_KERNEL_TC : -GDR_ERR_UNSUPPORTED;
+    case GDR_KERNEL_SIMT: return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
+    default: break;
+    }
+    if (tc2_fits)
+        return GDR_KERNEL_TC2;
     if (tc)
         return GDR_KERNEL_TC;
     return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
@@ -80,7 +92,7 @@ extern "C" {
 gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, const void *v,
                          const float *g, const float *beta, const float *S0, int chunk,
                          gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode, void *o,
-                         float *S_final, void *stream)
+                         float *S_final, void *workspace, size_t workspace_bytes, void *stream)
 {
     gdr::Params p;
     gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
@@ -89,24 +101,72 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, c
     const bool has_tokens = (long)p.B * p.T > 0;
     if (has_tokens && (!q || !k || !v || !g || !beta || !o))
         return GDR_ERR_ARG;
-    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_final};
+    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_final, workspace};
     for (const void *ptr : ptrs)
         if (ptr != nullptr && !aligned16(ptr))
             return GDR_ERR_ALIGN;
-    const int which = choose(p, shape->kernel);
+    const int which = choose(p, shape->kernel, workspace != nullptr ? workspace_bytes : 0);
     if (which < 0)
         return static_cast<gdr_status>(-which);
     if (p.B == 0)
         return GDR_OK;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S0 = S0; p.o = o; p.S_final = S_final;
     auto s = static_cast<cudaStream_t>(stream);
-    const int rc = which == GDR_KERNEL_TC ? gdr::launch_tc(p, s) : gdr::launch_simt(p, s);
+    int rc;
+    if (which == GDR_KERNEL_TC2)
+        rc = gdr::launch_tc2(p, workspace, s);
+    else if (which == GDR_KERNEL_TC)
+        rc = gdr::launch_tc(p, s);
+    else
+        rc = gdr::launch_simt(p, s);
     return static_cast<gdr_status>(rc);
+}
+
+gdr_status gdr_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                               gdr_inverse_mode inverse_mode, size_t *bytes)
+{
+    if (bytes == nullptr)
+        return GDR_ERR_ARG;
+    gdr::Params p;
+    const gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return st;
+    const int which = choose(p, shape->kernel, SIZE_MAX);
+    if (which < 0)
+        return static_cast<gdr_status>(-which);
+    *bytes = which == GDR_KERNEL_TC2 ? gdr::tc2_workspace_bytes(p) : 0;
+    return GDR_OK;
+}
+
+gdr_status gdr_chunk_prepare(const gdr_shape *shape, const void *q, const void *k,
+                             const float *g, const float *beta, int chunk,
+                             gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode,
+                             void *factors, size_t factors_bytes, void *stream)
+{
+    gdr::Params p;
+    const gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return st;
+    const bool has_tokens = (long)p.B * p.T > 0;
+    if (has_tokens && (!q || !k || !g || !beta || !factors))
+        return GDR_ERR_ARG;
+    const void *ptrs[] = {q, k, g, beta, factors};
+    for (const void *ptr : ptrs)
+        if (ptr != nullptr && !aligned16(ptr))
+            return GDR_ERR_ALIGN;
+    if (!gdr::prepare_supports(p))
+        return GDR_ERR_UNSUPPORTED;
+    if (factors_bytes < gdr::prepare_bytes(p))
+        return GDR_ERR_WORKSPACE;
+    if (!has_tokens)
+        return GDR_OK;
+    p.q = q; p.k = k; p.g = g; p.beta = beta;
+    return static_cast<gdr_status>(gdr::launch_prepare(p, factors, static_cast<cudaStream_t>(stream)));
 }
 
 gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const gdr_io *dev,
                               int chunk, gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode,
-                              void *stream)
+                              void *workspace, size_t workspace_bytes, void *stream)
 {
     if (host == nullptr || dev == nullptr)
         return GDR_ERR_ARG;
@@ -142,7 +202,8 @@ gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const 
             return GDR_ERR_CUDA;
     }
     st = gdr_chunk_fwd(shape, dev->q, dev->k, dev->v, dev->g, dev->beta, dev->S0, chunk,
-                       gate_mode, inverse_mode, dev->o, dev->S_final, stream);
+                       gate_mode, inverse_mode, dev->o, dev->S_final, workspace, workspace_bytes,
+                       stream);
     if (st != GDR_OK)
         return st;
     if (has_tokens &&
@@ -162,7 +223,7 @@ int gdr_select_kernel(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode
     const gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
     if (st != GDR_OK)
         return -static_cast<int>(st);
-    return choose(p, shape->kernel);
+    return choose(p, shape->kernel, SIZE_MAX);
 }
 
 int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
@@ -172,10 +233,10 @@ int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
     const gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
     if (st != GDR_OK)
         return -static_cast<int>(st);
-    const int which = choose(p, shape->kernel);
+    const int which = choose(p, shape->kernel, SIZE_MAX);
     if (which < 0)
         return which;
-    return which == GDR_KERNEL_TC ? gdr::tc_kernel_chunk(p) : p.C;
+    return which == GDR_KERNEL_SIMT ? p.C : gdr::tc_kernel_chunk(p);
 }
 
 gdr_status gdr_device_status(void *stream)
@@ -200,6 +261,7 @@ const char *gdr_status_string(gdr_status status)
     case GDR_ERR_CUDA: return "CUDA runtime error";
     case GDR_ERR_TIMEOUT: return "a bounded device wait gave up";
     case GDR_ERR_NONFINITE: return "non-finite input";
+    case GDR_ERR_WORKSPACE: return "workspace smaller than the selected kernel needs";
     }
     return "unknown status";
 }

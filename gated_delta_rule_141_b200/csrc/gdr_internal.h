@@ -2,6 +2,7 @@
 // of libgdr.so (not part of the public ABI).
 #pragma once
 #include <cuda_runtime.h>
+#include <cstddef>
 #include <cstdint>
 
 namespace gdr {
@@ -39,5 +40,16 @@ bool tc_supports(const Params &p);
 // for C = 128 runs on the C = 64 kernels).
 int tc_kernel_chunk(const Params &p);
 int launch_tc(const Params &p, cudaStream_t stream);
+
+// Two-pass tensor-core path: the chunk-local factors of all chunks in parallel
+// (written to a caller-owned workspace), then the state pass that reads them.
+bool tc2_supports(const Params &p);
+size_t tc2_workspace_bytes(const Params &p);
+int launch_tc2(const Params &p, void *workspace, cudaStream_t stream);
+
+// The first pass alone, at the requested chunk length (public gdr_chunk_prepare).
+bool prepare_supports(const Params &p);
+size_t prepare_bytes(const Params &p);
+int launch_prepare(const Params &p, void *out, cudaStream_t stream);
 
 }  // namespace gdr

@@ -591,6 +591,8 @@ int launch_scalar(const Params &p, cudaStream_t stream)
 
 #include "gdr_tc_ws.cuh"
 #include "gdr_tc_gen.cuh"
+#include "gdr_tc_prep.cuh"
+#include "gdr_tc_split.cuh"
 
 }  // namespace
 
@@ -629,6 +631,34 @@ int launch_tc(const Params &p0, cudaStream_t stream)
     if (p.dk == 64)
         return p.out_bf16 ? launch_scalar<64, true>(p, stream) : launch_scalar<64, false>(p, stream);
     return 5;
+}
+
+bool tc2_supports(const Params &p0) { return split::supports(as_kernel_chunk(p0)); }
+
+size_t tc2_workspace_bytes(const Params &p0) { return prep::ws_bytes(as_kernel_chunk(p0)); }
+
+int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
+{
+    const Params p = as_kernel_chunk(p0);
+    if (!split::supports(p))
+        return 5;
+    const int rc = prep::launch<128>(p, workspace, prep::record_kind(p), stream);
+    if (rc != 0)
+        return rc;
+    return p.out_bf16 ? split::launch<true>(p, workspace, stream)
+                      : split::launch<false>(p, workspace, stream);
+}
+
+bool prepare_supports(const Params &p) { return prep::supports(p); }
+
+size_t prepare_bytes(const Params &p) { return prep::bytes(p); }
+
+int launch_prepare(const Params &p, void *out, cudaStream_t stream)
+{
+    if (!prep::supports(p))
+        return 5;
+    return p.dk == 128 ? prep::launch<128>(p, out, prep::REC_PLAIN, stream)
+                       : prep::launch<256>(p, out, prep::REC_PLAIN, stream);
 }
 
 }  // namespace gdr

@@ -1,0 +1,687 @@
+// gdr_tc_prep.cuh -- first pass of the two-pass tensor-core path: the
+// chunk-local factors of every (batch, key head, chunk), computed for all
+// chunks in parallel.  Included by gdr_tc.cu.
+//
+// Per chunk of C = 64 tokens ("Systolic Linear Attention: Co-Designing
+// Tile-Grouped Gated Delta Attention for TPUs", §2.1, §2.3 Table 2, §2.4.2;
+// "Kimi Linear" chunkwise KDA, decay pivots):
+//   1. TMA: q and k as one [q; k] tile of 128 rows (zero past T); beta and the
+//      log-gates g through plain loads (zero past T: the recurrence is then
+//      left untouched by the padding rows).
+//   2. Lambda = cumsum g per decay group (fp32).
+//   3. Decayed Grams on tcgen05, never dividing by a decay prefix:
+//        scalar gate: [Q; K] K^T once, then the factor e^{Lambda_t - Lambda_j}
+//          (t >= j, so <= 1) on the way out of TMEM;
+//        grouped / per-channel gate: four row blocks of 16 tokens, each with
+//          its own pivot p in the middle of the block.  Rows t of the block
+//          carry e^{Lambda_t - Lambda_p}, columns j carry e^{Lambda_p - Lambda_j};
+//          both factors are at most e^{(half-block decay span)}, and their
+//          product is the exact e^{Lambda_t - Lambda_j}.  A block whose half
+//          span exceeds kGuard nats is recomputed element by element in fp32.
+//      L_tj = (t >= j) q_t . k_j decayed,  M_tj = (t > j) beta_j k_t . k_j decayed.
+//   4. A = (I + M)^{-1}: exact fp32 block doubling, or the truncated Neumann
+//      series with Newton residual steps on tcgen05 ("When Good Enough Is
+//      Optimal: Multiplication-Only Matrix Inversion Approximation for
+//      Quantized Gated DeltaNet", Lemma 3.1, §4.1).
+//   5. Output, per chunk, two bf16 C x C tiles: T = diag(beta) A and L, each as
+//      the byte image of a 128-byte-swizzled shared-memory tile (64 rows x 128
+//      bytes, 16-byte chunk index XOR (row % 8)), so that the second pass can
+//      bring them in with one bulk copy each.  For grouped / per-channel gates
+//      the record the state pass reads also carries the decayed operands
+//      Qbar = q e^{Lambda_t}, Khat = k e^{Lambda_C - Lambda_t}, Kbar = k e^{Lambda_t}
+//      (C x dk bf16 images, 64-column blocks of 64 rows) and F = e^{Lambda_C}
+//      (dk fp32): every factor is the exponential of a non-positive difference.
+
+namespace prep {
+
+constexpr int NT = 256;
+constexpr int CC = 64;
+constexpr int LDM = gen::LDM;              // row stride of the fp32 C x C scratch
+constexpr int NROUND = 4;                  // pivot blocks of 16 rows
+constexpr float kGuard = 64.f;             // largest exponent a pivoted factor may take
+constexpr uint32_t IMG = CC * CC * 2;      // one bf16 C x C tile image
+constexpr uint32_t CHUNK_BYTES = 2 * IMG;  // T, then L
+// Records of the two-pass path's workspace (key width 128).
+// scalar gate: T, L, Abe = T diag(e^Lambda), e^{Lambda_t}, e^{Lambda_C - Lambda_t}, e^{Lambda_C}
+constexpr uint32_t SC_ABE = 2 * IMG, SC_EA = 3 * IMG, SC_EB = SC_EA + CC * 4, SC_F = SC_EB + CC * 4;
+constexpr uint32_t SC_BYTES = SC_F + 16;
+// grouped / per-channel gates: T, L, Qbar, Khat, Kbar, F
+constexpr uint32_t EXT_QB = 2 * IMG, EXT_KH = EXT_QB + 2 * IMG, EXT_KB = EXT_KH + 2 * IMG;
+constexpr uint32_t EXT_F = EXT_KB + 2 * IMG;
+constexpr uint32_t EXT_BYTES = EXT_F + 128 * 4;
+enum RecordKind { REC_PLAIN = 0, REC_SCALAR = 1, REC_EXT = 2 };
+
+__host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
+// TMEM column of round r's accumulator (rounds are 16, 32, 48, 64 columns wide)
+__host__ __device__ constexpr uint32_t round_col(int r) { return 8u * r * (r + 1); }
+
+struct Plan {
+    uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, lam, beta, bar, misc, total, tmem_cols, tn;
+};
+
+__host__ __device__ inline Plan plan(int dk, int G, bool neumann)
+{
+    Plan s;
+    uint32_t o = 0;
+    auto take = [&](uint32_t bytes) {
+        const uint32_t at = o;
+        o += (bytes + 1023u) & ~1023u;
+        return at;
+    };
+    const bool extra = G > 1 || neumann;
+    s.QK = take((dk / 64) * 128 * 128);          // rows 0-63 q, 64-127 k
+    if (extra) {
+        s.RA = take((dk / 64) * 64 * 128);        // round rows: 16 of q, 16 of k
+        s.KC = take((dk / 64) * 64 * 128);        // round columns
+    } else {
+        s.RA = s.KC = 0;
+    }
+    // fp32 scratch lives in tiles that are dead once the Grams are read
+    s.Mf = extra ? s.RA : s.QK;
+    s.Tf = s.Mf + CC * LDM * 4;
+    s.NB = s.QK;                                  // Neumann operands (QK is dead by then)
+    s.XB = s.QK + 8192;
+    s.RB = s.QK + 16384;
+    s.lam = take(CC * G * 4);
+    s.beta = take(CC * 4 + NROUND * 4);
+    s.bar = take(64);
+    s.misc = s.bar + 32;
+    s.total = o + 1024;
+    s.tmem_cols = G > 1 ? 256u : (neumann ? 128u : 64u);
+    s.tn = G > 1 ? 192u : 64u;                    // Neumann products
+    return s;
+}
+
+struct PrepArgs {
+    Params p;
+    uint8_t *out;      // [B * Hk * nchunks][rec_bytes]
+    int nchunks;
+    int kind;          // RecordKind: what besides T and L the record carries
+    uint32_t rec_bytes;
+};
+
+// Store 8 floats as bf16 into the 16-byte chunk of row r holding columns [c, c+8)
+// of a 64 x 64 tile image in global memory.
+__device__ __forceinline__ void st_img8(uint8_t *img, int r, int c, const float *v)
+{
+    const int cc = (c >> 3) ^ (r & 7);
+    *reinterpret_cast<uint4 *>(img + r * 128 + cc * 16) =
+        make_uint4(ptx::pack_bf16(v[0], v[1]), ptx::pack_bf16(v[2], v[3]),
+                   ptx::pack_bf16(v[4], v[5]), ptx::pack_bf16(v[6], v[7]));
+}
+
+template <int DK>
+__global__ void __launch_bounds__(NT, 3)
+prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+            const PrepArgs a)
+{
+    using namespace ptx;
+    extern __shared__ uint8_t smem_raw[];
+    const Params &p = a.p;
+    const int G = p.G;
+    const bool neu = p.neumann != 0;
+    const Plan Ly = plan(DK, G, neu);
+    const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t pad = base_u32 - smem_u32(smem_raw);
+    uint8_t *base = smem_raw + pad;
+    float *lam = reinterpret_cast<float *>(base + Ly.lam);
+    float *sbeta = reinterpret_cast<float *>(base + Ly.beta);
+    int *flag = reinterpret_cast<int *>(sbeta + CC);
+    float *Mf = reinterpret_cast<float *>(base + Ly.Mf);
+    float *Tf = reinterpret_cast<float *>(base + Ly.Tf);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const long kh = (long)b * p.Hk + hk;
+    const int T = p.T;
+    const long c0 = (long)c * CC;
+    const int Cl = (int)min((long)CC, T - c0);
+    const int wsh = __ffs(DK / G) - 1;      // channels per decay group = 2^wsh
+    const uint32_t QK = base_u32 + Ly.QK, RA = base_u32 + Ly.RA, KC = base_u32 + Ly.KC;
+    uint8_t *img_T = a.out + (size_t)(kh * a.nchunks + c) * a.rec_bytes;
+    uint8_t *img_L = img_T + IMG;
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);     // TMA
+        mbar_init(&bars[1], 1);     // MMA
+        fence_barrier_init();
+        mbar_arrive_expect_tx(&bars[0], 2u * CC * DK * 2u);
+        for (int kb = 0; kb < DK / 64; ++kb) {
+            tma_load_3d(base + Ly.QK + kb * 128 * 128, &tm_q, &bars[0], 64 * kb, (int)c0, (int)kh);
+            tma_load_3d(base + Ly.QK + kb * 128 * 128 + 64 * 128, &tm_k, &bars[0], 64 * kb, (int)c0,
+                        (int)kh);
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, Ly.tmem_cols);
+        tmem_relinquish();
+    }
+    for (int t = tid; t < CC; t += NT)
+        sbeta[t] = t < Cl ? p.beta[kh * T + c0 + t] : 0.f;
+    for (int u = tid; u < CC * G; u += NT)
+        lam[u] = (u / G) < Cl ? p.g[(kh * T + c0) * G + u] : 0.f;
+    if (tid < NROUND)
+        flag[tid] = 0;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+
+    // ---- Lambda = cumsum over the chunk per decay group
+    if (G <= 8) {
+        if (warp < G) {   // lane l holds rows 2l, 2l+1
+            const float v0 = lam[(2 * lane) * G + warp], v1 = lam[(2 * lane + 1) * G + warp];
+            float s = v0 + v1;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, s, d);
+                if (lane >= d)
+                    s += y;
+            }
+            const float r0 = (s - (v0 + v1)) + v0;
+            lam[(2 * lane) * G + warp] = r0;
+            lam[(2 * lane + 1) * G + warp] = r0 + v1;
+        }
+    } else {
+        for (int gi = tid; gi < G; gi += NT) {
+            float acc = 0.f;
+            for (int t0 = 0; t0 < CC; t0 += 8) {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v[e] = lam[(t0 + e) * G + gi];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    acc += v[e];
+                    lam[(t0 + e) * G + gi] = acc;
+                }
+            }
+        }
+    }
+    // decay span of the chunk per group: within kGuard nats a single pivot at the
+    // chunk end serves every pair; wider spans take the four pivoted row blocks
+    bool wide = false;
+    if (G > 1)
+        for (int gi = tid; gi < G; gi += NT)
+            wide |= (lam[gi] - lam[(CC - 1) * G + gi]) > kGuard;
+    wide = __syncthreads_or(wide ? 1 : 0) != 0;
+
+    uint32_t ph_mma = 0;
+    bool failed = false;
+    auto wait_bar = [&](int i, uint32_t ph) {
+        const bool gave_up = !mbar_wait(&bars[i], ph);
+        if (gave_up)
+            atomicExch(&g_device_status, kTimeoutStatus);
+        return __syncthreads_or(gave_up ? 1 : 0) != 0;
+    };
+    failed = wait_bar(0, 0);
+
+    const bool ext = a.kind == REC_EXT;
+    if (!failed && ext) {
+        float *fo = reinterpret_cast<float *>(img_T + EXT_F);
+        for (int i = tid; i < DK; i += NT)
+            fo[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);
+    }
+    if (!failed && a.kind == REC_SCALAR) {   // per-token factors of the scalar gate
+        float *ea = reinterpret_cast<float *>(img_T + SC_EA);
+        float *eb = reinterpret_cast<float *>(img_T + SC_EB);
+        const float lc = lam[CC - 1];
+        for (int t = tid; t < CC; t += NT) {
+            ea[t] = __expf(lam[t]);
+            eb[t] = __expf(lc - lam[t]);
+        }
+        if (tid < 4)
+            reinterpret_cast<float *>(img_T + SC_F)[tid] = __expf(lc);
+    }
+    if (!failed && ext && wide) {
+        // ---- decayed operands for the state pass, straight from the raw tiles
+        for (int u = tid; u < CC * (DK / 8); u += NT) {
+            const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+            float qv[8], kv[8], qb[8], kh8[8], kb[8];
+            ld_tile8(QK, 128, t, i0, qv);
+            ld_tile8(QK, 128, 64 + t, i0, kv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int gi = (i0 + e) >> wsh;
+                const float lt = lam[t * G + gi];
+                const float ea = __expf(lt), eb = __expf(lam[(CC - 1) * G + gi] - lt);
+                qb[e] = qv[e] * ea;
+                kb[e] = kv[e] * ea;
+                kh8[e] = kv[e] * eb;
+            }
+            const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
+            *reinterpret_cast<uint4 *>(img_T + EXT_QB + off) =
+                make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]), pack_bf16(qb[4], qb[5]),
+                           pack_bf16(qb[6], qb[7]));
+            *reinterpret_cast<uint4 *>(img_T + EXT_KH + off) =
+                make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
+                           pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
+            *reinterpret_cast<uint4 *>(img_T + EXT_KB + off) =
+                make_uint4(pack_bf16(kb[0], kb[1]), pack_bf16(kb[2], kb[3]), pack_bf16(kb[4], kb[5]),
+                           pack_bf16(kb[6], kb[7]));
+        }
+    }
+
+    if (!failed && !wide) {
+        if (G > 1) {
+            // ---- one pivot at the chunk end: rows carry e^{Lambda_t - Lambda_C} (at most
+            //      e^{kGuard}), columns Khat = k e^{Lambda_C - Lambda_j} (at most 1); the
+            //      state pass's decayed operands come out of the same sweep
+            for (int u = tid; u < CC * (DK / 8); u += NT) {
+                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                float qv[8], kv[8], kh8[8], qb[8], kb[8];
+                ld_tile8(QK, 128, t, i0, qv);
+                ld_tile8(QK, 128, 64 + t, i0, kv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int gi = (i0 + e) >> wsh;
+                    const float lt = lam[t * G + gi], lc = lam[(CC - 1) * G + gi];
+                    const float up = __expf(lt - lc), dn = __expf(lc - lt), ea = __expf(lt);
+                    qb[e] = qv[e] * ea;
+                    kb[e] = kv[e] * ea;
+                    kh8[e] = kv[e] * dn;
+                    qv[e] *= up;
+                    kv[e] *= up;
+                }
+                st_tile8(QK, 128, t, i0, qv);
+                st_tile8(QK, 128, 64 + t, i0, kv);
+                st_tile8(KC, 64, t, i0, kh8);
+                if (ext) {
+                    const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(img_T + EXT_QB + off) =
+                        make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]),
+                                   pack_bf16(qb[4], qb[5]), pack_bf16(qb[6], qb[7]));
+                    *reinterpret_cast<uint4 *>(img_T + EXT_KH + off) =
+                        make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
+                                   pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
+                    *reinterpret_cast<uint4 *>(img_T + EXT_KB + off) =
+                        make_uint4(pack_bf16(kb[0], kb[1]), pack_bf16(kb[2], kb[3]),
+                                   pack_bf16(kb[4], kb[5]), pack_bf16(kb[6], kb[7]));
+                }
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+        }
+        // ---- [Q; K] K^T (M = 128, N = 64, K = dk); for the scalar gate the decay and
+        //      beta are applied on the way out, for the others beta only
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, CC, false, false);
+            for (int k0 = 0; k0 < DK; k0 += 16)
+                mma_bf16(tmem, desc_kmajor(QK, 128, 0, k0),
+                         G == 1 ? desc_kmajor(QK, 128, 64, k0) : desc_kmajor(KC, 64, 0, k0), id, k0 > 0);
+            mma_commit(&bars[1]);
+        }
+        failed = wait_bar(1, ph_mma);
+        ph_mma ^= 1u;
+        if (!failed) {
+            tc_fence_after();
+            const int R = 32 * (warp & 3) + lane, half = warp >> 2, j0 = 32 * half;
+            float g0[16], g1[16];
+            tmem_ld16(tq + j0, g0);
+            tmem_ld16(tq + j0 + 16, g1);
+            tmem_ld_wait();
+            const bool qrow = R < CC;
+            const int t = qrow ? R : R - CC;
+            const float lt = lam[t * G];
+            float out[32];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int j = j0 + u;
+                const float d = u < 16 ? g0[u] : g1[u - 16];
+                const bool keep = qrow ? (j <= t) : (j < t);
+                float v = keep ? (G == 1 ? d * __expf(lt - lam[j]) : d) : 0.f;
+                if (!qrow)
+                    v *= sbeta[j];
+                out[u] = v;
+            }
+            if (qrow) {
+#pragma unroll
+                for (int u = 0; u < 32; u += 8)
+                    st_img8(img_L, t, j0 + u, &out[u]);
+            } else {
+                // Mf aliases the (now dead) [q; k] tile
+#pragma unroll
+                for (int u = 0; u < 32; u += 4)
+                    *reinterpret_cast<float4 *>(&Mf[t * LDM + j0 + u]) =
+                        make_float4(out[u], out[u + 1], out[u + 2], out[u + 3]);
+            }
+        }
+    } else if (!failed) {
+        // ---- pivoted rounds: row block r (rows 16r..16r+15), pivot 16r + 8
+        for (int r = 0; r < NROUND && !failed; ++r) {
+            const int p0 = 16 * r, pv = p0 + 8, n_r = 16 * (r + 1);
+            bool clamp = false;
+            for (int u = tid; u < (32 + n_r) * (DK / 8); u += NT) {
+                const int row = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                float v8[8];
+                if (row < 32) {
+                    const int t = p0 + (row & 15);
+                    ld_tile8(QK, 128, (row < 16 ? 0 : 64) + t, i0, v8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int gi = (i0 + e) >> wsh;
+                        float x = lam[t * G + gi] - lam[pv * G + gi];
+                        if (x > kGuard) {
+                            x = kGuard;
+                            clamp = true;
+                        }
+                        v8[e] *= __expf(x);
+                    }
+                    st_tile8(RA, 64, row, i0, v8);
+                } else {
+                    const int j = row - 32;
+                    ld_tile8(QK, 128, 64 + j, i0, v8);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int gi = (i0 + e) >> wsh;
+                        float x = lam[pv * G + gi] - lam[j * G + gi];
+                        if (x > kGuard) {
+                            x = kGuard;
+                            clamp = true;
+                        }
+                        v8[e] *= __expf(x);
+                    }
+                    st_tile8(KC, 64, j, i0, v8);
+                }
+            }
+            if (clamp)
+                flag[r] = 1;
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(64, n_r, false, false);
+                for (int k0 = 0; k0 < DK; k0 += 16)
+                    mma_bf16(tmem + round_col(r), desc_kmajor(RA, 64, 0, k0), desc_kmajor(KC, 64, 0, k0),
+                             id, k0 > 0);
+                mma_commit(&bars[1]);
+            }
+            failed = wait_bar(1, ph_mma);
+            ph_mma ^= 1u;
+        }
+        if (!failed) {
+            tc_fence_after();
+            // M = 64 accumulator: round rows 0-15 (scores) sit in lanes 0-15 of quarter 0,
+            // rows 16-31 (key Gram) in lanes 0-15 of quarter 1.  Mf aliases the round tiles.
+            const int q4 = warp & 3, half = warp >> 2;
+            if (q4 < 2) {
+                const bool qrow = q4 == 0;
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int r = half == 0 ? (rr == 0 ? 0 : 3) : (rr == 0 ? 1 : 2);
+                    const int n_r = 16 * (r + 1), t = 16 * r + (lane & 15);
+                    for (int cb = 0; cb < 4; ++cb) {
+                        float d[16];
+                        if (16 * cb < n_r) {
+                            tmem_ld16(tq + round_col(r) + 16 * cb, d);
+                            tmem_ld_wait();
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                d[e] = 0.f;
+                        }
+                        if (lane < 16) {
+                            float v[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int j = 16 * cb + e;
+                                v[e] = qrow ? ((j <= t) ? d[e] : 0.f) : ((j < t) ? sbeta[j] * d[e] : 0.f);
+                            }
+                            if (qrow) {
+                                st_img8(img_L, t, 16 * cb, &v[0]);
+                                st_img8(img_L, t, 16 * cb + 8, &v[8]);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 16; e += 4)
+                                    *reinterpret_cast<float4 *>(&Mf[t * LDM + 16 * cb + e]) =
+                                        make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                            }
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+            // blocks whose decay span overran the guard: exact fp32 rows from the raw tiles
+            for (int r = 0; r < NROUND; ++r) {
+                if (!flag[r])
+                    continue;
+                for (int u = tid; u < 16 * 8; u += NT) {
+                    const int t = 16 * r + (u >> 3), j0 = (u & 7) * 8;
+                    float lv[8], mv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        lv[e] = mv[e] = 0.f;
+                    for (int i0 = 0; i0 < DK; i0 += 8) {
+                        float qt[8], kt[8];
+                        ld_tile8(QK, 128, t, i0, qt);
+                        ld_tile8(QK, 128, 64 + t, i0, kt);
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = j0 + e;
+                            if (j > t)
+                                break;
+                            float kj[8];
+                            ld_tile8(QK, 128, 64 + j, i0, kj);
+#pragma unroll
+                            for (int f = 0; f < 8; ++f) {
+                                const int gi = (i0 + f) >> wsh;
+                                const float dcy = __expf(lam[t * G + gi] - lam[j * G + gi]);
+                                lv[e] += qt[f] * kj[f] * dcy;
+                                mv[e] += kt[f] * kj[f] * dcy;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = j0 + e;
+                        mv[e] = (j < t) ? sbeta[j] * mv[e] : 0.f;
+                        lv[e] = (j <= t) ? lv[e] : 0.f;
+                        Mf[t * LDM + j] = mv[e];
+                    }
+                    st_img8(img_L, t, j0, lv);
+                }
+            }
+        }
+    }
+    if (!failed) {
+        __syncthreads();
+        if (!neu) {
+            gen::inverse64_inplace(Mf, Tf, tid);
+        } else {
+            // ---- truncated Neumann series (Horner) + Newton residual steps, M = 64 on tcgen05
+            const uint32_t NB = base_u32 + Ly.NB, XB = base_u32 + Ly.XB, RB = base_u32 + Ly.RB;
+            const uint32_t tn = tmem + Ly.tn, tqn = tq + Ly.tn;
+            for (int u = tid; u < CC * 8; u += NT) {
+                const int t = u >> 3, j = (u & 7) * 8;
+                float v8[8], x8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    v8[e] = Mf[t * LDM + j + e];
+                    x8[e] = (t == j + e) ? 1.f : 0.f;
+                }
+                st_tile8(NB, 64, t, j, v8);
+                st_tile8(XB, 64, t, j, x8);
+            }
+            fence_proxy_async_smem();
+            __syncthreads();
+            const int rr = gen::row64g(warp, lane);
+            const int cb = 32 * (warp >> 2);
+            const uint32_t id = idesc_bf16(64, 64, false, true);
+            auto product = [&](uint32_t a_tile, uint32_t b_tile) {   // tn = A (K-major) * B (MN-major)
+                if (tid == 0) {
+                    tc_fence_after();
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tn, desc_kmajor(a_tile, 64, 0, k0), desc_mnmajor(b_tile, 64, k0, 0), id,
+                                 k0 > 0);
+                    mma_commit(&bars[1]);
+                }
+                const bool f = wait_bar(1, ph_mma);
+                ph_mma ^= 1u;
+                return f;
+            };
+            for (int pw = 1; pw <= p.neu_order && !failed; ++pw) {
+                if ((failed = product(NB, XB)))
+                    break;
+                tc_fence_after();
+                float d0[16], d1[16];
+                tmem_ld16(tqn + cb, d0);
+                tmem_ld16(tqn + cb + 16, d1);
+                tmem_ld_wait();
+                if (rr >= 0) {
+                    float x[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        x[u] = ((rr == cb + u) ? 1.f : 0.f) - (u < 16 ? d0[u] : d1[u - 16]);
+#pragma unroll
+                    for (int u = 0; u < 32; u += 8)
+                        st_tile8(XB, 64, rr, cb + u, &x[u]);
+                    if (pw == p.neu_order)
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            Mf[rr * LDM + cb + u] = x[u];
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+            }
+            if (!failed && p.neu_order == 0) {
+                for (int u = tid; u < CC * CC; u += NT)
+                    Mf[(u / CC) * LDM + (u % CC)] = ((u / CC) == (u % CC)) ? 1.f : 0.f;
+                __syncthreads();
+            }
+            // Newton: Rm = I - X - N X ; X <- X + X Rm
+            for (int st = 0; st < p.neu_resid && !failed; ++st) {
+                if ((failed = product(NB, XB)))
+                    break;
+                tc_fence_after();
+                float d0[16], d1[16];
+                tmem_ld16(tqn + cb, d0);
+                tmem_ld16(tqn + cb + 16, d1);
+                tmem_ld_wait();
+                if (rr >= 0) {
+                    float rm[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        rm[u] = ((rr == cb + u) ? 1.f : 0.f) - Mf[rr * LDM + cb + u] -
+                                (u < 16 ? d0[u] : d1[u - 16]);
+#pragma unroll
+                    for (int u = 0; u < 32; u += 8)
+                        st_tile8(RB, 64, rr, cb + u, &rm[u]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                if ((failed = product(XB, RB)))
+                    break;
+                tc_fence_after();
+                tmem_ld16(tqn + cb, d0);
+                tmem_ld16(tqn + cb + 16, d1);
+                tmem_ld_wait();
+                if (rr >= 0) {
+                    float x[32];
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        x[u] = Mf[rr * LDM + cb + u] + (u < 16 ? d0[u] : d1[u - 16]);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        Mf[rr * LDM + cb + u] = x[u];
+#pragma unroll
+                    for (int u = 0; u < 32; u += 8)
+                        st_tile8(XB, 64, rr, cb + u, &x[u]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+            }
+        }
+    }
+    if (!failed) {
+        __syncthreads();
+        // ---- T = diag(beta) A as a tile image: thread u writes 16-byte chunk u (coalesced)
+        for (int u = tid; u < CC * 8; u += NT) {
+            const int r = u >> 3, cc = (u & 7) ^ (r & 7);
+            const float bt = sbeta[r];
+            const float4 x0 = *reinterpret_cast<const float4 *>(&Mf[r * LDM + 8 * cc]);
+            const float4 x1 = *reinterpret_cast<const float4 *>(&Mf[r * LDM + 8 * cc + 4]);
+            *reinterpret_cast<uint4 *>(img_T + 16 * u) =
+                make_uint4(pack_bf16(bt * x0.x, bt * x0.y), pack_bf16(bt * x0.z, bt * x0.w),
+                           pack_bf16(bt * x1.x, bt * x1.y), pack_bf16(bt * x1.z, bt * x1.w));
+            if (a.kind == REC_SCALAR) {   // Abe = T diag(e^{Lambda_j}), e^{Lambda_j} <= 1
+                float e[8];
+#pragma unroll
+                for (int f = 0; f < 8; ++f)
+                    e[f] = bt * __expf(lam[8 * cc + f]);
+                *reinterpret_cast<uint4 *>(img_T + SC_ABE + 16 * u) =
+                    make_uint4(pack_bf16(e[0] * x0.x, e[1] * x0.y), pack_bf16(e[2] * x0.z, e[3] * x0.w),
+                               pack_bf16(e[4] * x1.x, e[5] * x1.y), pack_bf16(e[6] * x1.z, e[7] * x1.w));
+            }
+        }
+    }
+    // drain: whatever was started must finish before tensor memory is released (bounded)
+    if (tid == 0 && failed) {
+        mma_commit(&bars[1]);
+        mbar_wait(&bars[1], ph_mma, 200000000ull);
+        mbar_wait(&bars[0], 0, 200000000ull);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Ly.tmem_cols);
+    }
+}
+
+inline int nchunks(const Params &p) { return (p.T + CC - 1) / CC; }
+
+inline size_t bytes(const Params &p)
+{
+    return (size_t)p.B * p.Hk * nchunks(p) * CHUNK_BYTES;
+}
+
+// Record of the two-pass path's workspace.
+inline int record_kind(const Params &p) { return p.G > 1 ? REC_EXT : REC_SCALAR; }
+
+inline uint32_t kind_bytes(int kind)
+{
+    return kind == REC_EXT ? EXT_BYTES : (kind == REC_SCALAR ? SC_BYTES : CHUNK_BYTES);
+}
+
+inline uint32_t rec_bytes(const Params &p) { return kind_bytes(record_kind(p)); }
+
+inline size_t ws_bytes(const Params &p) { return (size_t)p.B * p.Hk * nchunks(p) * rec_bytes(p); }
+
+inline bool supports(const Params &p)
+{
+    return p.in_bf16 && p.C == CC && (p.dk == 128 || p.dk == 256) && p.G >= 1 &&
+           p.G <= gmax(p.dk) && p.Hk <= 65535 && p.B <= 65535;
+}
+
+template <int DK>
+int launch(const Params &p, void *out, int kind, cudaStream_t stream)
+{
+    const int N = nchunks(p);
+    if (N == 0 || p.B == 0)
+        return 0;
+    CUtensorMap mq, mk;
+    const long sk = (long)p.B * p.Hk;
+    if (!make_map(&mq, p.q, DK, p.T, sk, CC) || !make_map(&mk, p.k, DK, p.T, sk, CC))
+        return 6;
+    const Plan Ly = plan(DK, p.G, p.neumann != 0);
+    auto kern = prep_kernel<DK>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
+        cudaSuccess)
+        return 6;
+    PrepArgs a;
+    a.p = p;
+    a.out = static_cast<uint8_t *>(out);
+    a.nchunks = N;
+    a.kind = kind;
+    a.rec_bytes = kind_bytes(kind);
+    dim3 grid(N, p.Hk, p.B);
+    kern<<<grid, NT, Ly.total, stream>>>(mq, mk, a);
+    return cudaGetLastError() == cudaSuccess ? 0 : 6;
+}
+
+}  // namespace prep

@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(PKG, "libgdr.so")
 
 # gdr_status
 OK, ERR_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, \
-    ERR_NONFINITE = range(9)
+    ERR_NONFINITE, ERR_WORKSPACE = range(10)
 # gdr_dtype
 F32, BF16 = 0, 1
 # gdr_gate_mode
@@ -23,14 +23,22 @@ GATE_SCALAR, GATE_GROUP64, GATE_CHANNEL = 0, 1, 2
 # gdr_inverse_mode
 INV_EXACT, INV_NEUMANN = 0, 1
 # gdr_kernel
-KERNEL_AUTO, KERNEL_SIMT, KERNEL_TC = 0, 1, 2
+KERNEL_AUTO, KERNEL_SIMT, KERNEL_TC, KERNEL_TC2 = 0, 1, 2, 3
 
-_KERNELS = {"auto": KERNEL_AUTO, "simt": KERNEL_SIMT, "tc": KERNEL_TC}
+_KERNELS = {"auto": KERNEL_AUTO, "simt": KERNEL_SIMT, "tc": KERNEL_TC, "tc2": KERNEL_TC2}
+KERNEL_NAMES = {KERNEL_SIMT: "simt", KERNEL_TC: "tc", KERNEL_TC2: "tc2"}
+
+# bytes of one chunk record written by gdr_chunk_prepare (T then L, 64 x 64 bf16 each)
+PREP_CHUNK_BYTES = 16384
+# bytes of one workspace record of the two-pass kernel: scalar gate, grouped / per-channel gates
+TC2_SCALAR_RECORD_BYTES = 25104
+TC2_EXT_RECORD_BYTES = 66048
 _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN}
 
 # Every symbol include/gdr.h declares.
-EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_host", "gdr_select_kernel", "gdr_kernel_chunk",
-           "gdr_device_status", "gdr_status_string", "gdr_version")
+EXPORTS = ("gdr_chunk_fwd", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
+           "gdr_select_kernel", "gdr_kernel_chunk", "gdr_device_status", "gdr_status_string",
+           "gdr_version")
 
 
 class GdrShape(ctypes.Structure):
@@ -65,12 +73,17 @@ def load(path: str = LIB_PATH):
         raise RuntimeError("libgdr.so not found at %s; build it with "
                            "`python -m gated_delta_rule_141_b200.build`" % path)
     lib = ctypes.CDLL(path)
-    vp, i = ctypes.c_void_p, ctypes.c_int
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     lib.gdr_chunk_fwd.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i, i,
-                                  vp, vp, vp]
+                                  vp, vp, vp, sz, vp]
     lib.gdr_chunk_fwd.restype = i
+    lib.gdr_workspace_bytes.argtypes = [ctypes.POINTER(GdrShape), i, i, i, ctypes.POINTER(sz)]
+    lib.gdr_workspace_bytes.restype = i
+    lib.gdr_chunk_prepare.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, i, i, i, vp, sz,
+                                      vp]
+    lib.gdr_chunk_prepare.restype = i
     lib.gdr_chunk_fwd_host.argtypes = [ctypes.POINTER(GdrShape), ctypes.POINTER(GdrIO),
-                                       ctypes.POINTER(GdrIO), i, i, i, vp]
+                                       ctypes.POINTER(GdrIO), i, i, i, vp, sz, vp]
     lib.gdr_chunk_fwd_host.restype = i
     lib.gdr_select_kernel.argtypes = [ctypes.POINTER(GdrShape), i, i, i]
     lib.gdr_select_kernel.restype = i
@@ -122,6 +135,16 @@ def kernel_chunk(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "ex
                                        _INVERSES[inverse]))
 
 
+def workspace_bytes(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "exact") -> int:
+    """Device workspace gdr_chunk_fwd needs for this request (raises if rejected)."""
+    n = ctypes.c_size_t(0)
+    st = load().gdr_workspace_bytes(ctypes.byref(shape), int(chunk), int(gate_mode),
+                                    _INVERSES[inverse], ctypes.byref(n))
+    if st != OK:
+        raise GdrError(st, "gdr_workspace_bytes")
+    return int(n.value)
+
+
 def device_status(stream=None) -> int:
     return int(load().gdr_device_status(_stream_handle(stream)))
 
@@ -148,13 +171,14 @@ def _ptr(t):
 
 def chunk_fwd(q, k, v, g, beta, S0=None, chunk=64, gate_mode=None, inverse="exact",
               neumann_order=4, neumann_residual_steps=1, out_dtype=None, o=None,
-              S_final=None, want_state=True, kernel="auto", stream=None):
+              S_final=None, want_state=True, kernel="auto", workspace=None, stream=None):
     """Chunkwise gated delta-rule forward on the current CUDA device.
 
     q, k [B,Hk,T,dk] and v [B,Hv,T,dv] (bf16 or fp32, same dtype); g [B,Hk,T,G] and
     beta [B,Hk,T] fp32; S0 [B,Hv,dk,dv] fp32 or None.  Returns (o, S_final);
-    S_final is None when want_state is False.  Outputs are allocated with torch
-    unless passed in.  Runs asynchronously on `stream` (default: torch's current).
+    S_final is None when want_state is False.  Outputs and the workspace the selected
+    kernel needs are allocated with torch unless passed in.  Runs asynchronously on
+    `stream` (default: torch's current).
     """
     import torch
     B, Hk, T, dk = q.shape
@@ -174,17 +198,43 @@ def chunk_fwd(q, k, v, g, beta, S0=None, chunk=64, gate_mode=None, inverse="exac
         S_final = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
     shape = make_shape(B, T, Hk, Hv, dk, dv, _dtype_code(q.dtype), _dtype_code(o.dtype),
                        neumann_order, neumann_residual_steps, kernel)
+    if workspace is None:
+        nbytes = workspace_bytes(shape, chunk, gate_mode, inverse)
+        workspace = (torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None)
     st = load().gdr_chunk_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                               _ptr(beta), _ptr(S0), int(chunk), int(gate_mode),
-                              _INVERSES[inverse], _ptr(o), _ptr(S_final),
+                              _INVERSES[inverse], _ptr(o), _ptr(S_final), _ptr(workspace),
+                              0 if workspace is None else workspace.numel(),
                               _stream_handle(stream))
     if st != OK:
         raise GdrError(st)
     return o, S_final
 
 
+def chunk_prepare(q, k, g, beta, chunk=64, gate_mode=None, inverse="exact", neumann_order=4,
+                  neumann_residual_steps=1, factors=None, stream=None):
+    """gdr_chunk_prepare: the chunk factors T = diag(beta) (I + M)^{-1} and L of every
+    chunk.  Returns a uint8 device tensor [B, Hk, ceil(T/64), 16384] of tile images
+    (see include/gdr.h for the byte layout)."""
+    import torch
+    B, Hk, T, dk = q.shape
+    if gate_mode is None:
+        gate_mode = gate_mode_for(g.shape[-1], dk)
+    nch = (T + 63) // 64
+    if factors is None:
+        factors = torch.empty((B, Hk, nch, PREP_CHUNK_BYTES), dtype=torch.uint8, device=q.device)
+    shape = make_shape(B, T, Hk, Hk, dk, dk, _dtype_code(q.dtype), BF16, neumann_order,
+                       neumann_residual_steps)
+    st = load().gdr_chunk_prepare(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(g), _ptr(beta),
+                                  int(chunk), int(gate_mode), _INVERSES[inverse], _ptr(factors),
+                                  factors.numel(), _stream_handle(stream))
+    if st != OK:
+        raise GdrError(st, "gdr_chunk_prepare")
+    return factors
+
+
 def chunk_fwd_host(host: dict, dev: dict, shape: GdrShape, chunk: int, gate_mode: int,
-                   inverse: str = "exact", stream=None):
+                   inverse: str = "exact", workspace=None, stream=None):
     """gdr_chunk_fwd_host: inputs/outputs in (pinned) host tensors, device buffers
     supplied by the caller.  Both dicts map q, k, v, g, beta, S0, o, S_final to
     tensors (S0 / S_final may be None)."""
@@ -193,6 +243,7 @@ def chunk_fwd_host(host: dict, dev: dict, shape: GdrShape, chunk: int, gate_mode
     d = GdrIO(*[_ptr(dev.get(n)) for n in names])
     st = load().gdr_chunk_fwd_host(ctypes.byref(shape), ctypes.byref(h), ctypes.byref(d),
                                    int(chunk), int(gate_mode), _INVERSES[inverse],
+                                   _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                    _stream_handle(stream))
     if st != OK:
         raise GdrError(st, "gdr_chunk_fwd_host")

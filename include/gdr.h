@@ -34,6 +34,8 @@
 #ifndef GDR_H_
 #define GDR_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -47,7 +49,8 @@ typedef enum {
     GDR_ERR_UNSUPPORTED = 5, /* valid request no kernel here implements        */
     GDR_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed           */
     GDR_ERR_TIMEOUT = 7,     /* a bounded on-device wait gave up               */
-    GDR_ERR_NONFINITE = 8    /* reserved: non-finite input detected            */
+    GDR_ERR_NONFINITE = 8,   /* reserved: non-finite input detected            */
+    GDR_ERR_WORKSPACE = 9    /* workspace smaller than the selected kernel needs */
 } gdr_status;
 
 typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
@@ -65,12 +68,21 @@ typedef enum { GDR_GATE_SCALAR = 0, GDR_GATE_GROUP64 = 1, GDR_GATE_CHANNEL = 2 }
  *          (Multiplication-Only Matrix Inversion ..., Lemma 3.1, §4.1)      */
 typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1 } gdr_inverse_mode;
 
-/* Kernel selection.  AUTO picks the tensor-core kernel whenever the request
- * is inside its envelope (bf16 inputs, dk in {64,128,256}, dv % 16 == 0,
- * chunk in {64,128}) and the CUDA-core kernel otherwise.  SIMT forces the
- * fp32 CUDA-core kernel; TC forces the tensor-core kernel and fails with
- * GDR_ERR_UNSUPPORTED outside its envelope.                                 */
-typedef enum { GDR_KERNEL_AUTO = 0, GDR_KERNEL_SIMT = 1, GDR_KERNEL_TC = 2 } gdr_kernel;
+/* Kernel selection.
+ *  TC    one fused tensor-core kernel per (batch, value head, 64 value
+ *        columns) that walks the chunks in order (bf16 inputs, dk in
+ *        {64,128,256}, dv % 64 == 0, chunk 64, or 128 in exact mode).
+ *  TC2   two tensor-core passes: the chunk-local factors of every chunk in
+ *        parallel (gdr_chunk_prepare), written to the caller's workspace, then
+ *        the state pass that reads them (bf16 inputs, dk = 128, dv % 64 == 0,
+ *        chunk 64, or 128 in exact mode).  Needs gdr_workspace_bytes() of
+ *        device workspace.
+ *  SIMT  the fp32 CUDA-core kernel (any dtype, chunk 1..128).
+ *  AUTO  TC2 when it applies and the call's workspace is large enough, else
+ *        TC when it applies, else SIMT.  Forcing a kernel outside its
+ *        envelope fails with GDR_ERR_UNSUPPORTED.                           */
+typedef enum { GDR_KERNEL_AUTO = 0, GDR_KERNEL_SIMT = 1, GDR_KERNEL_TC = 2,
+               GDR_KERNEL_TC2 = 3 } gdr_kernel;
 
 typedef struct {
     int B;      /* batch, >= 0                                               */
@@ -102,6 +114,8 @@ typedef struct {
  *   o      [B, Hv, T, dv]  out_dtype
  *   S_final[B, Hv, dk, dv] fp32 state after token T, or NULL to skip
  * chunk: chunk length C, 1..128 (see gdr_kernel_chunk for the blocking used).
+ * workspace, workspace_bytes: device scratch for the TC2 kernel (see
+ *   gdr_workspace_bytes), or NULL, 0; the one-pass kernels use none.
  * Returns GDR_OK once the work is queued on `stream`.  Kernel-side wait
  * timeouts are reported through gdr_device_status().
  */
@@ -109,7 +123,41 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape,
                          const void *q, const void *k, const void *v,
                          const float *g, const float *beta, const float *S0,
                          int chunk, gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode,
-                         void *o, float *S_final, void *stream);
+                         void *o, float *S_final,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device workspace (bytes) that gdr_chunk_fwd needs for this request with the
+ * kernel AUTO or shape->kernel selects when given enough: 0 for the one-pass
+ * kernels; for TC2, B * Hk * ceil(T / 64) records of 25104 bytes (scalar gate)
+ * or 66048 bytes (grouped / per-channel gates): the chunk factors T and L plus
+ * the decayed operands and decay factors the second pass reads.  The caller allocates it
+ * (16-byte aligned) and passes it with its size; its contents on entry do not
+ * matter.  A call
+ * whose workspace is smaller falls back (AUTO) or fails with
+ * GDR_ERR_WORKSPACE (TC2 forced).  Calls that share a workspace must not
+ * overlap on the GPU. */
+gdr_status gdr_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                               gdr_inverse_mode inverse_mode, size_t *bytes);
+
+/*
+ * gdr_chunk_prepare -- the chunk-local factors of every chunk, all chunks in
+ * parallel (the first pass of TC2).  Per (b, hk, chunk n) of C = 64 tokens,
+ * with Lambda = cumsum of g inside the chunk and decays exp(Lambda_t - Lambda_j):
+ *   L_tj = (t >= j) sum_i q_ti k_ji exp(Lambda_ti - Lambda_ji)
+ *   M_tj = (t >  j) beta_j sum_i k_ti k_ji exp(Lambda_ti - Lambda_ji)
+ *   T    = diag(beta) (I + M)^{-1}  (exact or Neumann, as inverse_mode)
+ * (SLA §2.1, §2.3 Table 2; rows past T are zero).
+ * Output `factors` (device, written): [B][Hk][ceil(T/64)] records of 16384
+ * bytes: T then L, each a 64 x 64 bf16 matrix stored as 64 rows of 128 bytes
+ * in which the 16-byte piece holding columns 8c..8c+7 of row r sits at
+ * position (c XOR (r mod 8)) -- the 128-byte-swizzled tile layout.
+ * factors_bytes must be at least B * Hk * ceil(T/64) * 16384.  Needs bf16
+ * q, k, dk in {128, 256} and chunk 64; q, k, g, beta as for gdr_chunk_fwd.
+ */
+gdr_status gdr_chunk_prepare(const gdr_shape *shape, const void *q, const void *k,
+                             const float *g, const float *beta, int chunk,
+                             gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode,
+                             void *factors, size_t factors_bytes, void *stream);
 
 /* Buffers of one call, either all on the host or all on the device. */
 typedef struct {
@@ -125,15 +173,17 @@ typedef struct {
  * (cudaMemcpyAsync, one copy per tensor; pinned host memory makes them
  * asynchronous), runs gdr_chunk_fwd on them and copies o and S_final back to
  * `host`, all on `stream`.  The host outputs are valid after the stream
- * synchronises.  `dev` must satisfy gdr_chunk_fwd's rules; host pointers
- * need no alignment.
+ * synchronises.  `dev` and the device `workspace` must satisfy
+ * gdr_chunk_fwd's rules; host pointers need no alignment.
  */
 gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const gdr_io *dev,
                               int chunk, gdr_gate_mode gate_mode,
-                              gdr_inverse_mode inverse_mode, void *stream);
+                              gdr_inverse_mode inverse_mode,
+                              void *workspace, size_t workspace_bytes, void *stream);
 
-/* Which kernel gdr_chunk_fwd would launch for this request: GDR_KERNEL_SIMT or
- * GDR_KERNEL_TC, or a negative gdr_status value if it would be rejected. */
+/* Which kernel gdr_chunk_fwd would launch for this request when given the
+ * workspace gdr_workspace_bytes asks for: GDR_KERNEL_SIMT, GDR_KERNEL_TC or
+ * GDR_KERNEL_TC2, or a negative gdr_status value if it would be rejected. */
 int gdr_select_kernel(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
                       gdr_inverse_mode inverse_mode);
 

@@ -39,29 +39,32 @@ def test_enums_match_header():
         return int(re.search(r"\b%s\s*=\s*(\d+)" % name, text).group(1))
     assert [val("GDR_OK"), val("GDR_ERR_ARG"), val("GDR_ERR_SHAPE"), val("GDR_ERR_DTYPE"),
             val("GDR_ERR_ALIGN"), val("GDR_ERR_UNSUPPORTED"), val("GDR_ERR_CUDA"),
-            val("GDR_ERR_TIMEOUT"), val("GDR_ERR_NONFINITE")] == list(range(9))
+            val("GDR_ERR_TIMEOUT"), val("GDR_ERR_NONFINITE"), val("GDR_ERR_WORKSPACE")] == list(range(10))
+    assert val("GDR_ERR_WORKSPACE") == gdr.ERR_WORKSPACE
     assert (val("GDR_F32"), val("GDR_BF16")) == (gdr.F32, gdr.BF16)
     assert (val("GDR_GATE_SCALAR"), val("GDR_GATE_GROUP64"), val("GDR_GATE_CHANNEL")) == (
         gdr.GATE_SCALAR, gdr.GATE_GROUP64, gdr.GATE_CHANNEL)
     assert (val("GDR_INV_EXACT"), val("GDR_INV_NEUMANN")) == (gdr.INV_EXACT, gdr.INV_NEUMANN)
-    assert (val("GDR_KERNEL_AUTO"), val("GDR_KERNEL_SIMT"), val("GDR_KERNEL_TC")) == (
-        gdr.KERNEL_AUTO, gdr.KERNEL_SIMT, gdr.KERNEL_TC)
+    assert (val("GDR_KERNEL_AUTO"), val("GDR_KERNEL_SIMT"), val("GDR_KERNEL_TC"),
+            val("GDR_KERNEL_TC2")) == (gdr.KERNEL_AUTO, gdr.KERNEL_SIMT, gdr.KERNEL_TC,
+                                       gdr.KERNEL_TC2)
     # struct layout: 11 ints
     assert ctypes.sizeof(gdr.GdrShape) == 44
 
 
 def test_status_strings_and_version(lib):
-    for s in range(9):
-        assert gdr.status_string(s)
+    for s in range(10):
+        assert gdr.status_string(s) != "unknown status"
     assert gdr.status_string(123) == "unknown status"
     assert gdr.version() >= 100
 
 
-def _call(shape, ptrs=None, chunk=64, gate=gdr.GATE_SCALAR, inv=gdr.INV_EXACT):
+def _call(shape, ptrs=None, chunk=64, gate=gdr.GATE_SCALAR, inv=gdr.INV_EXACT, ws=None,
+          ws_bytes=0):
     # fake but 16-byte-aligned device addresses: validation fails before any use
     p = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(8)] if ptrs is None else ptrs
     return gdr.load().gdr_chunk_fwd(ctypes.byref(shape), p[0], p[1], p[2], p[3], p[4], p[5],
-                                    chunk, gate, inv, p[6], p[7], None)
+                                    chunk, gate, inv, p[6], p[7], ws, ws_bytes, None)
 
 
 def test_rejects_bad_shapes(lib):
@@ -88,7 +91,7 @@ def test_rejects_bad_enums_and_dtypes(lib):
     assert _call(gdr.make_shape(**ok, out_dtype=5)) == gdr.ERR_DTYPE
     assert _call(gdr.make_shape(**ok, kernel=9)) == gdr.ERR_ARG
     assert gdr.load().gdr_chunk_fwd(None, None, None, None, None, None, None, 64, 0, 0,
-                                    None, None, None) == gdr.ERR_ARG
+                                    None, None, None, 0, None) == gdr.ERR_ARG
 
 
 def test_rejects_null_and_misaligned(lib):
@@ -111,7 +114,11 @@ def test_empty_batch_is_a_no_op(lib):
 
 def test_kernel_selection(lib):
     bf = gdr.make_shape(4, 4096, 16, 16, 128, 128)
-    assert gdr.select_kernel(bf, 64, gdr.GATE_SCALAR) in (gdr.KERNEL_TC, gdr.KERNEL_SIMT)
+    assert gdr.select_kernel(bf, 64, gdr.GATE_SCALAR) == gdr.KERNEL_TC2
+    assert gdr.select_kernel(gdr.make_shape(4, 4096, 16, 16, 128, 128, kernel="tc"), 64,
+                             gdr.GATE_SCALAR) == gdr.KERNEL_TC
+    assert gdr.select_kernel(gdr.make_shape(2, 8192, 8, 32, 256, 128), 64,
+                             gdr.GATE_GROUP64) == gdr.KERNEL_TC
     f32 = gdr.make_shape(1, 256, 2, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
     assert gdr.select_kernel(f32, 64, gdr.GATE_SCALAR) == gdr.KERNEL_SIMT
     forced = gdr.make_shape(1, 256, 2, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32,
@@ -125,7 +132,7 @@ def test_kernel_chunk(lib):
     # Exact mode: chunk 128 on the tensor-core kernel blocks by 64 (same function);
     # the Neumann inverse depends on C and keeps the requested blocking.
     kda = gdr.make_shape(2, 8192, 32, 32, 128, 128)
-    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL) == gdr.KERNEL_TC
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL) == gdr.KERNEL_TC2
     assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL) == 64
     assert gdr.kernel_chunk(kda, 64, gdr.GATE_CHANNEL) == 64
     assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL, "neumann") == 128
@@ -140,6 +147,52 @@ def test_host_entry_validates(lib):
     shape = gdr.make_shape(1, 64, 2, 4, 64, 64)
     io = gdr.GdrIO()
     assert gdr.load().gdr_chunk_fwd_host(ctypes.byref(shape), None, ctypes.byref(io), 64, 0, 0,
-                                         None) == gdr.ERR_ARG
+                                         None, 0, None) == gdr.ERR_ARG
     assert gdr.load().gdr_chunk_fwd_host(ctypes.byref(shape), ctypes.byref(io),
-                                         ctypes.byref(io), 64, 0, 0, None) == gdr.ERR_ARG
+                                         ctypes.byref(io), 64, 0, 0, None, 0, None) == gdr.ERR_ARG
+
+
+def test_workspace_rules(lib):
+    # two-pass path: dk = 128 bf16; the workspace is B * Hk * ceil(T/64) chunk records
+    sh = gdr.make_shape(2, 200, 3, 6, 128, 128)
+    need = gdr.workspace_bytes(sh, 64, gdr.GATE_CHANNEL)
+    assert need == 2 * 3 * 4 * gdr.TC2_EXT_RECORD_BYTES
+    assert gdr.workspace_bytes(sh, 64, gdr.GATE_SCALAR) == 2 * 3 * 4 * gdr.TC2_SCALAR_RECORD_BYTES
+    assert gdr.select_kernel(sh, 64, gdr.GATE_CHANNEL) == gdr.KERNEL_TC2
+    # exact C = 128 runs blocked by 64 on the two-pass path too
+    assert gdr.workspace_bytes(sh, 128, gdr.GATE_CHANNEL) == need
+    forced = gdr.make_shape(2, 200, 3, 6, 128, 128, kernel="tc2")
+    assert _call(forced, gate=gdr.GATE_CHANNEL) == gdr.ERR_WORKSPACE
+    assert _call(forced, gate=gdr.GATE_CHANNEL, ws=ctypes.c_void_p(0x900000),
+                 ws_bytes=need - 16) == gdr.ERR_WORKSPACE
+    assert _call(forced, gate=gdr.GATE_CHANNEL, ws=ctypes.c_void_p(0x900004),
+                 ws_bytes=need) == gdr.ERR_ALIGN
+    # the one-pass kernels need none; forcing the two-pass kernel outside its envelope
+    assert gdr.workspace_bytes(gdr.make_shape(1, 64, 1, 1, 256, 128), 64, gdr.GATE_SCALAR) == 0
+    assert gdr.workspace_bytes(gdr.make_shape(1, 64, 1, 1, 64, 64, in_dtype=gdr.F32,
+                                              out_dtype=gdr.F32), 64, gdr.GATE_SCALAR) == 0
+    with pytest.raises(gdr.GdrError):
+        gdr.workspace_bytes(gdr.make_shape(1, 64, 1, 1, 256, 128, kernel="tc2"), 64,
+                            gdr.GATE_SCALAR)
+    n = ctypes.c_size_t(0)
+    assert lib.gdr_workspace_bytes(ctypes.byref(sh), 64, 0, 0, None) == gdr.ERR_ARG
+    assert lib.gdr_workspace_bytes(ctypes.byref(sh), 64, 0, 7, ctypes.byref(n)) == gdr.ERR_ARG
+
+
+def test_prepare_validates(lib):
+    sh = gdr.make_shape(1, 130, 2, 2, 128, 128)
+    need = 1 * 2 * 3 * gdr.PREP_CHUNK_BYTES
+    p = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(5)]
+    call = lambda shape, ptrs, chunk=64, nbytes=need: lib.gdr_chunk_prepare(
+        ctypes.byref(shape), ptrs[0], ptrs[1], ptrs[2], ptrs[3], chunk, gdr.GATE_SCALAR,
+        gdr.INV_EXACT, ptrs[4], nbytes, None)
+    assert call(sh, p, nbytes=need - 1) == gdr.ERR_WORKSPACE
+    assert call(sh, p, chunk=32) == gdr.ERR_UNSUPPORTED
+    assert call(gdr.make_shape(1, 130, 2, 2, 64, 64), p) == gdr.ERR_UNSUPPORTED
+    for i in range(5):
+        q = list(p)
+        q[i] = None
+        assert call(sh, q) == gdr.ERR_ARG, i
+        q[i] = ctypes.c_void_p(0x10000 * (i + 1) + 8)
+        assert call(sh, q) == gdr.ERR_ALIGN, i
+    assert call(gdr.make_shape(0, 130, 2, 2, 128, 128), [None] * 5) == gdr.OK

@@ -52,6 +52,15 @@ SMALL = [
     (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 128, "exact", "tc"),
     (3, dict(B=1, Hk=1, Hv=4, T=384 - 37), 128, "exact", "tc"),
     (4, dict(Hk=2, Hv=2, T=640), 128, "exact", "tc"),
+    # two-pass tensor-core path (chunk factors in a workspace, then the state pass)
+    (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 64, "exact", "tc2"),
+    (1, dict(B=2, Hk=1, Hv=3, T=256, dv=192), 64, "exact", "tc2"),      # grouped values, 3 tiles
+    (1, dict(B=1, Hk=1, Hv=1, T=256), 64, "neumann", "tc2"),
+    (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 64, "exact", "tc2"),
+    (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 64, "exact", "tc2"),
+    (2, dict(B=1, Hk=2, Hv=2, T=256), 64, "neumann", "tc2"),
+    (4, dict(Hk=2, Hv=2, T=640 - 5), 128, "exact", "tc2"),               # strong decay, S0
+    (4, dict(Hk=1, Hv=1, T=64), 64, "exact", "tc2"),                     # a single chunk
 ]
 
 
@@ -103,7 +112,9 @@ def test_host_entry_matches_device_entry():
     dev["o"] = torch.empty_like(o_dev)
     dev["S_final"] = torch.empty_like(S_dev)
     shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv)
-    gdr.chunk_fwd_host(host, dev, shape, 64, gdr.GATE_SCALAR)
+    ws = torch.empty(gdr.workspace_bytes(shape, 64, gdr.GATE_SCALAR), dtype=torch.uint8,
+                     device="cuda")
+    gdr.chunk_fwd_host(host, dev, shape, 64, gdr.GATE_SCALAR, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(host["o"], o_dev.cpu())
     assert torch.equal(host["S_final"], S_dev.cpu())
