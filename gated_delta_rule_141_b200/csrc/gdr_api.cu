@@ -262,6 +262,8 @@ const char *gdr_status_string(gdr_status status)
     case GDR_ERR_TIMEOUT: return "a bounded device wait gave up";
     case GDR_ERR_NONFINITE: return "non-finite input";
     case GDR_ERR_WORKSPACE: return "workspace smaller than the selected kernel needs";
+    case GDR_ERR_SCRATCH_LIMIT:
+        return "request needs more than the GDR_STATIC_SCRATCH_BYTES scratch of gdr_chunk_fwd_static";
     }
     return "unknown status";
 }

@@ -15,7 +15,10 @@ LIB_PATH = os.path.join(PKG, "libgdr.so")
 
 # gdr_status
 OK, ERR_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, \
-    ERR_NONFINITE, ERR_WORKSPACE = range(10)
+    ERR_NONFINITE, ERR_WORKSPACE, ERR_SCRATCH_LIMIT = range(11)
+
+# size of the fixed device array gdr_chunk_fwd_static uses as its workspace
+STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
 # gdr_dtype
 F32, BF16 = 0, 1
 # gdr_gate_mode
@@ -37,6 +40,7 @@ _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN}
 
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_chunk_fwd", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
+           "gdr_chunk_fwd_static",
            "gdr_select_kernel", "gdr_kernel_chunk", "gdr_device_status", "gdr_status_string",
            "gdr_version")
 
@@ -77,6 +81,9 @@ def load(path: str = LIB_PATH):
     lib.gdr_chunk_fwd.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i, i,
                                   vp, vp, vp, sz, vp]
     lib.gdr_chunk_fwd.restype = i
+    lib.gdr_chunk_fwd_static.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i,
+                                         i, vp, vp, vp]
+    lib.gdr_chunk_fwd_static.restype = i
     lib.gdr_workspace_bytes.argtypes = [ctypes.POINTER(GdrShape), i, i, i, ctypes.POINTER(sz)]
     lib.gdr_workspace_bytes.restype = i
     lib.gdr_chunk_prepare.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, i, i, i, vp, sz,

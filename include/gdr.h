@@ -50,7 +50,9 @@ typedef enum {
     GDR_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed           */
     GDR_ERR_TIMEOUT = 7,     /* a bounded on-device wait gave up               */
     GDR_ERR_NONFINITE = 8,   /* reserved: non-finite input detected            */
-    GDR_ERR_WORKSPACE = 9    /* workspace smaller than the selected kernel needs */
+    GDR_ERR_WORKSPACE = 9,   /* workspace smaller than the selected kernel needs */
+    GDR_ERR_SCRATCH_LIMIT = 10 /* request needs more scratch than
+                                  gdr_chunk_fwd_static's fixed array holds      */
 } gdr_status;
 
 typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
@@ -180,6 +182,41 @@ gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const 
                               int chunk, gdr_gate_mode gate_mode,
                               gdr_inverse_mode inverse_mode,
                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Size of the device array gdr_chunk_fwd_static uses as its workspace. */
+#define GDR_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * gdr_chunk_fwd_static -- gdr_chunk_fwd on the TC2 kernel, with no workspace
+ * argument: for callers that may not allocate device memory on their call
+ * path, such as a serving engine whose memory planner owns all device memory
+ * once it has started, or a latency-critical loop that cannot afford the
+ * device-wide synchronisation an allocation can cause.  (The paper has no
+ * counterpart; this is a deployment convenience of this library.)
+ *
+ * Arguments, layouts, alignment and errors are those of gdr_chunk_fwd, with
+ * shape->kernel AUTO or TC2 (anything else: GDR_ERR_UNSUPPORTED; requests
+ * outside TC2's envelope fail as a forced TC2 call does).  The workspace is a
+ * fixed array of GDR_STATIC_SCRATCH_BYTES inside the library, which every GPU
+ * that loads the library's device code holds until the process exits; a
+ * request whose TC2 workspace (gdr_workspace_bytes) is larger fails with
+ * GDR_ERR_SCRATCH_LIMIT before anything is launched.  Nothing is allocated:
+ * no cudaMalloc, no cudaFree, no allocating library call.
+ *  - Set-up: the first call on a device, made with that device current, looks
+ *    up the array's device address (cudaGetSymbolAddress) and remembers it;
+ *    make that first call before any stream capture.
+ *  - Sharing: every call on a device uses the same array, which keeps what the
+ *    last call left there.  Nothing in it needs clearing between calls (each
+ *    call rewrites all it reads), but two calls that overlap on the GPU (other
+ *    streams, other host threads) race on it: order them on one stream or
+ *    synchronise between them.
+ */
+gdr_status gdr_chunk_fwd_static(const gdr_shape *shape,
+                                const void *q, const void *k, const void *v,
+                                const float *g, const float *beta, const float *S0,
+                                int chunk, gdr_gate_mode gate_mode,
+                                gdr_inverse_mode inverse_mode,
+                                void *o, float *S_final, void *stream);
 
 /* Which kernel gdr_chunk_fwd would launch for this request when given the
  * workspace gdr_workspace_bytes asks for: GDR_KERNEL_SIMT, GDR_KERNEL_TC or

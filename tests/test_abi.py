@@ -39,7 +39,10 @@ def test_enums_match_header():
         return int(re.search(r"\b%s\s*=\s*(\d+)" % name, text).group(1))
     assert [val("GDR_OK"), val("GDR_ERR_ARG"), val("GDR_ERR_SHAPE"), val("GDR_ERR_DTYPE"),
             val("GDR_ERR_ALIGN"), val("GDR_ERR_UNSUPPORTED"), val("GDR_ERR_CUDA"),
-            val("GDR_ERR_TIMEOUT"), val("GDR_ERR_NONFINITE"), val("GDR_ERR_WORKSPACE")] == list(range(10))
+            val("GDR_ERR_TIMEOUT"), val("GDR_ERR_NONFINITE"), val("GDR_ERR_WORKSPACE"),
+            val("GDR_ERR_SCRATCH_LIMIT")] == list(range(11))
+    assert int(re.search(r"GDR_STATIC_SCRATCH_BYTES \((\d+)u \* 1024u \* 1024u\)", text).group(1)) \
+        * 1024 * 1024 == gdr.STATIC_SCRATCH_BYTES
     assert val("GDR_ERR_WORKSPACE") == gdr.ERR_WORKSPACE
     assert (val("GDR_F32"), val("GDR_BF16")) == (gdr.F32, gdr.BF16)
     assert (val("GDR_GATE_SCALAR"), val("GDR_GATE_GROUP64"), val("GDR_GATE_CHANNEL")) == (
@@ -53,7 +56,7 @@ def test_enums_match_header():
 
 
 def test_status_strings_and_version(lib):
-    for s in range(10):
+    for s in range(11):
         assert gdr.status_string(s) != "unknown status"
     assert gdr.status_string(123) == "unknown status"
     assert gdr.version() >= 100
