@@ -113,15 +113,16 @@ def files_fingerprint(files):
     return h.hexdigest()[:12]
 
 
-def recorded_traffic(workload_name: str, chunk: int, inverse: str):
-    """DRAM bytes per launch from a committed ncu summary (profiles/traffic.json),
-    or None if there is none or the kernel's source files changed since."""
+def recorded_traffic(workload_name: str, chunk: int, inverse: str, kernel: str):
+    """DRAM bytes per step (all of the step's launches) from a committed ncu summary
+    (profiles/traffic.json), or None if there is none or the kernels' source files
+    changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    e = d.get("%s/C%d/%s" % (workload_name, chunk, inverse))
+    e = d.get("%s/C%d/%s/%s" % (workload_name, chunk, inverse, kernel))
     if not e:
         return None
     try:
@@ -366,7 +367,8 @@ def main():
         roof = {"bound": "tensor", "achieved": flop / (ms_step * 1e-3) / 1e12,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tc_frac}
     roof["peak_source"] = peak_src + " (burst)"
-    roof["traffic"] = recorded_traffic(w.name, chunk, args.inverse)
+    roof["traffic"] = recorded_traffic(w.name, chunk, args.inverse,
+                                       gdr.KERNEL_NAMES.get(kern, str(kern)))
     roof["tflops"] = flop / (ms_step * 1e-3) / 1e12
     roof["tc_frac"] = tc_frac
     roof["hbm_frac"] = hbm_frac

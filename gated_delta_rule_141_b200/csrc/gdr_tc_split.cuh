@@ -17,9 +17,10 @@
 // Roles (warp-specialised, hand-offs through mbarriers):
 //   warp 0      producer: TMA q, k, v; bulk copies of T and L; 2-stage ring
 //   warp 1      MMA issuer (one thread)
-//   warps 2-5   state chain: S (fp32, TMEM) -> bf16 operand, E = U - P
-//   warps 6-9   W read-back: TMEM fp32 -> bf16 operand tile (one chunk ahead)
-//   warps 10-11 epilogue: O = f (Q S) + L E from TMEM to global memory
+//   warps 2-9   state chain: S (fp32, TMEM) -> bf16 operand, E = U - P; two
+//               warps per TMEM lane quarter, each lane on 32 of the 64 columns
+//   warps 10-13 W read-back: TMEM fp32 -> bf16 operand tile (one chunk ahead)
+//   warps 14-15 epilogue: O = f (Q S) + L E from TMEM to global memory
 // Everything decayed (Abe, Qbar, Khat, Kbar, the per-token factors, F) comes
 // from the first pass's record, so no role here evaluates an exponential.
 // Stage s holds [W | Q | K] (rows 0-63 | 64-127 | 128-191, 128 columns),
@@ -31,13 +32,13 @@
 
 namespace split {
 
-constexpr int NWARP = 12;
-constexpr int NTHR = NWARP * 32;   // 384
+constexpr int NWARP = 16;
+constexpr int NTHR = NWARP * 32;   // 512
 constexpr int CC = 64;
 constexpr int KD = 128;
 constexpr int NVC = 64;
-constexpr int W_PROD = 0, W_MMA = 1, W_STATE0 = 2, W_PREP0 = 6, W_EPI0 = 10;
-constexpr int N_STATE = 128, N_PREP = 128, N_EPI = 64;
+constexpr int W_PROD = 0, W_MMA = 1, W_STATE0 = 2, W_PREP0 = 10, W_EPI0 = 14;
+constexpr int N_STATE = 256, N_PREP = 128, N_EPI = 64;
 constexpr int NB_STATE = 1, NB_PREP = 2, NB_EPI = 3;   // named barriers
 
 constexpr uint32_t T_U = 0;        // [Ab; *] V              64 cols
@@ -284,21 +285,22 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     } else if (warp < W_PREP0) {
         // ------------------------------------------------------------ state chain
         const int stid = tid - W_STATE0 * 32;
+        const int cs = 32 * ((warp - W_STATE0) >> 2);   // this lane's 32 of the 64 columns
+        {
+            float sv[32];
 #pragma unroll
-        for (int cb = 0; cb < NVC; cb += 16) {
-            float sv[16];
-#pragma unroll
-            for (int n = 0; n < 16; ++n)
+            for (int n = 0; n < 32; ++n)
                 sv[n] = 0.f;
             if (p.S0 != nullptr) {
-                const float *src = p.S0 + (vh * KD + R) * p.dv + n0 + cb;
+                const float *src = p.S0 + (vh * KD + R) * p.dv + n0 + cs;
 #pragma unroll
-                for (int n = 0; n < 16; n += 4) {
+                for (int n = 0; n < 32; n += 4) {
                     const float4 v4 = *reinterpret_cast<const float4 *>(src + n);
                     sv[n] = v4.x; sv[n + 1] = v4.y; sv[n + 2] = v4.z; sv[n + 3] = v4.w;
                 }
             }
-            tmem_st16(tq + T_S + cb, sv);
+            tmem_st16(tq + T_S + cs, *reinterpret_cast<float(*)[16]>(&sv[0]));
+            tmem_st16(tq + T_S + cs + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
         }
         tmem_st_wait();
         bool ok = true;
@@ -319,17 +321,22 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const Gates *gt = gates_of(s);
             const float F = scalar ? gt->F[0] : gt->F[R];
             // S_{c-1} -> bf16 operand; T_S <- F S_{c-1} (the update MMA accumulates onto it)
-#pragma unroll
-            for (int cb = 0; cb < NVC; cb += 16) {
-                float sv[16];
-                tmem_ld16(tq + T_S + cb, sv);
+            {
+                float s0[16], s1[16];
+                tmem_ld16(tq + T_S + cs, s0);
+                tmem_ld16(tq + T_S + cs + 16, s1);
                 tmem_ld_wait();
-                st_tile8(S_T, KD, R, cb, &sv[0]);
-                st_tile8(S_T, KD, R, cb + 8, &sv[8]);
+                st_tile8(S_T, KD, R, cs, &s0[0]);
+                st_tile8(S_T, KD, R, cs + 8, &s0[8]);
+                st_tile8(S_T, KD, R, cs + 16, &s1[0]);
+                st_tile8(S_T, KD, R, cs + 24, &s1[8]);
 #pragma unroll
-                for (int n = 0; n < 16; ++n)
-                    sv[n] *= F;
-                tmem_st16(tq + T_S + cb, sv);
+                for (int n = 0; n < 16; ++n) {
+                    s0[n] *= F;
+                    s1[n] *= F;
+                }
+                tmem_st16(tq + T_S + cs, s0);
+                tmem_st16(tq + T_S + cs + 16, s1);
             }
             tmem_st_wait();
             fence_proxy_async_smem();
@@ -344,24 +351,31 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tc_fence_after();
             if (R < CC) {   // warps of lane quarters 0 and 1: rows t of E
                 const float f = scalar ? gt->eb[R] : 1.f;
+                float p0[16], p1[16], u0[16], u1[16];
+                tmem_ld16(tq + T_PO + 64 * ob + cs, p0);
+                tmem_ld16(tq + T_PO + 64 * ob + cs + 16, p1);
+                tmem_ld16(tq + T_U + cs, u0);
+                tmem_ld16(tq + T_U + cs + 16, u1);
+                tmem_ld_wait();
 #pragma unroll
-                for (int cb = 0; cb < NVC; cb += 16) {
-                    float pv[16], uv[16], e[16];
-                    tmem_ld16(tq + T_PO + 64 * ob + cb, pv);
-                    tmem_ld16(tq + T_U + cb, uv);
-                    tmem_ld_wait();
+                for (int n = 0; n < 16; ++n) {
+                    u0[n] -= p0[n];
+                    u1[n] -= p1[n];
+                }
+                st_tile8(E_T, CC, R, cs, &u0[0]);
+                st_tile8(E_T, CC, R, cs + 8, &u0[8]);
+                st_tile8(E_T, CC, R, cs + 16, &u1[0]);
+                st_tile8(E_T, CC, R, cs + 24, &u1[8]);
+                if (scalar) {
 #pragma unroll
-                    for (int n = 0; n < 16; ++n)
-                        e[n] = uv[n] - pv[n];
-                    st_tile8(E_T, CC, R, cb, &e[0]);
-                    st_tile8(E_T, CC, R, cb + 8, &e[8]);
-                    if (scalar) {
-#pragma unroll
-                        for (int n = 0; n < 16; ++n)
-                            e[n] *= f;
-                        st_tile8(EH_T, CC, R, cb, &e[0]);
-                        st_tile8(EH_T, CC, R, cb + 8, &e[8]);
+                    for (int n = 0; n < 16; ++n) {
+                        u0[n] *= f;
+                        u1[n] *= f;
                     }
+                    st_tile8(EH_T, CC, R, cs, &u0[0]);
+                    st_tile8(EH_T, CC, R, cs + 8, &u0[8]);
+                    st_tile8(EH_T, CC, R, cs + 16, &u1[0]);
+                    st_tile8(EH_T, CC, R, cs + 24, &u1[8]);
                 }
             }
             fence_proxy_async_smem();
@@ -375,15 +389,15 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             ok = false;
         if (ok && p.S_final != nullptr) {
             tc_fence_after();
-            float *dst = p.S_final + (vh * KD + R) * p.dv + n0;
+            float *dst = p.S_final + (vh * KD + R) * p.dv + n0 + cs;
+            float s0[16], s1[16];
+            tmem_ld16(tq + T_S + cs, s0);
+            tmem_ld16(tq + T_S + cs + 16, s1);
+            tmem_ld_wait();
 #pragma unroll
-            for (int cb = 0; cb < NVC; cb += 16) {
-                float sv[16];
-                tmem_ld16(tq + T_S + cb, sv);
-                tmem_ld_wait();
-#pragma unroll
-                for (int n = 0; n < 16; n += 4)
-                    *reinterpret_cast<float4 *>(dst + cb + n) = make_float4(sv[n], sv[n + 1], sv[n + 2], sv[n + 3]);
+            for (int n = 0; n < 16; n += 4) {
+                *reinterpret_cast<float4 *>(dst + n) = make_float4(s0[n], s0[n + 1], s0[n + 2], s0[n + 3]);
+                *reinterpret_cast<float4 *>(dst + 16 + n) = make_float4(s1[n], s1[n + 1], s1[n + 2], s1[n + 3]);
             }
         }
     } else if (warp < W_EPI0) {
