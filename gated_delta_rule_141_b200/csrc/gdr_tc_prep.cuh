@@ -41,13 +41,15 @@ constexpr int NROUND = 4;                  // pivot blocks of 16 rows
 constexpr float kGuard = 64.f;             // largest exponent a pivoted factor may take
 constexpr uint32_t IMG = CC * CC * 2;      // one bf16 C x C tile image
 constexpr uint32_t CHUNK_BYTES = 2 * IMG;  // T, then L
-// Records of the two-pass path's workspace (key width 128).
-// scalar gate: T, L, Abe = T diag(e^Lambda), e^{Lambda_t}, e^{Lambda_C - Lambda_t}, e^{Lambda_C}
-constexpr uint32_t SC_ABE = 2 * IMG, SC_EA = 3 * IMG, SC_EB = SC_EA + CC * 4, SC_F = SC_EB + CC * 4;
+// Records of the two-pass path's workspace (key width 128).  Both start with T,
+// L and W = diag(beta) A Kbar (64 x 128 bf16: two 64-column images).
+// scalar gate: then e^{Lambda_t}, e^{Lambda_C - Lambda_t}, e^{Lambda_C}
+constexpr uint32_t REC_W = 2 * IMG;
+constexpr uint32_t SC_EA = 4 * IMG, SC_EB = SC_EA + CC * 4, SC_F = SC_EB + CC * 4;
 constexpr uint32_t SC_BYTES = SC_F + 16;
-// grouped / per-channel gates: T, L, Qbar, Khat, Kbar, F
-constexpr uint32_t EXT_QB = 2 * IMG, EXT_KH = EXT_QB + 2 * IMG, EXT_KB = EXT_KH + 2 * IMG;
-constexpr uint32_t EXT_F = EXT_KB + 2 * IMG;
+// grouped / per-channel gates: then Qbar, Khat (64 x 128 bf16 each) and F (128 fp32)
+constexpr uint32_t EXT_QB = 4 * IMG, EXT_KH = EXT_QB + 2 * IMG;
+constexpr uint32_t EXT_F = EXT_KH + 2 * IMG;
 constexpr uint32_t EXT_BYTES = EXT_F + 128 * 4;
 enum RecordKind { REC_PLAIN = 0, REC_SCALAR = 1, REC_EXT = 2 };
 
@@ -56,7 +58,7 @@ __host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
 __host__ __device__ constexpr uint32_t round_col(int r) { return 8u * r * (r + 1); }
 
 struct Plan {
-    uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, lam, beta, bar, misc, total, tmem_cols, tn;
+    uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, TB, lam, beta, bar, misc, total, tmem_cols, tn;
 };
 
 __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
@@ -68,26 +70,32 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
         o += (bytes + 1023u) & ~1023u;
         return at;
     };
-    const bool extra = G > 1 || neumann;
+    // The k rows of QK outlive the inverse (W = T Kbar reads them at the end);
+    // the q rows are dead after the Grams and hold T (bf16) for that product.
     s.QK = take((dk / 64) * 128 * 128);          // rows 0-63 q, 64-127 k
-    if (extra) {
+    s.TB = s.QK;
+    if (G > 1) {
         s.RA = take((dk / 64) * 64 * 128);        // round rows: 16 of q, 16 of k
         s.KC = take((dk / 64) * 64 * 128);        // round columns
+        s.Mf = s.RA;                              // fp32 scratch, once the Grams are read
     } else {
         s.RA = s.KC = 0;
+        s.Mf = take(CC * LDM * 4 + 32 * 36 * 4);
     }
-    // fp32 scratch lives in tiles that are dead once the Grams are read
-    s.Mf = extra ? s.RA : s.QK;
     s.Tf = s.Mf + CC * LDM * 4;
-    s.NB = s.QK;                                  // Neumann operands (QK is dead by then)
-    s.XB = s.QK + 8192;
-    s.RB = s.QK + 16384;
-    s.lam = take(CC * G * 4);
-    s.beta = take(CC * 4 + NROUND * 4);
-    s.bar = take(64);
-    s.misc = s.bar + 32;
+    if (neumann) {                                // Neumann operands
+        s.NB = take(3 * 8192);
+        s.XB = s.NB + 8192;
+        s.RB = s.NB + 16384;
+    } else {
+        s.NB = s.XB = s.RB = 0;
+    }
+    s.lam = take(CC * G * 4 + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
+    s.beta = s.lam + CC * G * 4;
+    s.bar = (s.beta + CC * 4 + NROUND * 4 + 7u) & ~7u;
+    s.misc = s.bar + 16;
     s.total = o + 1024;
-    s.tmem_cols = G > 1 ? 256u : (neumann ? 128u : 64u);
+    s.tmem_cols = G > 1 ? 256u : 128u;            // W (M = 64, N = 128) needs 128 columns
     s.tn = G > 1 ? 192u : 64u;                    // Neumann products
     return s;
 }
@@ -110,15 +118,17 @@ __device__ __forceinline__ void st_img8(uint8_t *img, int r, int c, const float 
                    ptx::pack_bf16(v[4], v[5]), ptx::pack_bf16(v[6], v[7]));
 }
 
-template <int DK>
-__global__ void __launch_bounds__(NT, 3)
+// SCALAR: the scalar-gate instantiation (no pivoting machinery, four CTAs per SM);
+// otherwise grouped / per-channel gates (two CTAs per SM: the gate tile is larger).
+template <int DK, bool SCALAR>
+__global__ void __launch_bounds__(NT, SCALAR ? 4 : 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const PrepArgs a)
 {
     using namespace ptx;
     extern __shared__ uint8_t smem_raw[];
     const Params &p = a.p;
-    const int G = p.G;
+    const int G = SCALAR ? 1 : p.G;
     const bool neu = p.neumann != 0;
     const Plan Ly = plan(DK, G, neu);
     const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -204,7 +214,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // decay span of the chunk per group: within kGuard nats a single pivot at the
     // chunk end serves every pair; wider spans take the four pivoted row blocks
     bool wide = false;
-    if (G > 1)
+    if (!SCALAR)
         for (int gi = tid; gi < G; gi += NT)
             wide |= (lam[gi] - lam[(CC - 1) * G + gi]) > kGuard;
     wide = __syncthreads_or(wide ? 1 : 0) != 0;
@@ -240,7 +250,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // ---- decayed operands for the state pass, straight from the raw tiles
         for (int u = tid; u < CC * (DK / 8); u += NT) {
             const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-            float qv[8], kv[8], qb[8], kh8[8], kb[8];
+            float qv[8], kv[8], qb[8], kh8[8];
             ld_tile8(QK, 128, t, i0, qv);
             ld_tile8(QK, 128, 64 + t, i0, kv);
 #pragma unroll
@@ -249,7 +259,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float lt = lam[t * G + gi];
                 const float ea = __expf(lt), eb = __expf(lam[(CC - 1) * G + gi] - lt);
                 qb[e] = qv[e] * ea;
-                kb[e] = kv[e] * ea;
                 kh8[e] = kv[e] * eb;
             }
             const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
@@ -259,20 +268,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             *reinterpret_cast<uint4 *>(img_T + EXT_KH + off) =
                 make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
                            pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
-            *reinterpret_cast<uint4 *>(img_T + EXT_KB + off) =
-                make_uint4(pack_bf16(kb[0], kb[1]), pack_bf16(kb[2], kb[3]), pack_bf16(kb[4], kb[5]),
-                           pack_bf16(kb[6], kb[7]));
         }
     }
 
     if (!failed && !wide) {
-        if (G > 1) {
+        if (!SCALAR) {
             // ---- one pivot at the chunk end: rows carry e^{Lambda_t - Lambda_C} (at most
             //      e^{kGuard}), columns Khat = k e^{Lambda_C - Lambda_j} (at most 1); the
             //      state pass's decayed operands come out of the same sweep
             for (int u = tid; u < CC * (DK / 8); u += NT) {
                 const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float qv[8], kv[8], kh8[8], qb[8], kb[8];
+                float qv[8], kv[8], kh8[8], qb[8];
                 ld_tile8(QK, 128, t, i0, qv);
                 ld_tile8(QK, 128, 64 + t, i0, kv);
 #pragma unroll
@@ -281,7 +287,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const float lt = lam[t * G + gi], lc = lam[(CC - 1) * G + gi];
                     const float up = __expf(lt - lc), dn = __expf(lc - lt), ea = __expf(lt);
                     qb[e] = qv[e] * ea;
-                    kb[e] = kv[e] * ea;
                     kh8[e] = kv[e] * dn;
                     qv[e] *= up;
                     kv[e] *= up;
@@ -297,9 +302,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<uint4 *>(img_T + EXT_KH + off) =
                         make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
                                    pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
-                    *reinterpret_cast<uint4 *>(img_T + EXT_KB + off) =
-                        make_uint4(pack_bf16(kb[0], kb[1]), pack_bf16(kb[2], kb[3]),
-                                   pack_bf16(kb[4], kb[5]), pack_bf16(kb[6], kb[7]));
                 }
             }
             fence_proxy_async_smem();
@@ -312,7 +314,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const uint32_t id = idesc_bf16(128, CC, false, false);
             for (int k0 = 0; k0 < DK; k0 += 16)
                 mma_bf16(tmem, desc_kmajor(QK, 128, 0, k0),
-                         G == 1 ? desc_kmajor(QK, 128, 64, k0) : desc_kmajor(KC, 64, 0, k0), id, k0 > 0);
+                         SCALAR ? desc_kmajor(QK, 128, 64, k0) : desc_kmajor(KC, 64, 0, k0), id, k0 > 0);
             mma_commit(&bars[1]);
         }
         failed = wait_bar(1, ph_mma);
@@ -333,7 +335,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int j = j0 + u;
                 const float d = u < 16 ? g0[u] : g1[u - 16];
                 const bool keep = qrow ? (j <= t) : (j < t);
-                float v = keep ? (G == 1 ? d * __expf(lt - lam[j]) : d) : 0.f;
+                float v = 0.f;
+                if (keep)
+                    v = SCALAR ? d * __expf(lt - lam[j]) : d;
                 if (!qrow)
                     v *= sbeta[j];
                 out[u] = v;
@@ -597,25 +601,83 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
     }
+    const bool with_w = a.kind != REC_PLAIN;
     if (!failed) {
         __syncthreads();
-        // ---- T = diag(beta) A as a tile image: thread u writes 16-byte chunk u (coalesced)
+        if (with_w && !SCALAR) {
+            // Kbar = k e^{Lambda_t} in place in the k rows (they hold raw k after the
+            // pivoted blocks, k e^{Lambda_t - Lambda_C} after the chunk-end pivot)
+            for (int u = tid; u < CC * (DK / 8); u += NT) {
+                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                float kv[8];
+                ld_tile8(QK, 128, 64 + t, i0, kv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int gi = (i0 + e) >> wsh;
+                    kv[e] *= __expf(wide ? lam[t * G + gi] : lam[(CC - 1) * G + gi]);
+                }
+                st_tile8(QK, 128, 64 + t, i0, kv);
+            }
+        }
+        // ---- T = diag(beta) A as a tile image: thread u writes 16-byte chunk u (coalesced).
+        //      For W the same chunk goes to the bf16 operand tile in the dead q rows,
+        //      scaled by e^{Lambda_j} for the scalar gate (W = T diag(e^Lambda) K).
+        const uint32_t TB = base_u32 + Ly.TB;
         for (int u = tid; u < CC * 8; u += NT) {
             const int r = u >> 3, cc = (u & 7) ^ (r & 7);
             const float bt = sbeta[r];
             const float4 x0 = *reinterpret_cast<const float4 *>(&Mf[r * LDM + 8 * cc]);
             const float4 x1 = *reinterpret_cast<const float4 *>(&Mf[r * LDM + 8 * cc + 4]);
-            *reinterpret_cast<uint4 *>(img_T + 16 * u) =
+            const uint4 tv =
                 make_uint4(pack_bf16(bt * x0.x, bt * x0.y), pack_bf16(bt * x0.z, bt * x0.w),
                            pack_bf16(bt * x1.x, bt * x1.y), pack_bf16(bt * x1.z, bt * x1.w));
-            if (a.kind == REC_SCALAR) {   // Abe = T diag(e^{Lambda_j}), e^{Lambda_j} <= 1
-                float e[8];
+            *reinterpret_cast<uint4 *>(img_T + 16 * u) = tv;
+            if (with_w) {
+                if (SCALAR) {
+                    float e[8];
 #pragma unroll
-                for (int f = 0; f < 8; ++f)
-                    e[f] = bt * __expf(lam[8 * cc + f]);
-                *reinterpret_cast<uint4 *>(img_T + SC_ABE + 16 * u) =
-                    make_uint4(pack_bf16(e[0] * x0.x, e[1] * x0.y), pack_bf16(e[2] * x0.z, e[3] * x0.w),
-                               pack_bf16(e[4] * x1.x, e[5] * x1.y), pack_bf16(e[6] * x1.z, e[7] * x1.w));
+                    for (int f = 0; f < 8; ++f)
+                        e[f] = bt * __expf(lam[8 * cc + f]);
+                    st_shared_v4(TB + 16 * u, pack_bf16(e[0] * x0.x, e[1] * x0.y),
+                                 pack_bf16(e[2] * x0.z, e[3] * x0.w), pack_bf16(e[4] * x1.x, e[5] * x1.y),
+                                 pack_bf16(e[6] * x1.z, e[7] * x1.w));
+                } else {
+                    st_shared_v4(TB + 16 * u, tv.x, tv.y, tv.z, tv.w);
+                }
+            }
+        }
+        if (with_w) {
+            // ---- W = TB Kbar (M = 64, N = 128, K = 64) on tcgen05, read back as an image
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(64, 128, false, true);
+                for (int k0 = 0; k0 < CC; k0 += 16)
+                    mma_bf16(tmem, desc_kmajor(TB, 64, 0, k0), desc_mnmajor(QK, 128, 64 + k0, 0), id,
+                             k0 > 0);
+                mma_commit(&bars[1]);
+            }
+            failed = wait_bar(1, ph_mma);
+            ph_mma ^= 1u;
+            if (!failed) {
+                tc_fence_after();
+                const int rr = gen::row64g(warp, lane);
+                const int cw = 64 * (warp >> 2);
+#pragma unroll
+                for (int cb = 0; cb < 64; cb += 32) {
+                    float w0[16], w1[16];
+                    tmem_ld16(tq + cw + cb, w0);
+                    tmem_ld16(tq + cw + cb + 16, w1);
+                    tmem_ld_wait();
+                    if (rr >= 0) {
+                        uint8_t *img_W = img_T + REC_W + (cw >> 6) * IMG;
+                        st_img8(img_W, rr, cb, &w0[0]);
+                        st_img8(img_W, rr, cb + 8, &w0[8]);
+                        st_img8(img_W, rr, cb + 16, &w1[0]);
+                        st_img8(img_W, rr, cb + 24, &w1[8]);
+                    }
+                }
             }
         }
     }
@@ -669,7 +731,7 @@ int launch(const Params &p, void *out, int kind, cudaStream_t stream)
     if (!make_map(&mq, p.q, DK, p.T, sk, CC) || !make_map(&mk, p.k, DK, p.T, sk, CC))
         return 6;
     const Plan Ly = plan(DK, p.G, p.neumann != 0);
-    auto kern = prep_kernel<DK>;
+    auto kern = p.G == 1 ? prep_kernel<DK, true> : prep_kernel<DK, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
         cudaSuccess)
         return 6;

@@ -1,54 +1,54 @@
 // gdr_tc_split.cuh -- second pass of the two-pass tensor-core path: the
 // inter-chunk state recurrence and the readout, for key width dk = 128, chunk
 // C = 64, 64 value columns per CTA, any decay grouping.  The chunk-local
-// factors T = diag(beta) (I + M)^{-1} and L come from the first pass
-// (gdr_tc_prep.cuh), so the serial chain per chunk holds only the state
+// factors T = diag(beta) (I + M)^{-1}, L and W = T Kbar come from the first
+// pass (gdr_tc_prep.cuh), so the serial chain per chunk holds only the state
 // products ("Systolic Linear Attention: Co-Designing Tile-Grouped Gated Delta
 // Attention for TPUs", §2.1, §2.3 Table 2, §2.4.2):
-//   W = T Kbar,  U = T V                     (off the chain, one chunk ahead)
+//   U = T V                                  (off the chain, one chunk ahead)
 //   P = W S,  E = U - P                      (chain)
 //   S <- F S + Khat^T E,  O = Qbar S + L E   (chain; O leaves off the chain)
 // with Kbar = k e^{Lambda_t}, Khat = k e^{Lambda_C - Lambda_t},
-// Qbar = q e^{Lambda_t}, F = diag(e^{Lambda_C}) -- all factors <= 1.
-// For the scalar gate the factors are row / column scalings:
-// W = (T diag(e^Lambda)) K, Khat^T E = K^T (diag(e^{Lambda_C - Lambda}) E) and
-// Qbar S = diag(e^Lambda) (Q S), applied by the epilogue.
+// Qbar = q e^{Lambda_t}, F = diag(e^{Lambda_C}) -- all factors <= 1.  For the
+// scalar gate Khat^T E = K^T (diag(e^{Lambda_C - Lambda}) E) and
+// Qbar S = diag(e^Lambda) (Q S) (the epilogue applies it), so q and k are used
+// as loaded; for grouped / per-channel gates Qbar and Khat come decayed from
+// the first pass.  Nothing here evaluates an exponential.
 //
-// Roles (warp-specialised, hand-offs through mbarriers):
-//   warp 0      producer: TMA q, k, v; bulk copies of T and L; 2-stage ring
-//   warp 1      MMA issuer (one thread)
-//   warps 2-9   state chain: S (fp32, TMEM) -> bf16 operand, E = U - P; two
+// Roles (warp-specialised, hand-offs through mbarriers; every wait bounded):
+//   warps 0-1   epilogue: O = f (Q S) + L E from TMEM to global memory
+//   warp 2      producer: TMA / bulk copies into a 2-stage ring
+//   warp 3      MMA issuer (one thread)
+//   warps 4-11  state chain: S (fp32, TMEM) -> bf16 operand, E = U - P; two
 //               warps per TMEM lane quarter, each lane on 32 of the 64 columns
-//   warps 10-13 W read-back: TMEM fp32 -> bf16 operand tile (one chunk ahead)
-//   warps 14-15 epilogue: O = f (Q S) + L E from TMEM to global memory
-// Everything decayed (Abe, Qbar, Khat, Kbar, the per-token factors, F) comes
-// from the first pass's record, so no role here evaluates an exponential.
-// Stage s holds [W | Q | K] (rows 0-63 | 64-127 | 128-191, 128 columns),
-// [V | L] (rows 0-63 | 64-127, 64 columns) and [Ab | Abe] (T, and for the
-// scalar gate T diag(e^Lambda)).  MMA operands are stacked so that M = 128:
-//   [Ab; Abe] V -> U (rows 0-63),  [Ab; Abe] K -> W (rows 64-127, scalar gate)
-//   or [Ab; *] Kbar -> W (rows 0-63),  [W; Q] S -> P, Q S (Q = Qbar for
-//   grouped / per-channel gates), Khat^T E onto S,  [V; L] E -> L E (rows 64-127).
+// A stage is loaded in two groups with their own barriers, so that it can be
+// refilled as soon as each group's last reader is done:
+//   X = {W, Q, T, V, factors}: read by U, P and the state warps -> free once E
+//       of the chunk is formed;
+//   Y = {K, L}: read by the update and the readout -> free after them.
+// MMA operands are stacked so that M = 128 and no product reads a tile that a
+// load may be refilling:
+//   [0; T] V -> U (rows 64-127),  [Q; W] S -> Q S (rows 0-63), P (rows 64-127),
+//   Khat^T E onto F S,  [L; 0] E -> L E (rows 0-63).
 
 namespace split {
 
-constexpr int NWARP = 16;
-constexpr int NTHR = NWARP * 32;   // 512
+constexpr int NWARP = 12;
+constexpr int NTHR = NWARP * 32;   // 384
 constexpr int CC = 64;
 constexpr int KD = 128;
 constexpr int NVC = 64;
-constexpr int W_PROD = 0, W_MMA = 1, W_STATE0 = 2, W_PREP0 = 10, W_EPI0 = 14;
-constexpr int N_STATE = 256, N_PREP = 128, N_EPI = 64;
-constexpr int NB_STATE = 1, NB_PREP = 2, NB_EPI = 3;   // named barriers
+constexpr int W_EPI0 = 0, W_PROD = 2, W_MMA = 3, W_STATE0 = 4;
+constexpr int N_STATE = 256, N_EPI = 64;
+constexpr int NB_STATE = 1, NB_EPI = 2;   // named barriers
 
-constexpr uint32_t T_U = 0;        // [Ab; *] V              64 cols
-constexpr uint32_t T_W = 64;       // [Ab; Abe] K / [Ab; *] Kbar   128 cols
-constexpr uint32_t T_PO = 192;     // two buffers of 64 cols: [W; Q] S
-constexpr uint32_t T_S = 320;      // fp32 state, 64 cols
-constexpr uint32_t T_LE = 384;     // two buffers of 64 cols: [V; L] E
+constexpr uint32_t T_U = 0;        // two buffers of 64 cols: [0; T] V (rows 64-127)
+constexpr uint32_t T_PO = 128;     // two buffers of 64 cols: [Q; W] S
+constexpr uint32_t T_S = 256;      // fp32 state, 64 cols
+constexpr uint32_t T_LE = 320;     // two buffers of 64 cols: [L; 0] E (rows 0-63)
 constexpr uint32_t TMEM_COLS = 512;
 
-enum Bar { FULL0, FULL1, FREE0, FREE1, WU_FULL, W_READY, S_READY, P_FULL, E_READY,
+enum Bar { FULLX0, FULLX1, FULLY0, FULLY1, FREEX0, FREEX1, FREEY0, FREEY1, S_READY, P_FULL, E_READY,
            UPD_DONE, OUT0, OUT1, OFREE0, OFREE1, DRAIN, NBARS };
 
 struct Gates {                        // landed by bulk copies from the first pass's record
@@ -57,11 +57,12 @@ struct Gates {                        // landed by bulk copies from the first pa
 };
 
 struct Plan {
-    uint32_t wqk[2], vl[2], ab[2], gates[2], kb[2];
+    uint32_t qwk[2], lz[2], v[2], ab[2], gates[2];
     uint32_t S, E, Eh, bar, misc, total;
 };
 
-// Scalar gate: an E_hat tile; grouped / per-channel gates: a Kbar tile per stage.
+// Stage: [Q | W | K] (rows 0-63 | 64-127 | 128-191, 128 columns), [L | 0]
+// (64 + 64 rows), V (64 rows) and [0 | T] (64 + 64 rows), 64 columns each.
 __host__ __device__ inline Plan plan(bool scalar)
 {
     Plan s;
@@ -72,11 +73,11 @@ __host__ __device__ inline Plan plan(bool scalar)
         return at;
     };
     for (int i = 0; i < 2; ++i) {
-        s.wqk[i] = take((KD / 64) * 192 * 128);
-        s.vl[i] = take(128 * 128);
+        s.qwk[i] = take((KD / 64) * 192 * 128);
+        s.lz[i] = take(128 * 128);
+        s.v[i] = take(64 * 128);
         s.ab[i] = take(128 * 128);
         s.gates[i] = take(sizeof(Gates));
-        s.kb[i] = scalar ? 0 : take((KD / 64) * CC * 128);
     }
     s.S = take(KD * NVC * 2);
     s.E = take(CC * NVC * 2);
@@ -90,10 +91,34 @@ __host__ __device__ inline Plan plan(bool scalar)
 struct SplitArgs {
     Params p;
     const uint8_t *factors;   // first-pass output, [B * Hk * nchunks][rec_bytes]
-    uint32_t rec_bytes;       // prep::CHUNK_BYTES (scalar gate) or prep::EXT_BYTES
+    uint32_t rec_bytes;       // prep::SC_BYTES (scalar gate) or prep::EXT_BYTES
     int nvt;
     int nchunks;
 };
+
+// Bounded wait without sleeping between probes: every hand-off in this kernel
+// is on or next to the per-chunk critical chain, where a back-off sleep would
+// add its length to the chunk period.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag)
+{
+    if (ptx::mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (ptx::mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 255) == 0) {
+            if (*abort_flag)
+                return false;
+            if (ptx::globaltimer_ns() - t0 > 2000000000ull) {
+                *abort_flag = 1;
+                atomicExch(&g_device_status, kTimeoutStatus);
+                return false;
+            }
+        }
+    }
+}
 
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(NTHR, 1)
@@ -101,7 +126,6 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
              const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
 {
     using namespace ptx;
-    using ws::wait_or_abort;
     using ws::named_sync;
     using ws::named_vote_or;
     extern __shared__ uint8_t smem_raw[];
@@ -126,9 +150,6 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 4);
     auto gates_of = [&](int s) { return reinterpret_cast<Gates *>(base + Ly.gates[s]); };
-    auto wqk_of = [&](int s) { return base_u32 + Ly.wqk[s]; };
-    auto vl_of = [&](int s) { return base_u32 + Ly.vl[s]; };
-    auto ab_of = [&](int s) { return base_u32 + Ly.ab[s]; };
     const uint32_t S_T = base_u32 + Ly.S, E_T = base_u32 + Ly.E, EH_T = base_u32 + Ly.Eh;
 
     if (tid == 0) {
@@ -144,6 +165,14 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
+    // the zero halves of [L; 0] and [0; T] (never loaded)
+    for (int i = tid; i < 2 * 64 * 8; i += NTHR) {
+        const int st = i >> 9, r = (i >> 3) & 63, c = (i & 7) * 8;
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        st_tile8(base_u32 + Ly.lz[st], 128, 64 + r, c, z);
+        st_tile8(base_u32 + Ly.ab[st], 128, r, c, z);
+    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -153,76 +182,84 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     if (warp == W_PROD) {
         // ------------------------------------------------------------ producer
-        uint32_t pend = 0, par0 = 0, par1 = 0;
+        int armx[2] = {0, 0}, army[2] = {0, 0};   // loads armed per stage and group
         for (int c = 0; c < N; ++c) {
             const int s = c & 1;
+            const long c0 = (long)c * CC;
+            const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
+            uint8_t *qwk = base + Ly.qwk[s];
+            // group X: W, Q (or Qbar), T, V, the decay factors
             if (c >= 2) {
-                const bool ok = wait_or_abort(&bars[FREE0 + s], ((c >> 1) - 1) & 1, abort_flag);
+                const bool ok = wait_or_abort(&bars[FREEX0 + s], ((c >> 1) - 1) & 1, abort_flag);
                 if (__any_sync(0xffffffffu, !ok))
                     break;
             }
-            const long c0 = (long)c * CC;
             if (lane == 0) {
-                const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
-                uint64_t *full = &bars[FULL0 + s];
-                if (scalar) {
-                    // q, k as loaded; Abe and the per-token factors from the first pass
-                    constexpr uint32_t fac_bytes = prep::SC_BYTES - prep::SC_EA;
-                    mbar_arrive_expect_tx(full, 2u * CC * KD * 2 + CC * NVC * 2 + 3 * prep::IMG + fac_bytes);
-                    for (int kb = 0; kb < KD / 64; ++kb) {
-                        uint8_t *blk = base + Ly.wqk[s] + kb * 192 * 128;
-                        tma_load_3d(blk + 64 * 128, &tm_q, full, 64 * kb, (int)c0, (int)kh);
-                        tma_load_3d(blk + 128 * 128, &tm_k, full, 64 * kb, (int)c0, (int)kh);
-                    }
-                    bulk_load(base + Ly.ab[s] + 64 * 128, fac + prep::SC_ABE, prep::IMG, full);
-                    bulk_load(gates_of(s)->ea, fac + prep::SC_EA, fac_bytes, full);
-                } else {
-                    // Qbar, Khat (per 64-column block), Kbar and F, decayed by the first pass
-                    mbar_arrive_expect_tx(full, 8u * prep::IMG + KD * 4 + CC * NVC * 2);
-                    for (int kb = 0; kb < KD / 64; ++kb) {
-                        uint8_t *blk = base + Ly.wqk[s] + kb * 192 * 128;
-                        bulk_load(blk + 64 * 128, fac + prep::EXT_QB + kb * prep::IMG, prep::IMG, full);
-                        bulk_load(blk + 128 * 128, fac + prep::EXT_KH + kb * prep::IMG, prep::IMG, full);
-                    }
-                    bulk_load(base + Ly.kb[s], fac + prep::EXT_KB, 2 * prep::IMG, full);
-                    bulk_load(gates_of(s)->F, fac + prep::EXT_F, KD * 4, full);
+                uint64_t *full = &bars[FULLX0 + s];
+                const uint32_t fac_bytes = scalar ? prep::SC_BYTES - prep::SC_EA : KD * 4;
+                // W, Q: two 64-column images each; T: one; V: 64 x 64 bf16
+                mbar_arrive_expect_tx(full, 5u * prep::IMG + CC * NVC * 2 + fac_bytes);
+                for (int kb = 0; kb < KD / 64; ++kb) {
+                    uint8_t *blk = qwk + kb * 192 * 128;
+                    bulk_load(blk + 64 * 128, fac + prep::REC_W + kb * prep::IMG, prep::IMG, full);
+                    if (scalar)
+                        tma_load_3d(blk, &tm_q, full, 64 * kb, (int)c0, (int)kh);
+                    else
+                        bulk_load(blk, fac + prep::EXT_QB + kb * prep::IMG, prep::IMG, full);
                 }
-                tma_load_3d(base + Ly.vl[s], &tm_v, full, n0, (int)c0, (int)vh);
-                bulk_load(base + Ly.ab[s], fac, prep::IMG, full);
-                bulk_load(base + Ly.vl[s] + 64 * 128, fac + prep::IMG, prep::IMG, full);
+                bulk_load(base + Ly.ab[s] + 64 * 128, fac, prep::IMG, full);
+                tma_load_3d(base + Ly.v[s], &tm_v, full, n0, (int)c0, (int)vh);
+                if (scalar)
+                    bulk_load(gates_of(s)->ea, fac + prep::SC_EA, fac_bytes, full);
+                else
+                    bulk_load(gates_of(s)->F, fac + prep::EXT_F, fac_bytes, full);
             }
-            pend |= 1u << s;
-            if (s)
-                par1 = (c >> 1) & 1;
-            else
-                par0 = (c >> 1) & 1;
+            armx[s] += 1;
+            // group Y: K (or Khat), L
+            if (c >= 2) {
+                const bool ok = wait_or_abort(&bars[FREEY0 + s], ((c >> 1) - 1) & 1, abort_flag);
+                if (__any_sync(0xffffffffu, !ok))
+                    break;
+            }
+            if (lane == 0) {
+                uint64_t *full = &bars[FULLY0 + s];
+                mbar_arrive_expect_tx(full, 3u * prep::IMG);
+                for (int kb = 0; kb < KD / 64; ++kb) {
+                    uint8_t *blk = qwk + kb * 192 * 128 + 128 * 128;
+                    if (scalar)
+                        tma_load_3d(blk, &tm_k, full, 64 * kb, (int)c0, (int)kh);
+                    else
+                        bulk_load(blk, fac + prep::EXT_KH + kb * prep::IMG, prep::IMG, full);
+                }
+                bulk_load(base + Ly.lz[s], fac + prep::IMG, prep::IMG, full);
+            }
+            army[s] += 1;
         }
-        if (lane == 0) {   // drain loads that may still be landing (bounded)
-            if (pend & 1u)
-                mbar_wait(&bars[FULL0], par0, 200000000ull);
-            if (pend & 2u)
-                mbar_wait(&bars[FULL1], par1, 200000000ull);
+        // drain loads that may still be landing (bounded): the last armed phase of
+        // each barrier, whether or not a consumer saw it
+        if (lane == 0) {
+            for (int s = 0; s < 2; ++s) {
+                if (armx[s] > 0)
+                    mbar_wait(&bars[FULLX0 + s], (armx[s] - 1) & 1, 200000000ull);
+                if (army[s] > 0)
+                    mbar_wait(&bars[FULLY0 + s], (army[s] - 1) & 1, 200000000ull);
+            }
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_u = idesc_bf16(128, NVC, false, true);
-            const uint32_t id_w = idesc_bf16(128, KD, false, true);
             const uint32_t id_po = idesc_bf16(128, NVC, false, true);
             const uint32_t id_s = idesc_bf16(KD, NVC, true, true);
-            // descriptors at k = 0; a K step adds its byte offset / 16 to the start field
-            // (K-major: 32 bytes per 16 columns inside a 64-column block, rows * 128 per
-            // block; MN-major: 16 rows of 128 bytes per 16-deep step)
-            // (stage 1 sits a fixed byte distance after stage 0: one more add)
-            const uint64_t d_ab0 = desc_kmajor(ab_of(0), 128, 0, 0);
-            const uint64_t d_v0 = desc_mnmajor(vl_of(0), 128, 0, 0);
-            const uint64_t d_wq0 = desc_kmajor(wqk_of(0), 192, 0, 0);
-            const uint64_t d_kt0 = desc_mnmajor(wqk_of(0), 192, 128, 0);
-            const uint64_t d_vl0 = desc_kmajor(vl_of(0), 128, 0, 0);
-            const uint64_t d_kb0 = scalar ? 0 : desc_mnmajor(base_u32 + Ly.kb[0], CC, 0, 0);
-            const uint64_t dkb = (Ly.kb[1] - Ly.kb[0]) >> 4;
-            const uint64_t dab = (Ly.ab[1] - Ly.ab[0]) >> 4, dvl = (Ly.vl[1] - Ly.vl[0]) >> 4;
-            const uint64_t dwq = (Ly.wqk[1] - Ly.wqk[0]) >> 4;
+            // descriptors at k = 0 of stage 0; a K step adds its byte offset / 16 to the
+            // start field, stage 1 a fixed distance
+            const uint64_t d_ab0 = desc_kmajor(base_u32 + Ly.ab[0], 128, 0, 0);
+            const uint64_t d_v0 = desc_mnmajor(base_u32 + Ly.v[0], 64, 0, 0);
+            const uint64_t d_qw0 = desc_kmajor(base_u32 + Ly.qwk[0], 192, 0, 0);
+            const uint64_t d_kt0 = desc_mnmajor(base_u32 + Ly.qwk[0], 192, 128, 0);
+            const uint64_t d_lz0 = desc_kmajor(base_u32 + Ly.lz[0], 128, 0, 0);
+            const uint64_t dab = (Ly.ab[1] - Ly.ab[0]) >> 4, dv = (Ly.v[1] - Ly.v[0]) >> 4;
+            const uint64_t dqw = (Ly.qwk[1] - Ly.qwk[0]) >> 4, dlz = (Ly.lz[1] - Ly.lz[0]) >> 4;
             const uint64_t d_s = desc_mnmajor(S_T, KD, 0, 0);
             const uint64_t d_e = desc_mnmajor(scalar ? EH_T : E_T, CC, 0, 0);
             const uint64_t d_eo = desc_mnmajor(E_T, CC, 0, 0);
@@ -230,82 +267,83 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 return static_cast<uint64_t>(((k0 >> 6) * rows * 128 + (k0 & 63) * 2) >> 4);
             };
             auto mstep = [](int k0) { return static_cast<uint64_t>(k0 * 8); };
-            auto wu = [&](int st) {
-                const uint64_t a0 = d_ab0 + st * dab, v0 = d_v0 + st * dvl;
-                const uint64_t k0d = scalar ? d_kt0 + st * dwq : d_kb0 + st * dkb;
-                for (int k0 = 0; k0 < CC; k0 += 16) {
-                    mma_bf16(tmem + T_U, a0 + kstep(k0, 128), v0 + mstep(k0), id_u, k0 > 0);
-                    mma_bf16(tmem + T_W, a0 + kstep(k0, 128), k0d + mstep(k0), id_w, k0 > 0);
-                }
-                mma_commit(&bars[WU_FULL]);
+            auto issue_u = [&](int st) {   // U of the chunk in stage st -> T_U buffer st
+                const uint64_t a0 = d_ab0 + st * dab, v0 = d_v0 + st * dv;
+                for (int k0 = 0; k0 < CC; k0 += 16)
+                    mma_bf16(tmem + T_U + 64 * st, a0 + kstep(k0, 128), v0 + mstep(k0), id_u, k0 > 0);
             };
-            bool ok = true;
-            if (N > 0) {
-                ok = wait_or_abort(&bars[FULL0], 0, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    wu(0);
-                }
-            }
+            bool ok = true, u_ready = false;
             for (int c = 0; c < N && ok; ++c) {
-                const int s = c & 1, ob = c & 1;
+                const int s = c & 1;
                 const uint32_t par = c & 1;
-                if (!(ok = wait_or_abort(&bars[W_READY], par, abort_flag)))
+                if (!(ok = wait_or_abort(&bars[FULLX0 + s], (c >> 1) & 1, abort_flag)))
                     break;
+                if (!u_ready) {
+                    tc_fence_after();
+                    issue_u(s);
+                }
                 if (!(ok = wait_or_abort(&bars[S_READY], par, abort_flag)))
                     break;
-                if (c >= 2 && !(ok = wait_or_abort(&bars[OFREE0 + ob], ((c >> 1) - 1) & 1, abort_flag)))
+                if (c >= 2 && !(ok = wait_or_abort(&bars[OFREE0 + s], ((c >> 1) - 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
-                const uint64_t wq = d_wq0 + s * dwq, kt = d_kt0 + s * dwq, vl = d_vl0 + s * dvl;
+                const uint64_t qw = d_qw0 + s * dqw, kt = d_kt0 + s * dqw, lz = d_lz0 + s * dlz;
                 for (int k0 = 0; k0 < KD; k0 += 16)
-                    mma_bf16(tmem + T_PO + 64 * ob, wq + kstep(k0, 192), d_s + mstep(k0), id_po, k0 > 0);
+                    mma_bf16(tmem + T_PO + 64 * s, qw + kstep(k0, 192), d_s + mstep(k0), id_po, k0 > 0);
                 mma_commit(&bars[P_FULL]);
+                // the next chunk's U overlaps this chunk's E step when its tiles are in
+                u_ready = false;
+                if (c + 1 < N && mbar_test(&bars[FULLX0 + (s ^ 1)], ((c + 1) >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_u(s ^ 1);
+                    u_ready = true;
+                }
                 if (!(ok = wait_or_abort(&bars[E_READY], par, abort_flag)))
+                    break;
+                // group X of this stage has no reader left: P and U finished before
+                // the state warps formed E (they waited for P_FULL)
+                mbar_arrive(&bars[FREEX0 + s]);
+                if (!(ok = wait_or_abort(&bars[FULLY0 + s], (c >> 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(tmem + T_S, kt + mstep(k0), d_e + mstep(k0), id_s, 1u);
                 mma_commit(&bars[UPD_DONE]);
                 for (int k0 = 0; k0 < CC; k0 += 16)
-                    mma_bf16(tmem + T_LE + 64 * ob, vl + kstep(k0, 128), d_eo + mstep(k0), id_po, k0 > 0);
-                mma_commit(&bars[OUT0 + ob]);
-                mma_commit(&bars[FREE0 + s]);
-                if (c + 1 < N) {
-                    if (!(ok = wait_or_abort(&bars[FULL0 + (s ^ 1)], ((c + 1) >> 1) & 1, abort_flag)))
-                        break;
-                    tc_fence_after();
-                    wu(s ^ 1);
-                }
+                    mma_bf16(tmem + T_LE + 64 * s, lz + kstep(k0, 128), d_eo + mstep(k0), id_po, k0 > 0);
+                mma_commit(&bars[OUT0 + s]);
+                mma_commit(&bars[FREEY0 + s]);
             }
             // whatever was issued must finish before tensor memory is released
             mma_commit(&bars[DRAIN]);
             mbar_wait(&bars[DRAIN], 0, 200000000ull);
         }
-    } else if (warp < W_PREP0) {
+    } else if (warp >= W_STATE0) {
         // ------------------------------------------------------------ state chain
         const int stid = tid - W_STATE0 * 32;
         const int cs = 32 * ((warp - W_STATE0) >> 2);   // this lane's 32 of the 64 columns
         {
-            float sv[32];
+            float s0[16], s1[16];
 #pragma unroll
-            for (int n = 0; n < 32; ++n)
-                sv[n] = 0.f;
+            for (int n = 0; n < 16; ++n)
+                s0[n] = s1[n] = 0.f;
             if (p.S0 != nullptr) {
                 const float *src = p.S0 + (vh * KD + R) * p.dv + n0 + cs;
 #pragma unroll
-                for (int n = 0; n < 32; n += 4) {
-                    const float4 v4 = *reinterpret_cast<const float4 *>(src + n);
-                    sv[n] = v4.x; sv[n + 1] = v4.y; sv[n + 2] = v4.z; sv[n + 3] = v4.w;
+                for (int n = 0; n < 16; n += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(src + n);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(src + 16 + n);
+                    s0[n] = a4.x; s0[n + 1] = a4.y; s0[n + 2] = a4.z; s0[n + 3] = a4.w;
+                    s1[n] = b4.x; s1[n + 1] = b4.y; s1[n + 2] = b4.z; s1[n + 3] = b4.w;
                 }
             }
-            tmem_st16(tq + T_S + cs, *reinterpret_cast<float(*)[16]>(&sv[0]));
-            tmem_st16(tq + T_S + cs + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
+            tmem_st16(tq + T_S + cs, s0);
+            tmem_st16(tq + T_S + cs + 16, s1);
         }
         tmem_st_wait();
         bool ok = true;
         for (int c = 0; c < N; ++c) {
-            const int s = c & 1, ob = c & 1;
+            const int s = c & 1;
             const uint32_t par = c & 1;
             if (c >= 1 &&
                 named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[UPD_DONE], (c - 1) & 1, abort_flag))) {
@@ -313,7 +351,7 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 break;
             }
             if (named_vote_or(NB_STATE, N_STATE,
-                              !wait_or_abort(&bars[FULL0 + s], (c >> 1) & 1, abort_flag))) {
+                              !wait_or_abort(&bars[FULLX0 + s], (c >> 1) & 1, abort_flag))) {
                 ok = false;
                 break;
             }
@@ -349,33 +387,34 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 break;
             }
             tc_fence_after();
-            if (R < CC) {   // warps of lane quarters 0 and 1: rows t of E
-                const float f = scalar ? gt->eb[R] : 1.f;
+            if (R >= CC) {   // warps of lane quarters 2 and 3: rows t of P, U and E
+                const int t = R - CC;
+                const float f = scalar ? gt->eb[t] : 1.f;
                 float p0[16], p1[16], u0[16], u1[16];
-                tmem_ld16(tq + T_PO + 64 * ob + cs, p0);
-                tmem_ld16(tq + T_PO + 64 * ob + cs + 16, p1);
-                tmem_ld16(tq + T_U + cs, u0);
-                tmem_ld16(tq + T_U + cs + 16, u1);
+                tmem_ld16(tq + T_PO + 64 * s + cs, p0);
+                tmem_ld16(tq + T_PO + 64 * s + cs + 16, p1);
+                tmem_ld16(tq + T_U + 64 * s + cs, u0);
+                tmem_ld16(tq + T_U + 64 * s + cs + 16, u1);
                 tmem_ld_wait();
 #pragma unroll
                 for (int n = 0; n < 16; ++n) {
                     u0[n] -= p0[n];
                     u1[n] -= p1[n];
                 }
-                st_tile8(E_T, CC, R, cs, &u0[0]);
-                st_tile8(E_T, CC, R, cs + 8, &u0[8]);
-                st_tile8(E_T, CC, R, cs + 16, &u1[0]);
-                st_tile8(E_T, CC, R, cs + 24, &u1[8]);
+                st_tile8(E_T, CC, t, cs, &u0[0]);
+                st_tile8(E_T, CC, t, cs + 8, &u0[8]);
+                st_tile8(E_T, CC, t, cs + 16, &u1[0]);
+                st_tile8(E_T, CC, t, cs + 24, &u1[8]);
                 if (scalar) {
 #pragma unroll
                     for (int n = 0; n < 16; ++n) {
                         u0[n] *= f;
                         u1[n] *= f;
                     }
-                    st_tile8(EH_T, CC, R, cs, &u0[0]);
-                    st_tile8(EH_T, CC, R, cs + 8, &u0[8]);
-                    st_tile8(EH_T, CC, R, cs + 16, &u1[0]);
-                    st_tile8(EH_T, CC, R, cs + 24, &u1[8]);
+                    st_tile8(EH_T, CC, t, cs, &u0[0]);
+                    st_tile8(EH_T, CC, t, cs + 8, &u0[8]);
+                    st_tile8(EH_T, CC, t, cs + 16, &u1[0]);
+                    st_tile8(EH_T, CC, t, cs + 24, &u1[8]);
                 }
             }
             fence_proxy_async_smem();
@@ -400,37 +439,10 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 *reinterpret_cast<float4 *>(dst + 16 + n) = make_float4(s1[n], s1[n + 1], s1[n + 2], s1[n + 3]);
             }
         }
-    } else if (warp < W_EPI0) {
-        // ------------------------------------------------------------ W read-back
-        const int ptid = tid - W_PREP0 * 32;
-        for (int c = 0; c < N; ++c) {
-            const uint32_t wqk = wqk_of(c & 1);
-            // W read-back: rows 64-127 of T_W (scalar gate) or rows 0-63
-            if (named_vote_or(NB_PREP, N_PREP, !wait_or_abort(&bars[WU_FULL], c & 1, abort_flag)))
-                break;
-            tc_fence_after();
-            const bool mine = scalar ? (R >= CC) : (R < CC);
-            if (mine) {
-                const int t = scalar ? R - CC : R;
-#pragma unroll
-                for (int cb = 0; cb < KD; cb += 16) {
-                    float wv[16];
-                    tmem_ld16(tq + T_W + cb, wv);
-                    tmem_ld_wait();
-                    st_tile8(wqk, 192, t, cb, &wv[0]);
-                    st_tile8(wqk, 192, t, cb + 8, &wv[8]);
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_sync(NB_PREP, N_PREP);
-            if (ptid == 0)
-                mbar_arrive(&bars[W_READY]);
-        }
     } else {
-        // ------------------------------------------------------------ epilogue (O rows in lanes 64-127)
+        // ------------------------------------------------------------ epilogue (rows t in lanes 0-63)
         const int etid = tid - W_EPI0 * 32;
-        const int t = R - CC;
+        const int t = R;
         for (int c = 0; c < N; ++c) {
             const int ob = c & 1;
             const long c0 = (long)c * CC;

@@ -34,7 +34,7 @@ KERNEL_NAMES = {KERNEL_SIMT: "simt", KERNEL_TC: "tc", KERNEL_TC2: "tc2"}
 # bytes of one chunk record written by gdr_chunk_prepare (T then L, 64 x 64 bf16 each)
 PREP_CHUNK_BYTES = 16384
 # bytes of one workspace record of the two-pass kernel: scalar gate, grouped / per-channel gates
-TC2_SCALAR_RECORD_BYTES = 25104
+TC2_SCALAR_RECORD_BYTES = 33296
 TC2_EXT_RECORD_BYTES = 66048
 _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN}
 

@@ -130,7 +130,7 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape,
 
 /* Device workspace (bytes) that gdr_chunk_fwd needs for this request with the
  * kernel AUTO or shape->kernel selects when given enough: 0 for the one-pass
- * kernels; for TC2, B * Hk * ceil(T / 64) records of 25104 bytes (scalar gate)
+ * kernels; for TC2, B * Hk * ceil(T / 64) records of 33296 bytes (scalar gate)
  * or 66048 bytes (grouped / per-channel gates): the chunk factors T and L plus
  * the decayed operands and decay factors the second pass reads.  The caller allocates it
  * (16-byte aligned) and passes it with its size; its contents on entry do not
