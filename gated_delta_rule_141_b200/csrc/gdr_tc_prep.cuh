@@ -12,7 +12,9 @@
 //   3. Decayed Grams on tcgen05, never dividing by a decay prefix:
 //        scalar gate: [Q; K] K^T once, then the factor e^{Lambda_t - Lambda_j}
 //          (t >= j, so <= 1) on the way out of TMEM;
-//        grouped / per-channel gate: four row blocks of 16 tokens, each with
+//        grouped / per-channel gate: when the chunk's decay span is within kGuard
+//          nats, one pivot at the chunk end (rows scaled by e^{Lambda_t - Lambda_C},
+//          columns by e^{Lambda_C - Lambda_j}); otherwise two row blocks of 32 tokens, each with
 //          its own pivot p in the middle of the block.  Rows t of the block
 //          carry e^{Lambda_t - Lambda_p}, columns j carry e^{Lambda_p - Lambda_j};
 //          both factors are at most e^{(half-block decay span)}, and their
@@ -37,7 +39,7 @@ namespace prep {
 constexpr int NT = 256;
 constexpr int CC = 64;
 constexpr int LDM = gen::LDM;              // row stride of the fp32 C x C scratch
-constexpr int NROUND = 4;                  // pivot blocks of 16 rows
+constexpr int NROUND = 2;                  // pivot blocks of 32 rows
 constexpr float kGuard = 64.f;             // largest exponent a pivoted factor may take
 constexpr uint32_t IMG = CC * CC * 2;      // one bf16 C x C tile image
 constexpr uint32_t CHUNK_BYTES = 2 * IMG;  // T, then L
@@ -54,8 +56,6 @@ constexpr uint32_t EXT_BYTES = EXT_F + 128 * 4;
 enum RecordKind { REC_PLAIN = 0, REC_SCALAR = 1, REC_EXT = 2 };
 
 __host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
-// TMEM column of round r's accumulator (rounds are 16, 32, 48, 64 columns wide)
-__host__ __device__ constexpr uint32_t round_col(int r) { return 8u * r * (r + 1); }
 
 struct Plan {
     uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, TB, lam, beta, bar, misc, total, tmem_cols, tn;
@@ -355,16 +355,18 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
     } else if (!failed) {
-        // ---- pivoted rounds: row block r (rows 16r..16r+15), pivot 16r + 8
-        for (int r = 0; r < NROUND && !failed; ++r) {
-            const int p0 = 16 * r, pv = p0 + 8, n_r = 16 * (r + 1);
+        // ---- two row blocks of 32 tokens, each pivoted at its middle row p = 32r + 16:
+        //      rows t of the block carry e^{Lambda_t - Lambda_p}, columns j <= end of the
+        //      block carry e^{Lambda_p - Lambda_j}; growth is bounded by a 16-token span
+        for (int r = 0; r < 2 && !failed; ++r) {
+            const int p0 = 32 * r, pv = p0 + 16, n_r = 32 * (r + 1);
             bool clamp = false;
-            for (int u = tid; u < (32 + n_r) * (DK / 8); u += NT) {
+            for (int u = tid; u < (64 + n_r) * (DK / 8); u += NT) {
                 const int row = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
                 float v8[8];
-                if (row < 32) {
-                    const int t = p0 + (row & 15);
-                    ld_tile8(QK, 128, (row < 16 ? 0 : 64) + t, i0, v8);
+                if (row < 64) {   // rows 0-31: q of the block, 32-63: k of the block
+                    const int t = p0 + (row & 31);
+                    ld_tile8(QK, 128, (row < 32 ? 0 : 64) + t, i0, v8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int gi = (i0 + e) >> wsh;
@@ -377,19 +379,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
                     st_tile8(RA, 64, row, i0, v8);
                 } else {
-                    const int j = row - 32;
-                    ld_tile8(QK, 128, 64 + j, i0, v8);
+                    const int jj = row - 64;
+                    ld_tile8(QK, 128, 64 + jj, i0, v8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int gi = (i0 + e) >> wsh;
-                        float x = lam[pv * G + gi] - lam[j * G + gi];
+                        float x = lam[pv * G + gi] - lam[jj * G + gi];
                         if (x > kGuard) {
                             x = kGuard;
                             clamp = true;
                         }
                         v8[e] *= __expf(x);
                     }
-                    st_tile8(KC, 64, j, i0, v8);
+                    st_tile8(KC, 64, jj, i0, v8);
                 }
             }
             if (clamp)
@@ -400,8 +402,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 tc_fence_after();
                 const uint32_t id = idesc_bf16(64, n_r, false, false);
                 for (int k0 = 0; k0 < DK; k0 += 16)
-                    mma_bf16(tmem + round_col(r), desc_kmajor(RA, 64, 0, k0), desc_kmajor(KC, 64, 0, k0),
-                             id, k0 > 0);
+                    mma_bf16(tmem + 32 * r, desc_kmajor(RA, 64, 0, k0), desc_kmajor(KC, 64, 0, k0), id,
+                             k0 > 0);
                 mma_commit(&bars[1]);
             }
             failed = wait_bar(1, ph_mma);
@@ -409,51 +411,56 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         if (!failed) {
             tc_fence_after();
-            // M = 64 accumulator: round rows 0-15 (scores) sit in lanes 0-15 of quarter 0,
-            // rows 16-31 (key Gram) in lanes 0-15 of quarter 1.  Mf aliases the round tiles.
+            // M = 64 accumulator: row m at lane 32 (m / 16) + m % 16.  Block rows of q
+            // (m < 32) are in quarters 0-1, of k in quarters 2-3; row t = 32r + 16 (q & 1)
+            // + lane.  Each warp takes half of the round's columns; Mf aliases the round tiles.
             const int q4 = warp & 3, half = warp >> 2;
-            if (q4 < 2) {
-                const bool qrow = q4 == 0;
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int r = half == 0 ? (rr == 0 ? 0 : 3) : (rr == 0 ? 1 : 2);
-                    const int n_r = 16 * (r + 1), t = 16 * r + (lane & 15);
-                    for (int cb = 0; cb < 4; ++cb) {
-                        float d[16];
-                        if (16 * cb < n_r) {
-                            tmem_ld16(tq + round_col(r) + 16 * cb, d);
-                            tmem_ld_wait();
+            const bool qrow = q4 < 2;
+            for (int r = 0; r < 2; ++r) {
+                const int n_r = 32 * (r + 1), w = n_r / 2, c0 = half * w;
+                const int t = 32 * r + 16 * (q4 & 1) + (lane & 15);
+                for (int cb = 0; cb < w; cb += 16) {
+                    float d[16];
+                    tmem_ld16(tq + 32 * r + c0 + cb, d);
+                    tmem_ld_wait();
+                    if (lane < 16) {
+                        float v[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int jj = c0 + cb + e;
+                            v[e] = qrow ? ((jj <= t) ? d[e] : 0.f) : ((jj < t) ? sbeta[jj] * d[e] : 0.f);
+                        }
+                        if (qrow) {
+                            st_img8(img_L, t, c0 + cb, &v[0]);
+                            st_img8(img_L, t, c0 + cb + 8, &v[8]);
                         } else {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                d[e] = 0.f;
+                            for (int e = 0; e < 16; e += 4)
+                                *reinterpret_cast<float4 *>(&Mf[t * LDM + c0 + cb + e]) =
+                                    make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                         }
-                        if (lane < 16) {
-                            float v[16];
+                    }
+                }
+                if (r == 0 && lane < 16) {   // columns 32-63 of block 0's rows: above the diagonal
+                    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const int zc = 32 + 16 * half;
+                    if (qrow) {
+                        st_img8(img_L, t, zc, z);
+                        st_img8(img_L, t, zc + 8, z);
+                    } else {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const int j = 16 * cb + e;
-                                v[e] = qrow ? ((j <= t) ? d[e] : 0.f) : ((j < t) ? sbeta[j] * d[e] : 0.f);
-                            }
-                            if (qrow) {
-                                st_img8(img_L, t, 16 * cb, &v[0]);
-                                st_img8(img_L, t, 16 * cb + 8, &v[8]);
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < 16; e += 4)
-                                    *reinterpret_cast<float4 *>(&Mf[t * LDM + 16 * cb + e]) =
-                                        make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                            }
-                        }
+                        for (int e = 0; e < 16; e += 4)
+                            *reinterpret_cast<float4 *>(&Mf[t * LDM + zc + e]) = make_float4(0.f, 0.f, 0.f, 0.f);
                     }
                 }
             }
             __syncthreads();
             // blocks whose decay span overran the guard: exact fp32 rows from the raw tiles
-            for (int r = 0; r < NROUND; ++r) {
+            for (int r = 0; r < 2; ++r) {
                 if (!flag[r])
                     continue;
-                for (int u = tid; u < 16 * 8; u += NT) {
-                    const int t = 16 * r + (u >> 3), j0 = (u & 7) * 8;
+                for (int u = tid; u < 32 * 8; u += NT) {
+                    const int t = 32 * r + (u >> 3), j0 = (u & 7) * 8;
                     float lv[8], mv[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
