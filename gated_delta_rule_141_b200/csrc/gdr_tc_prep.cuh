@@ -93,7 +93,7 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
     s.lam = take(CC * G * 4 + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
     s.beta = s.lam + CC * G * 4;
     s.bar = (s.beta + CC * 4 + NROUND * 4 + 7u) & ~7u;
-    s.misc = s.bar + 16;
+    s.misc = s.bar + 24;
     s.total = o + 1024;
     s.tmem_cols = G > 1 ? 256u : 128u;            // W (M = 64, N = 128) needs 128 columns
     s.tn = G > 1 ? 192u : 64u;                    // Neumann products
@@ -116,6 +116,27 @@ __device__ __forceinline__ void st_img8(uint8_t *img, int r, int c, const float 
     *reinterpret_cast<uint4 *>(img + r * 128 + cc * 16) =
         make_uint4(ptx::pack_bf16(v[0], v[1]), ptx::pack_bf16(v[2], v[3]),
                    ptx::pack_bf16(v[4], v[5]), ptx::pack_bf16(v[6], v[7]));
+}
+
+// Lambda of row t at the eight channels [i0, i0 + 8).  Per-channel gates read two
+// vectors; grouped gates (64 or more channels a group) one broadcast value.
+__device__ __forceinline__ void lam8(const float *lam, int G, int wsh, int t, int i0, float *o)
+{
+    if (wsh == 0) {
+        const float4 a = *reinterpret_cast<const float4 *>(lam + t * G + i0);
+        const float4 b = *reinterpret_cast<const float4 *>(lam + t * G + i0 + 4);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+        o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+    } else if (wsh >= 3) {
+        const float x = lam[t * G + (i0 >> wsh)];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            o[e] = x;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            o[e] = lam[t * G + ((i0 + e) >> wsh)];
+    }
 }
 
 // SCALAR: the scalar-gate instantiation (no pivoting machinery, four CTAs per SM);
@@ -153,10 +174,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     uint8_t *img_T = a.out + (size_t)(kh * a.nchunks + c) * a.rec_bytes;
     uint8_t *img_L = img_T + IMG;
 
+    // The log-gates of a grouped / per-channel chunk are one contiguous run of Cl x G
+    // floats: one bulk copy when it is 16-byte aligned, else plain loads.
+    const float *g_src = p.g + (kh * T + c0) * G;
+    const uint32_t g_bytes = (uint32_t)(Cl * G * 4);
+    const bool g_bulk = !SCALAR && (g_bytes & 15u) == 0 && (reinterpret_cast<uintptr_t>(g_src) & 15u) == 0;
     if (tid == 0) {
-        mbar_init(&bars[0], 1);     // TMA
+        mbar_init(&bars[0], 1);     // TMA of q, k
         mbar_init(&bars[1], 1);     // MMA
+        mbar_init(&bars[2], 1);     // bulk copy of the log-gates
         fence_barrier_init();
+        if (g_bulk) {
+            mbar_arrive_expect_tx(&bars[2], g_bytes);
+            bulk_load(lam, g_src, g_bytes, &bars[2]);
+        }
         mbar_arrive_expect_tx(&bars[0], 2u * CC * DK * 2u);
         for (int kb = 0; kb < DK / 64; ++kb) {
             tma_load_3d(base + Ly.QK + kb * 128 * 128, &tm_q, &bars[0], 64 * kb, (int)c0, (int)kh);
@@ -170,8 +201,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     for (int t = tid; t < CC; t += NT)
         sbeta[t] = t < Cl ? p.beta[kh * T + c0 + t] : 0.f;
-    for (int u = tid; u < CC * G; u += NT)
-        lam[u] = (u / G) < Cl ? p.g[(kh * T + c0) * G + u] : 0.f;
+    if (g_bulk) {
+        for (int u = Cl * G + tid; u < CC * G; u += NT)   // rows past T (not copied)
+            lam[u] = 0.f;
+    } else {
+        for (int u = tid; u < CC * G; u += NT)
+            lam[u] = (u / G) < Cl ? g_src[u] : 0.f;
+    }
     if (tid < NROUND)
         flag[tid] = 0;
     tc_fence_before();
@@ -179,6 +215,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+
+    uint32_t ph_mma = 0;
+    bool failed = false;
+    auto wait_bar = [&](int i, uint32_t ph) {
+        const bool gave_up = !mbar_wait(&bars[i], ph);
+        if (gave_up)
+            atomicExch(&g_device_status, kTimeoutStatus);
+        return __syncthreads_or(gave_up ? 1 : 0) != 0;
+    };
+    if (g_bulk)
+        failed = wait_bar(2, 0);
 
     // ---- Lambda = cumsum over the chunk per decay group
     if (G <= 8) {
@@ -218,22 +265,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int gi = tid; gi < G; gi += NT)
             wide |= (lam[gi] - lam[(CC - 1) * G + gi]) > kGuard;
     wide = __syncthreads_or(wide ? 1 : 0) != 0;
-
-    uint32_t ph_mma = 0;
-    bool failed = false;
-    auto wait_bar = [&](int i, uint32_t ph) {
-        const bool gave_up = !mbar_wait(&bars[i], ph);
-        if (gave_up)
-            atomicExch(&g_device_status, kTimeoutStatus);
-        return __syncthreads_or(gave_up ? 1 : 0) != 0;
-    };
-    failed = wait_bar(0, 0);
+    failed = wait_bar(0, 0) || failed;
 
     const bool ext = a.kind == REC_EXT;
     if (!failed && ext) {
         float *fo = reinterpret_cast<float *>(img_T + EXT_F);
         for (int i = tid; i < DK; i += NT)
-            fo[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);
+            fo[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);   // F = e^{Lambda_C}
     }
     if (!failed && a.kind == REC_SCALAR) {   // per-token factors of the scalar gate
         float *ea = reinterpret_cast<float *>(img_T + SC_EA);
@@ -250,16 +288,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // ---- decayed operands for the state pass, straight from the raw tiles
         for (int u = tid; u < CC * (DK / 8); u += NT) {
             const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-            float qv[8], kv[8], qb[8], kh8[8];
+            float qv[8], kv[8], qb[8], kh8[8], lt[8], lc[8];
             ld_tile8(QK, 128, t, i0, qv);
             ld_tile8(QK, 128, 64 + t, i0, kv);
+            lam8(lam, G, wsh, t, i0, lt);
+            lam8(lam, G, wsh, CC - 1, i0, lc);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int gi = (i0 + e) >> wsh;
-                const float lt = lam[t * G + gi];
-                const float ea = __expf(lt), eb = __expf(lam[(CC - 1) * G + gi] - lt);
-                qb[e] = qv[e] * ea;
-                kh8[e] = kv[e] * eb;
+                qb[e] = qv[e] * __expf(lt[e]);
+                kh8[e] = kv[e] * __expf(lc[e] - lt[e]);
             }
             const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
             *reinterpret_cast<uint4 *>(img_T + EXT_QB + off) =
@@ -278,15 +315,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             //      state pass's decayed operands come out of the same sweep
             for (int u = tid; u < CC * (DK / 8); u += NT) {
                 const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float qv[8], kv[8], kh8[8], qb[8];
+                float qv[8], kv[8], kh8[8], qb[8], lt[8], lc[8];
                 ld_tile8(QK, 128, t, i0, qv);
                 ld_tile8(QK, 128, 64 + t, i0, kv);
+                lam8(lam, G, wsh, t, i0, lt);
+                lam8(lam, G, wsh, CC - 1, i0, lc);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int gi = (i0 + e) >> wsh;
-                    const float lt = lam[t * G + gi], lc = lam[(CC - 1) * G + gi];
-                    const float up = __expf(lt - lc), dn = __expf(lc - lt), ea = __expf(lt);
-                    qb[e] = qv[e] * ea;
+                    const float up = __expf(lt[e] - lc[e]), dn = __expf(lc[e] - lt[e]);
+                    qb[e] = qv[e] * __expf(lt[e]);
                     kh8[e] = kv[e] * dn;
                     qv[e] *= up;
                     kv[e] *= up;
@@ -363,14 +400,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             bool clamp = false;
             for (int u = tid; u < (64 + n_r) * (DK / 8); u += NT) {
                 const int row = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float v8[8];
+                float v8[8], la[8], lb[8];
                 if (row < 64) {   // rows 0-31: q of the block, 32-63: k of the block
                     const int t = p0 + (row & 31);
                     ld_tile8(QK, 128, (row < 32 ? 0 : 64) + t, i0, v8);
+                    lam8(lam, G, wsh, t, i0, la);
+                    lam8(lam, G, wsh, pv, i0, lb);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int gi = (i0 + e) >> wsh;
-                        float x = lam[t * G + gi] - lam[pv * G + gi];
+                        float x = la[e] - lb[e];
                         if (x > kGuard) {
                             x = kGuard;
                             clamp = true;
@@ -381,10 +419,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 } else {
                     const int jj = row - 64;
                     ld_tile8(QK, 128, 64 + jj, i0, v8);
+                    lam8(lam, G, wsh, pv, i0, la);
+                    lam8(lam, G, wsh, jj, i0, lb);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int gi = (i0 + e) >> wsh;
-                        float x = lam[pv * G + gi] - lam[jj * G + gi];
+                        float x = la[e] - lb[e];
                         if (x > kGuard) {
                             x = kGuard;
                             clamp = true;
@@ -611,21 +650,26 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const bool with_w = a.kind != REC_PLAIN;
     if (!failed) {
         __syncthreads();
-        if (with_w && !SCALAR) {
-            // Kbar = k e^{Lambda_t} in place in the k rows (they hold raw k after the
-            // pivoted blocks, k e^{Lambda_t - Lambda_C} after the chunk-end pivot)
+        if (with_w && !SCALAR && wide) {
+            // Kbar = k e^{Lambda_t} in place in the raw k rows of the pivoted blocks
             for (int u = tid; u < CC * (DK / 8); u += NT) {
                 const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float kv[8];
+                float kv[8], lt[8];
                 ld_tile8(QK, 128, 64 + t, i0, kv);
+                lam8(lam, G, wsh, t, i0, lt);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int gi = (i0 + e) >> wsh;
-                    kv[e] *= __expf(wide ? lam[t * G + gi] : lam[(CC - 1) * G + gi]);
-                }
+                for (int e = 0; e < 8; ++e)
+                    kv[e] *= __expf(lt[e]);
                 st_tile8(QK, 128, 64 + t, i0, kv);
             }
         }
+        // After the chunk-end pivot the k rows hold k e^{Lambda_t - Lambda_C}: W is then
+        // (T that) diag(e^{Lambda_C}), the column factors applied on the way out of TMEM
+        // (held in the inverse's scratch, free by now).
+        const bool w_cols = with_w && !SCALAR && !wide;
+        if (w_cols)
+            for (int i = tid; i < DK; i += NT)
+                Tf[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);
         // ---- T = diag(beta) A as a tile image: thread u writes 16-byte chunk u (coalesced).
         //      For W the same chunk goes to the bf16 operand tile in the dead q rows,
         //      scaled by e^{Lambda_j} for the scalar gate (W = T diag(e^Lambda) K).
@@ -678,6 +722,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     tmem_ld16(tq + cw + cb + 16, w1);
                     tmem_ld_wait();
                     if (rr >= 0) {
+                        if (w_cols) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                w0[e] *= Tf[cw + cb + e];
+                                w1[e] *= Tf[cw + cb + 16 + e];
+                            }
+                        }
                         uint8_t *img_W = img_T + REC_W + (cw >> 6) * IMG;
                         st_img8(img_W, rr, cb, &w0[0]);
                         st_img8(img_W, rr, cb + 8, &w0[8]);
@@ -693,6 +744,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mma_commit(&bars[1]);
         mbar_wait(&bars[1], ph_mma, 200000000ull);
         mbar_wait(&bars[0], 0, 200000000ull);
+        if (g_bulk)
+            mbar_wait(&bars[2], 0, 200000000ull);
     }
     tc_fence_before();
     __syncthreads();

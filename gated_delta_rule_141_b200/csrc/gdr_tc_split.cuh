@@ -350,24 +350,30 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 ok = false;
                 break;
             }
+            tc_fence_after();
+            // S_{c-1} -> bf16 operand of P; only then T_S <- F S_{c-1} (the update MMA
+            // accumulates onto it), which nothing reads before E_READY
+            float s0[16], s1[16];
+            tmem_ld16(tq + T_S + cs, s0);
+            tmem_ld16(tq + T_S + cs + 16, s1);
+            tmem_ld_wait();
+            st_tile8(S_T, KD, R, cs, &s0[0]);
+            st_tile8(S_T, KD, R, cs + 8, &s0[8]);
+            st_tile8(S_T, KD, R, cs + 16, &s1[0]);
+            st_tile8(S_T, KD, R, cs + 24, &s1[8]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_sync(NB_STATE, N_STATE);
+            if (stid == 0)
+                mbar_arrive(&bars[S_READY]);
             if (named_vote_or(NB_STATE, N_STATE,
                               !wait_or_abort(&bars[FULLX0 + s], (c >> 1) & 1, abort_flag))) {
                 ok = false;
                 break;
             }
-            tc_fence_after();
             const Gates *gt = gates_of(s);
-            const float F = scalar ? gt->F[0] : gt->F[R];
-            // S_{c-1} -> bf16 operand; T_S <- F S_{c-1} (the update MMA accumulates onto it)
             {
-                float s0[16], s1[16];
-                tmem_ld16(tq + T_S + cs, s0);
-                tmem_ld16(tq + T_S + cs + 16, s1);
-                tmem_ld_wait();
-                st_tile8(S_T, KD, R, cs, &s0[0]);
-                st_tile8(S_T, KD, R, cs + 8, &s0[8]);
-                st_tile8(S_T, KD, R, cs + 16, &s1[0]);
-                st_tile8(S_T, KD, R, cs + 24, &s1[8]);
+                const float F = scalar ? gt->F[0] : gt->F[R];
 #pragma unroll
                 for (int n = 0; n < 16; ++n) {
                     s0[n] *= F;
@@ -376,12 +382,6 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tmem_st16(tq + T_S + cs, s0);
                 tmem_st16(tq + T_S + cs + 16, s1);
             }
-            tmem_st_wait();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_sync(NB_STATE, N_STATE);
-            if (stid == 0)
-                mbar_arrive(&bars[S_READY]);
             if (named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[P_FULL], par, abort_flag))) {
                 ok = false;
                 break;
@@ -417,12 +417,14 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     st_tile8(EH_T, CC, t, cs + 24, &u1[8]);
                 }
             }
+            tmem_st_wait();
             fence_proxy_async_smem();
             tc_fence_before();
             named_sync(NB_STATE, N_STATE);
             if (stid == 0)
                 mbar_arrive(&bars[E_READY]);
         }
+        tmem_st_wait();   // a chunk left early may still have its F S store in flight
         if (ok && N > 0 &&
             named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[UPD_DONE], (N - 1) & 1, abort_flag)))
             ok = false;

@@ -58,6 +58,8 @@ SMALL = [
     (1, dict(B=1, Hk=1, Hv=1, T=256), 64, "neumann", "tc2"),
     (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 64, "exact", "tc2"),
     (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 64, "exact", "tc2"),
+    # odd T: the second head's gate rows start off a 16-byte boundary (plain loads)
+    (2, dict(B=1, Hk=2, Hv=2, T=256 - 27, gate_mode=W.GATE_GROUP64), 64, "exact", "tc2"),
     (2, dict(B=1, Hk=2, Hv=2, T=256), 64, "neumann", "tc2"),
     (4, dict(Hk=2, Hv=2, T=640 - 5), 128, "exact", "tc2"),               # strong decay, S0
     (4, dict(Hk=1, Hv=1, T=64), 64, "exact", "tc2"),                     # a single chunk
