@@ -91,22 +91,53 @@ struct GenArgs {
 // Row of an M = 64 accumulator held by this thread (lanes 0-15 of each quarter).
 __device__ __forceinline__ int row64g(int warp, int lane) { return lane < 16 ? 16 * (warp & 3) + lane : -1; }
 
+// acc[i][n] = sum over l in [l0, K) of A[i * a_step + l] * B[l * ldb + n], n < 4: a 4 x 4
+// block of a product, the inner index in ascending order.
+template <int K>
+__device__ __forceinline__ void block_product4x4(float (&acc)[4][4], const float *A, int a_step,
+                                                 const float *B, int ldb, int l0)
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+            acc[i][n] = 0.f;
+#pragma unroll 4
+    for (int l = l0; l < K; ++l) {
+        float a[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            a[i] = A[i * a_step + l];
+        const float4 b = *reinterpret_cast<const float4 *>(B + l * ldb);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[i][0] += a[i] * b.x;
+            acc[i][1] += a[i] * b.y;
+            acc[i][2] += a[i] * b.z;
+            acc[i][3] += a[i] * b.w;
+        }
+    }
+}
+
 // In-place exact inverse of I + M (64 x 64, M strictly lower) by block doubling.
 __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
 {
-    // diagonal 16 x 16 blocks, exact forward substitution (into Tf, then back)
+    // diagonal 16 x 16 blocks, exact forward substitution (into Tf, then back).
+    // Column cc of the block's inverse, right-looking: once x_j is final it is
+    // applied to every later row at once, so the dependent chain is 15 steps
+    // long (each x_t still sums its terms in the order j = 0, 1, ...).
     if (tid < 64) {
         const int blk = tid >> 4, cc = tid & 15, o = 16 * blk;
         float x[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const float *mrow = Mf + (o + t) * LDM + o;
-            float acc = (t == cc) ? 1.f : 0.f;
+        for (int t = 0; t < 16; ++t)
+            x[t] = (t == cc) ? 1.f : 0.f;
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (j < t)
-                    acc -= mrow[j] * x[j];
-            x[t] = acc;
+        for (int j = 0; j < 15; ++j) {
+            const float xj = x[j];
+#pragma unroll
+            for (int t = j + 1; t < 16; ++t)
+                x[t] -= Mf[(o + t) * LDM + o + j] * xj;
         }
 #pragma unroll
         for (int t = 0; t < 16; ++t)
@@ -118,80 +149,47 @@ __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
         Mf[(16 * blk + t) * LDM + 16 * blk + cc] = Tf[idx];
     }
     __syncthreads();
-    // 16 -> 32 (two pairs): T = M21 X11, X21 = -X22 T
-    {
-        const int pr = tid >> 7, r = (tid >> 3) & 15, c2 = (tid & 7) * 2, o = 32 * pr;
-        float mr[16];
+    // The doubling steps are products of small dense blocks.  Each thread owns a
+    // 4 x 4 block of the product: per step of the inner index it loads four A
+    // values (shared by the lanes of a row group) and one float4 of B, which is
+    // half the shared-memory traffic per FMA of one output row per thread.
+    const int warp = tid >> 5, lane = tid & 31;
+    // 16 -> 32, pair pr in warp pr (lanes 0-15): T = M21 X11, X21 = -X22 T (16 x 16 blocks)
+    if (warp < 2 && lane < 16) {
+        const int pr = warp, rg = lane >> 2, c0 = 4 * (lane & 3), o = 32 * pr;
+        float acc[4][4];
+        block_product4x4<16>(acc, Mf + (o + 16 + rg) * LDM + o, 4 * LDM, Mf + o * LDM + o + c0, LDM, 0);
 #pragma unroll
-        for (int l = 0; l < 16; l += 4) {
-            const float4 m4 = *reinterpret_cast<const float4 *>(&Mf[(o + 16 + r) * LDM + o + l]);
-            mr[l] = m4.x; mr[l + 1] = m4.y; mr[l + 2] = m4.z; mr[l + 3] = m4.w;
-        }
-        float t0 = 0.f, t1 = 0.f;
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(&Tf[(pr * 16 + rg + 4 * i) * 36 + c0]) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        __syncwarp(0x0000ffffu);
+        block_product4x4<16>(acc, Mf + (o + 16 + rg) * LDM + o + 16, 4 * LDM, Tf + pr * 16 * 36 + c0, 36, 0);
 #pragma unroll
-        for (int l = 0; l < 16; ++l) {
-            const float2 a2 = *reinterpret_cast<const float2 *>(&Mf[(o + l) * LDM + o + c2]);
-            t0 += mr[l] * a2.x;
-            t1 += mr[l] * a2.y;
-        }
-        __syncthreads();
-        *reinterpret_cast<float2 *>(&Tf[(pr * 16 + r) * 36 + c2]) = make_float2(t0, t1);
-        __syncthreads();
-        float ar[16];
-#pragma unroll
-        for (int l = 0; l < 16; l += 4) {
-            const float4 a4 = *reinterpret_cast<const float4 *>(&Mf[(o + 16 + r) * LDM + o + 16 + l]);
-            ar[l] = a4.x; ar[l + 1] = a4.y; ar[l + 2] = a4.z; ar[l + 3] = a4.w;
-        }
-        float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l) {
-            const float2 t2 = *reinterpret_cast<const float2 *>(&Tf[(pr * 16 + l) * 36 + c2]);
-            x0 += ar[l] * t2.x;
-            x1 += ar[l] * t2.y;
-        }
-        *reinterpret_cast<float2 *>(&Mf[(o + 16 + r) * LDM + o + c2]) = make_float2(-x0, -x1);
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(&Mf[(o + 16 + rg + 4 * i) * LDM + o + c0]) =
+                make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
     }
     __syncthreads();
-    // 32 -> 64
-    {
-        const int r = tid >> 3, c4 = (tid & 7) * 4;
-        float mr[32];
+    // 32 -> 64 on warps 0-1: rows rg + 8i of the 32-row block, columns 16 warp + c0.
+    // X11 is lower triangular, so its rows above 16 warp vanish in those columns.
+    const int rg = lane >> 2, c0 = 16 * warp + 4 * (lane & 3);
+    if (warp < 2) {
+        float acc[4][4];
+        block_product4x4<32>(acc, Mf + (32 + rg) * LDM, 8 * LDM, Mf + c0, LDM, 16 * warp);
 #pragma unroll
-        for (int l = 0; l < 32; l += 4) {
-            const float4 m4 = *reinterpret_cast<const float4 *>(&Mf[(32 + r) * LDM + l]);
-            mr[l] = m4.x; mr[l + 1] = m4.y; mr[l + 2] = m4.z; mr[l + 3] = m4.w;
-        }
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(&Tf[(rg + 8 * i) * 36 + c0]) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    }
+    __syncthreads();
+    if (warp < 2) {
+        float acc[4][4];
+        block_product4x4<32>(acc, Mf + (32 + rg) * LDM + 32, 8 * LDM, Tf + c0, 36, 0);
 #pragma unroll
-        for (int l = 0; l < 32; l += 2) {
-            const float4 a = *reinterpret_cast<const float4 *>(&Mf[l * LDM + c4]);
-            const float4 b2 = *reinterpret_cast<const float4 *>(&Mf[(l + 1) * LDM + c4]);
-            acc.x += mr[l] * a.x; acc.y += mr[l] * a.y; acc.z += mr[l] * a.z; acc.w += mr[l] * a.w;
-            acc2.x += mr[l + 1] * b2.x; acc2.y += mr[l + 1] * b2.y;
-            acc2.z += mr[l + 1] * b2.z; acc2.w += mr[l + 1] * b2.w;
-        }
-        *reinterpret_cast<float4 *>(&Tf[r * 36 + c4]) =
-            make_float4(acc.x + acc2.x, acc.y + acc2.y, acc.z + acc2.z, acc.w + acc2.w);
-        __syncthreads();
-        float ar[32];
-#pragma unroll
-        for (int l = 0; l < 32; l += 4) {
-            const float4 a4 = *reinterpret_cast<const float4 *>(&Mf[(32 + r) * LDM + 32 + l]);
-            ar[l] = a4.x; ar[l + 1] = a4.y; ar[l + 2] = a4.z; ar[l + 3] = a4.w;
-        }
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f), x2 = x;
-#pragma unroll
-        for (int l = 0; l < 32; l += 2) {
-            const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[l * 36 + c4]);
-            const float4 u4 = *reinterpret_cast<const float4 *>(&Tf[(l + 1) * 36 + c4]);
-            x.x += ar[l] * t4.x; x.y += ar[l] * t4.y; x.z += ar[l] * t4.z; x.w += ar[l] * t4.w;
-            x2.x += ar[l + 1] * u4.x; x2.y += ar[l + 1] * u4.y;
-            x2.z += ar[l + 1] * u4.z; x2.w += ar[l + 1] * u4.w;
-        }
-        __syncthreads();
-        *reinterpret_cast<float4 *>(&Mf[(32 + r) * LDM + c4]) =
-            make_float4(-(x.x + x2.x), -(x.y + x2.y), -(x.z + x2.z), -(x.w + x2.w));
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(&Mf[(32 + rg + 8 * i) * LDM + c0]) =
+                make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
     }
     __syncthreads();
 }

@@ -366,29 +366,33 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const bool qrow = R < CC;
             const int t = qrow ? R : R - CC;
             const float lt = lam[t * G];
-            float out[32];
+            // two halves of 16 columns (fewer live registers)
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int j = j0 + u;
-                const float d = u < 16 ? g0[u] : g1[u - 16];
-                const bool keep = qrow ? (j <= t) : (j < t);
-                float v = 0.f;
-                if (keep)
-                    v = SCALAR ? d * __expf(lt - lam[j]) : d;
-                if (!qrow)
-                    v *= sbeta[j];
-                out[u] = v;
-            }
-            if (qrow) {
+            for (int h = 0; h < 2; ++h) {
+                const int jh = j0 + 16 * h;
+                float out[16];
 #pragma unroll
-                for (int u = 0; u < 32; u += 8)
-                    st_img8(img_L, t, j0 + u, &out[u]);
-            } else {
-                // Mf aliases the (now dead) [q; k] tile
+                for (int u = 0; u < 16; ++u) {
+                    const int j = jh + u;
+                    const float d = h == 0 ? g0[u] : g1[u];
+                    const bool keep = qrow ? (j <= t) : (j < t);
+                    float v = 0.f;
+                    if (keep)
+                        v = SCALAR ? d * __expf(lt - lam[j]) : d;
+                    if (!qrow)
+                        v *= sbeta[j];
+                    out[u] = v;
+                }
+                if (qrow) {
+                    st_img8(img_L, t, jh, &out[0]);
+                    st_img8(img_L, t, jh + 8, &out[8]);
+                } else {
+                    // Mf holds the k rows' products in fp32
 #pragma unroll
-                for (int u = 0; u < 32; u += 4)
-                    *reinterpret_cast<float4 *>(&Mf[t * LDM + j0 + u]) =
-                        make_float4(out[u], out[u + 1], out[u + 2], out[u + 3]);
+                    for (int u = 0; u < 16; u += 4)
+                        *reinterpret_cast<float4 *>(&Mf[t * LDM + jh + u]) =
+                            make_float4(out[u], out[u + 1], out[u + 2], out[u + 3]);
+                }
             }
         }
     } else if (!failed) {
