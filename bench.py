@@ -308,7 +308,9 @@ def main():
     ws_bytes = gdr.workspace_bytes(shape_run, chunk, gm_run, args.inverse)
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda") if ws_bytes else None
     kern = gdr.select_kernel(shape_run, chunk, gm_run, args.inverse)
-    launches_per_step = 2 if kern == gdr.KERNEL_TC2 else 1
+    # the two-pass path: pass 1, then one state pass, or three when segmented
+    nseg = gdr.state_segments(shape_run, chunk, gm_run, args.inverse) if kern == gdr.KERNEL_TC2 else 0
+    launches_per_step = (1 + (1 if nseg == 1 else 3)) if kern == gdr.KERNEL_TC2 else 1
     # with an L2 flush between steps, only the launches themselves are timed
     step_events = []
 
@@ -417,7 +419,8 @@ def main():
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.in_dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
-        "config": dict(config_dict(w, chunk, args.inverse, world), kernel_chunk=kchunk),
+        "config": dict(config_dict(w, chunk, args.inverse, world), kernel_chunk=kchunk,
+                       state_segments=nseg),
         "tflops": roof["tflops"], "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step, "kernel": gdr.KERNEL_NAMES.get(kern, str(kern)),
         "clocks": sampler.summary(),

@@ -239,6 +239,19 @@ int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
     return which == GDR_KERNEL_SIMT ? p.C : gdr::tc_kernel_chunk(p);
 }
 
+int gdr_state_segments(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                       gdr_inverse_mode inverse_mode)
+{
+    gdr::Params p;
+    const gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return -static_cast<int>(st);
+    const int which = choose(p, shape->kernel, SIZE_MAX);
+    if (which < 0)
+        return which;
+    return which == GDR_KERNEL_TC2 ? gdr::tc2_state_segments(p) : 0;
+}
+
 gdr_status gdr_device_status(void *stream)
 {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)

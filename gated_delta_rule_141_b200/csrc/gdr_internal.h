@@ -46,6 +46,8 @@ int launch_tc(const Params &p, cudaStream_t stream);
 bool tc2_supports(const Params &p);
 size_t tc2_workspace_bytes(const Params &p);
 int launch_tc2(const Params &p, void *workspace, cudaStream_t stream);
+// Segments per sequence of its state pass (1: sequential; more: segment-parallel).
+int tc2_state_segments(const Params &p);
 
 // The first pass alone, at the requested chunk length (public gdr_chunk_prepare).
 bool prepare_supports(const Params &p);

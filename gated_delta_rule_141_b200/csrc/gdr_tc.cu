@@ -635,7 +635,15 @@ int launch_tc(const Params &p0, cudaStream_t stream)
 
 bool tc2_supports(const Params &p0) { return split::supports(as_kernel_chunk(p0)); }
 
-size_t tc2_workspace_bytes(const Params &p0) { return prep::ws_bytes(as_kernel_chunk(p0)); }
+size_t tc2_workspace_bytes(const Params &p0)
+{
+    // the records, then (for few long sequences) the segmented state pass's buffers
+    const Params p = as_kernel_chunk(p0);
+    const size_t rec = prep::ws_bytes(p), seg = split::seg_bytes(p);
+    return seg == 0 ? rec : ((rec + 255) & ~size_t(255)) + seg;
+}
+
+int tc2_state_segments(const Params &p0) { return split::seg_plan(as_kernel_chunk(p0)).nseg; }
 
 int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
 {

@@ -17,14 +17,17 @@
 //
 // Roles (warp-specialised, hand-offs through mbarriers; every wait bounded):
 //   warps 0-1   epilogue: O = f (Q S) + L E from TMEM to global memory
-//   warp 2      producer: TMA / bulk copies into a 2-stage ring
+//   warps 2, 12 producers: TMA / bulk copies into a 2-stage ring.  A thread's
+//               bulk copies are accepted one after another (about 30 bytes a
+//               cycle), so two threads share a stage: warp 2 issues W, Q and
+//               the factors, warp 12 T and V, then group Y
 //   warp 3      MMA issuer (one thread)
 //   warps 4-11  state chain: S (fp32, TMEM) -> bf16 operand, E = U - P; two
 //               warps per TMEM lane quarter, each lane on 32 of the 64 columns
 // A stage is loaded in two groups with their own barriers, so that it can be
 // refilled as soon as each group's last reader is done:
-//   X = {W, Q, T, V, factors}: read by U, P and the state warps -> free once E
-//       of the chunk is formed;
+//   X = {W, Q, T, V, factors}: read by U, P and the state warps (which copy their
+//       factors to registers early) -> free once P is done;
 //   Y = {K, L}: read by the update and the readout -> free after them.
 // MMA operands are stacked so that M = 128 and no product reads a tile that a
 // load may be refilling:
@@ -33,12 +36,12 @@
 
 namespace split {
 
-constexpr int NWARP = 12;
-constexpr int NTHR = NWARP * 32;   // 384
+constexpr int NWARP = 13;
+constexpr int NTHR = NWARP * 32;   // 416
 constexpr int CC = 64;
 constexpr int KD = 128;
 constexpr int NVC = 64;
-constexpr int W_EPI0 = 0, W_PROD = 2, W_MMA = 3, W_STATE0 = 4;
+constexpr int W_EPI0 = 0, W_PROD = 2, W_MMA = 3, W_STATE0 = 4, W_PROD_Y = 12;
 constexpr int N_STATE = 256, N_EPI = 64;
 constexpr int NB_STATE = 1, NB_EPI = 2;   // named barriers
 
@@ -88,13 +91,74 @@ __host__ __device__ inline Plan plan(bool scalar)
     return s;
 }
 
+// How a launch walks the chunks.  MODE_SEQ: every CTA walks its whole sequence.
+// The segment-parallel form cuts each sequence into nseg segments of seg_len
+// chunks (grid.z = segment) and composes the affine maps S -> A_c S + B_c of the
+// chunks, A_c = F_c - Khat_c^T W_c and B_c = Khat_c^T U_c:
+//   MODE_SEG_AB: value-tile CTAs run their segment from S = 0 and store its end
+//     state Btil (no outputs); transition CTAs (grid.x past the value tiles, two
+//     per key head) run it from the identity with no values and store
+//     Atil = prod A_c, 64 of its columns each;
+//   seg_combine_kernel: S_start(0) = S0, S_start(g + 1) = Atil_g S_start(g) + Btil_g;
+//   MODE_SEG_C: every segment runs from its S_start and writes o; the last one
+//     writes S_final.
+enum Mode { MODE_SEQ = 0, MODE_SEG_AB = 1, MODE_SEG_C = 2 };
+
 struct SplitArgs {
     Params p;
     const uint8_t *factors;   // first-pass output, [B * Hk * nchunks][rec_bytes]
     uint32_t rec_bytes;       // prep::SC_BYTES (scalar gate) or prep::EXT_BYTES
     int nvt;
     int nchunks;
+    int mode;                 // Mode
+    int nseg, seg_len;        // segments per sequence and chunks per segment
+    float *seg_end;           // [B][Hv][nseg][KD][dv]: Btil of each segment
+    float *seg_trans;         // [B][Hk][nseg][KD][KD]: Atil of each segment
+    float *seg_start;         // [B][Hv][nseg][KD][dv]: the state each segment starts from
 };
+
+// Segment count for the state pass of a request: cost model in chunk periods, one
+// resident CTA per SM on kSMs SMs.  The segmented form does about three times the
+// chain work (values from zero, the transition, values again), so it pays only
+// when the sequential pass leaves most SMs idle.
+constexpr int kSMs = 148;
+constexpr int kMinSegChunks = 16;
+
+struct SegPlan {
+    int nseg, seg_len;
+};
+
+inline SegPlan seg_plan(const Params &p)
+{
+    const int N = prep::nchunks(p);
+    const long nvh = (long)(p.dv / NVC) * p.Hv * p.B;
+    const long ntr = (long)(KD / NVC) * p.Hk * p.B;
+    auto waves = [](long ctas) { return (ctas + kSMs - 1) / kSMs; };
+    const long seq_cost = waves(nvh) * (long)N;
+    SegPlan best{1, N};
+    long best_cost = seq_cost;
+    for (int ns = 2; ns <= N / kMinSegChunks; ++ns) {
+        const int L = (N + ns - 1) / ns;
+        const int nsg = (N + L - 1) / L;
+        const long cost = (waves((nvh + ntr) * nsg) + waves(nvh * nsg)) * (long)L + nsg;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = SegPlan{nsg, L};
+        }
+    }
+    return (best.nseg > 1 && best_cost * 5 <= seq_cost * 4) ? best : SegPlan{1, N};
+}
+
+// Bytes past the records that the segmented form needs (256-byte aligned pieces).
+inline size_t seg_bytes(const Params &p)
+{
+    const SegPlan sp = seg_plan(p);
+    if (sp.nseg == 1)
+        return 0;
+    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t per_v = (size_t)p.B * p.Hv * sp.nseg * KD * p.dv * 4;
+    return 2 * al(per_v) + al((size_t)p.B * p.Hk * sp.nseg * KD * KD * 4);
+}
 
 // Bounded wait without sleeping between probes: every hand-off in this kernel
 // is on or next to the per-chunk critical chain, where a back-off sleep would
@@ -136,15 +200,25 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint8_t *base = smem_raw + (base_u32 - smem_u32(smem_raw));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nt = blockIdx.x % args.nvt;
-    const int hv = blockIdx.x / args.nvt;
+    const int nvh = args.nvt * p.Hv;   // value-tile CTAs per batch entry
+    // a transition CTA of the segmented form: identity start, no values, no outputs
+    const bool trans = args.mode == MODE_SEG_AB && (int)blockIdx.x >= nvh;
+    const int xi = trans ? (int)blockIdx.x - nvh : (int)blockIdx.x;
+    const int nt = trans ? xi % (KD / NVC) : xi % args.nvt;
+    const int hv = trans ? 0 : xi / args.nvt;
     const int b = blockIdx.y;
-    const int hk = hv / p.R;
+    const int hk = trans ? xi / (KD / NVC) : hv / p.R;
     const int n0 = nt * NVC;
     const long kh = (long)b * p.Hk + hk;
     const long vh = (long)b * p.Hv + hv;
     const int T = p.T;
     const int N = args.nchunks;
+    const bool outputs = args.mode != MODE_SEG_AB;   // o is written
+    // this CTA's chunks: cbeg .. cbeg + nloc - 1 (local index i = c - cbeg drives the
+    // ring stages and barrier phases)
+    const int seg = blockIdx.z;
+    const int cbeg = seg * args.seg_len;
+    const int nloc = min(args.seg_len, N - cbeg);
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
@@ -153,8 +227,8 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint32_t S_T = base_u32 + Ly.S, E_T = base_u32 + Ly.E, EH_T = base_u32 + Ly.Eh;
 
     if (tid == 0) {
-        for (int i = 0; i < NBARS; ++i)
-            mbar_init(&bars[i], 1);
+        for (int i = 0; i < NBARS; ++i)   // FREEX: the MMAs' commit and the state warps
+            mbar_init(&bars[i], (i == FREEX0 || i == FREEX1) ? 2 : 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
@@ -182,15 +256,16 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     if (warp == W_PROD) {
         // ------------------------------------------------------------ producer
-        int armx[2] = {0, 0}, army[2] = {0, 0};   // loads armed per stage and group
-        for (int c = 0; c < N; ++c) {
-            const int s = c & 1;
+        int armx[2] = {0, 0};   // group X loads armed per stage
+        for (int i = 0; i < nloc; ++i) {
+            const int c = cbeg + i, s = i & 1;
             const long c0 = (long)c * CC;
             const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
             uint8_t *qwk = base + Ly.qwk[s];
-            // group X: W, Q (or Qbar), T, V, the decay factors
-            if (c >= 2) {
-                const bool ok = wait_or_abort(&bars[FREEX0 + s], ((c >> 1) - 1) & 1, abort_flag);
+            // group X: W, Q (or Qbar), T, V, the decay factors.  Q only where o is
+            // written; T and V not for a transition CTA.
+            if (i >= 2) {
+                const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
                 if (__any_sync(0xffffffffu, !ok))
                     break;
             }
@@ -198,32 +273,65 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 uint64_t *full = &bars[FULLX0 + s];
                 const uint32_t fac_bytes = scalar ? prep::SC_BYTES - prep::SC_EA : KD * 4;
                 // W, Q: two 64-column images each; T: one; V: 64 x 64 bf16
-                mbar_arrive_expect_tx(full, 5u * prep::IMG + CC * NVC * 2 + fac_bytes);
+                mbar_arrive_expect_tx(full, 2u * prep::IMG + (outputs ? 2u * prep::IMG : 0u) +
+                                                (trans ? 0u : prep::IMG + CC * NVC * 2) + fac_bytes);
                 for (int kb = 0; kb < KD / 64; ++kb) {
                     uint8_t *blk = qwk + kb * 192 * 128;
                     bulk_load(blk + 64 * 128, fac + prep::REC_W + kb * prep::IMG, prep::IMG, full);
+                    if (!outputs)
+                        continue;
                     if (scalar)
                         tma_load_3d(blk, &tm_q, full, 64 * kb, (int)c0, (int)kh);
                     else
                         bulk_load(blk, fac + prep::EXT_QB + kb * prep::IMG, prep::IMG, full);
                 }
-                bulk_load(base + Ly.ab[s] + 64 * 128, fac, prep::IMG, full);
-                tma_load_3d(base + Ly.v[s], &tm_v, full, n0, (int)c0, (int)vh);
                 if (scalar)
                     bulk_load(gates_of(s)->ea, fac + prep::SC_EA, fac_bytes, full);
                 else
                     bulk_load(gates_of(s)->F, fac + prep::EXT_F, fac_bytes, full);
             }
             armx[s] += 1;
-            // group Y: K (or Khat), L
-            if (c >= 2) {
-                const bool ok = wait_or_abort(&bars[FREEY0 + s], ((c >> 1) - 1) & 1, abort_flag);
+        }
+        // drain loads that may still be landing (bounded): the last armed phase of
+        // each barrier, whether or not a consumer saw it
+        if (lane == 0) {
+            for (int s = 0; s < 2; ++s)
+                if (armx[s] > 0)
+                    mbar_wait(&bars[FULLX0 + s], (armx[s] - 1) & 1, 200000000ull);
+        }
+    } else if (warp == W_PROD_Y) {
+        // ------------------------------------------------------------ second producer
+        // T and V of group X (their bytes are part of what warp W_PROD expects on FULLX,
+        // so the phase completes only when both threads' copies have landed), then
+        // group Y.
+        int army[2] = {0, 0};   // group Y loads armed per stage
+        for (int i = 0; i < nloc; ++i) {
+            const int c = cbeg + i, s = i & 1;
+            const long c0 = (long)c * CC;
+            const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
+            uint8_t *qwk = base + Ly.qwk[s];
+            // T and V of group X (counted in the FULLX bytes that warp W_PROD expects)
+            if (!trans) {
+                if (i >= 2) {
+                    const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
+                    if (__any_sync(0xffffffffu, !ok))
+                        break;
+                }
+                if (lane == 0) {
+                    uint64_t *full = &bars[FULLX0 + s];
+                    bulk_load(base + Ly.ab[s] + 64 * 128, fac, prep::IMG, full);
+                    tma_load_3d(base + Ly.v[s], &tm_v, full, n0, (int)c0, (int)vh);
+                }
+            }
+            // group Y: K (or Khat), L (L only where o is written)
+            if (i >= 2) {
+                const bool ok = wait_or_abort(&bars[FREEY0 + s], ((i >> 1) - 1) & 1, abort_flag);
                 if (__any_sync(0xffffffffu, !ok))
                     break;
             }
             if (lane == 0) {
                 uint64_t *full = &bars[FULLY0 + s];
-                mbar_arrive_expect_tx(full, 3u * prep::IMG);
+                mbar_arrive_expect_tx(full, (outputs ? 3u : 2u) * prep::IMG);
                 for (int kb = 0; kb < KD / 64; ++kb) {
                     uint8_t *blk = qwk + kb * 192 * 128 + 128 * 128;
                     if (scalar)
@@ -231,19 +339,15 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     else
                         bulk_load(blk, fac + prep::EXT_KH + kb * prep::IMG, prep::IMG, full);
                 }
-                bulk_load(base + Ly.lz[s], fac + prep::IMG, prep::IMG, full);
+                if (outputs)
+                    bulk_load(base + Ly.lz[s], fac + prep::IMG, prep::IMG, full);
             }
             army[s] += 1;
         }
-        // drain loads that may still be landing (bounded): the last armed phase of
-        // each barrier, whether or not a consumer saw it
         if (lane == 0) {
-            for (int s = 0; s < 2; ++s) {
-                if (armx[s] > 0)
-                    mbar_wait(&bars[FULLX0 + s], (armx[s] - 1) & 1, 200000000ull);
+            for (int s = 0; s < 2; ++s)
                 if (army[s] > 0)
                     mbar_wait(&bars[FULLY0 + s], (army[s] - 1) & 1, 200000000ull);
-            }
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
@@ -272,11 +376,12 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(tmem + T_U + 64 * st, a0 + kstep(k0, 128), v0 + mstep(k0), id_u, k0 > 0);
             };
-            bool ok = true, u_ready = false;
-            for (int c = 0; c < N && ok; ++c) {
-                const int s = c & 1;
-                const uint32_t par = c & 1;
-                if (!(ok = wait_or_abort(&bars[FULLX0 + s], (c >> 1) & 1, abort_flag)))
+            // a transition CTA has no values: U = 0 and no U product (u_ready stays true)
+            bool ok = true, u_ready = trans;
+            for (int i = 0; i < nloc && ok; ++i) {
+                const int s = i & 1;
+                const uint32_t par = i & 1;
+                if (!(ok = wait_or_abort(&bars[FULLX0 + s], (i >> 1) & 1, abort_flag)))
                     break;
                 if (!u_ready) {
                     tc_fence_after();
@@ -284,26 +389,26 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
                 if (!(ok = wait_or_abort(&bars[S_READY], par, abort_flag)))
                     break;
-                if (c >= 2 && !(ok = wait_or_abort(&bars[OFREE0 + s], ((c >> 1) - 1) & 1, abort_flag)))
+                if (i >= 2 && !(ok = wait_or_abort(&bars[OFREE0 + s], ((i >> 1) - 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
                 const uint64_t qw = d_qw0 + s * dqw, kt = d_kt0 + s * dqw, lz = d_lz0 + s * dlz;
                 for (int k0 = 0; k0 < KD; k0 += 16)
                     mma_bf16(tmem + T_PO + 64 * s, qw + kstep(k0, 192), d_s + mstep(k0), id_po, k0 > 0);
                 mma_commit(&bars[P_FULL]);
+                // U and P are the last tensor-core readers of group X (the state warps
+                // hold their factors in registers by then and arrive themselves)
+                mma_commit(&bars[FREEX0 + s]);
                 // the next chunk's U overlaps this chunk's E step when its tiles are in
-                u_ready = false;
-                if (c + 1 < N && mbar_test(&bars[FULLX0 + (s ^ 1)], ((c + 1) >> 1) & 1)) {
+                u_ready = trans;
+                if (!trans && i + 1 < nloc && mbar_test(&bars[FULLX0 + (s ^ 1)], ((i + 1) >> 1) & 1)) {
                     tc_fence_after();
                     issue_u(s ^ 1);
                     u_ready = true;
                 }
                 if (!(ok = wait_or_abort(&bars[E_READY], par, abort_flag)))
                     break;
-                // group X of this stage has no reader left: P and U finished before
-                // the state warps formed E (they waited for P_FULL)
-                mbar_arrive(&bars[FREEX0 + s]);
-                if (!(ok = wait_or_abort(&bars[FULLY0 + s], (c >> 1) & 1, abort_flag)))
+                if (!(ok = wait_or_abort(&bars[FULLY0 + s], (i >> 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
                 for (int k0 = 0; k0 < CC; k0 += 16)
@@ -323,12 +428,20 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int stid = tid - W_STATE0 * 32;
         const int cs = 32 * ((warp - W_STATE0) >> 2);   // this lane's 32 of the 64 columns
         {
+            // start state: S0 (or zero) for a whole sequence, zero for a segment's end
+            // state, the identity's columns for a transition, S_start of the segment
             float s0[16], s1[16];
 #pragma unroll
-            for (int n = 0; n < 16; ++n)
-                s0[n] = s1[n] = 0.f;
-            if (p.S0 != nullptr) {
-                const float *src = p.S0 + (vh * KD + R) * p.dv + n0 + cs;
+            for (int n = 0; n < 16; ++n) {
+                s0[n] = (trans && R == n0 + cs + n) ? 1.f : 0.f;
+                s1[n] = (trans && R == n0 + cs + 16 + n) ? 1.f : 0.f;
+            }
+            const float *src = nullptr;
+            if (args.mode == MODE_SEQ && p.S0 != nullptr)
+                src = p.S0 + (vh * KD + R) * p.dv + n0 + cs;
+            else if (args.mode == MODE_SEG_C)
+                src = args.seg_start + (((size_t)vh * args.nseg + seg) * KD + R) * p.dv + n0 + cs;
+            if (src != nullptr) {
 #pragma unroll
                 for (int n = 0; n < 16; n += 4) {
                     const float4 a4 = *reinterpret_cast<const float4 *>(src + n);
@@ -342,11 +455,11 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
         tmem_st_wait();
         bool ok = true;
-        for (int c = 0; c < N; ++c) {
-            const int s = c & 1;
-            const uint32_t par = c & 1;
-            if (c >= 1 &&
-                named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[UPD_DONE], (c - 1) & 1, abort_flag))) {
+        for (int i = 0; i < nloc; ++i) {
+            const int s = i & 1;
+            const uint32_t par = i & 1;
+            if (i >= 1 &&
+                named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[UPD_DONE], (i - 1) & 1, abort_flag))) {
                 ok = false;
                 break;
             }
@@ -367,11 +480,14 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (stid == 0)
                 mbar_arrive(&bars[S_READY]);
             if (named_vote_or(NB_STATE, N_STATE,
-                              !wait_or_abort(&bars[FULLX0 + s], (c >> 1) & 1, abort_flag))) {
+                              !wait_or_abort(&bars[FULLX0 + s], (i >> 1) & 1, abort_flag))) {
                 ok = false;
                 break;
             }
             const Gates *gt = gates_of(s);
+            // this thread's factors of the stage, read now: group X is refilled as soon
+            // as P is done
+            const float f_eb = (scalar && R >= CC) ? gt->eb[R - CC] : 1.f;
             {
                 const float F = scalar ? gt->F[0] : gt->F[R];
 #pragma unroll
@@ -386,15 +502,23 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 ok = false;
                 break;
             }
+            if (stid == 0)   // every state thread has read its factors (the vote above)
+                mbar_arrive(&bars[FREEX0 + s]);
             tc_fence_after();
             if (R >= CC) {   // warps of lane quarters 2 and 3: rows t of P, U and E
                 const int t = R - CC;
-                const float f = scalar ? gt->eb[t] : 1.f;
+                const float f = f_eb;
                 float p0[16], p1[16], u0[16], u1[16];
                 tmem_ld16(tq + T_PO + 64 * s + cs, p0);
                 tmem_ld16(tq + T_PO + 64 * s + cs + 16, p1);
-                tmem_ld16(tq + T_U + 64 * s + cs, u0);
-                tmem_ld16(tq + T_U + 64 * s + cs + 16, u1);
+                if (trans) {
+#pragma unroll
+                    for (int n = 0; n < 16; ++n)
+                        u0[n] = u1[n] = 0.f;
+                } else {
+                    tmem_ld16(tq + T_U + 64 * s + cs, u0);
+                    tmem_ld16(tq + T_U + 64 * s + cs + 16, u1);
+                }
                 tmem_ld_wait();
 #pragma unroll
                 for (int n = 0; n < 16; ++n) {
@@ -425,12 +549,18 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mbar_arrive(&bars[E_READY]);
         }
         tmem_st_wait();   // a chunk left early may still have its F S store in flight
-        if (ok && N > 0 &&
-            named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[UPD_DONE], (N - 1) & 1, abort_flag)))
+        if (ok && nloc > 0 &&
+            named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[UPD_DONE], (nloc - 1) & 1, abort_flag)))
             ok = false;
-        if (ok && p.S_final != nullptr) {
+        // end state: S_final (whole sequence, or the last segment), Btil or Atil of a segment
+        float *dst = nullptr;
+        if (args.mode == MODE_SEG_AB)
+            dst = trans ? args.seg_trans + (((size_t)kh * args.nseg + seg) * KD + R) * KD + n0 + cs
+                        : args.seg_end + (((size_t)vh * args.nseg + seg) * KD + R) * p.dv + n0 + cs;
+        else if (p.S_final != nullptr && seg == args.nseg - 1)
+            dst = p.S_final + (vh * KD + R) * p.dv + n0 + cs;
+        if (ok && dst != nullptr) {
             tc_fence_after();
-            float *dst = p.S_final + (vh * KD + R) * p.dv + n0 + cs;
             float s0[16], s1[16];
             tmem_ld16(tq + T_S + cs, s0);
             tmem_ld16(tq + T_S + cs + 16, s1);
@@ -445,8 +575,8 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // ------------------------------------------------------------ epilogue (rows t in lanes 0-63)
         const int etid = tid - W_EPI0 * 32;
         const int t = R;
-        for (int c = 0; c < N; ++c) {
-            const int ob = c & 1;
+        for (int i = 0; i < nloc; ++i) {
+            const int c = cbeg + i, ob = i & 1;
             const long c0 = (long)c * CC;
             const int Cl = (int)min((long)CC, T - c0);
             // Qbar S = e^{Lambda_t} (Q S) for the scalar gate (factor from the record)
@@ -454,10 +584,10 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                          args.factors + (size_t)(kh * N + c) * args.rec_bytes +
                                          prep::SC_EA)[t]
                                    : 1.f;
-            if (named_vote_or(NB_EPI, N_EPI, !wait_or_abort(&bars[OUT0 + ob], (c >> 1) & 1, abort_flag)))
+            if (named_vote_or(NB_EPI, N_EPI, !wait_or_abort(&bars[OUT0 + ob], (i >> 1) & 1, abort_flag)))
                 break;
             tc_fence_after();
-            const bool live = t < Cl;
+            const bool live = outputs && t < Cl;
             const long orow = (vh * T + c0 + t) * p.dv + n0;
 #pragma unroll
             for (int cb = 0; cb < NVC; cb += 16) {
@@ -497,6 +627,60 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
 }
 
+// Start state of every segment: S_start(0) = S0 (or zero), S_start(g + 1) =
+// Atil_g S_start(g) + Btil_g, in fp32 on the CUDA cores.  One CTA per (batch, value
+// head, 16 value columns); thread (r, j0) keeps row r, columns j0..j0+7 of S.
+constexpr int CMB_COLS = 16, CMB_LDA = KD + 1;
+constexpr uint32_t CMB_SMEM = (KD * CMB_LDA + KD * CMB_COLS) * 4;
+
+__global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
+{
+    extern __shared__ float cmb[];
+    float *As = cmb, *Ss = cmb + KD * CMB_LDA;   // Atil_g (rows padded), S_start(g)
+    const Params &p = a.p;
+    const int ncg = p.dv / CMB_COLS;
+    const int cg = blockIdx.x % ncg, hv = blockIdx.x / ncg, b = blockIdx.y;
+    const long vh = (long)b * p.Hv + hv, kh = (long)b * p.Hk + hv / p.R;
+    const int tid = threadIdx.x, r = tid >> 1, j0 = (tid & 1) * 8, col = cg * CMB_COLS + j0;
+    float sv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        sv[j] = p.S0 != nullptr ? p.S0[(vh * KD + r) * p.dv + col + j] : 0.f;
+    for (int g = 0; g < a.nseg; ++g) {
+        float *st = a.seg_start + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            st[j] = sv[j];
+        if (g + 1 == a.nseg)
+            break;
+        __syncthreads();   // the previous step's readers of As and Ss are done
+        const float *At = a.seg_trans + ((size_t)kh * a.nseg + g) * KD * KD;
+        for (int u = tid; u < KD * KD / 4; u += 256) {
+            const float4 x = reinterpret_cast<const float4 *>(At)[u];
+            float *d = As + (u / (KD / 4)) * CMB_LDA + (u % (KD / 4)) * 4;
+            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            Ss[r * CMB_COLS + j0 + j] = sv[j];
+        __syncthreads();
+        const float *Bt = a.seg_end + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            acc[j] = Bt[j];
+        for (int l = 0; l < KD; ++l) {
+            const float al = As[r * CMB_LDA + l];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                acc[j] += al * Ss[l * CMB_COLS + j0 + j];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            sv[j] = acc[j];
+    }
+}
+
 inline bool supports(const Params &p)
 {
     return prep::supports(p) && p.dk == KD && p.dv % NVC == 0 && p.G <= KD && p.T >= 1;
@@ -521,8 +705,30 @@ int launch(const Params &p, const void *factors, cudaStream_t stream)
     a.rec_bytes = prep::rec_bytes(p);
     a.nvt = p.dv / NVC;
     a.nchunks = prep::nchunks(p);
-    dim3 grid(a.nvt * p.Hv, p.B);
-    kern<<<grid, NTHR, Ly.total, stream>>>(mq, mk, mv, a);
+    const SegPlan sp = seg_plan(p);
+    a.nseg = sp.nseg;
+    a.seg_len = sp.seg_len;
+    a.seg_end = a.seg_trans = a.seg_start = nullptr;
+    if (sp.nseg == 1) {
+        a.mode = MODE_SEQ;
+        kern<<<dim3(a.nvt * p.Hv, p.B, 1), NTHR, Ly.total, stream>>>(mq, mk, mv, a);
+        return cudaGetLastError() == cudaSuccess ? 0 : 6;
+    }
+    // segmented: buffers past the records (sizes as seg_bytes)
+    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+    uint8_t *w = static_cast<uint8_t *>(const_cast<void *>(factors)) + al(prep::ws_bytes(p));
+    const size_t per_v = al((size_t)p.B * p.Hv * sp.nseg * KD * p.dv * 4);
+    a.seg_end = reinterpret_cast<float *>(w);
+    a.seg_start = reinterpret_cast<float *>(w + per_v);
+    a.seg_trans = reinterpret_cast<float *>(w + 2 * per_v);
+    if (cudaFuncSetAttribute(seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)CMB_SMEM) != cudaSuccess)
+        return 6;
+    a.mode = MODE_SEG_AB;
+    kern<<<dim3(a.nvt * p.Hv + (KD / NVC) * p.Hk, p.B, sp.nseg), NTHR, Ly.total, stream>>>(mq, mk, mv, a);
+    seg_combine_kernel<<<dim3((p.dv / CMB_COLS) * p.Hv, p.B), 256, CMB_SMEM, stream>>>(a);
+    a.mode = MODE_SEG_C;
+    kern<<<dim3(a.nvt * p.Hv, p.B, sp.nseg), NTHR, Ly.total, stream>>>(mq, mk, mv, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }
 

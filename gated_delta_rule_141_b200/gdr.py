@@ -41,7 +41,8 @@ _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN}
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_chunk_fwd", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
            "gdr_chunk_fwd_static",
-           "gdr_select_kernel", "gdr_kernel_chunk", "gdr_device_status", "gdr_status_string",
+           "gdr_select_kernel", "gdr_kernel_chunk", "gdr_state_segments", "gdr_device_status",
+           "gdr_status_string",
            "gdr_version")
 
 
@@ -96,6 +97,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_select_kernel.restype = i
     lib.gdr_kernel_chunk.argtypes = [ctypes.POINTER(GdrShape), i, i, i]
     lib.gdr_kernel_chunk.restype = i
+    lib.gdr_state_segments.argtypes = [ctypes.POINTER(GdrShape), i, i, i]
+    lib.gdr_state_segments.restype = i
     lib.gdr_device_status.argtypes = [vp]
     lib.gdr_device_status.restype = i
     lib.gdr_status_string.argtypes = [i]
@@ -140,6 +143,13 @@ def kernel_chunk(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "ex
     """Chunk length the selected kernel blocks by (negative status if rejected)."""
     return int(load().gdr_kernel_chunk(ctypes.byref(shape), int(chunk), int(gate_mode),
                                        _INVERSES[inverse]))
+
+
+def state_segments(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "exact") -> int:
+    """Segments per sequence of the two-pass path's state pass (1: sequential,
+    n > 1: segment-parallel, 0: another kernel; negative status if rejected)."""
+    return int(load().gdr_state_segments(ctypes.byref(shape), int(chunk), int(gate_mode),
+                                         _INVERSES[inverse]))
 
 
 def workspace_bytes(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = "exact") -> int:

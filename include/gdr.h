@@ -132,9 +132,13 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape,
  * kernel AUTO or shape->kernel selects when given enough: 0 for the one-pass
  * kernels; for TC2, B * Hk * ceil(T / 64) records of 33296 bytes (scalar gate)
  * or 66048 bytes (grouped / per-channel gates): the chunk factors T and L plus
- * the decayed operands and decay factors the second pass reads.  The caller allocates it
- * (16-byte aligned) and passes it with its size; its contents on entry do not
- * matter.  A call
+ * the decayed operands and decay factors the second pass reads.  When the
+ * sequences are few and long enough that the state pass runs segment-parallel
+ * (each sequence cut into segments whose state maps are composed), three
+ * fp32 states per segment and head (end state, start state: dk x dv per value
+ * head; transition: dk x dk per key head) follow the records, 256-byte
+ * aligned.  The caller allocates it (16-byte aligned) and passes it with its
+ * size; its contents on entry do not matter.  A call
  * whose workspace is smaller falls back (AUTO) or fails with
  * GDR_ERR_WORKSPACE (TC2 forced).  Calls that share a workspace must not
  * overlap on the GPU. */
@@ -233,6 +237,17 @@ int gdr_select_kernel(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode
  * the chunk length and is never re-blocked. */
 int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
                      gdr_inverse_mode inverse_mode);
+
+/* Segments per sequence of the TC2 state pass for this request, when TC2 is
+ * the kernel selected given the workspace gdr_workspace_bytes asks for: 1 when
+ * the pass walks every sequence whole (one launch after the first pass); n > 1
+ * when few long sequences are each cut into n segments whose state maps
+ * S -> A S + B are formed in parallel, composed in order and applied (three
+ * launches after the first pass; an affine two-level scan of the chunk
+ * recurrence); 0 when another kernel is selected; a negative gdr_status value
+ * if the request would be rejected.  Host only, no GPU work. */
+int gdr_state_segments(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                       gdr_inverse_mode inverse_mode);
 
 /* Synchronises `stream`, then returns and clears the device status word that
  * kernels set when a bounded wait gives up (GDR_OK or GDR_ERR_TIMEOUT), or

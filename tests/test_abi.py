@@ -146,6 +146,28 @@ def test_kernel_chunk(lib):
                             gdr.GATE_SCALAR) == -gdr.ERR_SHAPE
 
 
+def test_state_segments(lib):
+    # The two-pass state pass stays sequential while the value tiles of all
+    # sequences fill the SMs, and cuts few long sequences into segments whose
+    # state maps are composed; the segment buffers then follow the records in the
+    # workspace.
+    many = gdr.make_shape(4, 4096, 16, 16, 128, 128)
+    assert gdr.state_segments(many, 64, gdr.GATE_SCALAR) == 1
+    assert gdr.workspace_bytes(many, 64, gdr.GATE_SCALAR) == 4 * 16 * 64 * gdr.TC2_SCALAR_RECORD_BYTES
+    assert gdr.state_segments(gdr.make_shape(1, 256, 1, 1, 128, 128), 64, gdr.GATE_SCALAR) == 1
+    long = gdr.make_shape(1, 65536, 16, 16, 128, 128)
+    nseg = gdr.state_segments(long, 128, gdr.GATE_CHANNEL)
+    assert 2 <= nseg <= 1024 // 16
+    recs = 16 * 1024 * gdr.TC2_EXT_RECORD_BYTES
+    # two dk x dv fp32 states per value head and a dk x dk one per key head, per segment
+    assert gdr.workspace_bytes(long, 128, gdr.GATE_CHANNEL) == recs + nseg * 16 * 3 * 128 * 128 * 4
+    # other kernels: 0; rejected requests: the negative status
+    simt = gdr.make_shape(1, 256, 2, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
+    assert gdr.state_segments(simt, 64, gdr.GATE_SCALAR) == 0
+    assert gdr.state_segments(gdr.make_shape(1, 256, 2, 3, 64, 64), 64,
+                              gdr.GATE_SCALAR) == -gdr.ERR_SHAPE
+
+
 def test_host_entry_validates(lib):
     shape = gdr.make_shape(1, 64, 2, 4, 64, 64)
     io = gdr.GdrIO()
