@@ -273,6 +273,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int i = tid; i < DK; i += NT)
             fo[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);   // F = e^{Lambda_C}
     }
+    // Scalar gate: e^{Lambda_t - Lambda_j} = e^{Lambda_t - Lambda_p} e^{Lambda_p - Lambda_j} with
+    // the pivot p in the middle of the chunk; while the chunk's decay span is within
+    // 2 kGuard both factors stay below e^{kGuard}.  The row and column factors go to
+    // the inverse's scratch (free until the inverse), read back with the Gram.
+    const bool sc_piv = SCALAR && (lam[0] - lam[CC - 1]) <= 2.f * kGuard;
+    if (!failed && sc_piv)
+        for (int t = tid; t < CC; t += NT) {
+            Tf[t] = __expf(lam[t] - lam[CC / 2]);
+            Tf[CC + t] = __expf(lam[CC / 2] - lam[t]);
+        }
     if (!failed && a.kind == REC_SCALAR) {   // per-token factors of the scalar gate
         float *ea = reinterpret_cast<float *>(img_T + SC_EA);
         float *eb = reinterpret_cast<float *>(img_T + SC_EB);
@@ -378,7 +388,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const bool keep = qrow ? (j <= t) : (j < t);
                     float v = 0.f;
                     if (keep)
-                        v = SCALAR ? d * __expf(lt - lam[j]) : d;
+                        v = !SCALAR ? d : sc_piv ? d * (Tf[t] * Tf[CC + j]) : d * __expf(lt - lam[j]);
                     if (!qrow)
                         v *= sbeta[j];
                     out[u] = v;
@@ -402,39 +412,42 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int r = 0; r < 2 && !failed; ++r) {
             const int p0 = 32 * r, pv = p0 + 16, n_r = 32 * (r + 1);
             bool clamp = false;
-            for (int u = tid; u < (64 + n_r) * (DK / 8); u += NT) {
+            // rows 0-31 of RA: q of the block, 32-63: k of the block; the q and k rows of
+            // a token share their factors
+            for (int u = tid; u < (32 + n_r) * (DK / 8); u += NT) {
                 const int row = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float v8[8], la[8], lb[8];
-                if (row < 64) {   // rows 0-31: q of the block, 32-63: k of the block
-                    const int t = p0 + (row & 31);
-                    ld_tile8(QK, 128, (row < 32 ? 0 : 64) + t, i0, v8);
-                    lam8(lam, G, wsh, t, i0, la);
-                    lam8(lam, G, wsh, pv, i0, lb);
+                float la[8], lb[8], f8[8];
+                const bool rowop = row < 32;
+                const int t = p0 + row, jj = row - 32;
+                lam8(lam, G, wsh, rowop ? t : pv, i0, la);
+                lam8(lam, G, wsh, rowop ? pv : jj, i0, lb);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float x = la[e] - lb[e];
+                    if (x > kGuard) {
+                        x = kGuard;
+                        clamp = true;
+                    }
+                    f8[e] = __expf(x);
+                }
+                if (rowop) {
+                    float q8[8], k8[8];
+                    ld_tile8(QK, 128, t, i0, q8);
+                    ld_tile8(QK, 128, 64 + t, i0, k8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        float x = la[e] - lb[e];
-                        if (x > kGuard) {
-                            x = kGuard;
-                            clamp = true;
-                        }
-                        v8[e] *= __expf(x);
+                        q8[e] *= f8[e];
+                        k8[e] *= f8[e];
                     }
-                    st_tile8(RA, 64, row, i0, v8);
+                    st_tile8(RA, 64, row, i0, q8);
+                    st_tile8(RA, 64, 32 + row, i0, k8);
                 } else {
-                    const int jj = row - 64;
-                    ld_tile8(QK, 128, 64 + jj, i0, v8);
-                    lam8(lam, G, wsh, pv, i0, la);
-                    lam8(lam, G, wsh, jj, i0, lb);
+                    float k8[8];
+                    ld_tile8(QK, 128, 64 + jj, i0, k8);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float x = la[e] - lb[e];
-                        if (x > kGuard) {
-                            x = kGuard;
-                            clamp = true;
-                        }
-                        v8[e] *= __expf(x);
-                    }
-                    st_tile8(KC, 64, jj, i0, v8);
+                    for (int e = 0; e < 8; ++e)
+                        k8[e] *= f8[e];
+                    st_tile8(KC, 64, jj, i0, k8);
                 }
             }
             if (clamp)
@@ -674,6 +687,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (w_cols)
             for (int i = tid; i < DK; i += NT)
                 Tf[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);
+        if (SCALAR && with_w) {   // e^{Lambda_j} for W's operand, once per token
+            for (int t = tid; t < CC; t += NT)
+                Tf[2 * CC + t] = __expf(lam[t]);
+            __syncthreads();
+        }
         // ---- T = diag(beta) A as a tile image: thread u writes 16-byte chunk u (coalesced).
         //      For W the same chunk goes to the bf16 operand tile in the dead q rows,
         //      scaled by e^{Lambda_j} for the scalar gate (W = T diag(e^Lambda) K).
@@ -692,7 +710,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     float e[8];
 #pragma unroll
                     for (int f = 0; f < 8; ++f)
-                        e[f] = bt * __expf(lam[8 * cc + f]);
+                        e[f] = bt * Tf[2 * CC + 8 * cc + f];
                     st_shared_v4(TB + 16 * u, pack_bf16(e[0] * x0.x, e[1] * x0.y),
                                  pack_bf16(e[2] * x0.z, e[3] * x0.w), pack_bf16(e[4] * x1.x, e[5] * x1.y),
                                  pack_bf16(e[6] * x1.z, e[7] * x1.w));

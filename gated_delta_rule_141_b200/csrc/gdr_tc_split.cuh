@@ -629,23 +629,35 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
 // Start state of every segment: S_start(0) = S0 (or zero), S_start(g + 1) =
 // Atil_g S_start(g) + Btil_g, in fp32 on the CUDA cores.  One CTA per (batch, value
-// head, 16 value columns); thread (r, j0) keeps row r, columns j0..j0+7 of S.
-constexpr int CMB_COLS = 16, CMB_LDA = KD + 1;
-constexpr uint32_t CMB_SMEM = (KD * CMB_LDA + KD * CMB_COLS) * 4;
+// head, 16 value columns); thread (r, j0) keeps row r, columns j0..j0+7 of S.  The
+// steps are sequential, so Atil_{g+1} is copied in (cp.async, second buffer) while
+// step g computes.
+constexpr int CMB_COLS = 16, CMB_LDA = KD + 4;   // rows 16-byte aligned, 2-way bank spread
+constexpr uint32_t CMB_SMEM = (2 * KD * CMB_LDA + KD * CMB_COLS) * 4;
 
 __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
 {
-    extern __shared__ float cmb[];
-    float *As = cmb, *Ss = cmb + KD * CMB_LDA;   // Atil_g (rows padded), S_start(g)
+    using namespace ptx;
+    extern __shared__ __align__(16) float cmb[];
+    float *Ss = cmb + 2 * KD * CMB_LDA;   // S_start(g), 16 columns
     const Params &p = a.p;
     const int ncg = p.dv / CMB_COLS;
     const int cg = blockIdx.x % ncg, hv = blockIdx.x / ncg, b = blockIdx.y;
     const long vh = (long)b * p.Hv + hv, kh = (long)b * p.Hk + hv / p.R;
     const int tid = threadIdx.x, r = tid >> 1, j0 = (tid & 1) * 8, col = cg * CMB_COLS + j0;
+    auto fetch = [&](int g) {   // Atil_g into buffer g % 2
+        const float *At = a.seg_trans + ((size_t)kh * a.nseg + g) * KD * KD;
+        float *As = cmb + (g & 1) * KD * CMB_LDA;
+        for (int u = tid; u < KD * KD / 4; u += 256)
+            cp_async16(smem_u32(As + (u / (KD / 4)) * CMB_LDA + (u % (KD / 4)) * 4), At + 4 * u, 16u);
+        cp_async_commit();
+    };
     float sv[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
         sv[j] = p.S0 != nullptr ? p.S0[(vh * KD + r) * p.dv + col + j] : 0.f;
+    if (a.nseg > 1)
+        fetch(0);
     for (int g = 0; g < a.nseg; ++g) {
         float *st = a.seg_start + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
 #pragma unroll
@@ -653,17 +665,15 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
             st[j] = sv[j];
         if (g + 1 == a.nseg)
             break;
-        __syncthreads();   // the previous step's readers of As and Ss are done
-        const float *At = a.seg_trans + ((size_t)kh * a.nseg + g) * KD * KD;
-        for (int u = tid; u < KD * KD / 4; u += 256) {
-            const float4 x = reinterpret_cast<const float4 *>(At)[u];
-            float *d = As + (u / (KD / 4)) * CMB_LDA + (u % (KD / 4)) * 4;
-            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
-        }
+        cp_async_wait_all();   // Atil_g has landed (this thread's share)
+        __syncthreads();       // ... everyone's; the previous step's readers are done
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             Ss[r * CMB_COLS + j0 + j] = sv[j];
         __syncthreads();
+        if (g + 2 < a.nseg)
+            fetch(g + 1);
+        const float *As = cmb + (g & 1) * KD * CMB_LDA;
         const float *Bt = a.seg_end + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
         float acc[8];
 #pragma unroll
@@ -679,6 +689,7 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
         for (int j = 0; j < 8; ++j)
             sv[j] = acc[j];
     }
+    cp_async_wait_all();
 }
 
 inline bool supports(const Params &p)
