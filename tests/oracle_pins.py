@@ -315,6 +315,30 @@ def pin_resume(seed=10):
     return worst
 
 
+# P12b: the state after a stretch of tokens is affine in the state before it,
+# S_end = A S_start + B, with A the end state from the identity when no value is
+# written (v = 0, state dk x dk) and B the end state from zero; composing two
+# stretches' maps gives the state of one pass over both (the segment-parallel
+# state pass composes such maps).
+def pin_affine_segments(seed=12):
+    rng = np.random.default_rng(seed)
+    T, T1, dk, dv = 40, 17, 8, 5
+    q, k, v, g, beta, S0 = rand_inputs(rng, 1, T, 1, 1, dk, dv, dk)
+    _, Sf = oracle.recurrent(q, k, v, g, beta, S0)
+
+    def maps(sl):
+        qs, ks, vs, gs, bs = q[:, :, sl], k[:, :, sl], v[:, :, sl], g[:, :, sl], beta[:, :, sl]
+        zero_v = np.zeros(vs.shape[:3] + (dk,))
+        _, A = oracle.recurrent(qs, ks, zero_v, gs, bs, np.eye(dk)[None, None])
+        _, Bm = oracle.recurrent(qs, ks, vs, gs, bs, None)
+        return A[0, 0], Bm[0, 0]
+
+    A1, B1 = maps(slice(0, T1))
+    A2, B2 = maps(slice(T1, T))
+    S_seg = A2 @ (A1 @ S0[0, 0] + B1) + B2
+    return _rel(S_seg, Sf[0, 0])
+
+
 # P13: the chunked Neumann mode at order >= C-1 is the exact chunked form; at
 # low order on a contractive chunk it stays close (reported, loosely bounded).
 def pin_chunked_neumann(seed=11):
@@ -338,6 +362,7 @@ ALL_PINS = {
     "gate_consistency": (pin_gate_consistency, 1e-12),
     "gva": (pin_gva, 1e-13),
     "resume": (pin_resume, 1e-12),
+    "affine_segments": (pin_affine_segments, 1e-12),
     "chunked_neumann": (pin_chunked_neumann, 1e-11),
 }
 
