@@ -9,9 +9,10 @@ The arithmetic lives in ``gdr_oracle.c`` (plain C99 + OpenMP, fp64); this file
 only marshals numpy arrays.  Citations for each routine are in the C source:
 the token recurrence follows "Systolic Linear Attention: Co-Designing
 Tile-Grouped Gated Delta Attention for TPUs" §2.1 Eq. (2); the chunkwise WY
-form follows its §2.3 Table 2 and §2.4.2; the truncated Neumann inverse follows
-"When Good Enough Is Optimal: Multiplication-Only Matrix Inversion
-Approximation for Quantized Gated DeltaNet" (Lemma 3.1, §4.1).
+form follows its §2.3 Table 2 and §2.4.2, its 1-Step Neumann block inverse
+§2.4.3; the truncated Neumann inverse follows "When Good Enough Is Optimal:
+Multiplication-Only Matrix Inversion Approximation for Quantized Gated DeltaNet"
+(Lemma 3.1, §4.1).
 
 Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
 closed forms, invariants and hand-worked examples in ``tests/golden/``.
@@ -32,6 +33,7 @@ _lib = None
 
 INV_EXACT = 0
 INV_NEUMANN = 1
+INV_NEUMANN1 = 2   # 1-Step Neumann, blocks of 16 rows
 NV_NEWTON = 0      # residual step X <- X + X (I - (I+N) X)
 NV_REFINE = 1      # residual step X <- X + X0 (I - (I+N) X)
 NV_BANDCUT = 2     # zero X0 outside the band i - j <= order
@@ -59,10 +61,12 @@ def load_library(path: str):
     lib.gdro_chunked.argtypes = [i] * 12 + [dp] * 8 + [i]
     lib.gdro_tril_inverse.argtypes = [i, dp, dp]
     lib.gdro_neumann_inverse.argtypes = [i, dp, i, i, i, dp]
+    lib.gdro_block_neumann1_inverse.argtypes = [i, dp, i, dp]
     lib.gdro_chunk_matrices.argtypes = [i, i, i] + [dp] * 7
     lib.gdro_max_threads.argtypes = []
     for f in (lib.gdro_recurrent, lib.gdro_chunked, lib.gdro_tril_inverse,
-              lib.gdro_neumann_inverse, lib.gdro_chunk_matrices, lib.gdro_max_threads):
+              lib.gdro_neumann_inverse, lib.gdro_block_neumann1_inverse,
+              lib.gdro_chunk_matrices, lib.gdro_max_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -129,12 +133,13 @@ def recurrent(q, k, v, g, beta, S0=None, nthreads=0):
 
 def chunked(q, k, v, g, beta, S0=None, chunk=64, inverse="exact", order=4, resid=1,
             variant=NV_NEWTON, nthreads=0):
-    """Chunkwise WY form in fp64 with an exact (forward substitution) or truncated
-    Neumann chunk inverse.  Returns (o, S_final)."""
+    """Chunkwise WY form in fp64 with an exact (forward substitution), truncated
+    Neumann ("neumann") or 1-Step Neumann in blocks of 16 ("neumann1") chunk
+    inverse.  Returns (o, S_final)."""
     q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
     S0 = None if S0 is None else _f64(S0)
     B, T, Hk, Hv, dk, dv, G = _dims(q, v, g)
-    mode = {"exact": INV_EXACT, "neumann": INV_NEUMANN}[inverse]
+    mode = {"exact": INV_EXACT, "neumann": INV_NEUMANN, "neumann1": INV_NEUMANN1}[inverse]
     o = np.zeros((B, Hv, T, dv), np.float64)
     Sf = np.zeros((B, Hv, dk, dv), np.float64)
     _check(_load().gdro_chunked(B, T, Hk, Hv, dk, dv, G, int(chunk), mode, int(order),
@@ -161,6 +166,17 @@ def neumann_inverse(N, order=4, resid=1, variant=NV_NEWTON):
     X = np.zeros((n, n), np.float64)
     _check(_load().gdro_neumann_inverse(n, _ptr(N), int(order), int(resid), int(variant),
                                         _ptr(X)), "gdro_neumann_inverse")
+    return X
+
+
+def block_neumann1_inverse(N, blk=16):
+    """1-Step Neumann approximation (I - Nb) D^{-1} of (I + N)^{-1}: D the
+    block-diagonal part of I + N in blocks of `blk`, Nb = D^{-1} N_off."""
+    N = _f64(N)
+    n = N.shape[0]
+    X = np.zeros((n, n), np.float64)
+    _check(_load().gdro_block_neumann1_inverse(n, _ptr(N), int(blk), _ptr(X)),
+           "gdro_block_neumann1_inverse")
     return X
 
 

@@ -41,6 +41,8 @@
  * defines its own enums). */
 #define GDRO_INV_EXACT 0
 #define GDRO_INV_NEUMANN 1
+#define GDRO_INV_NEUMANN1 2  /* [SLA] 1-Step Neumann, blocks of GDRO_BLK1 rows */
+#define GDRO_BLK1 16
 #define GDRO_NV_REFINE 1   /* residual step uses X0 instead of X_k        */
 #define GDRO_NV_BANDCUT 2  /* zero X0 outside the band i - j <= order      */
 
@@ -251,6 +253,52 @@ int gdro_neumann_inverse(int n, const double *N, int order, int resid, int varia
 }
 
 /*
+ * 1-Step Neumann of [SLA] §2.4.3 ("Block-doubling and block-Neumann
+ * factorization").  Write I + N = D (I + Nb): D is the block-diagonal part of
+ * I + N in blocks of `blk` rows (the last block may be shorter) and
+ * Nb = D^{-1} N_off, N_off the part of N below the diagonal blocks.  Nb is
+ * nilpotent, so (I + N)^{-1} = sum_s (-Nb)^s D^{-1}; the 1-Step variant keeps the
+ * terms s = 0 and 1:
+ *   X = (I - Nb) D^{-1}.
+ * D^{-1} block by block by forward substitution (gdro_tril_inverse).
+ */
+int gdro_block_neumann1_inverse(int n, const double *N, int blk, double *X)
+{
+    if (n < 0 || blk < 1)
+        return GDRO_ERR_ARG;
+    const size_t nn = (size_t)n * n;
+    double *Dinv = (double *)calloc(nn ? nn : 1, sizeof(double));
+    double *Noff = (double *)calloc(nn ? nn : 1, sizeof(double));
+    double *Nb = (double *)malloc(sizeof(double) * (nn ? nn : 1));
+    double *Bi = (double *)malloc(sizeof(double) * (size_t)blk * blk);
+    double *Bx = (double *)malloc(sizeof(double) * (size_t)blk * blk);
+    if (!Dinv || !Noff || !Nb || !Bi || !Bx) {
+        free(Dinv); free(Noff); free(Nb); free(Bi); free(Bx);
+        return GDRO_ERR_NOMEM;
+    }
+    for (int b0 = 0; b0 < n; b0 += blk) {
+        const int nb = (n - b0 < blk) ? n - b0 : blk;
+        for (int i = 0; i < nb; ++i)
+            for (int j = 0; j < nb; ++j)
+                Bi[i * nb + j] = N[(b0 + i) * n + b0 + j];
+        gdro_tril_inverse(nb, Bi, Bx);
+        for (int i = 0; i < nb; ++i)
+            for (int j = 0; j < nb; ++j)
+                Dinv[(b0 + i) * n + b0 + j] = Bx[i * nb + j];
+    }
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j)
+            if (j / blk < i / blk)
+                Noff[i * n + j] = N[i * n + j];
+    matmul_nn(n, Dinv, Noff, Nb);
+    matmul_nn(n, Nb, Dinv, X);            /* Nb D^{-1} */
+    for (size_t e = 0; e < nn; ++e)
+        X[e] = Dinv[e] - X[e];            /* (I - Nb) D^{-1} */
+    free(Dinv); free(Noff); free(Nb); free(Bi); free(Bx);
+    return 0;
+}
+
+/*
  * Chunk matrices of one chunk for one key head, [SLA] §2.2 Bottleneck 2 and
  * §2.3 Table 2 (Gram M, score L, cumulative log-decay Lambda):
  *   Lam[t][i] = sum_{s<=t} g_s(i)                       (summed, never log o exp)
@@ -316,7 +364,8 @@ int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
 {
     if (check_dims(B, T, Hk, Hv, dk, dv, G) || C <= 0)
         return GDRO_ERR_ARG;
-    if (inverse_mode != GDRO_INV_EXACT && inverse_mode != GDRO_INV_NEUMANN)
+    if (inverse_mode != GDRO_INV_EXACT && inverse_mode != GDRO_INV_NEUMANN &&
+        inverse_mode != GDRO_INV_NEUMANN1)
         return GDRO_ERR_ARG;
     if (inverse_mode == GDRO_INV_NEUMANN && (neumann_order < 0 || neumann_resid < 0))
         return GDRO_ERR_ARG;
@@ -361,7 +410,13 @@ int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
             chunk_matrices(Cl, dk, G, qc, kc, gc, bc, Lam, M, L);
             if (inverse_mode == GDRO_INV_EXACT)
                 gdro_tril_inverse(Cl, M, A);
-            else if (gdro_neumann_inverse(Cl, M, neumann_order, neumann_resid,
+            else if (inverse_mode == GDRO_INV_NEUMANN1) {
+                if (gdro_block_neumann1_inverse(Cl, M, GDRO_BLK1, A) != 0) {
+#pragma omp atomic write
+                    err = GDRO_ERR_NOMEM;
+                    break;
+                }
+            } else if (gdro_neumann_inverse(Cl, M, neumann_order, neumann_resid,
                                           neumann_variant, A) != 0) {
 #pragma omp atomic write
                 err = GDRO_ERR_NOMEM;

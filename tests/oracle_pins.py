@@ -349,6 +349,45 @@ def pin_chunked_neumann(seed=11):
     return max(_rel(o2, o1), _rel(S2, S1))
 
 
+# P13 ("Systolic Linear Attention ...", §2.4.3, block-doubling and block-Neumann
+# factorization): with 8 blocks of 16 at C = 128, Nb = D^{-1} N_off (D the
+# block-diagonal part of I + N) is nilpotent, so sum_{s<=7} (-Nb)^s equals
+# (I + Nb^4)(I + Nb^2)(I - Nb) and sum_s (-Nb)^s D^{-1} is the exact inverse.  The
+# oracle's 1-Step Neumann must be the exact inverse minus the pages' truncation
+# sum_{s=2}^{7} (-Nb)^s D^{-1}; it is exact on the diagonal blocks and the first
+# block sub-diagonal.  D^{-1}, the exact inverse and the powers come from LAPACK
+# and numpy, not from the oracle.
+def pin_block_neumann(seed=13):
+    rng = np.random.default_rng(seed)
+    n, blk = 128, 16
+    N = np.tril(rng.standard_normal((n, n)) * 0.15, -1)
+    bl = np.arange(n) // blk
+    I = np.eye(n)
+    Dinv = np.linalg.inv(I + np.where(bl[:, None] == bl[None, :], N, 0.0))
+    Nb = Dinv @ np.where(bl[:, None] > bl[None, :], N, 0.0)
+    powers = [np.linalg.matrix_power(-Nb, s) for s in range(8)]
+    exact = np.linalg.inv(I + N)
+    X1 = oracle.block_neumann1_inverse(N, blk)
+    lag = bl[:, None] - bl[None, :]
+    return max(_rel(sum(powers), (I + powers[4]) @ (I + Nb @ Nb) @ (I - Nb)),
+               _rel(sum(powers) @ Dinv, exact),
+               _rel(X1, exact - sum(powers[2:]) @ Dinv),
+               np.abs((X1 - exact)[lag <= 1]).max() / np.abs(exact).max())
+
+
+# The 1-Step Neumann chunk form is exact while a chunk holds at most two blocks
+# of 16 (no block lag above 1): at C = 32 it is the token recurrence.
+def pin_neumann1_short_chunks(seed=14):
+    rng = np.random.default_rng(seed)
+    q, k, v, g, beta, S0 = rand_inputs(rng, 1, 70, 2, 2, 8, 4, 8)
+    o, Sf = oracle.recurrent(q, k, v, g, beta, S0)
+    worst = 0.0
+    for C in (16, 32):
+        o1, S1 = oracle.chunked(q, k, v, g, beta, S0, chunk=C, inverse="neumann1")
+        worst = max(worst, _rel(o1, o), _rel(S1, Sf))
+    return worst
+
+
 ALL_PINS = {
     "golden_examples": (pin_golden_examples, 1e-12),
     "golden_inverse": (pin_golden_inverse, 1e-12),
@@ -363,6 +402,8 @@ ALL_PINS = {
     "gva": (pin_gva, 1e-13),
     "resume": (pin_resume, 1e-12),
     "affine_segments": (pin_affine_segments, 1e-12),
+    "block_neumann": (pin_block_neumann, 1e-10),
+    "neumann1_short_chunks": (pin_neumann1_short_chunks, 1e-12),
     "chunked_neumann": (pin_chunked_neumann, 1e-11),
 }
 
