@@ -53,7 +53,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=1)
     ap.add_argument("--chunk", type=int, default=0)
-    ap.add_argument("--inverse", default="exact", choices=["exact", "neumann"])
+    ap.add_argument("--inverse", default="exact", choices=["exact", "neumann", "neumann1"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -67,7 +67,15 @@ def algorithmic(w: W.Workload, chunk: int, inverse: str, order=4, resid=1):
     C, dk, Dv, G = chunk, w.dk, w.R * w.dv, w.G
     s_in = 4 if w.in_dtype == "f32" else 2
     s_out = s_in
-    inv = C * C / 3.0 if inverse == "exact" else (order - 1 + 2 * resid) * C * C / 3.0
+    if inverse == "exact":
+        inv = C * C / 3.0
+    elif inverse == "neumann1":
+        # 16 x 16 diagonal blocks (triangular solves) and two triangular-times-dense
+        # 16 x 16 products per block pair below them, per token of the chunk
+        nb = (C + 15) // 16
+        inv = (2.0 * nb * 16 ** 3 / 3.0 + nb * (nb - 1) * 16 ** 3) / C
+    else:
+        inv = (order - 1 + 2 * resid) * C * C / 3.0
     flop_tok = 3 * C * dk + 2 * C * Dv + 6 * dk * Dv + inv
     byte_tok = 2 * dk * s_in + Dv * s_in + Dv * s_out + 4 * G + 4
     units = w.B * w.Hk * w.T
@@ -212,7 +220,7 @@ def oracle_sample(w: W.Workload, x: dict, chunk: int, inverse: str, budget_s: fl
                              nthreads=threads)
         else:
             oracle.chunked(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["S0"],
-                           chunk=chunk, inverse="neumann", nthreads=threads)
+                           chunk=chunk, inverse=inverse, nthreads=threads)
         return time.perf_counter() - t0
 
     n = min(total, threads)
@@ -224,7 +232,7 @@ def oracle_sample(w: W.Workload, x: dict, chunk: int, inverse: str, budget_s: fl
         dt = run(n2)
         n = n2
     tokens = n * w.T / w.Hv            # value-head sequences -> tokens of B*T
-    kind = "recurrent" if inverse == "exact" else "chunked-neumann"
+    kind = "recurrent" if inverse == "exact" else "chunked-" + inverse
     desc = "%d of %d (batch, value-head) sequences, all %d tokens each, fp64 %s" % (
         n, total, w.T, kind)
     return tokens / dt, threads, desc, dt

@@ -44,7 +44,7 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
     case GDR_GATE_CHANNEL: G = s->dk; break;
     default: return GDR_ERR_ARG;
     }
-    if (im != GDR_INV_EXACT && im != GDR_INV_NEUMANN)
+    if (im != GDR_INV_EXACT && im != GDR_INV_NEUMANN && im != GDR_INV_NEUMANN1)
         return GDR_ERR_ARG;
     if (im == GDR_INV_NEUMANN &&
         (s->neumann_order < 0 || s->neumann_order > 256 || s->neumann_residual_steps < 0 ||
@@ -56,6 +56,7 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
     p->in_bf16 = s->in_dtype == GDR_BF16;
     p->out_bf16 = s->out_dtype == GDR_BF16;
     p->neumann = im == GDR_INV_NEUMANN;
+    p->neumann1 = im == GDR_INV_NEUMANN1;
     p->neu_order = p->neumann ? s->neumann_order : 0;
     p->neu_resid = p->neumann ? s->neumann_residual_steps : 0;
     return GDR_OK;

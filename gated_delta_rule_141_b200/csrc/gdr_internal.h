@@ -16,6 +16,7 @@ struct Params {
     int in_bf16;    // q, k, v are bf16 (else fp32)
     int out_bf16;   // o is bf16 (else fp32)
     int neumann;    // 0 exact inverse, 1 truncated Neumann
+    int neumann1;   // 1-Step Neumann in blocks of 16 (neumann is 0 then)
     int neu_order;  // Neumann order m
     int neu_resid;  // Newton residual corrections
     const void *q, *k, *v;

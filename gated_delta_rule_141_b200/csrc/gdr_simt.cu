@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
     extern __shared__ float sm[];
     const int C = p.C, G = p.G, dk = p.dk, dv = p.dv, T = p.T;
     const bool neu = p.neumann != 0;
-    const SimtLayout Ly = simt_layout(C, G, dk, neu, p.neu_resid, NV);
+    const bool blk1 = p.neumann1 != 0;   // 1-Step Neumann: X is its scratch
+    const SimtLayout Ly = simt_layout(C, G, dk, neu || blk1, p.neu_resid, NV);
     float *lam = sm + Ly.lam, *A = sm + Ly.A, *P = sm + Ly.P, *X = sm + Ly.X;
     float *S = sm + Ly.S, *rhs = sm + Ly.rhs, *qs = sm + Ly.qs, *E = sm + Ly.E;
     float *blk = sm + Ly.blk, *sbeta = sm + Ly.beta, *row = sm + Ly.row;
@@ -131,19 +132,49 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
         __syncthreads();
         // --- chunk inverse
         if (!neu) {
-            // forward substitution in place: row t of M becomes row t of A
+            // forward substitution in place: row t of M becomes row t of A.  For the
+            // 1-Step Neumann inverse only within each 16-row diagonal block (the
+            // exact D^{-1}); the blocks below keep M until the step after.
             for (int t = tid; t < Cl; t += NT)
                 A[t * C + t] = 1.f;
             __syncthreads();
             for (int t = 1; t < Cl; ++t) {
-                for (int j = tid; j < t; j += NT)
+                const int b0 = blk1 ? (t / 16) * 16 : 0;
+                for (int j = b0 + tid; j < t; j += NT)
                     row[j] = A[t * C + j];
                 __syncthreads();
-                for (int c = tid; c < t; c += NT) {
+                for (int c = b0 + tid; c < t; c += NT) {
                     float acc = -row[c];
                     for (int j = c + 1; j < t; ++j)
                         acc -= row[j] * A[j * C + c];
                     A[t * C + c] = acc;
+                }
+                __syncthreads();
+            }
+            if (blk1) {
+                // ("Systolic Linear Attention ...", §2.4.3) A = (I - D^{-1} M_off) D^{-1}:
+                // below the diagonal blocks A_ij = -D_ii^{-1} M_ij D_jj^{-1}; first
+                // X = M_off D^{-1}, then A_off = -D^{-1} X (row i reads its own diagonal
+                // block, which this step does not write)
+                for (int idx = tid; idx < Cl * Cl; idx += NT) {
+                    const int i = idx / Cl, c = idx % Cl;
+                    if (c >= (i / 16) * 16)
+                        continue;
+                    const int ce = min((c / 16) * 16 + 16, Cl);
+                    float acc = 0.f;
+                    for (int l = c; l < ce; ++l)
+                        acc += A[i * C + l] * A[l * C + c];
+                    X[i * C + c] = acc;
+                }
+                __syncthreads();
+                for (int idx = tid; idx < Cl * Cl; idx += NT) {
+                    const int i = idx / Cl, c = idx % Cl, b0 = (i / 16) * 16;
+                    if (c >= b0)
+                        continue;
+                    float acc = 0.f;
+                    for (int l = b0; l <= i; ++l)
+                        acc += A[i * C + l] * X[l * C + c];
+                    A[i * C + c] = -acc;
                 }
                 __syncthreads();
             }
@@ -339,7 +370,8 @@ constexpr int kMaxSmem = 227 * 1024;
 
 int smem_for(const Params &p, int NV)
 {
-    return simt_layout(p.C, p.G, p.dk, p.neumann != 0, p.neu_resid, NV).total * (int)sizeof(float);
+    return simt_layout(p.C, p.G, p.dk, p.neumann != 0 || p.neumann1 != 0, p.neu_resid, NV).total *
+           (int)sizeof(float);
 }
 
 template <int NV>

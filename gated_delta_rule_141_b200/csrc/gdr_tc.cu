@@ -603,7 +603,7 @@ int launch_scalar(const Params &p, cudaStream_t stream)
 static Params as_kernel_chunk(const Params &p)
 {
     Params q = p;
-    if (!p.neumann && p.C == 128)
+    if (!p.neumann && !p.neumann1 && p.C == 128)   // the exact form only
         q.C = CH;
     return q;
 }
@@ -615,7 +615,8 @@ bool tc_supports(const Params &p0)
     const Params p = as_kernel_chunk(p0);
     const bool scalar64 = p.in_bf16 && p.G == 1 && p.C == CH && p.dk == 64 && p.dv % NV == 0 &&
                           !p.neumann && p.T >= 1 && p.B <= 65535;
-    return ws::supports(p) || scalar64 || gen::supports(p);
+    // the one-pass kernels have no 1-Step Neumann inverse
+    return !p.neumann1 && (ws::supports(p) || scalar64 || gen::supports(p));
 }
 
 int launch_tc(const Params &p0, cudaStream_t stream)

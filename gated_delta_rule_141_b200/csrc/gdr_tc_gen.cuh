@@ -119,8 +119,9 @@ __device__ __forceinline__ void block_product4x4(float (&acc)[4][4], const float
     }
 }
 
-// In-place exact inverse of I + M (64 x 64, M strictly lower) by block doubling.
-__device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
+// The four diagonal 16 x 16 blocks of I + M (64 x 64, M strictly lower) replaced
+// in place by their exact inverses; the blocks below them are left as they are.
+__device__ __forceinline__ void diag16_inverse_inplace(float *Mf, float *Tf, int tid)
 {
     // diagonal 16 x 16 blocks, exact forward substitution (into Tf, then back).
     // Column cc of the block's inverse, right-looking: once x_j is final it is
@@ -149,6 +150,12 @@ __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
         Mf[(16 * blk + t) * LDM + 16 * blk + cc] = Tf[idx];
     }
     __syncthreads();
+}
+
+// In-place exact inverse of I + M (64 x 64, M strictly lower) by block doubling.
+__device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
+{
+    diag16_inverse_inplace(Mf, Tf, tid);
     // The doubling steps are products of small dense blocks.  Each thread owns a
     // 4 x 4 block of the product: per step of the inner index it loads four A
     // values (shared by the lanes of a row group) and one float4 of B, which is
@@ -190,6 +197,47 @@ __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
         for (int i = 0; i < 4; ++i)
             *reinterpret_cast<float4 *>(&Mf[(32 + rg + 8 * i) * LDM + c0]) =
                 make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
+    }
+    __syncthreads();
+}
+
+// In-place 1-Step Neumann approximation of (I + M)^{-1} ("Systolic Linear
+// Attention ...", §2.4.3): with D the block-diagonal part of I + M in 16-row
+// blocks and N = D^{-1} M_off, A = (I - N) D^{-1}, i.e. the exact inverses D_ii^{-1}
+// on the diagonal and A_ij = -D_ii^{-1} M_ij D_jj^{-1} below it (i > j).  The six
+// products T_ij = M_ij D_jj^{-1} go to the (zero) block above the diagonal at
+// (j, i) first, one 16-thread group per block (4 x 4 outputs a thread).
+__device__ __forceinline__ void block_neumann1_64_inplace(float *Mf, float *Tf, int tid)
+{
+    diag16_inverse_inplace(Mf, Tf, tid);
+    const int pi = tid >> 4;                      // block pair 0..5 for tid < 96
+    const int bi = pi < 1 ? 1 : pi < 3 ? 2 : 3;   // (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+    const int bj = pi < 1 ? 0 : pi < 3 ? pi - 1 : pi - 3;
+    const int rg = (tid & 15) >> 2, c0 = 4 * (tid & 3);
+    if (tid < 96) {
+        float acc[4][4];
+        block_product4x4<16>(acc, Mf + (16 * bi + rg) * LDM + 16 * bj, 4 * LDM,
+                             Mf + 16 * bj * LDM + 16 * bj + c0, LDM, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(&Mf[(16 * bj + rg + 4 * i) * LDM + 16 * bi + c0]) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    }
+    __syncthreads();
+    if (tid < 96) {
+        float acc[4][4];
+        block_product4x4<16>(acc, Mf + (16 * bi + rg) * LDM + 16 * bi, 4 * LDM,
+                             Mf + 16 * bj * LDM + 16 * bi + c0, LDM, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(&Mf[(16 * bi + rg + 4 * i) * LDM + 16 * bj + c0]) =
+                make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
+    }
+    __syncthreads();
+    for (int u = tid; u < 6 * 256; u += NT) {     // the scratch blocks back to zero
+        const int q = u >> 8, r = (u >> 4) & 15, c = u & 15;
+        const int qi = q < 1 ? 1 : q < 3 ? 2 : 3, qj = q < 1 ? 0 : q < 3 ? q - 1 : q - 3;
+        Mf[(16 * qj + r) * LDM + 16 * qi + c] = 0.f;
     }
     __syncthreads();
 }

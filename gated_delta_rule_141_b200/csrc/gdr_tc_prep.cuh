@@ -555,7 +555,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (!failed) {
         __syncthreads();
         if (!neu) {
-            gen::inverse64_inplace(Mf, Tf, tid);
+            if (p.neumann1)
+                gen::block_neumann1_64_inplace(Mf, Tf, tid);
+            else
+                gen::inverse64_inplace(Mf, Tf, tid);
         } else {
             // ---- truncated Neumann series (Horner) + Newton residual steps, M = 64 on tcgen05
             const uint32_t NB = base_u32 + Ly.NB, XB = base_u32 + Ly.XB, RB = base_u32 + Ly.RB;

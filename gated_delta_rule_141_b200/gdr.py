@@ -24,7 +24,7 @@ F32, BF16 = 0, 1
 # gdr_gate_mode
 GATE_SCALAR, GATE_GROUP64, GATE_CHANNEL = 0, 1, 2
 # gdr_inverse_mode
-INV_EXACT, INV_NEUMANN = 0, 1
+INV_EXACT, INV_NEUMANN, INV_NEUMANN1 = 0, 1, 2
 # gdr_kernel
 KERNEL_AUTO, KERNEL_SIMT, KERNEL_TC, KERNEL_TC2 = 0, 1, 2, 3
 
@@ -36,7 +36,7 @@ PREP_CHUNK_BYTES = 16384
 # bytes of one workspace record of the two-pass kernel: scalar gate, grouped / per-channel gates
 TC2_SCALAR_RECORD_BYTES = 33296
 TC2_EXT_RECORD_BYTES = 66048
-_INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN}
+_INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN, "neumann1": INV_NEUMANN1}
 
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_chunk_fwd", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",

@@ -64,11 +64,15 @@ typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
 typedef enum { GDR_GATE_SCALAR = 0, GDR_GATE_GROUP64 = 1, GDR_GATE_CHANNEL = 2 } gdr_gate_mode;
 
 /* Chunk inverse A_c = (I + M_c)^{-1}:
- *  EXACT   block-doubling inverse, exact up to rounding (SLA §2.4.3)
- *  NEUMANN sum_{p<=order} (-M)^p with masking, then `neumann_residual_steps`
- *          Newton residual corrections X <- X + X (I - (I + M) X)
- *          (Multiplication-Only Matrix Inversion ..., Lemma 3.1, §4.1)      */
-typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1 } gdr_inverse_mode;
+ *  EXACT    block-doubling inverse, exact up to rounding (SLA §2.4.3)
+ *  NEUMANN  sum_{p<=order} (-M)^p with masking, then `neumann_residual_steps`
+ *           Newton residual corrections X <- X + X (I - (I + M) X)
+ *           (Multiplication-Only Matrix Inversion ..., Lemma 3.1, §4.1)
+ *  NEUMANN1 1-Step Neumann (SLA §2.4.3): with D the block-diagonal part of
+ *           I + M in blocks of 16 rows and N = D^{-1} M_off, A = (I - N) D^{-1}
+ *           (exact on the diagonal blocks and the first block below them);
+ *           depends on the chunk length, which is never re-blocked          */
+typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1, GDR_INV_NEUMANN1 = 2 } gdr_inverse_mode;
 
 /* Kernel selection.
  *  TC    one fused tensor-core kernel per (batch, value head, 64 value

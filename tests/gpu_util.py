@@ -70,11 +70,12 @@ def slice_sequences(inputs: dict, R: int, seqs):
 
 def oracle_reference(inputs: dict, chunk: int, inverse: str, order: int = 4, resid: int = 1):
     """The oracle's answer: the token recurrence for the exact mode (the
-    definition), the chunked Neumann form for the Neumann mode."""
+    definition), the chunked form with the same approximate inverse otherwise
+    ("neumann": truncated Neumann; "neumann1": 1-Step Neumann in blocks of 16)."""
     args = (inputs["q"], inputs["k"], inputs["v"], inputs["g"], inputs["beta"], inputs["S0"])
     if inverse == "exact":
         return oracle.recurrent(*args)
-    return oracle.chunked(*args, chunk=chunk, inverse="neumann", order=order, resid=resid)
+    return oracle.chunked(*args, chunk=chunk, inverse=inverse, order=order, resid=resid)
 
 
 def sample_sequences(w: W.Workload, count: int = 3):

@@ -146,6 +146,23 @@ def test_kernel_chunk(lib):
                             gdr.GATE_SCALAR) == -gdr.ERR_SHAPE
 
 
+def test_neumann1_selection(lib):
+    # 1-Step Neumann depends on the chunk length (blocks of 16 in a chunk), so it is
+    # never re-blocked: chunk 64 runs the two-pass path, chunk 128 the CUDA-core
+    # kernel; the fused one-pass kernels do not implement it.
+    kda = gdr.make_shape(2, 8192, 32, 32, 128, 128)
+    assert gdr.select_kernel(kda, 64, gdr.GATE_CHANNEL, "neumann1") == gdr.KERNEL_TC2
+    assert gdr.kernel_chunk(kda, 64, gdr.GATE_CHANNEL, "neumann1") == 64
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann1") == gdr.KERNEL_SIMT
+    assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL, "neumann1") == 128
+    forced = gdr.make_shape(1, 256, 2, 2, 128, 128, kernel="tc")
+    assert gdr.select_kernel(forced, 64, gdr.GATE_SCALAR, "neumann1") == -gdr.ERR_UNSUPPORTED
+    sla = gdr.make_shape(2, 8192, 8, 32, 256, 128)      # dk = 256: no two-pass path
+    assert gdr.select_kernel(sla, 64, gdr.GATE_GROUP64, "neumann1") == gdr.KERNEL_SIMT
+    sh = gdr.make_shape(1, 64, 1, 1, 128, 128)
+    assert lib.gdr_kernel_chunk(ctypes.byref(sh), 64, 0, 3) == -gdr.ERR_ARG   # no mode 3
+
+
 def test_state_segments(lib):
     # The two-pass state pass stays sequential while the value tiles of all
     # sequences fill the SMs, and cuts few long sequences into segments whose

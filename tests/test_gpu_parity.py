@@ -63,6 +63,13 @@ SMALL = [
     (2, dict(B=1, Hk=2, Hv=2, T=256), 64, "neumann", "tc2"),
     (4, dict(Hk=2, Hv=2, T=640 - 5), 128, "exact", "tc2"),               # strong decay, S0
     (4, dict(Hk=1, Hv=1, T=64), 64, "exact", "tc2"),                     # a single chunk
+    # 1-Step Neumann inverse (blocks of 16): two-pass path at chunk 64, CUDA-core
+    # kernel at chunk 128 (eight blocks, as in the pages)
+    (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 64, "neumann1", "tc2"),
+    (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 64, "neumann1", "tc2"),
+    (4, dict(Hk=1, Hv=1, T=384), 64, "neumann1", "tc2"),                # pivoted blocks
+    (0, {}, 128, "neumann1", "auto"),                                   # fp32
+    (4, dict(Hk=1, Hv=1, T=300), 128, "neumann1", "auto"),
 ]
 
 
