@@ -62,10 +62,12 @@ def load_library(path: str):
     lib.gdro_tril_inverse.argtypes = [i, dp, dp]
     lib.gdro_neumann_inverse.argtypes = [i, dp, i, i, i, dp]
     lib.gdro_block_neumann1_inverse.argtypes = [i, dp, i, dp]
+    lib.gdro_output_gate_rmsnorm.argtypes = [i, i, dp, dp, dp, ctypes.c_double, dp]
     lib.gdro_chunk_matrices.argtypes = [i, i, i] + [dp] * 7
     lib.gdro_max_threads.argtypes = []
     for f in (lib.gdro_recurrent, lib.gdro_chunked, lib.gdro_tril_inverse,
               lib.gdro_neumann_inverse, lib.gdro_block_neumann1_inverse,
+              lib.gdro_output_gate_rmsnorm,
               lib.gdro_chunk_matrices, lib.gdro_max_threads):
         f.restype = ctypes.c_int
     return lib
@@ -178,6 +180,19 @@ def block_neumann1_inverse(N, blk=16):
     _check(_load().gdro_block_neumann1_inverse(n, _ptr(N), int(blk), _ptr(X)),
            "gdro_block_neumann1_inverse")
     return X
+
+
+def output_gate_rmsnorm(o, z, w=None, eps=1e-6):
+    """sigmoid(z) * RMSNorm(o) over the last axis (dv) of o and z, with weight w [dv]
+    (ones when None): the readout epilogue of the SLA recurrence."""
+    o, z = _f64(o), _f64(z)
+    dv = o.shape[-1]
+    rows = o.size // dv if dv else 0
+    out = np.zeros(o.shape, np.float64)
+    wv = None if w is None else _f64(w)
+    _check(_load().gdro_output_gate_rmsnorm(int(rows), int(dv), _ptr(o), _ptr(z), _ptr(wv),
+                                            float(eps), _ptr(out)), "gdro_output_gate_rmsnorm")
+    return out
 
 
 def chunk_matrices(qc, kc, gc, bc):

@@ -477,3 +477,28 @@ int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
     }
     return err;
 }
+
+/*
+ * Output gate and per-value-head RMSNorm of the readout, [SLA] §2.3 Eq. (5):
+ *   out_t = sigmoid(z_t) * RMSNorm(o_t),  RMSNorm(x) = x / sqrt(mean_i x_i^2 + eps) * w
+ * over the dv channels of one (token, value head) row.  o, z, out: [rows][dv];
+ * w: [dv] per-channel weight, or NULL for ones.  out may alias o.
+ */
+int gdro_output_gate_rmsnorm(int rows, int dv, const double *o, const double *z, const double *w,
+                             double eps, double *out)
+{
+    if (rows < 0 || dv < 1 || eps < 0.0)
+        return GDRO_ERR_ARG;
+    for (int r = 0; r < rows; ++r) {
+        const double *x = o + (size_t)r * dv;
+        double ss = 0.0;
+        for (int i = 0; i < dv; ++i)
+            ss += x[i] * x[i];
+        const double inv = 1.0 / sqrt(ss / dv + eps);
+        for (int i = 0; i < dv; ++i) {
+            const double gate = 1.0 / (1.0 + exp(-z[(size_t)r * dv + i]));
+            out[(size_t)r * dv + i] = gate * x[i] * inv * (w ? w[i] : 1.0);
+        }
+    }
+    return 0;
+}

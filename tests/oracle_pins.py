@@ -388,6 +388,25 @@ def pin_neumann1_short_chunks(seed=14):
     return worst
 
 
+# Readout epilogue ("Systolic Linear Attention ...", §2.3 Eq. (5): output gate
+# times per-value-head RMSNorm): a hand-worked row, unit mean square with the
+# gate open (z large), eps = 0 and unit weight, invariance to a positive scale of
+# o, and the weight applied channel by channel.
+def pin_output_epilogue(seed=15):
+    # o = (3, 4): mean square 12.5; z = 0 gates by 1/2
+    out = oracle.output_gate_rmsnorm(np.array([[3.0, 4.0]]), np.zeros((1, 2)), eps=0.0)
+    worst = _rel(out, np.array([[1.5, 2.0]]) / np.sqrt(12.5))
+    rng = np.random.default_rng(seed)
+    o, z = rng.standard_normal((5, 7, 16)), rng.standard_normal((5, 7, 16))
+    w = rng.standard_normal(16)
+    opened = oracle.output_gate_rmsnorm(o, np.full_like(o, 60.0), eps=0.0)
+    worst = max(worst, np.abs(np.mean(opened ** 2, axis=-1) - 1.0).max())
+    a = oracle.output_gate_rmsnorm(o, z, w, eps=0.0)
+    worst = max(worst, _rel(a, oracle.output_gate_rmsnorm(3.7 * o, z, w, eps=0.0)))
+    worst = max(worst, _rel(a, oracle.output_gate_rmsnorm(o, z, None, eps=0.0) * w))
+    return worst
+
+
 ALL_PINS = {
     "golden_examples": (pin_golden_examples, 1e-12),
     "golden_inverse": (pin_golden_inverse, 1e-12),
@@ -404,6 +423,7 @@ ALL_PINS = {
     "affine_segments": (pin_affine_segments, 1e-12),
     "block_neumann": (pin_block_neumann, 1e-10),
     "neumann1_short_chunks": (pin_neumann1_short_chunks, 1e-12),
+    "output_epilogue": (pin_output_epilogue, 1e-13),
     "chunked_neumann": (pin_chunked_neumann, 1e-11),
 }
 
