@@ -58,6 +58,9 @@ def parse_args():
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--epilogue", action="store_true",
+                    help="add the readout epilogue (output gate times per-value-head RMSNorm, "
+                         "unit weight) to every step, device-timed and end to end")
     return ap.parse_args()
 
 
@@ -319,6 +322,11 @@ def main():
     # the two-pass path: pass 1, then one state pass, or three when segmented
     nseg = gdr.state_segments(shape_run, chunk, gm_run, args.inverse) if kern == gdr.KERNEL_TC2 else 0
     launches_per_step = (1 + (1 if nseg == 1 else 3)) if kern == gdr.KERNEL_TC2 else 1
+    zgate = None
+    if args.epilogue:   # output-gate logits z ~ N(0, 1), seeded apart from the workload's draws
+        zr = np.random.default_rng(7000 + args.workload).standard_normal(tuple(o.shape)).astype(np.float32)
+        zgate = torch.from_numpy(zr).cuda().to(o.dtype)
+        launches_per_step += 1
     # with an L2 flush between steps, only the launches themselves are timed
     step_events = []
 
@@ -331,6 +339,8 @@ def main():
         gdr.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
                       chunk=chunk, inverse=args.inverse, o=o, S_final=Sf, kernel=args.kernel,
                       workspace=workspace, stream=stream)
+        if zgate is not None:
+            gdr.output_gate_rmsnorm(o, zgate, None, eps=1e-6, stream=stream)
         if timed and flush is not None:
             e1.record(stream)
             step_events.append((e0, e1))
@@ -366,6 +376,8 @@ def main():
     # kernel-only launch time, for the roofline (no L2 flush between launches
     # when the inputs exceed L2 anyway)
     flop, byts = algorithmic(w, chunk, args.inverse)
+    if args.epilogue:   # the epilogue reads o and z and writes o once more
+        byts += 3 * o.numel() * o.element_size()
     peaks, peak_src = measured_peaks()
     hbm_frac = (byts / (ms_step * 1e-3)) / (peaks["hbm_gbs"] * 1e9)
     tc_frac = (flop / (ms_step * 1e-3)) / (peaks["bf16_tflops"] * 1e12)
@@ -398,12 +410,33 @@ def main():
                   if t is not None and n not in ("o", "S_final"))
         d2h = host["o"].numel() * host["o"].element_size() + host["S_final"].numel() * 4
         e2e_steps = max(3, min(args.steps, 20))
+        if zgate is not None:
+            host["z"], dbuf["z"] = zgate.cpu().pin_memory(), torch.empty_like(zgate)
+            h2d += host["z"].numel() * host["z"].element_size()
+
+        def e2e_step():
+            if zgate is None:
+                gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, workspace, stream)
+                return
+            # with the epilogue: the same copies around the device entry points
+            with torch.cuda.stream(stream):
+                for n in dev:
+                    if host[n] is not None:
+                        dbuf[n].copy_(host[n], non_blocking=True)
+                dbuf["z"].copy_(host["z"], non_blocking=True)
+                gdr.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["S0"],
+                              chunk=chunk, inverse=args.inverse, o=dbuf["o"], S_final=dbuf["S_final"],
+                              kernel=args.kernel, workspace=workspace, stream=stream)
+                gdr.output_gate_rmsnorm(dbuf["o"], dbuf["z"], None, eps=1e-6, stream=stream)
+                host["o"].copy_(dbuf["o"], non_blocking=True)
+                host["S_final"].copy_(dbuf["S_final"], non_blocking=True)
+
         for _ in range(2):
-            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, workspace, stream)
+            e2e_step()
         barrier()
         ev0.record(stream)
         for _ in range(e2e_steps):
-            gdr.chunk_fwd_host(host, dbuf, shape, chunk, gm, args.inverse, workspace, stream)
+            e2e_step()
         ev1.record(stream)
         barrier()
         ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), dist, torch.device("cuda", local))
@@ -428,7 +461,7 @@ def main():
         "dtype": "bf16" if w.in_dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
         "config": dict(config_dict(w, chunk, args.inverse, world), kernel_chunk=kchunk,
-                       state_segments=nseg),
+                       state_segments=nseg, epilogue=bool(args.epilogue)),
         "tflops": roof["tflops"], "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step, "kernel": gdr.KERNEL_NAMES.get(kern, str(kern)),
         "clocks": sampler.summary(),

@@ -41,6 +41,7 @@ _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN, "neumann1": INV_NEUMANN
 # Every symbol include/gdr.h declares.
 EXPORTS = ("gdr_chunk_fwd", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
            "gdr_chunk_fwd_static",
+           "gdr_output_gate_rmsnorm",
            "gdr_select_kernel", "gdr_kernel_chunk", "gdr_state_segments", "gdr_device_status",
            "gdr_status_string",
            "gdr_version")
@@ -99,6 +100,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_kernel_chunk.restype = i
     lib.gdr_state_segments.argtypes = [ctypes.POINTER(GdrShape), i, i, i]
     lib.gdr_state_segments.restype = i
+    lib.gdr_output_gate_rmsnorm.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, ctypes.c_float, vp]
+    lib.gdr_output_gate_rmsnorm.restype = i
     lib.gdr_device_status.argtypes = [vp]
     lib.gdr_device_status.restype = i
     lib.gdr_status_string.argtypes = [i]
@@ -226,6 +229,24 @@ def chunk_fwd(q, k, v, g, beta, S0=None, chunk=64, gate_mode=None, inverse="exac
     if st != OK:
         raise GdrError(st)
     return o, S_final
+
+
+def output_gate_rmsnorm(o, z, weight=None, eps=1e-6, stream=None):
+    """In place: o <- sigmoid(z) * RMSNorm(o) * weight over the last axis of o
+    [B, Hv, T, dv] (the readout epilogue); z like o, weight [dv] fp32 or None."""
+    B, Hv, T, dv = o.shape
+    if tuple(z.shape) != tuple(o.shape) or z.dtype != o.dtype:
+        raise ValueError("z must match o in shape and dtype")
+    if not (o.is_contiguous() and z.is_contiguous()):
+        raise ValueError("o and z must be contiguous")
+    if weight is not None and (tuple(weight.shape) != (dv,) or not weight.is_contiguous()):
+        raise ValueError("weight must be a contiguous [dv] fp32 tensor")
+    shape = make_shape(B, T, 1, Hv, 1, dv, out_dtype=_dtype_code(o.dtype))
+    st = load().gdr_output_gate_rmsnorm(ctypes.byref(shape), _ptr(o), _ptr(z), _ptr(weight),
+                                        float(eps), _stream_handle(stream))
+    if st != OK:
+        raise GdrError(st, "gdr_output_gate_rmsnorm")
+    return o
 
 
 def chunk_prepare(q, k, g, beta, chunk=64, gate_mode=None, inverse="exact", neumann_order=4,

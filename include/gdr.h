@@ -253,6 +253,23 @@ int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
 int gdr_state_segments(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
                        gdr_inverse_mode inverse_mode);
 
+/*
+ * gdr_output_gate_rmsnorm -- the readout epilogue of the SLA recurrence (SLA
+ * §2.3 Eq. (5)), in place on the output of gdr_chunk_fwd:
+ *   o_{t,m} <- sigmoid(z_{t,m}) * o_{t,m} / sqrt(mean_i o_{t,m,i}^2 + eps) * weight
+ * for every (batch, value head m, token t) row of dv channels.
+ *   o      [B, Hv, T, dv] out_dtype, device, read and written
+ *   z      [B, Hv, T, dv] out_dtype output-gate logits, device, read only
+ *   weight [dv] fp32 per-channel RMSNorm weight shared by the value heads, or
+ *          NULL for ones; device, read only
+ *   eps    >= 0 (1e-6 is usual)
+ * Uses B, T, Hv, dv and out_dtype of `shape` (dv <= 256).  Statistics in fp32.
+ * Asynchronous on `stream`; validation happens before any launch (GDR_ERR_ARG
+ * for NULL o or z or a bad eps, GDR_ERR_SHAPE, GDR_ERR_DTYPE).
+ */
+gdr_status gdr_output_gate_rmsnorm(const gdr_shape *shape, void *o, const void *z,
+                                   const float *weight, float eps, void *stream);
+
 /* Synchronises `stream`, then returns and clears the device status word that
  * kernels set when a bounded wait gives up (GDR_OK or GDR_ERR_TIMEOUT), or
  * GDR_ERR_CUDA if the stream reported an error. */

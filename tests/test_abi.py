@@ -163,6 +163,19 @@ def test_neumann1_selection(lib):
     assert lib.gdr_kernel_chunk(ctypes.byref(sh), 64, 0, 3) == -gdr.ERR_ARG   # no mode 3
 
 
+def test_output_epilogue_validates(lib):
+    # validation happens before any launch (no GPU needed for these)
+    f = gdr.load().gdr_output_gate_rmsnorm
+    big = gdr.make_shape(1, 4, 1, 1, 1, 300)                 # dv > 256
+    assert f(ctypes.byref(big), None, None, None, ctypes.c_float(1e-6), None) == gdr.ERR_SHAPE
+    empty = gdr.make_shape(1, 0, 1, 1, 1, 128)               # nothing to do
+    assert f(ctypes.byref(empty), None, None, None, ctypes.c_float(1e-6), None) == gdr.OK
+    sh = gdr.make_shape(1, 4, 1, 1, 1, 128)
+    assert f(ctypes.byref(sh), None, None, None, ctypes.c_float(-1.0), None) == gdr.ERR_ARG
+    assert f(ctypes.byref(sh), None, None, None, ctypes.c_float(1e-6), None) == gdr.ERR_ARG
+    assert f(None, None, None, None, ctypes.c_float(1e-6), None) == gdr.ERR_ARG
+
+
 def test_state_segments(lib):
     # The two-pass state pass stays sequential while the value tiles of all
     # sequences fill the SMs, and cuts few long sequences into segments whose
