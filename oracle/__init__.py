@@ -59,13 +59,15 @@ def load_library(path: str):
     i = ctypes.c_int
     lib.gdro_recurrent.argtypes = [i] * 7 + [dp] * 8 + [i]
     lib.gdro_chunked.argtypes = [i] * 12 + [dp] * 8 + [i]
+    lib.gdro_chunked_momentum.argtypes = ([i] * 12 + [ctypes.c_double, ctypes.POINTER(i)]
+                                          + [dp] * 8 + [i])
     lib.gdro_tril_inverse.argtypes = [i, dp, dp]
     lib.gdro_neumann_inverse.argtypes = [i, dp, i, i, i, dp]
     lib.gdro_block_neumann1_inverse.argtypes = [i, dp, i, dp]
     lib.gdro_output_gate_rmsnorm.argtypes = [i, i, dp, dp, dp, ctypes.c_double, dp]
     lib.gdro_chunk_matrices.argtypes = [i, i, i] + [dp] * 7
     lib.gdro_max_threads.argtypes = []
-    for f in (lib.gdro_recurrent, lib.gdro_chunked, lib.gdro_tril_inverse,
+    for f in (lib.gdro_recurrent, lib.gdro_chunked, lib.gdro_chunked_momentum, lib.gdro_tril_inverse,
               lib.gdro_neumann_inverse, lib.gdro_block_neumann1_inverse,
               lib.gdro_output_gate_rmsnorm,
               lib.gdro_chunk_matrices, lib.gdro_max_threads):
@@ -134,20 +136,35 @@ def recurrent(q, k, v, g, beta, S0=None, nthreads=0):
 
 
 def chunked(q, k, v, g, beta, S0=None, chunk=64, inverse="exact", order=4, resid=1,
-            variant=NV_NEWTON, nthreads=0):
+            variant=NV_NEWTON, nthreads=0, mu=None, kappa=None):
     """Chunkwise WY form in fp64 with an exact (forward substitution), truncated
     Neumann ("neumann") or 1-Step Neumann in blocks of 16 ("neumann1") chunk
-    inverse.  Returns (o, S_final)."""
+    inverse.  With `mu` (and optionally `kappa`, [B, ceil(T/chunk)] reset
+    indicators in {0, 1}) the state carries chunk-boundary momentum.  Returns
+    (o, S_final)."""
     q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
     S0 = None if S0 is None else _f64(S0)
     B, T, Hk, Hv, dk, dv, G = _dims(q, v, g)
     mode = {"exact": INV_EXACT, "neumann": INV_NEUMANN, "neumann1": INV_NEUMANN1}[inverse]
     o = np.zeros((B, Hv, T, dv), np.float64)
     Sf = np.zeros((B, Hv, dk, dv), np.float64)
-    _check(_load().gdro_chunked(B, T, Hk, Hv, dk, dv, G, int(chunk), mode, int(order),
-                                int(resid), int(variant), _ptr(q), _ptr(k), _ptr(v),
-                                _ptr(g), _ptr(beta), _ptr(S0), _ptr(o), _ptr(Sf),
-                                int(nthreads)), "gdro_chunked")
+    if mu is None and kappa is None:
+        _check(_load().gdro_chunked(B, T, Hk, Hv, dk, dv, G, int(chunk), mode, int(order),
+                                    int(resid), int(variant), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(g), _ptr(beta), _ptr(S0), _ptr(o), _ptr(Sf),
+                                    int(nthreads)), "gdro_chunked")
+        return o, Sf
+    kp = None
+    if kappa is not None:
+        kappa = np.ascontiguousarray(kappa, dtype=np.int32)
+        if kappa.shape != (B, (T + int(chunk) - 1) // int(chunk)):
+            raise ValueError("kappa must be [B, ceil(T / chunk)]")
+        kp = kappa.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    _check(_load().gdro_chunked_momentum(B, T, Hk, Hv, dk, dv, G, int(chunk), mode, int(order),
+                                         int(resid), int(variant), float(mu or 0.0), kp,
+                                         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(S0), _ptr(o), _ptr(Sf), int(nthreads)),
+           "gdro_chunked_momentum")
     return o, Sf
 
 

@@ -356,11 +356,12 @@ int gdro_chunk_matrices(int Cl, int dk, int G, const double *qc, const double *k
  * Processed per value head (one S of dk x dv), so the packed grouped-value
  * form is reached by running the R value heads of a key head separately.
  */
-int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
-                 int inverse_mode, int neumann_order, int neumann_resid,
-                 int neumann_variant, const double *q, const double *k,
-                 const double *v, const double *g, const double *beta,
-                 const double *S0, double *o, double *S_final, int nthreads)
+static int chunked_impl(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
+                        int inverse_mode, int neumann_order, int neumann_resid,
+                        int neumann_variant, int momentum, double mu, const int *kappa,
+                        const double *q, const double *k, const double *v, const double *g,
+                        const double *beta, const double *S0, double *o, double *S_final,
+                        int nthreads)
 {
     if (check_dims(B, T, Hk, Hv, dk, dv, G) || C <= 0)
         return GDRO_ERR_ARG;
@@ -389,9 +390,13 @@ int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
         double *Qb = (double *)malloc(sizeof(double) * (size_t)C * dk);
         double *Kh = (double *)malloc(sizeof(double) * (size_t)C * dk);
         double *F = (double *)malloc(sizeof(double) * (size_t)dk);
-        if (!S || !Lam || !M || !L || !A || !RHS || !E || !Kb || !Qb || !Kh || !F) {
+        /* momentum: the chunk-entry state and the velocity buffer Z (zero at the start) */
+        double *Sp = momentum ? (double *)malloc(sizeof(double) * (size_t)dk * dv) : NULL;
+        double *Z = momentum ? (double *)calloc((size_t)dk * dv, sizeof(double)) : NULL;
+        if (!S || !Lam || !M || !L || !A || !RHS || !E || !Kb || !Qb || !Kh || !F ||
+            (momentum && (!Sp || !Z))) {
             free(S); free(Lam); free(M); free(L); free(A); free(RHS); free(E);
-            free(Kb); free(Qb); free(Kh); free(F);
+            free(Kb); free(Qb); free(Kh); free(F); free(Sp); free(Z);
 #pragma omp atomic write
             err = GDRO_ERR_NOMEM;
             continue;
@@ -461,6 +466,8 @@ int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
                     ot[n] = acc;
                 }
             }
+            if (momentum)
+                memcpy(Sp, S, sizeof(double) * (size_t)dk * dv);
             /* S <- F S + Kh^T E */
             for (int i = 0; i < dk; ++i)
                 for (int n = 0; n < dv; ++n) {
@@ -469,13 +476,58 @@ int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
                         acc += Kh[t * dk + i] * E[t * dv + n];
                     S[i * dv + n] = acc;
                 }
+            if (momentum) {
+                /* chunk-boundary momentum ([SLA] §2.3): with S the chunk update just
+                 * formed (S~_c) and Sp the chunk-entry state S_{c-1},
+                 *   Z_c = mu kappa_c Z_{c-1} + (S~_c - F_c S_{c-1}),  S_c = F_c S_{c-1} + Z_c */
+                const long nch = (T + C - 1) / C;
+                const double mk = mu * (kappa ? (double)kappa[b * nch + c0 / C] : 1.0);
+                for (int i = 0; i < dk; ++i)
+                    for (int n = 0; n < dv; ++n) {
+                        const double fs = F[i] * Sp[i * dv + n];
+                        Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] - fs);
+                        S[i * dv + n] = fs + Z[i * dv + n];
+                    }
+            }
         }
         if (S_final)
             memcpy(S_final + s * (long)dk * dv, S, sizeof(double) * (size_t)dk * dv);
         free(S); free(Lam); free(M); free(L); free(A); free(RHS); free(E);
-        free(Kb); free(Qb); free(Kh); free(F);
+        free(Kb); free(Qb); free(Kh); free(F); free(Sp); free(Z);
     }
     return err;
+}
+
+int gdro_chunked(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
+                 int inverse_mode, int neumann_order, int neumann_resid,
+                 int neumann_variant, const double *q, const double *k,
+                 const double *v, const double *g, const double *beta,
+                 const double *S0, double *o, double *S_final, int nthreads)
+{
+    return chunked_impl(B, T, Hk, Hv, dk, dv, G, C, inverse_mode, neumann_order, neumann_resid,
+                        neumann_variant, 0, 0.0, NULL, q, k, v, g, beta, S0, o, S_final,
+                        nthreads);
+}
+
+/*
+ * The chunked form with chunk-boundary momentum ([SLA] §2.3, the momentum
+ * equation after Eq. (5), and §2.3's notation table): every chunk's state update
+ * S~_c (the chunked form above, from S_{c-1}) is blended with a velocity buffer,
+ *   Z_c = mu kappa_c Z_{c-1} + (S~_c - F_c S_{c-1}),  S_c = F_c S_{c-1} + Z_c,
+ * Z_0 = 0.  kappa: [B][ceil(T / C)] reset indicators (0 where a document reset
+ * falls inside the chunk), or NULL for ones.  The outputs of chunk c come from
+ * the chunk computation started at S_{c-1}, as without momentum.
+ */
+int gdro_chunked_momentum(int B, int T, int Hk, int Hv, int dk, int dv, int G, int C,
+                          int inverse_mode, int neumann_order, int neumann_resid,
+                          int neumann_variant, double mu, const int *kappa, const double *q,
+                          const double *k, const double *v, const double *g,
+                          const double *beta, const double *S0, double *o, double *S_final,
+                          int nthreads)
+{
+    return chunked_impl(B, T, Hk, Hv, dk, dv, G, C, inverse_mode, neumann_order, neumann_resid,
+                        neumann_variant, 1, mu, kappa, q, k, v, g, beta, S0, o, S_final,
+                        nthreads);
 }
 
 /*

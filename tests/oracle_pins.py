@@ -407,6 +407,44 @@ def pin_output_epilogue(seed=15):
     return worst
 
 
+# Chunk-boundary momentum ("Systolic Linear Attention ...", §2.3): with mu = 0,
+# or with every reset indicator kappa_c = 0, the momentum form is the plain
+# chunked form.
+def pin_momentum_reduces(seed=16):
+    rng = np.random.default_rng(seed)
+    q, k, v, g, beta, S0 = rand_inputs(rng, 2, 50, 2, 4, 8, 3, 8)
+    o, Sf = oracle.chunked(q, k, v, g, beta, S0, chunk=8)
+    worst = 0.0
+    for kw in (dict(mu=0.0), dict(mu=0.25, kappa=np.zeros((2, 7), np.int32))):
+        om, Sm = oracle.chunked(q, k, v, g, beta, S0, chunk=8, **kw)
+        worst = max(worst, _rel(om, o), _rel(Sm, Sf))
+    return worst
+
+
+# The same momentum written as the pages' joint affine step of (S, Z) (§3.3,
+# context parallelism): [S_c; Z_c] = [[J_c, mu kappa_c I], [J_c - F_c, mu kappa_c I]]
+# [S_{c-1}; Z_{c-1}] + [B_c; B_c], with J_c the chunk's state map from the
+# identity with no values, B_c its map from zero (both from plain chunked runs of
+# that chunk alone) and F_c = diag(exp(sum of its log-decays)).
+def pin_momentum_block_form(seed=17):
+    rng = np.random.default_rng(seed)
+    T, C, dk, dv, mu = 40, 8, 6, 3, 0.25
+    q, k, v, g, beta, S0 = rand_inputs(rng, 1, T, 1, 1, dk, dv, dk)
+    kappa = np.array([[1, 1, 0, 1, 1]], np.int32)
+    _, Sm = oracle.chunked(q, k, v, g, beta, S0, chunk=C, mu=mu, kappa=kappa)
+    S, Z = S0[0, 0].copy(), np.zeros((dk, dv))
+    for c in range(T // C):
+        sl = slice(c * C, (c + 1) * C)
+        qs, ks, vs, gs, bs = q[:, :, sl], k[:, :, sl], v[:, :, sl], g[:, :, sl], beta[:, :, sl]
+        _, J = oracle.chunked(qs, ks, np.zeros((1, 1, C, dk)), gs, bs, np.eye(dk)[None, None], chunk=C)
+        _, Bc = oracle.chunked(qs, ks, vs, gs, bs, None, chunk=C)
+        J, Bc = J[0, 0], Bc[0, 0]
+        F = np.diag(np.exp(gs[0, 0].sum(axis=0)))
+        m = mu * kappa[0, c]
+        S, Z = J @ S + m * Z + Bc, (J - F) @ S + m * Z + Bc
+    return _rel(S, Sm[0, 0])
+
+
 ALL_PINS = {
     "golden_examples": (pin_golden_examples, 1e-12),
     "golden_inverse": (pin_golden_inverse, 1e-12),
@@ -424,6 +462,8 @@ ALL_PINS = {
     "block_neumann": (pin_block_neumann, 1e-10),
     "neumann1_short_chunks": (pin_neumann1_short_chunks, 1e-12),
     "output_epilogue": (pin_output_epilogue, 1e-13),
+    "momentum_reduces": (pin_momentum_reduces, 1e-13),
+    "momentum_block_form": (pin_momentum_block_form, 1e-12),
     "chunked_neumann": (pin_chunked_neumann, 1e-11),
 }
 

@@ -29,6 +29,13 @@ MUTANTS = [
     ("neumann_resid_sign", "X[e] += T1[e];", "X[e] -= T1[e];"),
     ("lam_not_cumulative", "acc += gc[(long)t * G + (long)i * G / dk];",
      "acc = gc[(long)t * G + (long)i * G / dk];"),
+    ("neumann1_sign", "X[e] = Dinv[e] - X[e];", "X[e] = Dinv[e] + X[e];"),
+    ("epilogue_gate_sign", "const double gate = 1.0 / (1.0 + exp(-z[(size_t)r * dv + i]));",
+     "const double gate = 1.0 / (1.0 + exp(z[(size_t)r * dv + i]));"),
+    ("momentum_velocity_sign", "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] - fs);",
+     "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] + fs);"),
+    ("momentum_no_carry", "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] - fs);",
+     "Z[i * dv + n] = (S[i * dv + n] - fs);"),
 ]
 
 
