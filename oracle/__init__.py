@@ -65,11 +65,12 @@ def load_library(path: str):
     lib.gdro_neumann_inverse.argtypes = [i, dp, i, i, i, dp]
     lib.gdro_block_neumann1_inverse.argtypes = [i, dp, i, dp]
     lib.gdro_output_gate_rmsnorm.argtypes = [i, i, dp, dp, dp, ctypes.c_double, dp]
+    lib.gdro_recurrent_grad.argtypes = [i] * 7 + [dp] * 14 + [i]
     lib.gdro_chunk_matrices.argtypes = [i, i, i] + [dp] * 7
     lib.gdro_max_threads.argtypes = []
     for f in (lib.gdro_recurrent, lib.gdro_chunked, lib.gdro_chunked_momentum, lib.gdro_tril_inverse,
               lib.gdro_neumann_inverse, lib.gdro_block_neumann1_inverse,
-              lib.gdro_output_gate_rmsnorm,
+              lib.gdro_output_gate_rmsnorm, lib.gdro_recurrent_grad,
               lib.gdro_chunk_matrices, lib.gdro_max_threads):
         f.restype = ctypes.c_int
     return lib
@@ -133,6 +134,26 @@ def recurrent(q, k, v, g, beta, S0=None, nthreads=0):
                                   _ptr(g), _ptr(beta), _ptr(S0), _ptr(o), _ptr(Sf),
                                   int(nthreads)), "gdro_recurrent")
     return o, Sf
+
+
+def recurrent_grad(q, k, v, g, beta, S0, dO, dSf=None, nthreads=0):
+    """Gradients of sum(dO * o) + sum(dSf * S_final) of the token recurrence with
+    respect to (q, k, v, g, beta, S0), by a reverse sweep over the tokens.
+    Returns a dict with those keys (dS0 is the gradient at the initial state,
+    zero or S0)."""
+    q, k, v, g, beta, dO = map(_f64, (q, k, v, g, beta, dO))
+    S0 = None if S0 is None else _f64(S0)
+    dSf = None if dSf is None else _f64(dSf)
+    B, T, Hk, Hv, dk, dv, G = _dims(q, v, g)
+    out = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v),
+           "g": np.zeros_like(g), "beta": np.zeros_like(beta),
+           "S0": np.zeros((B, Hv, dk, dv), np.float64)}
+    _check(_load().gdro_recurrent_grad(B, T, Hk, Hv, dk, dv, G, _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(g), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dSf),
+                                       _ptr(out["q"]), _ptr(out["k"]), _ptr(out["v"]),
+                                       _ptr(out["g"]), _ptr(out["beta"]), _ptr(out["S0"]),
+                                       int(nthreads)), "gdro_recurrent_grad")
+    return out
 
 
 def chunked(q, k, v, g, beta, S0=None, chunk=64, inverse="exact", order=4, resid=1,

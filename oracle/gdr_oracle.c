@@ -554,3 +554,152 @@ int gdro_output_gate_rmsnorm(int rows, int dv, const double *o, const double *z,
     }
     return 0;
 }
+
+/* f_i = exp(g of channel i's group) for one token's gate row gt[G] */
+static void decay_factors(double *f, const double *gt, int dk, int G)
+{
+    for (int i = 0; i < dk; ++i) {
+        const long grp = (long)i * G / dk;
+        f[i] = exp(gt[grp]);
+    }
+}
+
+/*
+ * Gradients of the token recurrence ([SLA] §2.1 Eq. (2), the definition the
+ * oracle's forward follows) by a reverse sweep over the tokens: for upstream
+ * gradients dO [B,Hv,T,dv] and dSf [B,Hv,dk,dv] (NULL for zero), the gradients
+ * of sum(dO * o) + sum(dSf * S_final) with respect to q, k [B,Hk,T,dk],
+ * v [B,Hv,T,dv], g [B,Hk,T,G], beta [B,Hk,T] and S0 [B,Hv,dk,dv] (the initial
+ * state, zero when S0 is NULL).  Per token, with S' = F_t S_{t-1}, u = v - S'^T k,
+ * S_t = S' + beta k u^T and o = S_t^T q, backwards:
+ *   dS += q do^T, dq = S_t do;
+ *   du = beta dS^T k, dbeta = k^T dS u, dk = beta dS u - S' du, dv = du,
+ *   dS' = dS - k du^T;
+ *   dS_{t-1} = F_t dS', dg (per group) += sum_{i in group} f_i sum_n dS'_in S_{t-1,in}.
+ * Key-head inputs collect the gradients of all their value heads.  The states
+ * are recomputed forward and kept per token (T dk dv doubles per value head).
+ */
+int gdro_recurrent_grad(int B, int T, int Hk, int Hv, int dk, int dv, int G, const double *q,
+                        const double *k, const double *v, const double *g, const double *beta,
+                        const double *S0, const double *dO, const double *dSf, double *dq,
+                        double *dkk, double *dvv, double *dg, double *dbeta, double *dS0,
+                        int nthreads)
+{
+    if (check_dims(B, T, Hk, Hv, dk, dv, G) || !dO)
+        return GDRO_ERR_ARG;
+    const int R = Hv / Hk;
+    const long nkh = (long)B * Hk;
+    const size_t SS = (size_t)dk * dv;
+    int err = 0;
+    memset(dq, 0, sizeof(double) * (size_t)nkh * T * dk);
+    memset(dkk, 0, sizeof(double) * (size_t)nkh * T * dk);
+    memset(dg, 0, sizeof(double) * (size_t)nkh * T * G);
+    memset(dbeta, 0, sizeof(double) * (size_t)nkh * T);
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long kh = 0; kh < nkh; ++kh) {   /* one key head and its R value heads */
+        const long b = kh / Hk, hk = kh % Hk;
+        double *Sall = (double *)malloc(sizeof(double) * SS * (size_t)(T + 1));
+        double *Sp = (double *)malloc(sizeof(double) * SS);
+        double *dS = (double *)malloc(sizeof(double) * SS);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *du = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *f = (double *)malloc(sizeof(double) * (size_t)dk);
+        if (!Sall || !Sp || !dS || !u || !du || !f) {
+            free(Sall); free(Sp); free(dS); free(u); free(du); free(f);
+#pragma omp atomic write
+            err = GDRO_ERR_NOMEM;
+            continue;
+        }
+        for (int m = 0; m < R; ++m) {
+            const long s = b * Hv + hk * R + m;   /* value-head sequence */
+            /* forward, keeping S_{t-1} of every token in Sall[t] */
+            if (S0)
+                memcpy(Sall, S0 + s * (long)SS, sizeof(double) * SS);
+            else
+                memset(Sall, 0, sizeof(double) * SS);
+            for (long t = 0; t < T; ++t) {
+                const double *kt = k + (kh * T + t) * dk, *vt = v + (s * T + t) * dv;
+                const double *gt = g + (kh * T + t) * G;
+                const double bt = beta[kh * T + t];
+                const double *Sprev = Sall + SS * t;
+                double *Snew = Sall + SS * (t + 1);
+                decay_factors(f, gt, dk, G);
+                for (int n = 0; n < dv; ++n) {
+                    double r = 0.0;
+                    for (int i = 0; i < dk; ++i)
+                        r += f[i] * Sprev[i * dv + n] * kt[i];
+                    u[n] = vt[n] - r;
+                }
+                for (int i = 0; i < dk; ++i)
+                    for (int n = 0; n < dv; ++n)
+                        Snew[i * dv + n] = f[i] * Sprev[i * dv + n] + bt * kt[i] * u[n];
+            }
+            /* reverse sweep */
+            if (dSf)
+                memcpy(dS, dSf + s * (long)SS, sizeof(double) * SS);
+            else
+                memset(dS, 0, sizeof(double) * SS);
+            for (long t = T - 1; t >= 0; --t) {
+                const double *qt = q + (kh * T + t) * dk, *kt = k + (kh * T + t) * dk;
+                const double *vt = v + (s * T + t) * dv, *gt = g + (kh * T + t) * G;
+                const double *dot = dO + (s * T + t) * dv;
+                const double bt = beta[kh * T + t];
+                const double *Sprev = Sall + SS * t, *Snew = Sall + SS * (t + 1);
+                double *dqt = dq + (kh * T + t) * dk, *dkt = dkk + (kh * T + t) * dk;
+                double *dvt = dvv + (s * T + t) * dv, *dgt = dg + (kh * T + t) * G;
+                decay_factors(f, gt, dk, G);
+                for (int i = 0; i < dk; ++i)
+                    for (int n = 0; n < dv; ++n)
+                        Sp[i * dv + n] = f[i] * Sprev[i * dv + n];
+                for (int n = 0; n < dv; ++n) {
+                    double r = 0.0;
+                    for (int i = 0; i < dk; ++i)
+                        r += Sp[i * dv + n] * kt[i];
+                    u[n] = vt[n] - r;
+                }
+                /* readout o = S_t^T q */
+                for (int i = 0; i < dk; ++i) {
+                    double acc = 0.0;
+                    for (int n = 0; n < dv; ++n) {
+                        dS[i * dv + n] += qt[i] * dot[n];
+                        acc += Snew[i * dv + n] * dot[n];
+                    }
+                    dqt[i] += acc;
+                }
+                /* write S_t = S' + beta k u^T, u = v - S'^T k */
+                double db = 0.0;
+                for (int n = 0; n < dv; ++n) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i)
+                        acc += kt[i] * dS[i * dv + n];
+                    du[n] = bt * acc;
+                    db += acc * u[n];
+                    dvt[n] = du[n];
+                }
+                dbeta[kh * T + t] += db;
+                for (int i = 0; i < dk; ++i) {
+                    double a1 = 0.0, a2 = 0.0;
+                    for (int n = 0; n < dv; ++n) {
+                        a1 += dS[i * dv + n] * u[n];
+                        a2 += Sp[i * dv + n] * du[n];
+                    }
+                    dkt[i] += bt * a1 - a2;
+                }
+                /* dS' = dS - k du^T, then through the decay S' = F_t S_{t-1} */
+                for (int i = 0; i < dk; ++i) {
+                    double df = 0.0;
+                    for (int n = 0; n < dv; ++n) {
+                        const double dsp = dS[i * dv + n] - kt[i] * du[n];
+                        df += dsp * Sprev[i * dv + n];
+                        dS[i * dv + n] = f[i] * dsp;
+                    }
+                    dgt[(long)i * G / dk] += df * f[i];
+                }
+            }
+            memcpy(dS0 + s * (long)SS, dS, sizeof(double) * SS);
+        }
+        free(Sall); free(Sp); free(dS); free(u); free(du); free(f);
+    }
+    return err;
+}

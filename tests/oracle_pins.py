@@ -445,6 +445,39 @@ def pin_momentum_block_form(seed=17):
     return _rel(S, Sm[0, 0])
 
 
+# Gradients of the recurrence (the backward of NEXT #2 starts from this): the
+# oracle's reverse sweep against central finite differences of its forward, for
+# every input element of a tiny problem with two value heads per key head (the
+# key-head gradients sum over them), per-channel and scalar gates, and S0.
+def pin_grad_finite_differences(seed=18):
+    rng = np.random.default_rng(seed)
+    worst = 0.0
+    for G in (3, 1):
+        q, k, v, g, beta, S0 = rand_inputs(rng, 1, 5, 1, 2, 3, 2, G)
+        Wo = rng.standard_normal((1, 2, 5, 2))
+        Ws = rng.standard_normal((1, 2, 3, 2))
+        x = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "S0": S0}
+
+        def loss(x):
+            o, Sf = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
+            return float(np.sum(o * Wo) + np.sum(Sf * Ws))
+
+        grads = oracle.recurrent_grad(q, k, v, g, beta, S0, Wo, Ws)
+        h = 1e-6
+        for name, arr in x.items():
+            fd = np.zeros_like(arr)
+            for idx in np.ndindex(arr.shape):
+                old = arr[idx]
+                arr[idx] = old + h
+                lp = loss(x)
+                arr[idx] = old - h
+                lm = loss(x)
+                arr[idx] = old
+                fd[idx] = (lp - lm) / (2 * h)
+            worst = max(worst, np.abs(grads[name] - fd).max() / max(np.abs(fd).max(), 1e-30))
+    return worst
+
+
 ALL_PINS = {
     "golden_examples": (pin_golden_examples, 1e-12),
     "golden_inverse": (pin_golden_inverse, 1e-12),
@@ -464,6 +497,7 @@ ALL_PINS = {
     "output_epilogue": (pin_output_epilogue, 1e-13),
     "momentum_reduces": (pin_momentum_reduces, 1e-13),
     "momentum_block_form": (pin_momentum_block_form, 1e-12),
+    "grad_finite_differences": (pin_grad_finite_differences, 1e-6),
     "chunked_neumann": (pin_chunked_neumann, 1e-11),
 }
 

@@ -36,6 +36,12 @@ MUTANTS = [
      "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] + fs);"),
     ("momentum_no_carry", "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] - fs);",
      "Z[i * dv + n] = (S[i * dv + n] - fs);"),
+    ("grad_decay_group", "f[i] = exp(gt[grp]);", "f[i] = exp(gt[0]);"),
+    ("grad_dk_drops_state_term", "dkt[i] += bt * a1 - a2;", "dkt[i] += bt * a1;"),
+    ("grad_dS_misses_write", "const double dsp = dS[i * dv + n] - kt[i] * du[n];",
+     "const double dsp = dS[i * dv + n];"),
+    ("grad_dg_no_factor", "dgt[(long)i * G / dk] += df * f[i];", "dgt[(long)i * G / dk] += df;"),
+    ("grad_dq_old_state", "acc += Snew[i * dv + n] * dot[n];", "acc += Sprev[i * dv + n] * dot[n];"),
 ]
 
 
