@@ -33,7 +33,8 @@ struct SimtLayout {      // offsets in floats into dynamic shared memory
 
 // Neumann mode keeps N (in A) and the series X; a third C x C buffer P is only
 // needed for more than one residual step (the single-step correction writes
-// its residual over N).  Q S is staged in X once X has been applied.
+// its residual over N).  Q S (C x NV) is staged in X once X has been applied,
+// when X is large enough to hold it (C >= NV).
 __host__ __device__ inline SimtLayout simt_layout(int C, int G, int dk, bool neumann, int resid,
                                                   int NV)
 {
@@ -45,8 +46,9 @@ __host__ __device__ inline SimtLayout simt_layout(int C, int G, int dk, bool neu
     s.P = off;    off += (neumann && resid > 1) ? C * C : 0;
     s.S = off;    off += dk * NV;
     s.rhs = off;  off += C * NV;
-    s.qs = neumann ? s.X : off;
-    off += neumann ? 0 : C * NV;
+    const bool qs_in_x = neumann && C >= NV;
+    s.qs = qs_in_x ? s.X : off;
+    off += qs_in_x ? 0 : C * NV;
     s.E = off;    off += C * NV;
     s.blk = off;  off += LB * C;
     s.beta = off; off += C;
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
             E[t * NV + n] = sbeta[t] * acc;
         }
         __syncthreads();
-        // --- Qbar S, Qbar_t = q_t e^{Lambda_t} (staged in X in Neumann mode: X is spent)
+        // --- Qbar S, Qbar_t = q_t e^{Lambda_t} (staged in X in Neumann mode when it fits: X is spent)
         for (int idx = tid; idx < Cl * (NV / 8); idx += NT) {
             const int t = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
             float aq[8];
