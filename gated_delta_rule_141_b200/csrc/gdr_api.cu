@@ -123,6 +123,40 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, c
     return static_cast<gdr_status>(rc);
 }
 
+gdr_status gdr_chunk_fwd_momentum(const gdr_shape *shape, const void *q, const void *k,
+                                  const void *v, const float *g, const float *beta,
+                                  const float *S0, int chunk, gdr_gate_mode gate_mode,
+                                  gdr_inverse_mode inverse_mode, float mu, const int32_t *kappa,
+                                  void *o, float *S_final, void *stream)
+{
+    gdr::Params p;
+    gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    if (st != GDR_OK)
+        return st;
+    if (!(mu > -1e30f && mu < 1e30f))   // finite (NaN fails both)
+        return GDR_ERR_ARG;
+    const bool has_tokens = (long)p.B * p.T > 0;
+    if (has_tokens && (!q || !k || !v || !g || !beta || !o))
+        return GDR_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_final};
+    for (const void *ptr : ptrs)
+        if (ptr != nullptr && !aligned16(ptr))
+            return GDR_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(kappa) & 3u) != 0)
+        return GDR_ERR_ALIGN;
+    if (shape->kernel != GDR_KERNEL_AUTO && shape->kernel != GDR_KERNEL_SIMT)
+        return GDR_ERR_UNSUPPORTED;
+    p.momentum = 1;
+    p.mu = mu;
+    p.kappa = kappa;
+    if (gdr::simt_smem_bytes(p) > 227 * 1024)
+        return GDR_ERR_UNSUPPORTED;
+    if (p.B == 0)
+        return GDR_OK;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S0 = S0; p.o = o; p.S_final = S_final;
+    return static_cast<gdr_status>(gdr::launch_simt(p, static_cast<cudaStream_t>(stream)));
+}
+
 gdr_status gdr_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
                                gdr_inverse_mode inverse_mode, size_t *bytes)
 {

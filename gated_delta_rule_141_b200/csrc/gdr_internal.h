@@ -19,6 +19,9 @@ struct Params {
     int neumann1;   // 1-Step Neumann in blocks of 16 (neumann is 0 then)
     int neu_order;  // Neumann order m
     int neu_resid;  // Newton residual corrections
+    int momentum;   // chunk-boundary momentum (CUDA-core kernel only)
+    float mu;       // momentum coefficient
+    const int *kappa;  // [B][ceil(T / C)] momentum gates, or nullptr for ones
     const void *q, *k, *v;
     const float *g, *beta, *S0;
     void *o;

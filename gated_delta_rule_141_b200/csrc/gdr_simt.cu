@@ -16,6 +16,12 @@
 // Approximation for Quantized Gated DeltaNet" (masked powers, Lemma 3.1, then
 // Newton residual corrections).
 //
+// With chunk-boundary momentum (the same paper, §2.3) the state update of each
+// chunk is blended with a velocity Z (zero at the start), kept beside S:
+//   Z <- mu kappa_c Z + Khat^T E,  S <- F S + Z,
+// where Khat^T E is exactly the plain update minus F S; the chunk's outputs are
+// those of the plain chunk computation from the entry state.
+//
 // One CTA owns one value head and NV value columns; chunks run in order.
 #include <cuda_bf16.h>
 
@@ -28,7 +34,7 @@ constexpr int NT = 256;  // threads per CTA
 constexpr int LB = 16;   // rows per row block (L readout, Neumann products)
 
 struct SimtLayout {      // offsets in floats into dynamic shared memory
-    int lam, A, P, X, S, rhs, qs, E, blk, beta, row, total;
+    int lam, A, P, X, S, rhs, qs, E, blk, beta, row, Z, total;
 };
 
 // Neumann mode keeps N (in A) and the series X; a third C x C buffer P is only
@@ -36,7 +42,7 @@ struct SimtLayout {      // offsets in floats into dynamic shared memory
 // its residual over N).  Q S (C x NV) is staged in X once X has been applied,
 // when X is large enough to hold it (C >= NV).
 __host__ __device__ inline SimtLayout simt_layout(int C, int G, int dk, bool neumann, int resid,
-                                                  int NV)
+                                                  int NV, bool momentum)
 {
     SimtLayout s;
     int off = 0;
@@ -53,6 +59,7 @@ __host__ __device__ inline SimtLayout simt_layout(int C, int G, int dk, bool neu
     s.blk = off;  off += LB * C;
     s.beta = off; off += C;
     s.row = off;  off += C;
+    s.Z = off;    off += momentum ? dk * NV : 0;   // momentum velocity, last
     s.total = off;
     return s;
 }
@@ -75,17 +82,18 @@ __device__ __forceinline__ void st_out(void *p, long i, float x)
         static_cast<float *>(p)[i] = x;
 }
 
-template <bool IN_BF16, bool OUT_BF16, int NV>
+template <bool IN_BF16, bool OUT_BF16, int NV, bool MOM>
 __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
 {
     extern __shared__ float sm[];
     const int C = p.C, G = p.G, dk = p.dk, dv = p.dv, T = p.T;
     const bool neu = p.neumann != 0;
     const bool blk1 = p.neumann1 != 0;   // 1-Step Neumann: X is its scratch
-    const SimtLayout Ly = simt_layout(C, G, dk, neu || blk1, p.neu_resid, NV);
+    const SimtLayout Ly = simt_layout(C, G, dk, neu || blk1, p.neu_resid, NV, MOM);
     float *lam = sm + Ly.lam, *A = sm + Ly.A, *P = sm + Ly.P, *X = sm + Ly.X;
     float *S = sm + Ly.S, *rhs = sm + Ly.rhs, *qs = sm + Ly.qs, *E = sm + Ly.E;
     float *blk = sm + Ly.blk, *sbeta = sm + Ly.beta, *row = sm + Ly.row;
+    float *Z = sm + Ly.Z;   // momentum only
 
     const int tid = threadIdx.x;
     const int n0 = blockIdx.x * NV;           // first value column of this CTA
@@ -99,6 +107,8 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
     for (int idx = tid; idx < dk * NV; idx += NT) {
         const int i = idx / NV, n = idx % NV;
         S[idx] = (p.S0 != nullptr && n < nv) ? p.S0[(vh * dk + i) * dv + n0 + n] : 0.f;
+        if constexpr (MOM)
+            Z[idx] = 0.f;
     }
 
     for (int c0 = 0; c0 < T; c0 += C) {
@@ -328,6 +338,12 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
             __syncthreads();
         }
         // --- S <- F S + Khat^T E,  F = e^{Lambda_C}, Khat_t = k_t e^{Lambda_C - Lambda_t}
+        //     (momentum: Z <- mu kappa_c Z + Khat^T E, S <- F S + Z)
+        float mk = 0.f;
+        if constexpr (MOM) {
+            const long nch = (T + C - 1) / C;
+            mk = p.mu * (p.kappa != nullptr ? (float)p.kappa[(long)b * nch + c0 / C] : 1.f);
+        }
         for (int idx = tid; idx < dk * (NV / 8); idx += NT) {
             const int i = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
             const float lc = lam[(Cl - 1) * G + i / width];
@@ -335,7 +351,7 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
             float acc[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                acc[u] = f * S[i * NV + nb + u];
+                acc[u] = MOM ? 0.f : f * S[i * NV + nb + u];
             for (int t = 0; t < Cl; ++t) {
                 const float w = ld_in<IN_BF16>(p.k, (kh * T + c0 + t) * dk + i) *
                                 expf(lc - lam[t * G + i / width]);
@@ -344,8 +360,15 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
                     acc[u] += w * E[t * NV + nb + u];
             }
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                S[i * NV + nb + u] = acc[u];
+            for (int u = 0; u < 8; ++u) {
+                if constexpr (MOM) {
+                    const float z = mk * Z[i * NV + nb + u] + acc[u];
+                    Z[i * NV + nb + u] = z;
+                    S[i * NV + nb + u] = f * S[i * NV + nb + u] + z;
+                } else {
+                    S[i * NV + nb + u] = acc[u];
+                }
+            }
         }
     }
     __syncthreads();
@@ -357,10 +380,10 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
         }
 }
 
-template <bool I, bool O, int NV>
+template <bool I, bool O, int NV, bool MOM>
 int launch_variant(const Params &p, int smem, cudaStream_t stream)
 {
-    auto kern = simt_fwd_kernel<I, O, NV>;
+    auto kern = simt_fwd_kernel<I, O, NV, MOM>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 6;  // GDR_ERR_CUDA
     dim3 grid((p.dv + NV - 1) / NV, p.Hv, p.B);
@@ -372,18 +395,25 @@ constexpr int kMaxSmem = 227 * 1024;
 
 int smem_for(const Params &p, int NV)
 {
-    return simt_layout(p.C, p.G, p.dk, p.neumann != 0 || p.neumann1 != 0, p.neu_resid, NV).total *
+    return simt_layout(p.C, p.G, p.dk, p.neumann != 0 || p.neumann1 != 0, p.neu_resid, NV,
+                       p.momentum != 0).total *
            (int)sizeof(float);
+}
+
+template <int NV, bool MOM>
+int launch_io(const Params &p, int smem, cudaStream_t stream)
+{
+    if (p.in_bf16)
+        return p.out_bf16 ? launch_variant<true, true, NV, MOM>(p, smem, stream)
+                          : launch_variant<true, false, NV, MOM>(p, smem, stream);
+    return p.out_bf16 ? launch_variant<false, true, NV, MOM>(p, smem, stream)
+                      : launch_variant<false, false, NV, MOM>(p, smem, stream);
 }
 
 template <int NV>
 int launch_nv(const Params &p, int smem, cudaStream_t stream)
 {
-    if (p.in_bf16)
-        return p.out_bf16 ? launch_variant<true, true, NV>(p, smem, stream)
-                          : launch_variant<true, false, NV>(p, smem, stream);
-    return p.out_bf16 ? launch_variant<false, true, NV>(p, smem, stream)
-                      : launch_variant<false, false, NV>(p, smem, stream);
+    return p.momentum ? launch_io<NV, true>(p, smem, stream) : launch_io<NV, false>(p, smem, stream);
 }
 
 }  // namespace

@@ -39,7 +39,7 @@ TC2_EXT_RECORD_BYTES = 66048
 _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN, "neumann1": INV_NEUMANN1}
 
 # Every symbol include/gdr.h declares.
-EXPORTS = ("gdr_chunk_fwd", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
+EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_momentum", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
            "gdr_chunk_fwd_static",
            "gdr_output_gate_rmsnorm",
            "gdr_select_kernel", "gdr_kernel_chunk", "gdr_state_segments", "gdr_device_status",
@@ -83,6 +83,9 @@ def load(path: str = LIB_PATH):
     lib.gdr_chunk_fwd.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i, i,
                                   vp, vp, vp, sz, vp]
     lib.gdr_chunk_fwd.restype = i
+    lib.gdr_chunk_fwd_momentum.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i,
+                                           i, ctypes.c_float, vp, vp, vp, vp]
+    lib.gdr_chunk_fwd_momentum.restype = i
     lib.gdr_chunk_fwd_static.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i,
                                          i, vp, vp, vp]
     lib.gdr_chunk_fwd_static.restype = i
@@ -228,6 +231,46 @@ def chunk_fwd(q, k, v, g, beta, S0=None, chunk=64, gate_mode=None, inverse="exac
                               _stream_handle(stream))
     if st != OK:
         raise GdrError(st)
+    return o, S_final
+
+
+def chunk_fwd_momentum(q, k, v, g, beta, S0=None, mu=0.0, kappa=None, chunk=64, gate_mode=None,
+                       inverse="exact", neumann_order=4, neumann_residual_steps=1,
+                       out_dtype=None, o=None, S_final=None, want_state=True, kernel="auto",
+                       stream=None):
+    """chunk_fwd with chunk-boundary momentum: each chunk's state update is blended
+    with a velocity Z (zero at the start), Z <- mu kappa_c Z + (S~_c - F_c S), S <-
+    F_c S + Z.  kappa: int32 [B, ceil(T / chunk)] CUDA tensor of per-chunk gates on
+    the carried velocity, or None for ones.  Other arguments as chunk_fwd (no
+    workspace: the CUDA-core kernel runs it)."""
+    import torch
+    B, Hk, T, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[3]
+    G = g.shape[-1]
+    if gate_mode is None:
+        gate_mode = gate_mode_for(G, dk)
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("S0", S0),
+                    ("kappa", kappa)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    if kappa is not None and (kappa.dtype != torch.int32 or
+                              tuple(kappa.shape) != (B, (T + int(chunk) - 1) // int(chunk))):
+        raise ValueError("kappa must be an int32 [B, ceil(T / chunk)] tensor")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if o is None:
+        o = torch.empty((B, Hv, T, dv), dtype=out_dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    shape = make_shape(B, T, Hk, Hv, dk, dv, _dtype_code(q.dtype), _dtype_code(o.dtype),
+                       neumann_order, neumann_residual_steps, kernel)
+    st = load().gdr_chunk_fwd_momentum(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                       _ptr(beta), _ptr(S0), int(chunk), int(gate_mode),
+                                       _INVERSES[inverse], float(mu), _ptr(kappa), _ptr(o),
+                                       _ptr(S_final), _stream_handle(stream))
+    if st != OK:
+        raise GdrError(st, "gdr_chunk_fwd_momentum")
     return o, S_final
 
 

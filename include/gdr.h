@@ -35,6 +35,7 @@
 #define GDR_H_
 
 #include <stddef.h>
+#include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -131,6 +132,33 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape,
                          int chunk, gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode,
                          void *o, float *S_final,
                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdr_chunk_fwd_momentum -- gdr_chunk_fwd with chunk-boundary momentum
+ * ("Systolic Linear Attention: Co-Designing Tile-Grouped Gated Delta Attention
+ * for TPUs", §2.3, the momentum update after Eq. (5)).  Each chunk's state
+ * update is blended with a velocity buffer Z that starts at zero:
+ *   Z_c = mu kappa_c Z_{c-1} + (S~_c - F_c S_{c-1}),  S_c = F_c S_{c-1} + Z_c,
+ * with S~_c the plain chunk update from S_{c-1} and F_c the chunk's total decay;
+ * the outputs of chunk c are those of the plain chunk computation from S_{c-1}.
+ * Inputs, outputs and chunk / gate / inverse arguments as gdr_chunk_fwd, plus:
+ *   mu     momentum coefficient (finite; mu = 0 gives gdr_chunk_fwd's result)
+ *   kappa  [B, ceil(T / chunk)] int32 device array of per-chunk gates on the
+ *          carried velocity (0 where a document reset falls in the chunk), or
+ *          NULL for ones; 4-byte aligned (GDR_ERR_ALIGN otherwise)
+ * Chunks are taken at exactly `chunk` tokens (no re-blocking).  Runs on the
+ * CUDA-core kernel (fp32 arithmetic); shape->kernel must be AUTO or SIMT
+ * (anything else: GDR_ERR_UNSUPPORTED).  The velocity takes one more dk x 32
+ * fp32 tile of shared memory; a request that then does not fit also returns
+ * GDR_ERR_UNSUPPORTED.  The velocity is not returned.  No workspace.
+ * Asynchronous on `stream`.
+ */
+gdr_status gdr_chunk_fwd_momentum(const gdr_shape *shape,
+                                  const void *q, const void *k, const void *v,
+                                  const float *g, const float *beta, const float *S0,
+                                  int chunk, gdr_gate_mode gate_mode,
+                                  gdr_inverse_mode inverse_mode, float mu,
+                                  const int32_t *kappa, void *o, float *S_final, void *stream);
 
 /* Device workspace (bytes) that gdr_chunk_fwd needs for this request with the
  * kernel AUTO or shape->kernel selects when given enough: 0 for the one-pass

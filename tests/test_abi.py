@@ -176,6 +176,36 @@ def test_output_epilogue_validates(lib):
     assert f(None, None, None, None, ctypes.c_float(1e-6), None) == gdr.ERR_ARG
 
 
+def test_momentum_validates(lib):
+    # chunk-boundary momentum: host validation only (nothing launches on these)
+    f = gdr.load().gdr_chunk_fwd_momentum
+    nul = [None] * 6
+
+    def call(shape, mu=0.5, kappa=None, chunk=64, inverse=gdr.INV_EXACT):
+        return f(ctypes.byref(shape), *nul, chunk, gdr.GATE_SCALAR, inverse, ctypes.c_float(mu),
+                 kappa, None, None, None)
+
+    sh = gdr.make_shape(2, 100, 1, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
+    assert call(sh) == gdr.ERR_ARG                                 # tokens but no buffers
+    assert call(sh, mu=float("nan")) == gdr.ERR_ARG
+    assert call(sh, mu=float("inf")) == gdr.ERR_ARG
+    assert call(sh, chunk=0) == gdr.ERR_SHAPE
+    empty = gdr.make_shape(0, 100, 1, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
+    assert call(empty) == gdr.OK                                   # nothing to do
+    assert call(empty, kappa=ctypes.c_void_p(2)) == gdr.ERR_ALIGN  # int32 gates, 4-byte aligned
+    tc = gdr.make_shape(0, 100, 1, 2, 64, 64, kernel=gdr.KERNEL_TC2)
+    assert call(tc) == gdr.ERR_UNSUPPORTED                         # CUDA-core kernel only
+    # the velocity tile takes shared memory: dk = 256 with per-channel gates and
+    # exact chunks of 118 fits the plain kernel but not the momentum one
+    wide = gdr.make_shape(0, 1000, 1, 1, 256, 256, in_dtype=gdr.F32, out_dtype=gdr.F32,
+                          kernel="simt")
+    assert gdr.select_kernel(wide, 118, gdr.GATE_CHANNEL) == gdr.KERNEL_SIMT
+    assert f(ctypes.byref(wide), *nul, 118, gdr.GATE_CHANNEL, gdr.INV_EXACT, ctypes.c_float(0.5),
+             None, None, None, None) == gdr.ERR_UNSUPPORTED
+    assert f(ctypes.byref(wide), *nul, 64, gdr.GATE_CHANNEL, gdr.INV_EXACT, ctypes.c_float(0.5),
+             None, None, None, None) == gdr.OK
+
+
 def test_state_segments(lib):
     # The two-pass state pass stays sequential while the value tiles of all
     # sequences fill the SMs, and cuts few long sequences into segments whose
