@@ -1,0 +1,21 @@
+/* Host stand-in for the few CUDA runtime names that gdr_simt.cu's kernel uses,
+ * so that its source compiles as plain C++ for the host-emulation test: one
+ * thread per CTA, CTAs run one after another, __syncthreads() is a no-op (with
+ * a single thread every phase completes before the next begins). */
+#pragma once
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+using std::max;
+using std::min;
+typedef void *cudaStream_t;
+struct host_uint3 { unsigned x, y, z; };
+extern thread_local host_uint3 threadIdx, blockIdx;
+#define __global__
+#define __device__
+#define __host__
+#define __forceinline__ inline
+#define __launch_bounds__(...)
+#define __shared__
+#define __syncthreads() ((void)0)
