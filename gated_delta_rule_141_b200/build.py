@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgdr.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-SOURCES = ["gdr_api.cu", "gdr_simt.cu", "gdr_tc.cu", "gdr_static.cu", "gdr_epilogue.cu"]
+SOURCES = ["gdr_api.cu", "gdr_simt.cu", "gdr_bwd.cu", "gdr_tc.cu", "gdr_static.cu", "gdr_epilogue.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

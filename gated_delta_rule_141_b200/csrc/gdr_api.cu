@@ -123,6 +123,51 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, c
     return static_cast<gdr_status>(rc);
 }
 
+gdr_status gdr_bwd_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                                   size_t *bytes)
+{
+    if (bytes == nullptr)
+        return GDR_ERR_ARG;
+    gdr::Params p;
+    const gdr_status st = make_params(shape, chunk, gate_mode, GDR_INV_EXACT, &p);
+    if (st != GDR_OK)
+        return st;
+    *bytes = gdr::bwd_workspace_bytes(p);
+    return GDR_OK;
+}
+
+gdr_status gdr_chunk_bwd(const gdr_shape *shape, const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, const float *S0, const float *dO,
+                         const float *dS_final, int chunk, gdr_gate_mode gate_mode, float *dq,
+                         float *dk, float *dv, float *dg, float *dbeta, float *dS0,
+                         void *workspace, size_t workspace_bytes, void *stream)
+{
+    gdr::Params p;
+    gdr_status st = make_params(shape, chunk, gate_mode, GDR_INV_EXACT, &p);
+    if (st != GDR_OK)
+        return st;
+    const bool has_tokens = (long)p.B * p.T > 0;
+    if (has_tokens && (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv || !dg || !dbeta))
+        return GDR_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, dO, dS_final, dq, dk, dv, dg, dbeta, dS0, workspace};
+    for (const void *ptr : ptrs)
+        if (ptr != nullptr && !aligned16(ptr))
+            return GDR_ERR_ALIGN;
+    if (shape->kernel != GDR_KERNEL_AUTO && shape->kernel != GDR_KERNEL_SIMT)
+        return GDR_ERR_UNSUPPORTED;
+    if (gdr::bwd_smem_bytes(p) > 227 * 1024 || gdr::simt_smem_bytes(p) > 227 * 1024)
+        return GDR_ERR_UNSUPPORTED;
+    const size_t need = gdr::bwd_workspace_bytes(p);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return GDR_ERR_WORKSPACE;
+    if (p.B == 0)
+        return GDR_OK;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S0 = S0;
+    p.dO = dO; p.dS_final = dS_final;
+    p.grad_q = dq; p.grad_k = dk; p.grad_v = dv; p.grad_g = dg; p.grad_beta = dbeta; p.grad_S0 = dS0;
+    return static_cast<gdr_status>(gdr::launch_bwd(p, workspace, static_cast<cudaStream_t>(stream)));
+}
+
 gdr_status gdr_chunk_fwd_momentum(const gdr_shape *shape, const void *q, const void *k,
                                   const void *v, const float *g, const float *beta,
                                   const float *S0, int chunk, gdr_gate_mode gate_mode,

@@ -24,8 +24,12 @@ struct Params {
     const int *kappa;  // [B][ceil(T / C)] momentum gates, or nullptr for ones
     const void *q, *k, *v;
     const float *g, *beta, *S0;
-    void *o;
+    void *o;          // may be nullptr for the CUDA-core kernel (states only)
     float *S_final;
+    float *S_chunks;  // CUDA-core kernel: [B][Hv][ceil(T/C)][dk][dv] state at each chunk's start, or nullptr
+    // backward (gdr_chunk_bwd): upstream gradients in, gradients out (fp32)
+    const float *dO, *dS_final;
+    float *grad_q, *grad_k, *grad_v, *grad_g, *grad_beta, *grad_S0;
 };
 
 // Status word that kernels set when a bounded wait gives up (0 = fine).  It
@@ -37,6 +41,13 @@ int read_and_clear_device_status();
 // code if the request does not fit the kernel's shared-memory budget.
 int simt_smem_bytes(const Params &p);
 int launch_simt(const Params &p, cudaStream_t stream);
+
+// Backward of the chunked forward (exact inverse), CUDA cores, fp32: the states
+// at the chunk starts are recomputed by the forward kernel into the workspace,
+// then one reverse sweep over the chunks per value tile.
+size_t bwd_workspace_bytes(const Params &p);
+int bwd_smem_bytes(const Params &p);
+int launch_bwd(const Params &p, void *workspace, cudaStream_t stream);
 
 // Tensor-core kernel (tcgen05 + TMEM + TMA, bf16 operands, fp32 accumulate).
 bool tc_supports(const Params &p);

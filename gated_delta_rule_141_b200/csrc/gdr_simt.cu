@@ -114,6 +114,14 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
     for (int c0 = 0; c0 < T; c0 += C) {
         const int Cl = min(C, T - c0);        // a ragged last chunk is shorter
         __syncthreads();
+        if (p.S_chunks != nullptr) {          // the chunk's entry state, for the backward
+            float *dst = p.S_chunks + ((vh * ((T + C - 1) / C) + c0 / C) * dk) * (long)dv + n0;
+            for (int idx = tid; idx < dk * NV; idx += NT) {
+                const int i = idx / NV, n = idx % NV;
+                if (n < nv)
+                    dst[(long)i * dv + n] = S[idx];
+            }
+        }
         // --- write gates and cumulative log-decay Lambda (summed, per group)
         for (int t = tid; t < Cl; t += NT)
             sbeta[t] = p.beta[kh * T + c0 + t];
@@ -289,53 +297,57 @@ __global__ void __launch_bounds__(NT) simt_fwd_kernel(const Params p)
             E[t * NV + n] = sbeta[t] * acc;
         }
         __syncthreads();
-        // --- Qbar S, Qbar_t = q_t e^{Lambda_t} (staged in X in Neumann mode when it fits: X is spent)
-        for (int idx = tid; idx < Cl * (NV / 8); idx += NT) {
-            const int t = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
-            float aq[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                aq[u] = 0.f;
-            const long qt = (kh * T + c0 + t) * dk;
-            for (int i = 0; i < dk; ++i) {
-                const float qb = ld_in<IN_BF16>(p.q, qt + i) * expf(lam[t * G + i / width]);
+        // --- outputs (skipped when only the chunk-start states are wanted: a uniform
+        //     condition, so every thread takes the same barriers)
+        if (p.o != nullptr) {
+            // --- Qbar S, Qbar_t = q_t e^{Lambda_t} (staged in X in Neumann mode when it fits: X is spent)
+            for (int idx = tid; idx < Cl * (NV / 8); idx += NT) {
+                const int t = idx / (NV / 8), nb = (idx % (NV / 8)) * 8;
+                float aq[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
-                    aq[u] += qb * S[i * NV + nb + u];
-            }
+                    aq[u] = 0.f;
+                const long qt = (kh * T + c0 + t) * dk;
+                for (int i = 0; i < dk; ++i) {
+                    const float qb = ld_in<IN_BF16>(p.q, qt + i) * expf(lam[t * G + i / width]);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                qs[t * NV + nb + u] = aq[u];
-        }
-        __syncthreads();
-        // --- O = Qbar S + L E, L formed one row block at a time
-        for (int r0 = 0; r0 < Cl; r0 += LB) {
-            const int nr = min(LB, Cl - r0);
-            for (int idx = tid; idx < nr * Cl; idx += NT) {
-                const int r = idx / Cl, j = idx % Cl, t = r0 + r;
-                float l = 0.f;
-                if (j <= t) {
-                    const long qt = (kh * T + c0 + t) * dk, kj = (kh * T + c0 + j) * dk;
-                    for (int gi = 0; gi < G; ++gi) {
-                        float s = 0.f;
-                        for (int i = gi * width; i < (gi + 1) * width; ++i)
-                            s += ld_in<IN_BF16>(p.q, qt + i) * ld_in<IN_BF16>(p.k, kj + i);
-                        l += expf(lam[t * G + gi] - lam[j * G + gi]) * s;
+                    for (int u = 0; u < 8; ++u)
+                        aq[u] += qb * S[i * NV + nb + u];
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    qs[t * NV + nb + u] = aq[u];
+            }
+            __syncthreads();
+            // --- O = Qbar S + L E, L formed one row block at a time
+            for (int r0 = 0; r0 < Cl; r0 += LB) {
+                const int nr = min(LB, Cl - r0);
+                for (int idx = tid; idx < nr * Cl; idx += NT) {
+                    const int r = idx / Cl, j = idx % Cl, t = r0 + r;
+                    float l = 0.f;
+                    if (j <= t) {
+                        const long qt = (kh * T + c0 + t) * dk, kj = (kh * T + c0 + j) * dk;
+                        for (int gi = 0; gi < G; ++gi) {
+                            float s = 0.f;
+                            for (int i = gi * width; i < (gi + 1) * width; ++i)
+                                s += ld_in<IN_BF16>(p.q, qt + i) * ld_in<IN_BF16>(p.k, kj + i);
+                            l += expf(lam[t * G + gi] - lam[j * G + gi]) * s;
+                        }
+                    }
+                    blk[r * C + j] = l;
+                }
+                __syncthreads();
+                for (int idx = tid; idx < nr * NV; idx += NT) {
+                    const int r = idx / NV, n = idx % NV, t = r0 + r;
+                    if (n < nv) {
+                        float acc = qs[t * NV + n];
+                        for (int j = 0; j <= t; ++j)
+                            acc += blk[r * C + j] * E[j * NV + n];
+                        st_out<OUT_BF16>(p.o, (vh * T + c0 + t) * dv + n0 + n, acc);
                     }
                 }
-                blk[r * C + j] = l;
+                __syncthreads();
             }
-            __syncthreads();
-            for (int idx = tid; idx < nr * NV; idx += NT) {
-                const int r = idx / NV, n = idx % NV, t = r0 + r;
-                if (n < nv) {
-                    float acc = qs[t * NV + n];
-                    for (int j = 0; j <= t; ++j)
-                        acc += blk[r * C + j] * E[j * NV + n];
-                    st_out<OUT_BF16>(p.o, (vh * T + c0 + t) * dv + n0 + n, acc);
-                }
-            }
-            __syncthreads();
         }
         // --- S <- F S + Khat^T E,  F = e^{Lambda_C}, Khat_t = k_t e^{Lambda_C - Lambda_t}
         //     (momentum: Z <- mu kappa_c Z + Khat^T E, S <- F S + Z)

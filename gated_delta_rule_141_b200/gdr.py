@@ -39,7 +39,8 @@ TC2_EXT_RECORD_BYTES = 66048
 _INVERSES = {"exact": INV_EXACT, "neumann": INV_NEUMANN, "neumann1": INV_NEUMANN1}
 
 # Every symbol include/gdr.h declares.
-EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_momentum", "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
+EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_momentum", "gdr_chunk_bwd", "gdr_bwd_workspace_bytes",
+           "gdr_workspace_bytes", "gdr_chunk_prepare", "gdr_chunk_fwd_host",
            "gdr_chunk_fwd_static",
            "gdr_output_gate_rmsnorm",
            "gdr_select_kernel", "gdr_kernel_chunk", "gdr_state_segments", "gdr_device_status",
@@ -86,6 +87,10 @@ def load(path: str = LIB_PATH):
     lib.gdr_chunk_fwd_momentum.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i,
                                            i, ctypes.c_float, vp, vp, vp, vp]
     lib.gdr_chunk_fwd_momentum.restype = i
+    lib.gdr_chunk_bwd.argtypes = [ctypes.POINTER(GdrShape)] + [vp] * 8 + [i, i] + [vp] * 7 + [sz, vp]
+    lib.gdr_chunk_bwd.restype = i
+    lib.gdr_bwd_workspace_bytes.argtypes = [ctypes.POINTER(GdrShape), i, i, ctypes.POINTER(sz)]
+    lib.gdr_bwd_workspace_bytes.restype = i
     lib.gdr_chunk_fwd_static.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i,
                                          i, vp, vp, vp]
     lib.gdr_chunk_fwd_static.restype = i
@@ -272,6 +277,59 @@ def chunk_fwd_momentum(q, k, v, g, beta, S0=None, mu=0.0, kappa=None, chunk=64, 
     if st != OK:
         raise GdrError(st, "gdr_chunk_fwd_momentum")
     return o, S_final
+
+
+def bwd_workspace_bytes(shape: GdrShape, chunk: int, gate_mode: int) -> int:
+    """Workspace bytes gdr_chunk_bwd needs (the fp32 state at every chunk start)."""
+    out = ctypes.c_size_t(0)
+    st = load().gdr_bwd_workspace_bytes(ctypes.byref(shape), int(chunk), int(gate_mode),
+                                        ctypes.byref(out))
+    if st != OK:
+        raise GdrError(st, "gdr_bwd_workspace_bytes")
+    return out.value
+
+
+def chunk_bwd(q, k, v, g, beta, S0, dO, dS_final=None, chunk=64, gate_mode=None, kernel="auto",
+              workspace=None, want_dS0=True, stream=None):
+    """Gradients of sum(dO * o) + sum(dS_final * S_final) of the chunkwise forward
+    (exact inverse) with respect to q, k, v, g, beta and S0.  Inputs as chunk_fwd;
+    dO [B,Hv,T,dv] and dS_final [B,Hv,dk,dv] (or None) fp32 CUDA tensors.  Returns a
+    dict of fp32 tensors with keys q, k, v, g, beta, S0 (None unless want_dS0)."""
+    import torch
+    B, Hk, T, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[3]
+    G = g.shape[-1]
+    if gate_mode is None:
+        gate_mode = gate_mode_for(G, dk)
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("S0", S0),
+                    ("dO", dO), ("dS_final", dS_final)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    if dO.dtype != torch.float32 or tuple(dO.shape) != (B, Hv, T, dv):
+        raise ValueError("dO must be an fp32 [B, Hv, T, dv] tensor")
+    if dS_final is not None and (dS_final.dtype != torch.float32 or
+                                 tuple(dS_final.shape) != (B, Hv, dk, dv)):
+        raise ValueError("dS_final must be an fp32 [B, Hv, dk, dv] tensor")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    grads = {"q": torch.empty((B, Hk, T, dk), **f32), "k": torch.empty((B, Hk, T, dk), **f32),
+             "v": torch.empty((B, Hv, T, dv), **f32), "g": torch.empty((B, Hk, T, G), **f32),
+             "beta": torch.empty((B, Hk, T), **f32),
+             "S0": torch.empty((B, Hv, dk, dv), **f32) if want_dS0 else None}
+    shape = make_shape(B, T, Hk, Hv, dk, dv, _dtype_code(q.dtype), F32, kernel=kernel)
+    if workspace is None:
+        nbytes = bwd_workspace_bytes(shape, chunk, gate_mode)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    st = load().gdr_chunk_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                              _ptr(S0), _ptr(dO), _ptr(dS_final), int(chunk), int(gate_mode),
+                              _ptr(grads["q"]), _ptr(grads["k"]), _ptr(grads["v"]),
+                              _ptr(grads["g"]), _ptr(grads["beta"]), _ptr(grads["S0"]),
+                              _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                              _stream_handle(stream))
+    if st != OK:
+        raise GdrError(st, "gdr_chunk_bwd")
+    return grads
 
 
 def output_gate_rmsnorm(o, z, weight=None, eps=1e-6, stream=None):

@@ -134,6 +134,42 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gdr_chunk_bwd -- gradients of the chunkwise forward (exact chunk inverse):
+ * given the upstream gradients dO of o and dS_final of S_final, the gradients
+ * of sum(dO * o) + sum(dS_final * S_final) with respect to every input
+ * ("Systolic Linear Attention: Co-Designing Tile-Grouped Gated Delta Attention
+ * for TPUs", §2.5: only the state at each chunk's start is kept, and a reverse
+ * scan over the chunks recomputes the chunk's factors from it).
+ * Device inputs (read only): q, k, v, g, beta, S0 as gdr_chunk_fwd (S0 may be
+ *   NULL: zero initial state);
+ *   dO       [B, Hv, T, dv]  fp32
+ *   dS_final [B, Hv, dk, dv] fp32, or NULL for zero
+ * Device outputs (written, fp32): dq, dk [B, Hk, T, dk]; dv [B, Hv, T, dv];
+ *   dg [B, Hk, T, G]; dbeta [B, Hk, T]; dS0 [B, Hv, dk, dv] or NULL to skip.
+ *   The key-side gradients (dq, dk, dg, dbeta) sum the contributions of all
+ *   value heads of a key head, added with fp32 atomics: their last bits may
+ *   differ from run to run.
+ * workspace: at least gdr_bwd_workspace_bytes (the fp32 state at the start of
+ *   every chunk, [B, Hv, ceil(T / chunk), dk, dv]); GDR_ERR_WORKSPACE if
+ *   smaller.  shape->in_dtype gives the dtype of q, k, v; out_dtype is unused.
+ * Runs on the CUDA cores (fp32): shape->kernel AUTO or SIMT (otherwise
+ * GDR_ERR_UNSUPPORTED, as for a request whose shared memory does not fit,
+ * e.g. dk = 256 with per-channel gates at chunk 128).  Asynchronous on
+ * `stream`.
+ */
+gdr_status gdr_chunk_bwd(const gdr_shape *shape,
+                         const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, const float *S0,
+                         const float *dO, const float *dS_final,
+                         int chunk, gdr_gate_mode gate_mode,
+                         float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                         float *dS0, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes gdr_chunk_bwd needs for this request (into *bytes). */
+gdr_status gdr_bwd_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
+                                   size_t *bytes);
+
+/*
  * gdr_chunk_fwd_momentum -- gdr_chunk_fwd with chunk-boundary momentum
  * ("Systolic Linear Attention: Co-Designing Tile-Grouped Gated Delta Attention
  * for TPUs", §2.3, the momentum update after Eq. (5)).  Each chunk's state

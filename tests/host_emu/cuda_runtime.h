@@ -11,7 +11,7 @@ using std::max;
 using std::min;
 typedef void *cudaStream_t;
 struct host_uint3 { unsigned x, y, z; };
-extern thread_local host_uint3 threadIdx, blockIdx;
+extern thread_local host_uint3 threadIdx, blockIdx, gridDim;
 #define __global__
 #define __device__
 #define __host__
@@ -19,3 +19,10 @@ extern thread_local host_uint3 threadIdx, blockIdx;
 #define __launch_bounds__(...)
 #define __shared__
 #define __syncthreads() ((void)0)
+/* one thread at a time: an atomic add is a plain add */
+inline float atomicAdd(float *a, float v)
+{
+    const float old = *a;
+    *a = old + v;
+    return old;
+}

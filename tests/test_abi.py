@@ -206,6 +206,42 @@ def test_momentum_validates(lib):
              None, None, None, None) == gdr.OK
 
 
+def test_backward_validates(lib):
+    # the backward: workspace size and host validation (nothing launches on these)
+    f = gdr.load().gdr_chunk_bwd
+    sh = gdr.make_shape(2, 100, 1, 2, 64, 48, in_dtype=gdr.F32, out_dtype=gdr.F32)
+    # the fp32 state at every chunk start: B Hv ceil(T / C) dk dv floats
+    assert gdr.bwd_workspace_bytes(sh, 32, gdr.GATE_SCALAR) == 4 * 2 * 2 * 4 * 64 * 48
+    assert gdr.bwd_workspace_bytes(sh, 100, gdr.GATE_CHANNEL) == 4 * 2 * 2 * 1 * 64 * 48
+
+    def call(shape, chunk=32, gate=gdr.GATE_SCALAR, ptrs=None, ws=None, ws_bytes=0):
+        ptrs = ptrs or [None] * 8
+        return f(ctypes.byref(shape), *ptrs, chunk, gate, *([None] * 6), ws, ws_bytes, None)
+
+    assert call(sh) == gdr.ERR_ARG                                  # tokens but no buffers
+    assert call(sh, chunk=129) == gdr.ERR_SHAPE
+    # fake but aligned device addresses: every call below fails validation first (on a
+    # machine without a GPU a launch would return GDR_ERR_CUDA and fail the test)
+    full = [ctypes.c_void_p(1 << 20)] * 8
+
+    def call_all(shape, chunk=32, gate=gdr.GATE_SCALAR, ws=None, ws_bytes=0, align=0):
+        outs = [ctypes.c_void_p((1 << 21) + align)] + [ctypes.c_void_p(1 << 21)] * 5
+        return f(ctypes.byref(shape), *full, chunk, gate, *outs, ws, ws_bytes, None)
+
+    need = gdr.bwd_workspace_bytes(sh, 32, gdr.GATE_SCALAR)
+    assert call_all(sh, ws=None) == gdr.ERR_WORKSPACE
+    assert call_all(sh, ws=ctypes.c_void_p(1 << 22), ws_bytes=need - 1) == gdr.ERR_WORKSPACE
+    assert call_all(sh, ws=ctypes.c_void_p(1 << 22), ws_bytes=need, align=4) == gdr.ERR_ALIGN
+    tc = gdr.make_shape(2, 100, 1, 2, 64, 48, kernel="tc2")
+    assert call_all(tc, ws=ctypes.c_void_p(1 << 22), ws_bytes=need) == gdr.ERR_UNSUPPORTED
+    # dk = 256 with per-channel gates at chunk 128 does not fit the backward's shared memory
+    wide = gdr.make_shape(1, 100, 1, 1, 256, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
+    assert call_all(wide, chunk=128, gate=gdr.GATE_CHANNEL, ws=ctypes.c_void_p(1 << 22),
+                    ws_bytes=1 << 30) == gdr.ERR_UNSUPPORTED
+    empty = gdr.make_shape(0, 100, 1, 2, 64, 48, in_dtype=gdr.F32, out_dtype=gdr.F32)
+    assert call(empty) == gdr.OK
+
+
 def test_state_segments(lib):
     # The two-pass state pass stays sequential while the value tiles of all
     # sequences fill the SMs, and cuts few long sequences into segments whose

@@ -1,5 +1,5 @@
-"""The CUDA-core kernel's own source (gdr_simt.cu) compiled for the host and
-compared with the oracle, without a GPU.
+"""The CUDA-core kernels' own source (the forward of gdr_simt.cu, the backward of
+gdr_bwd.cu) compiled for the host and compared with the oracle, without a GPU.
 
 The kernel is written as phases separated by __syncthreads(), each phase a loop
 `for (idx = tid; idx < n; idx += NT)`.  With NT = 1 and the barriers as no-ops
@@ -29,9 +29,9 @@ SMEM_FLOATS = 227 * 1024 // 4
 CANARY = 4096
 
 RUNNER = r'''
-}  // namespace host_emu
+}  // namespace host_emu_bwd
 }  // namespace gdr
-thread_local host_uint3 threadIdx, blockIdx;
+thread_local host_uint3 threadIdx, blockIdx, gridDim;
 static float host_smem[%(smem)d + %(canary)d];
 static const uint32_t kCanary = 0x7fc0dead;   // a NaN pattern
 
@@ -87,6 +87,48 @@ extern "C" int emu_run(const gdr::Params *p)
     const int NV = emu_tile(p);
     return NV == 32 ? run_nv<32>(*p) : NV == 16 ? run_nv<16>(*p) : -3;
 }
+
+// the backward kernel over its grid (the caller has run the forward for the
+// chunk-start states and zeroed the accumulated gradients)
+template <bool I, int NV>
+static int run_bwd_grid(const gdr::Params &p)
+{
+    const int total = gdr::host_emu_bwd::bwd_layout(p.C, p.G, p.dk, NV).total;
+    if (total > %(smem)d)
+        return -1;
+    for (unsigned b = 0; b < (unsigned)p.B; ++b)
+        for (unsigned h = 0; h < (unsigned)p.Hv; ++h)
+            for (unsigned x = 0; x < (unsigned)((p.dv + NV - 1) / NV); ++x) {
+                threadIdx = {0, 0, 0};
+                blockIdx = {x, h, b};
+                std::memset(host_smem, 0xff, sizeof(float) * total);
+                for (int c = 0; c < %(canary)d; ++c)
+                    std::memcpy(&host_smem[total + c], &kCanary, 4);
+                gdr::host_emu_bwd::simt_bwd_kernel<I, NV>(p);
+                for (int c = 0; c < %(canary)d; ++c)
+                    if (std::memcmp(&host_smem[total + c], &kCanary, 4) != 0)
+                        return -2;
+            }
+    return 0;
+}
+
+extern "C" int emu_bwd_tile(const gdr::Params *p)
+{
+    for (int NV : {32, 16})
+        if (gdr::host_emu_bwd::bwd_layout(p->C, p->G, p->dk, NV).total * 4 <= 227 * 1024)
+            return NV;
+    return 0;
+}
+
+extern "C" int emu_bwd(const gdr::Params *p)
+{
+    const int NV = emu_bwd_tile(p);
+    if (NV == 32)
+        return p->in_bf16 ? run_bwd_grid<true, 32>(*p) : run_bwd_grid<false, 32>(*p);
+    if (NV == 16)
+        return p->in_bf16 ? run_bwd_grid<true, 16>(*p) : run_bwd_grid<false, 16>(*p);
+    return -3;
+}
 '''
 
 
@@ -96,19 +138,28 @@ class Params(ctypes.Structure):
                  "B T Hk Hv dk dv G C R in_bf16 out_bf16 neumann neumann1 neu_order neu_resid "
                  "momentum".split()] +
                 [("mu", ctypes.c_float), ("kappa", ctypes.c_void_p)] +
-                [(n, ctypes.c_void_p) for n in "q k v g beta S0 o S_final".split()])
+                [(n, ctypes.c_void_p) for n in
+                 "q k v g beta S0 o S_final S_chunks dO dS_final grad_q grad_k grad_v grad_g "
+                 "grad_beta grad_S0".split()])
 
 
 @pytest.fixture(scope="module")
 def emu(tmp_path_factory):
-    src = open(os.path.join(CSRC, "gdr_simt.cu")).read()
-    cut = src.index("template <bool I, bool O, int NV, bool MOM>\nint launch_variant")
-    body = src[:cut]
-    for old, new in (("constexpr int NT = 256;", "constexpr int NT = 1;"),
-                     ("namespace {", "namespace host_emu {"),
-                     ("extern __shared__ float sm[];", "float *const sm = host_smem_ptr();")):
-        assert body.count(old) == 1, old
-        body = body.replace(old, new)
+    def kernel_part(name, marker, ns):
+        src = open(os.path.join(CSRC, name)).read()
+        body = src[:src.index(marker)]
+        for old, new in (("constexpr int NT = 256;", "constexpr int NT = 1;"),
+                         ("namespace {", "namespace %s {" % ns),
+                         ("extern __shared__ float sm[];", "float *const sm = host_smem_ptr();")):
+            assert body.count(old) == 1, old
+            body = body.replace(old, new)
+        return body
+
+    fwd = kernel_part("gdr_simt.cu", "template <bool I, bool O, int NV, bool MOM>\nint launch_variant",
+                      "host_emu")
+    bwd = kernel_part("gdr_bwd.cu", "template <bool I, int NV>\nint launch_bwd_variant", "host_emu_bwd")
+    # each part ends inside `namespace gdr { namespace ... {`; close the first
+    body = fwd + "}  // namespace host_emu\n}  // namespace gdr\n" + bwd
     head = "float *host_smem_ptr();\n"
     tail = RUNNER % {"smem": SMEM_FLOATS, "canary": CANARY} + "float *host_smem_ptr() { return host_smem; }\n"
     d = tmp_path_factory.mktemp("host_emu")
@@ -121,6 +172,8 @@ def emu(tmp_path_factory):
     lib = ctypes.CDLL(str(so))
     lib.emu_run.argtypes = [ctypes.POINTER(Params)]
     lib.emu_tile.argtypes = [ctypes.POINTER(Params)]
+    lib.emu_bwd.argtypes = [ctypes.POINTER(Params)]
+    lib.emu_bwd_tile.argtypes = [ctypes.POINTER(Params)]
     return lib
 
 
@@ -194,7 +247,7 @@ CASES = [
 def test_host_kernel_matches_oracle(emu, case):
     T, Hk, Hv, dk, dv, G, chunk, inverse, order, resid, with_s0 = case
     rng = np.random.default_rng(zlib.crc32(repr(case).encode()))
-    q, k, v, g, beta, S0 = P.rand_inputs(rng, 1, T, Hk, Hv // Hk, dk, dv, G)
+    q, k, v, g, beta, S0 = P.rand_inputs(rng, 1, T, Hk, Hv, dk, dv, G)
     x = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "S0": S0 if with_s0 else None}
     o, S = run_host(emu, x, chunk, inverse, order, resid)
     args = (x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
@@ -223,3 +276,69 @@ def test_host_kernel_bf16_io(emu):
     o_ref, S_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
     assert rel(S, S_ref) <= 1e-5
     assert rel(o, o_ref) <= 2.0 ** -8
+
+
+def run_host_bwd(lib, x, chunk, dO, dSf, bf16=False):
+    """The library's backward on the host: the forward kernel for the chunk-start
+    states (no outputs), then the backward kernel; returns the gradients."""
+    q = x["q"]
+    B, Hk, T, dk = q.shape
+    Hv, dv, G = x["v"].shape[1], x["v"].shape[3], x["g"].shape[3]
+    conv = _bf16_bits if bf16 else (lambda a: np.ascontiguousarray(a, np.float32))
+    qq, kk, vv = conv(x["q"]), conv(x["k"]), conv(x["v"])
+    g = np.ascontiguousarray(x["g"], np.float32)
+    beta = np.ascontiguousarray(x["beta"], np.float32)
+    S0 = None if x["S0"] is None else np.ascontiguousarray(x["S0"], np.float32)
+    nch = (T + chunk - 1) // chunk
+    guard = 64
+    f32 = lambda n: np.full(n + 2 * guard, 12345.0, np.float32)
+    Sc = f32(B * Hv * nch * dk * dv)
+    outs = {"q": (B, Hk, T, dk), "k": (B, Hk, T, dk), "v": (B, Hv, T, dv), "g": (B, Hk, T, G),
+            "beta": (B, Hk, T), "S0": (B, Hv, dk, dv)}
+    bufs = {n: f32(int(np.prod(s))) for n, s in outs.items()}
+    for n in ("q", "k", "g", "beta"):       # accumulated: the library zeroes them first
+        bufs[n][guard:-guard] = 0.0
+    dO32 = np.ascontiguousarray(dO, np.float32)
+    dS32 = None if dSf is None else np.ascontiguousarray(dSf, np.float32)
+    ptr = lambda a, off=0: None if a is None else a.ctypes.data + off * a.itemsize
+    p = Params(B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, G=G, C=chunk, R=Hv // Hk,
+               in_bf16=int(bf16), out_bf16=0, neumann=0, neumann1=0, neu_order=0, neu_resid=0,
+               momentum=0, mu=0.0, kappa=None, q=ptr(qq), k=ptr(kk), v=ptr(vv), g=ptr(g),
+               beta=ptr(beta), S0=ptr(S0), o=None, S_final=None, S_chunks=ptr(Sc, guard))
+    assert lib.emu_run(ctypes.byref(p)) == 0
+    p.S_chunks = ptr(Sc, guard)
+    p.dO, p.dS_final = ptr(dO32), ptr(dS32)
+    p.grad_q, p.grad_k, p.grad_v = ptr(bufs["q"], guard), ptr(bufs["k"], guard), ptr(bufs["v"], guard)
+    p.grad_g, p.grad_beta, p.grad_S0 = ptr(bufs["g"], guard), ptr(bufs["beta"], guard), ptr(bufs["S0"], guard)
+    assert lib.emu_bwd_tile(ctypes.byref(p)) in (16, 32)
+    rc = lib.emu_bwd(ctypes.byref(p))
+    assert rc == 0, "host backward failed (%d: -2 = shared-memory canary overwritten)" % rc
+    for buf in [Sc] + list(bufs.values()):
+        assert np.all(buf[:guard] == 12345.0) and np.all(buf[-guard:] == 12345.0)
+    return {n: bufs[n][guard:-guard].reshape(s).astype(np.float64) for n, s in outs.items()}
+
+
+# (T, Hk, Hv, dk, dv, G, chunk, with S0, with dS_final)
+BWD_CASES = [
+    (37, 1, 2, 32, 48, 1, 16, True, True),      # ragged tail, two value heads, two value tiles
+    (70, 1, 1, 64, 32, 64, 32, True, False),    # per-channel decay
+    (45, 2, 4, 64, 20, 1, 64, False, True),     # one short chunk, dv not a multiple of 8
+    (50, 1, 1, 128, 16, 2, 16, True, True),     # 64-channel groups
+    (9, 1, 1, 16, 8, 16, 1, True, True),        # chunks of one token
+    (0, 1, 1, 32, 32, 1, 64, True, True),       # no tokens: dS0 = dS_final
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=["T%d-R%d-dk%d-dv%d-G%d-C%d" % (c[0], c[2] // c[1], c[3], c[4], c[5], c[6])
+                                                 for c in BWD_CASES])
+def test_host_backward_matches_oracle(emu, case):
+    T, Hk, Hv, dk, dv, G, chunk, with_s0, with_dsf = case
+    rng = np.random.default_rng(zlib.crc32(repr(case).encode()))
+    q, k, v, g, beta, S0 = P.rand_inputs(rng, 1, T, Hk, Hv, dk, dv, G)
+    x = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "S0": S0 if with_s0 else None}
+    dO = rng.standard_normal((1, Hv, T, dv))
+    dSf = rng.standard_normal((1, Hv, dk, dv)) if with_dsf else None
+    got = run_host_bwd(emu, x, chunk, dO, dSf)
+    ref = oracle.recurrent_grad(q, k, v, g, beta, x["S0"], dO, dSf)
+    for n in ("q", "k", "v", "g", "beta", "S0"):
+        assert rel(got[n], ref[n]) <= 1e-4, (n, rel(got[n], ref[n]))
