@@ -20,6 +20,9 @@ chunks) with inputs resident in HBM.  Prints ONE JSON line on rank 0.
   of the same workload (rank 0, N = 1 only).
 * --impl reference: the oracle alone on the host cores (a bounded sample per
   step), the only comparison arm this method has.
+* --pass backward / --momentum MU: the same line for gdr_chunk_bwd (seeded
+  upstream gradients) or gdr_chunk_fwd_momentum (seeded per-chunk kappa), both
+  CUDA-core kernels; their roofline is fp32 FMA issue ("alu").
 """
 from __future__ import annotations
 
@@ -44,6 +47,8 @@ METRIC = "tokens/s and TFLOP/s (% of bf16 TC peak) for chunkwise gated-delta fwd
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA issue on the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz (max SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse_args():
@@ -61,6 +66,10 @@ def parse_args():
     ap.add_argument("--epilogue", action="store_true",
                     help="add the readout epilogue (output gate times per-value-head RMSNorm, "
                          "unit weight) to every step, device-timed and end to end")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="backward: time gdr_chunk_bwd (exact inverse; seeded upstream gradients)")
+    ap.add_argument("--momentum", type=float, default=None,
+                    help="time gdr_chunk_fwd_momentum with this mu (seeded 0/1 kappa per chunk)")
     return ap.parse_args()
 
 
@@ -279,6 +288,201 @@ def config_dict(w, chunk, inverse, world):
                    else "L2 flushed between steps")}
 
 
+def oracle_variant_sample(w, x, chunk, up, mu, kappa, budget_s=12.0, t_cap=256):
+    """The oracle on a bounded sample for the backward (recurrent_grad over whole key
+    heads, the first t_cap tokens: it keeps every token's state) or for momentum
+    (the chunked form with momentum, whole sequences).  Returns (tokens/s, threads,
+    description)."""
+    import oracle
+    threads = max(1, oracle.max_threads())
+
+    def run(n):
+        heads = [(s // w.Hk, s % w.Hk) for s in range(n)]
+        vh = lambda b, hk: [x_ for x_ in range(hk * w.R, (hk + 1) * w.R)]
+        T = min(w.T, t_cap) if up is not None else w.T
+        key = lambda name: np.stack([x[name][b, hk, :T] for b, hk in heads])[:, None]
+        val = lambda arr: np.stack([arr[b, vh(b, hk), :T] for b, hk in heads])
+        q, k, g, beta = key("q"), key("k"), key("g"), key("beta")
+        v = val(x["v"])
+        S0 = None if x["S0"] is None else np.stack([x["S0"][b, vh(b, hk)] for b, hk in heads])
+        t0 = time.perf_counter()
+        if up is not None:
+            oracle.recurrent_grad(q, k, v, g, beta, S0, val(up[0]), None, nthreads=threads)
+        else:
+            kap = None if kappa is None else np.stack([kappa[b] for b, _ in heads])
+            oracle.chunked(q, k, v, g, beta, S0, chunk=chunk, mu=mu, kappa=kap, nthreads=threads)
+        return time.perf_counter() - t0, T
+
+    total = w.B * w.Hk
+    n = min(total, threads)
+    dt, T = run(n)
+    want = int(n * max(1.0, budget_s / max(dt, 1e-3)))
+    n2 = min(total, max(n, (want // threads) * threads))
+    if n2 > n:
+        (dt, T), n = run(n2), n2
+    tokens = n * T / w.Hk
+    what = ("fp64 recurrent_grad (reverse sweep), first %d tokens" % T if up is not None
+            else "fp64 chunked form with momentum, all %d tokens" % T)
+    return tokens / dt, threads, "%d of %d (batch, key-head) sequences with their %d value heads, %s" % (
+        n, total, w.R, what)
+
+
+def run_variant(args, w, chunk, rank, world, local):
+    """--pass backward (gdr_chunk_bwd) or --momentum MU (gdr_chunk_fwd_momentum): the
+    same timing rules and JSON line as the forward, for these CUDA-core paths."""
+    import torch
+    from gated_delta_rule_141_b200 import gdr
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    backward = args.which == "backward"
+    x = W.make_inputs(w, rank_seed(args.workload, rank))
+    dt_in = torch.bfloat16 if w.in_dtype == "bf16" else torch.float32
+    dev = {n: torch.from_numpy(x[n]).to("cuda").to(dt_in) for n in ("q", "k", "v")}
+    dev["g"] = torch.from_numpy(x["g"]).cuda()
+    dev["beta"] = torch.from_numpy(x["beta"]).cuda()
+    dev["S0"] = None if x["S0"] is None else torch.from_numpy(x["S0"]).cuda()
+    rng = np.random.default_rng(7200 + args.workload + 7919 * rank)
+    up, kappa = None, None
+    if backward:   # upstream gradients ~ N(0, 1)
+        up = (rng.standard_normal((w.B, w.Hv, w.T, w.dv)).astype(np.float32),
+              rng.standard_normal((w.B, w.Hv, w.dk, w.dv)).astype(np.float32))
+        dev["dO"], dev["dS_final"] = torch.from_numpy(up[0]).cuda(), torch.from_numpy(up[1]).cuda()
+    else:          # kappa: 0 with probability 1/8 per chunk (a document reset inside it)
+        kappa = (rng.random((w.B, (w.T + chunk - 1) // chunk)) >= 0.125).astype(np.int32)
+        dev["kappa"] = torch.from_numpy(kappa).cuda()
+    shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
+                           gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                           gdr.BF16 if w.in_dtype == "bf16" else gdr.F32, kernel="simt")
+    gm = gdr.gate_mode_for(w.G, w.dk)
+    ws = None
+    if backward:
+        nb = gdr.bwd_workspace_bytes(shape, chunk, gm)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
+    in_bytes = sum(t.numel() * t.element_size() for t in dev.values() if t is not None)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if in_bytes < L2_BYTES else None
+    stream = torch.cuda.current_stream()
+    out = {}
+
+    def call(d):
+        if backward:
+            out["g"] = gdr.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], d["dO"],
+                                     d["dS_final"], chunk=chunk, gate_mode=gm, kernel="simt",
+                                     workspace=ws, stream=stream)
+        else:
+            out["o"] = gdr.chunk_fwd_momentum(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
+                                              mu=args.momentum, kappa=d["kappa"], chunk=chunk,
+                                              gate_mode=gm, kernel="simt", stream=stream)
+
+    step_events = []
+
+    def step(timed=False):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call(dev)
+        e1.record(stream)
+        if timed:
+            step_events.append((e0, e1))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier()
+        for _ in range(args.steps):
+            step(timed=True)
+        barrier()
+    ms_step = max_over_ranks(sum(a.elapsed_time(b) for a, b in step_events), dist,
+                             torch.device("cuda", local)) / args.steps
+    tokens_step = w.B * w.T
+    value = job_tokens_per_s(world, tokens_step, ms_step)
+    flop, byts = algorithmic(w, chunk, "exact")
+    if backward:   # the forward recomputed once, its chunk products run backwards twice
+        flop *= 3
+        byts = 2 * byts + 4 * w.B * w.Hv * w.T * w.dv * 2 + 4 * w.B * w.Hk * w.T * (2 * w.dk + w.G + 1)
+    achieved = flop / (ms_step * 1e-3) / 1e12
+    roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+            "frac": achieved / FP32_ALU_TFLOPS, "traffic": None,
+            "peak_source": "fp32 FMA on the CUDA cores from unit counts and the max SM clock",
+            "kernel": "simt", "hbm_gbs": byts / (ms_step * 1e-3) / 1e9}
+    # kernels launched per step: backward = forward recompute, 4 zero fills, the backward
+    launches = 6 if backward else 1
+
+    e2e = None
+    if not args.no_e2e:
+        host = {n: (None if t is None else t.cpu().pin_memory()) for n, t in dev.items()}
+        dbuf = {n: (None if t is None else torch.empty_like(t)) for n, t in dev.items()}
+        h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+        if backward:
+            res = {n: torch.empty(tuple(t.shape), dtype=torch.float32).pin_memory()
+                   for n, t in gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                                             dev["S0"], dev["dO"], dev["dS_final"], chunk=chunk,
+                                             gate_mode=gm, kernel="simt", workspace=ws,
+                                             stream=stream).items() if t is not None}
+        else:
+            res = {"o": torch.empty((w.B, w.Hv, w.T, w.dv), dtype=dt_in).pin_memory(),
+                   "S_final": torch.empty((w.B, w.Hv, w.dk, w.dv), dtype=torch.float32).pin_memory()}
+        d2h = sum(t.numel() * t.element_size() for t in res.values())
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for n in dev:
+                    if host[n] is not None:
+                        dbuf[n].copy_(host[n], non_blocking=True)
+                call(dbuf)
+                got = out["g"] if backward else dict(zip(("o", "S_final"), out["o"]))
+                for n, t in res.items():
+                    t.copy_(got[n], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        ev0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        ev1.record(stream)
+        barrier()
+        ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), dist, torch.device("cuda", local)) / n_e2e
+        e2e = {"value": job_tokens_per_s(world, tokens_step, ms_e2e), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, desc = oracle_variant_sample(w, x, chunk, up, args.momentum, kappa)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    what = "backward (gdr_chunk_bwd)" if backward else "forward with momentum mu=%g" % args.momentum
+    line = {
+        "metric": "tokens/s of the chunkwise gated-delta %s, CUDA-core kernels" % what,
+        "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
+        "config": dict(config_dict(w, chunk, "exact", world), which=what, kernel="simt"),
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps * launches, "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -288,6 +492,8 @@ def main():
     chunk = args.chunk or w.chunk
     if args.impl == "reference":
         return run_reference(args, w, chunk, rank)
+    if args.which == "backward" or args.momentum is not None:
+        return run_variant(args, w, chunk, rank, world, local)
 
     import torch
     from gated_delta_rule_141_b200 import gdr
