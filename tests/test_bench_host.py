@@ -1,0 +1,46 @@
+"""bench.py's host side on CPU: the reference arm's JSON line carries the keys of
+the bench contract, and the oracle samples of the backward and momentum modes
+run on a bounded slice of the workload."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from gated_delta_rule_141_b200 import workloads as W  # noqa: E402
+
+
+def test_reference_arm_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "0", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e", "impl"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 2
+    assert d["config"]["workload"] == W.WORKLOADS[0].name
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_variant_oracle_samples():
+    w = W.WORKLOADS[0]
+    x = W.make_inputs(w, bench.rank_seed(0, 0))
+    rng = np.random.default_rng(3)
+    up = (rng.standard_normal((w.B, w.Hv, w.T, w.dv)).astype(np.float32), None)
+    rate, threads, desc = bench.oracle_variant_sample(w, x, 64, up, None, None, budget_s=0.2)
+    assert rate > 0 and threads >= 1 and "recurrent_grad" in desc
+    kappa = np.ones((w.B, (w.T + 63) // 64), np.int32)
+    rate, threads, desc = bench.oracle_variant_sample(w, x, 64, None, 0.25, kappa, budget_s=0.2)
+    assert rate > 0 and "momentum" in desc
