@@ -74,3 +74,32 @@ def test_momentum_zero_is_plain_forward():
     torch.cuda.synchronize()
     assert U.rel_err(o1.cpu().numpy(), o2.cpu().numpy()) <= 1e-6
     assert U.rel_err(S1.cpu().numpy(), S2.cpu().numpy()) <= 1e-6
+
+
+def test_momentum_full_size_sampled():
+    # the gdn_scalar_bf16 workload at full size (B=4, H=16, T=4096, dk=dv=128) with the
+    # pages' mu = 0.25 and a seeded kappa, in the launch bench.py --momentum times;
+    # checked on a sample of sequences against the oracle
+    import torch
+    from gated_delta_rule_141_b200 import gdr
+    w, x = W.workload_inputs(1)
+    chunk, mu = w.chunk, 0.25
+    kappa = _kappa(w.B, w.T, chunk, 9100)
+    dev = U.to_device(x, w.in_dtype)
+    o, Sf = gdr.chunk_fwd_momentum(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
+                                   mu=mu, kappa=torch.from_numpy(kappa).to("cuda"), chunk=chunk,
+                                   kernel="simt")
+    torch.cuda.synchronize()
+    o = o.float().cpu().numpy().astype(np.float64)
+    Sf = Sf.cpu().numpy().astype(np.float64)
+    assert np.isfinite(o).all() and np.isfinite(Sf).all()
+    seqs = U.sample_sequences(w)
+    xs = U.slice_sequences(x, w.R, seqs)
+    kap = np.stack([kappa[b] for b, _ in seqs])
+    o_ref, S_ref = oracle.chunked(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["S0"],
+                                  chunk=chunk, inverse="exact", mu=mu, kappa=kap)
+    ib, ih = [b for b, _ in seqs], [h for _, h in seqs]
+    eo = U.rel_err(o[ib, ih][:, None], o_ref)
+    es = U.rel_err(Sf[ib, ih][:, None], S_ref)
+    print("rel err o %.3e  S_final %.3e" % (eo, es))
+    assert eo <= U.TOL_BF16 and es <= U.TOL_BF16

@@ -65,3 +65,34 @@ def test_backward_matches_exact_gradient(idx, over, chunk, with_dsf, with_s0):
     errs = {n: U.rel_err(got[n].cpu().numpy(), ref[n]) for n in ref}
     print(" ".join("d%s %.2e" % kv for kv in errs.items()))
     assert max(errs.values()) <= TOL, errs
+
+
+def test_backward_full_size_sampled():
+    # the gdn_scalar_bf16 workload at full size (B=4, H=16, T=4096, dk=dv=128), the
+    # launch bench.py --pass backward times; the oracle's gradient for a sample of
+    # key heads (with all their value heads) against the GPU's
+    import torch
+    from gated_delta_rule_141_b200 import gdr
+    w, x = W.workload_inputs(1)
+    dO, dSf = upstream(x, 7190, True)
+    dev = U.to_device(x, w.in_dtype)
+    got = gdr.chunk_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
+                        torch.from_numpy(dO.astype(np.float32)).to("cuda"),
+                        torch.from_numpy(dSf.astype(np.float32)).to("cuda"), chunk=w.chunk)
+    torch.cuda.synchronize()
+    got = {n: t.cpu().numpy().astype(np.float64) for n, t in got.items()}
+    for n, t in got.items():
+        assert np.isfinite(t).all(), n
+    heads = [(0, 0), (w.B - 1, w.Hk - 1)]              # (batch, key head)
+    for b, hk in heads:
+        hv = list(range(hk * w.R, (hk + 1) * w.R))
+        key = lambda a: a[b:b + 1, hk:hk + 1]
+        val = lambda a: a[b:b + 1, hv]
+        ref = oracle.recurrent_grad(key(x["q"]), key(x["k"]), val(x["v"]), key(x["g"]),
+                                    key(x["beta"]), None if x["S0"] is None else val(x["S0"]),
+                                    val(dO), val(dSf))
+        errs = {"q": U.rel_err(key(got["q"]), ref["q"]), "k": U.rel_err(key(got["k"]), ref["k"]),
+                "g": U.rel_err(key(got["g"]), ref["g"]), "beta": U.rel_err(key(got["beta"]), ref["beta"]),
+                "v": U.rel_err(val(got["v"]), ref["v"]), "S0": U.rel_err(val(got["S0"]), ref["S0"])}
+        print((b, hk), " ".join("d%s %.2e" % kv for kv in errs.items()))
+        assert max(errs.values()) <= TOL, errs
