@@ -10,9 +10,11 @@ only marshals numpy arrays.  Citations for each routine are in the C source:
 the token recurrence follows "Systolic Linear Attention: Co-Designing
 Tile-Grouped Gated Delta Attention for TPUs" §2.1 Eq. (2); the chunkwise WY
 form follows its §2.3 Table 2 and §2.4.2, its 1-Step Neumann block inverse
-§2.4.3; the truncated Neumann inverse follows "When Good Enough Is Optimal:
-Multiplication-Only Matrix Inversion Approximation for Quantized Gated DeltaNet"
-(Lemma 3.1, §4.1).
+§2.4.3, chunk-boundary momentum and the readout epilogue §2.3, and the gradient
+(``recurrent_grad``) is the exact derivative of the token recurrence that the
+backward of its §2.5 must reproduce; the truncated Neumann inverse follows "When
+Good Enough Is Optimal: Multiplication-Only Matrix Inversion Approximation for
+Quantized Gated DeltaNet" (Lemma 3.1, §4.1).
 
 Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
 closed forms, invariants and hand-worked examples in ``tests/golden/``.

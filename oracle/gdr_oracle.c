@@ -25,6 +25,16 @@
  *   o      [B, Hv, T, dv]      output o_t = S_t^T q_t (post-update state)
  *   S_final[B, Hv, dk, dv]     state after the last token
  *
+ * Routines: gdro_recurrent (the definition: token recurrence), gdro_chunked
+ * (the chunkwise WY form with the exact, truncated-Neumann or 1-Step Neumann
+ * inverse), gdro_chunked_momentum (the same with chunk-boundary momentum,
+ * [SLA] §2.3), gdro_recurrent_grad (the exact gradient of the token recurrence,
+ * a reverse sweep: what a backward, [SLA] §2.5, must reproduce), the chunk
+ * inverses alone (gdro_tril_inverse, gdro_neumann_inverse,
+ * gdro_block_neumann1_inverse), the chunk's factor matrices
+ * (gdro_chunk_matrices) and the readout epilogue (gdro_output_gate_rmsnorm,
+ * [SLA] §2.3 Eq. (5)).
+ *
  * Every function returns 0 on success and a negative code on a bad argument.
  */
 #include <math.h>
