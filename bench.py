@@ -60,7 +60,7 @@ def parse_args():
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--inverse", default="exact", choices=["exact", "neumann", "neumann1"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "simt"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "simt", "simt2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--epilogue", action="store_true",
@@ -527,7 +527,8 @@ def main():
     kern = gdr.select_kernel(shape_run, chunk, gm_run, args.inverse)
     # the two-pass path: pass 1, then one state pass, or three when segmented
     nseg = gdr.state_segments(shape_run, chunk, gm_run, args.inverse) if kern == gdr.KERNEL_TC2 else 0
-    launches_per_step = (1 + (1 if nseg == 1 else 3)) if kern == gdr.KERNEL_TC2 else 1
+    launches_per_step = ((1 + (1 if nseg == 1 else 3)) if kern == gdr.KERNEL_TC2
+                         else 2 if kern == gdr.KERNEL_SIMT2 else 1)
     zgate = None
     if args.epilogue:   # output-gate logits z ~ N(0, 1), seeded apart from the workload's draws
         zr = np.random.default_rng(7000 + args.workload).standard_normal(tuple(o.shape)).astype(np.float32)

@@ -25,7 +25,7 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
     if (s->out_dtype != GDR_F32 && s->out_dtype != GDR_BF16)
         return GDR_ERR_DTYPE;
     if (s->kernel != GDR_KERNEL_AUTO && s->kernel != GDR_KERNEL_SIMT && s->kernel != GDR_KERNEL_TC &&
-        s->kernel != GDR_KERNEL_TC2)
+        s->kernel != GDR_KERNEL_TC2 && s->kernel != GDR_KERNEL_SIMT2)
         return GDR_ERR_ARG;
     if (s->B < 0 || s->T < 0 || s->Hk < 1 || s->Hv < 1 || s->Hv % s->Hk != 0)
         return GDR_ERR_SHAPE;
@@ -62,8 +62,9 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
     return GDR_OK;
 }
 
-// GDR_KERNEL_SIMT / GDR_KERNEL_TC / GDR_KERNEL_TC2, or -status, for a call
-// that brings `ws_bytes` of workspace (SIZE_MAX: as much as TC2 asks for).
+// GDR_KERNEL_SIMT / GDR_KERNEL_TC / GDR_KERNEL_TC2 / GDR_KERNEL_SIMT2 (forced
+// only), or -status, for a call that brings `ws_bytes` of workspace (SIZE_MAX:
+// as much as the kernel asks for).
 int choose(const gdr::Params &p, gdr_kernel want, size_t ws_bytes)
 {
     const bool tc2 = gdr::tc2_supports(p);
@@ -77,6 +78,10 @@ int choose(const gdr::Params &p, gdr_kernel want, size_t ws_bytes)
         return tc2_fits ? GDR_KERNEL_TC2 : -GDR_ERR_WORKSPACE;
     case GDR_KERNEL_TC: return tc ? GDR_KERNEL_TC : -GDR_ERR_UNSUPPORTED;
     case GDR_KERNEL_SIMT: return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
+    case GDR_KERNEL_SIMT2:
+        if (!gdr::simt2_supports(p))
+            return -GDR_ERR_UNSUPPORTED;
+        return ws_bytes >= gdr::simt2_workspace_bytes(p) ? GDR_KERNEL_SIMT2 : -GDR_ERR_WORKSPACE;
     default: break;
     }
     if (tc2_fits)
@@ -116,6 +121,8 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, c
     int rc;
     if (which == GDR_KERNEL_TC2)
         rc = gdr::launch_tc2(p, workspace, s);
+    else if (which == GDR_KERNEL_SIMT2)
+        rc = gdr::launch_simt2(p, workspace, s);
     else if (which == GDR_KERNEL_TC)
         rc = gdr::launch_tc(p, s);
     else
@@ -214,7 +221,9 @@ gdr_status gdr_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode 
     const int which = choose(p, shape->kernel, SIZE_MAX);
     if (which < 0)
         return static_cast<gdr_status>(-which);
-    *bytes = which == GDR_KERNEL_TC2 ? gdr::tc2_workspace_bytes(p) : 0;
+    *bytes = which == GDR_KERNEL_TC2     ? gdr::tc2_workspace_bytes(p)
+             : which == GDR_KERNEL_SIMT2 ? gdr::simt2_workspace_bytes(p)
+                                         : 0;
     return GDR_OK;
 }
 
@@ -316,7 +325,7 @@ int gdr_kernel_chunk(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
     const int which = choose(p, shape->kernel, SIZE_MAX);
     if (which < 0)
         return which;
-    return which == GDR_KERNEL_SIMT ? p.C : gdr::tc_kernel_chunk(p);
+    return (which == GDR_KERNEL_SIMT || which == GDR_KERNEL_SIMT2) ? p.C : gdr::tc_kernel_chunk(p);
 }
 
 int gdr_state_segments(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,

@@ -27,6 +27,7 @@ struct Params {
     void *o;          // may be nullptr for the CUDA-core kernel (states only)
     float *S_final;
     float *S_chunks;  // CUDA-core kernel: [B][Hv][ceil(T/C)][dk][dv] state at each chunk's start, or nullptr
+    const float *factors;  // two-pass CUDA-core form: [B][Hk][ceil(T/C)][2][C][C] (inverse, L) records
     // backward (gdr_chunk_bwd): upstream gradients in, gradients out (fp32)
     const float *dO, *dS_final;
     float *grad_q, *grad_k, *grad_v, *grad_g, *grad_beta, *grad_S0;
@@ -41,6 +42,11 @@ int read_and_clear_device_status();
 // code if the request does not fit the kernel's shared-memory budget.
 int simt_smem_bytes(const Params &p);
 int launch_simt(const Params &p, cudaStream_t stream);
+// Two-pass CUDA-core form: the chunk inverse and L of every chunk in parallel
+// (into a workspace), then the value tiles' pass over the chunks.
+bool simt2_supports(const Params &p);
+size_t simt2_workspace_bytes(const Params &p);
+int launch_simt2(const Params &p, void *workspace, cudaStream_t stream);
 
 // Backward of the chunked forward (exact inverse), CUDA cores, fp32: the states
 // at the chunk starts are recomputed by the forward kernel into the workspace,

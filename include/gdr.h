@@ -85,11 +85,16 @@ typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1, GDR_INV_NEUMANN1 = 2 } gd
  *        chunk 64, or 128 in exact mode).  Needs gdr_workspace_bytes() of
  *        device workspace.
  *  SIMT  the fp32 CUDA-core kernel (any dtype, chunk 1..128).
+ *  SIMT2 the same arithmetic in two passes: the chunk inverse and score matrix
+ *        L of every chunk in parallel, written to the caller's workspace
+ *        (2 C^2 fp32 per (batch, key head, chunk); gdr_workspace_bytes), then
+ *        the value tiles' pass over the chunks that reads them.  Only when
+ *        forced; any dtype, chunk 1..128, every inverse mode.
  *  AUTO  TC2 when it applies and the call's workspace is large enough, else
  *        TC when it applies, else SIMT.  Forcing a kernel outside its
  *        envelope fails with GDR_ERR_UNSUPPORTED.                           */
 typedef enum { GDR_KERNEL_AUTO = 0, GDR_KERNEL_SIMT = 1, GDR_KERNEL_TC = 2,
-               GDR_KERNEL_TC2 = 3 } gdr_kernel;
+               GDR_KERNEL_TC2 = 3, GDR_KERNEL_SIMT2 = 4 } gdr_kernel;
 
 typedef struct {
     int B;      /* batch, >= 0                                               */
@@ -291,8 +296,9 @@ gdr_status gdr_chunk_fwd_static(const gdr_shape *shape,
                                 void *o, float *S_final, void *stream);
 
 /* Which kernel gdr_chunk_fwd would launch for this request when given the
- * workspace gdr_workspace_bytes asks for: GDR_KERNEL_SIMT, GDR_KERNEL_TC or
- * GDR_KERNEL_TC2, or a negative gdr_status value if it would be rejected. */
+ * workspace gdr_workspace_bytes asks for: GDR_KERNEL_SIMT, GDR_KERNEL_TC,
+ * GDR_KERNEL_TC2 or GDR_KERNEL_SIMT2, or a negative gdr_status value if it
+ * would be rejected. */
 int gdr_select_kernel(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
                       gdr_inverse_mode inverse_mode);
 

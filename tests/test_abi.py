@@ -49,8 +49,8 @@ def test_enums_match_header():
         gdr.GATE_SCALAR, gdr.GATE_GROUP64, gdr.GATE_CHANNEL)
     assert (val("GDR_INV_EXACT"), val("GDR_INV_NEUMANN")) == (gdr.INV_EXACT, gdr.INV_NEUMANN)
     assert (val("GDR_KERNEL_AUTO"), val("GDR_KERNEL_SIMT"), val("GDR_KERNEL_TC"),
-            val("GDR_KERNEL_TC2")) == (gdr.KERNEL_AUTO, gdr.KERNEL_SIMT, gdr.KERNEL_TC,
-                                       gdr.KERNEL_TC2)
+            val("GDR_KERNEL_TC2"), val("GDR_KERNEL_SIMT2")) == (
+        gdr.KERNEL_AUTO, gdr.KERNEL_SIMT, gdr.KERNEL_TC, gdr.KERNEL_TC2, gdr.KERNEL_SIMT2)
     # struct layout: 11 ints
     assert ctypes.sizeof(gdr.GdrShape) == 44
 
@@ -204,6 +204,26 @@ def test_momentum_validates(lib):
              None, None, None, None) == gdr.ERR_UNSUPPORTED
     assert f(ctypes.byref(wide), *nul, 64, gdr.GATE_CHANNEL, gdr.INV_EXACT, ctypes.c_float(0.5),
              None, None, None, None) == gdr.OK
+
+
+def test_two_pass_simt_selection(lib):
+    # the two-pass CUDA-core form runs only when forced; its workspace holds the
+    # chunk inverse and L of every chunk (2 C^2 fp32 each)
+    sh = gdr.make_shape(2, 1000, 8, 32, 256, 128, kernel="simt2")
+    assert gdr.select_kernel(sh, 128, gdr.GATE_GROUP64, "neumann") == gdr.KERNEL_SIMT2
+    assert gdr.kernel_chunk(sh, 128, gdr.GATE_GROUP64, "neumann") == 128
+    nch = (1000 + 127) // 128
+    assert gdr.workspace_bytes(sh, 128, gdr.GATE_GROUP64, "neumann") == 2 * 8 * nch * 2 * 128 * 128 * 4
+    auto = gdr.make_shape(2, 1000, 8, 32, 256, 128)
+    assert gdr.select_kernel(auto, 128, gdr.GATE_GROUP64, "neumann") == gdr.KERNEL_SIMT
+    # not enough workspace: nothing launched
+    full = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(8)]
+    assert _call(sh, full, chunk=128, gate=gdr.GATE_GROUP64, inv=gdr.INV_NEUMANN,
+                 ws=ctypes.c_void_p(0x900000), ws_bytes=1024) == gdr.ERR_WORKSPACE
+    # per-channel gates at chunk 128 with two Newton steps: the first pass does not fit
+    big = gdr.make_shape(1, 1000, 1, 1, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32,
+                         neumann_residual_steps=2, kernel="simt2")
+    assert gdr.select_kernel(big, 128, gdr.GATE_CHANNEL, "neumann") == -gdr.ERR_UNSUPPORTED
 
 
 def test_backward_validates(lib):

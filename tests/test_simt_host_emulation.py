@@ -35,11 +35,12 @@ thread_local host_uint3 threadIdx, blockIdx, gridDim;
 static float host_smem[%(smem)d + %(canary)d];
 static const uint32_t kCanary = 0x7fc0dead;   // a NaN pattern
 
-template <bool I, bool O, int NV, bool M>
+template <bool I, bool O, int NV, bool M, bool PRE>
 static int run_grid(const gdr::Params &p)
 {
     const gdr::host_emu::SimtLayout Ly = gdr::host_emu::simt_layout(
-        p.C, p.G, p.dk, p.neumann != 0 || p.neumann1 != 0, p.neu_resid, NV, p.momentum != 0);
+        p.C, p.G, p.dk, !PRE && (p.neumann != 0 || p.neumann1 != 0), PRE ? 0 : p.neu_resid, NV,
+        p.momentum != 0);
     if (Ly.total > %(smem)d)
         return -1;
     for (unsigned b = 0; b < (unsigned)p.B; ++b)
@@ -50,7 +51,7 @@ static int run_grid(const gdr::Params &p)
                 std::memset(host_smem, 0xff, sizeof(float) * Ly.total);   // NaN: unset reads show
                 for (int c = 0; c < %(canary)d; ++c)
                     std::memcpy(&host_smem[Ly.total + c], &kCanary, 4);
-                gdr::host_emu::simt_fwd_kernel<I, O, NV, M>(p);
+                gdr::host_emu::simt_fwd_kernel<I, O, NV, M, PRE>(p);
                 for (int c = 0; c < %(canary)d; ++c)
                     if (std::memcmp(&host_smem[Ly.total + c], &kCanary, 4) != 0)
                         return -2;
@@ -61,7 +62,9 @@ static int run_grid(const gdr::Params &p)
 template <bool I, bool O, int NV>
 static int run_m(const gdr::Params &p)
 {
-    return p.momentum ? run_grid<I, O, NV, true>(p) : run_grid<I, O, NV, false>(p);
+    if (p.factors != nullptr)   // second pass of the two-pass form
+        return run_grid<I, O, NV, false, true>(p);
+    return p.momentum ? run_grid<I, O, NV, true, false>(p) : run_grid<I, O, NV, false, false>(p);
 }
 
 template <int NV>
@@ -75,10 +78,40 @@ static int run_nv(const gdr::Params &p)
 // the value-tile width the library picks: 32 columns if they fit, else 16
 extern "C" int emu_tile(const gdr::Params *p)
 {
+    const bool pre = p->factors != nullptr;
     for (int NV : {32, 16})
-        if (gdr::host_emu::simt_layout(p->C, p->G, p->dk, p->neumann != 0 || p->neumann1 != 0,
-                                       p->neu_resid, NV, p->momentum != 0).total * 4 <= 227 * 1024)
+        if (gdr::host_emu::simt_layout(p->C, p->G, p->dk,
+                                       !pre && (p->neumann != 0 || p->neumann1 != 0),
+                                       pre ? 0 : p->neu_resid, NV, p->momentum != 0).total * 4 <=
+            227 * 1024)
             return NV;
+    return 0;
+}
+
+// first pass of the two-pass form over its grid (chunks x key heads x batch)
+extern "C" int emu_factors(const gdr::Params *p, float *rec)
+{
+    const gdr::host_emu::SimtLayout Ly = gdr::host_emu::simt_layout(
+        p->C, p->G, p->dk, p->neumann != 0 || p->neumann1 != 0, p->neu_resid, 8, false);
+    if (Ly.total * 4 > 227 * 1024)
+        return -1;
+    const int nch = (p->T + p->C - 1) / p->C;
+    for (unsigned b = 0; b < (unsigned)p->B; ++b)
+        for (unsigned h = 0; h < (unsigned)p->Hk; ++h)
+            for (unsigned c = 0; c < (unsigned)nch; ++c) {
+                threadIdx = {0, 0, 0};
+                blockIdx = {c, h, b};
+                std::memset(host_smem, 0xff, sizeof(float) * Ly.total);
+                for (int k = 0; k < %(canary)d; ++k)
+                    std::memcpy(&host_smem[Ly.total + k], &kCanary, 4);
+                if (p->in_bf16)
+                    gdr::host_emu::simt_factors_kernel<true>(*p, rec);
+                else
+                    gdr::host_emu::simt_factors_kernel<false>(*p, rec);
+                for (int k = 0; k < %(canary)d; ++k)
+                    if (std::memcmp(&host_smem[Ly.total + k], &kCanary, 4) != 0)
+                        return -2;
+            }
     return 0;
 }
 
@@ -139,7 +172,7 @@ class Params(ctypes.Structure):
                  "momentum".split()] +
                 [("mu", ctypes.c_float), ("kappa", ctypes.c_void_p)] +
                 [(n, ctypes.c_void_p) for n in
-                 "q k v g beta S0 o S_final S_chunks dO dS_final grad_q grad_k grad_v grad_g "
+                 "q k v g beta S0 o S_final S_chunks factors dO dS_final grad_q grad_k grad_v grad_g "
                  "grad_beta grad_S0".split()])
 
 
@@ -149,13 +182,13 @@ def emu(tmp_path_factory):
         src = open(os.path.join(CSRC, name)).read()
         body = src[:src.index(marker)]
         for old, new in (("constexpr int NT = 256;", "constexpr int NT = 1;"),
-                         ("namespace {", "namespace %s {" % ns),
-                         ("extern __shared__ float sm[];", "float *const sm = host_smem_ptr();")):
+                         ("namespace {", "namespace %s {" % ns)):
             assert body.count(old) == 1, old
             body = body.replace(old, new)
-        return body
+        assert "extern __shared__ float sm[];" in body     # every kernel's shared memory
+        return body.replace("extern __shared__ float sm[];", "float *const sm = host_smem_ptr();")
 
-    fwd = kernel_part("gdr_simt.cu", "template <bool I, bool O, int NV, bool MOM>\nint launch_variant",
+    fwd = kernel_part("gdr_simt.cu", "template <bool I, bool O, int NV, bool MOM, bool PRE>\nint launch_variant",
                       "host_emu")
     bwd = kernel_part("gdr_bwd.cu", "template <bool I, int NV>\nint launch_bwd_variant", "host_emu_bwd")
     # each part ends inside `namespace gdr { namespace ... {`; close the first
@@ -172,6 +205,7 @@ def emu(tmp_path_factory):
     lib = ctypes.CDLL(str(so))
     lib.emu_run.argtypes = [ctypes.POINTER(Params)]
     lib.emu_tile.argtypes = [ctypes.POINTER(Params)]
+    lib.emu_factors.argtypes = [ctypes.POINTER(Params), ctypes.c_void_p]
     lib.emu_bwd.argtypes = [ctypes.POINTER(Params)]
     lib.emu_bwd_tile.argtypes = [ctypes.POINTER(Params)]
     return lib
@@ -186,7 +220,8 @@ def _from_bf16(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
-def run_host(lib, x, chunk, inverse="exact", order=4, resid=1, bf16=False, mu=None, kappa=None):
+def run_host(lib, x, chunk, inverse="exact", order=4, resid=1, bf16=False, mu=None, kappa=None,
+             two_pass=False):
     q = x["q"]
     B, Hk, T, dk = q.shape
     Hv, dv, G = x["v"].shape[1], x["v"].shape[3], x["g"].shape[3]
@@ -209,6 +244,12 @@ def run_host(lib, x, chunk, inverse="exact", order=4, resid=1, bf16=False, mu=No
                momentum=int(mu is not None), mu=0.0 if mu is None else mu, kappa=ptr(kap),
                q=ptr(qq), k=ptr(kk), v=ptr(vv), g=ptr(g), beta=ptr(beta), S0=ptr(S0),
                o=ptr(o_buf, guard), S_final=ptr(s_buf, guard))
+    if two_pass:   # the first pass's records; NaN where a record is not written
+        nch = (T + chunk - 1) // chunk
+        rec = np.full(B * Hk * nch * 2 * chunk * chunk + 2 * guard, np.nan, np.float32)
+        assert lib.emu_factors(ctypes.byref(p), ptr(rec, guard)) == 0
+        assert np.all(np.isnan(rec[:guard])) and np.all(np.isnan(rec[-guard:]))
+        p.factors = ptr(rec, guard)
     assert lib.emu_tile(ctypes.byref(p)) in (16, 32)
     rc = lib.emu_run(ctypes.byref(p))
     assert rc == 0, "host run failed (%d: -2 = shared-memory canary overwritten)" % rc
@@ -250,6 +291,24 @@ def test_host_kernel_matches_oracle(emu, case):
     q, k, v, g, beta, S0 = P.rand_inputs(rng, 1, T, Hk, Hv, dk, dv, G)
     x = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "S0": S0 if with_s0 else None}
     o, S = run_host(emu, x, chunk, inverse, order, resid)
+    args = (x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
+    if inverse == "exact":
+        o_ref, S_ref = oracle.recurrent(*args)
+    else:
+        o_ref, S_ref = oracle.chunked(*args, chunk=chunk, inverse=inverse, order=order, resid=resid)
+    assert rel(o, o_ref) <= 1e-5 and rel(S, S_ref) <= 1e-5
+
+
+@pytest.mark.parametrize("case", CASES, ids=["T%d-R%d-dk%d-dv%d-G%d-C%d-%s" % (c[0], c[2] // c[1], c[3], c[4], c[5], c[6], c[7])
+                                             for c in CASES])
+def test_host_two_pass_matches_oracle(emu, case):
+    # the two-pass form (chunk factors of all chunks first, then the value tiles'
+    # pass reading them): the same results as the one-pass kernel computes
+    T, Hk, Hv, dk, dv, G, chunk, inverse, order, resid, with_s0 = case
+    rng = np.random.default_rng(zlib.crc32(repr(case).encode()))
+    q, k, v, g, beta, S0 = P.rand_inputs(rng, 1, T, Hk, Hv, dk, dv, G)
+    x = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "S0": S0 if with_s0 else None}
+    o, S = run_host(emu, x, chunk, inverse, order, resid, two_pass=True)
     args = (x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
     if inverse == "exact":
         o_ref, S_ref = oracle.recurrent(*args)
