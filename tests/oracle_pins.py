@@ -396,6 +396,10 @@ def pin_output_epilogue(seed=15):
     # o = (3, 4): mean square 12.5; z = 0 gates by 1/2
     out = oracle.output_gate_rmsnorm(np.array([[3.0, 4.0]]), np.zeros((1, 2)), eps=0.0)
     worst = _rel(out, np.array([[1.5, 2.0]]) / np.sqrt(12.5))
+    # per-channel gates sigmoid(0) = 1/2, sigmoid(ln 3) = 3/4, and eps = 7.5 inside the
+    # root: 1 / sqrt(12.5 + 7.5) = 1 / sqrt(20)
+    out = oracle.output_gate_rmsnorm(np.array([[3.0, 4.0]]), np.array([[0.0, np.log(3.0)]]), eps=7.5)
+    worst = max(worst, _rel(out, np.array([[1.5, 3.0]]) / np.sqrt(20.0)))
     rng = np.random.default_rng(seed)
     o, z = rng.standard_normal((5, 7, 16)), rng.standard_normal((5, 7, 16))
     w = rng.standard_normal(16)

@@ -32,6 +32,10 @@ MUTANTS = [
     ("neumann1_sign", "X[e] = Dinv[e] - X[e];", "X[e] = Dinv[e] + X[e];"),
     ("epilogue_gate_sign", "const double gate = 1.0 / (1.0 + exp(-z[(size_t)r * dv + i]));",
      "const double gate = 1.0 / (1.0 + exp(z[(size_t)r * dv + i]));"),
+    ("epilogue_eps_outside_root", "const double inv = 1.0 / sqrt(ss / dv + eps);",
+     "const double inv = 1.0 / (sqrt(ss / dv) + eps);"),
+    ("epilogue_gate_index", "const double gate = 1.0 / (1.0 + exp(-z[(size_t)r * dv + i]));",
+     "const double gate = 1.0 / (1.0 + exp(-z[(size_t)r * dv]));"),
     ("momentum_velocity_sign", "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] - fs);",
      "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] + fs);"),
     ("momentum_no_carry", "Z[i * dv + n] = mk * Z[i * dv + n] + (S[i * dv + n] - fs);",
