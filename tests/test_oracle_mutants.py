@@ -32,6 +32,10 @@ MUTANTS = [
     ("neumann1_sign", "X[e] = Dinv[e] - X[e];", "X[e] = Dinv[e] + X[e];"),
     ("epilogue_gate_sign", "const double gate = 1.0 / (1.0 + exp(-z[(size_t)r * dv + i]));",
      "const double gate = 1.0 / (1.0 + exp(z[(size_t)r * dv + i]));"),
+    ("gva_mapping_recurrent", "hk = hv / R;\n        double *S = (double *)malloc",
+     "hk = hv % Hk;\n        double *S = (double *)malloc"),
+    ("gva_mapping_chunked", "hk = hv / R;\n        const long kh = b * Hk + hk;\n        const size_t CC",
+     "hk = hv % Hk;\n        const long kh = b * Hk + hk;\n        const size_t CC"),
     ("epilogue_eps_outside_root", "const double inv = 1.0 / sqrt(ss / dv + eps);",
      "const double inv = 1.0 / (sqrt(ss / dv) + eps);"),
     ("epilogue_gate_index", "const double gate = 1.0 / (1.0 + exp(-z[(size_t)r * dv + i]));",
