@@ -16,13 +16,18 @@
 // Approximation for Quantized Gated DeltaNet" (masked powers, Lemma 3.1, then
 // Newton residual corrections).
 //
-// With chunk-boundary momentum (the same paper, §2.3) the state update of each
-// chunk is blended with a velocity Z (zero at the start), kept beside S:
+// With chunk-boundary momentum ("Systolic Linear Attention ...", §2.3) the state
+// update of each chunk is blended with a velocity Z (zero at the start), kept
+// beside S:
 //   Z <- mu kappa_c Z + Khat^T E,  S <- F S + Z,
 // where Khat^T E is exactly the plain update minus F S; the chunk's outputs are
 // those of the plain chunk computation from the entry state.
 //
-// One CTA owns one value head and NV value columns; chunks run in order.
+// One CTA owns one value head and NV value columns; chunks run in order.  In the
+// two-pass form (PRE) a first kernel computes every chunk's inverse and L at
+// once, and this kernel reads them instead of recomputing them per value tile.
+// With o == nullptr it only walks the states (writing the state at each chunk's
+// start to S_chunks when given: the backward's recomputation).
 #include <cuda_bf16.h>
 
 #include "gdr_internal.h"
