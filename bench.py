@@ -257,8 +257,22 @@ def run_reference(args, w, chunk, rank):
     x = W.make_inputs(w, rank_seed(args.workload, 0))
     times, rate_list = [], []
     desc, threads = "", 1
+    variant = args.which == "backward" or args.momentum is not None
+    up, kappa = None, None
+    if variant:   # the same seeded upstream gradients / kappa as the GPU arm's rank 0
+        rng = np.random.default_rng(7200 + args.workload)
+        if args.which == "backward":
+            up = (rng.standard_normal((w.B, w.Hv, w.T, w.dv)).astype(np.float32), None)
+        else:
+            kappa = (rng.random((w.B, (w.T + chunk - 1) // chunk)) >= 0.125).astype(np.int32)
     for step in range(args.warmup + args.steps):
-        rate, threads, desc, dt = oracle_sample(w, x, chunk, args.inverse, budget_s=2.0)
+        if variant:
+            t0 = time.perf_counter()
+            rate, threads, desc = oracle_variant_sample(w, x, chunk, up, args.momentum, kappa,
+                                                        budget_s=2.0)
+            dt = time.perf_counter() - t0
+        else:
+            rate, threads, desc, dt = oracle_sample(w, x, chunk, args.inverse, budget_s=2.0)
         if step >= args.warmup:
             rate_list.append(rate)
             times.append(dt)
@@ -268,7 +282,9 @@ def run_reference(args, w, chunk, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(w, chunk, args.inverse, args.gpus),
+        "config": (dict(config_dict(w, chunk, "exact", args.gpus),
+                        which=("backward" if args.which == "backward" else "momentum mu=%g" % args.momentum))
+                   if variant else config_dict(w, chunk, args.inverse, args.gpus)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": desc + " per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
