@@ -96,13 +96,16 @@ typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1, GDR_INV_NEUMANN1 = 2 } gd
 typedef enum { GDR_KERNEL_AUTO = 0, GDR_KERNEL_SIMT = 1, GDR_KERNEL_TC = 2,
                GDR_KERNEL_TC2 = 3, GDR_KERNEL_SIMT2 = 4 } gdr_kernel;
 
+/* Shape of a request.  Besides the per-field ranges, B * T * (Hk dk + Hv dv)
+ * must not exceed 2^40 elements (GDR_ERR_SHAPE otherwise). */
 typedef struct {
-    int B;      /* batch, >= 0                                               */
+    int B;      /* batch, 0..65535                                           */
     int T;      /* tokens per sequence, >= 0; any T (a ragged last chunk is
                    handled as a shorter chunk)                               */
     int Hk;     /* key heads, >= 1                                           */
-    int Hv;     /* value heads, multiple of Hk; value head hv reads key head
-                   hv / (Hv / Hk) (grouped value heads, SLA §2.4.1)          */
+    int Hv;     /* value heads, multiple of Hk, at most 65535; value head hv
+                   reads key head hv / (Hv / Hk) (grouped value heads,
+                   SLA §2.4.1)                                               */
     int dk;     /* key width, 1..256                                         */
     int dv;     /* value width per value head, 1..256                        */
     gdr_dtype in_dtype;   /* dtype of q, k, v                                */

@@ -86,6 +86,24 @@ def test_rejects_bad_shapes(lib):
                  inv=gdr.INV_NEUMANN) == gdr.ERR_SHAPE
 
 
+def test_rejects_sizes_past_the_grid_and_byte_limits(lib):
+    # batch and value heads index grid rows (<= 65535); at most 2^40 input elements
+    assert _call(gdr.make_shape(70000, 64, 1, 1, 64, 64)) == gdr.ERR_SHAPE
+    assert _call(gdr.make_shape(1, 64, 1, 70000, 64, 64)) == gdr.ERR_SHAPE
+    assert _call(gdr.make_shape(60000, 1 << 30, 1, 1, 64, 64)) == gdr.ERR_SHAPE
+    assert gdr.select_kernel(gdr.make_shape(65536, 64, 1, 1, 64, 64), 64, gdr.GATE_SCALAR) == \
+        -gdr.ERR_SHAPE
+    # just inside the bound the workspace sizes are exact (no wrap-around)
+    big = gdr.make_shape(64, 1 << 20, 16, 16, 128, 128)
+    nch = (1 << 20) // 64
+    assert gdr.state_segments(big, 64, gdr.GATE_SCALAR) == 1      # many sequences: no segments
+    assert gdr.workspace_bytes(big, 64, gdr.GATE_SCALAR) == 64 * 16 * nch * gdr.TC2_SCALAR_RECORD_BYTES
+    assert gdr.bwd_workspace_bytes(big, 64, gdr.GATE_SCALAR) == 4 * 64 * 16 * nch * 128 * 128
+    simt2 = gdr.make_shape(64, 1 << 20, 16, 16, 128, 128, kernel="simt2")
+    assert gdr.workspace_bytes(simt2, 128, gdr.GATE_CHANNEL, "neumann") == \
+        64 * 16 * (nch // 2) * 2 * 128 * 128 * 4
+
+
 def test_rejects_bad_enums_and_dtypes(lib):
     ok = dict(B=1, T=64, Hk=2, Hv=4, dk=64, dv=64)
     assert _call(gdr.make_shape(**ok), gate=7) == gdr.ERR_ARG
