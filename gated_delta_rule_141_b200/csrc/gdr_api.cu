@@ -33,7 +33,7 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
         return GDR_ERR_SHAPE;
     // batch and heads index grid rows (at most 65535), and at most 2^40 input
     // elements keep every byte count here (records, workspaces) far inside 64 bits
-    if (s->B > 65535 || s->Hv > 65535)
+    if (s->B > 65535 || s->Hv > 65535 || (long)s->B * s->Hv > 0x7fffffffL)   // and 32-bit sequence indices
         return GDR_ERR_SHAPE;
     if ((double)s->B * s->T * ((double)s->Hk * s->dk + (double)s->Hv * s->dv) > 1099511627776.0)
         return GDR_ERR_SHAPE;

@@ -96,8 +96,9 @@ typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1, GDR_INV_NEUMANN1 = 2 } gd
 typedef enum { GDR_KERNEL_AUTO = 0, GDR_KERNEL_SIMT = 1, GDR_KERNEL_TC = 2,
                GDR_KERNEL_TC2 = 3, GDR_KERNEL_SIMT2 = 4 } gdr_kernel;
 
-/* Shape of a request.  Besides the per-field ranges, B * T * (Hk dk + Hv dv)
- * must not exceed 2^40 elements (GDR_ERR_SHAPE otherwise). */
+/* Shape of a request.  Besides the per-field ranges, B * Hv must be below 2^31
+ * and B * T * (Hk dk + Hv dv) must not exceed 2^40 elements (GDR_ERR_SHAPE
+ * otherwise). */
 typedef struct {
     int B;      /* batch, 0..65535                                           */
     int T;      /* tokens per sequence, >= 0; any T (a ragged last chunk is

@@ -91,6 +91,7 @@ def test_rejects_sizes_past_the_grid_and_byte_limits(lib):
     assert _call(gdr.make_shape(70000, 64, 1, 1, 64, 64)) == gdr.ERR_SHAPE
     assert _call(gdr.make_shape(1, 64, 1, 70000, 64, 64)) == gdr.ERR_SHAPE
     assert _call(gdr.make_shape(60000, 1 << 30, 1, 1, 64, 64)) == gdr.ERR_SHAPE
+    assert _call(gdr.make_shape(65535, 1, 65535, 65535, 64, 64)) == gdr.ERR_SHAPE   # B Hv >= 2^31
     assert gdr.select_kernel(gdr.make_shape(65536, 64, 1, 1, 64, 64), 64, gdr.GATE_SCALAR) == \
         -gdr.ERR_SHAPE
     # just inside the bound the workspace sizes are exact (no wrap-around)
