@@ -37,8 +37,11 @@ namespace {
 constexpr int NT = 256;  // threads per CTA
 
 struct BwdLayout {       // offsets in floats into dynamic shared memory
-    int lam, beta, row, P, A, L, S, dS, Y, dO, dE, dR, DL, DLg, F, X, total;
+    int lam, beta, row, P, A, L, S, dS, Y, dO, dE, dR, DL, DLg, F, X, E1, total;
+    bool tab;            // scalar gate: e^{Lambda_t - Lambda_j} tabulated in E1
 };
+
+constexpr int kBwdSmemFloats = 227 * 1024 / 4;
 
 __host__ __device__ inline BwdLayout bwd_layout(int C, int G, int dk, int NV)
 {
@@ -60,6 +63,10 @@ __host__ __device__ inline BwdLayout bwd_layout(int C, int G, int dk, int NV)
     s.DLg = off;  off += (G < dk) ? C * G : 0;   // dLambda per (token, group)
     s.F = off;    off += dk;        // e^{Lambda_C} per channel
     s.X = off;    off += dk;        // gradient of Lambda_C per channel
+    // scalar gate: the pair factors depend on (t, j) only; tabulate them when
+    // they fit beside the rest (last, so the other offsets do not move)
+    s.tab = G == 1 && off + C * C <= kBwdSmemFloats;
+    s.E1 = off;   off += s.tab ? C * C : 0;
     s.total = off;
     return s;
 }
@@ -88,7 +95,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
     float *lam = sm + Ly.lam, *sbeta = sm + Ly.beta, *row = sm + Ly.row, *P = sm + Ly.P;
     float *A = sm + Ly.A, *L = sm + Ly.L, *S = sm + Ly.S, *dS = sm + Ly.dS, *Y = sm + Ly.Y;
     float *dO = sm + Ly.dO, *dE = sm + Ly.dE, *dR = sm + Ly.dR, *DL = sm + Ly.DL;
-    float *Fv = sm + Ly.F, *X = sm + Ly.X;
+    float *Fv = sm + Ly.F, *X = sm + Ly.X, *E1 = sm + Ly.E1;
+    const bool tab = Ly.tab;
     const int width = dk / G;                 // channels per decay group
     float *DLg = width > 1 ? sm + Ly.DLg : DL;   // per group (the same array when G = dk)
 
@@ -148,6 +156,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
                     const float e = expf(lam[t * G + gi] - lam[j * G + gi]);
                     pm += e * skk;
                     lm += e * sqk;
+                    if (tab)
+                        E1[t * C + j] = e;
                 }
                 if (j == t)
                     pm = 0.f;
@@ -278,14 +288,14 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             const float qti = ld_in<IN_BF16>(p.q, base + (long)t * dk);
             float a = 0.f, bb = 0.f, cc = 0.f, d = 0.f;
             for (int j = 0; j <= t; ++j) {
-                const float e = expf(lt - lam[j * G + gi]);
+                const float e = tab ? E1[t * C + j] : expf(lt - lam[j * G + gi]);
                 const float kji = ld_in<IN_BF16>(p.k, base + (long)j * dk);
                 if (j < t)
                     a += sbeta[j] * A[t * C + j] * kji * e;
                 cc += L[t * C + j] * kji * e;
             }
             for (int t2 = t; t2 < Cl; ++t2) {
-                const float e = expf(lam[t2 * G + gi] - lt);
+                const float e = tab ? E1[t2 * C + t] : expf(lam[t2 * G + gi] - lt);
                 if (t2 > t)
                     bb += sbeta[t] * A[t2 * C + t] * ld_in<IN_BF16>(p.k, base + (long)t2 * dk) * e;
                 d += L[t2 * C + t] * ld_in<IN_BF16>(p.q, base + (long)t2 * dk) * e;
@@ -356,7 +366,7 @@ int launch_bwd_variant(const Params &p, int smem, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }
 
-constexpr int kMaxSmem = 227 * 1024;
+constexpr int kMaxSmem = kBwdSmemFloats * 4;
 
 int bwd_smem_for(const Params &p, int NV)
 {
