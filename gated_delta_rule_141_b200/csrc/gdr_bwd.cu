@@ -38,8 +38,8 @@ constexpr int NT = 256;  // threads per CTA
 
 struct BwdLayout {       // offsets in floats into dynamic shared memory
     int lam, beta, row, P, A, L, S, dS, Y, dO, dE, dR, DL, DLg, F, X, E1, total;
-    bool tab;            // scalar gate: e^{Lambda_t - Lambda_j} tabulated in E1
-};
+    bool tab;            // scalar gate: e^{Lambda_t - Lambda_j} (C x C) and e^{Lambda_t} (C)
+};                       // tabulated in E1
 
 constexpr int kBwdSmemFloats = 227 * 1024 / 4;
 
@@ -65,8 +65,8 @@ __host__ __device__ inline BwdLayout bwd_layout(int C, int G, int dk, int NV)
     s.X = off;    off += dk;        // gradient of Lambda_C per channel
     // scalar gate: the pair factors depend on (t, j) only; tabulate them when
     // they fit beside the rest (last, so the other offsets do not move)
-    s.tab = G == 1 && off + C * C <= kBwdSmemFloats;
-    s.E1 = off;   off += s.tab ? C * C : 0;
+    s.tab = G == 1 && off + C * C + C <= kBwdSmemFloats;
+    s.E1 = off;   off += s.tab ? C * C + C : 0;
     s.total = off;
     return s;
 }
@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
     float *dO = sm + Ly.dO, *dE = sm + Ly.dE, *dR = sm + Ly.dR, *DL = sm + Ly.DL;
     float *Fv = sm + Ly.F, *X = sm + Ly.X, *E1 = sm + Ly.E1;
     const bool tab = Ly.tab;
+    float *Et = E1 + C * C;                   // tab: e^{Lambda_t}
     const int width = dk / G;                 // channels per decay group
     float *DLg = width > 1 ? sm + Ly.DLg : DL;   // per group (the same array when G = dk)
 
@@ -166,6 +167,9 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             A[t * C + j] = (j == t) ? 1.f : pm * sbeta[j];
             L[t * C + j] = lm;
         }
+        if (tab)
+            for (int t = tid; t < Cl; t += NT)
+                Et[t] = expf(lam[t]);
         __syncthreads();
         // --- A = (I + M)^{-1} by forward substitution in place (row t from the rows above)
         for (int t = 1; t < Cl; ++t) {
@@ -186,7 +190,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             const long kt = (kh * T + c0 + t) * dk;
             float acc = 0.f;
             for (int i = 0; i < dk; ++i)
-                acc += ld_in<IN_BF16>(p.k, kt + i) * expf(lam[t * G + i / width]) * S[i * NV + n];
+                acc += ld_in<IN_BF16>(p.k, kt + i) * (tab ? Et[t] : expf(lam[t * G + i / width])) *
+                       S[i * NV + n];
             const float vv = n < nv ? ld_in<IN_BF16>(p.v, (vh * T + c0 + t) * dv + n0 + n) : 0.f;
             dR[idx] = vv - acc;
         }
@@ -207,7 +212,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             const long kj = (kh * T + c0 + j) * dk;
             for (int i = 0; i < dk; ++i) {
                 const int gi = i / width;
-                acc += ld_in<IN_BF16>(p.k, kj + i) * expf(lam[(Cl - 1) * G + gi] - lam[j * G + gi]) *
+                acc += ld_in<IN_BF16>(p.k, kj + i) *
+                       (tab ? E1[(Cl - 1) * C + j] : expf(lam[(Cl - 1) * G + gi] - lam[j * G + gi])) *
                        dS[i * NV + n];
             }
             dE[idx] = acc;
@@ -261,7 +267,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             for (int n = 0; n < NV; ++n) {
                 float sn = f * S[i * NV + n];
                 for (int t = 0; t < Cl; ++t)
-                    sn += ld_in<IN_BF16>(p.k, (kh * T + c0 + t) * dk + i) * expf(lc - lam[t * G + gi]) *
+                    sn += ld_in<IN_BF16>(p.k, (kh * T + c0 + t) * dk + i) *
+                          (tab ? E1[(Cl - 1) * C + t] : expf(lc - lam[t * G + gi])) *
                           sbeta[t] * Y[t * NV + n];
                 x += dS[i * NV + n] * sn;
             }
@@ -307,7 +314,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
                 dkh += Y[t * NV + n] * dS[i * NV + n];
             }
             dkh *= sbeta[t];
-            const float et = expf(lt), eh = expf(lc - lt);
+            const float et = tab ? Et[t] : expf(lt);
+            const float eh = tab ? E1[(Cl - 1) * C + t] : expf(lc - lt);
             atomicAdd(&p.grad_q[base + (long)t * dk], cc + dqb * et);
             atomicAdd(&p.grad_k[base + (long)t * dk], a + bb + d + dkb * et + dkh * eh);
             DL[t * dk + i] = kti * (a - bb - d) + qti * cc + (dqb * qti + dkb * kti) * et - dkh * kti * eh;
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             float acc = Fv[i] * dS[idx];
             for (int t = 0; t < Cl; ++t) {
                 const long kt = (kh * T + c0 + t) * dk + i;
-                const float e = expf(lam[t * G + gi]);
+                const float e = tab ? Et[t] : expf(lam[t * G + gi]);
                 acc += e * (ld_in<IN_BF16>(p.q, kt) * dO[t * NV + n] - ld_in<IN_BF16>(p.k, kt) * dR[t * NV + n]);
             }
             dS[idx] = acc;
