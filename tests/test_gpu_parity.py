@@ -31,9 +31,6 @@ SMALL = [
     (0, dict(T=203, Hk=1, Hv=3, dv=40, s0_std=0.5), 64, "exact", "simt"),
     (0, dict(T=77, dk=32, dv=16, s0_std=0.3), 16, "exact", "simt"),
     (0, dict(T=130, gate_mode=W.GATE_CHANNEL), 32, "neumann", "simt"),
-    # chunks shorter than the 32-column value tile (Q S then has its own buffer)
-    (0, dict(T=101, s0_std=0.3), 16, "neumann", "simt"),
-    (0, dict(T=93, dv=40, gate_mode=W.GATE_CHANNEL), 24, "neumann1", "simt"),
     # bf16 inputs, each gate mode, both inverse modes, shrunk workloads
     (1, dict(B=1, Hk=2, Hv=2, T=320), 64, "exact", "auto"),
     (1, dict(B=1, Hk=2, Hv=2, T=320), 64, "exact", "simt"),
@@ -73,6 +70,9 @@ SMALL = [
     (4, dict(Hk=1, Hv=1, T=384), 64, "neumann1", "tc2"),                # pivoted blocks
     (0, {}, 128, "neumann1", "auto"),                                   # fp32
     (4, dict(Hk=1, Hv=1, T=300), 128, "neumann1", "auto"),
+    # chunks shorter than the 32-column value tile (Q S then has its own buffer)
+    (0, dict(T=101, s0_std=0.3), 16, "neumann", "simt"),
+    (0, dict(T=93, dv=40, gate_mode=W.GATE_CHANNEL), 24, "neumann1", "simt"),
 ]
 
 
