@@ -95,6 +95,22 @@ def algorithmic(w: W.Workload, chunk: int, inverse: str, order=4, resid=1):
     return flop_tok * units, byte_tok * units + state
 
 
+def roofline(flop: float, byts: float, ms: float, peaks: dict) -> dict:
+    """The bound (HBM or tensor) whose time at peak is the larger for this work,
+    the achieved rate against it, and both fractions."""
+    s = ms * 1e-3
+    hbm_frac = (byts / s) / (peaks["hbm_gbs"] * 1e9)
+    tc_frac = (flop / s) / (peaks["bf16_tflops"] * 1e12)
+    if byts / (peaks["hbm_gbs"] * 1e9) >= flop / (peaks["bf16_tflops"] * 1e12):
+        roof = {"bound": "hbm", "achieved": byts / s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm_frac}
+    else:
+        roof = {"bound": "tensor", "achieved": flop / s / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": tc_frac}
+    roof["hbm_frac"], roof["tc_frac"] = hbm_frac, tc_frac
+    return roof
+
+
 def rank_seed(workload_index: int, rank: int) -> int:
     """Each rank draws its own copy of the workload (weak scaling, independent
     sequences); rank 0 uses the standard seed."""
@@ -602,21 +618,11 @@ def main():
     if args.epilogue:   # the epilogue reads o and z and writes o once more
         byts += 3 * o.numel() * o.element_size()
     peaks, peak_src = measured_peaks()
-    hbm_frac = (byts / (ms_step * 1e-3)) / (peaks["hbm_gbs"] * 1e9)
-    tc_frac = (flop / (ms_step * 1e-3)) / (peaks["bf16_tflops"] * 1e12)
-    bound = "hbm" if byts / (peaks["hbm_gbs"] * 1e9) >= flop / (peaks["bf16_tflops"] * 1e12) else "tensor"
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": byts / (ms_step * 1e-3) / 1e9,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm_frac}
-    else:
-        roof = {"bound": "tensor", "achieved": flop / (ms_step * 1e-3) / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tc_frac}
+    roof = roofline(flop, byts, ms_step, peaks)
     roof["peak_source"] = peak_src + " (burst)"
     roof["traffic"] = recorded_traffic(w.name, chunk, args.inverse,
                                        gdr.KERNEL_NAMES.get(kern, str(kern)))
     roof["tflops"] = flop / (ms_step * 1e-3) / 1e12
-    roof["tc_frac"] = tc_frac
-    roof["hbm_frac"] = hbm_frac
     roof["kernel"] = gdr.KERNEL_NAMES.get(kern, str(kern))
     roof["launches_per_step"] = launches_per_step
 

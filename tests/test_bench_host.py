@@ -44,3 +44,18 @@ def test_variant_oracle_samples():
     kappa = np.ones((w.B, (w.T + 63) // 64), np.int32)
     rate, threads, desc = bench.oracle_variant_sample(w, x, 64, None, 0.25, kappa, budget_s=0.2)
     assert rate > 0 and "momentum" in desc
+
+
+def test_roofline_arithmetic():
+    peaks = {"hbm_gbs": 6448.0, "bf16_tflops": 1726.0}
+    # the gdn_scalar_bf16 step: 279 MB and 3.69e10 FLOP in 0.217 ms is HBM-bound
+    r = bench.roofline(3.69e10, 279e6, 0.217, peaks)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - 279e6 / 0.217e-3 / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6448.0) < 1e-12
+    assert abs(r["tc_frac"] - 3.69e10 / 0.217e-3 / 1726e12) < 1e-12
+    # at 324 FLOP per byte (above the ridge of ~268) the tensor bound applies
+    r = bench.roofline(1.34e11, 414e6, 0.1, peaks)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["frac"] - 1.34e11 / 1e-4 / 1726e12) < 1e-12
+    assert abs(r["hbm_frac"] - 414e6 / 1e-4 / 6448e9) < 1e-12
