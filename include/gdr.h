@@ -14,7 +14,10 @@
  * structural masking and residual correction ("When Good Enough Is Optimal:
  * Multiplication-Only Matrix Inversion Approximation for Quantized Gated
  * DeltaNet", Lemma 3.1); the state S stays on chip across chunks.  There is
- * no 1/sqrt(dk) query scale.
+ * no 1/sqrt(dk) query scale.  Beside the forward: its gradients
+ * (gdr_chunk_bwd, the custom-VJP backward of §2.5), the forward with
+ * chunk-boundary momentum (gdr_chunk_fwd_momentum, §2.3) and the readout
+ * epilogue (gdr_output_gate_rmsnorm, §2.3 Eq. (5)).
  *
  * Conventions shared by every entry point
  *  - Tensors are dense, row-major, contiguous, in the layouts given below.
@@ -22,14 +25,16 @@
  *    every buffer.  The library allocates no device memory on any call
  *    (tensor memory on chip is allocated and released inside each kernel).
  *  - Every device pointer must be 16-byte aligned (tensor-memory-access tile
- *    loads); otherwise GDR_ERR_ALIGN.
+ *    loads); otherwise GDR_ERR_ALIGN.  (The int32 kappa of
+ *    gdr_chunk_fwd_momentum needs 4 bytes.)
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL = the legacy default stream).  Arguments are validated on the host
  *    before anything is launched; on any error nothing is launched and the
  *    status says why.  No exception, abort or exit crosses the ABI.
- *  - Thread safety: calls may be issued from several host threads; the only
+ *  - Thread safety: calls may be issued from several host threads; the
  *    library-global state is the device status word read by
- *    gdr_device_status().
+ *    gdr_device_status() and the fixed scratch array of gdr_chunk_fwd_static
+ *    (calls of that entry point that overlap on the GPU race on it).
  */
 #ifndef GDR_H_
 #define GDR_H_
