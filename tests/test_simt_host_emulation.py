@@ -401,3 +401,14 @@ def test_host_backward_matches_oracle(emu, case):
     ref = oracle.recurrent_grad(q, k, v, g, beta, x["S0"], dO, dSf)
     for n in ("q", "k", "v", "g", "beta", "S0"):
         assert rel(got[n], ref[n]) <= 1e-4, (n, rel(got[n], ref[n]))
+
+
+def test_host_kernel_momentum_bf16_io(emu):
+    # momentum with bf16 q, k, v and bf16 o (the gdn_scalar_bf16 shapes, shortened)
+    w, x = W.workload_inputs(1, B=2, Hk=1, Hv=2, T=200)
+    kappa = (np.random.default_rng(9).random((2, 4)) < 0.7).astype(np.int32)
+    o, S = run_host(emu, x, 64, bf16=True, mu=0.25, kappa=kappa)
+    o_ref, S_ref = oracle.chunked(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], chunk=64,
+                                  mu=0.25, kappa=kappa)
+    assert rel(S, S_ref) <= 1e-5
+    assert rel(o, o_ref) <= 2.0 ** -8
