@@ -56,8 +56,12 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--workload", type=int, default=4,
+                    help="workload index (default 4: long_strong_decay_bf16, the largest)")
     ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--T", type=int, default=0,
+                    help="tokens per sequence instead of the workload's own (reduced-size "
+                         "profiling captures; the JSON config records it)")
     ap.add_argument("--inverse", default="exact", choices=["exact", "neumann", "neumann1"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "simt", "simt2"])
@@ -521,6 +525,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = W.WORKLOADS[args.workload]
+    if args.T:
+        w = w.scaled(T=args.T)
     chunk = args.chunk or w.chunk
     if args.impl == "reference":
         return run_reference(args, w, chunk, rank)

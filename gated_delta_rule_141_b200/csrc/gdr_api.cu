@@ -97,33 +97,37 @@ int choose(const gdr::Params &p, gdr_kernel want, size_t ws_bytes)
     return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
 }
 
-}  // namespace
-
-extern "C" {
-
-gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, const void *v,
-                         const float *g, const float *beta, const float *S0, int chunk,
-                         gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode, void *o,
-                         float *S_final, void *workspace, size_t workspace_bytes, void *stream)
+// Every check gdr_chunk_fwd makes before it launches anything: the request, the
+// device pointers, their alignment and the kernel choice given the workspace.
+// On GDR_OK *p holds the request with its pointers and *which the kernel.
+gdr_status validate_fwd(const gdr_shape *shape, const void *q, const void *k, const void *v,
+                        const float *g, const float *beta, const float *S0, int chunk,
+                        gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode, void *o,
+                        float *S_final, void *workspace, size_t workspace_bytes, gdr::Params *p,
+                        int *which)
 {
-    gdr::Params p;
-    gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, p);
     if (st != GDR_OK)
         return st;
-    const bool has_tokens = (long)p.B * p.T > 0;
+    const bool has_tokens = (long)p->B * p->T > 0;
     if (has_tokens && (!q || !k || !v || !g || !beta || !o))
         return GDR_ERR_ARG;
     const void *ptrs[] = {q, k, v, g, beta, S0, o, S_final, workspace};
     for (const void *ptr : ptrs)
         if (ptr != nullptr && !aligned16(ptr))
             return GDR_ERR_ALIGN;
-    const int which = choose(p, shape->kernel, workspace != nullptr ? workspace_bytes : 0);
-    if (which < 0)
-        return static_cast<gdr_status>(-which);
+    const int w = choose(*p, shape->kernel, workspace != nullptr ? workspace_bytes : 0);
+    if (w < 0)
+        return static_cast<gdr_status>(-w);
+    p->q = q; p->k = k; p->v = v; p->g = g; p->beta = beta; p->S0 = S0; p->o = o; p->S_final = S_final;
+    *which = w;
+    return GDR_OK;
+}
+
+gdr_status launch_fwd(const gdr::Params &p, int which, void *workspace, cudaStream_t s)
+{
     if (p.B == 0)
         return GDR_OK;
-    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S0 = S0; p.o = o; p.S_final = S_final;
-    auto s = static_cast<cudaStream_t>(stream);
     int rc;
     if (which == GDR_KERNEL_TC2)
         rc = gdr::launch_tc2(p, workspace, s);
@@ -134,6 +138,24 @@ gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, c
     else
         rc = gdr::launch_simt(p, s);
     return static_cast<gdr_status>(rc);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdr_status gdr_chunk_fwd(const gdr_shape *shape, const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, const float *S0, int chunk,
+                         gdr_gate_mode gate_mode, gdr_inverse_mode inverse_mode, void *o,
+                         float *S_final, void *workspace, size_t workspace_bytes, void *stream)
+{
+    gdr::Params p;
+    int which = 0;
+    const gdr_status st = validate_fwd(shape, q, k, v, g, beta, S0, chunk, gate_mode, inverse_mode,
+                                       o, S_final, workspace, workspace_bytes, &p, &which);
+    if (st != GDR_OK)
+        return st;
+    return launch_fwd(p, which, workspace, static_cast<cudaStream_t>(stream));
 }
 
 gdr_status gdr_bwd_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,
@@ -265,8 +287,13 @@ gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const 
 {
     if (host == nullptr || dev == nullptr)
         return GDR_ERR_ARG;
+    // the whole device-side request is validated before any copy is queued, so
+    // that a refused call leaves nothing on the stream
     gdr::Params p;
-    gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
+    int which = 0;
+    gdr_status st = validate_fwd(shape, dev->q, dev->k, dev->v, dev->g, dev->beta, dev->S0, chunk,
+                                 gate_mode, inverse_mode, dev->o, dev->S_final, workspace,
+                                 workspace_bytes, &p, &which);
     if (st != GDR_OK)
         return st;
     const bool has_tokens = (long)p.B * p.T > 0;
@@ -291,14 +318,10 @@ gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const 
     for (const Copy &c : in) {
         if (c.bytes == 0 || c.src == nullptr)
             continue;
-        if (c.dst == nullptr)
-            return GDR_ERR_ARG;
         if (cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
             return GDR_ERR_CUDA;
     }
-    st = gdr_chunk_fwd(shape, dev->q, dev->k, dev->v, dev->g, dev->beta, dev->S0, chunk,
-                       gate_mode, inverse_mode, dev->o, dev->S_final, workspace, workspace_bytes,
-                       stream);
+    st = launch_fwd(p, which, workspace, s);
     if (st != GDR_OK)
         return st;
     if (has_tokens &&
@@ -355,6 +378,13 @@ gdr_status gdr_device_status(void *stream)
     if (v < 0)
         return GDR_ERR_CUDA;
     return v == 0 ? GDR_OK : GDR_ERR_TIMEOUT;
+}
+
+gdr_status gdr_selftest_bounded_wait(uint64_t limit_ns, void *stream)
+{
+    if (limit_ns < 1000u || limit_ns > 1000000000u)
+        return GDR_ERR_ARG;
+    return static_cast<gdr_status>(gdr::launch_wait_probe(limit_ns, static_cast<cudaStream_t>(stream)));
 }
 
 const char *gdr_status_string(gdr_status status)

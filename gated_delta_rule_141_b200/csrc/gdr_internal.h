@@ -38,6 +38,10 @@ struct Params {
 // (after the caller synchronised) and clears it.  Returns -1 on a CUDA error.
 int read_and_clear_device_status();
 
+// One warp that waits on an mbarrier nothing arrives on, for limit_ns, then sets
+// the status word to the timeout code and releases its tensor memory.
+int launch_wait_probe(uint64_t limit_ns, cudaStream_t stream);
+
 // CUDA-core kernel (fp32 arithmetic).  Returns 0 on launch, or a gdr_status
 // code if the request does not fit the kernel's shared-memory budget.
 int simt_smem_bytes(const Params &p);

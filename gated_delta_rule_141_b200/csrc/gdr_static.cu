@@ -6,10 +6,11 @@
 // on which the library's device code is loaded keeps it until the process
 // exits.  In host code its name only stands in for the symbol (it is not a
 // device address), so the address the kernels receive comes from
-// cudaGetSymbolAddress, looked up once per device on the first call made with
-// that device current.
+// cudaGetSymbolAddress, asked again on every call with the caller's device
+// current: the answer belongs to the device context current at that moment,
+// and a remembered one could outlive its context (after cudaDeviceReset, or
+// when the caller switches contexts).  The lookup allocates nothing.
 #include <cstddef>
-#include <mutex>
 
 #include "gdr.h"
 #include "gdr_internal.h"
@@ -18,24 +19,13 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[GDR_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_static_scratch on the current device (set up on first use).
+// Device address of g_static_scratch in the current device context, or nullptr.
 void *scratch_on_current_device()
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess)
         return nullptr;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void *addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || addr == nullptr)
-            return nullptr;
-        g_scratch_addr[dev] = addr;
-    }
-    return g_scratch_addr[dev];
+    return addr;
 }
 
 }  // namespace

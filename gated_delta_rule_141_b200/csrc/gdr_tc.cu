@@ -589,6 +589,29 @@ int launch_scalar(const Params &p, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }
 
+// Self-test of the bounded-wait path every tensor-core kernel relies on: one
+// warp takes tensor memory, waits on an mbarrier that nothing ever arrives on,
+// gives up after limit_ns of wall time exactly as the production waits do (the
+// status word becomes the timeout code), releases the tensor memory and returns.
+__global__ void __launch_bounds__(32, 1) wait_probe_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t slot;
+    tmem_alloc(&slot, 32);
+    tmem_relinquish();
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    tc_fence_before();
+    __syncwarp();
+    tc_fence_after();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit_ns))
+        atomicExch(&g_device_status, kTimeoutStatus);
+    __syncwarp();
+    tmem_dealloc(slot, 32);
+}
+
 #include "gdr_tc_ws.cuh"
 #include "gdr_tc_gen.cuh"
 #include "gdr_tc_prep.cuh"
@@ -656,6 +679,12 @@ int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
         return rc;
     return p.out_bf16 ? split::launch<true>(p, workspace, stream)
                       : split::launch<false>(p, workspace, stream);
+}
+
+int launch_wait_probe(uint64_t limit_ns, cudaStream_t stream)
+{
+    wait_probe_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }
 
 bool prepare_supports(const Params &p) { return prep::supports(p); }

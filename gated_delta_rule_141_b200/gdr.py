@@ -45,6 +45,7 @@ EXPORTS = ("gdr_chunk_fwd", "gdr_chunk_fwd_momentum", "gdr_chunk_bwd", "gdr_bwd_
            "gdr_chunk_fwd_static",
            "gdr_output_gate_rmsnorm",
            "gdr_select_kernel", "gdr_kernel_chunk", "gdr_state_segments", "gdr_device_status",
+           "gdr_selftest_bounded_wait",
            "gdr_status_string",
            "gdr_version")
 
@@ -113,6 +114,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_output_gate_rmsnorm.restype = i
     lib.gdr_device_status.argtypes = [vp]
     lib.gdr_device_status.restype = i
+    lib.gdr_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+    lib.gdr_selftest_bounded_wait.restype = i
     lib.gdr_status_string.argtypes = [i]
     lib.gdr_status_string.restype = ctypes.c_char_p
     lib.gdr_version.argtypes = []
@@ -176,6 +179,12 @@ def workspace_bytes(shape: GdrShape, chunk: int, gate_mode: int, inverse: str = 
 
 def device_status(stream=None) -> int:
     return int(load().gdr_device_status(_stream_handle(stream)))
+
+
+def selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    """Launch the library's bounded-wait self-test (a wait nothing ends, given up
+    after limit_ns); its status shows in device_status()."""
+    return int(load().gdr_selftest_bounded_wait(int(limit_ns), _stream_handle(stream)))
 
 
 def _stream_handle(stream):

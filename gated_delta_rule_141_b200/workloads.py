@@ -124,10 +124,11 @@ def make_inputs(w: Workload, seed: int) -> dict:
     return dict(q=q, k=k, v=v, g=g, beta=beta, S0=S0)
 
 
-def workload_inputs(index: int, **overrides) -> tuple:
-    """(workload, inputs) for workload `index` with the standard seed 1000 + index;
-    `overrides` shrink a workload (e.g. T=512) while keeping its distributions."""
+def workload_inputs(index: int, seed=None, **overrides) -> tuple:
+    """(workload, inputs) for workload `index` with the standard seed 1000 + index
+    (or `seed`); `overrides` shrink a workload (e.g. T=512) while keeping its
+    distributions."""
     w = WORKLOADS[index]
     if overrides:
         w = w.scaled(**overrides)
-    return w, make_inputs(w, 1000 + index)
+    return w, make_inputs(w, 1000 + index if seed is None else seed)

@@ -288,9 +288,11 @@ gdr_status gdr_chunk_fwd_host(const gdr_shape *shape, const gdr_io *host, const 
  * request whose TC2 workspace (gdr_workspace_bytes) is larger fails with
  * GDR_ERR_SCRATCH_LIMIT before anything is launched.  Nothing is allocated:
  * no cudaMalloc, no cudaFree, no allocating library call.
- *  - Set-up: the first call on a device, made with that device current, looks
- *    up the array's device address (cudaGetSymbolAddress) and remembers it;
- *    make that first call before any stream capture.
+ *  - Set-up: every call looks up the array's device address in the device
+ *    context current at that moment (cudaGetSymbolAddress, which allocates
+ *    nothing), so the address is never stale after a cudaDeviceReset or a
+ *    context switch.  The first call on a device can load the library's
+ *    device code there; make that first call before any stream capture.
  *  - Sharing: every call on a device uses the same array, which keeps what the
  *    last call left there.  Nothing in it needs clearing between calls (each
  *    call rewrites all it reads), but two calls that overlap on the GPU (other
@@ -353,6 +355,18 @@ gdr_status gdr_output_gate_rmsnorm(const gdr_shape *shape, void *o, const void *
  * kernels set when a bounded wait gives up (GDR_OK or GDR_ERR_TIMEOUT), or
  * GDR_ERR_CUDA if the stream reported an error. */
 gdr_status gdr_device_status(void *stream);
+
+/*
+ * gdr_selftest_bounded_wait -- test of the failure path of the kernels'
+ * bounded waits (no counterpart in the pages; a diagnostic of this library).
+ * Launches one warp on `stream` that takes tensor memory, waits on an
+ * mbarrier nothing arrives on, gives up after limit_ns nanoseconds of wall
+ * time (1e3 .. 1e9, else GDR_ERR_ARG), sets the status word that
+ * gdr_device_status() reports as GDR_ERR_TIMEOUT, releases the tensor memory
+ * and returns: the CUDA context stays usable.  No forward entry point
+ * reaches it.
+ */
+gdr_status gdr_selftest_bounded_wait(uint64_t limit_ns, void *stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char *gdr_status_string(gdr_status status);

@@ -17,7 +17,7 @@ def pytest_configure(config):
 # that a failure in an extension (under -x) cannot hide them; the static-
 # workspace file stays last, as its name intends.  The sort is stable.
 _GPU_ORDER = ["test_gpu_parity", "test_gpu_prepare", "test_gpu_segmented", "test_gpu_epilogue",
-              "test_gpu_momentum", "test_gpu_two_pass_simt", "test_gpu_vjp"]
+              "test_gpu_momentum", "test_gpu_two_pass_simt", "test_gpu_vjp", "test_gpu_timeout"]
 
 
 def pytest_collection_modifyitems(session, config, items):

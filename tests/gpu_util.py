@@ -78,8 +78,17 @@ def oracle_reference(inputs: dict, chunk: int, inverse: str, order: int = 4, res
     return oracle.chunked(*args, chunk=chunk, inverse=inverse, order=order, resid=resid)
 
 
-def sample_sequences(w: W.Workload, count: int = 3):
-    """Deterministic sample of (b, hv) pairs: first, last and a middle one."""
+def sample_sequences(w: W.Workload, count: int = 8):
+    """Deterministic sample of at least `count` (b, hv) pairs (all of them when
+    there are fewer): the first and the last sequence, every value head of the
+    middle key head of a middle batch entry (all R heads that share one key
+    head's factors), then sequences spread evenly over the grid."""
     total = w.B * w.Hv
-    picks = sorted(set([0, total - 1, total // 2, (7 * total) // 13][:count]))
-    return [(s // w.Hv, s % w.Hv) for s in picks]
+    picks = {0, total - 1}
+    bm, hk = w.B // 2, w.Hk // 2
+    picks.update(bm * w.Hv + hk * w.R + r for r in range(w.R))
+    j = 0
+    while len(picks) < min(count, total):
+        picks.add((j * total) // count + (j * 3) % max(1, total // count))
+        j += 1
+    return [(s // w.Hv, s % w.Hv) for s in sorted(picks)]

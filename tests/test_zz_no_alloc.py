@@ -1,8 +1,9 @@
 """gdr_chunk_fwd_static -- the entry point for callers that may not allocate
 device memory on their call path (its workspace is a fixed array inside the
-library).  Called through the C ABI twice in a row, it must give what
-gdr_chunk_fwd gives with a caller-owned workspace, within the bf16 bound of the
-parity tests; requests too large for the array are refused before any launch.
+library).  Called through the C ABI twice in a row on different inputs, it must give
+exactly what gdr_chunk_fwd gives with a caller-owned workspace, and match the
+oracle within the bf16 bound of the parity tests; requests too large for the
+array are refused before any launch.
 
 The file is named so that pytest collects it after every other test file."""
 import ctypes
@@ -41,32 +42,41 @@ def _static_call(lib, dev, shape, chunk, gate, o, Sf):
                                     stream)
 
 
-# (workload, overrides): scalar gate with grouped values; per-channel decay with a ragged tail
-CASES = [(1, dict(B=2, Hk=2, Hv=4, T=320)), (2, dict(B=1, Hk=2, Hv=2, T=448 - 37))]
+# (workload, overrides): scalar gate with grouped values; per-channel decay with a
+# ragged tail; one long sequence, whose state pass runs segment-parallel (its
+# segment states live in the array too)
+CASES = [(1, dict(B=2, Hk=2, Hv=4, T=320)), (2, dict(B=1, Hk=2, Hv=2, T=448 - 37)),
+         (1, dict(B=1, Hk=1, Hv=1, T=64 * 48 + 1))]
 
 
-@pytest.mark.parametrize("idx,over", CASES, ids=["w%d" % c[0] for c in CASES])
+@pytest.mark.parametrize("idx,over", CASES, ids=["w%d-T%d" % (c[0], c[1]["T"]) for c in CASES])
 def test_static_entry_matches_workspace_entry(lib, idx, over):
+    """Two calls in a row on different seeded inputs: each must equal, bit for bit,
+    gdr_chunk_fwd with a caller-owned workspace on the same inputs (the same kernels
+    with no atomics, so the same bits), and match the oracle within the bf16
+    bound.  Different inputs make stale contents of the shared array visible."""
     import torch
     from gated_delta_rule_141_b200 import gdr
-    w, x = W.workload_inputs(idx, **over)
-    dev = U.to_device(x, "bf16")
+    w, _ = W.workload_inputs(idx, **over)
     gate = gdr.gate_mode_for(w.G, w.dk)
     shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv)
-    o_ref, S_ref = gdr.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
-                                 chunk=64, gate_mode=gate, kernel="tc2")
-    torch.cuda.synchronize()
-    o_ref = o_ref.float().cpu().numpy()
-    S_ref = S_ref.cpu().numpy()
+    if over["T"] > 64 * 32:
+        assert gdr.state_segments(shape, 64, gate) > 1
     for call in range(2):
+        _, x = W.workload_inputs(idx, seed=5000 + 17 * call + idx, **over)
+        dev = U.to_device(x, "bf16")
+        o_ref, S_ref = gdr.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                                     dev["S0"], chunk=64, gate_mode=gate, kernel="tc2")
         o = torch.full((w.B, w.Hv, w.T, w.dv), float("nan"), dtype=torch.bfloat16, device="cuda")
         Sf = torch.full((w.B, w.Hv, w.dk, w.dv), float("nan"), dtype=torch.float32, device="cuda")
         assert _static_call(lib, dev, shape, 64, gate, o, Sf) == gdr.OK
         torch.cuda.synchronize()
         assert gdr.device_status() == gdr.OK
-        eo = U.rel_err(o.float().cpu().numpy(), o_ref)
-        es = U.rel_err(Sf.cpu().numpy(), S_ref)
-        print("call %d: rel err o %.3e  S_final %.3e" % (call, eo, es))
+        assert torch.equal(o, o_ref) and torch.equal(Sf, S_ref), "call %d differs" % call
+        oo, So = U.oracle_reference(x, 64, "exact")
+        eo = U.rel_err(o.float().cpu().numpy(), oo)
+        es = U.rel_err(Sf.cpu().numpy(), So)
+        print("call %d: rel err vs oracle o %.3e  S_final %.3e" % (call, eo, es))
         assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
 
 
