@@ -17,6 +17,8 @@ struct Params {
     int out_bf16;   // o is bf16 (else fp32)
     int neumann;    // 0 exact inverse, 1 truncated Neumann
     int neumann1;   // 1-Step Neumann in blocks of 16 (neumann is 0 then)
+    int pair;       // two-pass path: the request's chunk of 2C runs as pairs of C-token
+                    // halves, the second half corrected by the pair's Y (internal)
     int neu_order;  // Neumann order m
     int neu_resid;  // Newton residual corrections
     int momentum;   // chunk-boundary momentum (CUDA-core kernel only)

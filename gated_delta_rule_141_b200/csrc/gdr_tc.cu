@@ -615,6 +615,7 @@ __global__ void __launch_bounds__(32, 1) wait_probe_kernel(uint64_t limit_ns)
 #include "gdr_tc_ws.cuh"
 #include "gdr_tc_gen.cuh"
 #include "gdr_tc_prep.cuh"
+#include "gdr_tc_pair.cuh"
 #include "gdr_tc_split.cuh"
 
 }  // namespace
@@ -622,20 +623,30 @@ __global__ void __launch_bounds__(32, 1) wait_probe_kernel(uint64_t limit_ns)
 // In exact mode the chunkwise form reaches the token recurrence exactly for any
 // chunk length (the WY equivalence of the SLA paper, §2.4.2), so a request for
 // C = 128 runs on the C = 64 kernels: the same function, blocked more finely.
-// The truncated Neumann inverse depends on C and is never re-blocked.
+// The truncated Neumann inverse depends on C: at C = 128 the two-pass path runs
+// it as pairs of 64-token halves with the pair correction (gdr_tc_pair.cuh),
+// which the one-pass kernels do not have.
 static Params as_kernel_chunk(const Params &p)
 {
     Params q = p;
-    if (!p.neumann && !p.neumann1 && p.C == 128)   // the exact form only
+    if (!p.neumann1 && p.C == 128) {
         q.C = CH;
+        q.pair = p.neumann;
+    }
     return q;
 }
 
-int tc_kernel_chunk(const Params &p) { return as_kernel_chunk(p).C; }
+int tc_kernel_chunk(const Params &p)
+{
+    const Params q = as_kernel_chunk(p);
+    return q.pair ? 2 * q.C : q.C;
+}
 
 bool tc_supports(const Params &p0)
 {
     const Params p = as_kernel_chunk(p0);
+    if (p.pair)
+        return false;
     const bool scalar64 = p.in_bf16 && p.G == 1 && p.C == CH && p.dk == 64 && p.dv % NV == 0 &&
                           !p.neumann && p.T >= 1 && p.B <= 65535;
     // the one-pass kernels have no 1-Step Neumann inverse
@@ -645,6 +656,8 @@ bool tc_supports(const Params &p0)
 int launch_tc(const Params &p0, cudaStream_t stream)
 {
     const Params p = as_kernel_chunk(p0);
+    if (p.pair)
+        return 5;
     if (ws::supports(p))
         return p.out_bf16 ? ws::launch<true>(p, stream) : ws::launch<false>(p, stream);
     if (gen::supports(p)) {
@@ -674,7 +687,9 @@ int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
     const Params p = as_kernel_chunk(p0);
     if (!split::supports(p))
         return 5;
-    const int rc = prep::launch<128>(p, workspace, prep::record_kind(p), stream);
+    int rc = prep::launch<128>(p, workspace, prep::record_kind(p), stream, p.pair);
+    if (rc == 0 && p.pair)
+        rc = pair::launch<128>(p, workspace, stream);
     if (rc != 0)
         return rc;
     return p.out_bf16 ? split::launch<true>(p, workspace, stream)

@@ -1,0 +1,420 @@
+// gdr_tc_pair.cuh -- the truncated Neumann inverse at chunk 2C = 128 on the
+// two-pass path, with the state pass stepping by C = 64.  Included by gdr_tc.cu.
+//
+// "When Good Enough Is Optimal: Multiplication-Only Matrix Inversion
+// Approximation for Quantized Gated DeltaNet" (§4.1, Lemma 3.1) truncates the
+// Neumann series of (I + M)^{-1} for a whole chunk; the result depends on the
+// chunk length, so a 128-token request cannot simply be blocked by 64 as the
+// exact inverse can.  Split the chunk into halves 1 and 2.  With G the chunk's
+// decayed Gram (G_tj = sum_i k_ti k_ji e^{Lambda_ti - Lambda_ji}, t > j),
+// M = G diag(beta), A the truncated series with its Newton steps and
+// T = diag(beta) A, the blocks of powers and products of block-lower-triangular
+// matrices are the products of their blocks, so T11 and T22 are exactly the
+// 64-token factors of each half (what the first pass writes).  Only T21 is
+// unseen by a state pass that steps half by half.  Stepping half 2 from the
+// state at the half boundary gives
+//   E2' = T22 (V2 - Kbar2 S) - T22 G21 E1,
+// while the 128-token chunk has E2 = T21 (V1 - Kbar1 S) + T22 (V2 - Kbar2 S),
+// with S the pair's start state and E1 = T11 (V1 - Kbar1 S) the first half's E.
+// In the similar form Atil = diag(beta) A diag(beta)^{-1} (the same series of
+// Ntil = diag(beta) G, beta on the rows; unit lower triangular),
+// T21 = Atil21 diag(beta1) and T11 = Atil11 diag(beta1), hence
+//   E2 = E2' + Y E1,   Y = Atil21 Atil11^{-1} + Atil22 Ntil21,
+// and the half's output and state update follow from that E2 unchanged.  (For
+// the exact inverse Y = 0: that is why exact requests at 128 run by 64.)
+//
+// pair_kernel, one CTA (256 threads) per (batch, key head, pair of halves):
+//   1. bulk copies of Ntil11, Ntil22 (first-pass images) and the operands of
+//      G21 = Kbar2' Khat1^T (Kbar2' = k2 e^{Lambda_t - Lambda_mid},
+//      Khat1 = k1 e^{Lambda_mid - Lambda_j}: both <= 1, no pivot needed);
+//   2. G21 on tcgen05, Ntil21 = diag(beta2) G21 into the 128 x 128 Ntil tile;
+//   3. Atil by Horner's rule (X <- I - Ntil X, m times) and r Newton steps
+//      (X <- X + X (I - X - Ntil X)), all products M = N = K = 128 on tcgen05,
+//      X kept in fp32 in tensor memory and as a bf16 operand in shared memory;
+//   4. Atil11^{-1} exactly in fp32 (block doubling), Y in fp32 on the CUDA cores;
+//   5. Y as a bf16 image into the first half's record.
+// The state pass loads Y under L ([L; Y] tile), so its [L; Y] E product of the
+// first half leaves Y E1 in the tensor-memory rows it reads for the second.
+
+namespace pair {
+
+constexpr int NT = 256;
+constexpr int CC = 64;
+constexpr int LDM = gen::LDM;
+constexpr uint32_t TMEM_COLS = 256;   // product (128 columns), X in fp32 (128 columns)
+constexpr uint32_t T_D = 0, T_X = 128;
+
+struct Plan {
+    uint32_t NTL, XT, RT, Tf, beta, bar, misc, total;
+};
+
+__host__ __device__ inline Plan plan()
+{
+    Plan s;
+    uint32_t o = 0;
+    auto take = [&](uint32_t bytes) {
+        const uint32_t at = o;
+        o += (bytes + 1023u) & ~1023u;
+        return at;
+    };
+    s.NTL = take(2 * 128 * 128);        // Ntil, 128 x 128 bf16
+    s.XT = take(2 * 128 * 128);         // X, 128 x 128 bf16
+    s.RT = take(2 * 128 * 128);         // Newton residual; first the G21 operands
+    s.Tf = take(32 * 36 * 4 + 1024);    // scratch of the fp32 block inverse
+    s.beta = take(3 * CC * 4);          // beta2, then (scalar gate) ea2, eb1
+    s.bar = take(64);
+    s.misc = s.bar + 32;
+    s.total = o + 1024;
+    return s;
+}
+
+struct PairArgs {
+    Params p;                 // the request at the half length (C = 64, pair = 1)
+    uint8_t *rec;             // the first pass's records, [B * Hk * nchunks][rec_bytes]
+    int nchunks;              // halves per sequence
+    uint32_t rec_bytes;
+    uint32_t base_bytes;      // offset of the pair extras in a record
+    int ext;                  // grouped / per-channel records (else the scalar gate's)
+};
+
+// fp32 views of the regions freed once the series is done (stride LDM)
+__device__ __forceinline__ float *f32(uint8_t *base, uint32_t off) { return reinterpret_cast<float *>(base + off); }
+
+template <int DK>
+__global__ void __launch_bounds__(NT, 2)
+pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
+{
+    using namespace ptx;
+    extern __shared__ uint8_t smem_raw[];
+    const Params &p = a.p;
+    const Plan Ly = plan();
+    const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *base = smem_raw + (base_u32 - smem_u32(smem_raw));
+    const uint32_t NTL = base_u32 + Ly.NTL, XT = base_u32 + Ly.XT, RT = base_u32 + Ly.RT;
+    float *Tf = f32(base, Ly.Tf);
+    float *sbeta = f32(base, Ly.beta);          // beta of half 2
+    float *ea2 = sbeta + CC, *eb1 = sbeta + 2 * CC;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pr = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const long kh = (long)b * p.Hk + hk;
+    const int c1 = 2 * pr, c2 = c1 + 1;
+    const int T = p.T;
+    uint8_t *rec1 = a.rec + (size_t)(kh * a.nchunks + c1) * a.rec_bytes;
+    uint8_t *img_Y = rec1 + a.base_bytes + prep::PAIR_Y;
+
+    // no second half (odd number of halves): nothing follows, Y = 0
+    if (c2 >= a.nchunks) {
+        for (int u = tid; u < CC * 8; u += NT)
+            reinterpret_cast<uint4 *>(img_Y)[u] = make_uint4(0u, 0u, 0u, 0u);
+        return;
+    }
+    const uint8_t *rec2 = rec1 + a.rec_bytes;
+    const long c0_2 = (long)c2 * CC;
+    const int Cl2 = (int)min((long)CC, T - c0_2);
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);   // loads
+        mbar_init(&bars[1], 1);   // MMA
+        fence_barrier_init();
+        uint64_t *full = &bars[0];
+        const uint32_t opnd = (uint32_t)(CC * DK * 2);   // one 64-row operand tile
+        mbar_arrive_expect_tx(full, 2u * prep::IMG + 2u * opnd);
+        bulk_load(base + Ly.NTL, rec1 + a.base_bytes + prep::PAIR_N, prep::IMG, full);
+        bulk_load(base + Ly.NTL + 128 * 128 + 64 * 128, rec2 + a.base_bytes + prep::PAIR_N, prep::IMG, full);
+        if (a.ext) {
+            // Khat1 (the first half's record) and Kbar2 (the second half's pair extra),
+            // 64-row tiles of DK / 64 column blocks, as the records store them
+            bulk_load(base + Ly.RT, rec1 + prep::EXT_KH, opnd, full);
+            bulk_load(base + Ly.RT + opnd, rec2 + a.base_bytes + prep::PAIR_KB, opnd, full);
+        } else {
+            for (int kb = 0; kb < DK / 64; ++kb) {
+                tma_load_3d(base + Ly.RT + kb * 64 * 128, &tm_k, full, 64 * kb, c1 * CC, (int)kh);
+                tma_load_3d(base + Ly.RT + opnd + kb * 64 * 128, &tm_k, full, 64 * kb, (int)c0_2, (int)kh);
+            }
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    for (int t = tid; t < CC; t += NT) {
+        sbeta[t] = t < Cl2 ? p.beta[kh * T + c0_2 + t] : 0.f;
+        if (!a.ext) {   // e^{Lambda_t} of half 2, e^{Lambda_mid - Lambda_j} of half 1
+            ea2[t] = reinterpret_cast<const float *>(rec2 + prep::SC_EA)[t];
+            eb1[t] = reinterpret_cast<const float *>(rec1 + prep::SC_EB)[t];
+        }
+    }
+    // the zero block of Ntil (rows 0-63 of columns 64-127), X = I
+    for (int u = tid; u < 64 * 8; u += NT) {
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        st_tile8(NTL, 128, u >> 3, 64 + (u & 7) * 8, z);
+    }
+    for (int u = tid; u < 128 * 16; u += NT) {
+        const int r = u >> 4, c = (u & 15) * 8;
+        float x8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            x8[e] = (r == c + e) ? 1.f : 0.f;
+        st_tile8(XT, 128, r, c, x8);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+
+    uint32_t ph_mma = 0;
+    bool failed = false;
+    auto wait_bar = [&](int i, uint32_t ph) {
+        const bool gave_up = !mbar_wait(&bars[i], ph);
+        if (gave_up)
+            atomicExch(&g_device_status, kTimeoutStatus);
+        return __syncthreads_or(gave_up ? 1 : 0) != 0;
+    };
+    failed = wait_bar(0, 0);
+    const uint32_t KH1 = RT, KB2 = RT + (uint32_t)(CC * DK * 2);
+    if (!failed && !a.ext) {   // scalar gate: scale the raw k rows by their decay factors
+        for (int u = tid; u < 2 * CC * (DK / 8); u += NT) {
+            const int h = u / (CC * (DK / 8)), r = (u / (DK / 8)) % CC, i0 = (u % (DK / 8)) * 8;
+            const uint32_t tile = h == 0 ? KH1 : KB2;
+            const float f = h == 0 ? eb1[r] : ea2[r];
+            float v8[8];
+            ld_tile8(tile, 64, r, i0, v8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                v8[e] *= f;
+            st_tile8(tile, 64, r, i0, v8);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    // ---- G21 = Kbar2' Khat1^T (M = 64, N = 64, K = DK)
+    if (!failed) {
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(64, 64, false, false);
+            for (int k0 = 0; k0 < DK; k0 += 16)
+                mma_bf16(tmem + T_D, desc_kmajor(KB2, 64, 0, k0), desc_kmajor(KH1, 64, 0, k0), id, k0 > 0);
+            mma_commit(&bars[1]);
+        }
+        failed = wait_bar(1, ph_mma);
+        ph_mma ^= 1u;
+    }
+    if (!failed) {
+        tc_fence_after();
+        const int rr = gen::row64g(warp, lane);
+        const int cb = 32 * (warp >> 2);
+        float d0[16], d1[16];
+        tmem_ld16(tq + T_D + cb, d0);
+        tmem_ld16(tq + T_D + cb + 16, d1);
+        tmem_ld_wait();
+        if (rr >= 0) {
+            const float bt = sbeta[rr];
+            float n[32];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                n[u] = bt * d0[u];
+                n[16 + u] = bt * d1[u];
+            }
+#pragma unroll
+            for (int u = 0; u < 32; u += 8)
+                st_tile8(NTL, 128, 64 + rr, cb + u, &n[u]);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- the 128 x 128 series: products D = A B with M = N = K = 128
+    const int R = 32 * (warp & 3) + lane;   // row of this thread (lane of its quarter)
+    const int ch = 64 * (warp >> 2);        // its 64 columns
+    const uint32_t id128 = idesc_bf16(128, 128, false, true);
+    auto product = [&](uint32_t a_tile, uint32_t b_tile) {
+        if (tid == 0) {
+            tc_fence_after();
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma_bf16(tmem + T_D, desc_kmajor(a_tile, 128, 0, k0), desc_mnmajor(b_tile, 128, k0, 0),
+                         id128, k0 > 0);
+            mma_commit(&bars[1]);
+        }
+        const bool f = wait_bar(1, ph_mma);
+        ph_mma ^= 1u;
+        if (!f)
+            tc_fence_after();
+        return f;
+    };
+    // X (fp32, tensor memory) and its bf16 operand: this thread's row R, 16 columns at a time
+    auto put_x = [&](int c, const float (&x)[16]) {
+        tmem_st16(tq + T_X + c, x);
+        st_tile8(XT, 128, R, c, &x[0]);
+        st_tile8(XT, 128, R, c + 8, &x[8]);
+    };
+    if (!failed && p.neu_order == 0) {
+        for (int c = ch; c < ch + 64; c += 16) {
+            float x[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                x[e] = (R == c + e) ? 1.f : 0.f;
+            tmem_st16(tq + T_X + c, x);
+        }
+    }
+    for (int pw = 1; pw <= p.neu_order && !failed; ++pw) {   // X <- I - Ntil X
+        if ((failed = product(NTL, XT)))
+            break;
+        for (int c = ch; c < ch + 64; c += 16) {
+            float d[16], x[16];
+            tmem_ld16(tq + T_D + c, d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                x[e] = ((R == c + e) ? 1.f : 0.f) - d[e];
+            put_x(c, x);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    }
+    for (int st = 0; st < p.neu_resid && !failed; ++st) {   // Newton: X <- X + X (I - X - Ntil X)
+        if ((failed = product(NTL, XT)))
+            break;
+        for (int c = ch; c < ch + 64; c += 16) {
+            float d[16], x[16];
+            tmem_ld16(tq + T_D + c, d);
+            tmem_ld16(tq + T_X + c, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                d[e] = ((R == c + e) ? 1.f : 0.f) - x[e] - d[e];
+            st_tile8(RT, 128, R, c, &d[0]);
+            st_tile8(RT, 128, R, c + 8, &d[8]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if ((failed = product(XT, RT)))
+            break;
+        for (int c = ch; c < ch + 64; c += 16) {
+            float d[16], x[16];
+            tmem_ld16(tq + T_D + c, d);
+            tmem_ld16(tq + T_X + c, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                x[e] += d[e];
+            put_x(c, x);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    // ---- Y = Atil21 Atil11^{-1} + Atil22 Ntil21 in fp32 (regions of the dead tiles)
+    float *N21f = f32(base, Ly.XT);                      // 64 x LDM each
+    float *A11f = N21f + CC * LDM;
+    float *A21f = A11f + CC * LDM;
+    float *A22f = f32(base, Ly.NTL);                     // once Ntil21 is copied out
+    if (!failed) {
+        tc_fence_after();
+        // Atil from tensor memory: rows 0-63 x columns 0-63 (strict lower part, as I + H
+        // for the inverse), rows 64-127 x columns 0-63 (Atil21)
+        if (ch == 0) {
+            for (int c = 0; c < 64; c += 16) {
+                float x[16];
+                tmem_ld16(tq + T_X + c, x);
+                tmem_ld_wait();
+                if (R < 64) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        A11f[R * LDM + c + e] = (R > c + e) ? x[e] : 0.f;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        A21f[(R - 64) * LDM + c + e] = x[e];
+                }
+            }
+        }
+        for (int u = tid; u < CC * 8; u += NT) {          // Ntil21 as the bf16 the series used
+            const int t = u >> 3, j0 = (u & 7) * 8;
+            float v8[8];
+            ld_tile8(NTL, 128, 64 + t, j0, v8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                N21f[t * LDM + j0 + e] = v8[e];
+        }
+    }
+    __syncthreads();
+    if (!failed && ch == 64 && R >= 64) {                 // Atil22: rows and columns 64-127
+        for (int c = 64; c < 128; c += 16) {
+            float x[16];
+            tmem_ld16(tq + T_X + c, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                A22f[(R - 64) * LDM + c - 64 + e] = x[e];
+        }
+    }
+    __syncthreads();
+    if (!failed) {
+        gen::inverse64_inplace(A11f, Tf, tid);            // Atil11^{-1}, lower triangular
+        const int rg = tid >> 4, c0 = 4 * (tid & 15);     // rows rg + 16 i, columns c0..c0+3
+        float y[4][4], z[4][4];
+        gen::block_product4x4<64>(y, A21f + rg * LDM, 16 * LDM, A11f + c0, LDM, c0);
+        gen::block_product4x4<64>(z, A22f + rg * LDM, 16 * LDM, N21f + c0, LDM, 0);
+        __syncthreads();                                  // every read of A21f done
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+                A21f[(rg + 16 * i) * LDM + c0 + n] = y[i][n] + z[i][n];
+        __syncthreads();
+        for (int u = tid; u < CC * 8; u += NT) {          // Y as a 128-byte-swizzled image
+            const int t = u >> 3, j0 = (u & 7) * 8;
+            prep::st_img8(img_Y, t, j0, A21f + t * LDM + j0);
+        }
+    }
+    if (tid == 0 && failed) {   // drain what was started before releasing tensor memory
+        mma_commit(&bars[1]);
+        mbar_wait(&bars[1], ph_mma, 200000000ull);
+        mbar_wait(&bars[0], 0, 200000000ull);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+inline int npairs(int nchunks) { return (nchunks + 1) / 2; }
+
+template <int DK>
+int launch(const Params &p, void *records, cudaStream_t stream)
+{
+    const int N = prep::nchunks(p);
+    if (N == 0 || p.B == 0)
+        return 0;
+    CUtensorMap mk;
+    if (!make_map(&mk, p.k, DK, p.T, (long)p.B * p.Hk, CC))
+        return 6;
+    const Plan Ly = plan();
+    if (cudaFuncSetAttribute(pair_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
+        cudaSuccess)
+        return 6;
+    PairArgs a;
+    a.p = p;
+    a.rec = static_cast<uint8_t *>(records);
+    a.nchunks = N;
+    a.rec_bytes = prep::rec_bytes(p);
+    a.base_bytes = prep::kind_bytes(prep::record_kind(p));
+    a.ext = prep::record_kind(p) == prep::REC_EXT;
+    pair_kernel<DK><<<dim3(npairs(N), p.Hk, p.B), NT, Ly.total, stream>>>(mk, a);
+    return cudaGetLastError() == cudaSuccess ? 0 : 6;
+}
+
+}  // namespace pair

@@ -54,6 +54,14 @@ constexpr uint32_t EXT_QB = 4 * IMG, EXT_KH = EXT_QB + 2 * IMG;
 constexpr uint32_t EXT_F = EXT_KH + 2 * IMG;
 constexpr uint32_t EXT_BYTES = EXT_F + 128 * 4;
 enum RecordKind { REC_PLAIN = 0, REC_SCALAR = 1, REC_EXT = 2 };
+// Pair records (the truncated Neumann inverse at C = 128 run as two 64-token
+// halves): the base record, then Y (the pair's correction, written by
+// pair_kernel into the record of the pair's first half), Ntil = diag(beta) x the
+// decayed Gram of the half (beta on the rows: strictly lower, bf16 image) and,
+// for grouped / per-channel gates, Kbar = k e^{Lambda_t} (64 x 128 bf16, two
+// images).
+constexpr uint32_t PAIR_Y = 0, PAIR_N = IMG, PAIR_KB = 2 * IMG;   // offsets past the base record
+__host__ __device__ constexpr uint32_t pair_extra(int kind) { return kind == REC_EXT ? 4 * IMG : 2 * IMG; }
 
 __host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
 
@@ -106,6 +114,8 @@ struct PrepArgs {
     int nchunks;
     int kind;          // RecordKind: what besides T and L the record carries
     uint32_t rec_bytes;
+    uint32_t base_bytes;   // the kind's own record; pair extras follow it (pair != 0)
+    int pair;              // also write the pair extras (Ntil, and Kbar for REC_EXT)
 };
 
 // Store 8 floats as bf16 into the 16-byte chunk of row r holding columns [c, c+8)
@@ -389,7 +399,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     float v = 0.f;
                     if (keep)
                         v = !SCALAR ? d : sc_piv ? d * (Tf[t] * Tf[CC + j]) : d * __expf(lt - lam[j]);
-                    if (!qrow)
+                    if (!qrow && !a.pair)   // pairs: the raw Gram, beta applied before the inverse
                         v *= sbeta[j];
                     out[u] = v;
                 }
@@ -484,7 +494,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int jj = c0 + cb + e;
-                            v[e] = qrow ? ((jj <= t) ? d[e] : 0.f) : ((jj < t) ? sbeta[jj] * d[e] : 0.f);
+                            v[e] = qrow ? ((jj <= t) ? d[e] : 0.f)
+                                        : ((jj < t) ? (a.pair ? d[e] : sbeta[jj] * d[e]) : 0.f);
                         }
                         if (qrow) {
                             st_img8(img_L, t, c0 + cb, &v[0]);
@@ -543,13 +554,33 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = j0 + e;
-                        mv[e] = (j < t) ? sbeta[j] * mv[e] : 0.f;
+                        mv[e] = (j < t) ? (a.pair ? mv[e] : sbeta[j] * mv[e]) : 0.f;
                         lv[e] = (j <= t) ? lv[e] : 0.f;
                         Mf[t * LDM + j] = mv[e];
                     }
                     st_img8(img_L, t, j0, lv);
                 }
             }
+        }
+    }
+    if (!failed && a.pair) {
+        // Mf holds the decayed Gram of the k rows (strictly lower): the pair kernel's
+        // Ntil = diag(beta) Gram (beta on the rows) as an image, then M = Gram diag(beta)
+        __syncthreads();
+        uint8_t *img_N = img_T + a.base_bytes + PAIR_N;
+        for (int u = tid; u < CC * 8; u += NT) {
+            const int t = u >> 3, j0 = (u & 7) * 8;
+            float nv[8], mv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float gr = Mf[t * LDM + j0 + e];
+                nv[e] = sbeta[t] * gr;
+                mv[e] = gr * sbeta[j0 + e];
+            }
+            st_img8(img_N, t, j0, nv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                Mf[t * LDM + j0 + e] = mv[e];
         }
     }
     if (!failed) {
@@ -690,6 +721,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (w_cols)
             for (int i = tid; i < DK; i += NT)
                 Tf[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);
+        if (a.pair && !SCALAR) {
+            // Kbar = k e^{Lambda_t} for the pair kernel: the k rows hold it after the
+            // pivoted blocks; after the chunk-end pivot they hold k e^{Lambda_t - Lambda_C}
+            __syncthreads();
+            uint8_t *img_K = img_T + a.base_bytes + PAIR_KB;
+            for (int u = tid; u < CC * (DK / 8); u += NT) {
+                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                float kv[8];
+                ld_tile8(QK, 128, 64 + t, i0, kv);
+                if (w_cols)   // Tf holds e^{Lambda_C} per channel here
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        kv[e] *= Tf[i0 + e];
+                st_img8(img_K + (i0 >> 6) * IMG, t, i0 & 63, kv);
+            }
+        }
         if (SCALAR && with_w) {   // e^{Lambda_j} for W's operand, once per token
             for (int t = tid; t < CC; t += NT)
                 Tf[2 * CC + t] = __expf(lam[t]);
@@ -795,7 +842,10 @@ inline uint32_t kind_bytes(int kind)
     return kind == REC_EXT ? EXT_BYTES : (kind == REC_SCALAR ? SC_BYTES : CHUNK_BYTES);
 }
 
-inline uint32_t rec_bytes(const Params &p) { return kind_bytes(record_kind(p)); }
+inline uint32_t rec_bytes(const Params &p)
+{
+    return kind_bytes(record_kind(p)) + (p.pair ? pair_extra(record_kind(p)) : 0u);
+}
 
 inline size_t ws_bytes(const Params &p) { return (size_t)p.B * p.Hk * nchunks(p) * rec_bytes(p); }
 
@@ -806,7 +856,7 @@ inline bool supports(const Params &p)
 }
 
 template <int DK>
-int launch(const Params &p, void *out, int kind, cudaStream_t stream)
+int launch(const Params &p, void *out, int kind, cudaStream_t stream, int pair = 0)
 {
     const int N = nchunks(p);
     if (N == 0 || p.B == 0)
@@ -825,7 +875,9 @@ int launch(const Params &p, void *out, int kind, cudaStream_t stream)
     a.out = static_cast<uint8_t *>(out);
     a.nchunks = N;
     a.kind = kind;
-    a.rec_bytes = kind_bytes(kind);
+    a.base_bytes = kind_bytes(kind);
+    a.pair = pair;
+    a.rec_bytes = a.base_bytes + (pair ? pair_extra(kind) : 0u);
     dim3 grid(N, p.Hk, p.B);
     kern<<<grid, NT, Ly.total, stream>>>(mq, mk, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;

@@ -115,6 +115,8 @@ struct SplitArgs {
     float *seg_end;           // [B][Hv][nseg][KD][dv]: Btil of each segment
     float *seg_trans;         // [B][Hk][nseg][KD][KD]: Atil of each segment
     float *seg_start;         // [B][Hv][nseg][KD][dv]: the state each segment starts from
+    int pair;                 // chunks of 128 run as pairs of 64-token halves (Neumann inverse)
+    uint32_t pair_y;          // byte offset of the pair correction Y in a record
 };
 
 // Segment count for the state pass of a request: cost model in chunk periods, one
@@ -131,6 +133,7 @@ struct SegPlan {
 inline SegPlan seg_plan(const Params &p)
 {
     const int N = prep::nchunks(p);
+    const int even = p.pair ? 2 : 1;   // pairs never straddle a segment boundary
     const long nvh = (long)(p.dv / NVC) * p.Hv * p.B;
     const long ntr = (long)(KD / NVC) * p.Hk * p.B;
     auto waves = [](long ctas) { return (ctas + kSMs - 1) / kSMs; };
@@ -138,7 +141,7 @@ inline SegPlan seg_plan(const Params &p)
     SegPlan best{1, N};
     long best_cost = seq_cost;
     for (int ns = 2; ns <= N / kMinSegChunks; ++ns) {
-        const int L = (N + ns - 1) / ns;
+        const int L = ((N + ns - 1) / ns + even - 1) / even * even;
         const int nsg = (N + L - 1) / L;
         const long cost = (waves((nvh + ntr) * nsg) + waves(nvh * nsg)) * (long)L + nsg;
         if (cost < best_cost) {
@@ -329,9 +332,14 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 if (__any_sync(0xffffffffu, !ok))
                     break;
             }
+            // pairs: the first half's Y goes under its L ([L; Y]); stage 0 holds first
+            // halves, since every segment starts at an even chunk
+            const bool with_y = args.pair && s == 0;
             if (lane == 0) {
                 uint64_t *full = &bars[FULLY0 + s];
-                mbar_arrive_expect_tx(full, (outputs ? 3u : 2u) * prep::IMG);
+                mbar_arrive_expect_tx(full, (outputs ? 3u : 2u) * prep::IMG + (with_y ? prep::IMG : 0u));
+                if (with_y)
+                    bulk_load(base + Ly.lz[s] + 64 * 128, fac + args.pair_y, prep::IMG, full);
                 for (int kb = 0; kb < KD / 64; ++kb) {
                     uint8_t *blk = qwk + kb * 192 * 128 + 128 * 128;
                     if (scalar)
@@ -519,12 +527,26 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     tmem_ld16(tq + T_U + 64 * s + cs, u0);
                     tmem_ld16(tq + T_U + 64 * s + cs + 16, u1);
                 }
+                // second half of a pair: + Y E1, left by the first half's [L; Y] E product in
+                // rows 64-127 of its LE buffer (complete: it was issued before this P)
+                const bool corr = args.pair && (i & 1);
+                float y0[16], y1[16];
+                if (corr) {
+                    tmem_ld16(tq + T_LE + cs, y0);
+                    tmem_ld16(tq + T_LE + cs + 16, y1);
+                }
                 tmem_ld_wait();
 #pragma unroll
                 for (int n = 0; n < 16; ++n) {
                     u0[n] -= p0[n];
                     u1[n] -= p1[n];
                 }
+                if (corr)
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) {
+                        u0[n] += y0[n];
+                        u1[n] += y1[n];
+                    }
                 st_tile8(E_T, CC, t, cs, &u0[0]);
                 st_tile8(E_T, CC, t, cs + 8, &u0[8]);
                 st_tile8(E_T, CC, t, cs + 16, &u1[0]);
@@ -720,6 +742,8 @@ int launch(const Params &p, const void *factors, cudaStream_t stream)
     a.nseg = sp.nseg;
     a.seg_len = sp.seg_len;
     a.seg_end = a.seg_trans = a.seg_start = nullptr;
+    a.pair = p.pair;
+    a.pair_y = prep::kind_bytes(prep::record_kind(p)) + prep::PAIR_Y;
     if (sp.nseg == 1) {
         a.mode = MODE_SEQ;
         kern<<<dim3(a.nvt * p.Hv, p.B, 1), NTHR, Ly.total, stream>>>(mq, mk, mv, a);

@@ -214,7 +214,10 @@ gdr_status gdr_chunk_fwd_momentum(const gdr_shape *shape,
  * kernel AUTO or shape->kernel selects when given enough: 0 for the one-pass
  * kernels; for TC2, B * Hk * ceil(T / 64) records of 33296 bytes (scalar gate)
  * or 66048 bytes (grouped / per-channel gates): the chunk factors T and L plus
- * the decayed operands and decay factors the second pass reads.  When the
+ * the decayed operands and decay factors the second pass reads.  The truncated
+ * Neumann inverse at chunk 128 runs as pairs of 64-token halves, and its records
+ * carry the pair correction and its inputs: 16384 more bytes (scalar gate) or
+ * 32768 more (grouped / per-channel gates).  When the
  * sequences are few and long enough that the state pass runs segment-parallel
  * (each sequence cut into segments whose state maps are composed), three
  * fp32 states per segment and head (end state, start state: dk x dv per value

@@ -158,6 +158,20 @@ def test_kernel_chunk(lib):
     assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL) == 64
     assert gdr.kernel_chunk(kda, 64, gdr.GATE_CHANNEL) == 64
     assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL, "neumann") == 128
+    # ... which the two-pass path runs as pairs of 64-token halves (records with the
+    # pair extras: Y, Ntil and, for per-channel gates, Kbar); the one-pass kernels
+    # have no pair correction
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann") == gdr.KERNEL_TC2
+    many = gdr.make_shape(4, 4096, 16, 16, 128, 128)
+    for gate, rec in ((gdr.GATE_CHANNEL, gdr.TC2_EXT_RECORD_BYTES + 4 * 8192),
+                      (gdr.GATE_SCALAR, gdr.TC2_SCALAR_RECORD_BYTES + 2 * 8192)):
+        assert gdr.state_segments(many, 128, gate, "neumann") == 1
+        assert gdr.workspace_bytes(many, 128, gate, "neumann") == 4 * 16 * 64 * rec
+    assert gdr.select_kernel(gdr.make_shape(1, 4096, 1, 1, 128, 128, kernel="tc"), 128,
+                             gdr.GATE_CHANNEL, "neumann") == -gdr.ERR_UNSUPPORTED
+    # segments of the segment-parallel state pass start on pair boundaries
+    long = gdr.make_shape(1, 65536, 16, 16, 128, 128)
+    assert gdr.state_segments(long, 128, gdr.GATE_CHANNEL, "neumann") >= 2
     simt = gdr.make_shape(1, 256, 2, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
     assert gdr.kernel_chunk(simt, 128, gdr.GATE_SCALAR) == 128
     assert gdr.kernel_chunk(simt, 32, gdr.GATE_SCALAR) == 32

@@ -70,6 +70,17 @@ SMALL = [
     (4, dict(Hk=1, Hv=1, T=384), 64, "neumann1", "tc2"),                # pivoted blocks
     (0, {}, 128, "neumann1", "auto"),                                   # fp32
     (4, dict(Hk=1, Hv=1, T=300), 128, "neumann1", "auto"),
+    # truncated Neumann at chunk 128 on the two-pass path: pairs of 64-token halves
+    # with the pair correction; an odd number of halves (no second half in the last
+    # pair), a partial second half, weak and strong per-channel decay, grouped and
+    # scalar gates, grouped value heads
+    (4, dict(Hk=2, Hv=2, T=640), 128, "neumann", "tc2"),
+    (4, dict(Hk=1, Hv=1, T=704 - 37), 128, "neumann", "tc2"),
+    (4, dict(Hk=1, Hv=1, T=600), 128, "neumann", "tc2"),
+    (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 128, "neumann", "tc2"),
+    (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 128, "neumann", "tc2"),
+    (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 128, "neumann", "tc2"),
+    (1, dict(B=2, Hk=1, Hv=3, T=256, dv=192), 128, "neumann", "tc2"),
 ]
 
 
@@ -184,3 +195,31 @@ def test_short_chunk_neumann_parity(idx, over, chunk, inverse):
     eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
     print("rel err o %.3e  S_final %.3e" % (eo, es))
     assert eo <= U.TOL_F32 and es <= U.TOL_F32
+
+
+# The pair correction at other Neumann orders and residual steps (order 0 with one
+# Newton step; order 2 without; order 3 with two), and on a long single sequence
+# whose state pass runs segment-parallel (segments start on pair boundaries).
+PAIR_ORDERS = [(0, 1), (2, 0), (3, 2)]
+
+
+@pytest.mark.parametrize("order,resid", PAIR_ORDERS, ids=["m%d-r%d" % c for c in PAIR_ORDERS])
+def test_pair_neumann_orders(order, resid):
+    w, x = W.workload_inputs(2, B=1, Hk=1, Hv=1, T=384 - 5)
+    o, Sf = U.run_gpu(x, w.in_dtype, 128, "neumann", order=order, resid=resid, kernel="tc2")
+    o_ref, S_ref = U.oracle_reference(x, 128, "neumann", order=order, resid=resid)
+    eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
+    print("rel err o %.3e  S_final %.3e" % (eo, es))
+    assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
+
+
+def test_pair_neumann_segmented():
+    from gated_delta_rule_141_b200 import gdr
+    w, x = W.workload_inputs(4, Hk=1, Hv=1, T=64 * 60 + 17)
+    shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv)
+    assert gdr.state_segments(shape, 128, gdr.GATE_CHANNEL, "neumann") > 1
+    o, Sf = U.run_gpu(x, w.in_dtype, 128, "neumann", kernel="tc2")
+    o_ref, S_ref = U.oracle_reference(x, 128, "neumann")
+    eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
+    print("rel err o %.3e  S_final %.3e" % (eo, es))
+    assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
