@@ -623,15 +623,15 @@ __global__ void __launch_bounds__(32, 1) wait_probe_kernel(uint64_t limit_ns)
 // In exact mode the chunkwise form reaches the token recurrence exactly for any
 // chunk length (the WY equivalence of the SLA paper, §2.4.2), so a request for
 // C = 128 runs on the C = 64 kernels: the same function, blocked more finely.
-// The truncated Neumann inverse depends on C: at C = 128 the two-pass path runs
-// it as pairs of 64-token halves with the pair correction (gdr_tc_pair.cuh),
-// which the one-pass kernels do not have.
+// The truncated and 1-Step Neumann inverses depend on C: at C = 128 the two-pass
+// path runs them as pairs of 64-token halves with the pair correction
+// (gdr_tc_pair.cuh), which the one-pass kernels do not have.
 static Params as_kernel_chunk(const Params &p)
 {
     Params q = p;
-    if (!p.neumann1 && p.C == 128) {
+    if (p.C == 128) {
         q.C = CH;
-        q.pair = p.neumann;
+        q.pair = p.neumann || p.neumann1;
     }
     return q;
 }

@@ -32,6 +32,8 @@
 //      (X <- X + X (I - X - Ntil X)), all products M = N = K = 128 on tcgen05,
 //      X kept in fp32 in tensor memory and as a bf16 operand in shared memory;
 //   4. Atil11^{-1} exactly in fp32 (block doubling), Y in fp32 on the CUDA cores;
+//      (the 1-Step Neumann inverse of §2.4.3 instead of 3: Atil from the diagonal
+//      16 x 16 blocks in fp32, with the same correction;)
 //   5. Y as a bf16 image into the first half's record.
 // The state pass loads Y under L ([L; Y] tile), so its [L; Y] E product of the
 // first half leaves Y E1 in the tensor-memory rows it reads for the second.
@@ -319,47 +321,101 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
     float *A11f = N21f + CC * LDM;
     float *A21f = A11f + CC * LDM;
     float *A22f = f32(base, Ly.NTL);                     // once Ntil21 is copied out
-    if (!failed) {
-        tc_fence_after();
-        // Atil from tensor memory: rows 0-63 x columns 0-63 (strict lower part, as I + H
-        // for the inverse), rows 64-127 x columns 0-63 (Atil21)
-        if (ch == 0) {
-            for (int c = 0; c < 64; c += 16) {
+    if (!p.neumann1) {
+        if (!failed) {
+            tc_fence_after();
+            // Atil from tensor memory: rows 0-63 x columns 0-63 (strict lower part, as I + H
+            // for the inverse), rows 64-127 x columns 0-63 (Atil21)
+            if (ch == 0) {
+                for (int c = 0; c < 64; c += 16) {
+                    float x[16];
+                    tmem_ld16(tq + T_X + c, x);
+                    tmem_ld_wait();
+                    if (R < 64) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            A11f[R * LDM + c + e] = (R > c + e) ? x[e] : 0.f;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            A21f[(R - 64) * LDM + c + e] = x[e];
+                    }
+                }
+            }
+            for (int u = tid; u < CC * 8; u += NT) {          // Ntil21 as the bf16 the series used
+                const int t = u >> 3, j0 = (u & 7) * 8;
+                float v8[8];
+                ld_tile8(NTL, 128, 64 + t, j0, v8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    N21f[t * LDM + j0 + e] = v8[e];
+            }
+        }
+        __syncthreads();
+        if (!failed && ch == 64 && R >= 64) {                 // Atil22: rows and columns 64-127
+            for (int c = 64; c < 128; c += 16) {
                 float x[16];
                 tmem_ld16(tq + T_X + c, x);
                 tmem_ld_wait();
-                if (R < 64) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        A11f[R * LDM + c + e] = (R > c + e) ? x[e] : 0.f;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        A21f[(R - 64) * LDM + c + e] = x[e];
-                }
+                for (int e = 0; e < 16; ++e)
+                    A22f[(R - 64) * LDM + c - 64 + e] = x[e];
             }
         }
-        for (int u = tid; u < CC * 8; u += NT) {          // Ntil21 as the bf16 the series used
+        __syncthreads();
+    } else if (!failed) {
+        // 1-Step Neumann ("Systolic Linear Attention ...", §2.4.3), in fp32 from the bf16
+        // blocks: Atil = Dtil^{-1} - Dtil^{-1} Ntil_off Dtil^{-1}, Dtil the diagonal 16 x 16
+        // blocks of I + Ntil; per half that is the first pass's 64-token factor, and across
+        // the halves Atil21 = -bd(Atil22) Ntil21 bd(Atil11) (bd: the diagonal blocks)
+        for (int u = tid; u < CC * 8; u += NT) {
             const int t = u >> 3, j0 = (u & 7) * 8;
-            float v8[8];
-            ld_tile8(NTL, 128, 64 + t, j0, v8);
+            float a8[8], n8[8];
+            ld_tile8(NTL, 128, t, j0, a8);
+            ld_tile8(NTL, 128, 64 + t, j0, n8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                A11f[t * LDM + j0 + e] = (t > j0 + e) ? a8[e] : 0.f;
+                N21f[t * LDM + j0 + e] = n8[e];
+            }
+        }
+        __syncthreads();
+        for (int u = tid; u < CC * 8; u += NT) {   // Ntil22 lies past the bytes of A22f
+            const int t = u >> 3, j0 = (u & 7) * 8;
+            float a8[8];
+            ld_tile8(NTL, 128, 64 + t, 64 + j0, a8);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                N21f[t * LDM + j0 + e] = v8[e];
+                A22f[t * LDM + j0 + e] = (t > j0 + e) ? a8[e] : 0.f;
         }
-    }
-    __syncthreads();
-    if (!failed && ch == 64 && R >= 64) {                 // Atil22: rows and columns 64-127
-        for (int c = 64; c < 128; c += 16) {
-            float x[16];
-            tmem_ld16(tq + T_X + c, x);
-            tmem_ld_wait();
+        __syncthreads();
+        gen::block_neumann1_64_inplace(A11f, Tf, tid);
+        gen::block_neumann1_64_inplace(A22f, Tf, tid);
+        const int rg = tid >> 4, c0 = 4 * (tid & 15), lb = c0 & ~15, lr = 16 * (rg >> 2);
+        float acc[4][4];
+        // Z = Ntil21 bd(Atil11): rows rg + 16 i, columns c0..c0+3 (one 16-column block)
+        gen::block_product4x4<16>(acc, N21f + rg * LDM + lb, 16 * LDM, A11f + lb * LDM + c0, LDM, 0);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                A22f[(R - 64) * LDM + c - 64 + e] = x[e];
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+                A21f[(rg + 16 * i) * LDM + c0 + n] = acc[i][n];
+        __syncthreads();
+        // Atil21 = -bd(Atil22) Z: rows 4 rg .. 4 rg + 3 (one 16-row block)
+        gen::block_product4x4<16>(acc, A22f + (4 * rg) * LDM + lr, LDM, A21f + lr * LDM + c0, LDM, 0);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+                A21f[(4 * rg + i) * LDM + c0 + n] = -acc[i][n];
+        for (int u = tid; u < CC * CC; u += NT) {   // Atil11 as I + H for the exact inverse
+            const int t = u / CC, j = u % CC;
+            if (t <= j)
+                A11f[t * LDM + j] = 0.f;
         }
+        __syncthreads();
     }
-    __syncthreads();
     if (!failed) {
         gen::inverse64_inplace(A11f, Tf, tid);            // Atil11^{-1}, lower triangular
         const int rg = tid >> 4, c0 = 4 * (tid & 15);     // rows rg + 16 i, columns c0..c0+3

@@ -12,9 +12,12 @@
 //   3. Decayed Grams on tcgen05, never dividing by a decay prefix:
 //        scalar gate: [Q; K] K^T once, then the factor e^{Lambda_t - Lambda_j}
 //          (t >= j, so <= 1) on the way out of TMEM;
-//        grouped / per-channel gate: when the chunk's decay span is within kGuard
-//          nats, one pivot at the chunk end (rows scaled by e^{Lambda_t - Lambda_C},
-//          columns by e^{Lambda_C - Lambda_j}); otherwise two row blocks of 32 tokens, each with
+//        grouped / per-channel gate: when each half of the chunk spans at most
+//          kGuard nats of decay, one pivot p = 32 in the middle of the chunk (rows
+//          scaled by e^{Lambda_t - Lambda_p}, columns by e^{Lambda_p - Lambda_j}, each
+//          at most e^{kGuard}, from two exponentials per element: every decayed
+//          operand of the record is these times a per-channel constant); otherwise
+//          two row blocks of 32 tokens, each with
 //          its own pivot p in the middle of the block.  Rows t of the block
 //          carry e^{Lambda_t - Lambda_p}, columns j carry e^{Lambda_p - Lambda_j};
 //          both factors are at most e^{(half-block decay span)}, and their
@@ -66,7 +69,7 @@ __host__ __device__ constexpr uint32_t pair_extra(int kind) { return kind == REC
 __host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
 
 struct Plan {
-    uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, TB, lam, beta, bar, misc, total, tmem_cols, tn;
+    uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, TB, lam, beta, piv, bar, misc, total, tmem_cols, tn;
 };
 
 __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
@@ -100,6 +103,7 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
     }
     s.lam = take(CC * G * 4 + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
     s.beta = s.lam + CC * G * 4;
+    s.piv = G > 1 ? take(2 * dk * 4) : 0;   // per channel: e^{Lambda_p}, e^{Lambda_C - Lambda_p}
     s.bar = (s.beta + CC * 4 + NROUND * 4 + 7u) & ~7u;
     s.misc = s.bar + 24;
     s.total = o + 1024;
@@ -268,13 +272,26 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
     }
-    // decay span of the chunk per group: within kGuard nats a single pivot at the
-    // chunk end serves every pair; wider spans take the four pivoted row blocks
+    // decay span of each half of the chunk per group: within kGuard nats a single
+    // pivot in the middle of the chunk serves every pair; wider spans take the two
+    // pivoted row blocks
+    constexpr int PV = CC / 2;
+    float *piv = reinterpret_cast<float *>(base + Ly.piv);   // e^{Lambda_p}, e^{Lambda_C - Lambda_p}
     bool wide = false;
     if (!SCALAR)
-        for (int gi = tid; gi < G; gi += NT)
-            wide |= (lam[gi] - lam[(CC - 1) * G + gi]) > kGuard;
+        for (int gi = tid; gi < G; gi += NT) {
+            const float l0 = lam[gi], lp = lam[PV * G + gi], lc = lam[(CC - 1) * G + gi];
+            wide |= (l0 - lp) > kGuard || (lp - lc) > kGuard;
+        }
     wide = __syncthreads_or(wide ? 1 : 0) != 0;
+    if (!SCALAR && !wide) {
+        for (int i = tid; i < DK; i += NT) {
+            const float lp = lam[PV * G + (i >> wsh)], lc = lam[(CC - 1) * G + (i >> wsh)];
+            piv[i] = __expf(lp);
+            piv[DK + i] = __expf(lc - lp);
+        }
+        __syncthreads();
+    }
     failed = wait_bar(0, 0) || failed;
 
     const bool ext = a.kind == REC_EXT;
@@ -330,27 +347,30 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     if (!failed && !wide) {
         if (!SCALAR) {
-            // ---- one pivot at the chunk end: rows carry e^{Lambda_t - Lambda_C} (at most
-            //      e^{kGuard}), columns Khat = k e^{Lambda_C - Lambda_j} (at most 1); the
-            //      state pass's decayed operands come out of the same sweep
+            // ---- one pivot p in the middle of the chunk: rows carry a_t = e^{Lambda_t - Lambda_p},
+            //      columns b_j = e^{Lambda_p - Lambda_j} (each at most e^{kGuard}); the state
+            //      pass's operands from the same two exponentials, Qbar = q a e^{Lambda_p} and
+            //      Khat = k b e^{Lambda_C - Lambda_p}; the k rows keep k a (Kbar = k a e^{Lambda_p}
+            //      is W's operand, its per-channel factor applied on the way out of TMEM)
             for (int u = tid; u < CC * (DK / 8); u += NT) {
                 const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float qv[8], kv[8], kh8[8], qb[8], lt[8], lc[8];
+                float qv[8], kv[8], kc[8], kh8[8], qb[8], lt[8], lp[8];
                 ld_tile8(QK, 128, t, i0, qv);
                 ld_tile8(QK, 128, 64 + t, i0, kv);
                 lam8(lam, G, wsh, t, i0, lt);
-                lam8(lam, G, wsh, CC - 1, i0, lc);
+                lam8(lam, G, wsh, PV, i0, lp);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float up = __expf(lt[e] - lc[e]), dn = __expf(lc[e] - lt[e]);
-                    qb[e] = qv[e] * __expf(lt[e]);
-                    kh8[e] = kv[e] * dn;
-                    qv[e] *= up;
-                    kv[e] *= up;
+                    const float a = __expf(lt[e] - lp[e]), b = __expf(lp[e] - lt[e]);
+                    qv[e] *= a;
+                    kc[e] = kv[e] * b;
+                    kv[e] *= a;
+                    qb[e] = qv[e] * piv[i0 + e];
+                    kh8[e] = kc[e] * piv[DK + i0 + e];
                 }
                 st_tile8(QK, 128, t, i0, qv);
                 st_tile8(QK, 128, 64 + t, i0, kv);
-                st_tile8(KC, 64, t, i0, kh8);
+                st_tile8(KC, 64, t, i0, kc);
                 if (ext) {
                     const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
                     *reinterpret_cast<uint4 *>(img_T + EXT_QB + off) =
@@ -714,13 +734,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 st_tile8(QK, 128, 64 + t, i0, kv);
             }
         }
-        // After the chunk-end pivot the k rows hold k e^{Lambda_t - Lambda_C}: W is then
-        // (T that) diag(e^{Lambda_C}), the column factors applied on the way out of TMEM
-        // (held in the inverse's scratch, free by now).
+        // After the middle pivot the k rows hold k e^{Lambda_t - Lambda_p}: W is then
+        // (T that) diag(e^{Lambda_p}), the column factors applied on the way out of TMEM
+        // (copied into the inverse's scratch, free by now).
         const bool w_cols = with_w && !SCALAR && !wide;
         if (w_cols)
             for (int i = tid; i < DK; i += NT)
-                Tf[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);
+                Tf[i] = piv[i];
         if (a.pair && !SCALAR) {
             // Kbar = k e^{Lambda_t} for the pair kernel: the k rows hold it after the
             // pivoted blocks; after the chunk-end pivot they hold k e^{Lambda_t - Lambda_C}
@@ -730,7 +750,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
                 float kv[8];
                 ld_tile8(QK, 128, 64 + t, i0, kv);
-                if (w_cols)   // Tf holds e^{Lambda_C} per channel here
+                if (w_cols)   // Tf holds e^{Lambda_p} per channel here
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         kv[e] *= Tf[i0 + e];

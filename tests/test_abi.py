@@ -181,12 +181,13 @@ def test_kernel_chunk(lib):
 
 def test_neumann1_selection(lib):
     # 1-Step Neumann depends on the chunk length (blocks of 16 in a chunk), so it is
-    # never re-blocked: chunk 64 runs the two-pass path, chunk 128 the CUDA-core
-    # kernel; the fused one-pass kernels do not implement it.
+    # never re-blocked: chunk 64 runs the two-pass path, chunk 128 the two-pass path
+    # as pairs of 64-token halves with the pair correction (the function of the
+    # 128-token chunk); the fused one-pass kernels do not implement it.
     kda = gdr.make_shape(2, 8192, 32, 32, 128, 128)
     assert gdr.select_kernel(kda, 64, gdr.GATE_CHANNEL, "neumann1") == gdr.KERNEL_TC2
     assert gdr.kernel_chunk(kda, 64, gdr.GATE_CHANNEL, "neumann1") == 64
-    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann1") == gdr.KERNEL_SIMT
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann1") == gdr.KERNEL_TC2
     assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL, "neumann1") == 128
     forced = gdr.make_shape(1, 256, 2, 2, 128, 128, kernel="tc")
     assert gdr.select_kernel(forced, 64, gdr.GATE_SCALAR, "neumann1") == -gdr.ERR_UNSUPPORTED

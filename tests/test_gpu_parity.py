@@ -81,6 +81,10 @@ SMALL = [
     (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 128, "neumann", "tc2"),
     (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 128, "neumann", "tc2"),
     (1, dict(B=2, Hk=1, Hv=3, T=256, dv=192), 128, "neumann", "tc2"),
+    # 1-Step Neumann at chunk 128 (eight blocks of 16, as in the pages) the same way
+    (4, dict(Hk=2, Hv=2, T=640 - 27), 128, "neumann1", "tc2"),
+    (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 128, "neumann1", "tc2"),
+    (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 128, "neumann1", "tc2"),
 ]
 
 

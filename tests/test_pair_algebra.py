@@ -21,6 +21,18 @@ def neumann(N, order, resid):
     return X
 
 
+def one_step_neumann(M, blk):
+    """1-Step Neumann approximation of (I + M)^{-1}: with D the block-diagonal part
+    of I + M in blocks of `blk` rows, D^{-1} - D^{-1} M_off D^{-1}."""
+    n = M.shape[0]
+    D = np.eye(n)
+    for b0 in range(0, n, blk):
+        s = slice(b0, min(n, b0 + blk))
+        D[s, s] += M[s, s]
+    Dinv = np.linalg.inv(D)
+    return Dinv - Dinv @ (M - (D - np.eye(n))) @ Dinv
+
+
 def chunk_step(q, k, v, lam, beta, S, A_of):
     """One chunk of the chunkwise form: decays relative to the chunk start
     (lam[t] = Lambda_t per channel, lam[-1] the chunk end), T = diag(beta) A(M)."""
@@ -45,8 +57,11 @@ def chunk_step(q, k, v, lam, beta, S, A_of):
 
 
 @pytest.mark.parametrize("h,order,resid,seed", [(8, 4, 1, 0), (8, 2, 0, 1), (6, 3, 2, 2),
-                                                (16, 4, 1, 3), (5, 0, 1, 4)])
+                                                (16, 4, 1, 3), (5, 0, 1, 4), (8, -1, 4, 5),
+                                                (12, -1, 4, 6)])
 def test_pair_correction_reproduces_the_whole_chunk(h, order, resid, seed):
+    """order >= 0: truncated Neumann of that order with `resid` Newton steps;
+    order -1: 1-Step Neumann in blocks of `resid` rows (blocks inside each half)."""
     rng = np.random.default_rng(seed)
     dk, dv, C = 6, 5, 2 * h
     q = rng.standard_normal((C, dk))
@@ -56,7 +71,8 @@ def test_pair_correction_reproduces_the_whole_chunk(h, order, resid, seed):
     g = -np.log1p(np.exp(rng.standard_normal((C, dk))))      # -softplus, per channel
     beta = 1 / (1 + np.exp(-rng.standard_normal(C)))
     S = 0.3 * rng.standard_normal((dk, dv))
-    A_of = lambda M: neumann(M, order, resid)
+    A_of = ((lambda M: neumann(M, order, resid)) if order >= 0
+            else (lambda M: one_step_neumann(M, resid)))
     lam = np.cumsum(g, axis=0)
     O_ref, S_ref, _, G = chunk_step(q, k, v, lam, beta, S, A_of)
 
@@ -86,7 +102,7 @@ def test_pair_correction_reproduces_the_whole_chunk(h, order, resid, seed):
     assert np.abs(O - O_ref).max() <= 1e-10 * np.abs(O_ref).max()
     assert np.abs(S_end - S_ref).max() <= 1e-10 * np.abs(S_ref).max()
     # and the correction is not trivially zero when the series is truncated
-    if order < C - 1 and resid == 0:
+    if 0 <= order < C - 1 and resid == 0:
         assert np.abs(Y @ E1).max() > 1e-8
 
 
