@@ -566,7 +566,7 @@ def main():
     # the two-pass path: pass 1, then one state pass, or three when segmented
     nseg = gdr.state_segments(shape_run, chunk, gm_run, args.inverse) if kern == gdr.KERNEL_TC2 else 0
     # Neumann at chunk 128 on the two-pass path adds the pair kernel after pass 1
-    pair = kern == gdr.KERNEL_TC2 and args.inverse == "neumann" and chunk == 128
+    pair = kern == gdr.KERNEL_TC2 and args.inverse in ("neumann", "neumann1") and chunk == 128
     launches_per_step = ((1 + (1 if nseg == 1 else 3) + (1 if pair else 0)) if kern == gdr.KERNEL_TC2
                          else 2 if kern == gdr.KERNEL_SIMT2 else 1)
     zgate = None

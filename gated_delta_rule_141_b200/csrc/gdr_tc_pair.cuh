@@ -129,7 +129,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         if (a.ext) {
             // Khat1 (the first half's record) and Kbar2 (the second half's pair extra),
             // 64-row tiles of DK / 64 column blocks, as the records store them
-            bulk_load(base + Ly.RT, rec1 + prep::EXT_KH, opnd, full);
+            bulk_load(base + Ly.RT, rec1 + prep::ext_kh(DK), opnd, full);
             bulk_load(base + Ly.RT + opnd, rec2 + a.base_bytes + prep::PAIR_KB, opnd, full);
         } else {
             for (int kb = 0; kb < DK / 64; ++kb) {
@@ -467,7 +467,7 @@ int launch(const Params &p, void *records, cudaStream_t stream)
     a.rec = static_cast<uint8_t *>(records);
     a.nchunks = N;
     a.rec_bytes = prep::rec_bytes(p);
-    a.base_bytes = prep::kind_bytes(prep::record_kind(p));
+    a.base_bytes = prep::kind_bytes(prep::record_kind(p), DK);
     a.ext = prep::record_kind(p) == prep::REC_EXT;
     pair_kernel<DK><<<dim3(npairs(N), p.Hk, p.B), NT, Ly.total, stream>>>(mk, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;

@@ -52,19 +52,26 @@ constexpr uint32_t CHUNK_BYTES = 2 * IMG;  // T, then L
 constexpr uint32_t REC_W = 2 * IMG;
 constexpr uint32_t SC_EA = 4 * IMG, SC_EB = SC_EA + CC * 4, SC_F = SC_EB + CC * 4;
 constexpr uint32_t SC_BYTES = SC_F + 16;
-// grouped / per-channel gates: then Qbar, Khat (64 x 128 bf16 each) and F (128 fp32)
-constexpr uint32_t EXT_QB = 4 * IMG, EXT_KH = EXT_QB + 2 * IMG;
-constexpr uint32_t EXT_F = EXT_KH + 2 * IMG;
-constexpr uint32_t EXT_BYTES = EXT_F + 128 * 4;
+// grouped / per-channel gates: then Qbar, Khat (64 x dk bf16 each, dk / 64 images)
+// and F (dk fp32); offsets for key width dk:
+__host__ __device__ constexpr uint32_t ext_qb(int dk) { return (2u + dk / 64) * IMG; }
+__host__ __device__ constexpr uint32_t ext_kh(int dk) { return (2u + 2 * (dk / 64)) * IMG; }
+__host__ __device__ constexpr uint32_t ext_f(int dk) { return (2u + 3 * (dk / 64)) * IMG; }
+__host__ __device__ constexpr uint32_t ext_bytes(int dk) { return ext_f(dk) + dk * 4; }
+constexpr uint32_t EXT_QB = ext_qb(128), EXT_KH = ext_kh(128), EXT_F = ext_f(128);
+constexpr uint32_t EXT_BYTES = ext_bytes(128);
 enum RecordKind { REC_PLAIN = 0, REC_SCALAR = 1, REC_EXT = 2 };
 // Pair records (the truncated Neumann inverse at C = 128 run as two 64-token
 // halves): the base record, then Y (the pair's correction, written by
 // pair_kernel into the record of the pair's first half), Ntil = diag(beta) x the
 // decayed Gram of the half (beta on the rows: strictly lower, bf16 image) and,
-// for grouped / per-channel gates, Kbar = k e^{Lambda_t} (64 x 128 bf16, two
+// for grouped / per-channel gates, Kbar = k e^{Lambda_t} (64 x dk bf16, dk / 64
 // images).
 constexpr uint32_t PAIR_Y = 0, PAIR_N = IMG, PAIR_KB = 2 * IMG;   // offsets past the base record
-__host__ __device__ constexpr uint32_t pair_extra(int kind) { return kind == REC_EXT ? 4 * IMG : 2 * IMG; }
+__host__ __device__ constexpr uint32_t pair_extra(int kind, int dk = 128)
+{
+    return kind == REC_EXT ? (2u + dk / 64) * IMG : 2 * IMG;
+}
 
 __host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
 
@@ -107,7 +114,7 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
     s.bar = (s.beta + CC * 4 + NROUND * 4 + 7u) & ~7u;
     s.misc = s.bar + 24;
     s.total = o + 1024;
-    s.tmem_cols = G > 1 ? 256u : 128u;            // W (M = 64, N = 128) needs 128 columns
+    s.tmem_cols = (G > 1 || dk > 128) ? 256u : 128u;   // W (M = 64, N = dk) needs dk columns
     s.tn = G > 1 ? 192u : 64u;                    // Neumann products
     return s;
 }
@@ -296,7 +303,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     const bool ext = a.kind == REC_EXT;
     if (!failed && ext) {
-        float *fo = reinterpret_cast<float *>(img_T + EXT_F);
+        float *fo = reinterpret_cast<float *>(img_T + ext_f(DK));
         for (int i = tid; i < DK; i += NT)
             fo[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);   // F = e^{Lambda_C}
     }
@@ -336,10 +343,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 kh8[e] = kv[e] * __expf(lc[e] - lt[e]);
             }
             const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
-            *reinterpret_cast<uint4 *>(img_T + EXT_QB + off) =
+            *reinterpret_cast<uint4 *>(img_T + ext_qb(DK) + off) =
                 make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]), pack_bf16(qb[4], qb[5]),
                            pack_bf16(qb[6], qb[7]));
-            *reinterpret_cast<uint4 *>(img_T + EXT_KH + off) =
+            *reinterpret_cast<uint4 *>(img_T + ext_kh(DK) + off) =
                 make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
                            pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
         }
@@ -373,10 +380,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 st_tile8(KC, 64, t, i0, kc);
                 if (ext) {
                     const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(img_T + EXT_QB + off) =
+                    *reinterpret_cast<uint4 *>(img_T + ext_qb(DK) + off) =
                         make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]),
                                    pack_bf16(qb[4], qb[5]), pack_bf16(qb[6], qb[7]));
-                    *reinterpret_cast<uint4 *>(img_T + EXT_KH + off) =
+                    *reinterpret_cast<uint4 *>(img_T + ext_kh(DK) + off) =
                         make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
                                    pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
                 }
@@ -790,12 +797,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
         if (with_w) {
-            // ---- W = TB Kbar (M = 64, N = 128, K = 64) on tcgen05, read back as an image
+            // ---- W = TB Kbar (M = 64, N = dk, K = 64) on tcgen05, read back as an image
             fence_proxy_async_smem();
             __syncthreads();
             if (tid == 0) {
                 tc_fence_after();
-                const uint32_t id = idesc_bf16(64, 128, false, true);
+                const uint32_t id = idesc_bf16(64, DK, false, true);
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(tmem, desc_kmajor(TB, 64, 0, k0), desc_mnmajor(QK, 128, 64 + k0, 0), id,
                              k0 > 0);
@@ -806,9 +813,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (!failed) {
                 tc_fence_after();
                 const int rr = gen::row64g(warp, lane);
-                const int cw = 64 * (warp >> 2);
+                const int cw = (DK / 2) * (warp >> 2);   // this warp's half of the dk columns
 #pragma unroll
-                for (int cb = 0; cb < 64; cb += 32) {
+                for (int cb = 0; cb < DK / 2; cb += 32) {
                     float w0[16], w1[16];
                     tmem_ld16(tq + cw + cb, w0);
                     tmem_ld16(tq + cw + cb + 16, w1);
@@ -821,11 +828,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                 w1[e] *= Tf[cw + cb + 16 + e];
                             }
                         }
-                        uint8_t *img_W = img_T + REC_W + (cw >> 6) * IMG;
-                        st_img8(img_W, rr, cb, &w0[0]);
-                        st_img8(img_W, rr, cb + 8, &w0[8]);
-                        st_img8(img_W, rr, cb + 16, &w1[0]);
-                        st_img8(img_W, rr, cb + 24, &w1[8]);
+                        const int col = cw + cb;   // 32 columns inside one 64-column image
+                        uint8_t *img_W = img_T + REC_W + (col >> 6) * IMG;
+                        st_img8(img_W, rr, col & 63, &w0[0]);
+                        st_img8(img_W, rr, (col & 63) + 8, &w0[8]);
+                        st_img8(img_W, rr, (col & 63) + 16, &w1[0]);
+                        st_img8(img_W, rr, (col & 63) + 24, &w1[8]);
                     }
                 }
             }
@@ -857,14 +865,14 @@ inline size_t bytes(const Params &p)
 // Record of the two-pass path's workspace.
 inline int record_kind(const Params &p) { return p.G > 1 ? REC_EXT : REC_SCALAR; }
 
-inline uint32_t kind_bytes(int kind)
+inline uint32_t kind_bytes(int kind, int dk = 128)
 {
-    return kind == REC_EXT ? EXT_BYTES : (kind == REC_SCALAR ? SC_BYTES : CHUNK_BYTES);
+    return kind == REC_EXT ? ext_bytes(dk) : (kind == REC_SCALAR ? SC_BYTES : CHUNK_BYTES);
 }
 
 inline uint32_t rec_bytes(const Params &p)
 {
-    return kind_bytes(record_kind(p)) + (p.pair ? pair_extra(record_kind(p)) : 0u);
+    return kind_bytes(record_kind(p), p.dk) + (p.pair ? pair_extra(record_kind(p), p.dk) : 0u);
 }
 
 inline size_t ws_bytes(const Params &p) { return (size_t)p.B * p.Hk * nchunks(p) * rec_bytes(p); }
@@ -895,9 +903,9 @@ int launch(const Params &p, void *out, int kind, cudaStream_t stream, int pair =
     a.out = static_cast<uint8_t *>(out);
     a.nchunks = N;
     a.kind = kind;
-    a.base_bytes = kind_bytes(kind);
+    a.base_bytes = kind_bytes(kind, DK);
     a.pair = pair;
-    a.rec_bytes = a.base_bytes + (pair ? pair_extra(kind) : 0u);
+    a.rec_bytes = a.base_bytes + (pair ? pair_extra(kind, DK) : 0u);
     dim3 grid(N, p.Hk, p.B);
     kern<<<grid, NT, Ly.total, stream>>>(mq, mk, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;

@@ -743,7 +743,7 @@ int launch(const Params &p, const void *factors, cudaStream_t stream)
     a.seg_len = sp.seg_len;
     a.seg_end = a.seg_trans = a.seg_start = nullptr;
     a.pair = p.pair;
-    a.pair_y = prep::kind_bytes(prep::record_kind(p)) + prep::PAIR_Y;
+    a.pair_y = prep::kind_bytes(prep::record_kind(p), p.dk) + prep::PAIR_Y;
     if (sp.nseg == 1) {
         a.mode = MODE_SEQ;
         kern<<<dim3(a.nvt * p.Hv, p.B, 1), NTHR, Ly.total, stream>>>(mq, mk, mv, a);
