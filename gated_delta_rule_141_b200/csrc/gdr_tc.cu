@@ -687,13 +687,24 @@ int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
     const Params p = as_kernel_chunk(p0);
     if (!split::supports(p))
         return 5;
-    int rc = prep::launch<128>(p, workspace, prep::record_kind(p), stream, p.pair);
+    const int kind = prep::record_kind(p);
+    int rc;
+    if (p.dk == 256) {
+        rc = prep::launch<256>(p, workspace, kind, stream, p.pair);
+        if (rc == 0 && p.pair)
+            rc = pair::launch<256>(p, workspace, stream);
+        if (rc != 0)
+            return rc;
+        return p.out_bf16 ? split::launch<256, true>(p, workspace, stream)
+                          : split::launch<256, false>(p, workspace, stream);
+    }
+    rc = prep::launch<128>(p, workspace, kind, stream, p.pair);
     if (rc == 0 && p.pair)
         rc = pair::launch<128>(p, workspace, stream);
     if (rc != 0)
         return rc;
-    return p.out_bf16 ? split::launch<true>(p, workspace, stream)
-                      : split::launch<false>(p, workspace, stream);
+    return p.out_bf16 ? split::launch<128, true>(p, workspace, stream)
+                      : split::launch<128, false>(p, workspace, stream);
 }
 
 int launch_wait_probe(uint64_t limit_ns, cudaStream_t stream)

@@ -50,6 +50,7 @@ struct Plan {
     uint32_t NTL, XT, RT, Tf, beta, bar, misc, total;
 };
 
+template <int DK>
 __host__ __device__ inline Plan plan()
 {
     Plan s;
@@ -61,7 +62,8 @@ __host__ __device__ inline Plan plan()
     };
     s.NTL = take(2 * 128 * 128);        // Ntil, 128 x 128 bf16
     s.XT = take(2 * 128 * 128);         // X, 128 x 128 bf16
-    s.RT = take(2 * 128 * 128);         // Newton residual; first the G21 operands
+    // Newton residual; first the G21 operands (two 64 x dk tiles)
+    s.RT = take(2 * 128 * 128 > 2 * CC * DK * 2 ? 2 * 128 * 128 : 2 * CC * DK * 2);
     s.Tf = take(32 * 36 * 4 + 1024);    // scratch of the fp32 block inverse
     s.beta = take(3 * CC * 4);          // beta2, then (scalar gate) ea2, eb1
     s.bar = take(64);
@@ -89,7 +91,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
     using namespace ptx;
     extern __shared__ uint8_t smem_raw[];
     const Params &p = a.p;
-    const Plan Ly = plan();
+    const Plan Ly = plan<DK>();
     const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *base = smem_raw + (base_u32 - smem_u32(smem_raw));
     const uint32_t NTL = base_u32 + Ly.NTL, XT = base_u32 + Ly.XT, RT = base_u32 + Ly.RT;
@@ -458,7 +460,7 @@ int launch(const Params &p, void *records, cudaStream_t stream)
     CUtensorMap mk;
     if (!make_map(&mk, p.k, DK, p.T, (long)p.B * p.Hk, CC))
         return 6;
-    const Plan Ly = plan();
+    const Plan Ly = plan<DK>();
     if (cudaFuncSetAttribute(pair_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
         cudaSuccess)
         return 6;

@@ -39,7 +39,7 @@ namespace split {
 constexpr int NWARP = 13;
 constexpr int NTHR = NWARP * 32;   // 416
 constexpr int CC = 64;
-constexpr int KD = 128;
+constexpr int KD = 128;             // key width of the segment-parallel form
 constexpr int NVC = 64;
 constexpr int W_EPI0 = 0, W_PROD = 2, W_MMA = 3, W_STATE0 = 4, W_PROD_Y = 12;
 constexpr int N_STATE = 256, N_EPI = 64;
@@ -47,16 +47,18 @@ constexpr int NB_STATE = 1, NB_EPI = 2;   // named barriers
 
 constexpr uint32_t T_U = 0;        // two buffers of 64 cols: [0; T] V (rows 64-127)
 constexpr uint32_t T_PO = 128;     // two buffers of 64 cols: [Q; W] S
-constexpr uint32_t T_S = 256;      // fp32 state, 64 cols
-constexpr uint32_t T_LE = 320;     // two buffers of 64 cols: [L; 0] E (rows 0-63)
+constexpr uint32_t T_S = 256;      // fp32 state, 64 cols per 128 key rows
+// two buffers of 64 cols after the state: [L; 0] E (rows 0-63)
+__host__ __device__ constexpr uint32_t t_le(int dk) { return T_S + dk / 2; }
 constexpr uint32_t TMEM_COLS = 512;
 
 enum Bar { FULLX0, FULLX1, FULLY0, FULLY1, FREEX0, FREEX1, FREEY0, FREEY1, S_READY, P_FULL, E_READY,
            UPD_DONE, OUT0, OUT1, OFREE0, OFREE1, DRAIN, NBARS };
 
+template <int DK>
 struct Gates {                        // landed by bulk copies from the first pass's record
     float ea[CC], eb[CC];             // scalar gate: e^{Lambda_t}, e^{Lambda_C - Lambda_t}
-    float F[KD];                      // e^{Lambda_C} per key channel (F[0] for the scalar gate)
+    float F[DK];                      // e^{Lambda_C} per key channel (F[0] for the scalar gate)
 };
 
 struct Plan {
@@ -64,8 +66,12 @@ struct Plan {
     uint32_t S, E, Eh, bar, misc, total;
 };
 
-// Stage: [Q | W | K] (rows 0-63 | 64-127 | 128-191, 128 columns), [L | 0]
-// (64 + 64 rows), V (64 rows) and [0 | T] (64 + 64 rows), 64 columns each.
+// Stage: [Q | W | K] (rows 0-63 | 64-127 | 128-191, dk columns), [L | 0]
+// (64 + 64 rows), V (64 rows) and [0 | T] (64 + 64 rows), 64 columns each.  At
+// dk = 256 the [Q | W | K] tile (96 KB) has one buffer shared by both stages:
+// the next chunk's W and Q land once P has read this chunk's, its K once the
+// update has (the other parts keep two stages).
+template <int DK>
 __host__ __device__ inline Plan plan(bool scalar)
 {
     Plan s;
@@ -76,13 +82,13 @@ __host__ __device__ inline Plan plan(bool scalar)
         return at;
     };
     for (int i = 0; i < 2; ++i) {
-        s.qwk[i] = take((KD / 64) * 192 * 128);
+        s.qwk[i] = (i == 0 || DK == 128) ? take((DK / 64) * 192 * 128) : s.qwk[0];
         s.lz[i] = take(128 * 128);
         s.v[i] = take(64 * 128);
         s.ab[i] = take(128 * 128);
-        s.gates[i] = take(sizeof(Gates));
+        s.gates[i] = take(sizeof(Gates<DK>));
     }
-    s.S = take(KD * NVC * 2);
+    s.S = take(DK * NVC * 2);
     s.E = take(CC * NVC * 2);
     s.Eh = scalar ? take(CC * NVC * 2) : s.E;
     s.bar = take(NBARS * 8 + 16);
@@ -133,6 +139,8 @@ struct SegPlan {
 inline SegPlan seg_plan(const Params &p)
 {
     const int N = prep::nchunks(p);
+    if (p.dk != KD)   // the segment-parallel form is built for dk = 128
+        return SegPlan{1, N};
     const int even = p.pair ? 2 : 1;   // pairs never straddle a segment boundary
     const long nvh = (long)(p.dv / NVC) * p.Hv * p.B;
     const long ntr = (long)(KD / NVC) * p.Hk * p.B;
@@ -187,7 +195,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
     }
 }
 
-template <bool OUT_BF16>
+template <int DK, bool OUT_BF16>
 __global__ void __launch_bounds__(NTHR, 1)
 split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
@@ -198,7 +206,10 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     const Params &p = args.p;
     const bool scalar = p.G == 1;
-    const Plan Ly = plan(scalar);
+    const Plan Ly = plan<DK>(scalar);
+    constexpr bool ONE = DK > 128;          // one [Q | W | K] buffer (see plan)
+    constexpr int NKB = DK / 64;            // 64-column blocks of a key-side tile
+    constexpr uint32_t T_LE = t_le(DK);
     const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *base = smem_raw + (base_u32 - smem_u32(smem_raw));
 
@@ -207,10 +218,10 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // a transition CTA of the segmented form: identity start, no values, no outputs
     const bool trans = args.mode == MODE_SEG_AB && (int)blockIdx.x >= nvh;
     const int xi = trans ? (int)blockIdx.x - nvh : (int)blockIdx.x;
-    const int nt = trans ? xi % (KD / NVC) : xi % args.nvt;
+    const int nt = trans ? xi % (DK / NVC) : xi % args.nvt;
     const int hv = trans ? 0 : xi / args.nvt;
     const int b = blockIdx.y;
-    const int hk = trans ? xi / (KD / NVC) : hv / p.R;
+    const int hk = trans ? xi / (DK / NVC) : hv / p.R;
     const int n0 = nt * NVC;
     const long kh = (long)b * p.Hk + hk;
     const long vh = (long)b * p.Hv + hv;
@@ -226,7 +237,21 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 4);
-    auto gates_of = [&](int s) { return reinterpret_cast<Gates *>(base + Ly.gates[s]); };
+    auto gates_of = [&](int s) { return reinterpret_cast<Gates<DK> *>(base + Ly.gates[s]); };
+    // Wait before loading chunk i into stage i & 1 until its previous contents are
+    // released (FREEX0 / FREEY0 and the stage's offset): with two buffers, their use by
+    // chunk i - 2; with one [Q | W | K] buffer, the previous chunk's release of the
+    // other stage, which also implies chunk i - 2's (the releases come in chunk order)
+    auto wait_free = [&](int bar0, int i) -> bool {
+        if (ONE) {
+            if (i < 1)
+                return true;
+            return wait_or_abort(&bars[bar0 + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort_flag);
+        }
+        if (i < 2)
+            return true;
+        return wait_or_abort(&bars[bar0 + (i & 1)], ((i >> 1) - 1) & 1, abort_flag);
+    };
     const uint32_t S_T = base_u32 + Ly.S, E_T = base_u32 + Ly.E, EH_T = base_u32 + Ly.Eh;
 
     if (tid == 0) {
@@ -267,18 +292,18 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             uint8_t *qwk = base + Ly.qwk[s];
             // group X: W, Q (or Qbar), T, V, the decay factors.  Q only where o is
             // written; T and V not for a transition CTA.
-            if (i >= 2) {
-                const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
+            {
+                const bool ok = wait_free(FREEX0, i);
                 if (__any_sync(0xffffffffu, !ok))
                     break;
             }
             if (lane == 0) {
                 uint64_t *full = &bars[FULLX0 + s];
-                const uint32_t fac_bytes = scalar ? prep::SC_BYTES - prep::SC_EA : KD * 4;
-                // W, Q: two 64-column images each; T: one; V: 64 x 64 bf16
-                mbar_arrive_expect_tx(full, 2u * prep::IMG + (outputs ? 2u * prep::IMG : 0u) +
+                const uint32_t fac_bytes = scalar ? prep::SC_BYTES - prep::SC_EA : DK * 4;
+                // W, Q: dk / 64 images each; T: one; V: 64 x 64 bf16
+                mbar_arrive_expect_tx(full, NKB * prep::IMG + (outputs ? NKB * prep::IMG : 0u) +
                                                 (trans ? 0u : prep::IMG + CC * NVC * 2) + fac_bytes);
-                for (int kb = 0; kb < KD / 64; ++kb) {
+                for (int kb = 0; kb < NKB; ++kb) {
                     uint8_t *blk = qwk + kb * 192 * 128;
                     bulk_load(blk + 64 * 128, fac + prep::REC_W + kb * prep::IMG, prep::IMG, full);
                     if (!outputs)
@@ -286,12 +311,12 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     if (scalar)
                         tma_load_3d(blk, &tm_q, full, 64 * kb, (int)c0, (int)kh);
                     else
-                        bulk_load(blk, fac + prep::EXT_QB + kb * prep::IMG, prep::IMG, full);
+                        bulk_load(blk, fac + prep::ext_qb(DK) + kb * prep::IMG, prep::IMG, full);
                 }
                 if (scalar)
                     bulk_load(gates_of(s)->ea, fac + prep::SC_EA, fac_bytes, full);
                 else
-                    bulk_load(gates_of(s)->F, fac + prep::EXT_F, fac_bytes, full);
+                    bulk_load(gates_of(s)->F, fac + prep::ext_f(DK), fac_bytes, full);
             }
             armx[s] += 1;
         }
@@ -315,8 +340,8 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             uint8_t *qwk = base + Ly.qwk[s];
             // T and V of group X (counted in the FULLX bytes that warp W_PROD expects)
             if (!trans) {
-                if (i >= 2) {
-                    const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
+                {
+                    const bool ok = wait_free(FREEX0, i);
                     if (__any_sync(0xffffffffu, !ok))
                         break;
                 }
@@ -327,8 +352,8 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
             }
             // group Y: K (or Khat), L (L only where o is written)
-            if (i >= 2) {
-                const bool ok = wait_or_abort(&bars[FREEY0 + s], ((i >> 1) - 1) & 1, abort_flag);
+            {
+                const bool ok = wait_free(FREEY0, i);
                 if (__any_sync(0xffffffffu, !ok))
                     break;
             }
@@ -337,15 +362,15 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const bool with_y = args.pair && s == 0;
             if (lane == 0) {
                 uint64_t *full = &bars[FULLY0 + s];
-                mbar_arrive_expect_tx(full, (outputs ? 3u : 2u) * prep::IMG + (with_y ? prep::IMG : 0u));
+                mbar_arrive_expect_tx(full, (NKB + (outputs ? 1u : 0u)) * prep::IMG + (with_y ? prep::IMG : 0u));
                 if (with_y)
                     bulk_load(base + Ly.lz[s] + 64 * 128, fac + args.pair_y, prep::IMG, full);
-                for (int kb = 0; kb < KD / 64; ++kb) {
+                for (int kb = 0; kb < NKB; ++kb) {
                     uint8_t *blk = qwk + kb * 192 * 128 + 128 * 128;
                     if (scalar)
                         tma_load_3d(blk, &tm_k, full, 64 * kb, (int)c0, (int)kh);
                     else
-                        bulk_load(blk, fac + prep::EXT_KH + kb * prep::IMG, prep::IMG, full);
+                        bulk_load(blk, fac + prep::ext_kh(DK) + kb * prep::IMG, prep::IMG, full);
                 }
                 if (outputs)
                     bulk_load(base + Ly.lz[s], fac + prep::IMG, prep::IMG, full);
@@ -362,7 +387,7 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (lane == 0) {
             const uint32_t id_u = idesc_bf16(128, NVC, false, true);
             const uint32_t id_po = idesc_bf16(128, NVC, false, true);
-            const uint32_t id_s = idesc_bf16(KD, NVC, true, true);
+            const uint32_t id_s = idesc_bf16(128, NVC, true, true);   // per 128 key rows
             // descriptors at k = 0 of stage 0; a K step adds its byte offset / 16 to the
             // start field, stage 1 a fixed distance
             const uint64_t d_ab0 = desc_kmajor(base_u32 + Ly.ab[0], 128, 0, 0);
@@ -372,7 +397,9 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const uint64_t d_lz0 = desc_kmajor(base_u32 + Ly.lz[0], 128, 0, 0);
             const uint64_t dab = (Ly.ab[1] - Ly.ab[0]) >> 4, dv = (Ly.v[1] - Ly.v[0]) >> 4;
             const uint64_t dqw = (Ly.qwk[1] - Ly.qwk[0]) >> 4, dlz = (Ly.lz[1] - Ly.lz[0]) >> 4;
-            const uint64_t d_s = desc_mnmajor(S_T, KD, 0, 0);
+            const uint64_t d_s = desc_mnmajor(S_T, DK, 0, 0);
+            // K^T's rows 128-255 (dk = 256): two 64-column blocks further on
+            const uint64_t dkt_hi = (uint64_t)((2 * 192 * 128) >> 4);
             const uint64_t d_e = desc_mnmajor(scalar ? EH_T : E_T, CC, 0, 0);
             const uint64_t d_eo = desc_mnmajor(E_T, CC, 0, 0);
             auto kstep = [](int k0, int rows) {
@@ -401,7 +428,7 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     break;
                 tc_fence_after();
                 const uint64_t qw = d_qw0 + s * dqw, kt = d_kt0 + s * dqw, lz = d_lz0 + s * dlz;
-                for (int k0 = 0; k0 < KD; k0 += 16)
+                for (int k0 = 0; k0 < DK; k0 += 16)
                     mma_bf16(tmem + T_PO + 64 * s, qw + kstep(k0, 192), d_s + mstep(k0), id_po, k0 > 0);
                 mma_commit(&bars[P_FULL]);
                 // U and P are the last tensor-core readers of group X (the state warps
@@ -419,8 +446,9 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 if (!(ok = wait_or_abort(&bars[FULLY0 + s], (i >> 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
-                for (int k0 = 0; k0 < CC; k0 += 16)
-                    mma_bf16(tmem + T_S, kt + mstep(k0), d_e + mstep(k0), id_s, 1u);
+                for (int h = 0; h < DK / 128; ++h)
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tmem + T_S + 64 * h, kt + h * dkt_hi + mstep(k0), d_e + mstep(k0), id_s, 1u);
                 mma_commit(&bars[UPD_DONE]);
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(tmem + T_LE + 64 * s, lz + kstep(k0, 128), d_eo + mstep(k0), id_po, k0 > 0);
@@ -435,20 +463,23 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // ------------------------------------------------------------ state chain
         const int stid = tid - W_STATE0 * 32;
         const int cs = 32 * ((warp - W_STATE0) >> 2);   // this lane's 32 of the 64 columns
-        {
+        constexpr int NH = DK / 128;                     // key rows R + 128 h of this thread
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
             // start state: S0 (or zero) for a whole sequence, zero for a segment's end
             // state, the identity's columns for a transition, S_start of the segment
+            const int row = R + 128 * h;
             float s0[16], s1[16];
 #pragma unroll
             for (int n = 0; n < 16; ++n) {
-                s0[n] = (trans && R == n0 + cs + n) ? 1.f : 0.f;
-                s1[n] = (trans && R == n0 + cs + 16 + n) ? 1.f : 0.f;
+                s0[n] = (trans && row == n0 + cs + n) ? 1.f : 0.f;
+                s1[n] = (trans && row == n0 + cs + 16 + n) ? 1.f : 0.f;
             }
             const float *src = nullptr;
             if (args.mode == MODE_SEQ && p.S0 != nullptr)
-                src = p.S0 + (vh * KD + R) * p.dv + n0 + cs;
+                src = p.S0 + (vh * DK + row) * p.dv + n0 + cs;
             else if (args.mode == MODE_SEG_C)
-                src = args.seg_start + (((size_t)vh * args.nseg + seg) * KD + R) * p.dv + n0 + cs;
+                src = args.seg_start + (((size_t)vh * args.nseg + seg) * KD + row) * p.dv + n0 + cs;
             if (src != nullptr) {
 #pragma unroll
                 for (int n = 0; n < 16; n += 4) {
@@ -458,8 +489,8 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     s1[n] = b4.x; s1[n + 1] = b4.y; s1[n + 2] = b4.z; s1[n + 3] = b4.w;
                 }
             }
-            tmem_st16(tq + T_S + cs, s0);
-            tmem_st16(tq + T_S + cs + 16, s1);
+            tmem_st16(tq + T_S + 64 * h + cs, s0);
+            tmem_st16(tq + T_S + 64 * h + cs + 16, s1);
         }
         tmem_st_wait();
         bool ok = true;
@@ -474,14 +505,20 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tc_fence_after();
             // S_{c-1} -> bf16 operand of P; only then T_S <- F S_{c-1} (the update MMA
             // accumulates onto it), which nothing reads before E_READY
-            float s0[16], s1[16];
-            tmem_ld16(tq + T_S + cs, s0);
-            tmem_ld16(tq + T_S + cs + 16, s1);
+            float s0[NH][16], s1[NH][16];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                tmem_ld16(tq + T_S + 64 * h + cs, s0[h]);
+                tmem_ld16(tq + T_S + 64 * h + cs + 16, s1[h]);
+            }
             tmem_ld_wait();
-            st_tile8(S_T, KD, R, cs, &s0[0]);
-            st_tile8(S_T, KD, R, cs + 8, &s0[8]);
-            st_tile8(S_T, KD, R, cs + 16, &s1[0]);
-            st_tile8(S_T, KD, R, cs + 24, &s1[8]);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                st_tile8(S_T, DK, R + 128 * h, cs, &s0[h][0]);
+                st_tile8(S_T, DK, R + 128 * h, cs + 8, &s0[h][8]);
+                st_tile8(S_T, DK, R + 128 * h, cs + 16, &s1[h][0]);
+                st_tile8(S_T, DK, R + 128 * h, cs + 24, &s1[h][8]);
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             named_sync(NB_STATE, N_STATE);
@@ -492,19 +529,20 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 ok = false;
                 break;
             }
-            const Gates *gt = gates_of(s);
+            const Gates<DK> *gt = gates_of(s);
             // this thread's factors of the stage, read now: group X is refilled as soon
             // as P is done
             const float f_eb = (scalar && R >= CC) ? gt->eb[R - CC] : 1.f;
-            {
-                const float F = scalar ? gt->F[0] : gt->F[R];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                const float F = scalar ? gt->F[0] : gt->F[R + 128 * h];
 #pragma unroll
                 for (int n = 0; n < 16; ++n) {
-                    s0[n] *= F;
-                    s1[n] *= F;
+                    s0[h][n] *= F;
+                    s1[h][n] *= F;
                 }
-                tmem_st16(tq + T_S + cs, s0);
-                tmem_st16(tq + T_S + cs + 16, s1);
+                tmem_st16(tq + T_S + 64 * h + cs, s0[h]);
+                tmem_st16(tq + T_S + 64 * h + cs + 16, s1[h]);
             }
             if (named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[P_FULL], par, abort_flag))) {
                 ok = false;
@@ -580,17 +618,22 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             dst = trans ? args.seg_trans + (((size_t)kh * args.nseg + seg) * KD + R) * KD + n0 + cs
                         : args.seg_end + (((size_t)vh * args.nseg + seg) * KD + R) * p.dv + n0 + cs;
         else if (p.S_final != nullptr && seg == args.nseg - 1)
-            dst = p.S_final + (vh * KD + R) * p.dv + n0 + cs;
+            dst = p.S_final + (vh * DK + R) * p.dv + n0 + cs;
         if (ok && dst != nullptr) {
             tc_fence_after();
-            float s0[16], s1[16];
-            tmem_ld16(tq + T_S + cs, s0);
-            tmem_ld16(tq + T_S + cs + 16, s1);
-            tmem_ld_wait();
 #pragma unroll
-            for (int n = 0; n < 16; n += 4) {
-                *reinterpret_cast<float4 *>(dst + n) = make_float4(s0[n], s0[n + 1], s0[n + 2], s0[n + 3]);
-                *reinterpret_cast<float4 *>(dst + 16 + n) = make_float4(s1[n], s1[n + 1], s1[n + 2], s1[n + 3]);
+            for (int h = 0; h < NH; ++h) {   // rows R + 128 h (the segment buffers: dk = 128)
+                float s0[16], s1[16];
+                tmem_ld16(tq + T_S + 64 * h + cs, s0);
+                tmem_ld16(tq + T_S + 64 * h + cs + 16, s1);
+                tmem_ld_wait();
+                float *d = dst + (size_t)128 * h * p.dv;
+#pragma unroll
+                for (int n = 0; n < 16; n += 4) {
+                    *reinterpret_cast<float4 *>(d + n) = make_float4(s0[n], s0[n + 1], s0[n + 2], s0[n + 3]);
+                    *reinterpret_cast<float4 *>(d + 16 + n) =
+                        make_float4(s1[n], s1[n + 1], s1[n + 2], s1[n + 3]);
+                }
             }
         }
     } else {
@@ -714,21 +757,24 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
     cp_async_wait_all();
 }
 
+// dk = 128 with any gate grouping; dk = 256 with grouped gates (records of the
+// grouped / per-channel kind: the scalar gate's record is built for dk = 128)
 inline bool supports(const Params &p)
 {
-    return prep::supports(p) && p.dk == KD && p.dv % NVC == 0 && p.G <= KD && p.T >= 1;
+    return prep::supports(p) && (p.dk == KD || (p.dk == 256 && p.G > 1)) && p.dv % NVC == 0 &&
+           p.G <= p.dk && p.T >= 1;
 }
 
-template <bool OB>
+template <int DK, bool OB>
 int launch(const Params &p, const void *factors, cudaStream_t stream)
 {
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, p.q, KD, p.T, (long)p.B * p.Hk, CC) ||
-        !make_map(&mk, p.k, KD, p.T, (long)p.B * p.Hk, CC) ||
+    if (!make_map(&mq, p.q, DK, p.T, (long)p.B * p.Hk, CC) ||
+        !make_map(&mk, p.k, DK, p.T, (long)p.B * p.Hk, CC) ||
         !make_map(&mv, p.v, p.dv, p.T, (long)p.B * p.Hv, CC))
         return 6;
-    const Plan Ly = plan(p.G == 1);
-    auto kern = split_kernel<OB>;
+    const Plan Ly = plan<DK>(p.G == 1);
+    auto kern = split_kernel<DK, OB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
         cudaSuccess)
         return 6;

@@ -139,7 +139,17 @@ def test_kernel_selection(lib):
     assert gdr.select_kernel(bf, 64, gdr.GATE_SCALAR) == gdr.KERNEL_TC2
     assert gdr.select_kernel(gdr.make_shape(4, 4096, 16, 16, 128, 128, kernel="tc"), 64,
                              gdr.GATE_SCALAR) == gdr.KERNEL_TC
-    assert gdr.select_kernel(gdr.make_shape(2, 8192, 8, 32, 256, 128), 64,
+    # dk = 256 with grouped gates: the two-pass path (one [Q | W | K] buffer); the
+    # scalar gate at dk = 256 has no two-pass record and takes the fused kernel
+    sla = gdr.make_shape(2, 8192, 8, 32, 256, 128)
+    assert gdr.select_kernel(sla, 64, gdr.GATE_GROUP64) == gdr.KERNEL_TC2
+    assert gdr.select_kernel(sla, 128, gdr.GATE_GROUP64, "neumann") == gdr.KERNEL_TC2
+    assert gdr.kernel_chunk(sla, 128, gdr.GATE_GROUP64, "neumann") == 128
+    assert gdr.state_segments(sla, 64, gdr.GATE_GROUP64) == 1
+    assert gdr.select_kernel(sla, 64, gdr.GATE_SCALAR) == gdr.KERNEL_TC
+    # records at dk = 256: T, L, then W, Qbar, Khat of four 64-column images and 256 F
+    assert gdr.workspace_bytes(sla, 64, gdr.GATE_GROUP64) == 2 * 8 * 128 * (14 * 8192 + 1024)
+    assert gdr.select_kernel(gdr.make_shape(2, 8192, 8, 32, 256, 128, kernel="tc"), 64,
                              gdr.GATE_GROUP64) == gdr.KERNEL_TC
     f32 = gdr.make_shape(1, 256, 2, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
     assert gdr.select_kernel(f32, 64, gdr.GATE_SCALAR) == gdr.KERNEL_SIMT
@@ -191,8 +201,8 @@ def test_neumann1_selection(lib):
     assert gdr.kernel_chunk(kda, 128, gdr.GATE_CHANNEL, "neumann1") == 128
     forced = gdr.make_shape(1, 256, 2, 2, 128, 128, kernel="tc")
     assert gdr.select_kernel(forced, 64, gdr.GATE_SCALAR, "neumann1") == -gdr.ERR_UNSUPPORTED
-    sla = gdr.make_shape(2, 8192, 8, 32, 256, 128)      # dk = 256: no two-pass path
-    assert gdr.select_kernel(sla, 64, gdr.GATE_GROUP64, "neumann1") == gdr.KERNEL_SIMT
+    sla = gdr.make_shape(2, 8192, 8, 32, 256, 128)      # dk = 256: two-pass path too
+    assert gdr.select_kernel(sla, 64, gdr.GATE_GROUP64, "neumann1") == gdr.KERNEL_TC2
     sh = gdr.make_shape(1, 64, 1, 1, 128, 128)
     assert lib.gdr_kernel_chunk(ctypes.byref(sh), 64, 0, 3) == -gdr.ERR_ARG   # no mode 3
 
@@ -249,7 +259,7 @@ def test_two_pass_simt_selection(lib):
     nch = (1000 + 127) // 128
     assert gdr.workspace_bytes(sh, 128, gdr.GATE_GROUP64, "neumann") == 2 * 8 * nch * 2 * 128 * 128 * 4
     auto = gdr.make_shape(2, 1000, 8, 32, 256, 128)
-    assert gdr.select_kernel(auto, 128, gdr.GATE_GROUP64, "neumann") == gdr.KERNEL_SIMT
+    assert gdr.select_kernel(auto, 128, gdr.GATE_GROUP64, "neumann") == gdr.KERNEL_TC2
     # not enough workspace: nothing launched
     full = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(8)]
     assert _call(sh, full, chunk=128, gate=gdr.GATE_GROUP64, inv=gdr.INV_NEUMANN,

@@ -81,6 +81,15 @@ SMALL = [
     (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 128, "neumann", "tc2"),
     (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 128, "neumann", "tc2"),
     (1, dict(B=2, Hk=1, Hv=3, T=256, dv=192), 128, "neumann", "tc2"),
+    # dk = 256 with grouped gates on the two-pass path (one [Q | W | K] buffer), grouped
+    # value heads, S0, ragged tails, both chunk lengths and every inverse
+    (3, dict(B=1, Hk=2, Hv=8, T=384), 64, "exact", "tc2"),
+    (3, dict(B=1, Hk=1, Hv=4, T=384 - 37, s0_std=0.05), 64, "exact", "tc2"),
+    (3, dict(B=2, Hk=1, Hv=2, T=256, dv=192), 128, "exact", "tc2"),
+    (3, dict(B=1, Hk=2, Hv=8, T=256), 64, "neumann", "tc2"),
+    (3, dict(B=1, Hk=1, Hv=4, T=384 - 37, s0_std=0.05), 128, "neumann", "tc2"),
+    (3, dict(B=1, Hk=1, Hv=4, T=320), 128, "neumann1", "tc2"),
+    (3, dict(B=1, Hk=1, Hv=2, T=200, gate_mode=W.GATE_SCALAR), 64, "exact", "auto"),
     # 1-Step Neumann at chunk 128 (eight blocks of 16, as in the pages) the same way
     (4, dict(Hk=2, Hv=2, T=640 - 27), 128, "neumann1", "tc2"),
     (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 128, "neumann1", "tc2"),
