@@ -201,6 +201,69 @@ __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
     __syncthreads();
 }
 
+// In-place exact inverse of I + M (64 x 64, M strictly lower) by block doubling,
+// the merges spread over all 256 threads: after the exact 16 x 16 diagonal
+// blocks, each merge X21 = -X22 (M21 X11) is two small dense products whose
+// every output element has its own thread (2 columns a thread for the 16 x 16
+// merges, 4 for the 32 x 32 one) and a loop over the full inner index (the zero
+// triangles multiply as zeros, so every lane of a warp runs the same trip
+// count).  Same arithmetic as inverse64_inplace (inner index ascending, fp32),
+// shorter dependent chains; Tf needs 32 x 36 floats.
+__device__ __forceinline__ void inverse64_par(float *Mf, float *Tf, int tid)
+{
+    diag16_inverse_inplace(Mf, Tf, tid);
+    {   // 16 -> 32: pair pr (rows 32 pr + 16 .. +31, columns 32 pr .. +15)
+        const int pr = tid >> 7, q = tid & 127, r = q >> 3, c0 = (q & 7) * 2, o = 32 * pr;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {   // T = M21 X11
+            const float m = Mf[(o + 16 + r) * LDM + o + l];
+            const float2 x = *reinterpret_cast<const float2 *>(&Mf[(o + l) * LDM + o + c0]);
+            a0 += m * x.x;
+            a1 += m * x.y;
+        }
+        *reinterpret_cast<float2 *>(&Tf[(16 * pr + r) * 36 + c0]) = make_float2(a0, a1);
+        __syncthreads();
+        a0 = a1 = 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {   // X21 = -X22 T
+            const float x = Mf[(o + 16 + r) * LDM + o + 16 + l];
+            const float2 t = *reinterpret_cast<const float2 *>(&Tf[(16 * pr + l) * 36 + c0]);
+            a0 += x * t.x;
+            a1 += x * t.y;
+        }
+        *reinterpret_cast<float2 *>(&Mf[(o + 16 + r) * LDM + o + c0]) = make_float2(-a0, -a1);
+        __syncthreads();
+    }
+    {   // 32 -> 64: rows 32 .. 63, columns 0 .. 31
+        const int r = tid >> 3, c0 = (tid & 7) * 4;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) {   // T = M21 X11
+            const float m = Mf[(32 + r) * LDM + l];
+            const float4 x = *reinterpret_cast<const float4 *>(&Mf[l * LDM + c0]);
+            a[0] += m * x.x;
+            a[1] += m * x.y;
+            a[2] += m * x.z;
+            a[3] += m * x.w;
+        }
+        *reinterpret_cast<float4 *>(&Tf[r * 36 + c0]) = make_float4(a[0], a[1], a[2], a[3]);
+        __syncthreads();
+        a[0] = a[1] = a[2] = a[3] = 0.f;
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) {   // X21 = -X22 T
+            const float x = Mf[(32 + r) * LDM + 32 + l];
+            const float4 t = *reinterpret_cast<const float4 *>(&Tf[l * 36 + c0]);
+            a[0] += x * t.x;
+            a[1] += x * t.y;
+            a[2] += x * t.z;
+            a[3] += x * t.w;
+        }
+        *reinterpret_cast<float4 *>(&Mf[(32 + r) * LDM + c0]) = make_float4(-a[0], -a[1], -a[2], -a[3]);
+        __syncthreads();
+    }
+}
+
 // In-place 1-Step Neumann approximation of (I + M)^{-1} ("Systolic Linear
 // Attention ...", §2.4.3): with D the block-diagonal part of I + M in 16-row
 // blocks and N = D^{-1} M_off, A = (I - N) D^{-1}, i.e. the exact inverses D_ii^{-1}

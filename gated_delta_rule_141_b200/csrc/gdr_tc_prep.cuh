@@ -76,7 +76,7 @@ __host__ __device__ constexpr uint32_t pair_extra(int kind, int dk = 128)
 __host__ __device__ constexpr int gmax(int dk) { return dk == 256 ? 8 : 128; }
 
 struct Plan {
-    uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, TB, lam, beta, piv, IT, bar, misc, total, tmem_cols, tn;
+    uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, TB, lam, beta, piv, bar, misc, total, tmem_cols, tn;
 };
 
 __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
@@ -111,13 +111,6 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
     s.lam = take(CC * G * 4 + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
     s.beta = s.lam + CC * G * 4;
     s.piv = G > 1 ? take(2 * dk * 4) : 0;   // per channel: e^{Lambda_p}, e^{Lambda_C - Lambda_p}
-    // four bf16 64 x 64 operand tiles of the tensor-core inverse (grouped / per-channel
-    // gates, middle pivot): in the Lambda tile or the Gram's column-operand tile, both
-    // dead by then, when one of them is large enough
-    s.IT = G == 1 ? 0u
-           : CC * G * 4 >= 4 * 8192          ? s.lam   // per-channel gates at dk = 128
-           : (dk / 64) * 64 * 128 >= 4 * 8192 ? s.KC    // the column operand tile, dk = 256
-                                               : take(4 * 8192);
     s.bar = (s.beta + CC * 4 + NROUND * 4 + 7u) & ~7u;
     s.misc = s.bar + 24;
     s.total = o + 1024;
@@ -167,122 +160,6 @@ __device__ __forceinline__ void lam8(const float *lam, int G, int wsh, int t, in
     }
 }
 
-__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
-
-// (I + M)^{-1} in place for the 64 x 64 strictly lower M in Mf (fp32, row stride
-// LDM) by block doubling ("Systolic Linear Attention ...", §2.4.3): the 16 x 16
-// diagonal blocks exactly in fp32 (forward substitution), then the two merges
-// X21 = -X22 M21 X11 (16 -> 32 -> 64) as products of whole 64 x 64 matrices on
-// tcgen05: with D the block-diagonal inverse and N the sub-diagonal blocks of M
-// at that level, the merged inverse is D - (D N) D (the products of the zero
-// blocks are exact zeros).  Each product takes bf16 operands split into high and
-// low parts (x = hi + lo, both bf16) and sums hi*hi + hi*lo + lo*hi in fp32, so
-// the merges carry about 16 bits of precision instead of bf16's 8.  Tiles: four
-// 64 x 64 bf16 operand tiles at `tile` (8 KB each, 1024-aligned); tensor memory:
-// 64 columns at `tmem` (M = 64 accumulator).  Returns true if a bounded wait gave
-// up (the status word is set).  All threads of the CTA call it.
-__device__ bool inverse64_tc(float *Mf, float *Tf, uint32_t tile, uint32_t tmem, uint32_t tq,
-                             uint64_t *bar, uint32_t &ph, int tid)
-{
-    using namespace ptx;
-    const int warp = tid >> 5, lane = tid & 31;
-    const uint32_t AH = tile, AL = tile + 8192, BH = tile + 16384, BL = tile + 24576;
-    gen::diag16_inverse_inplace(Mf, Tf, tid);
-    // hi / lo tiles of the entries of Mf selected by keep(t, j); zeros elsewhere
-    auto split = [&](uint32_t th, uint32_t tl, auto keep) {
-        for (int u = tid; u < CC * 8; u += NT) {
-            const int t = u >> 3, j0 = (u & 7) * 8;
-            float h[8], l[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float x = keep(t, j0 + e) ? Mf[t * LDM + j0 + e] : 0.f;
-                h[e] = bf16_round(x);
-                l[e] = x - h[e];
-            }
-            st_tile8(th, 64, t, j0, h);
-            st_tile8(tl, 64, t, j0, l);
-        }
-    };
-    // D[tmem] = A B over K = 64, A K-major (hi ah, lo al), B MN-major (hi bh, lo bl)
-    auto product = [&](uint32_t ah, uint32_t al, uint32_t bh, uint32_t bl) {
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(64, 64, false, true);
-            for (int k0 = 0; k0 < CC; k0 += 16)
-                mma_bf16(tmem, desc_kmajor(ah, 64, 0, k0), desc_mnmajor(bh, 64, k0, 0), id, k0 > 0);
-            for (int k0 = 0; k0 < CC; k0 += 16)
-                mma_bf16(tmem, desc_kmajor(ah, 64, 0, k0), desc_mnmajor(bl, 64, k0, 0), id, 1u);
-            for (int k0 = 0; k0 < CC; k0 += 16)
-                mma_bf16(tmem, desc_kmajor(al, 64, 0, k0), desc_mnmajor(bh, 64, k0, 0), id, 1u);
-            mma_commit(bar);
-        }
-        const bool gave_up = !mbar_wait(bar, ph);
-        if (gave_up)
-            atomicExch(&g_device_status, kTimeoutStatus);
-        ph ^= 1u;
-        const bool f = __syncthreads_or(gave_up ? 1 : 0) != 0;
-        tc_fence_after();
-        return f;
-    };
-    // this thread's row of the M = 64 accumulator (or -1) and its 32 columns
-    const int rr = gen::row64g(warp, lane), cb = 32 * (warp >> 2);
-    auto read = [&](float (&v)[32]) {
-        float a[16], b[16];
-        tmem_ld16(tq + cb, a);
-        tmem_ld16(tq + cb + 16, b);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            v[e] = a[e];
-            v[16 + e] = b[e];
-        }
-    };
-    // -P as hi / lo operand tiles (row rr, columns cb .. cb + 31)
-    auto put_neg = [&](const float (&v)[32]) {
-        if (rr < 0)
-            return;
-#pragma unroll
-        for (int c = 0; c < 32; c += 8) {
-            float h[8], l[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                h[e] = bf16_round(-v[c + e]);
-                l[e] = -v[c + e] - h[e];
-            }
-            st_tile8(BH, 64, rr, cb + c, h);
-            st_tile8(BL, 64, rr, cb + c, l);
-        }
-    };
-    for (int lvl = 0; lvl < 2; ++lvl) {
-        const int w = 16 << lvl;   // blocks of w rows merge into blocks of 2w
-        split(AH, AL, [w](int t, int j) { return t / w == j / w; });                        // D
-        split(BH, BL, [w](int t, int j) { return t / w == j / w + 1 && (t / w) % 2 == 1; });  // N
-        if (product(AH, AL, BH, BL))   // D N
-            return true;
-        float v[32];
-        read(v);
-        tc_fence_before();
-        __syncthreads();               // every read of the N tiles done
-        put_neg(v);
-        if (product(BH, BL, AH, AL))   // -(D N) D: the merged blocks below the diagonal
-            return true;
-        read(v);
-        if (rr >= 0)
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int c = cb + e;
-                if (rr / w == c / w + 1 && (rr / w) % 2 == 1)
-                    Mf[rr * LDM + c] = v[e];
-            }
-        tc_fence_before();
-        __syncthreads();
-    }
-    return false;
-}
-
 // SCALAR: the scalar-gate instantiation (no pivoting machinery, four CTAs per SM);
 // otherwise grouped / per-channel gates (two CTAs per SM: the gate tile is larger).
 template <int DK, bool SCALAR>
@@ -323,6 +200,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const float *g_src = p.g + (kh * T + c0) * G;
     const uint32_t g_bytes = (uint32_t)(Cl * G * 4);
     const bool g_bulk = !SCALAR && (g_bytes & 15u) == 0 && (reinterpret_cast<uintptr_t>(g_src) & 15u) == 0;
+    // beta of a full chunk: one 256-byte bulk copy on the q, k barrier when aligned
+    const float *b_src = p.beta + kh * T + c0;
+    const bool b_bulk = Cl == CC && (reinterpret_cast<uintptr_t>(b_src) & 15u) == 0;
     if (tid == 0) {
         mbar_init(&bars[0], 1);     // TMA of q, k
         mbar_init(&bars[1], 1);     // MMA
@@ -332,7 +212,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             mbar_arrive_expect_tx(&bars[2], g_bytes);
             bulk_load(lam, g_src, g_bytes, &bars[2]);
         }
-        mbar_arrive_expect_tx(&bars[0], 2u * CC * DK * 2u);
+        mbar_arrive_expect_tx(&bars[0], 2u * CC * DK * 2u + (b_bulk ? CC * 4u : 0u));
+        if (b_bulk)
+            bulk_load(sbeta, b_src, CC * 4u, &bars[0]);
         for (int kb = 0; kb < DK / 64; ++kb) {
             tma_load_3d(base + Ly.QK + kb * 128 * 128, &tm_q, &bars[0], 64 * kb, (int)c0, (int)kh);
             tma_load_3d(base + Ly.QK + kb * 128 * 128 + 64 * 128, &tm_k, &bars[0], 64 * kb, (int)c0,
@@ -343,8 +225,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_alloc(tmem_slot, Ly.tmem_cols);
         tmem_relinquish();
     }
-    for (int t = tid; t < CC; t += NT)
-        sbeta[t] = t < Cl ? p.beta[kh * T + c0 + t] : 0.f;
+    if (!b_bulk)
+        for (int t = tid; t < CC; t += NT)
+            sbeta[t] = t < Cl ? b_src[t] : 0.f;
     if (g_bulk) {
         for (int u = Cl * G + tid; u < CC * G; u += NT)   // rows past T (not copied)
             lam[u] = 0.f;
@@ -738,10 +621,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!neu) {
             if (p.neumann1)
                 gen::block_neumann1_64_inplace(Mf, Tf, tid);
-            else if (SCALAR || wide)
-                gen::inverse64_inplace(Mf, Tf, tid);
             else
-                failed = inverse64_tc(Mf, Tf, base_u32 + Ly.IT, tmem, tq, &bars[1], ph_mma, tid);
+                gen::inverse64_par(Mf, Tf, tid);
         } else {
             // ---- truncated Neumann series (Horner) + Newton residual steps, M = 64 on tcgen05
             const uint32_t NB = base_u32 + Ly.NB, XB = base_u32 + Ly.XB, RB = base_u32 + Ly.RB;
