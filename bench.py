@@ -64,7 +64,7 @@ def parse_args():
                          "profiling captures; the JSON config records it)")
     ap.add_argument("--inverse", default="exact", choices=["exact", "neumann", "neumann1"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "simt", "simt2"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tc", "tc2", "tc2w", "simt", "simt2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--epilogue", action="store_true",
@@ -564,10 +564,11 @@ def main():
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda") if ws_bytes else None
     kern = gdr.select_kernel(shape_run, chunk, gm_run, args.inverse)
     # the two-pass path: pass 1, then one state pass, or three when segmented
-    nseg = gdr.state_segments(shape_run, chunk, gm_run, args.inverse) if kern == gdr.KERNEL_TC2 else 0
+    two_pass = kern in (gdr.KERNEL_TC2, gdr.KERNEL_TC2W)
+    nseg = gdr.state_segments(shape_run, chunk, gm_run, args.inverse) if two_pass else 0
     # Neumann at chunk 128 on the two-pass path adds the pair kernel after pass 1
-    pair = kern == gdr.KERNEL_TC2 and args.inverse in ("neumann", "neumann1") and chunk == 128
-    launches_per_step = ((1 + (1 if nseg == 1 else 3) + (1 if pair else 0)) if kern == gdr.KERNEL_TC2
+    pair = two_pass and args.inverse in ("neumann", "neumann1") and chunk == 128
+    launches_per_step = ((1 + (1 if nseg == 1 else 3) + (1 if pair else 0)) if two_pass
                          else 2 if kern == gdr.KERNEL_SIMT2 else 1)
     zgate = None
     if args.epilogue:   # output-gate logits z ~ N(0, 1), seeded apart from the workload's draws

@@ -25,7 +25,7 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
     if (s->out_dtype != GDR_F32 && s->out_dtype != GDR_BF16)
         return GDR_ERR_DTYPE;
     if (s->kernel != GDR_KERNEL_AUTO && s->kernel != GDR_KERNEL_SIMT && s->kernel != GDR_KERNEL_TC &&
-        s->kernel != GDR_KERNEL_TC2 && s->kernel != GDR_KERNEL_SIMT2)
+        s->kernel != GDR_KERNEL_TC2 && s->kernel != GDR_KERNEL_SIMT2 && s->kernel != GDR_KERNEL_TC2W)
         return GDR_ERR_ARG;
     if (s->B < 0 || s->T < 0 || s->Hk < 1 || s->Hv < 1 || s->Hv % s->Hk != 0)
         return GDR_ERR_SHAPE;
@@ -65,6 +65,7 @@ gdr_status make_params(const gdr_shape *s, int chunk, gdr_gate_mode gm, gdr_inve
     p->neumann1 = im == GDR_INV_NEUMANN1;
     p->neu_order = p->neumann ? s->neumann_order : 0;
     p->neu_resid = p->neumann ? s->neumann_residual_steps : 0;
+    p->wide_state = s->kernel == GDR_KERNEL_TC2W;
     return GDR_OK;
 }
 
@@ -82,6 +83,10 @@ int choose(const gdr::Params &p, gdr_kernel want, size_t ws_bytes)
         if (!tc2)
             return -GDR_ERR_UNSUPPORTED;
         return tc2_fits ? GDR_KERNEL_TC2 : -GDR_ERR_WORKSPACE;
+    case GDR_KERNEL_TC2W:
+        if (!gdr::tc2w_supports(p))
+            return -GDR_ERR_UNSUPPORTED;
+        return tc2_fits ? GDR_KERNEL_TC2W : -GDR_ERR_WORKSPACE;
     case GDR_KERNEL_TC: return tc ? GDR_KERNEL_TC : -GDR_ERR_UNSUPPORTED;
     case GDR_KERNEL_SIMT: return simt ? GDR_KERNEL_SIMT : -GDR_ERR_UNSUPPORTED;
     case GDR_KERNEL_SIMT2:
@@ -129,7 +134,7 @@ gdr_status launch_fwd(const gdr::Params &p, int which, void *workspace, cudaStre
     if (p.B == 0)
         return GDR_OK;
     int rc;
-    if (which == GDR_KERNEL_TC2)
+    if (which == GDR_KERNEL_TC2 || which == GDR_KERNEL_TC2W)
         rc = gdr::launch_tc2(p, workspace, s);
     else if (which == GDR_KERNEL_SIMT2)
         rc = gdr::launch_simt2(p, workspace, s);
@@ -249,7 +254,7 @@ gdr_status gdr_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode 
     const int which = choose(p, shape->kernel, SIZE_MAX);
     if (which < 0)
         return static_cast<gdr_status>(-which);
-    *bytes = which == GDR_KERNEL_TC2     ? gdr::tc2_workspace_bytes(p)
+    *bytes = which == GDR_KERNEL_TC2 || which == GDR_KERNEL_TC2W ? gdr::tc2_workspace_bytes(p)
              : which == GDR_KERNEL_SIMT2 ? gdr::simt2_workspace_bytes(p)
                                          : 0;
     return GDR_OK;
@@ -367,7 +372,7 @@ int gdr_state_segments(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mod
     const int which = choose(p, shape->kernel, SIZE_MAX);
     if (which < 0)
         return which;
-    return which == GDR_KERNEL_TC2 ? gdr::tc2_state_segments(p) : 0;
+    return (which == GDR_KERNEL_TC2 || which == GDR_KERNEL_TC2W) ? gdr::tc2_state_segments(p) : 0;
 }
 
 gdr_status gdr_device_status(void *stream)

@@ -19,6 +19,8 @@ struct Params {
     int neumann1;   // 1-Step Neumann in blocks of 16 (neumann is 0 then)
     int pair;       // two-pass path: the request's chunk of 2C runs as pairs of C-token
                     // halves, the second half corrected by the pair's Y (internal)
+    int wide_state; // two-pass path: 1 forces the 128-column state pass, 0 leaves it
+                    // to the segment cost model
     int neu_order;  // Neumann order m
     int neu_resid;  // Newton residual corrections
     int momentum;   // chunk-boundary momentum (CUDA-core kernel only)
@@ -71,6 +73,8 @@ int launch_tc(const Params &p, cudaStream_t stream);
 // Two-pass tensor-core path: the chunk-local factors of all chunks in parallel
 // (written to a caller-owned workspace), then the state pass that reads them.
 bool tc2_supports(const Params &p);
+// ... with the 128-column state pass (GDR_KERNEL_TC2W)
+bool tc2w_supports(const Params &p);
 size_t tc2_workspace_bytes(const Params &p);
 int launch_tc2(const Params &p, void *workspace, cudaStream_t stream);
 // Segments per sequence of its state pass (1: sequential; more: segment-parallel).

@@ -617,6 +617,7 @@ __global__ void __launch_bounds__(32, 1) wait_probe_kernel(uint64_t limit_ns)
 #include "gdr_tc_prep.cuh"
 #include "gdr_tc_pair.cuh"
 #include "gdr_tc_split.cuh"
+#include "gdr_tc_split128.cuh"
 
 }  // namespace
 
@@ -672,15 +673,17 @@ int launch_tc(const Params &p0, cudaStream_t stream)
 
 bool tc2_supports(const Params &p0) { return split::supports(as_kernel_chunk(p0)); }
 
+bool tc2w_supports(const Params &p0) { return split::supports128(as_kernel_chunk(p0)); }
+
 size_t tc2_workspace_bytes(const Params &p0)
 {
     // the records, then (for few long sequences) the segmented state pass's buffers
     const Params p = as_kernel_chunk(p0);
-    const size_t rec = prep::ws_bytes(p), seg = split::seg_bytes(p);
+    const size_t rec = prep::ws_bytes(p), seg = split::state_seg_bytes(p);
     return seg == 0 ? rec : ((rec + 255) & ~size_t(255)) + seg;
 }
 
-int tc2_state_segments(const Params &p0) { return split::seg_plan(as_kernel_chunk(p0)).nseg; }
+int tc2_state_segments(const Params &p0) { return split::state_seg_plan(as_kernel_chunk(p0)).nseg; }
 
 int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
 {
@@ -698,11 +701,15 @@ int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
         return p.out_bf16 ? split::launch<256, true>(p, workspace, stream)
                           : split::launch<256, false>(p, workspace, stream);
     }
-    rc = prep::launch<128>(p, workspace, kind, stream, p.pair);
+    const bool wide = split::use128(p);   // the 128-column state pass (stores -W)
+    rc = prep::launch<128>(p, workspace, kind, stream, p.pair, wide ? 1 : 0);
     if (rc == 0 && p.pair)
         rc = pair::launch<128>(p, workspace, stream);
     if (rc != 0)
         return rc;
+    if (wide)
+        return p.out_bf16 ? split::launch128<true>(p, workspace, stream)
+                          : split::launch128<false>(p, workspace, stream);
     return p.out_bf16 ? split::launch<128, true>(p, workspace, stream)
                       : split::launch<128, false>(p, workspace, stream);
 }

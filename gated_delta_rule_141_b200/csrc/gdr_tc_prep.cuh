@@ -127,6 +127,7 @@ struct PrepArgs {
     uint32_t rec_bytes;
     uint32_t base_bytes;   // the kind's own record; pair extras follow it (pair != 0)
     int pair;              // also write the pair extras (Ntil, and Kbar for REC_EXT)
+    int neg_w;             // store -W (the 128-column state pass accumulates U - W S)
 };
 
 // Store 8 floats as bf16 into the 16-byte chunk of row r holding columns [c, c+8)
@@ -834,6 +835,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                 w1[e] *= Tf[cw + cb + 16 + e];
                             }
                         }
+                        if (a.neg_w) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                w0[e] = -w0[e];
+                                w1[e] = -w1[e];
+                            }
+                        }
                         const int col = cw + cb;   // 32 columns inside one 64-column image
                         uint8_t *img_W = img_T + REC_W + (col >> 6) * IMG;
                         st_img8(img_W, rr, col & 63, &w0[0]);
@@ -890,7 +898,7 @@ inline bool supports(const Params &p)
 }
 
 template <int DK>
-int launch(const Params &p, void *out, int kind, cudaStream_t stream, int pair = 0)
+int launch(const Params &p, void *out, int kind, cudaStream_t stream, int pair = 0, int neg_w = 0)
 {
     const int N = nchunks(p);
     if (N == 0 || p.B == 0)
@@ -911,6 +919,7 @@ int launch(const Params &p, void *out, int kind, cudaStream_t stream, int pair =
     a.kind = kind;
     a.base_bytes = kind_bytes(kind, DK);
     a.pair = pair;
+    a.neg_w = neg_w;
     a.rec_bytes = a.base_bytes + (pair ? pair_extra(kind, DK) : 0u);
     dim3 grid(N, p.Hk, p.B);
     kern<<<grid, NT, Ly.total, stream>>>(mq, mk, a);

@@ -26,11 +26,12 @@ GATE_SCALAR, GATE_GROUP64, GATE_CHANNEL = 0, 1, 2
 # gdr_inverse_mode
 INV_EXACT, INV_NEUMANN, INV_NEUMANN1 = 0, 1, 2
 # gdr_kernel
-KERNEL_AUTO, KERNEL_SIMT, KERNEL_TC, KERNEL_TC2, KERNEL_SIMT2 = 0, 1, 2, 3, 4
+KERNEL_AUTO, KERNEL_SIMT, KERNEL_TC, KERNEL_TC2, KERNEL_SIMT2, KERNEL_TC2W = 0, 1, 2, 3, 4, 5
 
 _KERNELS = {"auto": KERNEL_AUTO, "simt": KERNEL_SIMT, "tc": KERNEL_TC, "tc2": KERNEL_TC2,
-            "simt2": KERNEL_SIMT2}
-KERNEL_NAMES = {KERNEL_SIMT: "simt", KERNEL_TC: "tc", KERNEL_TC2: "tc2", KERNEL_SIMT2: "simt2"}
+            "simt2": KERNEL_SIMT2, "tc2w": KERNEL_TC2W}
+KERNEL_NAMES = {KERNEL_SIMT: "simt", KERNEL_TC: "tc", KERNEL_TC2: "tc2", KERNEL_SIMT2: "simt2",
+                KERNEL_TC2W: "tc2w"}
 
 # bytes of one chunk record written by gdr_chunk_prepare (T then L, 64 x 64 bf16 each)
 PREP_CHUNK_BYTES = 16384

@@ -86,9 +86,16 @@ typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1, GDR_INV_NEUMANN1 = 2 } gd
  *        {64,128,256}, dv % 64 == 0, chunk 64, or 128 in exact mode).
  *  TC2   two tensor-core passes: the chunk-local factors of every chunk in
  *        parallel (gdr_chunk_prepare), written to the caller's workspace, then
- *        the state pass that reads them (bf16 inputs, dk = 128, dv % 64 == 0,
- *        chunk 64, or 128 in exact mode).  Needs gdr_workspace_bytes() of
- *        device workspace.
+ *        the state pass that reads them (bf16 inputs, dk = 128 with any gate
+ *        grouping or dk = 256 with grouped / per-channel gates, dv % 64 == 0,
+ *        chunk 64 or 128, every inverse mode).  Needs gdr_workspace_bytes() of
+ *        device workspace.  For few long sequences its state pass runs
+ *        segment-parallel, with 128 value columns per CTA when that is the
+ *        cheaper.
+ *  TC2W  TC2 with the 128-column state pass forced (grouped / per-channel
+ *        gates, dk = 128, dv % 128 == 0, exact inverse or chunk 64): a test
+ *        and benchmark switch; gdr_select_kernel reports TC2 for what AUTO
+ *        picks.
  *  SIMT  the fp32 CUDA-core kernel (any dtype, chunk 1..128).
  *  SIMT2 the same arithmetic in two passes: the chunk inverse and score matrix
  *        L of every chunk in parallel, written to the caller's workspace
@@ -99,7 +106,7 @@ typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1, GDR_INV_NEUMANN1 = 2 } gd
  *        TC when it applies, else SIMT.  Forcing a kernel outside its
  *        envelope fails with GDR_ERR_UNSUPPORTED.                           */
 typedef enum { GDR_KERNEL_AUTO = 0, GDR_KERNEL_SIMT = 1, GDR_KERNEL_TC = 2,
-               GDR_KERNEL_TC2 = 3, GDR_KERNEL_SIMT2 = 4 } gdr_kernel;
+               GDR_KERNEL_TC2 = 3, GDR_KERNEL_SIMT2 = 4, GDR_KERNEL_TC2W = 5 } gdr_kernel;
 
 /* Shape of a request.  Besides the per-field ranges, B * Hv must be below 2^31
  * and B * T * (Hk dk + Hv dv) must not exceed 2^40 elements (GDR_ERR_SHAPE

@@ -49,8 +49,9 @@ def test_enums_match_header():
         gdr.GATE_SCALAR, gdr.GATE_GROUP64, gdr.GATE_CHANNEL)
     assert (val("GDR_INV_EXACT"), val("GDR_INV_NEUMANN")) == (gdr.INV_EXACT, gdr.INV_NEUMANN)
     assert (val("GDR_KERNEL_AUTO"), val("GDR_KERNEL_SIMT"), val("GDR_KERNEL_TC"),
-            val("GDR_KERNEL_TC2"), val("GDR_KERNEL_SIMT2")) == (
-        gdr.KERNEL_AUTO, gdr.KERNEL_SIMT, gdr.KERNEL_TC, gdr.KERNEL_TC2, gdr.KERNEL_SIMT2)
+            val("GDR_KERNEL_TC2"), val("GDR_KERNEL_SIMT2"), val("GDR_KERNEL_TC2W")) == (
+        gdr.KERNEL_AUTO, gdr.KERNEL_SIMT, gdr.KERNEL_TC, gdr.KERNEL_TC2, gdr.KERNEL_SIMT2,
+        gdr.KERNEL_TC2W)
     # struct layout: 11 ints
     assert ctypes.sizeof(gdr.GdrShape) == 44
 
@@ -304,6 +305,27 @@ def test_backward_validates(lib):
                     ws_bytes=1 << 30) == gdr.ERR_UNSUPPORTED
     empty = gdr.make_shape(0, 100, 1, 2, 64, 48, in_dtype=gdr.F32, out_dtype=gdr.F32)
     assert call(empty) == gdr.OK
+
+
+def test_wide_state_pass_selection(lib):
+    # the 128-column state pass: forced with TC2W (grouped / per-channel gates, dk = 128,
+    # dv % 128 == 0, no pair correction); AUTO takes it for few long sequences
+    kda = gdr.make_shape(1, 4096, 1, 1, 128, 128, kernel="tc2w")
+    assert gdr.select_kernel(kda, 64, gdr.GATE_CHANNEL) == gdr.KERNEL_TC2W
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL) == gdr.KERNEL_TC2W
+    assert gdr.select_kernel(kda, 64, gdr.GATE_SCALAR) == -gdr.ERR_UNSUPPORTED
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann") == -gdr.ERR_UNSUPPORTED
+    assert gdr.select_kernel(gdr.make_shape(1, 4096, 1, 1, 128, 64, kernel="tc2w"), 64,
+                             gdr.GATE_CHANNEL) == -gdr.ERR_UNSUPPORTED
+    long = gdr.make_shape(1, 65536, 16, 16, 128, 128)
+    assert gdr.select_kernel(long, 128, gdr.GATE_CHANNEL) == gdr.KERNEL_TC2
+    nseg = gdr.state_segments(long, 128, gdr.GATE_CHANNEL)
+    assert nseg >= 2
+    # the workspace follows the plan of the pass that runs
+    forced = gdr.make_shape(1, 65536, 16, 16, 128, 128, kernel="tc2w")
+    assert gdr.state_segments(forced, 128, gdr.GATE_CHANNEL) == nseg
+    assert gdr.workspace_bytes(forced, 128, gdr.GATE_CHANNEL) == \
+        gdr.workspace_bytes(long, 128, gdr.GATE_CHANNEL)
 
 
 def test_state_segments(lib):

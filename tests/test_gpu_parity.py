@@ -81,6 +81,12 @@ SMALL = [
     (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 128, "neumann", "tc2"),
     (1, dict(B=1, Hk=2, Hv=2, T=320 - 13), 128, "neumann", "tc2"),
     (1, dict(B=2, Hk=1, Hv=3, T=256, dv=192), 128, "neumann", "tc2"),
+    # the 128-column state pass forced (sequential here: one segment), both decays,
+    # grouped gates, two value tiles, the Neumann inverse at chunk 64
+    (4, dict(Hk=2, Hv=2, T=640 - 5), 128, "exact", "tc2w"),
+    (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 64, "exact", "tc2w"),
+    (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 64, "exact", "tc2w"),
+    (2, dict(B=1, Hk=1, Hv=2, T=300, dv=256), 64, "neumann", "tc2w"),
     # dk = 256 with grouped gates on the two-pass path (one [Q | W | K] buffer), grouped
     # value heads, S0, ragged tails, both chunk lengths and every inverse
     (3, dict(B=1, Hk=2, Hv=8, T=384), 64, "exact", "tc2"),

@@ -52,3 +52,30 @@ def test_segmented_state_pass(idx, over):
     print("rel err o %.3e  S_final %.3e" % (eo, es))
     assert np.isfinite(o).all() and np.isfinite(Sf).all()
     assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
+
+
+# The 128-column state pass (forced): one value CTA per head and one transition CTA
+# per key head per segment, U / P / E / O sharing one tensor-memory buffer.
+WIDE = [
+    (4, dict(Hk=1, Hv=1, T=64 * 60 + 17)),        # strong per-channel decay, S0
+    (2, dict(B=1, Hk=1, Hv=2, T=64 * 52 - 9)),    # two value heads, one transition
+    (2, dict(B=1, Hk=1, Hv=1, T=64 * 48, dv=256, gate_mode=W.GATE_GROUP64)),   # two value tiles
+]
+
+
+@pytest.mark.parametrize("idx,over", WIDE,
+                         ids=["w%d-%s" % (c[0], "-".join("%s%s" % kv for kv in c[1].items())) for c in WIDE])
+def test_wide_segmented_state_pass(idx, over):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from gated_delta_rule_141_b200 import gdr
+    w, x = W.workload_inputs(idx, **over)
+    shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, kernel="tc2w")
+    assert gdr.state_segments(shape, 64, gdr.gate_mode_for(w.G, w.dk)) > 1
+    o, Sf = U.run_gpu(x, w.in_dtype, 64, "exact", kernel="tc2w")
+    o_ref, S_ref = U.oracle_reference(x, 64, "exact")
+    eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
+    print("rel err o %.3e  S_final %.3e" % (eo, es))
+    assert np.isfinite(o).all() and np.isfinite(Sf).all()
+    assert eo <= U.TOL_BF16 and es <= U.TOL_BF16

@@ -168,7 +168,7 @@ extern "C" int emu_bwd(const gdr::Params *p)
 class Params(ctypes.Structure):
     # gdr::Params of gdr_internal.h, field for field
     _fields_ = ([(n, ctypes.c_int) for n in
-                 "B T Hk Hv dk dv G C R in_bf16 out_bf16 neumann neumann1 pair neu_order neu_resid "
+                 "B T Hk Hv dk dv G C R in_bf16 out_bf16 neumann neumann1 pair wide_state neu_order neu_resid "
                  "momentum".split()] +
                 [("mu", ctypes.c_float), ("kappa", ctypes.c_void_p)] +
                 [(n, ctypes.c_void_p) for n in
