@@ -101,15 +101,15 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
         s.Mf = take(CC * LDM * 4 + 32 * 36 * 4);
     }
     s.Tf = s.Mf + CC * LDM * 4;
-    if (neumann) {                                // Neumann operands
-        s.NB = take(3 * 8192);
+    s.lam = take(CC * G * 4 + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
+    s.beta = s.lam + CC * G * 4;
+    if (neumann) {   // Neumann operands: in the Lambda tile (dead by the inverse) when it is large enough
+        s.NB = CC * G * 4 >= 3 * 8192 ? s.lam : take(3 * 8192);
         s.XB = s.NB + 8192;
         s.RB = s.NB + 16384;
     } else {
         s.NB = s.XB = s.RB = 0;
     }
-    s.lam = take(CC * G * 4 + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
-    s.beta = s.lam + CC * G * 4;
     s.piv = G > 1 ? take(2 * dk * 4) : 0;   // per channel: e^{Lambda_p}, e^{Lambda_C - Lambda_p}
     s.bar = (s.beta + CC * 4 + NROUND * 4 + 7u) & ~7u;
     s.misc = s.bar + 24;
@@ -597,6 +597,21 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
         }
     }
+    if (!failed && a.kind != REC_PLAIN && !SCALAR && wide) {
+        // Kbar = k e^{Lambda_t} in place in the raw k rows of the pivoted blocks, before the
+        // inverse: the last use of Lambda there, whose tile then holds the Neumann operands
+        __syncthreads();
+        for (int u = tid; u < CC * (DK / 8); u += NT) {
+            const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+            float kv[8], lt[8];
+            ld_tile8(QK, 128, 64 + t, i0, kv);
+            lam8(lam, G, wsh, t, i0, lt);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                kv[e] *= __expf(lt[e]);
+            st_tile8(QK, 128, 64 + t, i0, kv);
+        }
+    }
     if (!failed && a.pair) {
         // Mf holds the decayed Gram of the k rows (strictly lower): the pair kernel's
         // Ntil = diag(beta) Gram (beta on the rows) as an image, then M = Gram diag(beta)
@@ -735,19 +750,6 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const bool with_w = a.kind != REC_PLAIN;
     if (!failed) {
         __syncthreads();
-        if (with_w && !SCALAR && wide) {
-            // Kbar = k e^{Lambda_t} in place in the raw k rows of the pivoted blocks
-            for (int u = tid; u < CC * (DK / 8); u += NT) {
-                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float kv[8], lt[8];
-                ld_tile8(QK, 128, 64 + t, i0, kv);
-                lam8(lam, G, wsh, t, i0, lt);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    kv[e] *= __expf(lt[e]);
-                st_tile8(QK, 128, 64 + t, i0, kv);
-            }
-        }
         // After the middle pivot the k rows hold k e^{Lambda_t - Lambda_p}: W is then
         // (T that) diag(e^{Lambda_p}), the column factors applied on the way out of TMEM
         // (copied into the inverse's scratch, free by now).
