@@ -391,14 +391,26 @@ def run_variant(args, w, chunk, rank, world, local):
     else:          # kappa: 0 with probability 1/8 per chunk (a document reset inside it)
         kappa = (rng.random((w.B, (w.T + chunk - 1) // chunk)) >= 0.125).astype(np.int32)
         dev["kappa"] = torch.from_numpy(kappa).cuda()
+    # the backward runs on the CUDA cores; momentum on the two-pass tensor-core path when
+    # it applies (bf16, dk = 128, chunk 64), else on the CUDA cores
+    vkernel = "simt" if backward else ("auto" if args.kernel == "auto" else args.kernel)
     shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
                            gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
-                           gdr.BF16 if w.in_dtype == "bf16" else gdr.F32, kernel="simt")
+                           gdr.BF16 if w.in_dtype == "bf16" else gdr.F32, kernel=vkernel)
     gm = gdr.gate_mode_for(w.G, w.dk)
     ws = None
     if backward:
         nb = gdr.bwd_workspace_bytes(shape, chunk, gm)
         ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
+    on_tc2 = False
+    if not backward and vkernel != "simt":
+        tc2_shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, gdr.BF16 if w.in_dtype == "bf16"
+                                   else gdr.F32, gdr.BF16 if w.in_dtype == "bf16" else gdr.F32,
+                                   kernel="tc2")
+        on_tc2 = (w.in_dtype == "bf16" and w.dk == 128 and chunk == 64 and w.dv % 64 == 0)
+        if on_tc2:
+            nb = gdr.workspace_bytes(tc2_shape, chunk, gm)
+            ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
     in_bytes = sum(t.numel() * t.element_size() for t in dev.values() if t is not None)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if in_bytes < L2_BYTES else None
     stream = torch.cuda.current_stream()
@@ -412,7 +424,8 @@ def run_variant(args, w, chunk, rank, world, local):
         else:
             out["o"] = gdr.chunk_fwd_momentum(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
                                               mu=args.momentum, kappa=d["kappa"], chunk=chunk,
-                                              gate_mode=gm, kernel="simt", stream=stream)
+                                              gate_mode=gm, kernel="tc2" if on_tc2 else "simt",
+                                              workspace=ws, stream=stream)
 
     step_events = []
 
@@ -449,12 +462,19 @@ def run_variant(args, w, chunk, rank, world, local):
         flop *= 3
         byts = 2 * byts + 4 * w.B * w.Hv * w.T * w.dv * 2 + 4 * w.B * w.Hk * w.T * (2 * w.dk + w.G + 1)
     achieved = flop / (ms_step * 1e-3) / 1e12
-    roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-            "frac": achieved / FP32_ALU_TFLOPS, "traffic": None,
-            "peak_source": "fp32 FMA on the CUDA cores from unit counts and the max SM clock",
-            "kernel": "simt", "hbm_gbs": byts / (ms_step * 1e-3) / 1e9}
-    # kernels launched per step: backward = forward recompute, 4 zero fills, the backward
-    launches = 6 if backward else 1
+    if on_tc2:   # the forward's roofline: the same algorithmic work, the same two passes
+        peaks, peak_src = measured_peaks()
+        roof = roofline(flop, byts, ms_step, peaks)
+        roof.update(peak_source=peak_src + " (burst)", traffic=None, kernel="tc2",
+                    tflops=achieved)
+    else:
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_ALU_TFLOPS, "traffic": None,
+                "peak_source": "fp32 FMA on the CUDA cores from unit counts and the max SM clock",
+                "kernel": "simt", "hbm_gbs": byts / (ms_step * 1e-3) / 1e9}
+    # kernels launched per step: backward = forward recompute, 4 zero fills, the backward;
+    # momentum on the two-pass path: pass 1 and the state pass
+    launches = 6 if backward else (2 if on_tc2 else 1)
 
     e2e = None
     if not args.no_e2e:
@@ -507,11 +527,14 @@ def run_variant(args, w, chunk, rank, world, local):
         return 0
     what = "backward (gdr_chunk_bwd)" if backward else "forward with momentum mu=%g" % args.momentum
     line = {
-        "metric": "tokens/s of the chunkwise gated-delta %s, CUDA-core kernels" % what,
+        "metric": "tokens/s of the chunkwise gated-delta %s, %s" % (
+            what, "two-pass tensor-core path" if on_tc2 else "CUDA-core kernels"),
         "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
-        "config": dict(config_dict(w, chunk, "exact", world), which=what, kernel="simt"),
+        "dtype": "bf16" if on_tc2 else "f32",
+        "data": "synthetic (seeded numpy PCG64, distributions of the workload)",
+        "config": dict(config_dict(w, chunk, "exact", world), which=what,
+                       kernel="tc2" if on_tc2 else "simt"),
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * launches, "clocks": sampler.summary(),
     }

@@ -212,7 +212,8 @@ gdr_status gdr_chunk_fwd_momentum(const gdr_shape *shape, const void *q, const v
                                   const void *v, const float *g, const float *beta,
                                   const float *S0, int chunk, gdr_gate_mode gate_mode,
                                   gdr_inverse_mode inverse_mode, float mu, const int32_t *kappa,
-                                  void *o, float *S_final, void *stream)
+                                  void *o, float *S_final, void *workspace, size_t workspace_bytes,
+                                  void *stream)
 {
     gdr::Params p;
     gdr_status st = make_params(shape, chunk, gate_mode, inverse_mode, &p);
@@ -223,23 +224,30 @@ gdr_status gdr_chunk_fwd_momentum(const gdr_shape *shape, const void *q, const v
     const bool has_tokens = (long)p.B * p.T > 0;
     if (has_tokens && (!q || !k || !v || !g || !beta || !o))
         return GDR_ERR_ARG;
-    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_final};
+    const void *ptrs[] = {q, k, v, g, beta, S0, o, S_final, workspace};
     for (const void *ptr : ptrs)
         if (ptr != nullptr && !aligned16(ptr))
             return GDR_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(kappa) & 3u) != 0)
         return GDR_ERR_ALIGN;
-    if (shape->kernel != GDR_KERNEL_AUTO && shape->kernel != GDR_KERNEL_SIMT)
+    const gdr_kernel want = shape->kernel;
+    if (want != GDR_KERNEL_AUTO && want != GDR_KERNEL_SIMT && want != GDR_KERNEL_TC2)
         return GDR_ERR_UNSUPPORTED;
     p.momentum = 1;
     p.mu = mu;
     p.kappa = kappa;
-    if (gdr::simt_smem_bytes(p) > 227 * 1024)
+    // the two-pass tensor-core path when it applies and the workspace suffices
+    const bool tc2 = want != GDR_KERNEL_SIMT && gdr::tc2_supports(p) && workspace != nullptr &&
+                     workspace_bytes >= gdr::tc2_workspace_bytes(p);
+    if (want == GDR_KERNEL_TC2 && !tc2)
+        return gdr::tc2_supports(p) ? GDR_ERR_WORKSPACE : GDR_ERR_UNSUPPORTED;
+    if (!tc2 && gdr::simt_smem_bytes(p) > 227 * 1024)
         return GDR_ERR_UNSUPPORTED;
     if (p.B == 0)
         return GDR_OK;
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.S0 = S0; p.o = o; p.S_final = S_final;
-    return static_cast<gdr_status>(gdr::launch_simt(p, static_cast<cudaStream_t>(stream)));
+    auto s = static_cast<cudaStream_t>(stream);
+    return static_cast<gdr_status>(tc2 ? gdr::launch_tc2(p, workspace, s) : gdr::launch_simt(p, s));
 }
 
 gdr_status gdr_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_mode gate_mode,

@@ -630,7 +630,7 @@ __global__ void __launch_bounds__(32, 1) wait_probe_kernel(uint64_t limit_ns)
 static Params as_kernel_chunk(const Params &p)
 {
     Params q = p;
-    if (p.C == 128) {
+    if (p.C == 128 && !p.momentum) {   // momentum acts at the request's chunk boundaries
         q.C = CH;
         q.pair = p.neumann || p.neumann1;
     }

@@ -50,6 +50,8 @@ constexpr uint32_t T_PO = 128;     // two buffers of 64 cols: [Q; W] S
 constexpr uint32_t T_S = 256;      // fp32 state, 64 cols per 128 key rows
 // two buffers of 64 cols after the state: [L; 0] E (rows 0-63)
 __host__ __device__ constexpr uint32_t t_le(int dk) { return T_S + dk / 2; }
+// chunk-boundary momentum (dk = 128): the velocity Z, fp32, 64 cols after the LE buffers
+constexpr uint32_t T_Z = 448;
 constexpr uint32_t TMEM_COLS = 512;
 
 enum Bar { FULLX0, FULLX1, FULLY0, FULLY1, FREEX0, FREEX1, FREEY0, FREEY1, S_READY, P_FULL, E_READY,
@@ -139,7 +141,7 @@ struct SegPlan {
 inline SegPlan seg_plan(const Params &p)
 {
     const int N = prep::nchunks(p);
-    if (p.dk != KD)   // the segment-parallel form is built for dk = 128
+    if (p.dk != KD || p.momentum)   // built for dk = 128 and a state without velocity
         return SegPlan{1, N};
     const int even = p.pair ? 2 : 1;   // pairs never straddle a segment boundary
     const long nvh = (long)(p.dv / NVC) * p.Hv * p.B;
@@ -449,6 +451,9 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 for (int h = 0; h < DK / 128; ++h)
                     for (int k0 = 0; k0 < CC; k0 += 16)
                         mma_bf16(tmem + T_S + 64 * h, kt + h * dkt_hi + mstep(k0), d_e + mstep(k0), id_s, 1u);
+                if (p.momentum)   // the same update into the velocity (dk = 128)
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tmem + T_Z, kt + mstep(k0), d_e + mstep(k0), id_s, 1u);
                 mma_commit(&bars[UPD_DONE]);
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(tmem + T_LE + 64 * s, lz + kstep(k0, 128), d_eo + mstep(k0), id_po, k0 > 0);
@@ -492,6 +497,14 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tmem_st16(tq + T_S + 64 * h + cs, s0);
             tmem_st16(tq + T_S + 64 * h + cs + 16, s1);
         }
+        if (p.momentum) {   // Z_0 = 0
+            float z[16];
+#pragma unroll
+            for (int n = 0; n < 16; ++n)
+                z[n] = 0.f;
+            tmem_st16(tq + T_Z + cs, z);
+            tmem_st16(tq + T_Z + cs + 16, z);
+        }
         tmem_st_wait();
         bool ok = true;
         for (int i = 0; i < nloc; ++i) {
@@ -533,6 +546,25 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             // this thread's factors of the stage, read now: group X is refilled as soon
             // as P is done
             const float f_eb = (scalar && R >= CC) ? gt->eb[R - CC] : 1.f;
+            // chunk-boundary momentum: Z <- mu kappa_c Z, and S <- F S + that Z, so that the
+            // update, added to both, leaves Z_c = mu kappa_c Z_{c-1} + Khat^T E and
+            // S_c = F S_{c-1} + Z_c
+            float zk = 0.f;
+            float z0[16], z1[16];
+            if (p.momentum) {
+                const int c = cbeg + i;
+                zk = p.mu * (p.kappa != nullptr ? (float)p.kappa[(long)b * N + c] : 1.f);
+                tmem_ld16(tq + T_Z + cs, z0);
+                tmem_ld16(tq + T_Z + cs + 16, z1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int n = 0; n < 16; ++n) {
+                    z0[n] *= zk;
+                    z1[n] *= zk;
+                }
+                tmem_st16(tq + T_Z + cs, z0);
+                tmem_st16(tq + T_Z + cs + 16, z1);
+            }
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
                 const float F = scalar ? gt->F[0] : gt->F[R + 128 * h];
@@ -541,6 +573,12 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     s0[h][n] *= F;
                     s1[h][n] *= F;
                 }
+                if (p.momentum)   // dk = 128: h = 0 only
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) {
+                        s0[h][n] += z0[n];
+                        s1[h][n] += z1[n];
+                    }
                 tmem_st16(tq + T_S + 64 * h + cs, s0[h]);
                 tmem_st16(tq + T_S + 64 * h + cs + 16, s1[h]);
             }
@@ -762,7 +800,7 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
 inline bool supports(const Params &p)
 {
     return prep::supports(p) && (p.dk == KD || (p.dk == 256 && p.G > 1)) && p.dv % NVC == 0 &&
-           p.G <= p.dk && p.T >= 1;
+           p.G <= p.dk && p.T >= 1 && (!p.momentum || (p.dk == KD && !p.pair));
 }
 
 template <int DK, bool OB>

@@ -414,7 +414,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
 // sequences are few and long enough to run segment-parallel, and no pair correction.
 inline bool supports128(const Params &p)
 {
-    return supports(p) && p.dk == KD && p.G > 1 && p.dv % NVC2 == 0 && !p.pair;
+    return supports(p) && p.dk == KD && p.G > 1 && p.dv % NVC2 == 0 && !p.pair && !p.momentum;
 }
 
 // Segment plan of the 128-column pass (one value CTA per head and 128 columns, one

@@ -88,7 +88,7 @@ def load(path: str = LIB_PATH):
                                   vp, vp, vp, sz, vp]
     lib.gdr_chunk_fwd.restype = i
     lib.gdr_chunk_fwd_momentum.argtypes = [ctypes.POINTER(GdrShape), vp, vp, vp, vp, vp, vp, i, i,
-                                           i, ctypes.c_float, vp, vp, vp, vp]
+                                           i, ctypes.c_float, vp, vp, vp, vp, sz, vp]
     lib.gdr_chunk_fwd_momentum.restype = i
     lib.gdr_chunk_bwd.argtypes = [ctypes.POINTER(GdrShape)] + [vp] * 8 + [i, i] + [vp] * 7 + [sz, vp]
     lib.gdr_chunk_bwd.restype = i
@@ -253,12 +253,13 @@ def chunk_fwd(q, k, v, g, beta, S0=None, chunk=64, gate_mode=None, inverse="exac
 def chunk_fwd_momentum(q, k, v, g, beta, S0=None, mu=0.0, kappa=None, chunk=64, gate_mode=None,
                        inverse="exact", neumann_order=4, neumann_residual_steps=1,
                        out_dtype=None, o=None, S_final=None, want_state=True, kernel="auto",
-                       stream=None):
+                       workspace=None, stream=None):
     """chunk_fwd with chunk-boundary momentum: each chunk's state update is blended
     with a velocity Z (zero at the start), Z <- mu kappa_c Z + (S~_c - F_c S), S <-
     F_c S + Z.  kappa: int32 [B, ceil(T / chunk)] CUDA tensor of per-chunk gates on
-    the carried velocity, or None for ones.  Other arguments as chunk_fwd (no
-    workspace: the CUDA-core kernel runs it)."""
+    the carried velocity, or None for ones.  Other arguments as chunk_fwd; the
+    workspace (allocated here unless passed in) lets the two-pass tensor-core path
+    run it."""
     import torch
     B, Hk, T, dk = q.shape
     Hv, dv = v.shape[1], v.shape[3]
@@ -281,10 +282,18 @@ def chunk_fwd_momentum(q, k, v, g, beta, S0=None, mu=0.0, kappa=None, chunk=64, 
         S_final = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
     shape = make_shape(B, T, Hk, Hv, dk, dv, _dtype_code(q.dtype), _dtype_code(o.dtype),
                        neumann_order, neumann_residual_steps, kernel)
+    if workspace is None and kernel != "simt":
+        try:
+            nbytes = workspace_bytes(shape, chunk, gate_mode, inverse)
+        except GdrError:
+            nbytes = 0
+        workspace = (torch.empty(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None)
     st = load().gdr_chunk_fwd_momentum(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                        _ptr(beta), _ptr(S0), int(chunk), int(gate_mode),
                                        _INVERSES[inverse], float(mu), _ptr(kappa), _ptr(o),
-                                       _ptr(S_final), _stream_handle(stream))
+                                       _ptr(S_final), _ptr(workspace),
+                                       0 if workspace is None else workspace.numel(),
+                                       _stream_handle(stream))
     if st != OK:
         raise GdrError(st, "gdr_chunk_fwd_momentum")
     return o, S_final

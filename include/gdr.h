@@ -203,19 +203,23 @@ gdr_status gdr_bwd_workspace_bytes(const gdr_shape *shape, int chunk, gdr_gate_m
  *   kappa  [B, ceil(T / chunk)] int32 device array of per-chunk gates on the
  *          carried velocity (0 where a document reset falls in the chunk), or
  *          NULL for ones; 4-byte aligned (GDR_ERR_ALIGN otherwise)
- * Chunks are taken at exactly `chunk` tokens (no re-blocking).  Runs on the
- * CUDA-core kernel (fp32 arithmetic); shape->kernel must be AUTO or SIMT
- * (anything else: GDR_ERR_UNSUPPORTED).  The velocity takes one more dk x 32
- * fp32 tile of shared memory; a request that then does not fit also returns
- * GDR_ERR_UNSUPPORTED.  The velocity is not returned.  No workspace.
- * Asynchronous on `stream`.
+ * Chunks are taken at exactly `chunk` tokens (no re-blocking).  Kernels:
+ * TC2 (bf16 inputs, dk = 128, dv % 64 == 0, chunk 64, any gate grouping and
+ * inverse; the velocity is one more fp32 tensor-memory tile of the state pass,
+ * which then walks every sequence whole) when shape->kernel is AUTO or TC2 and
+ * the call brings gdr_workspace_bytes() of workspace for the same request;
+ * otherwise the CUDA-core kernel (fp32 arithmetic; SIMT forces it), whose
+ * velocity takes one more dk x 32 fp32 tile of shared memory (a request that
+ * then does not fit returns GDR_ERR_UNSUPPORTED).  Other kernels:
+ * GDR_ERR_UNSUPPORTED.  The velocity is not returned.  Asynchronous on `stream`.
  */
 gdr_status gdr_chunk_fwd_momentum(const gdr_shape *shape,
                                   const void *q, const void *k, const void *v,
                                   const float *g, const float *beta, const float *S0,
                                   int chunk, gdr_gate_mode gate_mode,
                                   gdr_inverse_mode inverse_mode, float mu,
-                                  const int32_t *kappa, void *o, float *S_final, void *stream);
+                                  const int32_t *kappa, void *o, float *S_final,
+                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /* Device workspace (bytes) that gdr_chunk_fwd needs for this request with the
  * kernel AUTO or shape->kernel selects when given enough: 0 for the one-pass

@@ -228,7 +228,7 @@ def test_momentum_validates(lib):
 
     def call(shape, mu=0.5, kappa=None, chunk=64, inverse=gdr.INV_EXACT):
         return f(ctypes.byref(shape), *nul, chunk, gdr.GATE_SCALAR, inverse, ctypes.c_float(mu),
-                 kappa, None, None, None)
+                 kappa, None, None, None, 0, None)
 
     sh = gdr.make_shape(2, 100, 1, 2, 64, 64, in_dtype=gdr.F32, out_dtype=gdr.F32)
     assert call(sh) == gdr.ERR_ARG                                 # tokens but no buffers
@@ -239,16 +239,21 @@ def test_momentum_validates(lib):
     assert call(empty) == gdr.OK                                   # nothing to do
     assert call(empty, kappa=ctypes.c_void_p(2)) == gdr.ERR_ALIGN  # int32 gates, 4-byte aligned
     tc = gdr.make_shape(0, 100, 1, 2, 64, 64, kernel=gdr.KERNEL_TC2)
-    assert call(tc) == gdr.ERR_UNSUPPORTED                         # CUDA-core kernel only
+    assert call(tc) == gdr.ERR_UNSUPPORTED                         # the two-pass path: dk = 128
+    tc128 = gdr.make_shape(0, 100, 1, 2, 128, 64, kernel=gdr.KERNEL_TC2)
+    assert call(tc128) == gdr.ERR_WORKSPACE                        # ... given its workspace
+    assert call(tc128, chunk=128) == gdr.ERR_UNSUPPORTED           # ... at chunk 64
+    assert call(gdr.make_shape(0, 100, 1, 2, 128, 64, kernel=gdr.KERNEL_TC), chunk=64) == \
+        gdr.ERR_UNSUPPORTED
     # the velocity tile takes shared memory: dk = 256 with per-channel gates and
     # exact chunks of 118 fits the plain kernel but not the momentum one
     wide = gdr.make_shape(0, 1000, 1, 1, 256, 256, in_dtype=gdr.F32, out_dtype=gdr.F32,
                           kernel="simt")
     assert gdr.select_kernel(wide, 118, gdr.GATE_CHANNEL) == gdr.KERNEL_SIMT
     assert f(ctypes.byref(wide), *nul, 118, gdr.GATE_CHANNEL, gdr.INV_EXACT, ctypes.c_float(0.5),
-             None, None, None, None) == gdr.ERR_UNSUPPORTED
+             None, None, None, None, 0, None) == gdr.ERR_UNSUPPORTED
     assert f(ctypes.byref(wide), *nul, 64, gdr.GATE_CHANNEL, gdr.INV_EXACT, ctypes.c_float(0.5),
-             None, None, None, None) == gdr.OK
+             None, None, None, None, 0, None) == gdr.OK
 
 
 def test_two_pass_simt_selection(lib):

@@ -1,7 +1,8 @@
 """Chunk-boundary momentum ("Systolic Linear Attention: Co-Designing Tile-Grouped
-Gated Delta Attention for TPUs", §2.3): the CUDA-core kernel through the C ABI
-(gdr_chunk_fwd_momentum) against the oracle's chunked form with momentum, on the
-same seeded inputs; kappa is a seeded 0/1 array of per-chunk gates."""
+Gated Delta Attention for TPUs", §2.3): the CUDA-core kernel and the two-pass
+tensor-core path through the C ABI (gdr_chunk_fwd_momentum) against the oracle's
+chunked form with momentum, on the same seeded inputs; kappa is a seeded 0/1
+array of per-chunk gates."""
 import numpy as np
 import pytest
 
@@ -30,6 +31,18 @@ CASES = [
     (2, dict(B=1, Hk=2, Hv=2, T=256), 64, "exact", 0.7, True),         # bf16, per-channel decay
 ]
 
+# the same on the two-pass tensor-core path (the velocity in tensor memory): scalar,
+# grouped and per-channel gates, ragged tails, S0, grouped value heads, the Neumann
+# inverses, strong decay
+TC2_CASES = [
+    (1, dict(B=2, Hk=2, Hv=4, T=320 - 13), 64, "exact", 0.9, True),
+    (1, dict(B=1, Hk=1, Hv=1, T=256), 64, "exact", 0.25, False),
+    (2, dict(B=1, Hk=2, Hv=2, T=256 - 27), 64, "exact", 0.7, True),
+    (2, dict(B=1, Hk=1, Hv=2, T=200, gate_mode=W.GATE_GROUP64), 64, "neumann", 0.5, True),
+    (2, dict(B=1, Hk=1, Hv=1, T=192), 64, "neumann1", -0.3, True),
+    (4, dict(Hk=1, Hv=1, T=640 - 5), 64, "exact", 0.25, True),
+]
+
 
 def _kappa(B, T, chunk, seed):
     rng = np.random.default_rng(seed)
@@ -49,7 +62,7 @@ def test_momentum_parity(idx, over, chunk, inverse, mu, with_kappa):
     dev = U.to_device(x, w.in_dtype)
     kd = None if kappa is None else torch.from_numpy(kappa).to("cuda")
     o, Sf = gdr.chunk_fwd_momentum(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
-                                   mu=mu, kappa=kd, chunk=chunk, inverse=inverse)
+                                   mu=mu, kappa=kd, chunk=chunk, inverse=inverse, kernel="simt")
     torch.cuda.synchronize()
     o = o.float().cpu().numpy().astype(np.float64)
     Sf = Sf.cpu().numpy().astype(np.float64)
@@ -59,6 +72,30 @@ def test_momentum_parity(idx, over, chunk, inverse, mu, with_kappa):
     eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
     print("rel err o %.3e  S_final %.3e  (tol %.0e)" % (eo, es, tol))
     assert eo <= tol and es <= tol
+
+
+@pytest.mark.parametrize("idx,over,chunk,inverse,mu,with_kappa", TC2_CASES,
+                         ids=["w%d-C%d-%s-mu%g-%s" % (c[0], c[2], c[3], c[4], "kappa" if c[5] else "ones")
+                              for c in TC2_CASES])
+def test_momentum_parity_tensor_cores(idx, over, chunk, inverse, mu, with_kappa):
+    import torch
+    from gated_delta_rule_141_b200 import gdr
+    w, x = W.workload_inputs(idx, **over)
+    B, T = x["q"].shape[0], x["q"].shape[2]
+    kappa = _kappa(B, T, chunk, 9200 + idx) if with_kappa else None
+    dev = U.to_device(x, w.in_dtype)
+    kd = None if kappa is None else torch.from_numpy(kappa).to("cuda")
+    o, Sf = gdr.chunk_fwd_momentum(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
+                                   mu=mu, kappa=kd, chunk=chunk, inverse=inverse, kernel="tc2")
+    torch.cuda.synchronize()
+    assert gdr.device_status() == gdr.OK
+    o = o.float().cpu().numpy().astype(np.float64)
+    Sf = Sf.cpu().numpy().astype(np.float64)
+    o_ref, S_ref = oracle.chunked(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], chunk=chunk,
+                                  inverse=inverse, mu=mu, kappa=kappa)
+    eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
+    print("rel err o %.3e  S_final %.3e" % (eo, es))
+    assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
 
 
 def test_momentum_zero_is_plain_forward():
@@ -78,7 +115,8 @@ def test_momentum_zero_is_plain_forward():
 
 def test_momentum_full_size_sampled():
     # the gdn_scalar_bf16 workload at full size (B=4, H=16, T=4096, dk=dv=128) with the
-    # pages' mu = 0.25 and a seeded kappa, in the launch bench.py --momentum times;
+    # pages' mu = 0.25 and a seeded kappa, in the launch bench.py --momentum times (the
+    # two-pass tensor-core path);
     # checked on a sample of sequences against the oracle
     import torch
     from gated_delta_rule_141_b200 import gdr
@@ -87,8 +125,7 @@ def test_momentum_full_size_sampled():
     kappa = _kappa(w.B, w.T, chunk, 9100)
     dev = U.to_device(x, w.in_dtype)
     o, Sf = gdr.chunk_fwd_momentum(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev["S0"],
-                                   mu=mu, kappa=torch.from_numpy(kappa).to("cuda"), chunk=chunk,
-                                   kernel="simt")
+                                   mu=mu, kappa=torch.from_numpy(kappa).to("cuda"), chunk=chunk)
     torch.cuda.synchronize()
     o = o.float().cpu().numpy().astype(np.float64)
     Sf = Sf.cpu().numpy().astype(np.float64)
