@@ -419,7 +419,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         __syncthreads();
     }
     if (!failed) {
-        gen::inverse64_inplace(A11f, Tf, tid);            // Atil11^{-1}, lower triangular
+        gen::inverse64_par(A11f, Tf, tid);                // Atil11^{-1}, lower triangular
         const int rg = tid >> 4, c0 = 4 * (tid & 15);     // rows rg + 16 i, columns c0..c0+3
         float y[4][4], z[4][4];
         gen::block_product4x4<64>(y, A21f + rg * LDM, 16 * LDM, A11f + c0, LDM, c0);
