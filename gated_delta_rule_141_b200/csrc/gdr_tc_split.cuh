@@ -548,39 +548,33 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const float f_eb = (scalar && R >= CC) ? gt->eb[R - CC] : 1.f;
             // chunk-boundary momentum: Z <- mu kappa_c Z, and S <- F S + that Z, so that the
             // update, added to both, leaves Z_c = mu kappa_c Z_{c-1} + Khat^T E and
-            // S_c = F S_{c-1} + Z_c
-            float zk = 0.f;
-            float z0[16], z1[16];
-            if (p.momentum) {
-                const int c = cbeg + i;
-                zk = p.mu * (p.kappa != nullptr ? (float)p.kappa[(long)b * N + c] : 1.f);
-                tmem_ld16(tq + T_Z + cs, z0);
-                tmem_ld16(tq + T_Z + cs + 16, z1);
-                tmem_ld_wait();
-#pragma unroll
-                for (int n = 0; n < 16; ++n) {
-                    z0[n] *= zk;
-                    z1[n] *= zk;
-                }
-                tmem_st16(tq + T_Z + cs, z0);
-                tmem_st16(tq + T_Z + cs + 16, z1);
-            }
+            // S_c = F S_{c-1} + Z_c (dk = 128: one row per thread); 16 columns at a time
+            const float zk = p.momentum ? p.mu * (p.kappa != nullptr ? (float)p.kappa[(long)b * N + cbeg + i]
+                                                                     : 1.f)
+                                        : 0.f;
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
                 const float F = scalar ? gt->F[0] : gt->F[R + 128 * h];
 #pragma unroll
-                for (int n = 0; n < 16; ++n) {
-                    s0[h][n] *= F;
-                    s1[h][n] *= F;
-                }
-                if (p.momentum)   // dk = 128: h = 0 only
+                for (int part = 0; part < 2; ++part) {
+                    float *sv = part == 0 ? s0[h] : s1[h];
+                    const uint32_t col = 64 * h + cs + 16 * part;
 #pragma unroll
-                    for (int n = 0; n < 16; ++n) {
-                        s0[h][n] += z0[n];
-                        s1[h][n] += z1[n];
+                    for (int n = 0; n < 16; ++n)
+                        sv[n] *= F;
+                    if (p.momentum) {
+                        float z[16];
+                        tmem_ld16(tq + T_Z + cs + 16 * part, z);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int n = 0; n < 16; ++n) {
+                            z[n] *= zk;
+                            sv[n] += z[n];
+                        }
+                        tmem_st16(tq + T_Z + cs + 16 * part, z);
                     }
-                tmem_st16(tq + T_S + 64 * h + cs, s0[h]);
-                tmem_st16(tq + T_S + 64 * h + cs + 16, s1[h]);
+                    tmem_st16(tq + T_S + col, *reinterpret_cast<const float(*)[16]>(sv));
+                }
             }
             if (named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[P_FULL], par, abort_flag))) {
                 ok = false;

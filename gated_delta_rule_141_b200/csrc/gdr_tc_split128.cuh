@@ -376,23 +376,31 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             tc_fence_after();
             const bool live = outputs && t < Cl;
             const long orow = (vh * T + c0 + t) * p.dv + n0;
+            // 64 columns per tensor-memory wait: the epilogue must finish within about one
+            // chunk period, or the next chunk but one waits for its buffer
 #pragma unroll
-            for (int cb = 0; cb < NVC2; cb += 16) {
-                float ov[16];
-                tmem_ld16(tq + T_R + 128 * ob + cb, ov);
+            for (int half = 0; half < NVC2; half += 64) {
+                float ov[64];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    tmem_ld16(tq + T_R + 128 * ob + half + 16 * q, *reinterpret_cast<float(*)[16]>(&ov[16 * q]));
                 tmem_ld_wait();
                 if (live) {
-                    if constexpr (OUT_BF16) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow + cb);
-                        dst[0] = make_uint4(pack_bf16(ov[0], ov[1]), pack_bf16(ov[2], ov[3]),
-                                            pack_bf16(ov[4], ov[5]), pack_bf16(ov[6], ov[7]));
-                        dst[1] = make_uint4(pack_bf16(ov[8], ov[9]), pack_bf16(ov[10], ov[11]),
-                                            pack_bf16(ov[12], ov[13]), pack_bf16(ov[14], ov[15]));
-                    } else {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + cb);
 #pragma unroll
-                        for (int n = 0; n < 4; ++n)
-                            dst[n] = make_float4(ov[4 * n], ov[4 * n + 1], ov[4 * n + 2], ov[4 * n + 3]);
+                    for (int cb = 0; cb < 64; cb += 16) {
+                        const float *v = &ov[cb];
+                        if constexpr (OUT_BF16) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow + half + cb);
+                            dst[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+                            dst[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                                                pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+                        } else {
+                            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + half + cb);
+#pragma unroll
+                            for (int n = 0; n < 4; ++n)
+                                dst[n] = make_float4(v[4 * n], v[4 * n + 1], v[4 * n + 2], v[4 * n + 3]);
+                        }
                     }
                 }
             }
