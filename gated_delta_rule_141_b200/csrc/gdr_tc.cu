@@ -617,6 +617,7 @@ __global__ void __launch_bounds__(32, 1) wait_probe_kernel(uint64_t limit_ns)
 #include "gdr_tc_prep.cuh"
 #include "gdr_tc_pair.cuh"
 #include "gdr_tc_split.cuh"
+#include "gdr_tc_ab128.cuh"
 #include "gdr_tc_split128.cuh"
 
 }  // namespace

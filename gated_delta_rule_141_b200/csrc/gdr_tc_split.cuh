@@ -106,7 +106,8 @@ __host__ __device__ inline Plan plan(bool scalar)
 //   MODE_SEG_AB: value-tile CTAs run their segment from S = 0 and store its end
 //     state Btil (no outputs); transition CTAs (grid.x past the value tiles, two
 //     per key head) run it from the identity with no values and store
-//     Atil = prod A_c, 64 of its columns each;
+//     Atil = prod A_c, 64 of its columns each (the 128-column pass runs both
+//     chains of a key head in one CTA, ab128_kernel);
 //   seg_combine_kernel: S_start(0) = S0, S_start(g + 1) = Atil_g S_start(g) + Btil_g;
 //   MODE_SEG_C: every segment runs from its S_start and writes o; the last one
 //     writes S_final.

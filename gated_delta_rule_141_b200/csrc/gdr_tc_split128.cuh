@@ -1,13 +1,15 @@
 // gdr_tc_split128.cuh -- the state pass with 128 value columns per CTA, for
 // few long sequences (the segment-parallel form).  Included by gdr_tc.cu after
-// gdr_tc_split.cuh.
+// gdr_tc_split.cuh and gdr_tc_ab128.cuh: this kernel runs the whole sequence
+// (MODE_SEQ) or each segment from its start state with outputs (MODE_SEG_C); the
+// segments' end states and transitions (MODE_SEG_AB) come from ab128_kernel.
 //
 // The same chunk recurrence as split_kernel ("Systolic Linear Attention:
 // Co-Designing Tile-Grouped Gated Delta Attention for TPUs", §2.1, §2.3 Table 2,
 // §2.4.2), E = T V - W S, S <- F S + Khat^T E, O = Qbar S + L E, arranged for
 // fewer, wider chain steps:
-//   * one CTA holds 128 value columns (a whole dv = 128 head, or a 128-column
-//     block of the identity for a transition), so every product has N = 128: an
+//   * one CTA holds 128 value columns (a whole dv = 128 head), so every product
+//     has N = 128: an
 //     N = 64 product reads as many operand bytes from shared memory per output
 //     column as it computes, N = 128 half as many;
 //   * U, P, E and O share one fp32 tensor-memory buffer R (two, alternating by
@@ -77,19 +79,15 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     uint8_t *base = smem_raw + (base_u32 - smem_u32(smem_raw));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nvh = args.nvt * p.Hv;   // value-tile CTAs per batch entry
-    const bool trans = args.mode == MODE_SEG_AB && (int)blockIdx.x >= nvh;
-    const int xi = trans ? (int)blockIdx.x - nvh : (int)blockIdx.x;
-    const int nt = trans ? 0 : xi % args.nvt;
-    const int hv = trans ? 0 : xi / args.nvt;
+    const int nt = (int)blockIdx.x % args.nvt;
+    const int hv = (int)blockIdx.x / args.nvt;
     const int b = blockIdx.y;
-    const int hk = trans ? xi : hv / p.R;
+    const int hk = hv / p.R;
     const int n0 = nt * NVC2;
     const long kh = (long)b * p.Hk + hk;
     const long vh = (long)b * p.Hv + hv;
     const int T = p.T;
     const int N = args.nchunks;
-    const bool outputs = args.mode != MODE_SEG_AB;
     const int seg = blockIdx.z;
     const int cbeg = seg * args.seg_len;
     const int nloc = min(args.seg_len, N - cbeg);
@@ -140,13 +138,11 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             }
             if (lane == 0) {
                 uint64_t *full = &bars[FULLX0 + s];
-                mbar_arrive_expect_tx(full, 2u * prep::IMG + (outputs ? 2u * prep::IMG : 0u) +
-                                                (trans ? 0u : prep::IMG + CC * NVC2 * 2) + KD * 4);
+                mbar_arrive_expect_tx(full, 5u * prep::IMG + CC * NVC2 * 2 + KD * 4);
                 for (int kb = 0; kb < KD / 64; ++kb) {
                     uint8_t *blk = qwk + kb * 192 * 128;
                     bulk_load(blk + 64 * 128, fac + prep::REC_W + kb * prep::IMG, prep::IMG, full);
-                    if (outputs)
-                        bulk_load(blk, fac + prep::EXT_QB + kb * prep::IMG, prep::IMG, full);
+                    bulk_load(blk, fac + prep::EXT_QB + kb * prep::IMG, prep::IMG, full);
                 }
                 bulk_load(fgate(s), fac + prep::EXT_F, KD * 4, full);
             }
@@ -166,18 +162,16 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
             uint8_t *qwk = base + Ly.qwk[s];
             uint8_t *lzt = base + Ly.lzt[s];
-            if (!trans) {
-                if (i >= 2) {
-                    const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
-                    if (__any_sync(0xffffffffu, !ok))
-                        break;
-                }
-                if (lane == 0) {
-                    uint64_t *full = &bars[FULLX0 + s];
-                    bulk_load(lzt + 128 * 128, fac, prep::IMG, full);   // T under the zeros
-                    tma_load_3d(base + Ly.v[s], &tm_v, full, n0, (int)c0, (int)vh);
-                    tma_load_3d(base + Ly.v[s] + 64 * 128, &tm_v, full, n0 + 64, (int)c0, (int)vh);
-                }
+            if (i >= 2) {
+                const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
+                if (__any_sync(0xffffffffu, !ok))
+                    break;
+            }
+            if (lane == 0) {
+                uint64_t *full = &bars[FULLX0 + s];
+                bulk_load(lzt + 128 * 128, fac, prep::IMG, full);   // T under the zeros
+                tma_load_3d(base + Ly.v[s], &tm_v, full, n0, (int)c0, (int)vh);
+                tma_load_3d(base + Ly.v[s] + 64 * 128, &tm_v, full, n0 + 64, (int)c0, (int)vh);
             }
             if (i >= 2) {
                 const bool ok = wait_or_abort(&bars[FREEY0 + s], ((i >> 1) - 1) & 1, abort_flag);
@@ -186,12 +180,11 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             }
             if (lane == 0) {
                 uint64_t *full = &bars[FULLY0 + s];
-                mbar_arrive_expect_tx(full, (outputs ? 3u : 2u) * prep::IMG);
+                mbar_arrive_expect_tx(full, 3u * prep::IMG);
                 for (int kb = 0; kb < KD / 64; ++kb)
                     bulk_load(qwk + kb * 192 * 128 + 128 * 128, fac + prep::EXT_KH + kb * prep::IMG,
                               prep::IMG, full);
-                if (outputs)
-                    bulk_load(lzt, fac + prep::IMG, prep::IMG, full);   // L above the zeros
+                bulk_load(lzt, fac + prep::IMG, prep::IMG, full);   // L above the zeros
             }
             army[s] += 1;
         }
@@ -223,17 +216,16 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 if (i >= 2 && !(ok = wait_or_abort(&bars[OFREE0 + s], ((i >> 1) - 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
-                if (!trans)   // U = [0; T] V into rows 64-127 of R(s), zeros into 0-63
-                    for (int k0 = 0; k0 < CC; k0 += 16)
-                        mma_bf16(rb, desc_kmajor(lzt + 64 * 128, 128, 0, k0),
-                                 desc_mnmajor(base_u32 + Ly.v[s], 64, k0, 0), id128, k0 > 0);
+                // U = [0; T] V into rows 64-127 of R(s), zeros into 0-63
+                for (int k0 = 0; k0 < CC; k0 += 16)
+                    mma_bf16(rb, desc_kmajor(lzt + 64 * 128, 128, 0, k0),
+                             desc_mnmajor(base_u32 + Ly.v[s], 64, k0, 0), id128, k0 > 0);
                 if (!(ok = wait_or_abort(&bars[S_READY], par, abort_flag)))
                     break;
                 tc_fence_after();
                 // [Qbar; -W] S: Qbar S into rows 0-63, U - W S = E into rows 64-127
                 for (int k0 = 0; k0 < KD; k0 += 16)
-                    mma_bf16(rb, desc_kmajor(qwk, 192, 0, 0) + kstep(k0, 192), d_s + mstep(k0), id128,
-                             (!trans || k0 > 0) ? 1u : 0u);
+                    mma_bf16(rb, desc_kmajor(qwk, 192, 0, 0) + kstep(k0, 192), d_s + mstep(k0), id128, 1u);
                 mma_commit(&bars[P_FULL]);
                 mma_commit(&bars[FREEX0 + s]);
                 if (!(ok = wait_or_abort(&bars[E_READY], par, abort_flag)))
@@ -262,7 +254,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             float sv[64];
 #pragma unroll
             for (int n = 0; n < 64; ++n)
-                sv[n] = (trans && R == cs + n) ? 1.f : 0.f;
+                sv[n] = 0.f;
             const float *src = nullptr;
             if (args.mode == MODE_SEQ && p.S0 != nullptr)
                 src = p.S0 + (vh * KD + R) * p.dv + n0 + cs;
@@ -347,10 +339,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[UPD_DONE], (nloc - 1) & 1, abort_flag)))
             ok = false;
         float *dst = nullptr;
-        if (args.mode == MODE_SEG_AB)
-            dst = trans ? args.seg_trans + (((size_t)kh * args.nseg + seg) * KD + R) * KD + cs
-                        : args.seg_end + (((size_t)vh * args.nseg + seg) * KD + R) * p.dv + n0 + cs;
-        else if (p.S_final != nullptr && seg == args.nseg - 1)
+        if (p.S_final != nullptr && seg == args.nseg - 1)
             dst = p.S_final + (vh * KD + R) * p.dv + n0 + cs;
         if (ok && dst != nullptr) {
             tc_fence_after();
@@ -374,7 +363,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             if (named_vote_or(NB_EPI, N_EPI, !wait_or_abort(&bars[OUT0 + ob], (i >> 1) & 1, abort_flag)))
                 break;
             tc_fence_after();
-            const bool live = outputs && t < Cl;
+            const bool live = t < Cl;
             const long orow = (vh * T + c0 + t) * p.dv + n0;
             // 64 columns per tensor-memory wait: the epilogue must finish within about one
             // chunk period, or the next chunk but one waits for its buffer
@@ -425,21 +414,21 @@ inline bool supports128(const Params &p)
     return supports(p) && p.dk == KD && p.G > 1 && p.dv % NVC2 == 0 && !p.pair && !p.momentum;
 }
 
-// Segment plan of the 128-column pass (one value CTA per head and 128 columns, one
-// transition CTA per key head); its chain step does twice the columns of the
-// 64-column pass's for about 1.3 times its time.
+// Segment plan of the 128-column pass (one CTA per head and 128 value columns in
+// both launches, the transitions riding with the first value tile of each key
+// head); its chain step does twice the columns of the 64-column pass's for about
+// 1.3 times its time.
 inline SegPlan seg_plan128(const Params &p)
 {
     const int N = prep::nchunks(p);
     const long nvh = (long)(p.dv / NVC2) * p.Hv * p.B;
-    const long ntr = (long)p.Hk * p.B;
     auto waves = [](long ctas) { return (ctas + kSMs - 1) / kSMs; };
     SegPlan best{1, N};
     long best_cost = waves(nvh) * (long)N;
     for (int ns = 2; ns <= N / kMinSegChunks; ++ns) {
         const int L = (N + ns - 1) / ns;
         const int nsg = (N + L - 1) / L;
-        const long cost = (waves((nvh + ntr) * nsg) + waves(nvh * nsg)) * (long)L + nsg;
+        const long cost = 2 * waves(nvh * nsg) * (long)L + nsg;
         if (cost < best_cost) {
             best_cost = cost;
             best = SegPlan{nsg, L};
@@ -461,9 +450,9 @@ inline bool use128(const Params &p)
         return false;
     auto waves = [](long ctas) { return (ctas + kSMs - 1) / kSMs; };
     const long nvh = (long)(p.dv / NVC) * p.Hv * p.B, ntr = (long)(KD / NVC) * p.Hk * p.B;
-    const long nvh2 = (long)(p.dv / NVC2) * p.Hv * p.B, ntr2 = (long)p.Hk * p.B;
+    const long nvh2 = (long)(p.dv / NVC2) * p.Hv * p.B;
     const long ca = (waves((nvh + ntr) * a.nseg) + waves(nvh * a.nseg)) * (long)a.seg_len * 10;
-    const long cw = (waves((nvh2 + ntr2) * w.nseg) + waves(nvh2 * w.nseg)) * (long)w.seg_len * 13;
+    const long cw = 2 * waves(nvh2 * w.nseg) * (long)w.seg_len * 13;
     return cw < ca;
 }
 
@@ -504,8 +493,12 @@ int launch128(const Params &p, const void *factors, cudaStream_t stream)
     if (cudaFuncSetAttribute(seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)CMB_SMEM) != cudaSuccess)
         return 6;
+    const ab::Plan La = ab::plan();
+    if (cudaFuncSetAttribute(ab::ab128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)La.total) != cudaSuccess)
+        return 6;
     a.mode = MODE_SEG_AB;
-    kern<<<dim3(a.nvt * p.Hv + p.Hk, p.B, sp.nseg), NTHR, Ly.total, stream>>>(mv, a);
+    ab::ab128_kernel<<<dim3(a.nvt * p.Hv, p.B, sp.nseg), ab::NTHR, La.total, stream>>>(mv, a);
     seg_combine_kernel<<<dim3((p.dv / CMB_COLS) * p.Hv, p.B), 256, CMB_SMEM, stream>>>(a);
     a.mode = MODE_SEG_C;
     kern<<<dim3(a.nvt * p.Hv, p.B, sp.nseg), NTHR, Ly.total, stream>>>(mv, a);

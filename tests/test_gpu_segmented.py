@@ -54,10 +54,12 @@ def test_segmented_state_pass(idx, over):
     assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
 
 
-# The 128-column state pass (forced): one value CTA per head and one transition CTA
-# per key head per segment, U / P / E / O sharing one tensor-memory buffer.
+# The 128-column state pass (forced): one CTA per head and 128 value columns per
+# segment, the first value tile of each key head also carrying its transition;
+# U / P / E / O sharing one tensor-memory buffer.
 WIDE = [
     (4, dict(Hk=1, Hv=1, T=64 * 60 + 17)),        # strong per-channel decay, S0
+    (4, dict(B=2, Hk=2, Hv=4, T=64 * 64 + 3)),    # two batch entries, two value heads per key head
     (2, dict(B=1, Hk=1, Hv=2, T=64 * 52 - 9)),    # two value heads, one transition
     (2, dict(B=1, Hk=1, Hv=1, T=64 * 48, dv=256, gate_mode=W.GATE_GROUP64)),   # two value tiles
 ]
