@@ -79,7 +79,12 @@ struct Plan {
     uint32_t QK, RA, KC, Mf, Tf, NB, XB, RB, TB, lam, beta, piv, bar, misc, total, tmem_cols, tn;
 };
 
-__host__ __device__ inline Plan plan(int dk, int G, bool neumann)
+// Rows of Lambda that the register-resident form (rl) keeps in shared memory.
+enum LamRow { LR_0 = 0, LR_P = 1, LR_C = 2, LR_16 = 3, LR_48 = 4, LR_N = 5 };
+
+// rl: per-channel Lambda lives in registers (dk = 128, grouped / per-channel gates,
+// extended records), so the 32 KB Lambda tile is gone and three CTAs fit on an SM.
+__host__ __device__ inline Plan plan(int dk, int G, bool neumann, bool rl = false)
 {
     Plan s;
     uint32_t o = 0;
@@ -101,9 +106,15 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
         s.Mf = take(CC * LDM * 4 + 32 * 36 * 4);
     }
     s.Tf = s.Mf + CC * LDM * 4;
-    s.lam = take(CC * G * 4 + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
-    s.beta = s.lam + CC * G * 4;
-    if (neumann) {   // Neumann operands: in the Lambda tile (dead by the inverse) when it is large enough
+    const uint32_t lam_bytes = rl ? LR_N * dk * 4 : CC * G * 4;
+    s.lam = take(lam_bytes + CC * 4 + NROUND * 4 + 64);   // Lambda, beta, flags, barriers
+    s.beta = s.lam + lam_bytes;
+    if (neumann && rl) {
+        // the q rows of QK (dead after the Grams) and the end of the inverse's scratch
+        s.NB = s.QK;
+        s.XB = s.QK + 2 * 8192;
+        s.RB = s.Mf + ((CC * LDM * 4 + 32 * 36 * 4 + 1023u) & ~1023u);
+    } else if (neumann) {   // in the Lambda tile (dead by the inverse) when it is large enough
         s.NB = CC * G * 4 >= 3 * 8192 ? s.lam : take(3 * 8192);
         s.XB = s.NB + 8192;
         s.RB = s.NB + 16384;
@@ -114,8 +125,10 @@ __host__ __device__ inline Plan plan(int dk, int G, bool neumann)
     s.bar = (s.beta + CC * 4 + NROUND * 4 + 7u) & ~7u;
     s.misc = s.bar + 24;
     s.total = o + 1024;
-    s.tmem_cols = (G > 1 || dk > 128) ? 256u : 128u;   // W (M = 64, N = dk) needs dk columns
-    s.tn = G > 1 ? 192u : 64u;                    // Neumann products
+    // W (M = 64, N = dk) needs dk columns; three CTAs a SM (rl) share the 512 columns, so
+    // their Neumann products reuse the Grams' columns 64-127 (read out by then)
+    s.tmem_cols = ((G > 1 && !rl) || dk > 128) ? 256u : 128u;
+    s.tn = (G > 1 && !rl) ? 192u : 64u;           // Neumann products
     return s;
 }
 
@@ -162,18 +175,25 @@ __device__ __forceinline__ void lam8(const float *lam, int G, int wsh, int t, in
 }
 
 // SCALAR: the scalar-gate instantiation (no pivoting machinery, four CTAs per SM);
-// otherwise grouped / per-channel gates (two CTAs per SM: the gate tile is larger).
-template <int DK, bool SCALAR>
-__global__ void __launch_bounds__(NT, SCALAR ? 4 : 2)
+// otherwise grouped / per-channel gates: RL keeps Lambda in registers (dk = 128,
+// extended records; three CTAs per SM), else in a shared-memory tile (two per SM).
+//
+// RL: thread (tb, cg) = (tid / 16, tid % 16) owns tokens 4 tb .. 4 tb + 3 at the
+// eight channels 8 cg .. 8 cg + 7 in every elementwise sweep; its Lambda values are
+// a blocked scan (within its four tokens, then over the 16 token blocks), and the
+// rows every thread needs (0, 16, 32, 48, 63) go to shared memory.
+template <int DK, bool SCALAR, bool RL = false>
+__global__ void __launch_bounds__(NT, SCALAR ? 4 : RL ? 3 : 2)
 prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const PrepArgs a)
 {
     using namespace ptx;
+    static_assert(!RL || (DK == 128 && !SCALAR), "register-resident Lambda: dk = 128, gated by group");
     extern __shared__ uint8_t smem_raw[];
     const Params &p = a.p;
     const int G = SCALAR ? 1 : p.G;
     const bool neu = p.neumann != 0;
-    const Plan Ly = plan(DK, G, neu);
+    const Plan Ly = plan(DK, G, neu, RL);
     const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t pad = base_u32 - smem_u32(smem_raw);
     uint8_t *base = smem_raw + pad;
@@ -193,14 +213,24 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int Cl = (int)min((long)CC, T - c0);
     const int wsh = __ffs(DK / G) - 1;      // channels per decay group = 2^wsh
     const uint32_t QK = base_u32 + Ly.QK, RA = base_u32 + Ly.RA, KC = base_u32 + Ly.KC;
+    // L and W leave as whole images by bulk copies from shared memory (a thread holds
+    // one row of them, so direct stores would each touch 16 or 32 lines): L is staged
+    // in the q rows (scalar gate; read before T lands there) or in the second half of
+    // the Grams' column tile, W in the inverse's scratch (dk = 128, read back before)
+    // or the column tile (dk = 256, after L has left).
+    const uint32_t Ls = SCALAR ? QK : KC + 8192;
+    const uint32_t Ws = DK == 128 ? base_u32 + Ly.Mf : KC;
+    constexpr bool W_STAGE = !(SCALAR && DK > 128);
     uint8_t *img_T = a.out + (size_t)(kh * a.nchunks + c) * a.rec_bytes;
     uint8_t *img_L = img_T + IMG;
 
     // The log-gates of a grouped / per-channel chunk are one contiguous run of Cl x G
-    // floats: one bulk copy when it is 16-byte aligned, else plain loads.
+    // floats: one bulk copy when it is 16-byte aligned (RL: into the Gram tiles, free
+    // until the scan has read it), else plain loads.
     const float *g_src = p.g + (kh * T + c0) * G;
     const uint32_t g_bytes = (uint32_t)(Cl * G * 4);
     const bool g_bulk = !SCALAR && (g_bytes & 15u) == 0 && (reinterpret_cast<uintptr_t>(g_src) & 15u) == 0;
+    float *g_tile = RL ? reinterpret_cast<float *>(base + Ly.RA) : lam;
     // beta of a full chunk: one 256-byte bulk copy on the q, k barrier when aligned
     const float *b_src = p.beta + kh * T + c0;
     const bool b_bulk = Cl == CC && (reinterpret_cast<uintptr_t>(b_src) & 15u) == 0;
@@ -211,7 +241,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         fence_barrier_init();
         if (g_bulk) {
             mbar_arrive_expect_tx(&bars[2], g_bytes);
-            bulk_load(lam, g_src, g_bytes, &bars[2]);
+            bulk_load(g_tile, g_src, g_bytes, &bars[2]);
         }
         mbar_arrive_expect_tx(&bars[0], 2u * CC * DK * 2u + (b_bulk ? CC * 4u : 0u));
         if (b_bulk)
@@ -229,7 +259,34 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (!b_bulk)
         for (int t = tid; t < CC; t += NT)
             sbeta[t] = t < Cl ? b_src[t] : 0.f;
-    if (g_bulk) {
+    // RL: this thread's log-gates (zero past T) into registers, from the bulk-copied
+    // tile or straight from global memory
+    const int cg = tid & 15, tb = tid >> 4, i0r = 8 * cg;
+    float lv[RL ? 4 : 1][8];
+    auto load_gates = [&](const float *src, bool vec) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int t = 4 * tb + k;
+            if (t >= Cl) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    lv[k][e] = 0.f;
+            } else if (vec) {
+                const float4 x0 = *reinterpret_cast<const float4 *>(src + t * G + i0r);
+                const float4 x1 = *reinterpret_cast<const float4 *>(src + t * G + i0r + 4);
+                lv[k][0] = x0.x; lv[k][1] = x0.y; lv[k][2] = x0.z; lv[k][3] = x0.w;
+                lv[k][4] = x1.x; lv[k][5] = x1.y; lv[k][6] = x1.z; lv[k][7] = x1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    lv[k][e] = src[t * G + ((i0r + e) >> wsh)];
+            }
+        }
+    };
+    if constexpr (RL) {
+        if (!g_bulk)
+            load_gates(g_src, wsh == 0 && (reinterpret_cast<uintptr_t>(p.g) & 15u) == 0);
+    } else if (g_bulk) {
         for (int u = Cl * G + tid; u < CC * G; u += NT)   // rows past T (not copied)
             lam[u] = 0.f;
     } else {
@@ -256,7 +313,53 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         failed = wait_bar(2, 0);
 
     // ---- Lambda = cumsum over the chunk per decay group
-    if (G <= 8) {
+    if constexpr (RL) {
+        if (g_bulk) {
+            load_gates(g_tile, wsh == 0);
+            __syncthreads();   // the gate tile has been read: its space takes the block totals
+        }
+        // blocked scan: the thread's four tokens, then the 16 token blocks in order
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int k = 1; k < 4; ++k)
+                lv[k][e] += lv[k - 1][e];
+        float *tot = reinterpret_cast<float *>(base + Ly.RA);   // [16][DK]: free until the Grams
+        *reinterpret_cast<float4 *>(tot + tb * DK + i0r) = make_float4(lv[3][0], lv[3][1], lv[3][2], lv[3][3]);
+        *reinterpret_cast<float4 *>(tot + tb * DK + i0r + 4) = make_float4(lv[3][4], lv[3][5], lv[3][6], lv[3][7]);
+        __syncthreads();
+        if (tid < DK) {   // exclusive prefix over the token blocks, one channel a thread
+            float run = 0.f;
+            for (int j = 0; j < 16; ++j) {
+                const float x = tot[j * DK + tid];
+                tot[j * DK + tid] = run;
+                run += x;
+            }
+        }
+        __syncthreads();
+        {
+            const float4 o0 = *reinterpret_cast<const float4 *>(tot + tb * DK + i0r);
+            const float4 o1 = *reinterpret_cast<const float4 *>(tot + tb * DK + i0r + 4);
+            const float off[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    lv[k][e] += off[e];
+        }
+        // the rows every thread reads: 0, 16, 32 (the pivot), 48 and 63 (the chunk's end)
+        auto put = [&](int row, int k) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                lam[row * DK + i0r + e] = lv[k][e];
+        };
+        if (tb == 0) put(LR_0, 0);
+        if (tb == 4) put(LR_16, 0);
+        if (tb == 8) put(LR_P, 0);
+        if (tb == 12) put(LR_48, 0);
+        if (tb == 15) put(LR_C, 3);
+        __syncthreads();
+    } else if (G <= 8) {
         if (warp < G) {   // lane l holds rows 2l, 2l+1
             const float v0 = lam[(2 * lane) * G + warp], v1 = lam[(2 * lane + 1) * G + warp];
             float s = v0 + v1;
@@ -291,16 +394,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // pivoted row blocks
     constexpr int PV = CC / 2;
     float *piv = reinterpret_cast<float *>(base + Ly.piv);   // e^{Lambda_p}, e^{Lambda_C - Lambda_p}
+    // Lambda at the pivot and at the chunk's end, channel i
+    auto lam_p = [&](int i) { return RL ? lam[LR_P * DK + i] : lam[PV * G + (i >> wsh)]; };
+    auto lam_c = [&](int i) { return RL ? lam[LR_C * DK + i] : lam[(CC - 1) * G + (i >> wsh)]; };
     bool wide = false;
-    if (!SCALAR)
+    if (RL) {
+        if (tid < DK) {
+            const float l0 = lam[LR_0 * DK + tid], lp = lam_p(tid), lc = lam_c(tid);
+            wide = (l0 - lp) > kGuard || (lp - lc) > kGuard;
+        }
+    } else if (!SCALAR) {
         for (int gi = tid; gi < G; gi += NT) {
             const float l0 = lam[gi], lp = lam[PV * G + gi], lc = lam[(CC - 1) * G + gi];
             wide |= (l0 - lp) > kGuard || (lp - lc) > kGuard;
         }
+    }
     wide = __syncthreads_or(wide ? 1 : 0) != 0;
     if (!SCALAR && !wide) {
         for (int i = tid; i < DK; i += NT) {
-            const float lp = lam[PV * G + (i >> wsh)], lc = lam[(CC - 1) * G + (i >> wsh)];
+            const float lp = lam_p(i), lc = lam_c(i);
             piv[i] = __expf(lp);
             piv[DK + i] = __expf(lc - lp);
         }
@@ -312,7 +424,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (!failed && ext) {
         float *fo = reinterpret_cast<float *>(img_T + ext_f(DK));
         for (int i = tid; i < DK; i += NT)
-            fo[i] = __expf(lam[(CC - 1) * G + (i >> wsh)]);   // F = e^{Lambda_C}
+            fo[i] = __expf(lam_c(i));   // F = e^{Lambda_C}
     }
     // Scalar gate: e^{Lambda_t - Lambda_j} = e^{Lambda_t - Lambda_p} e^{Lambda_p - Lambda_j} with
     // the pivot p in the middle of the chunk; while the chunk's decay span is within
@@ -335,29 +447,33 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (tid < 4)
             reinterpret_cast<float *>(img_T + SC_F)[tid] = __expf(lc);
     }
-    if (!failed && ext && wide) {
-        // ---- decayed operands for the state pass, straight from the raw tiles
+    // decayed operands for the state pass straight from the raw tiles (wide chunks):
+    // Qbar = q e^{Lambda_t}, Khat = k e^{Lambda_C - Lambda_t} at row t, channels i0 .. i0 + 7
+    auto raw_operands = [&](int t, int i0, const float *lt, const float *lc) {
+        float qv[8], kv[8], qb[8], kh8[8];
+        ld_tile8(QK, 128, t, i0, qv);
+        ld_tile8(QK, 128, 64 + t, i0, kv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            qb[e] = qv[e] * __expf(lt[e]);
+            kh8[e] = kv[e] * __expf(lc[e] - lt[e]);
+        }
+        const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
+        *reinterpret_cast<uint4 *>(img_T + ext_qb(DK) + off) =
+            make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]), pack_bf16(qb[4], qb[5]),
+                       pack_bf16(qb[6], qb[7]));
+        *reinterpret_cast<uint4 *>(img_T + ext_kh(DK) + off) =
+            make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
+                       pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
+    };
+    if (!RL && !failed && ext && wide)   // (RL: after the rounds, whose fp32 rows may need the area)
         for (int u = tid; u < CC * (DK / 8); u += NT) {
             const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-            float qv[8], kv[8], qb[8], kh8[8], lt[8], lc[8];
-            ld_tile8(QK, 128, t, i0, qv);
-            ld_tile8(QK, 128, 64 + t, i0, kv);
+            float lt[8], lc[8];
             lam8(lam, G, wsh, t, i0, lt);
             lam8(lam, G, wsh, CC - 1, i0, lc);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                qb[e] = qv[e] * __expf(lt[e]);
-                kh8[e] = kv[e] * __expf(lc[e] - lt[e]);
-            }
-            const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
-            *reinterpret_cast<uint4 *>(img_T + ext_qb(DK) + off) =
-                make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]), pack_bf16(qb[4], qb[5]),
-                           pack_bf16(qb[6], qb[7]));
-            *reinterpret_cast<uint4 *>(img_T + ext_kh(DK) + off) =
-                make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
-                           pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
+            raw_operands(t, i0, lt, lc);
         }
-    }
 
     if (!failed && !wide) {
         if (!SCALAR) {
@@ -366,13 +482,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             //      pass's operands from the same two exponentials, Qbar = q a e^{Lambda_p} and
             //      Khat = k b e^{Lambda_C - Lambda_p}; the k rows keep k a (Kbar = k a e^{Lambda_p}
             //      is W's operand, its per-channel factor applied on the way out of TMEM)
-            for (int u = tid; u < CC * (DK / 8); u += NT) {
-                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float qv[8], kv[8], kc[8], kh8[8], qb[8], lt[8], lp[8];
+            auto item = [&](int t, int i0, const float *lt, const float *lp) {
+                float qv[8], kv[8], kc[8], kh8[8], qb[8];
                 ld_tile8(QK, 128, t, i0, qv);
                 ld_tile8(QK, 128, 64 + t, i0, kv);
-                lam8(lam, G, wsh, t, i0, lt);
-                lam8(lam, G, wsh, PV, i0, lp);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float a = __expf(lt[e] - lp[e]), b = __expf(lp[e] - lt[e]);
@@ -393,6 +506,23 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     *reinterpret_cast<uint4 *>(img_T + ext_kh(DK) + off) =
                         make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
                                    pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
+                }
+            };
+            if constexpr (RL) {
+                float lp[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    lp[e] = lam[LR_P * DK + i0r + e];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    item(4 * tb + k, i0r, lv[k], lp);
+            } else {
+                for (int u = tid; u < CC * (DK / 8); u += NT) {
+                    const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                    float lt[8], lp[8];
+                    lam8(lam, G, wsh, t, i0, lt);
+                    lam8(lam, G, wsh, PV, i0, lp);
+                    item(t, i0, lt, lp);
                 }
             }
             fence_proxy_async_smem();
@@ -419,7 +549,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tmem_ld_wait();
             const bool qrow = R < CC;
             const int t = qrow ? R : R - CC;
-            const float lt = lam[t * G];
+            const float lt = SCALAR ? lam[t] : 0.f;   // (scalar gate: G = 1)
             // two halves of 16 columns (fewer live registers)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -438,8 +568,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     out[u] = v;
                 }
                 if (qrow) {
-                    st_img8(img_L, t, jh, &out[0]);
-                    st_img8(img_L, t, jh + 8, &out[8]);
+                    st_tile8(Ls, 64, t, jh, &out[0]);
+                    st_tile8(Ls, 64, t, jh + 8, &out[8]);
                 } else {
                     // Mf holds the k rows' products in fp32
 #pragma unroll
@@ -457,14 +587,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int p0 = 32 * r, pv = p0 + 16, n_r = 32 * (r + 1);
             bool clamp = false;
             // rows 0-31 of RA: q of the block, 32-63: k of the block; the q and k rows of
-            // a token share their factors
-            for (int u = tid; u < (32 + n_r) * (DK / 8); u += NT) {
-                const int row = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float la[8], lb[8], f8[8];
-                const bool rowop = row < 32;
-                const int t = p0 + row, jj = row - 32;
-                lam8(lam, G, wsh, rowop ? t : pv, i0, la);
-                lam8(lam, G, wsh, rowop ? pv : jj, i0, lb);
+            // a token share their factors.  Row operand of token t: factor e^{la - lb}
+            // with (la, lb) = (Lambda_t, Lambda_p); column operand of token jj:
+            // (Lambda_p, Lambda_jj).
+            auto operand = [&](bool rowop, int t, int i0, const float *la, const float *lb) {
+                float f8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     float x = la[e] - lb[e];
@@ -483,15 +610,39 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         q8[e] *= f8[e];
                         k8[e] *= f8[e];
                     }
-                    st_tile8(RA, 64, row, i0, q8);
-                    st_tile8(RA, 64, 32 + row, i0, k8);
+                    st_tile8(RA, 64, t - p0, i0, q8);
+                    st_tile8(RA, 64, 32 + t - p0, i0, k8);
                 } else {
                     float k8[8];
-                    ld_tile8(QK, 128, 64 + jj, i0, k8);
+                    ld_tile8(QK, 128, 64 + t, i0, k8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         k8[e] *= f8[e];
-                    st_tile8(KC, 64, jj, i0, k8);
+                    st_tile8(KC, 64, t, i0, k8);
+                }
+            };
+            if constexpr (RL) {
+                float lp[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    lp[e] = lam[(r == 0 ? LR_16 : LR_48) * DK + i0r + e];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int t = 4 * tb + k;
+                    if (t >= p0 && t < p0 + 32)
+                        operand(true, t, i0r, lv[k], lp);
+                    if (t < n_r)
+                        operand(false, t, i0r, lp, lv[k]);
+                }
+            } else {
+                for (int u = tid; u < (32 + n_r) * (DK / 8); u += NT) {
+                    const int row = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                    float la[8], lb[8];
+                    const bool rowop = row < 32;
+                    const int t = rowop ? p0 + row : row - 32;
+                    lam8(lam, G, wsh, rowop ? t : pv, i0, la);
+                    lam8(lam, G, wsh, rowop ? pv : t, i0, lb);
+                    operand(rowop, t, i0, la, lb);
                 }
             }
             if (clamp)
@@ -532,8 +683,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                         : ((jj < t) ? (a.pair ? d[e] : sbeta[jj] * d[e]) : 0.f);
                         }
                         if (qrow) {
-                            st_img8(img_L, t, c0 + cb, &v[0]);
-                            st_img8(img_L, t, c0 + cb + 8, &v[8]);
+                            st_tile8(Ls, 64, t, c0 + cb, &v[0]);
+                            st_tile8(Ls, 64, t, c0 + cb + 8, &v[8]);
                         } else {
 #pragma unroll
                             for (int e = 0; e < 16; e += 4)
@@ -546,8 +697,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                     const int zc = 32 + 16 * half;
                     if (qrow) {
-                        st_img8(img_L, t, zc, z);
-                        st_img8(img_L, t, zc + 8, z);
+                        st_tile8(Ls, 64, t, zc, z);
+                        st_tile8(Ls, 64, t, zc + 8, z);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; e += 4)
@@ -557,15 +708,27 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             __syncthreads();
             // blocks whose decay span overran the guard: exact fp32 rows from the raw tiles
+            // (RL: Lambda is spilled to the record's Qbar / Khat area first, rewritten below)
+            const float *lsc = reinterpret_cast<const float *>(img_T + ext_qb(DK));
+            if (RL && (flag[0] || flag[1])) {
+                float *lw = reinterpret_cast<float *>(img_T + ext_qb(DK));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float *dst = lw + (4 * tb + k) * DK + i0r;
+                    *reinterpret_cast<float4 *>(dst) = make_float4(lv[k][0], lv[k][1], lv[k][2], lv[k][3]);
+                    *reinterpret_cast<float4 *>(dst + 4) = make_float4(lv[k][4], lv[k][5], lv[k][6], lv[k][7]);
+                }
+                __syncthreads();
+            }
             for (int r = 0; r < 2; ++r) {
                 if (!flag[r])
                     continue;
                 for (int u = tid; u < 32 * 8; u += NT) {
                     const int t = 32 * r + (u >> 3), j0 = (u & 7) * 8;
-                    float lv[8], mv[8];
+                    float lv2[8], mv[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        lv[e] = mv[e] = 0.f;
+                        lv2[e] = mv[e] = 0.f;
                     for (int i0 = 0; i0 < DK; i0 += 8) {
                         float qt[8], kt[8];
                         ld_tile8(QK, 128, t, i0, qt);
@@ -579,8 +742,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                             for (int f = 0; f < 8; ++f) {
                                 const int gi = (i0 + f) >> wsh;
-                                const float dcy = __expf(lam[t * G + gi] - lam[j * G + gi]);
-                                lv[e] += qt[f] * kj[f] * dcy;
+                                const float dcy = RL ? __expf(lsc[t * DK + i0 + f] - lsc[j * DK + i0 + f])
+                                                     : __expf(lam[t * G + gi] - lam[j * G + gi]);
+                                lv2[e] += qt[f] * kj[f] * dcy;
                                 mv[e] += kt[f] * kj[f] * dcy;
                             }
                         }
@@ -589,27 +753,55 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int e = 0; e < 8; ++e) {
                         const int j = j0 + e;
                         mv[e] = (j < t) ? (a.pair ? mv[e] : sbeta[j] * mv[e]) : 0.f;
-                        lv[e] = (j <= t) ? lv[e] : 0.f;
+                        lv2[e] = (j <= t) ? lv2[e] : 0.f;
                         Mf[t * LDM + j] = mv[e];
                     }
-                    st_img8(img_L, t, j0, lv);
+                    st_tile8(Ls, 64, t, j0, lv2);
                 }
             }
+            if constexpr (RL) {   // the state pass's decayed operands, now that the area is free
+                __syncthreads();
+                float lc[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    lc[e] = lam[LR_C * DK + i0r + e];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    raw_operands(4 * tb + k, i0r, lv[k], lc);
+            }
+        }
+    }
+    if (!failed) {   // L leaves in one bulk copy
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(img_L, Ls, IMG);
+            bulk_commit();
         }
     }
     if (!failed && a.kind != REC_PLAIN && !SCALAR && wide) {
         // Kbar = k e^{Lambda_t} in place in the raw k rows of the pivoted blocks, before the
         // inverse: the last use of Lambda there, whose tile then holds the Neumann operands
         __syncthreads();
-        for (int u = tid; u < CC * (DK / 8); u += NT) {
-            const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-            float kv[8], lt[8];
+        auto kbar = [&](int t, int i0, const float *lt) {
+            float kv[8];
             ld_tile8(QK, 128, 64 + t, i0, kv);
-            lam8(lam, G, wsh, t, i0, lt);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 kv[e] *= __expf(lt[e]);
             st_tile8(QK, 128, 64 + t, i0, kv);
+        };
+        if constexpr (RL) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                kbar(4 * tb + k, i0r, lv[k]);
+        } else {
+            for (int u = tid; u < CC * (DK / 8); u += NT) {
+                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+                float lt[8];
+                lam8(lam, G, wsh, t, i0, lt);
+                kbar(t, i0, lt);
+            }
         }
     }
     if (!failed && a.pair) {
@@ -633,6 +825,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
     }
     if (!failed) {
+        if (tid == 0 && (SCALAR || (RL && neu)))   // T or the Neumann operands land on L's staging
+            bulk_wait_read();
         __syncthreads();
         if (!neu) {
             if (p.neumann1)
@@ -808,6 +1002,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (with_w) {
             // ---- W = TB Kbar (M = 64, N = dk, K = 64) on tcgen05, read back as an image
             fence_proxy_async_smem();
+            if (tid == 0 && DK > 128)   // W's staging is L's
+                bulk_wait_read();
             __syncthreads();
             if (tid == 0) {
                 tc_fence_after();
@@ -845,16 +1041,35 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                             }
                         }
                         const int col = cw + cb;   // 32 columns inside one 64-column image
-                        uint8_t *img_W = img_T + REC_W + (col >> 6) * IMG;
-                        st_img8(img_W, rr, col & 63, &w0[0]);
-                        st_img8(img_W, rr, (col & 63) + 8, &w0[8]);
-                        st_img8(img_W, rr, (col & 63) + 16, &w1[0]);
-                        st_img8(img_W, rr, (col & 63) + 24, &w1[8]);
+                        if constexpr (W_STAGE) {
+                            const uint32_t wi = Ws + (col >> 6) * IMG;
+                            st_tile8(wi, 64, rr, col & 63, &w0[0]);
+                            st_tile8(wi, 64, rr, (col & 63) + 8, &w0[8]);
+                            st_tile8(wi, 64, rr, (col & 63) + 16, &w1[0]);
+                            st_tile8(wi, 64, rr, (col & 63) + 24, &w1[8]);
+                        } else {
+                            uint8_t *img_W = img_T + REC_W + (col >> 6) * IMG;
+                            st_img8(img_W, rr, col & 63, &w0[0]);
+                            st_img8(img_W, rr, (col & 63) + 8, &w0[8]);
+                            st_img8(img_W, rr, (col & 63) + 16, &w1[0]);
+                            st_img8(img_W, rr, (col & 63) + 24, &w1[8]);
+                        }
+                    }
+                }
+                if constexpr (W_STAGE) {   // W leaves in one bulk copy
+                    fence_proxy_async_smem();
+                    __syncthreads();
+                    if (tid == 0) {
+                        bulk_store(img_T + REC_W, Ws, (DK / 64) * IMG);
+                        bulk_commit();
                     }
                 }
             }
         }
     }
+    // shared memory must outlive the bulk copies' reads of it
+    if (tid == 0)
+        bulk_wait_read();
     // drain: whatever was started must finish before tensor memory is released (bounded)
     if (tid == 0 && failed) {
         mma_commit(&bars[1]);
@@ -909,10 +1124,15 @@ int launch(const Params &p, void *out, int kind, cudaStream_t stream, int pair =
     const long sk = (long)p.B * p.Hk;
     if (!make_map(&mq, p.q, DK, p.T, sk, CC) || !make_map(&mk, p.k, DK, p.T, sk, CC))
         return 6;
-    const Plan Ly = plan(DK, p.G, p.neumann != 0);
-    auto kern = p.G == 1 ? prep_kernel<DK, true> : prep_kernel<DK, false>;
+    // Lambda in registers where it pays (per-channel / grouped gates at dk = 128 with the
+    // state pass's records: its fp32 rows use the record as scratch)
+    const bool rl = DK == 128 && p.G > 1 && kind == REC_EXT;
+    const Plan Ly = plan(DK, p.G, p.neumann != 0, rl);
+    auto kern = p.G == 1 ? prep_kernel<DK, true> : rl ? prep_kernel<DK, false, DK == 128> : prep_kernel<DK, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return 6;
     PrepArgs a;
     a.p = p;

@@ -116,6 +116,20 @@ def test_small_parity(idx, over, chunk, inverse, kernel):
     assert eo <= tol and es <= tol
 
 
+@pytest.mark.parametrize("inverse", ["exact", "neumann"])
+def test_decay_past_pivot_guard(inverse):
+    # log-gates x8: 16-token half blocks span more than the pivot guard, so the first
+    # pass recomputes those Gram rows element by element in fp32 (and rebuilds the
+    # state pass's decayed operands afterwards)
+    w, x = W.workload_inputs(4, Hk=1, Hv=1, T=192 - 11)
+    x["g"] = (x["g"] * 8.0).astype(np.float32)
+    o, Sf = U.run_gpu(x, w.in_dtype, 64, inverse, kernel="tc2")
+    o_ref, S_ref = U.oracle_reference(x, 64, inverse)
+    eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
+    print("rel err o %.3e  S_final %.3e" % (eo, es))
+    assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
+
+
 def test_edge_cases():
     # T = 0: no tokens, S_final = S0
     w, x = W.workload_inputs(0, T=0, s0_std=0.4)
