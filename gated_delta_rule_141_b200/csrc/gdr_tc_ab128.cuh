@@ -22,6 +22,10 @@
 //   [T; *] V -> U (rows 0-63),  [-W; Khat] S -> U - W S = E (rows 0-63),
 //   Khat^T E onto F S.
 // Tensor memory: R_A 0, R_B 128, S_A 256, S_B 384 (fp32, 128 columns each).
+// Pairs (the chunk-128 Neumann inverses run as 64-token halves): a second half adds
+// the first half's correction, E2 += Y E1, as one more product [Y; *] E1 onto its R
+// before the E phase; E1 is still the chain's bf16 E operand then, and Y (from the
+// first half's record) lands just above the second-half stage's [-W; Khat].
 //
 // Roles: warp 0 producer (W, Khat, F), warp 1 MMA issuer, warp 2 producer (T, V),
 // warp 3 idle, warps 4-19 state (S row in TMEM lane 32 (w % 4) + lane, 32 of the
@@ -43,7 +47,7 @@ enum Bar { FULL0, FULL1, FREE0, FREE1, S_READY_A, S_READY_B, P_FULL_A, P_FULL_B,
            E_READY_B, UPD_A, UPD_B, DRAIN, NBARS };
 
 struct Plan {
-    uint32_t wk[2], tv[2], gates[2];
+    uint32_t y, wk[2], tv[2], gates[2];
     uint32_t S[2], E[2], bar, misc, total;
 };
 
@@ -51,7 +55,7 @@ struct Plan {
 // directly followed by V (64 rows, two 64-column blocks): the U product's A operand
 // is the 128 rows from T, whose lower half (V's first block) only feeds rows that
 // nobody reads.
-__host__ __device__ inline Plan plan()
+__host__ __device__ inline Plan plan(bool pair = false)
 {
     Plan s;
     uint32_t o = 0;
@@ -60,7 +64,10 @@ __host__ __device__ inline Plan plan()
         o += (bytes + 1023u) & ~1023u;
         return at;
     };
+    s.y = 0;
     for (int i = 0; i < 2; ++i) {
+        if (pair && i == 1)   // second halves (segments start at even chunks)
+            s.y = take(prep::IMG);
         s.wk[i] = take((KD / 64) * 128 * 128);
         s.tv[i] = take(prep::IMG + 2 * 64 * 128);
     }
@@ -84,7 +91,8 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     using ws::named_vote_or;
     extern __shared__ uint8_t smem_raw[];
     const Params &p = args.p;
-    const Plan Ly = plan();
+    const bool pair = args.pair != 0;
+    const Plan Ly = plan(pair);
     const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *base = smem_raw + (base_u32 - smem_u32(smem_raw));
 
@@ -137,8 +145,11 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             }
             if (lane == 0) {
                 uint64_t *full = &bars[FULL0 + s];
-                if (px) {   // -W and Khat of both 64-column blocks, F
-                    mbar_arrive_expect_tx(full, 4u * prep::IMG + KD * 4);
+                if (px) {   // -W and Khat of both 64-column blocks, F (and a pair's Y)
+                    const bool with_y = pair && s == 1;
+                    mbar_arrive_expect_tx(full, (with_y ? 5u : 4u) * prep::IMG + KD * 4);
+                    if (with_y)
+                        bulk_load(base + Ly.y, fac - args.rec_bytes + args.pair_y, prep::IMG, full);
                     uint8_t *wk = base + Ly.wk[s];
                     for (int kb = 0; kb < KD / 64; ++kb) {
                         bulk_load(wk + kb * 128 * 128, fac + prep::REC_W + kb * prep::IMG, prep::IMG, full);
@@ -199,6 +210,10 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                     for (int k0 = 0; k0 < KD; k0 += 16)
                         mma_bf16(tr[x], desc_kmajor(wk, 128, 0, 0) + kstep(k0), d_s[x] + mstep(k0), id128,
                                  (x == 0 || k0 > 0) ? 1u : 0u);
+                    if (pair && s == 1)   // second half: + Y E1 (rows 0-63)
+                        for (int k0 = 0; k0 < CC; k0 += 16)
+                            mma_bf16(tr[x], desc_kmajor(base_u32 + Ly.y, 128, 0, k0), d_e[x] + mstep(k0),
+                                     id128, 1u);
                     mma_commit(&bars[P_FULL_A + x]);
                 }
                 // S <- F S + Khat^T E

@@ -55,7 +55,7 @@ constexpr uint32_t T_Z = 448;
 constexpr uint32_t TMEM_COLS = 512;
 
 enum Bar { FULLX0, FULLX1, FULLY0, FULLY1, FREEX0, FREEX1, FREEY0, FREEY1, S_READY, P_FULL, E_READY,
-           UPD_DONE, OUT0, OUT1, OFREE0, OFREE1, DRAIN, NBARS };
+           UPD_DONE, OUT0, OUT1, OFREE0, OFREE1, DRAIN, VFREE, NBARS };
 
 template <int DK>
 struct Gates {                        // landed by bulk copies from the first pass's record

@@ -32,6 +32,7 @@ namespace split {
 constexpr int NVC2 = 128;                 // value columns per CTA
 constexpr uint32_t T_R = 0;               // two buffers of 128 columns
 constexpr uint32_t T_S2 = 256;            // fp32 state, 128 columns
+constexpr uint32_t T_X = 384;             // pairs: Y E1 of the first half (rows 64-127)
 
 struct Plan128 {
     uint32_t qwk[2], lzt[2], v[2], gates[2];
@@ -39,8 +40,10 @@ struct Plan128 {
 };
 
 // Stage: [Qbar | -W | Khat] (rows 0-63 | 64-127 | 128-191, 128 columns), [L | 0 | T]
-// (3 x 64 rows, 64 columns), V (64 rows, 128 columns), F (128 fp32).
-__host__ __device__ inline Plan128 plan128()
+// (3 x 64 rows, 64 columns), V (64 rows, 128 columns), F (128 fp32).  Pairs: stage 0
+// (first halves) appends the pair's Y under T ([L | 0 | T | Y]) and V has one buffer
+// (the 16 KB that pays for Y), refilled as soon as the chunk's U product is done.
+__host__ __device__ inline Plan128 plan128(bool pair = false)
 {
     Plan128 s;
     uint32_t o = 0;
@@ -51,8 +54,8 @@ __host__ __device__ inline Plan128 plan128()
     };
     for (int i = 0; i < 2; ++i) {
         s.qwk[i] = take((KD / 64) * 192 * 128);
-        s.lzt[i] = take(192 * 128);
-        s.v[i] = take(2 * 64 * 128);
+        s.lzt[i] = take(((pair && i == 0) ? 256 : 192) * 128);
+        s.v[i] = (pair && i == 1) ? s.v[0] : take(2 * 64 * 128);
     }
     s.S = take(KD * NVC2 * 2);
     s.E = take(CC * NVC2 * 2);
@@ -74,7 +77,8 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     using ws::named_vote_or;
     extern __shared__ uint8_t smem_raw[];
     const Params &p = args.p;
-    const Plan128 Ly = plan128();
+    const bool pair = args.pair != 0;
+    const Plan128 Ly = plan128(pair);
     const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *base = smem_raw + (base_u32 - smem_u32(smem_raw));
 
@@ -167,6 +171,11 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 if (__any_sync(0xffffffffu, !ok))
                     break;
             }
+            if (pair && i >= 1) {   // one V buffer: the previous chunk's U product has read it
+                const bool ok = wait_or_abort(&bars[VFREE], (i - 1) & 1, abort_flag);
+                if (__any_sync(0xffffffffu, !ok))
+                    break;
+            }
             if (lane == 0) {
                 uint64_t *full = &bars[FULLX0 + s];
                 bulk_load(lzt + 128 * 128, fac, prep::IMG, full);   // T under the zeros
@@ -179,12 +188,17 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                     break;
             }
             if (lane == 0) {
+                // pairs: a first half (stage 0: segments start at even chunks) brings the
+                // pair's Y under its T
+                const bool with_y = pair && s == 0;
                 uint64_t *full = &bars[FULLY0 + s];
-                mbar_arrive_expect_tx(full, 3u * prep::IMG);
+                mbar_arrive_expect_tx(full, (with_y ? 4u : 3u) * prep::IMG);
                 for (int kb = 0; kb < KD / 64; ++kb)
                     bulk_load(qwk + kb * 192 * 128 + 128 * 128, fac + prep::EXT_KH + kb * prep::IMG,
                               prep::IMG, full);
                 bulk_load(lzt, fac + prep::IMG, prep::IMG, full);   // L above the zeros
+                if (with_y)
+                    bulk_load(lzt + 192 * 128, fac + args.pair_y, prep::IMG, full);
             }
             army[s] += 1;
         }
@@ -220,6 +234,8 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(rb, desc_kmajor(lzt + 64 * 128, 128, 0, k0),
                              desc_mnmajor(base_u32 + Ly.v[s], 64, k0, 0), id128, k0 > 0);
+                if (pair)
+                    mma_commit(&bars[VFREE]);
                 if (!(ok = wait_or_abort(&bars[S_READY], par, abort_flag)))
                     break;
                 tc_fence_after();
@@ -227,7 +243,8 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 for (int k0 = 0; k0 < KD; k0 += 16)
                     mma_bf16(rb, desc_kmajor(qwk, 192, 0, 0) + kstep(k0, 192), d_s + mstep(k0), id128, 1u);
                 mma_commit(&bars[P_FULL]);
-                mma_commit(&bars[FREEX0 + s]);
+                if (!pair)   // (pairs: T also feeds the first half's Y product below)
+                    mma_commit(&bars[FREEX0 + s]);
                 if (!(ok = wait_or_abort(&bars[E_READY], par, abort_flag)))
                     break;
                 if (!(ok = wait_or_abort(&bars[FULLY0 + s], (i >> 1) & 1, abort_flag)))
@@ -240,6 +257,12 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 // [L; 0] E onto R(s): O = Qbar S + L E in rows 0-63 (rows 64-127 unchanged)
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(rb, desc_kmajor(lzt, 128, 0, k0), d_e + mstep(k0), id128, 1u);
+                if (pair && s == 0)   // [T; Y] E1: Y E1 into rows 64-127 of X for the second half
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tmem + T_X, desc_kmajor(lzt + 128 * 128, 128, 0, k0), d_e + mstep(k0),
+                                 id128, k0 > 0);
+                if (pair)
+                    mma_commit(&bars[FREEX0 + s]);
                 mma_commit(&bars[OUT0 + s]);
                 mma_commit(&bars[FREEY0 + s]);
             }
@@ -316,7 +339,24 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             if (stid == 0)   // every state thread has read its factor (the vote above)
                 mbar_arrive(&bars[FREEX0 + s]);
             tc_fence_after();
-            if (R >= CC) {   // lanes 64-127: E of token t = R - 64, straight from R(s)
+            if (R >= CC && pair && s == 1) {   // second half of a pair: E2 + Y E1 (X, same lanes)
+                const int t = R - CC;
+#pragma unroll
+                for (int h = 0; h < 64; h += 32) {
+                    float ev[32], xv[32];
+                    tmem_ld16(tq + T_R + 128 * s + cs + h, *reinterpret_cast<float(*)[16]>(&ev[0]));
+                    tmem_ld16(tq + T_R + 128 * s + cs + h + 16, *reinterpret_cast<float(*)[16]>(&ev[16]));
+                    tmem_ld16(tq + T_X + cs + h, *reinterpret_cast<float(*)[16]>(&xv[0]));
+                    tmem_ld16(tq + T_X + cs + h + 16, *reinterpret_cast<float(*)[16]>(&xv[16]));
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int n = 0; n < 32; ++n)
+                        ev[n] += xv[n];
+#pragma unroll
+                    for (int n = 0; n < 32; n += 8)
+                        st_tile8(E_T, CC, t, cs + h + n, &ev[n]);
+                }
+            } else if (R >= CC) {   // lanes 64-127: E of token t = R - 64, straight from R(s)
                 const int t = R - CC;
                 float ev[64];
 #pragma unroll
@@ -408,10 +448,10 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
 }
 
 // The 128-column state pass serves grouped / per-channel gates at dk = 128 when the
-// sequences are few and long enough to run segment-parallel, and no pair correction.
+// sequences are few and long enough to run segment-parallel.
 inline bool supports128(const Params &p)
 {
-    return supports(p) && p.dk == KD && p.G > 1 && p.dv % NVC2 == 0 && !p.pair && !p.momentum;
+    return supports(p) && p.dk == KD && p.G > 1 && p.dv % NVC2 == 0 && !p.momentum;
 }
 
 // Segment plan of the 128-column pass (one CTA per head and 128 value columns in
@@ -423,10 +463,11 @@ inline SegPlan seg_plan128(const Params &p)
     const int N = prep::nchunks(p);
     const long nvh = (long)(p.dv / NVC2) * p.Hv * p.B;
     auto waves = [](long ctas) { return (ctas + kSMs - 1) / kSMs; };
+    const int even = p.pair ? 2 : 1;   // pairs never straddle a segment boundary
     SegPlan best{1, N};
     long best_cost = waves(nvh) * (long)N;
     for (int ns = 2; ns <= N / kMinSegChunks; ++ns) {
-        const int L = (N + ns - 1) / ns;
+        const int L = ((N + ns - 1) / ns + even - 1) / even * even;
         const int nsg = (N + L - 1) / L;
         const long cost = 2 * waves(nvh * nsg) * (long)L + nsg;
         if (cost < best_cost) {
@@ -462,7 +503,7 @@ int launch128(const Params &p, const void *factors, cudaStream_t stream)
     CUtensorMap mv;
     if (!make_map(&mv, p.v, p.dv, p.T, (long)p.B * p.Hv, CC))
         return 6;
-    const Plan128 Ly = plan128();
+    const Plan128 Ly = plan128(p.pair != 0);
     auto kern = split128_kernel<OB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly.total) !=
         cudaSuccess)
@@ -476,8 +517,8 @@ int launch128(const Params &p, const void *factors, cudaStream_t stream)
     const SegPlan sp = seg_plan128(p);
     a.nseg = sp.nseg;
     a.seg_len = sp.seg_len;
-    a.pair = 0;
-    a.pair_y = 0;
+    a.pair = p.pair;
+    a.pair_y = prep::kind_bytes(prep::record_kind(p), p.dk) + prep::PAIR_Y;
     a.seg_end = a.seg_trans = a.seg_start = nullptr;
     if (sp.nseg == 1) {   // one segment: the whole sequence from S0, with outputs
         a.mode = MODE_SEQ;
@@ -493,7 +534,7 @@ int launch128(const Params &p, const void *factors, cudaStream_t stream)
     if (cudaFuncSetAttribute(seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)CMB_SMEM) != cudaSuccess)
         return 6;
-    const ab::Plan La = ab::plan();
+    const ab::Plan La = ab::plan(p.pair != 0);
     if (cudaFuncSetAttribute(ab::ab128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)La.total) != cudaSuccess)
         return 6;

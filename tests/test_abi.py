@@ -314,12 +314,17 @@ def test_backward_validates(lib):
 
 def test_wide_state_pass_selection(lib):
     # the 128-column state pass: forced with TC2W (grouped / per-channel gates, dk = 128,
-    # dv % 128 == 0, no pair correction); AUTO takes it for few long sequences
+    # dv % 128 == 0, every inverse: the chunk-128 Neumann ones as corrected pairs); AUTO
+    # takes it for few long sequences
     kda = gdr.make_shape(1, 4096, 1, 1, 128, 128, kernel="tc2w")
     assert gdr.select_kernel(kda, 64, gdr.GATE_CHANNEL) == gdr.KERNEL_TC2W
     assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL) == gdr.KERNEL_TC2W
     assert gdr.select_kernel(kda, 64, gdr.GATE_SCALAR) == -gdr.ERR_UNSUPPORTED
-    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann") == -gdr.ERR_UNSUPPORTED
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann") == gdr.KERNEL_TC2W
+    assert gdr.select_kernel(kda, 128, gdr.GATE_CHANNEL, "neumann1") == gdr.KERNEL_TC2W
+    # pairs never straddle a segment boundary: segments hold an even number of halves
+    pairs = gdr.state_segments(kda, 128, gdr.GATE_CHANNEL, "neumann")
+    assert pairs > 1
     assert gdr.select_kernel(gdr.make_shape(1, 4096, 1, 1, 128, 64, kernel="tc2w"), 64,
                              gdr.GATE_CHANNEL) == -gdr.ERR_UNSUPPORTED
     long = gdr.make_shape(1, 65536, 16, 16, 128, 128)

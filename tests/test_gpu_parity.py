@@ -87,6 +87,10 @@ SMALL = [
     (2, dict(B=1, Hk=2, Hv=2, T=448 - 37), 64, "exact", "tc2w"),
     (2, dict(B=1, Hk=1, Hv=2, T=256, gate_mode=W.GATE_GROUP64), 64, "exact", "tc2w"),
     (2, dict(B=1, Hk=1, Hv=2, T=300, dv=256), 64, "neumann", "tc2w"),
+    # ... and its pairs of 64-token halves at chunk 128 (Y E1 added to a second half)
+    (4, dict(Hk=2, Hv=2, T=640 - 5), 128, "neumann", "tc2w"),
+    (4, dict(Hk=1, Hv=1, T=704 - 37), 128, "neumann", "tc2w"),
+    (2, dict(B=1, Hk=1, Hv=2, T=448 - 37), 128, "neumann1", "tc2w"),
     # dk = 256 with grouped gates on the two-pass path (one [Q | W | K] buffer), grouped
     # value heads, S0, ragged tails, both chunk lengths and every inverse
     (3, dict(B=1, Hk=2, Hv=8, T=384), 64, "exact", "tc2"),

@@ -81,3 +81,33 @@ def test_wide_segmented_state_pass(idx, over):
     print("rel err o %.3e  S_final %.3e" % (eo, es))
     assert np.isfinite(o).all() and np.isfinite(Sf).all()
     assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
+
+
+# The chunk-128 Neumann inverses run as pairs of 64-token halves: segments start at
+# even halves, a second half adds Y E1 in both launches (ends / transitions and
+# outputs); odd half counts leave a last half unpaired.
+WIDE_PAIRS = [
+    (4, dict(Hk=1, Hv=1, T=64 * 60 + 17), "neumann"),
+    (4, dict(B=2, Hk=2, Hv=4, T=64 * 66 + 3), "neumann"),
+    (2, dict(B=1, Hk=1, Hv=1, T=64 * 48, dv=256, gate_mode=W.GATE_GROUP64), "neumann1"),
+    (2, dict(B=1, Hk=1, Hv=2, T=64 * 52 - 9), "neumann1"),
+]
+
+
+@pytest.mark.parametrize("idx,over,inverse", WIDE_PAIRS,
+                         ids=["w%d-%s-%s" % (c[0], "-".join("%s%s" % kv for kv in c[1].items()), c[2])
+                              for c in WIDE_PAIRS])
+def test_wide_segmented_pairs(idx, over, inverse):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from gated_delta_rule_141_b200 import gdr
+    w, x = W.workload_inputs(idx, **over)
+    shape = gdr.make_shape(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, kernel="tc2w")
+    assert gdr.state_segments(shape, 128, gdr.gate_mode_for(w.G, w.dk), inverse) > 1
+    o, Sf = U.run_gpu(x, w.in_dtype, 128, inverse, kernel="tc2w")
+    o_ref, S_ref = U.oracle_reference(x, 128, inverse)
+    eo, es = U.rel_err(o, o_ref), U.rel_err(Sf, S_ref)
+    print("rel err o %.3e  S_final %.3e" % (eo, es))
+    assert np.isfinite(o).all() and np.isfinite(Sf).all()
+    assert eo <= U.TOL_BF16 and es <= U.TOL_BF16
