@@ -31,12 +31,14 @@
 //   3. Atil by Horner's rule (X <- I - Ntil X, m times) and r Newton steps
 //      (X <- X + X (I - X - Ntil X)), all products M = N = K = 128 on tcgen05,
 //      X kept in fp32 in tensor memory and as a bf16 operand in shared memory;
-//   4. Atil11^{-1} exactly in fp32 (block doubling), Y in fp32 on the CUDA cores;
-//      (the 1-Step Neumann inverse of §2.4.3 instead of 3: Atil from the diagonal
-//      16 x 16 blocks in fp32, with the same correction;)
+//   4. Atil11^{-1} exactly in fp32 (block doubling), then Y on tcgen05 from split
+//      bf16 operands (hi + lo parts: fp32-level products, which the cancellation
+//      between Y's two terms needs); (the 1-Step Neumann inverse of §2.4.3 instead
+//      of 3: Atil from the diagonal 16 x 16 blocks, Y in fp32 on the CUDA cores;)
 //   5. Y as a bf16 image into the first half's record.
-// The state pass loads Y under L ([L; Y] tile), so its [L; Y] E product of the
-// first half leaves Y E1 in the tensor-memory rows it reads for the second.
+// The state passes add Y E1 to the second half's E: the 64-column pass through an
+// [L; Y] tile whose E product of the first half leaves Y E1 in tensor memory, the
+// 128-column passes through their own products with Y.
 
 namespace pair {
 
@@ -318,122 +320,169 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         __syncthreads();
     }
 
-    // ---- Y = Atil21 Atil11^{-1} + Atil22 Ntil21 in fp32 (regions of the dead tiles)
-    float *N21f = f32(base, Ly.XT);                      // 64 x LDM each
-    float *A11f = N21f + CC * LDM;
-    float *A21f = A11f + CC * LDM;
-    float *A22f = f32(base, Ly.NTL);                     // once Ntil21 is copied out
     if (!p.neumann1) {
+        // ---- Y = Atil21 Atil11^{-1} + Atil22 Ntil21 on tcgen05 (M = N = K = 64) in split
+        //      bf16 terms: with P = Ph + Pl (Ph the bf16 rounding of the fp32 P, Pl that of
+        //      the rest), P Q ~ Ph Qh + Ph Ql + Pl Qh in fp32, the dropped Pl Ql being 2^-16
+        //      of the product; Ntil21 is exactly the bf16 operand the series used.  The
+        //      inverse Atil11^{-1} stays in fp32 on the CUDA cores (block doubling).
+        float *A11f = f32(base, Ly.XT);                  // strict lower part: I + H form
+        const uint32_t A21H = RT, A21L = RT + 8192, A22H = RT + 16384, A22L = RT + 24576;
+        const uint32_t IH = NTL + 128 * 128, IL = IH + 8192;   // the dead columns 64-127 of Ntil
+        auto split_store = [&](uint32_t th, uint32_t tl, int r, int c, const float *v) {
+            float hi[8], lo[8];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const uint32_t h = pack_bf16(v[e], v[e + 1]);
+                hi[e] = bf16lo(h);
+                hi[e + 1] = bf16hi(h);
+                lo[e] = v[e] - hi[e];
+                lo[e + 1] = v[e + 1] - hi[e + 1];
+            }
+            st_tile8(th, 64, r, c, hi);
+            st_tile8(tl, 64, r, c, lo);
+        };
         if (!failed) {
             tc_fence_after();
-            // Atil from tensor memory: rows 0-63 x columns 0-63 (strict lower part, as I + H
-            // for the inverse), rows 64-127 x columns 0-63 (Atil21)
-            if (ch == 0) {
-                for (int c = 0; c < 64; c += 16) {
-                    float x[16];
-                    tmem_ld16(tq + T_X + c, x);
-                    tmem_ld_wait();
-                    if (R < 64) {
+            // Atil from tensor memory: Atil11 (strict lower part) to fp32 for the inverse,
+            // Atil21 and Atil22 straight to their split operand tiles
+            for (int c = 0; c < 64; c += 16) {
+                float x[16];
+                tmem_ld16(tq + T_X + ch + c, x);
+                tmem_ld_wait();
+                if (ch == 0 && R < 64) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            A11f[R * LDM + c + e] = (R > c + e) ? x[e] : 0.f;
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            A21f[(R - 64) * LDM + c + e] = x[e];
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        A11f[R * LDM + c + e] = (R > c + e) ? x[e] : 0.f;
+                } else if (R >= 64) {
+                    const uint32_t th = ch == 0 ? A21H : A22H, tl = ch == 0 ? A21L : A22L;
+                    split_store(th, tl, R - 64, c, &x[0]);
+                    split_store(th, tl, R - 64, c + 8, &x[8]);
                 }
             }
-            for (int u = tid; u < CC * 8; u += NT) {          // Ntil21 as the bf16 the series used
+        }
+        __syncthreads();
+        if (!failed) {
+            gen::inverse64_par(A11f, Tf, tid);            // Atil11^{-1}, unit lower triangular
+            for (int u = tid; u < CC * 8; u += NT) {
+                const int r = u >> 3, c = (u & 7) * 8;
+                split_store(IH, IL, r, c, A11f + r * LDM + c);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (!failed) {
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id64 = idesc_bf16(64, 64, false, true);
+                for (int k0 = 0; k0 < CC; k0 += 16) {
+                    const uint64_t a21h = desc_kmajor(A21H, 64, 0, k0), a21l = desc_kmajor(A21L, 64, 0, k0);
+                    const uint64_t a22h = desc_kmajor(A22H, 64, 0, k0), a22l = desc_kmajor(A22L, 64, 0, k0);
+                    const uint64_t ih = desc_mnmajor(IH, 64, k0, 0), il = desc_mnmajor(IL, 64, k0, 0);
+                    const uint64_t n21 = desc_mnmajor(NTL, 128, 64 + k0, 0);
+                    mma_bf16(tmem + T_D, a21h, ih, id64, k0 > 0);
+                    mma_bf16(tmem + T_D, a21h, il, id64, 1u);
+                    mma_bf16(tmem + T_D, a21l, ih, id64, 1u);
+                    mma_bf16(tmem + T_D, a22h, n21, id64, 1u);
+                    mma_bf16(tmem + T_D, a22l, n21, id64, 1u);
+                }
+                mma_commit(&bars[1]);
+            }
+            failed = wait_bar(1, ph_mma);
+            ph_mma ^= 1u;
+        }
+        if (!failed) {   // Y (M = 64 accumulator: rows in lanes 0-15 of each quarter) as an image
+            tc_fence_after();
+            const int rr = gen::row64g(warp, lane);
+            const int cb = 32 * (warp >> 2);
+            float d0[16], d1[16];
+            tmem_ld16(tq + T_D + cb, d0);
+            tmem_ld16(tq + T_D + cb + 16, d1);
+            tmem_ld_wait();
+            if (rr >= 0) {
+                prep::st_img8(img_Y, rr, cb, &d0[0]);
+                prep::st_img8(img_Y, rr, cb + 8, &d0[8]);
+                prep::st_img8(img_Y, rr, cb + 16, &d1[0]);
+                prep::st_img8(img_Y, rr, cb + 24, &d1[8]);
+            }
+        }
+    } else {
+        // ---- the 1-Step Neumann inverse: Atil21 from the diagonal blocks, Y in fp32
+        float *N21f = f32(base, Ly.XT);                  // 64 x LDM each
+        float *A11f = N21f + CC * LDM;
+        float *A21f = A11f + CC * LDM;
+        float *A22f = f32(base, Ly.NTL);                 // once Ntil21 is copied out
+        if (!failed) {
+            // 1-Step Neumann ("Systolic Linear Attention ...", §2.4.3), in fp32 from the bf16
+            // blocks: Atil = Dtil^{-1} - Dtil^{-1} Ntil_off Dtil^{-1}, Dtil the diagonal 16 x 16
+            // blocks of I + Ntil; per half that is the first pass's 64-token factor, and across
+            // the halves Atil21 = -bd(Atil22) Ntil21 bd(Atil11) (bd: the diagonal blocks)
+            for (int u = tid; u < CC * 8; u += NT) {
                 const int t = u >> 3, j0 = (u & 7) * 8;
-                float v8[8];
-                ld_tile8(NTL, 128, 64 + t, j0, v8);
+                float a8[8], n8[8];
+                ld_tile8(NTL, 128, t, j0, a8);
+                ld_tile8(NTL, 128, 64 + t, j0, n8);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    A11f[t * LDM + j0 + e] = (t > j0 + e) ? a8[e] : 0.f;
+                    N21f[t * LDM + j0 + e] = n8[e];
+                }
+            }
+            __syncthreads();
+            for (int u = tid; u < CC * 8; u += NT) {   // Ntil22 lies past the bytes of A22f
+                const int t = u >> 3, j0 = (u & 7) * 8;
+                float a8[8];
+                ld_tile8(NTL, 128, 64 + t, 64 + j0, a8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    N21f[t * LDM + j0 + e] = v8[e];
+                    A22f[t * LDM + j0 + e] = (t > j0 + e) ? a8[e] : 0.f;
             }
-        }
-        __syncthreads();
-        if (!failed && ch == 64 && R >= 64) {                 // Atil22: rows and columns 64-127
-            for (int c = 64; c < 128; c += 16) {
-                float x[16];
-                tmem_ld16(tq + T_X + c, x);
-                tmem_ld_wait();
+            __syncthreads();
+            gen::block_neumann1_64_inplace(A11f, Tf, tid);
+            gen::block_neumann1_64_inplace(A22f, Tf, tid);
+            const int rg = tid >> 4, c0 = 4 * (tid & 15), lb = c0 & ~15, lr = 16 * (rg >> 2);
+            float acc[4][4];
+            // Z = Ntil21 bd(Atil11): rows rg + 16 i, columns c0..c0+3 (one 16-column block)
+            gen::block_product4x4<16>(acc, N21f + rg * LDM + lb, 16 * LDM, A11f + lb * LDM + c0, LDM, 0);
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    A22f[(R - 64) * LDM + c - 64 + e] = x[e];
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    A21f[(rg + 16 * i) * LDM + c0 + n] = acc[i][n];
+            __syncthreads();
+            // Atil21 = -bd(Atil22) Z: rows 4 rg .. 4 rg + 3 (one 16-row block)
+            gen::block_product4x4<16>(acc, A22f + (4 * rg) * LDM + lr, LDM, A21f + lr * LDM + c0, LDM, 0);
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    A21f[(4 * rg + i) * LDM + c0 + n] = -acc[i][n];
+            for (int u = tid; u < CC * CC; u += NT) {   // Atil11 as I + H for the exact inverse
+                const int t = u / CC, j = u % CC;
+                if (t <= j)
+                    A11f[t * LDM + j] = 0.f;
             }
+            __syncthreads();
         }
-        __syncthreads();
-    } else if (!failed) {
-        // 1-Step Neumann ("Systolic Linear Attention ...", §2.4.3), in fp32 from the bf16
-        // blocks: Atil = Dtil^{-1} - Dtil^{-1} Ntil_off Dtil^{-1}, Dtil the diagonal 16 x 16
-        // blocks of I + Ntil; per half that is the first pass's 64-token factor, and across
-        // the halves Atil21 = -bd(Atil22) Ntil21 bd(Atil11) (bd: the diagonal blocks)
-        for (int u = tid; u < CC * 8; u += NT) {
-            const int t = u >> 3, j0 = (u & 7) * 8;
-            float a8[8], n8[8];
-            ld_tile8(NTL, 128, t, j0, a8);
-            ld_tile8(NTL, 128, 64 + t, j0, n8);
+        if (!failed) {
+            gen::inverse64_par(A11f, Tf, tid);                // Atil11^{-1}, lower triangular
+            const int rg = tid >> 4, c0 = 4 * (tid & 15);     // rows rg + 16 i, columns c0..c0+3
+            float y[4][4], z[4][4];
+            gen::block_product4x4<64>(y, A21f + rg * LDM, 16 * LDM, A11f + c0, LDM, c0);
+            gen::block_product4x4<64>(z, A22f + rg * LDM, 16 * LDM, N21f + c0, LDM, 0);
+            __syncthreads();                                  // every read of A21f done
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                A11f[t * LDM + j0 + e] = (t > j0 + e) ? a8[e] : 0.f;
-                N21f[t * LDM + j0 + e] = n8[e];
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    A21f[(rg + 16 * i) * LDM + c0 + n] = y[i][n] + z[i][n];
+            __syncthreads();
+            for (int u = tid; u < CC * 8; u += NT) {          // Y as a 128-byte-swizzled image
+                const int t = u >> 3, j0 = (u & 7) * 8;
+                prep::st_img8(img_Y, t, j0, A21f + t * LDM + j0);
             }
-        }
-        __syncthreads();
-        for (int u = tid; u < CC * 8; u += NT) {   // Ntil22 lies past the bytes of A22f
-            const int t = u >> 3, j0 = (u & 7) * 8;
-            float a8[8];
-            ld_tile8(NTL, 128, 64 + t, 64 + j0, a8);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                A22f[t * LDM + j0 + e] = (t > j0 + e) ? a8[e] : 0.f;
-        }
-        __syncthreads();
-        gen::block_neumann1_64_inplace(A11f, Tf, tid);
-        gen::block_neumann1_64_inplace(A22f, Tf, tid);
-        const int rg = tid >> 4, c0 = 4 * (tid & 15), lb = c0 & ~15, lr = 16 * (rg >> 2);
-        float acc[4][4];
-        // Z = Ntil21 bd(Atil11): rows rg + 16 i, columns c0..c0+3 (one 16-column block)
-        gen::block_product4x4<16>(acc, N21f + rg * LDM + lb, 16 * LDM, A11f + lb * LDM + c0, LDM, 0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-                A21f[(rg + 16 * i) * LDM + c0 + n] = acc[i][n];
-        __syncthreads();
-        // Atil21 = -bd(Atil22) Z: rows 4 rg .. 4 rg + 3 (one 16-row block)
-        gen::block_product4x4<16>(acc, A22f + (4 * rg) * LDM + lr, LDM, A21f + lr * LDM + c0, LDM, 0);
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-                A21f[(4 * rg + i) * LDM + c0 + n] = -acc[i][n];
-        for (int u = tid; u < CC * CC; u += NT) {   // Atil11 as I + H for the exact inverse
-            const int t = u / CC, j = u % CC;
-            if (t <= j)
-                A11f[t * LDM + j] = 0.f;
-        }
-        __syncthreads();
-    }
-    if (!failed) {
-        gen::inverse64_par(A11f, Tf, tid);                // Atil11^{-1}, lower triangular
-        const int rg = tid >> 4, c0 = 4 * (tid & 15);     // rows rg + 16 i, columns c0..c0+3
-        float y[4][4], z[4][4];
-        gen::block_product4x4<64>(y, A21f + rg * LDM, 16 * LDM, A11f + c0, LDM, c0);
-        gen::block_product4x4<64>(z, A22f + rg * LDM, 16 * LDM, N21f + c0, LDM, 0);
-        __syncthreads();                                  // every read of A21f done
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-                A21f[(rg + 16 * i) * LDM + c0 + n] = y[i][n] + z[i][n];
-        __syncthreads();
-        for (int u = tid; u < CC * 8; u += NT) {          // Y as a 128-byte-swizzled image
-            const int t = u >> 3, j0 = (u & 7) * 8;
-            prep::st_img8(img_Y, t, j0, A21f + t * LDM + j0);
         }
     }
     if (tid == 0 && failed) {   // drain what was started before releasing tensor memory
