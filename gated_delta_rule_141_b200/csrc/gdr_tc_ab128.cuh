@@ -113,7 +113,7 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 4);
-    auto fgate = [&](int s) { return reinterpret_cast<float *>(base + Ly.gates[s]); };
+    auto fgate = [&](int s) { return reinterpret_cast<float *>(base + stage(Ly.gates, s)); };
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i)   // FULL: two producers; FREE: the MMAs and the state warps
@@ -134,7 +134,7 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     if (warp == W_PX || warp == W_PY) {
         // ------------------------------------------------------------ producers
         const bool px = warp == W_PX;
-        int armed[2] = {0, 0};
+        int armed0 = 0, armed1 = 0;   // copies issued on each stage's barrier
         for (int i = 0; i < nloc; ++i) {
             const int c = cbeg + i, s = i & 1;
             const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
@@ -150,7 +150,7 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                     mbar_arrive_expect_tx(full, (with_y ? 5u : 4u) * prep::IMG + KD * 4);
                     if (with_y)
                         bulk_load(base + Ly.y, fac - args.rec_bytes + args.pair_y, prep::IMG, full);
-                    uint8_t *wk = base + Ly.wk[s];
+                    uint8_t *wk = base + stage(Ly.wk, s);
                     for (int kb = 0; kb < KD / 64; ++kb) {
                         bulk_load(wk + kb * 128 * 128, fac + prep::REC_W + kb * prep::IMG, prep::IMG, full);
                         bulk_load(wk + kb * 128 * 128 + 64 * 128, fac + prep::EXT_KH + kb * prep::IMG,
@@ -159,19 +159,20 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                     bulk_load(fgate(s), fac + prep::EXT_F, KD * 4, full);
                 } else {    // T, then V
                     mbar_arrive_expect_tx(full, prep::IMG + CC * NV * 2);
-                    uint8_t *tv = base + Ly.tv[s];
+                    uint8_t *tv = base + stage(Ly.tv, s);
                     const long c0 = (long)c * CC;
                     bulk_load(tv, fac, prep::IMG, full);
                     tma_load_3d(tv + prep::IMG, &tm_v, full, n0, (int)c0, (int)vh);
                     tma_load_3d(tv + prep::IMG + 64 * 128, &tm_v, full, n0 + 64, (int)c0, (int)vh);
                 }
             }
-            armed[s] += 1;
+            armed0 += s == 0;
+            armed1 += s == 1;
         }
         if (lane == 0)   // no copy may still be in flight when the CTA exits
             for (int s = 0; s < 2; ++s)
-                if (armed[s] > 0)
-                    mbar_wait(&bars[FULL0 + s], (armed[s] - 1) & 1, 200000000ull);
+                if ((s == 0 ? armed0 : armed1) > 0)
+                    mbar_wait(&bars[FULL0 + s], ((s == 0 ? armed0 : armed1) - 1) & 1, 200000000ull);
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -181,23 +182,24 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 return static_cast<uint64_t>(((k0 >> 6) * 128 * 128 + (k0 & 63) * 2) >> 4);
             };
             auto mstep = [](int k0) { return static_cast<uint64_t>(k0 * 8); };
-            const uint64_t d_s[2] = {desc_mnmajor(base_u32 + Ly.S[0], KD, 0, 0),
-                                     desc_mnmajor(base_u32 + Ly.S[1], KD, 0, 0)};
-            const uint64_t d_e[2] = {desc_mnmajor(base_u32 + Ly.E[0], CC, 0, 0),
-                                     desc_mnmajor(base_u32 + Ly.E[1], CC, 0, 0)};
-            const uint32_t tr[2] = {tmem + T_RA, tmem + T_RB}, ts[2] = {tmem + T_SA, tmem + T_SB};
+            // per chain x (arithmetic, so that nothing lives in local memory)
+            const uint32_t dSE = Ly.S[1] - Ly.S[0];
+            auto d_s = [&](int x) { return desc_mnmajor(base_u32 + Ly.S[0] + x * dSE, KD, 0, 0); };
+            auto d_e = [&](int x) { return desc_mnmajor(base_u32 + Ly.E[0] + x * dSE, CC, 0, 0); };
+            auto tr = [&](int x) { return tmem + T_RA + (T_RB - T_RA) * x; };
+            auto ts = [&](int x) { return tmem + T_SA + (T_SB - T_SA) * x; };
             const int nch = dual ? 2 : 1;
             bool ok = true;
             for (int i = 0; i < nloc && ok; ++i) {
                 const int s = i & 1;
                 const uint32_t par = i & 1;
-                const uint32_t wk = base_u32 + Ly.wk[s], tv = base_u32 + Ly.tv[s];
+                const uint32_t wk = base_u32 + stage(Ly.wk, s), tv = base_u32 + stage(Ly.tv, s);
                 if (!(ok = wait_or_abort(&bars[FULL0 + s], (i >> 1) & 1, abort_flag)))
                     break;
                 tc_fence_after();
                 // U = [T; *] V into R_A (E_A of the previous chunk has been read)
                 for (int k0 = 0; k0 < CC; k0 += 16)
-                    mma_bf16(tr[0], desc_kmajor(tv, 128, 0, k0), desc_mnmajor(tv + prep::IMG, 64, k0, 0),
+                    mma_bf16(tr(0), desc_kmajor(tv, 128, 0, k0), desc_mnmajor(tv + prep::IMG, 64, k0, 0),
                              id128, k0 > 0);
                 // [-W; Khat] S: E = U - W S into rows 0-63 (value chain), -W S (transition)
 #pragma unroll
@@ -208,11 +210,11 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                         break;
                     tc_fence_after();
                     for (int k0 = 0; k0 < KD; k0 += 16)
-                        mma_bf16(tr[x], desc_kmajor(wk, 128, 0, 0) + kstep(k0), d_s[x] + mstep(k0), id128,
+                        mma_bf16(tr(x), desc_kmajor(wk, 128, 0, 0) + kstep(k0), d_s(x) + mstep(k0), id128,
                                  (x == 0 || k0 > 0) ? 1u : 0u);
                     if (pair && s == 1)   // second half: + Y E1 (rows 0-63)
                         for (int k0 = 0; k0 < CC; k0 += 16)
-                            mma_bf16(tr[x], desc_kmajor(base_u32 + Ly.y, 128, 0, k0), d_e[x] + mstep(k0),
+                            mma_bf16(tr(x), desc_kmajor(base_u32 + Ly.y, 128, 0, k0), d_e(x) + mstep(k0),
                                      id128, 1u);
                     mma_commit(&bars[P_FULL_A + x]);
                 }
@@ -226,7 +228,7 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                         break;
                     tc_fence_after();
                     for (int k0 = 0; k0 < CC; k0 += 16)
-                        mma_bf16(ts[x], kt + mstep(k0), d_e[x] + mstep(k0), id_s, 1u);
+                        mma_bf16(ts(x), kt + mstep(k0), d_e(x) + mstep(k0), id_s, 1u);
                     mma_commit(&bars[UPD_A + x]);
                 }
                 mma_commit(&bars[FREE0 + s]);
@@ -240,9 +242,11 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
         const int R = 32 * (warp & 3) + lane;            // S row (key channel), E row if < 64
         const int cs = 32 * ((warp - W_STATE0) >> 2);    // this thread's 32 of the 128 columns
         const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-        const uint32_t tr[2] = {tq + T_RA + cs, tq + T_RB + cs}, ts[2] = {tq + T_SA + cs, tq + T_SB + cs};
-        const uint32_t S_T[2] = {base_u32 + Ly.S[0], base_u32 + Ly.S[1]};
-        const uint32_t E_T[2] = {base_u32 + Ly.E[0], base_u32 + Ly.E[1]};
+        const uint32_t dSE = Ly.S[1] - Ly.S[0];
+        auto tr = [&](int x) { return tq + T_RA + (T_RB - T_RA) * x + cs; };
+        auto ts = [&](int x) { return tq + T_SA + (T_SB - T_SA) * x + cs; };
+        auto S_T = [&](int x) { return base_u32 + Ly.S[0] + x * dSE; };
+        auto E_T = [&](int x) { return base_u32 + Ly.E[0] + x * dSE; };
         const int nch = dual ? 2 : 1;
         // chain A from zero; chain B from the identity
 #pragma unroll
@@ -253,8 +257,8 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
 #pragma unroll
             for (int n = 0; n < 32; ++n)
                 sv[n] = (x == 1 && R == cs + n) ? 1.f : 0.f;
-            tmem_st16(ts[x], *reinterpret_cast<const float(*)[16]>(&sv[0]));
-            tmem_st16(ts[x] + 16, *reinterpret_cast<const float(*)[16]>(&sv[16]));
+            tmem_st16(ts(x), *reinterpret_cast<const float(*)[16]>(&sv[0]));
+            tmem_st16(ts(x) + 16, *reinterpret_cast<const float(*)[16]>(&sv[16]));
         }
         tmem_st_wait();
         bool ok = true;
@@ -273,12 +277,12 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 }
                 tc_fence_after();
                 float sv[32];
-                tmem_ld16(ts[x], *reinterpret_cast<float(*)[16]>(&sv[0]));
-                tmem_ld16(ts[x] + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
+                tmem_ld16(ts(x), *reinterpret_cast<float(*)[16]>(&sv[0]));
+                tmem_ld16(ts(x) + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
                 tmem_ld_wait();
 #pragma unroll
                 for (int n = 0; n < 32; n += 8)
-                    st_tile8(S_T[x], KD, R, cs + n, &sv[n]);
+                    st_tile8(S_T(x), KD, R, cs + n, &sv[n]);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 named_sync(NB_STATE, N_STATE);
@@ -293,8 +297,8 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
 #pragma unroll
                 for (int n = 0; n < 32; ++n)
                     sv[n] *= F;
-                tmem_st16(ts[x], *reinterpret_cast<const float(*)[16]>(&sv[0]));
-                tmem_st16(ts[x] + 16, *reinterpret_cast<const float(*)[16]>(&sv[16]));
+                tmem_st16(ts(x), *reinterpret_cast<const float(*)[16]>(&sv[0]));
+                tmem_st16(ts(x) + 16, *reinterpret_cast<const float(*)[16]>(&sv[16]));
             }
             if (!ok)
                 break;
@@ -312,12 +316,12 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 tc_fence_after();
                 if (R < CC) {
                     float ev[32];
-                    tmem_ld16(tr[x], *reinterpret_cast<float(*)[16]>(&ev[0]));
-                    tmem_ld16(tr[x] + 16, *reinterpret_cast<float(*)[16]>(&ev[16]));
+                    tmem_ld16(tr(x), *reinterpret_cast<float(*)[16]>(&ev[0]));
+                    tmem_ld16(tr(x) + 16, *reinterpret_cast<float(*)[16]>(&ev[16]));
                     tmem_ld_wait();
 #pragma unroll
                     for (int n = 0; n < 32; n += 8)
-                        st_tile8(E_T[x], CC, R, cs + n, &ev[n]);
+                        st_tile8(E_T(x), CC, R, cs + n, &ev[n]);
                 }
                 tmem_st_wait();
                 fence_proxy_async_smem();
@@ -342,8 +346,8 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             float *dst = x == 0 ? args.seg_end + (((size_t)vh * args.nseg + seg) * KD + R) * p.dv + n0 + cs
                                 : args.seg_trans + (((size_t)kh * args.nseg + seg) * KD + R) * KD + cs;
             float sv[32];
-            tmem_ld16(ts[x], *reinterpret_cast<float(*)[16]>(&sv[0]));
-            tmem_ld16(ts[x] + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
+            tmem_ld16(ts(x), *reinterpret_cast<float(*)[16]>(&sv[0]));
+            tmem_ld16(ts(x) + 16, *reinterpret_cast<float(*)[16]>(&sv[16]));
             tmem_ld_wait();
 #pragma unroll
             for (int n = 0; n < 32; n += 4)

@@ -57,6 +57,11 @@ constexpr uint32_t TMEM_COLS = 512;
 enum Bar { FULLX0, FULLX1, FULLY0, FULLY1, FREEX0, FREEX1, FREEY0, FREEY1, S_READY, P_FULL, E_READY,
            UPD_DONE, OUT0, OUT1, OFREE0, OFREE1, DRAIN, VFREE, NBARS };
 
+// The stage-s member of a two-stage plan array, selected rather than indexed, so that
+// a plan whose arrays are indexed by a runtime stage stays in registers (an indexed
+// array would live in local memory, one load on every use).
+__host__ __device__ __forceinline__ uint32_t stage(const uint32_t (&a)[2], int s) { return s ? a[1] : a[0]; }
+
 template <int DK>
 struct Gates {                        // landed by bulk copies from the first pass's record
     float ea[CC], eb[CC];             // scalar gate: e^{Lambda_t}, e^{Lambda_C - Lambda_t}
@@ -240,7 +245,7 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 4);
-    auto gates_of = [&](int s) { return reinterpret_cast<Gates<DK> *>(base + Ly.gates[s]); };
+    auto gates_of = [&](int s) { return reinterpret_cast<Gates<DK> *>(base + stage(Ly.gates, s)); };
     // Wait before loading chunk i into stage i & 1 until its previous contents are
     // released (FREEX0 / FREEY0 and the stage's offset): with two buffers, their use by
     // chunk i - 2; with one [Q | W | K] buffer, the previous chunk's release of the
@@ -274,8 +279,8 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     for (int i = tid; i < 2 * 64 * 8; i += NTHR) {
         const int st = i >> 9, r = (i >> 3) & 63, c = (i & 7) * 8;
         const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        st_tile8(base_u32 + Ly.lz[st], 128, 64 + r, c, z);
-        st_tile8(base_u32 + Ly.ab[st], 128, r, c, z);
+        st_tile8(base_u32 + stage(Ly.lz, st), 128, 64 + r, c, z);
+        st_tile8(base_u32 + stage(Ly.ab, st), 128, r, c, z);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -287,12 +292,12 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     if (warp == W_PROD) {
         // ------------------------------------------------------------ producer
-        int armx[2] = {0, 0};   // group X loads armed per stage
+        int narmx = 0;     // group X loads armed per stage
         for (int i = 0; i < nloc; ++i) {
             const int c = cbeg + i, s = i & 1;
             const long c0 = (long)c * CC;
             const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
-            uint8_t *qwk = base + Ly.qwk[s];
+            uint8_t *qwk = base + stage(Ly.qwk, s);
             // group X: W, Q (or Qbar), T, V, the decay factors.  Q only where o is
             // written; T and V not for a transition CTA.
             {
@@ -321,26 +326,26 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 else
                     bulk_load(gates_of(s)->F, fac + prep::ext_f(DK), fac_bytes, full);
             }
-            armx[s] += 1;
+            ++narmx;
         }
         // drain loads that may still be landing (bounded): the last armed phase of
         // each barrier, whether or not a consumer saw it
         if (lane == 0) {
             for (int s = 0; s < 2; ++s)
-                if (armx[s] > 0)
-                    mbar_wait(&bars[FULLX0 + s], (armx[s] - 1) & 1, 200000000ull);
+                if ((narmx + 1 - s) / 2 > 0)   // loads armed on stage s
+                    mbar_wait(&bars[FULLX0 + s], ((narmx + 1 - s) / 2 - 1) & 1, 200000000ull);
         }
     } else if (warp == W_PROD_Y) {
         // ------------------------------------------------------------ second producer
         // T and V of group X (their bytes are part of what warp W_PROD expects on FULLX,
         // so the phase completes only when both threads' copies have landed), then
         // group Y.
-        int army[2] = {0, 0};   // group Y loads armed per stage
+        int narmy = 0;     // group Y loads armed per stage
         for (int i = 0; i < nloc; ++i) {
             const int c = cbeg + i, s = i & 1;
             const long c0 = (long)c * CC;
             const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
-            uint8_t *qwk = base + Ly.qwk[s];
+            uint8_t *qwk = base + stage(Ly.qwk, s);
             // T and V of group X (counted in the FULLX bytes that warp W_PROD expects)
             if (!trans) {
                 {
@@ -350,8 +355,8 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
                 if (lane == 0) {
                     uint64_t *full = &bars[FULLX0 + s];
-                    bulk_load(base + Ly.ab[s] + 64 * 128, fac, prep::IMG, full);
-                    tma_load_3d(base + Ly.v[s], &tm_v, full, n0, (int)c0, (int)vh);
+                    bulk_load(base + stage(Ly.ab, s) + 64 * 128, fac, prep::IMG, full);
+                    tma_load_3d(base + stage(Ly.v, s), &tm_v, full, n0, (int)c0, (int)vh);
                 }
             }
             // group Y: K (or Khat), L (L only where o is written)
@@ -367,7 +372,7 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 uint64_t *full = &bars[FULLY0 + s];
                 mbar_arrive_expect_tx(full, (NKB + (outputs ? 1u : 0u)) * prep::IMG + (with_y ? prep::IMG : 0u));
                 if (with_y)
-                    bulk_load(base + Ly.lz[s] + 64 * 128, fac + args.pair_y, prep::IMG, full);
+                    bulk_load(base + stage(Ly.lz, s) + 64 * 128, fac + args.pair_y, prep::IMG, full);
                 for (int kb = 0; kb < NKB; ++kb) {
                     uint8_t *blk = qwk + kb * 192 * 128 + 128 * 128;
                     if (scalar)
@@ -376,14 +381,14 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         bulk_load(blk, fac + prep::ext_kh(DK) + kb * prep::IMG, prep::IMG, full);
                 }
                 if (outputs)
-                    bulk_load(base + Ly.lz[s], fac + prep::IMG, prep::IMG, full);
+                    bulk_load(base + stage(Ly.lz, s), fac + prep::IMG, prep::IMG, full);
             }
-            army[s] += 1;
+            ++narmy;
         }
         if (lane == 0) {
             for (int s = 0; s < 2; ++s)
-                if (army[s] > 0)
-                    mbar_wait(&bars[FULLY0 + s], (army[s] - 1) & 1, 200000000ull);
+                if ((narmy + 1 - s) / 2 > 0)   // loads armed on stage s
+                    mbar_wait(&bars[FULLY0 + s], ((narmy + 1 - s) / 2 - 1) & 1, 200000000ull);
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer

@@ -99,7 +99,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + Ly.misc + 4);
-    auto fgate = [&](int s) { return reinterpret_cast<float *>(base + Ly.gates[s]); };
+    auto fgate = [&](int s) { return reinterpret_cast<float *>(base + stage(Ly.gates, s)); };
     const uint32_t S_T = base_u32 + Ly.S, E_T = base_u32 + Ly.E;
 
     if (tid == 0) {
@@ -117,7 +117,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     for (int i = tid; i < 2 * 64 * 8; i += NTHR) {
         const int st = i >> 9, r = (i >> 3) & 63, c = (i & 7) * 8;
         const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        st_tile8(base_u32 + Ly.lzt[st], 192, 64 + r, c, z);
+        st_tile8(base_u32 + stage(Ly.lzt, st), 192, 64 + r, c, z);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -130,11 +130,11 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     if (warp == W_PROD) {
         // ------------------------------------------------------------ producer: X group
         // [Qbar; -W] (Qbar only where o is written) and F; warp 12 adds T and V
-        int armx[2] = {0, 0};
+        int narmx = 0;   // group X loads armed (both stages)
         for (int i = 0; i < nloc; ++i) {
             const int c = cbeg + i, s = i & 1;
             const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
-            uint8_t *qwk = base + Ly.qwk[s];
+            uint8_t *qwk = base + stage(Ly.qwk, s);
             if (i >= 2) {
                 const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
                 if (__any_sync(0xffffffffu, !ok))
@@ -150,22 +150,22 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 }
                 bulk_load(fgate(s), fac + prep::EXT_F, KD * 4, full);
             }
-            armx[s] += 1;
+            ++narmx;
         }
         if (lane == 0) {
             for (int s = 0; s < 2; ++s)
-                if (armx[s] > 0)
-                    mbar_wait(&bars[FULLX0 + s], (armx[s] - 1) & 1, 200000000ull);
+                if ((narmx + 1 - s) / 2 > 0)   // loads armed on stage s
+                    mbar_wait(&bars[FULLX0 + s], ((narmx + 1 - s) / 2 - 1) & 1, 200000000ull);
         }
     } else if (warp == W_PROD_Y) {
         // ------------------------------------------------------------ producer: T, V; Y group
-        int army[2] = {0, 0};
+        int narmy = 0;   // group Y loads armed (both stages)
         for (int i = 0; i < nloc; ++i) {
             const int c = cbeg + i, s = i & 1;
             const long c0 = (long)c * CC;
             const uint8_t *fac = args.factors + (size_t)(kh * N + c) * args.rec_bytes;
-            uint8_t *qwk = base + Ly.qwk[s];
-            uint8_t *lzt = base + Ly.lzt[s];
+            uint8_t *qwk = base + stage(Ly.qwk, s);
+            uint8_t *lzt = base + stage(Ly.lzt, s);
             if (i >= 2) {
                 const bool ok = wait_or_abort(&bars[FREEX0 + s], ((i >> 1) - 1) & 1, abort_flag);
                 if (__any_sync(0xffffffffu, !ok))
@@ -179,8 +179,8 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             if (lane == 0) {
                 uint64_t *full = &bars[FULLX0 + s];
                 bulk_load(lzt + 128 * 128, fac, prep::IMG, full);   // T under the zeros
-                tma_load_3d(base + Ly.v[s], &tm_v, full, n0, (int)c0, (int)vh);
-                tma_load_3d(base + Ly.v[s] + 64 * 128, &tm_v, full, n0 + 64, (int)c0, (int)vh);
+                tma_load_3d(base + stage(Ly.v, s), &tm_v, full, n0, (int)c0, (int)vh);
+                tma_load_3d(base + stage(Ly.v, s) + 64 * 128, &tm_v, full, n0 + 64, (int)c0, (int)vh);
             }
             if (i >= 2) {
                 const bool ok = wait_or_abort(&bars[FREEY0 + s], ((i >> 1) - 1) & 1, abort_flag);
@@ -200,12 +200,12 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 if (with_y)
                     bulk_load(lzt + 192 * 128, fac + args.pair_y, prep::IMG, full);
             }
-            army[s] += 1;
+            ++narmy;
         }
         if (lane == 0) {
             for (int s = 0; s < 2; ++s)
-                if (army[s] > 0)
-                    mbar_wait(&bars[FULLY0 + s], (army[s] - 1) & 1, 200000000ull);
+                if ((narmy + 1 - s) / 2 > 0)   // loads armed on stage s
+                    mbar_wait(&bars[FULLY0 + s], ((narmy + 1 - s) / 2 - 1) & 1, 200000000ull);
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
@@ -222,7 +222,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             for (int i = 0; i < nloc && ok; ++i) {
                 const int s = i & 1;
                 const uint32_t par = i & 1;
-                const uint32_t qwk = base_u32 + Ly.qwk[s], lzt = base_u32 + Ly.lzt[s];
+                const uint32_t qwk = base_u32 + stage(Ly.qwk, s), lzt = base_u32 + stage(Ly.lzt, s);
                 const uint32_t rb = tmem + T_R + 128 * s;
                 if (!(ok = wait_or_abort(&bars[FULLX0 + s], (i >> 1) & 1, abort_flag)))
                     break;
@@ -233,7 +233,7 @@ split128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 // U = [0; T] V into rows 64-127 of R(s), zeros into 0-63
                 for (int k0 = 0; k0 < CC; k0 += 16)
                     mma_bf16(rb, desc_kmajor(lzt + 64 * 128, 128, 0, k0),
-                             desc_mnmajor(base_u32 + Ly.v[s], 64, k0, 0), id128, k0 > 0);
+                             desc_mnmajor(base_u32 + stage(Ly.v, s), 64, k0, 0), id128, k0 > 0);
                 if (pair)
                     mma_commit(&bars[VFREE]);
                 if (!(ok = wait_or_abort(&bars[S_READY], par, abort_flag)))
