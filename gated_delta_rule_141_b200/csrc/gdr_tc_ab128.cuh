@@ -17,10 +17,9 @@
 // Value tiles beyond the first of a key head (dv > 128, or several value heads per
 // key head) run the value chain alone.
 //
-// Operands are stacked so that M = 128 with the chain's rows in 0-63; rows 64-127
-// of the R buffers hold products nobody reads:
-//   [T; *] V -> U (rows 0-63),  [-W; Khat] S -> U - W S = E (rows 0-63),
-//   Khat^T E onto F S.
+// The chunk's rows need only M = 64 products (the 64-row accumulator puts row m in
+// tensor-memory lane 32 (m / 16) + m % 16):
+//   T V -> U,  -W S onto it -> E = U - W S,  Khat^T E onto F S (M = dk = 128).
 // Tensor memory: R_A 0, R_B 128, S_A 256, S_B 384 (fp32, 128 columns each).
 // Pairs (the chunk-128 Neumann inverses run as 64-token halves): a second half adds
 // the first half's correction, E2 += Y E1, as one more product [Y; *] E1 onto its R
@@ -29,7 +28,7 @@
 //
 // Roles: warp 0 producer (W, Khat, F), warp 1 MMA issuer, warp 2 producer (T, V),
 // warp 3 idle, warps 4-19 state (S row in TMEM lane 32 (w % 4) + lane, 32 of the
-// 128 columns each; E rows in lanes 0-63, warps with w % 4 < 2).
+// 128 columns each; E row 16 (w % 4) + lane in lanes 0-15 of every warp).
 
 namespace split {
 
@@ -52,9 +51,7 @@ struct Plan {
 };
 
 // Stage: [-W | Khat] (rows 0-63 | 64-127, two 64-column blocks), then T (64 rows)
-// directly followed by V (64 rows, two 64-column blocks): the U product's A operand
-// is the 128 rows from T, whose lower half (V's first block) only feeds rows that
-// nobody reads.
+// and V (64 rows, two 64-column blocks).
 __host__ __device__ inline Plan plan(bool pair = false)
 {
     Plan s;
@@ -176,7 +173,7 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t id128 = idesc_bf16(128, NV, false, true);
+            const uint32_t id64 = idesc_bf16(64, NV, false, true);
             const uint32_t id_s = idesc_bf16(KD, NV, true, true);
             auto kstep = [](int k0) {   // K-major A of 128 rows, 64-column blocks
                 return static_cast<uint64_t>(((k0 >> 6) * 128 * 128 + (k0 & 63) * 2) >> 4);
@@ -199,9 +196,9 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 tc_fence_after();
                 // U = [T; *] V into R_A (E_A of the previous chunk has been read)
                 for (int k0 = 0; k0 < CC; k0 += 16)
-                    mma_bf16(tr(0), desc_kmajor(tv, 128, 0, k0), desc_mnmajor(tv + prep::IMG, 64, k0, 0),
-                             id128, k0 > 0);
-                // [-W; Khat] S: E = U - W S into rows 0-63 (value chain), -W S (transition)
+                    mma_bf16(tr(0), desc_kmajor(tv, 64, 0, k0), desc_mnmajor(tv + prep::IMG, 64, k0, 0),
+                             id64, k0 > 0);
+                // -W S: E = U - W S (value chain), -W S (transition)
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (x >= nch || !ok)
@@ -210,12 +207,12 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                         break;
                     tc_fence_after();
                     for (int k0 = 0; k0 < KD; k0 += 16)
-                        mma_bf16(tr(x), desc_kmajor(wk, 128, 0, 0) + kstep(k0), d_s(x) + mstep(k0), id128,
+                        mma_bf16(tr(x), desc_kmajor(wk, 128, 0, 0) + kstep(k0), d_s(x) + mstep(k0), id64,
                                  (x == 0 || k0 > 0) ? 1u : 0u);
-                    if (pair && s == 1)   // second half: + Y E1 (rows 0-63)
+                    if (pair && s == 1)   // second half: + Y E1
                         for (int k0 = 0; k0 < CC; k0 += 16)
                             mma_bf16(tr(x), desc_kmajor(base_u32 + Ly.y, 128, 0, k0), d_e(x) + mstep(k0),
-                                     id128, 1u);
+                                     id64, 1u);
                     mma_commit(&bars[P_FULL_A + x]);
                 }
                 // S <- F S + Khat^T E
@@ -266,10 +263,10 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             const int s = i & 1;
             const uint32_t par = i & 1;
             // S phases: S_{c-1} -> bf16 operand, then F S_{c-1} back (the update accumulates onto it)
-    #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            if (x >= nch)
-                break;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                if (x >= nch)
+                    break;
                 if (i >= 1 && named_vote_or(NB_STATE, N_STATE,
                                             !wait_or_abort(&bars[UPD_A + x], par ^ 1u, abort_flag))) {
                     ok = false;
@@ -302,11 +299,11 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
             }
             if (!ok)
                 break;
-            // E phases: E from rows 0-63 of R -> bf16 operand of the update
-    #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            if (x >= nch)
-                break;
+            // E phases: E from R -> bf16 operand of the update
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                if (x >= nch)
+                    break;
                 if (named_vote_or(NB_STATE, N_STATE, !wait_or_abort(&bars[P_FULL_A + x], par, abort_flag))) {
                     ok = false;
                     break;
@@ -314,14 +311,17 @@ ab128_kernel(const __grid_constant__ CUtensorMap tm_v, const SplitArgs args)
                 if (x == 0 && stid == 0)   // every state thread has read F (the vote above)
                     mbar_arrive(&bars[FREE0 + s]);
                 tc_fence_after();
-                if (R < CC) {
+                {   // E row t = 16 (w % 4) + lane in lanes 0-15 (M = 64 accumulator)
                     float ev[32];
                     tmem_ld16(tr(x), *reinterpret_cast<float(*)[16]>(&ev[0]));
                     tmem_ld16(tr(x) + 16, *reinterpret_cast<float(*)[16]>(&ev[16]));
                     tmem_ld_wait();
+                    if (lane < 16) {
+                        const int t = 16 * (warp & 3) + lane;
 #pragma unroll
-                    for (int n = 0; n < 32; n += 8)
-                        st_tile8(E_T(x), CC, R, cs + n, &ev[n]);
+                        for (int n = 0; n < 32; n += 8)
+                            st_tile8(E_T(x), CC, t, cs + n, &ev[n]);
+                    }
                 }
                 tmem_st_wait();
                 fence_proxy_async_smem();
