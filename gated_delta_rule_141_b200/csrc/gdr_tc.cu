@@ -705,7 +705,7 @@ int launch_tc2(const Params &p0, void *workspace, cudaStream_t stream)
     const bool wide = split::use128(p);   // the 128-column state pass (stores -W)
     rc = prep::launch<128>(p, workspace, kind, stream, p.pair, wide ? 1 : 0);
     if (rc == 0 && p.pair)
-        rc = pair::launch<128>(p, workspace, stream);
+        rc = pair::launch<128>(p, workspace, stream, wide ? 1 : 0);
     if (rc != 0)
         return rc;
     if (wide)

@@ -67,7 +67,7 @@ __host__ __device__ inline Plan plan()
     // Newton residual; first the G21 operands (two 64 x dk tiles)
     s.RT = take(2 * 128 * 128 > 2 * CC * DK * 2 ? 2 * 128 * 128 : 2 * CC * DK * 2);
     s.Tf = take(32 * 36 * 4 + 1024);    // scratch of the fp32 block inverse
-    s.beta = take(3 * CC * 4);          // beta2, then (scalar gate) ea2, eb1
+    s.beta = take(4 * CC * 4);          // beta2, then (scalar gate) ea2, eb1, then beta1
     s.bar = take(64);
     s.misc = s.bar + 32;
     s.total = o + 1024;
@@ -81,6 +81,8 @@ struct PairArgs {
     uint32_t rec_bytes;
     uint32_t base_bytes;      // offset of the pair extras in a record
     int ext;                  // grouped / per-channel records (else the scalar gate's)
+    int defer_tw;             // the first pass left the halves' T and W to this kernel
+    int neg_w;                // ... and the state pass reads -W
 };
 
 // fp32 views of the regions freed once the series is done (stride LDM)
@@ -99,7 +101,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
     const uint32_t NTL = base_u32 + Ly.NTL, XT = base_u32 + Ly.XT, RT = base_u32 + Ly.RT;
     float *Tf = f32(base, Ly.Tf);
     float *sbeta = f32(base, Ly.beta);          // beta of half 2
-    float *ea2 = sbeta + CC, *eb1 = sbeta + 2 * CC;
+    float *ea2 = sbeta + CC, *eb1 = sbeta + 2 * CC, *beta1 = sbeta + 3 * CC;
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + Ly.bar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + Ly.misc);
 
@@ -124,6 +126,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
     if (tid == 0) {
         mbar_init(&bars[0], 1);   // loads
         mbar_init(&bars[1], 1);   // MMA
+        mbar_init(&bars[2], 1);   // Kbar of the first half (deferred T and W)
         fence_barrier_init();
         uint64_t *full = &bars[0];
         const uint32_t opnd = (uint32_t)(CC * DK * 2);   // one 64-row operand tile
@@ -148,6 +151,8 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
     }
     for (int t = tid; t < CC; t += NT) {
         sbeta[t] = t < Cl2 ? p.beta[kh * T + c0_2 + t] : 0.f;
+        if (a.defer_tw)
+            beta1[t] = p.beta[kh * T + (long)c1 * CC + t];   // a first half is whole
         if (!a.ext) {   // e^{Lambda_t} of half 2, e^{Lambda_mid - Lambda_j} of half 1
             ea2[t] = reinterpret_cast<const float *>(rec2 + prep::SC_EA)[t];
             eb1[t] = reinterpret_cast<const float *>(rec1 + prep::SC_EB)[t];
@@ -174,6 +179,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
 
     uint32_t ph_mma = 0;
     bool failed = false;
+    bool kb_sent = false;    // (thread 0) the halves' Kbar are on their way
     auto wait_bar = [&](int i, uint32_t ph) {
         const bool gave_up = !mbar_wait(&bars[i], ph);
         if (gave_up)
@@ -318,6 +324,83 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+    }
+
+    // ---- the halves' own T and W, left by the first pass: T_h = diag(beta_h) A_hh =
+    //      Atil_hh diag(beta_h), Atil_hh the h-th diagonal block of X (the half's own
+    //      series), and W_h = T_h Kbar_h (M = 64, N = dk, K = 64), into the halves' records
+    //      as the first pass would have written them (W negated for the 128-column pass)
+    if (!failed && a.defer_tw && tid == 0) {   // both halves' Kbar over the dead residual tile
+        const uint32_t opnd = (uint32_t)(CC * DK * 2);
+        kb_sent = true;
+        mbar_arrive_expect_tx(&bars[2], 2u * opnd);
+        bulk_load(base + Ly.RT, rec1 + a.base_bytes + prep::PAIR_KB, opnd, &bars[2]);
+        bulk_load(base + Ly.RT + opnd, rec2 + a.base_bytes + prep::PAIR_KB, opnd, &bars[2]);
+    }
+    for (int h = 0; h < 2 && !failed && a.defer_tw; ++h) {
+        uint8_t *rec = h == 0 ? rec1 : rec1 + a.rec_bytes;
+        const float *bh = h == 0 ? beta1 : sbeta;
+        const uint32_t TBh = XT + h * 8192;      // X's bf16 operand is dead
+        tc_fence_after();
+        if ((R < 64) == (h == 0) && ch == 64 * h) {   // warps holding rows of the block
+            const int r = R - 64 * h;
+            for (int c = 0; c < 64; c += 16) {
+                float x[16];
+                tmem_ld16(tq + T_X + ch + c, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    x[e] *= bh[c + e];
+                prep::st_img8(rec, r, c, &x[0]);
+                prep::st_img8(rec, r, c + 8, &x[8]);
+                st_tile8(TBh, 64, r, c, &x[0]);
+                st_tile8(TBh, 64, r, c + 8, &x[8]);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (h == 0 && (failed = wait_bar(2, 0)))
+            break;
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(64, DK, false, true);
+            const uint32_t KBh = RT + h * (uint32_t)(CC * DK * 2);
+            for (int k0 = 0; k0 < CC; k0 += 16)
+                mma_bf16(tmem + T_D, desc_kmajor(TBh, 64, 0, k0), desc_mnmajor(KBh, 64, k0, 0), id, k0 > 0);
+            mma_commit(&bars[1]);
+        }
+        failed = wait_bar(1, ph_mma);
+        ph_mma ^= 1u;
+        if (!failed) {
+            tc_fence_after();
+            const int rr = gen::row64g(warp, lane);
+            const int cw = (DK / 2) * (warp >> 2);   // this warp's half of the dk columns
+#pragma unroll
+            for (int cb = 0; cb < DK / 2; cb += 32) {
+                float w0[16], w1[16];
+                tmem_ld16(tq + T_D + cw + cb, w0);
+                tmem_ld16(tq + T_D + cw + cb + 16, w1);
+                tmem_ld_wait();
+                if (rr >= 0) {
+                    if (a.neg_w) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            w0[e] = -w0[e];
+                            w1[e] = -w1[e];
+                        }
+                    }
+                    const int col = cw + cb;   // 32 columns inside one 64-column image
+                    uint8_t *img_W = rec + prep::REC_W + (col >> 6) * prep::IMG;
+                    prep::st_img8(img_W, rr, col & 63, &w0[0]);
+                    prep::st_img8(img_W, rr, (col & 63) + 8, &w0[8]);
+                    prep::st_img8(img_W, rr, (col & 63) + 16, &w1[0]);
+                    prep::st_img8(img_W, rr, (col & 63) + 24, &w1[8]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();   // the product is read back before the next one lands there
     }
 
     if (!p.neumann1) {
@@ -489,6 +572,8 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         mma_commit(&bars[1]);
         mbar_wait(&bars[1], ph_mma, 200000000ull);
         mbar_wait(&bars[0], 0, 200000000ull);
+        if (kb_sent)
+            mbar_wait(&bars[2], 0, 200000000ull);
     }
     tc_fence_before();
     __syncthreads();
@@ -501,7 +586,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
 inline int npairs(int nchunks) { return (nchunks + 1) / 2; }
 
 template <int DK>
-int launch(const Params &p, void *records, cudaStream_t stream)
+int launch(const Params &p, void *records, cudaStream_t stream, int neg_w = 0)
 {
     const int N = prep::nchunks(p);
     if (N == 0 || p.B == 0)
@@ -520,6 +605,10 @@ int launch(const Params &p, void *records, cudaStream_t stream)
     a.rec_bytes = prep::rec_bytes(p);
     a.base_bytes = prep::kind_bytes(prep::record_kind(p), DK);
     a.ext = prep::record_kind(p) == prep::REC_EXT;
+    // the first pass leaves T and W of paired halves here (truncated Neumann, dk = 128,
+    // grouped / per-channel records): the same condition as its own
+    a.defer_tw = DK == 128 && a.ext && p.neumann && !p.neumann1;
+    a.neg_w = neg_w;
     pair_kernel<DK><<<dim3(npairs(N), p.Hk, p.B), NT, Ly.total, stream>>>(mk, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }

@@ -824,7 +824,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 Mf[t * LDM + j0 + e] = mv[e];
         }
     }
-    if (!failed) {
+    // A chunk-128 truncated Neumann pair (grouped / per-channel records, dk = 128) leaves its
+    // halves' T and W to the pair kernel, whose 128-token series holds both halves' own
+    // series as its diagonal blocks; an unpaired last half computes its own.
+    const bool defer = DK == 128 && a.pair && neu && ext && ((c & 1) || c + 1 < a.nchunks);
+    if (!failed && !defer) {
         if (tid == 0 && (SCALAR || (RL && neu)))   // T or the Neumann operands land on L's staging
             bulk_wait_read();
         __syncthreads();
@@ -976,7 +980,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         //      For W the same chunk goes to the bf16 operand tile in the dead q rows,
         //      scaled by e^{Lambda_j} for the scalar gate (W = T diag(e^Lambda) K).
         const uint32_t TB = base_u32 + Ly.TB;
-        for (int u = tid; u < CC * 8; u += NT) {
+        for (int u = tid; u < (defer ? 0 : CC * 8); u += NT) {
             const int r = u >> 3, cc = (u & 7) ^ (r & 7);
             const float bt = sbeta[r];
             const float4 x0 = *reinterpret_cast<const float4 *>(&Mf[r * LDM + 8 * cc]);
@@ -999,7 +1003,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
         }
-        if (with_w) {
+        if (with_w && !defer) {
             // ---- W = TB Kbar (M = 64, N = dk, K = 64) on tcgen05, read back as an image
             fence_proxy_async_smem();
             if (tid == 0 && DK > 128)   // W's staging is L's
