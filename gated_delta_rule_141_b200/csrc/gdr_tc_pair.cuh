@@ -274,7 +274,62 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
             tmem_st16(tq + T_X + c, x);
         }
     }
-    for (int pw = 1; pw <= p.neu_order && !failed; ++pw) {   // X <- I - Ntil X
+    // order 4 (the default): X = I - N + N^2 - N^3 + N^4 = (I + P2) - N (I + P2) + P2 P2 with
+    // P2 = N^2, two product round trips instead of Horner's four (the same series, other
+    // rounding); the B operand -(I + P2) makes the sum one accumulation
+    const bool quad = p.neu_order == 4;
+    if (!failed && quad) {
+        if (!(failed = product(NTL, NTL))) {
+            for (int c = ch; c < ch + 64; c += 16) {
+                float d[16], x[16];
+                tmem_ld16(tq + T_D + c, d);
+                tmem_ld_wait();
+                tmem_st16(tq + T_X + c, d);                      // P2, fp32
+                st_tile8(RT, 128, R, c, &d[0]);                  // P2 (bf16, both operands)
+                st_tile8(RT, 128, R, c + 8, &d[8]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    x[e] = -(((R == c + e) ? 1.f : 0.f) + d[e]);
+                st_tile8(XT, 128, R, c, &x[0]);                  // -(I + P2)
+                st_tile8(XT, 128, R, c + 8, &x[8]);
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+        }
+        if (!failed) {
+            if (tid == 0) {
+                tc_fence_after();
+                for (int k0 = 0; k0 < 128; k0 += 16)
+                    mma_bf16(tmem + T_D, desc_kmajor(NTL, 128, 0, k0), desc_mnmajor(XT, 128, k0, 0), id128,
+                             k0 > 0);
+                for (int k0 = 0; k0 < 128; k0 += 16)
+                    mma_bf16(tmem + T_D, desc_kmajor(RT, 128, 0, k0), desc_mnmajor(RT, 128, k0, 0), id128, 1u);
+                mma_commit(&bars[1]);
+            }
+            failed = wait_bar(1, ph_mma);
+            ph_mma ^= 1u;
+        }
+        if (!failed) {
+            tc_fence_after();
+            for (int c = ch; c < ch + 64; c += 16) {
+                float d[16], x[16];
+                tmem_ld16(tq + T_D + c, d);
+                tmem_ld16(tq + T_X + c, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    x[e] += ((R == c + e) ? 1.f : 0.f) + d[e];
+                put_x(c, x);
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+        }
+    }
+    for (int pw = 1; pw <= (quad ? 0 : p.neu_order) && !failed; ++pw) {   // X <- I - Ntil X
         if ((failed = product(NTL, XT)))
             break;
         for (int c = ch; c < ch + 64; c += 16) {

@@ -763,9 +763,8 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
         fetch(0);
     for (int g = 0; g < a.nseg; ++g) {
         float *st = a.seg_start + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            st[j] = sv[j];
+        *reinterpret_cast<float4 *>(st) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+        *reinterpret_cast<float4 *>(st + 4) = make_float4(sv[4], sv[5], sv[6], sv[7]);
         if (g + 1 == a.nseg)
             break;
         cp_async_wait_all();   // Atil_g has landed (this thread's share)
@@ -779,14 +778,26 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
         const float *As = cmb + (g & 1) * KD * CMB_LDA;
         const float *Bt = a.seg_end + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
         float acc[8];
+        {
+            const float4 b0 = *reinterpret_cast<const float4 *>(Bt);
+            const float4 b1 = *reinterpret_cast<const float4 *>(Bt + 4);
+            acc[0] = b0.x; acc[1] = b0.y; acc[2] = b0.z; acc[3] = b0.w;
+            acc[4] = b1.x; acc[5] = b1.y; acc[6] = b1.z; acc[7] = b1.w;
+        }
+        // the inner index four at a time (one float4 of Atil's row, two of each S row),
+        // still in ascending order
+        for (int l = 0; l < KD; l += 4) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(&As[r * CMB_LDA + l]);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            acc[j] = Bt[j];
-        for (int l = 0; l < KD; ++l) {
-            const float al = As[r * CMB_LDA + l];
+            for (int u = 0; u < 4; ++u) {
+                const float4 s0 = *reinterpret_cast<const float4 *>(&Ss[(l + u) * CMB_COLS + j0]);
+                const float4 s1 = *reinterpret_cast<const float4 *>(&Ss[(l + u) * CMB_COLS + j0 + 4]);
+                const float sj[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                acc[j] += al * Ss[l * CMB_COLS + j0 + j];
+                for (int j = 0; j < 8; ++j)
+                    acc[j] += av[u] * sj[j];
+            }
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j)

@@ -91,6 +91,8 @@ WIDE_PAIRS = [
     (4, dict(B=2, Hk=2, Hv=4, T=64 * 66 + 3), "neumann"),
     (2, dict(B=1, Hk=1, Hv=1, T=64 * 48, dv=256, gate_mode=W.GATE_GROUP64), "neumann1"),
     (2, dict(B=1, Hk=1, Hv=2, T=64 * 52 - 9), "neumann1"),
+    # weak decay: the halves' W (written by the pair kernel) weigh on every output
+    (2, dict(B=1, Hk=1, Hv=2, T=64 * 52 - 9), "neumann"),
 ]
 
 
