@@ -34,7 +34,7 @@
 //   4. Atil11^{-1} exactly in fp32 (block doubling), then Y on tcgen05 from split
 //      bf16 operands (hi + lo parts: fp32-level products, which the cancellation
 //      between Y's two terms needs); (the 1-Step Neumann inverse of §2.4.3 instead
-//      of 3: Atil from the diagonal 16 x 16 blocks, Y in fp32 on the CUDA cores;)
+//      of 3: Atil from the diagonal 16 x 16 blocks in fp32, Y the same way;)
 //   5. Y as a bf16 image into the first half's record.
 // The state passes add Y E1 to the second half's E: the 64-column pass through an
 // [L; Y] tile whose E product of the first half leaves Y E1 in tensor memory, the
@@ -179,7 +179,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
 
     uint32_t ph_mma = 0;
     bool failed = false;
-    bool kb_sent = false;    // (thread 0) the halves' Kbar are on their way
+    int kb_loads = 0;        // (thread 0) phases armed on the Kbar barrier
     auto wait_bar = [&](int i, uint32_t ph) {
         const bool gave_up = !mbar_wait(&bars[i], ph);
         if (gave_up)
@@ -385,14 +385,15 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
     //      Atil_hh diag(beta_h), Atil_hh the h-th diagonal block of X (the half's own
     //      series), and W_h = T_h Kbar_h (M = 64, N = dk, K = 64), into the halves' records
     //      as the first pass would have written them (W negated for the 128-column pass)
-    if (!failed && a.defer_tw && tid == 0) {   // both halves' Kbar over the dead residual tile
+    const bool tw_series = a.defer_tw && !p.neumann1;   // (1-Step Neumann: in its branch below)
+    if (!failed && tw_series && tid == 0) {   // both halves' Kbar over the dead residual tile
         const uint32_t opnd = (uint32_t)(CC * DK * 2);
-        kb_sent = true;
+        kb_loads = 1;
         mbar_arrive_expect_tx(&bars[2], 2u * opnd);
         bulk_load(base + Ly.RT, rec1 + a.base_bytes + prep::PAIR_KB, opnd, &bars[2]);
         bulk_load(base + Ly.RT + opnd, rec2 + a.base_bytes + prep::PAIR_KB, opnd, &bars[2]);
     }
-    for (int h = 0; h < 2 && !failed && a.defer_tw; ++h) {
+    for (int h = 0; h < 2 && !failed && tw_series; ++h) {
         uint8_t *rec = h == 0 ? rec1 : rec1 + a.rec_bytes;
         const float *bh = h == 0 ? beta1 : sbeta;
         const uint32_t TBh = XT + h * 8192;      // X's bf16 operand is dead
@@ -579,6 +580,74 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
             __syncthreads();
             gen::block_neumann1_64_inplace(A11f, Tf, tid);
             gen::block_neumann1_64_inplace(A22f, Tf, tid);
+            // the halves' own T and W, left by the first pass: T_h = Atil_hh diag(beta_h) from
+            // the fp32 blocks, W_h = T_h Kbar_h, one half at a time in the residual tile's
+            // dead tail (Atil11's last rows end 2 KB into it)
+            for (int h = 0; h < 2 && a.defer_tw && !failed; ++h) {
+                uint8_t *rec = h == 0 ? rec1 : rec1 + a.rec_bytes;
+                const float *Ah = h == 0 ? A11f : A22f;
+                const float *bh = h == 0 ? beta1 : sbeta;
+                const uint32_t TBs = RT + 8192, KBs = RT + 16384;
+                if (tid == 0) {
+                    const uint32_t opnd = (uint32_t)(CC * DK * 2);
+                    kb_loads = h + 1;
+                    mbar_arrive_expect_tx(&bars[2], opnd);
+                    bulk_load(base + Ly.RT + 16384, rec + a.base_bytes + prep::PAIR_KB, opnd, &bars[2]);
+                }
+                for (int u = tid; u < CC * 8; u += NT) {
+                    const int r = u >> 3, c = (u & 7) * 8;
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        v[e] = Ah[r * LDM + c + e] * bh[c + e];
+                    prep::st_img8(rec, r, c, v);
+                    st_tile8(TBs, 64, r, c, v);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                if ((failed = wait_bar(2, (uint32_t)h)))
+                    break;
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(64, DK, false, true);
+                    for (int k0 = 0; k0 < CC; k0 += 16)
+                        mma_bf16(tmem + T_D, desc_kmajor(TBs, 64, 0, k0), desc_mnmajor(KBs, 64, k0, 0), id,
+                                 k0 > 0);
+                    mma_commit(&bars[1]);
+                }
+                failed = wait_bar(1, ph_mma);
+                ph_mma ^= 1u;
+                if (failed)
+                    break;
+                tc_fence_after();
+                const int rr = gen::row64g(warp, lane);
+                const int cw = (DK / 2) * (warp >> 2);
+#pragma unroll
+                for (int cb = 0; cb < DK / 2; cb += 32) {
+                    float w0[16], w1[16];
+                    tmem_ld16(tq + T_D + cw + cb, w0);
+                    tmem_ld16(tq + T_D + cw + cb + 16, w1);
+                    tmem_ld_wait();
+                    if (rr >= 0) {
+                        if (a.neg_w) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                w0[e] = -w0[e];
+                                w1[e] = -w1[e];
+                            }
+                        }
+                        const int col = cw + cb;
+                        uint8_t *img_W = rec + prep::REC_W + (col >> 6) * prep::IMG;
+                        prep::st_img8(img_W, rr, col & 63, &w0[0]);
+                        prep::st_img8(img_W, rr, (col & 63) + 8, &w0[8]);
+                        prep::st_img8(img_W, rr, (col & 63) + 16, &w1[0]);
+                        prep::st_img8(img_W, rr, (col & 63) + 24, &w1[8]);
+                    }
+                }
+                tc_fence_before();
+                __syncthreads();   // read back (and the tiles read) before the next half
+            }
             const int rg = tid >> 4, c0 = 4 * (tid & 15), lb = c0 & ~15, lr = 16 * (rg >> 2);
             float acc[4][4];
             // Z = Ntil21 bd(Atil11): rows rg + 16 i, columns c0..c0+3 (one 16-column block)
@@ -604,22 +673,96 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
             }
             __syncthreads();
         }
+        // ---- Y = Atil21 Atil11^{-1} + Atil22 Ntil21 on tcgen05 from split bf16 operands, as in
+        //      the truncated series' branch, in two stages for want of free tiles beside the
+        //      fp32 blocks: Atil22 Ntil21 (Ntil21 exact in bf16), then Atil21 Atil11^{-1} onto it
+        auto split_store = [&](uint32_t th, uint32_t tl, int r, int c, const float *v) {
+            float hi[8], lo[8];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const uint32_t hh = pack_bf16(v[e], v[e + 1]);
+                hi[e] = bf16lo(hh);
+                hi[e + 1] = bf16hi(hh);
+                lo[e] = v[e] - hi[e];
+                lo[e + 1] = v[e + 1] - hi[e + 1];
+            }
+            st_tile8(th, 64, r, c, hi);
+            st_tile8(tl, 64, r, c, lo);
+        };
+        const uint32_t id64 = idesc_bf16(64, 64, false, true);
         if (!failed) {
             gen::inverse64_par(A11f, Tf, tid);                // Atil11^{-1}, lower triangular
-            const int rg = tid >> 4, c0 = 4 * (tid & 15);     // rows rg + 16 i, columns c0..c0+3
-            float y[4][4], z[4][4];
-            gen::block_product4x4<64>(y, A21f + rg * LDM, 16 * LDM, A11f + c0, LDM, c0);
-            gen::block_product4x4<64>(z, A22f + rg * LDM, 16 * LDM, N21f + c0, LDM, 0);
-            __syncthreads();                                  // every read of A21f done
+            // stage 1 tiles: Ntil21 over the first 8 KB of its fp32 copy (read out first),
+            // Atil22 high / low past the fp32 blocks in the residual and Ntil tiles
+            const uint32_t N21T = XT, A22H = RT + 20480, A22L = NTL + 18432;
+            float nv[2][8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int k = 0; k < 2; ++k) {
+                const int u = tid + NT * k, r = u >> 3, c = (u & 7) * 8;
 #pragma unroll
-                for (int n = 0; n < 4; ++n)
-                    A21f[(rg + 16 * i) * LDM + c0 + n] = y[i][n] + z[i][n];
+                for (int e = 0; e < 8; ++e)
+                    nv[k][e] = N21f[r * LDM + c + e];
+                split_store(A22H, A22L, r, c, A22f + r * LDM + c);
+            }
             __syncthreads();
-            for (int u = tid; u < CC * 8; u += NT) {          // Y as a 128-byte-swizzled image
-                const int t = u >> 3, j0 = (u & 7) * 8;
-                prep::st_img8(img_Y, t, j0, A21f + t * LDM + j0);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int u = tid + NT * k;
+                st_tile8(N21T, 64, u >> 3, (u & 7) * 8, nv[k]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                for (int k0 = 0; k0 < CC; k0 += 16) {
+                    const uint64_t n21 = desc_mnmajor(N21T, 64, k0, 0);
+                    mma_bf16(tmem + T_D, desc_kmajor(A22H, 64, 0, k0), n21, id64, k0 > 0);
+                    mma_bf16(tmem + T_D, desc_kmajor(A22L, 64, 0, k0), n21, id64, 1u);
+                }
+                mma_commit(&bars[1]);
+            }
+            failed = wait_bar(1, ph_mma);
+            ph_mma ^= 1u;
+        }
+        if (!failed) {
+            // stage 2 tiles: over the dead fp32 Ntil21 / Atil22 and stage 1's Atil22 high part
+            const uint32_t A21H = XT + 8192, A21L = NTL, IH = NTL + 8192, IL = RT + 20480;
+            for (int u = tid; u < CC * 8; u += NT) {
+                const int r = u >> 3, c = (u & 7) * 8;
+                split_store(A21H, A21L, r, c, A21f + r * LDM + c);
+                split_store(IH, IL, r, c, A11f + r * LDM + c);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                for (int k0 = 0; k0 < CC; k0 += 16) {
+                    const uint64_t a21h = desc_kmajor(A21H, 64, 0, k0), a21l = desc_kmajor(A21L, 64, 0, k0);
+                    const uint64_t ih = desc_mnmajor(IH, 64, k0, 0), il = desc_mnmajor(IL, 64, k0, 0);
+                    mma_bf16(tmem + T_D, a21h, ih, id64, 1u);
+                    mma_bf16(tmem + T_D, a21h, il, id64, 1u);
+                    mma_bf16(tmem + T_D, a21l, ih, id64, 1u);
+                }
+                mma_commit(&bars[1]);
+            }
+            failed = wait_bar(1, ph_mma);
+            ph_mma ^= 1u;
+        }
+        if (!failed) {   // Y (M = 64 accumulator: rows in lanes 0-15 of each quarter) as an image
+            tc_fence_after();
+            const int rr = gen::row64g(warp, lane);
+            const int cb = 32 * (warp >> 2);
+            float d0[16], d1[16];
+            tmem_ld16(tq + T_D + cb, d0);
+            tmem_ld16(tq + T_D + cb + 16, d1);
+            tmem_ld_wait();
+            if (rr >= 0) {
+                prep::st_img8(img_Y, rr, cb, &d0[0]);
+                prep::st_img8(img_Y, rr, cb + 8, &d0[8]);
+                prep::st_img8(img_Y, rr, cb + 16, &d1[0]);
+                prep::st_img8(img_Y, rr, cb + 24, &d1[8]);
             }
         }
     }
@@ -627,8 +770,8 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         mma_commit(&bars[1]);
         mbar_wait(&bars[1], ph_mma, 200000000ull);
         mbar_wait(&bars[0], 0, 200000000ull);
-        if (kb_sent)
-            mbar_wait(&bars[2], 0, 200000000ull);
+        if (kb_loads > 0)
+            mbar_wait(&bars[2], (kb_loads - 1) & 1, 200000000ull);
     }
     tc_fence_before();
     __syncthreads();
@@ -660,9 +803,9 @@ int launch(const Params &p, void *records, cudaStream_t stream, int neg_w = 0)
     a.rec_bytes = prep::rec_bytes(p);
     a.base_bytes = prep::kind_bytes(prep::record_kind(p), DK);
     a.ext = prep::record_kind(p) == prep::REC_EXT;
-    // the first pass leaves T and W of paired halves here (truncated Neumann, dk = 128,
+    // the first pass leaves T and W of paired halves here (both Neumann inverses, dk = 128,
     // grouped / per-channel records): the same condition as its own
-    a.defer_tw = DK == 128 && a.ext && p.neumann && !p.neumann1;
+    a.defer_tw = DK == 128 && a.ext && (p.neumann || p.neumann1);
     a.neg_w = neg_w;
     pair_kernel<DK><<<dim3(npairs(N), p.Hk, p.B), NT, Ly.total, stream>>>(mk, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;

@@ -824,10 +824,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 Mf[t * LDM + j0 + e] = mv[e];
         }
     }
-    // A chunk-128 truncated Neumann pair (grouped / per-channel records, dk = 128) leaves its
-    // halves' T and W to the pair kernel, whose 128-token series holds both halves' own
-    // series as its diagonal blocks; an unpaired last half computes its own.
-    const bool defer = DK == 128 && a.pair && neu && ext && ((c & 1) || c + 1 < a.nchunks);
+    // A chunk-128 Neumann pair (grouped / per-channel records, dk = 128) leaves its halves'
+    // T and W to the pair kernel, which holds both halves' own factors as the diagonal
+    // blocks of its 128-token one; an unpaired last half computes its own.
+    const bool defer = DK == 128 && a.pair && (neu || p.neumann1) && ext && ((c & 1) || c + 1 < a.nchunks);
     if (!failed && !defer) {
         if (tid == 0 && (SCALAR || (RL && neu)))   // T or the Neumann operands land on L's staging
             bulk_wait_read();
