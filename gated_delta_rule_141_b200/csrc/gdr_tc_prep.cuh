@@ -583,6 +583,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // ---- two row blocks of 32 tokens, each pivoted at its middle row p = 32r + 16:
         //      rows t of the block carry e^{Lambda_t - Lambda_p}, columns j <= end of the
         //      block carry e^{Lambda_p - Lambda_j}; growth is bounded by a 16-token span
+        // RL: Lambda goes to the record's Qbar / Khat area (rewritten at the end of this path)
+        // and is read back from there, so that the common path keeps no registers for it
+        const float *lsc = reinterpret_cast<const float *>(img_T + ext_qb(DK));
+        auto lam_row = [&](int t, float *o) {   // this thread's eight channels of row t
+            const float4 a0 = *reinterpret_cast<const float4 *>(lsc + t * DK + i0r);
+            const float4 a1 = *reinterpret_cast<const float4 *>(lsc + t * DK + i0r + 4);
+            o[0] = a0.x; o[1] = a0.y; o[2] = a0.z; o[3] = a0.w;
+            o[4] = a1.x; o[5] = a1.y; o[6] = a1.z; o[7] = a1.w;
+        };
+        if constexpr (RL) {
+            float *lw = reinterpret_cast<float *>(img_T + ext_qb(DK));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float *dst = lw + (4 * tb + k) * DK + i0r;
+                *reinterpret_cast<float4 *>(dst) = make_float4(lv[k][0], lv[k][1], lv[k][2], lv[k][3]);
+                *reinterpret_cast<float4 *>(dst + 4) = make_float4(lv[k][4], lv[k][5], lv[k][6], lv[k][7]);
+            }
+            __syncthreads();
+        }
         for (int r = 0; r < 2 && !failed; ++r) {
             const int p0 = 32 * r, pv = p0 + 16, n_r = 32 * (r + 1);
             bool clamp = false;
@@ -626,13 +645,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     lp[e] = lam[(r == 0 ? LR_16 : LR_48) * DK + i0r + e];
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < 4; ++k) {
                     const int t = 4 * tb + k;
+                    float lt[8];
+                    lam_row(t, lt);
                     if (t >= p0 && t < p0 + 32)
-                        operand(true, t, i0r, lv[k], lp);
+                        operand(true, t, i0r, lt, lp);
                     if (t < n_r)
-                        operand(false, t, i0r, lp, lv[k]);
+                        operand(false, t, i0r, lp, lt);
                 }
             } else {
                 for (int u = tid; u < (32 + n_r) * (DK / 8); u += NT) {
@@ -708,18 +729,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             __syncthreads();
             // blocks whose decay span overran the guard: exact fp32 rows from the raw tiles
-            // (RL: Lambda is spilled to the record's Qbar / Khat area first, rewritten below)
-            const float *lsc = reinterpret_cast<const float *>(img_T + ext_qb(DK));
-            if (RL && (flag[0] || flag[1])) {
-                float *lw = reinterpret_cast<float *>(img_T + ext_qb(DK));
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float *dst = lw + (4 * tb + k) * DK + i0r;
-                    *reinterpret_cast<float4 *>(dst) = make_float4(lv[k][0], lv[k][1], lv[k][2], lv[k][3]);
-                    *reinterpret_cast<float4 *>(dst + 4) = make_float4(lv[k][4], lv[k][5], lv[k][6], lv[k][7]);
-                }
-                __syncthreads();
-            }
+            // (RL: Lambda from the record's Qbar / Khat area)
             for (int r = 0; r < 2; ++r) {
                 if (!flag[r])
                     continue;
@@ -759,15 +769,30 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     st_tile8(Ls, 64, t, j0, lv2);
                 }
             }
-            if constexpr (RL) {   // the state pass's decayed operands, now that the area is free
+            if constexpr (RL) {
+                // this thread's Lambda back, then (the area free) the state pass's decayed
+                // operands and Kbar = k e^{Lambda_t} in place in the raw k rows, the same rows
+                // the same thread has just read
+                float lr[4][8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    lam_row(4 * tb + k, lr[k]);
                 __syncthreads();
                 float lc[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     lc[e] = lam[LR_C * DK + i0r + e];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    raw_operands(4 * tb + k, i0r, lv[k], lc);
+                for (int k = 0; k < 4; ++k) {
+                    const int t = 4 * tb + k;
+                    raw_operands(t, i0r, lr[k], lc);
+                    float kv[8];
+                    ld_tile8(QK, 128, 64 + t, i0r, kv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        kv[e] *= __expf(lr[k][e]);
+                    st_tile8(QK, 128, 64 + t, i0r, kv);
+                }
             }
         }
     }
@@ -779,9 +804,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             bulk_commit();
         }
     }
-    if (!failed && a.kind != REC_PLAIN && !SCALAR && wide) {
+    if (!RL && !failed && a.kind != REC_PLAIN && !SCALAR && wide) {
         // Kbar = k e^{Lambda_t} in place in the raw k rows of the pivoted blocks, before the
         // inverse: the last use of Lambda there, whose tile then holds the Neumann operands
+        // (RL: at the end of the pivoted blocks' path)
         __syncthreads();
         auto kbar = [&](int t, int i0, const float *lt) {
             float kv[8];
@@ -791,17 +817,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 kv[e] *= __expf(lt[e]);
             st_tile8(QK, 128, 64 + t, i0, kv);
         };
-        if constexpr (RL) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                kbar(4 * tb + k, i0r, lv[k]);
-        } else {
-            for (int u = tid; u < CC * (DK / 8); u += NT) {
-                const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                float lt[8];
-                lam8(lam, G, wsh, t, i0, lt);
-                kbar(t, i0, lt);
-            }
+        for (int u = tid; u < CC * (DK / 8); u += NT) {
+            const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
+            float lt[8];
+            lam8(lam, G, wsh, t, i0, lt);
+            kbar(t, i0, lt);
         }
     }
     if (!failed && a.pair) {
