@@ -583,9 +583,10 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // ---- two row blocks of 32 tokens, each pivoted at its middle row p = 32r + 16:
         //      rows t of the block carry e^{Lambda_t - Lambda_p}, columns j <= end of the
         //      block carry e^{Lambda_p - Lambda_j}; growth is bounded by a 16-token span
-        // RL: Lambda goes to the record's Qbar / Khat area (rewritten at the end of this path)
-        // and is read back from there, so that the common path keeps no registers for it
-        const float *lsc = reinterpret_cast<const float *>(img_T + ext_qb(DK));
+        // RL: Lambda goes to the record's T / L / W area (written after this path: L leaves
+        // from its staging tile, T and W after the inverse) and is read back from there, so
+        // that the common path keeps no registers for it
+        const float *lsc = reinterpret_cast<const float *>(img_T);
         auto lam_row = [&](int t, float *o) {   // this thread's eight channels of row t
             const float4 a0 = *reinterpret_cast<const float4 *>(lsc + t * DK + i0r);
             const float4 a1 = *reinterpret_cast<const float4 *>(lsc + t * DK + i0r + 4);
@@ -593,7 +594,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             o[4] = a1.x; o[5] = a1.y; o[6] = a1.z; o[7] = a1.w;
         };
         if constexpr (RL) {
-            float *lw = reinterpret_cast<float *>(img_T + ext_qb(DK));
+            float *lw = reinterpret_cast<float *>(img_T);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 float *dst = lw + (4 * tb + k) * DK + i0r;
@@ -729,7 +730,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             __syncthreads();
             // blocks whose decay span overran the guard: exact fp32 rows from the raw tiles
-            // (RL: Lambda from the record's Qbar / Khat area)
+            // (RL: Lambda from the record)
             for (int r = 0; r < 2; ++r) {
                 if (!flag[r])
                     continue;
@@ -770,27 +771,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
             if constexpr (RL) {
-                // this thread's Lambda back, then (the area free) the state pass's decayed
-                // operands and Kbar = k e^{Lambda_t} in place in the raw k rows, the same rows
-                // the same thread has just read
-                float lr[4][8];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    lam_row(4 * tb + k, lr[k]);
+                // the state pass's decayed operands and Kbar = k e^{Lambda_t} in place in the
+                // raw k rows (every fp32 row has read them: the barrier), the same rows the same
+                // thread reads for the operands
                 __syncthreads();
                 float lc[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     lc[e] = lam[LR_C * DK + i0r + e];
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < 4; ++k) {
                     const int t = 4 * tb + k;
-                    raw_operands(t, i0r, lr[k], lc);
+                    float lt[8];
+                    lam_row(t, lt);
+                    raw_operands(t, i0r, lt, lc);
                     float kv[8];
                     ld_tile8(QK, 128, 64 + t, i0r, kv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        kv[e] *= __expf(lr[k][e]);
+                        kv[e] *= __expf(lt[e]);
                     st_tile8(QK, 128, 64 + t, i0r, kv);
                 }
             }
