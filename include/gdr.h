@@ -93,9 +93,10 @@ typedef enum { GDR_INV_EXACT = 0, GDR_INV_NEUMANN = 1, GDR_INV_NEUMANN1 = 2 } gd
  *        segment-parallel, with 128 value columns per CTA when that is the
  *        cheaper.
  *  TC2W  TC2 with the 128-column state pass forced (grouped / per-channel
- *        gates, dk = 128, dv % 128 == 0, exact inverse or chunk 64): a test
- *        and benchmark switch; gdr_select_kernel reports TC2 for what AUTO
- *        picks.
+ *        gates, dk = 128, dv % 128 == 0, every inverse mode: the chunk-128
+ *        Neumann inverses as corrected pairs of 64-token halves; no momentum):
+ *        a test and benchmark switch; gdr_select_kernel reports TC2 for what
+ *        AUTO picks.
  *  SIMT  the fp32 CUDA-core kernel (any dtype, chunk 1..128).
  *  SIMT2 the same arithmetic in two passes: the chunk inverse and score matrix
  *        L of every chunk in parallel, written to the caller's workspace
