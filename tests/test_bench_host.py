@@ -46,6 +46,17 @@ def test_variant_oracle_samples():
     assert rate > 0 and "momentum" in desc
 
 
+def test_forward_oracle_sample_is_bounded():
+    # long sequences: a token prefix first (the oracle's cost per token does not depend on
+    # the position), so the timed work stays near the budget; the rate counts B*T tokens
+    w, x = W.workload_inputs(4, T=4096)
+    rate, threads, desc, dt = bench.oracle_sample(w, x, 128, "exact", budget_s=0.05)
+    assert rate > 0 and threads >= 1
+    assert "the first 2048 of their 4096 tokens" in desc, desc
+    n = int(desc.split()[0])
+    assert abs(rate * dt - n * 2048 / w.Hv) <= 1e-6 * rate * dt
+
+
 def test_roofline_arithmetic():
     peaks = {"hbm_gbs": 6448.0, "bf16_tflops": 1726.0}
     # the gdn_scalar_bf16 step: 279 MB and 3.69e10 FLOP in 0.217 ms is HBM-bound
