@@ -37,13 +37,16 @@ namespace {
 constexpr int NT = 256;  // threads per CTA
 
 struct BwdLayout {       // offsets in floats into dynamic shared memory
-    int lam, beta, row, P, A, L, S, dS, Y, dO, dE, dR, DL, DLg, F, X, E1, total;
+    int lam, beta, row, P, A, L, S, dS, Y, dO, dE, dR, DL, DLg, F, X, E1, qk, ldq, total;
     bool tab;            // scalar gate: e^{Lambda_t - Lambda_j} (C x C) and e^{Lambda_t} (C)
-};                       // tabulated in E1
+                         // tabulated in E1
+    bool stage;          // the chunk's q and k rows staged at qk (row stride ldq elements)
+};
 
 constexpr int kBwdSmemFloats = 227 * 1024 / 4;
 
-__host__ __device__ inline BwdLayout bwd_layout(int C, int G, int dk, int NV)
+// in_bytes: the size of an input element (2 for bf16 q, k, v; 4 for fp32)
+__host__ __device__ inline BwdLayout bwd_layout(int C, int G, int dk, int NV, int in_bytes)
 {
     BwdLayout s;
     int off = 0;
@@ -67,9 +70,22 @@ __host__ __device__ inline BwdLayout bwd_layout(int C, int G, int dk, int NV)
     // they fit beside the rest (last, so the other offsets do not move)
     s.tab = G == 1 && off + C * C + C <= kBwdSmemFloats;
     s.E1 = off;   off += s.tab ? C * C + C : 0;
+    // the chunk's q and k rows in the input type, when they fit: every product of the chunk
+    // reads them 2 C to dk times, from here instead of global memory (rows padded by one
+    // word, so that a warp reading one column of many rows meets every bank once)
+    s.ldq = dk + 4 / in_bytes;
+    const int qk_floats = (2 * C * s.ldq * in_bytes + 3) / 4;
+    s.qk = off;
+    s.stage = off + qk_floats <= kBwdSmemFloats;
+    off += s.stage ? qk_floats : 0;
     s.total = off;
     return s;
 }
+
+template <bool BF> struct InElem { using type = float; };
+template <> struct InElem<true> { using type = __nv_bfloat16; };
+__device__ __forceinline__ float in_f(float x) { return x; }
+__device__ __forceinline__ float in_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 template <bool BF>
 __device__ __forceinline__ float ld_in(const void *p, long i)
@@ -91,7 +107,7 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
 {
     extern __shared__ float sm[];
     const int C = p.C, G = p.G, dk = p.dk, dv = p.dv, T = p.T;
-    const BwdLayout Ly = bwd_layout(C, G, dk, NV);
+    const BwdLayout Ly = bwd_layout(C, G, dk, NV, IN_BF16 ? 2 : 4);
     float *lam = sm + Ly.lam, *sbeta = sm + Ly.beta, *row = sm + Ly.row, *P = sm + Ly.P;
     float *A = sm + Ly.A, *L = sm + Ly.L, *S = sm + Ly.S, *dS = sm + Ly.dS, *Y = sm + Ly.Y;
     float *dO = sm + Ly.dO, *dE = sm + Ly.dE, *dR = sm + Ly.dR, *DL = sm + Ly.DL;
@@ -100,6 +116,11 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
     float *Et = E1 + C * C;                   // tab: e^{Lambda_t}
     const int width = dk / G;                 // channels per decay group
     float *DLg = width > 1 ? sm + Ly.DLg : DL;   // per group (the same array when G = dk)
+    using In = typename InElem<IN_BF16>::type;
+    In *qs = reinterpret_cast<In *>(sm + Ly.qk);
+    In *ks = qs + C * Ly.ldq;
+    const bool st = Ly.stage;
+    const int ldq = Ly.ldq;
 
     const int tid = threadIdx.x;
     const int n0 = blockIdx.x * NV;
@@ -118,6 +139,13 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
     for (int c = nch - 1; c >= 0; --c) {
         const int c0 = c * C;
         const int Cl = min(C, T - c0);
+        // q and k of token t (of the chunk) at channel i
+        auto qq = [&](int t, int i) {
+            return st ? in_f(qs[t * ldq + i]) : ld_in<IN_BF16>(p.q, (kh * T + c0 + t) * dk + i);
+        };
+        auto kk = [&](int t, int i) {
+            return st ? in_f(ks[t * ldq + i]) : ld_in<IN_BF16>(p.k, (kh * T + c0 + t) * dk + i);
+        };
         __syncthreads();
         // --- the chunk's start state, gates, Lambda, the dO tile
         {
@@ -140,19 +168,25 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             const int t = idx / NV, n = idx % NV;
             dO[idx] = n < nv ? p.dO[(vh * T + c0 + t) * dv + n0 + n] : 0.f;
         }
+        if (st)
+            for (int idx = tid; idx < Cl * dk; idx += NT) {
+                const int t = idx / dk, i = idx % dk;
+                const long g = (kh * T + c0 + t) * dk + i;
+                qs[t * ldq + i] = static_cast<const In *>(p.q)[g];
+                ks[t * ldq + i] = static_cast<const In *>(p.k)[g];
+            }
         __syncthreads();
         // --- P, M = P diag(beta) (into A), L
         for (int idx = tid; idx < Cl * Cl; idx += NT) {
             const int t = idx / Cl, j = idx % Cl;
             float pm = 0.f, lm = 0.f;
             if (j <= t) {
-                const long kt = (kh * T + c0 + t) * dk, kj = (kh * T + c0 + j) * dk;
                 for (int gi = 0; gi < G; ++gi) {
                     float skk = 0.f, sqk = 0.f;
                     for (int i = gi * width; i < (gi + 1) * width; ++i) {
-                        const float kji = ld_in<IN_BF16>(p.k, kj + i);
-                        skk += ld_in<IN_BF16>(p.k, kt + i) * kji;
-                        sqk += ld_in<IN_BF16>(p.q, kt + i) * kji;
+                        const float kji = kk(j, i);
+                        skk += kk(t, i) * kji;
+                        sqk += qq(t, i) * kji;
                     }
                     const float e = expf(lam[t * G + gi] - lam[j * G + gi]);
                     pm += e * skk;
@@ -187,11 +221,9 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
         // --- R = V - Kbar S (into dR), Kbar_t = k_t e^{Lambda_t}
         for (int idx = tid; idx < Cl * NV; idx += NT) {
             const int t = idx / NV, n = idx % NV;
-            const long kt = (kh * T + c0 + t) * dk;
             float acc = 0.f;
             for (int i = 0; i < dk; ++i)
-                acc += ld_in<IN_BF16>(p.k, kt + i) * (tab ? Et[t] : expf(lam[t * G + i / width])) *
-                       S[i * NV + n];
+                acc += kk(t, i) * (tab ? Et[t] : expf(lam[t * G + i / width])) * S[i * NV + n];
             const float vv = n < nv ? ld_in<IN_BF16>(p.v, (vh * T + c0 + t) * dv + n0 + n) : 0.f;
             dR[idx] = vv - acc;
         }
@@ -209,10 +241,9 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             float acc = 0.f;
             for (int t = j; t < Cl; ++t)
                 acc += L[t * C + j] * dO[t * NV + n];
-            const long kj = (kh * T + c0 + j) * dk;
             for (int i = 0; i < dk; ++i) {
                 const int gi = i / width;
-                acc += ld_in<IN_BF16>(p.k, kj + i) *
+                acc += kk(j, i) *
                        (tab ? E1[(Cl - 1) * C + j] : expf(lam[(Cl - 1) * G + gi] - lam[j * G + gi])) *
                        dS[i * NV + n];
             }
@@ -267,7 +298,7 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             for (int n = 0; n < NV; ++n) {
                 float sn = f * S[i * NV + n];
                 for (int t = 0; t < Cl; ++t)
-                    sn += ld_in<IN_BF16>(p.k, (kh * T + c0 + t) * dk + i) *
+                    sn += kk(t, i) *
                           (tab ? E1[(Cl - 1) * C + t] : expf(lc - lam[t * G + gi])) *
                           sbeta[t] * Y[t * NV + n];
                 x += dS[i * NV + n] * sn;
@@ -291,12 +322,12 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             const int t = idx / dk, i = idx % dk, gi = i / width;
             const float lt = lam[t * G + gi], lc = lam[(Cl - 1) * G + gi];
             const long base = (kh * T + c0) * dk + i;
-            const float kti = ld_in<IN_BF16>(p.k, base + (long)t * dk);
-            const float qti = ld_in<IN_BF16>(p.q, base + (long)t * dk);
+            const float kti = kk(t, i);
+            const float qti = qq(t, i);
             float a = 0.f, bb = 0.f, cc = 0.f, d = 0.f;
             for (int j = 0; j <= t; ++j) {
                 const float e = tab ? E1[t * C + j] : expf(lt - lam[j * G + gi]);
-                const float kji = ld_in<IN_BF16>(p.k, base + (long)j * dk);
+                const float kji = kk(j, i);
                 if (j < t)
                     a += sbeta[j] * A[t * C + j] * kji * e;
                 cc += L[t * C + j] * kji * e;
@@ -304,8 +335,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             for (int t2 = t; t2 < Cl; ++t2) {
                 const float e = tab ? E1[t2 * C + t] : expf(lam[t2 * G + gi] - lt);
                 if (t2 > t)
-                    bb += sbeta[t] * A[t2 * C + t] * ld_in<IN_BF16>(p.k, base + (long)t2 * dk) * e;
-                d += L[t2 * C + t] * ld_in<IN_BF16>(p.q, base + (long)t2 * dk) * e;
+                    bb += sbeta[t] * A[t2 * C + t] * kk(t2, i) * e;
+                d += L[t2 * C + t] * qq(t2, i) * e;
             }
             float dqb = 0.f, dkb = 0.f, dkh = 0.f;
             for (int n = 0; n < NV; ++n) {
@@ -347,9 +378,8 @@ __global__ void __launch_bounds__(NT) simt_bwd_kernel(const Params p)
             const int i = idx / NV, n = idx % NV, gi = i / width;
             float acc = Fv[i] * dS[idx];
             for (int t = 0; t < Cl; ++t) {
-                const long kt = (kh * T + c0 + t) * dk + i;
                 const float e = tab ? Et[t] : expf(lam[t * G + gi]);
-                acc += e * (ld_in<IN_BF16>(p.q, kt) * dO[t * NV + n] - ld_in<IN_BF16>(p.k, kt) * dR[t * NV + n]);
+                acc += e * (qq(t, i) * dO[t * NV + n] - kk(t, i) * dR[t * NV + n]);
             }
             dS[idx] = acc;
         }
@@ -378,7 +408,7 @@ constexpr int kMaxSmem = kBwdSmemFloats * 4;
 
 int bwd_smem_for(const Params &p, int NV)
 {
-    return bwd_layout(p.C, p.G, p.dk, NV).total * (int)sizeof(float);
+    return bwd_layout(p.C, p.G, p.dk, NV, p.in_bf16 ? 2 : 4).total * (int)sizeof(float);
 }
 
 int zero(float *a, long n, cudaStream_t stream)

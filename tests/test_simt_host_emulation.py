@@ -126,7 +126,7 @@ extern "C" int emu_run(const gdr::Params *p)
 template <bool I, int NV>
 static int run_bwd_grid(const gdr::Params &p)
 {
-    const int total = gdr::host_emu_bwd::bwd_layout(p.C, p.G, p.dk, NV).total;
+    const int total = gdr::host_emu_bwd::bwd_layout(p.C, p.G, p.dk, NV, I ? 2 : 4).total;
     if (total > %(smem)d)
         return -1;
     for (unsigned b = 0; b < (unsigned)p.B; ++b)
@@ -148,7 +148,7 @@ static int run_bwd_grid(const gdr::Params &p)
 extern "C" int emu_bwd_tile(const gdr::Params *p)
 {
     for (int NV : {32, 16})
-        if (gdr::host_emu_bwd::bwd_layout(p->C, p->G, p->dk, NV).total * 4 <= 227 * 1024)
+        if (gdr::host_emu_bwd::bwd_layout(p->C, p->G, p->dk, NV, p->in_bf16 ? 2 : 4).total * 4 <= 227 * 1024)
             return NV;
     return 0;
 }
