@@ -304,6 +304,23 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
                  "r"(d));
 }
 
+// A 16-byte store to global memory that the compiler does not see as a C++ store:
+// it cannot alias the shared-memory values a loop keeps in registers, so they are
+// not reloaded after it.  For record bytes that nothing in the kernel reads back.
+__device__ __forceinline__ void st_global_v4(void *dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(dst), "r"(a), "r"(b), "r"(c), "r"(d));
+}
+
+// Eight consecutive floats from 16-byte aligned shared memory, as two vector loads.
+__device__ __forceinline__ void ld8f(const float *src, float *o)
+{
+    const float4 x0 = *reinterpret_cast<const float4 *>(src);
+    const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+    o[0] = x0.x; o[1] = x0.y; o[2] = x0.z; o[3] = x0.w;
+    o[4] = x1.x; o[5] = x1.y; o[6] = x1.z; o[7] = x1.w;
+}
+
 __device__ __forceinline__ void ld_shared_v4(uint32_t saddr, uint32_t &a, uint32_t &b,
                                              uint32_t &c, uint32_t &d)
 {

@@ -202,14 +202,18 @@ __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
 }
 
 // In-place exact inverse of I + M (64 x 64, M strictly lower) by block doubling,
-// the merges spread over all 256 threads: after the exact 16 x 16 diagonal
-// blocks, each merge X21 = -X22 (M21 X11) is two small dense products whose
-// every output element has its own thread (2 columns a thread for the 16 x 16
-// merges, 4 for the 32 x 32 one) and a loop over the full inner index (the zero
-// triangles multiply as zeros, so every lane of a warp runs the same trip
-// count).  Same arithmetic as inverse64_inplace (inner index ascending, fp32),
-// shorter dependent chains; Tf needs 32 x 36 floats.
-__device__ __forceinline__ void inverse64_par(float *Mf, float *Tf, int tid)
+// the merges spread over the CTA: after the exact 16 x 16 diagonal blocks, each
+// merge X21 = -X22 (M21 X11) is two small dense products with a loop over the full
+// inner index (the zero triangles multiply as zeros, so every lane of a warp runs
+// the same trip count).  The 16 -> 32 merges give every output pair its own thread
+// (all 256); the 32 -> 64 one runs on warps 0-3, thread (rg, c0) owning rows rg
+// and rg + 16 of the 32-row block at columns c0 .. c0 + 3, so each step of the
+// inner index loads two values of the left factor and one float4 of the right one
+// for eight products: fewer shared-memory wavefronts than one output row a thread
+// (what bounds pass 1, several CTAs to an SM), shorter chains than 4 x 4 blocks on
+// two warps.  Same arithmetic as inverse64_inplace (inner index ascending, fp32);
+// Tf needs 32 x 36 floats.
+__device__ __forceinline__ void inverse64_mid(float *Mf, float *Tf, int tid)
 {
     diag16_inverse_inplace(Mf, Tf, tid);
     {   // 16 -> 32: pair pr (rows 32 pr + 16 .. +31, columns 32 pr .. +15)
@@ -235,33 +239,36 @@ __device__ __forceinline__ void inverse64_par(float *Mf, float *Tf, int tid)
         *reinterpret_cast<float2 *>(&Mf[(o + 16 + r) * LDM + o + c0]) = make_float2(-a0, -a1);
         __syncthreads();
     }
-    {   // 32 -> 64: rows 32 .. 63, columns 0 .. 31
-        const int r = tid >> 3, c0 = (tid & 7) * 4;
-        float a[4] = {0.f, 0.f, 0.f, 0.f};
+    // 32 -> 64: rows 32 + rg and 48 + rg, columns c0 .. c0 + 3
+    const int rg = (tid >> 3) & 15, c0 = (tid & 7) * 4;
+    if (tid < 128) {
+        float a[2][4] = {};
 #pragma unroll 8
         for (int l = 0; l < 32; ++l) {   // T = M21 X11
-            const float m = Mf[(32 + r) * LDM + l];
+            const float m0 = Mf[(32 + rg) * LDM + l], m1 = Mf[(48 + rg) * LDM + l];
             const float4 x = *reinterpret_cast<const float4 *>(&Mf[l * LDM + c0]);
-            a[0] += m * x.x;
-            a[1] += m * x.y;
-            a[2] += m * x.z;
-            a[3] += m * x.w;
+            a[0][0] += m0 * x.x; a[0][1] += m0 * x.y; a[0][2] += m0 * x.z; a[0][3] += m0 * x.w;
+            a[1][0] += m1 * x.x; a[1][1] += m1 * x.y; a[1][2] += m1 * x.z; a[1][3] += m1 * x.w;
         }
-        *reinterpret_cast<float4 *>(&Tf[r * 36 + c0]) = make_float4(a[0], a[1], a[2], a[3]);
-        __syncthreads();
-        a[0] = a[1] = a[2] = a[3] = 0.f;
+        *reinterpret_cast<float4 *>(&Tf[rg * 36 + c0]) = make_float4(a[0][0], a[0][1], a[0][2], a[0][3]);
+        *reinterpret_cast<float4 *>(&Tf[(rg + 16) * 36 + c0]) = make_float4(a[1][0], a[1][1], a[1][2], a[1][3]);
+    }
+    __syncthreads();
+    if (tid < 128) {
+        float a[2][4] = {};
 #pragma unroll 8
         for (int l = 0; l < 32; ++l) {   // X21 = -X22 T
-            const float x = Mf[(32 + r) * LDM + 32 + l];
+            const float x0 = Mf[(32 + rg) * LDM + 32 + l], x1 = Mf[(48 + rg) * LDM + 32 + l];
             const float4 t = *reinterpret_cast<const float4 *>(&Tf[l * 36 + c0]);
-            a[0] += x * t.x;
-            a[1] += x * t.y;
-            a[2] += x * t.z;
-            a[3] += x * t.w;
+            a[0][0] += x0 * t.x; a[0][1] += x0 * t.y; a[0][2] += x0 * t.z; a[0][3] += x0 * t.w;
+            a[1][0] += x1 * t.x; a[1][1] += x1 * t.y; a[1][2] += x1 * t.z; a[1][3] += x1 * t.w;
         }
-        *reinterpret_cast<float4 *>(&Mf[(32 + r) * LDM + c0]) = make_float4(-a[0], -a[1], -a[2], -a[3]);
-        __syncthreads();
+        *reinterpret_cast<float4 *>(&Mf[(32 + rg) * LDM + c0]) =
+            make_float4(-a[0][0], -a[0][1], -a[0][2], -a[0][3]);
+        *reinterpret_cast<float4 *>(&Mf[(48 + rg) * LDM + c0]) =
+            make_float4(-a[1][0], -a[1][1], -a[1][2], -a[1][3]);
     }
+    __syncthreads();
 }
 
 // In-place 1-Step Neumann approximation of (I + M)^{-1} ("Systolic Linear

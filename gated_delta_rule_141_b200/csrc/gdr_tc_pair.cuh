@@ -502,7 +502,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         }
         __syncthreads();
         if (!failed) {
-            gen::inverse64_par(A11f, Tf, tid);            // Atil11^{-1}, unit lower triangular
+            gen::inverse64_mid(A11f, Tf, tid);            // Atil11^{-1}, unit lower triangular
             for (int u = tid; u < CC * 8; u += NT) {
                 const int r = u >> 3, c = (u & 7) * 8;
                 split_store(IH, IL, r, c, A11f + r * LDM + c);
@@ -691,7 +691,7 @@ pair_kernel(const __grid_constant__ CUtensorMap tm_k, const PairArgs a)
         };
         const uint32_t id64 = idesc_bf16(64, 64, false, true);
         if (!failed) {
-            gen::inverse64_par(A11f, Tf, tid);                // Atil11^{-1}, lower triangular
+            gen::inverse64_mid(A11f, Tf, tid);                // Atil11^{-1}, lower triangular
             // stage 1 tiles: Ntil21 over the first 8 KB of its fp32 copy (read out first),
             // Atil22 high / low past the fp32 blocks in the residual and Ntil tiles
             const uint32_t N21T = XT, A22H = RT + 20480, A22L = NTL + 18432;

@@ -482,7 +482,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             //      pass's operands from the same two exponentials, Qbar = q a e^{Lambda_p} and
             //      Khat = k b e^{Lambda_C - Lambda_p}; the k rows keep k a (Kbar = k a e^{Lambda_p}
             //      is W's operand, its per-channel factor applied on the way out of TMEM)
-            auto item = [&](int t, int i0, const float *lt, const float *lp) {
+            // fq, fk: e^{Lambda_p} and e^{Lambda_C - Lambda_p} at the eight channels
+            auto item = [&](int t, int i0, const float *lt, const float *lp, const float *fq,
+                            const float *fk) {
                 float qv[8], kv[8], kc[8], kh8[8], qb[8];
                 ld_tile8(QK, 128, t, i0, qv);
                 ld_tile8(QK, 128, 64 + t, i0, kv);
@@ -492,37 +494,40 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     qv[e] *= a;
                     kc[e] = kv[e] * b;
                     kv[e] *= a;
-                    qb[e] = qv[e] * piv[i0 + e];
-                    kh8[e] = kc[e] * piv[DK + i0 + e];
+                    qb[e] = qv[e] * fq[e];
+                    kh8[e] = kc[e] * fk[e];
                 }
                 st_tile8(QK, 128, t, i0, qv);
                 st_tile8(QK, 128, 64 + t, i0, kv);
                 st_tile8(KC, 64, t, i0, kc);
                 if (ext) {
                     const uint32_t off = (i0 >> 6) * IMG + t * 128 + ((((i0 >> 3) & 7) ^ (t & 7)) << 4);
-                    *reinterpret_cast<uint4 *>(img_T + ext_qb(DK) + off) =
-                        make_uint4(pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]),
-                                   pack_bf16(qb[4], qb[5]), pack_bf16(qb[6], qb[7]));
-                    *reinterpret_cast<uint4 *>(img_T + ext_kh(DK) + off) =
-                        make_uint4(pack_bf16(kh8[0], kh8[1]), pack_bf16(kh8[2], kh8[3]),
-                                   pack_bf16(kh8[4], kh8[5]), pack_bf16(kh8[6], kh8[7]));
+                    st_global_v4(img_T + ext_qb(DK) + off, pack_bf16(qb[0], qb[1]), pack_bf16(qb[2], qb[3]),
+                                 pack_bf16(qb[4], qb[5]), pack_bf16(qb[6], qb[7]));
+                    st_global_v4(img_T + ext_kh(DK) + off, pack_bf16(kh8[0], kh8[1]),
+                                 pack_bf16(kh8[2], kh8[3]), pack_bf16(kh8[4], kh8[5]),
+                                 pack_bf16(kh8[6], kh8[7]));
                 }
             };
             if constexpr (RL) {
-                float lp[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    lp[e] = lam[LR_P * DK + i0r + e];
+                // the thread's eight channels are the same for its four tokens: the
+                // pivot's Lambda and the two per-channel factors are loaded once
+                float lp[8], fq[8], fk[8];
+                ld8f(lam + LR_P * DK + i0r, lp);
+                ld8f(piv + i0r, fq);
+                ld8f(piv + DK + i0r, fk);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    item(4 * tb + k, i0r, lv[k], lp);
+                    item(4 * tb + k, i0r, lv[k], lp, fq, fk);
             } else {
                 for (int u = tid; u < CC * (DK / 8); u += NT) {
                     const int t = u / (DK / 8), i0 = (u % (DK / 8)) * 8;
-                    float lt[8], lp[8];
+                    float lt[8], lp[8], fq[8], fk[8];
                     lam8(lam, G, wsh, t, i0, lt);
                     lam8(lam, G, wsh, PV, i0, lp);
-                    item(t, i0, lt, lp);
+                    ld8f(piv + i0, fq);
+                    ld8f(piv + DK + i0, fk);
+                    item(t, i0, lt, lp, fq, fk);
                 }
             }
             fence_proxy_async_smem();
@@ -554,6 +559,12 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int jh = j0 + 16 * h;
+                const bool with_beta = !qrow && !a.pair;   // pairs: the raw Gram, beta applied before the inverse
+                float bj[16];   // (grouped / per-channel gates: beta of the 16 columns at once)
+                if (!SCALAR && with_beta) {
+                    ld8f(sbeta + jh, bj);
+                    ld8f(sbeta + jh + 8, bj + 8);
+                }
                 float out[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
@@ -563,8 +574,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     float v = 0.f;
                     if (keep)
                         v = !SCALAR ? d : sc_piv ? d * (Tf[t] * Tf[CC + j]) : d * __expf(lt - lam[j]);
-                    if (!qrow && !a.pair)   // pairs: the raw Gram, beta applied before the inverse
-                        v *= sbeta[j];
+                    if (with_beta)
+                        v *= SCALAR ? sbeta[j] : bj[u];
                     out[u] = v;
                 }
                 if (qrow) {
@@ -855,7 +866,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (p.neumann1)
                 gen::block_neumann1_64_inplace(Mf, Tf, tid);
             else
-                gen::inverse64_par(Mf, Tf, tid);
+                gen::inverse64_mid(Mf, Tf, tid);
         } else {
             // ---- truncated Neumann series (Horner) + Newton residual steps, M = 64 on tcgen05
             const uint32_t NB = base_u32 + Ly.NB, XB = base_u32 + Ly.XB, RB = base_u32 + Ly.RB;
@@ -1051,9 +1062,15 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     if (rr >= 0) {
                         if (w_cols) {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                w0[e] *= Tf[cw + cb + e];
-                                w1[e] *= Tf[cw + cb + 16 + e];
+                            for (int e0 = 0; e0 < 16; e0 += 8) {
+                                float f0[8], f1[8];
+                                ld8f(Tf + cw + cb + e0, f0);
+                                ld8f(Tf + cw + cb + 16 + e0, f1);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    w0[e0 + e] *= f0[e];
+                                    w1[e0 + e] *= f1[e];
+                                }
                             }
                         }
                         if (a.neg_w) {
