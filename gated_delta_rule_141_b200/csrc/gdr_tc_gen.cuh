@@ -121,15 +121,16 @@ __device__ __forceinline__ void block_product4x4(float (&acc)[4][4], const float
 
 // The four diagonal 16 x 16 blocks of I + M (64 x 64, M strictly lower) replaced
 // in place by their exact inverses; the blocks below them are left as they are.
-__device__ __forceinline__ void diag16_inverse_inplace(float *Mf, float *Tf, int tid)
+__device__ __forceinline__ void diag16_inverse_inplace(float *Mf, int tid)
 {
-    // diagonal 16 x 16 blocks, exact forward substitution (into Tf, then back).
-    // Column cc of the block's inverse, right-looking: once x_j is final it is
-    // applied to every later row at once, so the dependent chain is 15 steps
-    // long (each x_t still sums its terms in the order j = 0, 1, ...).
+    // Exact forward substitution, column cc of a block's inverse a thread, in
+    // registers.  Right-looking: once x_j is final it is applied to every later row
+    // at once, so the dependent chain is 15 steps long (each x_t still sums its
+    // terms in the order j = 0, 1, ...).  The columns go back over the blocks once
+    // every thread has read them (a barrier, no staging copy).
+    const int blk = tid >> 4, cc = tid & 15, o = 16 * blk;
+    float x[16];
     if (tid < 64) {
-        const int blk = tid >> 4, cc = tid & 15, o = 16 * blk;
-        float x[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t)
             x[t] = (t == cc) ? 1.f : 0.f;
@@ -140,22 +141,19 @@ __device__ __forceinline__ void diag16_inverse_inplace(float *Mf, float *Tf, int
             for (int t = j + 1; t < 16; ++t)
                 x[t] -= Mf[(o + t) * LDM + o + j] * xj;
         }
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-            Tf[blk * 256 + t * 16 + cc] = x[t];
     }
     __syncthreads();
-    for (int idx = tid; idx < 4 * 256; idx += NT) {
-        const int blk = idx >> 8, t = (idx >> 4) & 15, cc = idx & 15;
-        Mf[(16 * blk + t) * LDM + 16 * blk + cc] = Tf[idx];
-    }
+    if (tid < 64)
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+            Mf[(o + t) * LDM + o + cc] = x[t];
     __syncthreads();
 }
 
 // In-place exact inverse of I + M (64 x 64, M strictly lower) by block doubling.
 __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
 {
-    diag16_inverse_inplace(Mf, Tf, tid);
+    diag16_inverse_inplace(Mf, tid);
     // The doubling steps are products of small dense blocks.  Each thread owns a
     // 4 x 4 block of the product: per step of the inner index it loads four A
     // values (shared by the lanes of a row group) and one float4 of B, which is
@@ -215,7 +213,7 @@ __device__ __forceinline__ void inverse64_inplace(float *Mf, float *Tf, int tid)
 // Tf needs 32 x 36 floats.
 __device__ __forceinline__ void inverse64_mid(float *Mf, float *Tf, int tid)
 {
-    diag16_inverse_inplace(Mf, Tf, tid);
+    diag16_inverse_inplace(Mf, tid);
     {   // 16 -> 32: pair pr (rows 32 pr + 16 .. +31, columns 32 pr .. +15)
         const int pr = tid >> 7, q = tid & 127, r = q >> 3, c0 = (q & 7) * 2, o = 32 * pr;
         float a0 = 0.f, a1 = 0.f;
@@ -279,7 +277,7 @@ __device__ __forceinline__ void inverse64_mid(float *Mf, float *Tf, int tid)
 // (j, i) first, one 16-thread group per block (4 x 4 outputs a thread).
 __device__ __forceinline__ void block_neumann1_64_inplace(float *Mf, float *Tf, int tid)
 {
-    diag16_inverse_inplace(Mf, Tf, tid);
+    diag16_inverse_inplace(Mf, tid);
     const int pi = tid >> 4;                      // block pair 0..5 for tid < 96
     const int bi = pi < 1 ? 1 : pi < 3 ? 2 : 3;   // (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
     const int bj = pi < 1 ? 0 : pi < 3 ? pi - 1 : pi - 3;

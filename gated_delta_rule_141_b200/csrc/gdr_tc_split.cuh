@@ -732,13 +732,18 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
 // Start state of every segment: S_start(0) = S0 (or zero), S_start(g + 1) =
 // Atil_g S_start(g) + Btil_g, in fp32 on the CUDA cores.  One CTA per (batch, value
-// head, 16 value columns); thread (r, j0) keeps row r, columns j0..j0+7 of S.  The
-// steps are sequential, so Atil_{g+1} is copied in (cp.async, second buffer) while
-// step g computes.
-constexpr int CMB_COLS = 16, CMB_LDA = KD + 4;   // rows 16-byte aligned, 2-way bank spread
+// head, 16 value columns), 128 threads; thread (rb, cb) keeps rows rb, rb + 32,
+// rb + 64, rb + 96 at columns 4 cb .. 4 cb + 3 of S, so that each step of the inner
+// index is four float4 loads of Atil's rows and one of S's for sixteen products (the
+// rows 32 apart fall in distinct bank groups).  Each output sums Btil, then the inner
+// index in ascending order.  The steps are sequential, so Atil_{g+1} is copied in
+// (cp.async, second buffer) and Btil_{g+1} loaded into registers while step g
+// computes.
+constexpr int CMB_COLS = 16, CMB_LDA = KD + 4;   // rows 16-byte aligned, 4-bank row offset
+constexpr int CMB_THREADS = 128;
 constexpr uint32_t CMB_SMEM = (2 * KD * CMB_LDA + KD * CMB_COLS) * 4;
 
-__global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
+__global__ void __launch_bounds__(CMB_THREADS) seg_combine_kernel(const SplitArgs a)
 {
     using namespace ptx;
     extern __shared__ __align__(16) float cmb[];
@@ -747,61 +752,84 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const SplitArgs a)
     const int ncg = p.dv / CMB_COLS;
     const int cg = blockIdx.x % ncg, hv = blockIdx.x / ncg, b = blockIdx.y;
     const long vh = (long)b * p.Hv + hv, kh = (long)b * p.Hk + hv / p.R;
-    const int tid = threadIdx.x, r = tid >> 1, j0 = (tid & 1) * 8, col = cg * CMB_COLS + j0;
+    const int tid = threadIdx.x, rb = tid >> 2, c4 = (tid & 3) * 4, col = cg * CMB_COLS + c4;
     auto fetch = [&](int g) {   // Atil_g into buffer g % 2
         const float *At = a.seg_trans + ((size_t)kh * a.nseg + g) * KD * KD;
         float *As = cmb + (g & 1) * KD * CMB_LDA;
-        for (int u = tid; u < KD * KD / 4; u += 256)
+        for (int u = tid; u < KD * KD / 4; u += CMB_THREADS)
             cp_async16(smem_u32(As + (u / (KD / 4)) * CMB_LDA + (u % (KD / 4)) * 4), At + 4 * u, 16u);
         cp_async_commit();
     };
-    float sv[8];
+    float sv[4][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        sv[j] = p.S0 != nullptr ? p.S0[(vh * KD + r) * p.dv + col + j] : 0.f;
-    if (a.nseg > 1)
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)   // (S0 is the caller's: no alignment assumed)
+            sv[i][j] = p.S0 != nullptr ? p.S0[(vh * KD + rb + 32 * i) * p.dv + col + j] : 0.f;
+    // Btil_g, loaded one step ahead (its latency hides behind the step before)
+    float bn[4][4];
+    auto load_b = [&](int g) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 bt = *reinterpret_cast<const float4 *>(
+                a.seg_end + (((size_t)vh * a.nseg + g) * KD + rb + 32 * i) * p.dv + col);
+            bn[i][0] = bt.x; bn[i][1] = bt.y; bn[i][2] = bt.z; bn[i][3] = bt.w;
+        }
+    };
+    if (a.nseg > 1) {
         fetch(0);
+        load_b(0);
+    }
     for (int g = 0; g < a.nseg; ++g) {
-        float *st = a.seg_start + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
-        *reinterpret_cast<float4 *>(st) = make_float4(sv[0], sv[1], sv[2], sv[3]);
-        *reinterpret_cast<float4 *>(st + 4) = make_float4(sv[4], sv[5], sv[6], sv[7]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float *st = a.seg_start + (((size_t)vh * a.nseg + g) * KD + rb + 32 * i) * p.dv + col;
+            *reinterpret_cast<float4 *>(st) = make_float4(sv[i][0], sv[i][1], sv[i][2], sv[i][3]);
+        }
         if (g + 1 == a.nseg)
             break;
         cp_async_wait_all();   // Atil_g has landed (this thread's share)
         __syncthreads();       // ... everyone's; the previous step's readers are done
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            Ss[r * CMB_COLS + j0 + j] = sv[j];
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4 *>(&Ss[(rb + 32 * i) * CMB_COLS + c4]) =
+                make_float4(sv[i][0], sv[i][1], sv[i][2], sv[i][3]);
         __syncthreads();
         if (g + 2 < a.nseg)
             fetch(g + 1);
         const float *As = cmb + (g & 1) * KD * CMB_LDA;
-        const float *Bt = a.seg_end + (((size_t)vh * a.nseg + g) * KD + r) * p.dv + col;
-        float acc[8];
-        {
-            const float4 b0 = *reinterpret_cast<const float4 *>(Bt);
-            const float4 b1 = *reinterpret_cast<const float4 *>(Bt + 4);
-            acc[0] = b0.x; acc[1] = b0.y; acc[2] = b0.z; acc[3] = b0.w;
-            acc[4] = b1.x; acc[5] = b1.y; acc[6] = b1.z; acc[7] = b1.w;
-        }
-        // the inner index four at a time (one float4 of Atil's row, two of each S row),
-        // still in ascending order
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[i][j] = bn[i][j];
+        if (g + 2 < a.nseg)
+            load_b(g + 1);
         for (int l = 0; l < KD; l += 4) {
-            const float4 a4 = *reinterpret_cast<const float4 *>(&As[r * CMB_LDA + l]);
-            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+            float av[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(&As[(rb + 32 * i) * CMB_LDA + l]);
+                av[i][0] = a4.x; av[i][1] = a4.y; av[i][2] = a4.z; av[i][3] = a4.w;
+            }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float4 s0 = *reinterpret_cast<const float4 *>(&Ss[(l + u) * CMB_COLS + j0]);
-                const float4 s1 = *reinterpret_cast<const float4 *>(&Ss[(l + u) * CMB_COLS + j0 + 4]);
-                const float sj[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                const float4 s4 = *reinterpret_cast<const float4 *>(&Ss[(l + u) * CMB_COLS + c4]);
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    acc[j] += av[u] * sj[j];
+                for (int i = 0; i < 4; ++i) {
+                    acc[i][0] += av[i][u] * s4.x;
+                    acc[i][1] += av[i][u] * s4.y;
+                    acc[i][2] += av[i][u] * s4.z;
+                    acc[i][3] += av[i][u] * s4.w;
+                }
             }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            sv[j] = acc[j];
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                sv[i][j] = acc[i][j];
     }
     cp_async_wait_all();
 }
@@ -856,7 +884,7 @@ int launch(const Params &p, const void *factors, cudaStream_t stream)
         return 6;
     a.mode = MODE_SEG_AB;
     kern<<<dim3(a.nvt * p.Hv + (KD / NVC) * p.Hk, p.B, sp.nseg), NTHR, Ly.total, stream>>>(mq, mk, mv, a);
-    seg_combine_kernel<<<dim3((p.dv / CMB_COLS) * p.Hv, p.B), 256, CMB_SMEM, stream>>>(a);
+    seg_combine_kernel<<<dim3((p.dv / CMB_COLS) * p.Hv, p.B), CMB_THREADS, CMB_SMEM, stream>>>(a);
     a.mode = MODE_SEG_C;
     kern<<<dim3(a.nvt * p.Hv, p.B, sp.nseg), NTHR, Ly.total, stream>>>(mq, mk, mv, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;

@@ -540,7 +540,7 @@ int launch128(const Params &p, const void *factors, cudaStream_t stream)
         return 6;
     a.mode = MODE_SEG_AB;
     ab::ab128_kernel<<<dim3(a.nvt * p.Hv, p.B, sp.nseg), ab::NTHR, La.total, stream>>>(mv, a);
-    seg_combine_kernel<<<dim3((p.dv / CMB_COLS) * p.Hv, p.B), 256, CMB_SMEM, stream>>>(a);
+    seg_combine_kernel<<<dim3((p.dv / CMB_COLS) * p.Hv, p.B), CMB_THREADS, CMB_SMEM, stream>>>(a);
     a.mode = MODE_SEG_C;
     kern<<<dim3(a.nvt * p.Hv, p.B, sp.nseg), NTHR, Ly.total, stream>>>(mv, a);
     return cudaGetLastError() == cudaSuccess ? 0 : 6;
