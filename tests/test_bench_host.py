@@ -70,3 +70,20 @@ def test_roofline_arithmetic():
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert abs(r["frac"] - 1.34e11 / 1e-4 / 1726e12) < 1e-12
     assert abs(r["hbm_frac"] - 414e6 / 1e-4 / 6448e9) < 1e-12
+
+
+def test_recorded_traffic_follows_the_sources(tmp_path, monkeypatch):
+    """A committed DRAM figure is reported only while the kernels' source files are the
+    ones it was measured on: any edit to them turns it into null."""
+    src = tmp_path / "k.cuh"
+    src.write_text("// kernel source\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    entry = {"files": ["k.cuh"], "fingerprint": bench.files_fingerprint(["k.cuh"]),
+             "bytes_per_launch": 4365551616}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"wl/C128/exact/tc2": entry}))
+    assert bench.recorded_traffic("wl", 128, "exact", "tc2") == 4365551616
+    assert bench.recorded_traffic("wl", 64, "exact", "tc2") is None   # no entry for that chunk
+    src.write_text("// kernel source, edited\n")
+    assert bench.recorded_traffic("wl", 128, "exact", "tc2") is None
+
